@@ -1,0 +1,87 @@
+"""Shared test helpers: oracle layers from the seeded generator, the top-k margin
+filter, and the output tolerance check."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+from workloads import synth
+
+# Output tolerance of the block: per-token relative L2 error and max-abs error
+# relative to the largest reference magnitude.
+REL_L2_TOL = 1e-3
+MAX_ABS_TOL = 5e-3
+# Minimum fp64 gap between the k-th and (k+1)-th logit of every test token, so that
+# routing is decided identically by any correct fp32 implementation.
+TOPK_MARGIN = 1e-3
+
+
+def oracle_layer_from(cfg: synth.Config, L: dict, *, norm_topk: int = 1, corr_on_output: int = 0,
+                      sh_gate_vec=None) -> oracle.OracleLayer:
+    """Pack a generated layer with the oracle's own packer."""
+    fmt = cfg.fmt
+    return oracle.OracleLayer(
+        d=cfg.d, n_experts=cfg.n_experts, top_k=cfg.top_k, ffn=cfg.ffn, fmt=fmt,
+        w_router=L["w_router"], w_delta=L["w_delta"],
+        gate_exps=oracle.pack(fmt, L["gate_codes"], L["gate_scales"]),
+        up_exps=oracle.pack(fmt, L["up_codes"], L["up_scales"]),
+        down_exps=oracle.pack(fmt, L["down_codes"], L["down_scales"]),
+        shared_ffn=cfg.shared_ffn,
+        sh_gate=L.get("sh_gate"), sh_up=L.get("sh_up"), sh_down=L.get("sh_down"),
+        sh_gate_vec=sh_gate_vec,
+        rank=cfg.rank, corr_a=L.get("corr_a"), corr_b=L.get("corr_b"),
+        norm_topk=norm_topk, corr_on_output=corr_on_output,
+    )
+
+
+def topk_gap(logits: np.ndarray, k: int) -> np.ndarray:
+    """Per-token fp64 gap between the k-th and (k+1)-th largest logit."""
+    s = -np.sort(-logits, axis=1)
+    if k >= logits.shape[1]:
+        return np.full(logits.shape[0], np.inf)
+    return s[:, k - 1] - s[:, k]
+
+
+def with_margin(cfg: synth.Config, layer: oracle.OracleLayer, x: np.ndarray, margin: float = TOPK_MARGIN,
+                seed: int = 12345, max_rounds: int = 50) -> np.ndarray:
+    """Replace tokens whose top-k margin (oracle fp64 logits) is below `margin` with fresh
+    draws from the generator until every token has the margin."""
+    x = x.copy()
+    bad = np.arange(x.shape[0])
+    for rnd in range(max_rounds):
+        logits, _, _ = oracle.route(layer, x[bad])
+        gap = topk_gap(logits, cfg.top_k)
+        bad = bad[gap < margin]
+        if bad.size == 0:
+            return x
+        x[bad] = synth.x_rows_host(cfg, bad.size, seed + 7919 * rnd)
+    raise RuntimeError("could not reach the top-k margin")
+
+
+def check_output(got: np.ndarray, ref: np.ndarray, rel_l2: float = REL_L2_TOL, max_abs: float = MAX_ABS_TOL):
+    """Per-token relative L2 <= rel_l2 and max |got-ref| <= max_abs * max|ref|."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    if ref.size == 0:
+        return
+    err = np.linalg.norm(got - ref, axis=1)
+    nrm = np.linalg.norm(ref, axis=1)
+    rel = err / np.maximum(nrm, 1e-300)
+    worst = int(np.argmax(rel))
+    assert rel.max() <= rel_l2, "token %d: relative L2 %.3e > %.1e" % (worst, rel.max(), rel_l2)
+    mx = np.abs(got - ref).max()
+    assert mx <= max_abs * np.abs(ref).max(), "max abs %.3e > %.1e * %.3e" % (mx, max_abs, np.abs(ref).max())
+
+
+def f16(bits: np.ndarray) -> np.ndarray:
+    """fp16 bit patterns -> float64 via numpy's float16 (a library routine)."""
+    return np.asarray(bits, np.uint16).view(np.float16).astype(np.float64)
+
+
+def bf16(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> float64 via torch's bfloat16 (a library routine)."""
+    import torch
+
+    t = torch.from_numpy(np.ascontiguousarray(bits, np.uint16).view(np.int16)).view(torch.bfloat16)
+    return t.double().numpy()
