@@ -1,0 +1,401 @@
+#!/usr/bin/env python
+"""MoE-layer throughput of the ternary MoE block forward on B200.
+
+Default workload: the 35B-A3B-class decode layer (d=2048, 256 experts, top-8 + shared
+expert, ffn 512, PQ2_0 experts, rank-512 correction).  One step = one forward at each
+decode batch size b in {1, 8, 32, 64} (105 tokens), each call on the next of 40
+independent layers (9.1 GB of weights, far above the 126 MB L2, so every call reads
+its weights from HBM).  Metric: tokens/s over the whole job.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl scion|reference]
+
+The block does not shard across GPUs (one GPU per layer replica): with N > 1 each
+rank runs an independent replica (weak scaling); NCCL is used only for the barrier
+and the max-over-ranks of the timed region.  `--impl reference` times the CPU
+oracle (the plain fp64 reference) on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s (decode b=1..64, prefill 4K/16K); % HBM or bf16 roofline"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="a3b_decode")
+    ap.add_argument("--impl", default="scion", choices=["scion", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0, help="override the number of cycled layers")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------- algorithmic work
+def workload_bytes(cfg, T, U):
+    """Algorithmic HBM bytes of one forward: U active experts' packed banks, the dense
+    bf16 weights (router + delta, shared expert, correction), x in and out."""
+    bb = 34 if cfg.fmt == 0 else 28
+    per_expert = 3 * cfg.ffn * cfg.d * bb // 128
+    fixed = (2 * cfg.n_experts * cfg.d + 3 * cfg.shared_ffn * cfg.d + 2 * cfg.rank * cfg.d) * 2
+    return U * per_expert + fixed + T * cfg.d * (2 + 4)
+
+
+def stage_bytes(cfg, T, U):
+    """Algorithmic bytes per launch of each kernel stage."""
+    bb = 34 if cfg.fmt == 0 else 28
+    d, F, k, Fs, r, E = cfg.d, cfg.ffn, cfg.top_k, cfg.shared_ffn, cfg.rank, cfg.n_experts
+    rf = 4 if cfg.router_f32 else 2
+    return {
+        "router_f32": 2 * E * d * 4 + T * d * 2 + T * E * 4,
+        "xproj": ((0 if cfg.router_f32 else 2 * E * d) + 2 * Fs * d + r * d) * 2 + T * d * 2 + T * E * 4
+        + T * (Fs + r) * 2,
+        "route": T * E * 4 + T * k * 12 + E * 12,
+        "gateup": U * 2 * F * d * bb // 128 + T * d * 2 + T * k * F * 2,
+        "down_routed": U * F * d * bb // 128 + T * k * F * 2 + T * d * 4,
+        "down_dense": d * (Fs + r) * 2 + T * (Fs + r) * 2 + T * d * 4,
+    }
+
+
+def workload_flops(cfg, T):
+    return 2 * T * (cfg.top_k * 3 * cfg.d * cfg.ffn + 3 * cfg.d * cfg.shared_ffn + 2 * cfg.n_experts * cfg.d
+                    + 2 * cfg.rank * cfg.d)
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons of one GPU through NVML (read-only)."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, torch_dev):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_dev).uuid)
+            h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                hi = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(hi)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    h = hi
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(0)
+            self.h, self.nv = h, pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover
+            self.err = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------- oracle baseline
+def oracle_sample(cfg, batches):
+    """Host-generated layer 0 of the workload and its oracle; returns (oracle layer, xs)."""
+    import oracle
+    from workloads import synth
+
+    L = synth.layer_host(cfg, 0)
+    banks = {n: oracle.pack(cfg.fmt, L[n + "_codes"], L[n + "_scales"]) for n in ("gate", "up", "down")}
+    for n in ("gate", "up", "down"):
+        del L[n + "_codes"]
+    ol = oracle.OracleLayer(
+        d=cfg.d, n_experts=cfg.n_experts, top_k=cfg.top_k, ffn=cfg.ffn, fmt=cfg.fmt, w_router=L["w_router"],
+        w_delta=L["w_delta"], gate_exps=banks["gate"], up_exps=banks["up"], down_exps=banks["down"],
+        shared_ffn=cfg.shared_ffn, sh_gate=L.get("sh_gate"), sh_up=L.get("sh_up"), sh_down=L.get("sh_down"),
+        rank=cfg.rank, corr_a=L.get("corr_a"), corr_b=L.get("corr_b"))
+    xs = [synth.x_host(cfg, T) for T in batches]
+    return ol, xs
+
+
+def cpu_baseline(cfg):
+    import oracle
+
+    batches = cfg.tokens if max(cfg.tokens) <= 64 else [64]
+    ol, xs = oracle_sample(cfg, batches)
+    t0 = time.perf_counter()
+    for x in xs:
+        oracle.forward(ol, x)
+    dt = time.perf_counter() - t0
+    ntok = sum(batches)
+    return {"value": ntok / dt, "unit": "tokens/s", "cores": oracle.cores_used(), "kind": "oracle",
+            "sample": "%s layer 0 (host-generated), one forward per batch %s = %d tokens, %.1f s"
+                      % (cfg.name, batches, ntok, dt)}
+
+
+def run_reference(args, rank):
+    """The oracle arm: plain fp64 C reference on the host cores, rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+    from workloads import synth
+
+    cfg = synth.CONFIGS[args.workload]
+    ol, xs = oracle_sample(cfg, [1])
+    x = xs[0]
+    for _ in range(args.warmup):
+        oracle.forward(ol, x)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.forward(ol, x)
+    dt = time.perf_counter() - t0
+    v = args.steps / dt
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": cfg.name, "d": cfg.d, "experts": cfg.n_experts, "top_k": cfg.top_k,
+                       "ffn": cfg.ffn, "format": "PQ2_0" if cfg.fmt == 0 else "PTQ1_0"},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.cores_used(), "kind": "oracle",
+                             "sample": "each step: one single-token forward on layer 0 of %s" % cfg.name},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- GPU arm
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import ternary_quantized_moe_b200 as tq
+    from workloads import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    cfg = synth.CONFIGS[args.workload]
+    n_layers = args.layers or cfg.n_layers
+    batches = list(cfg.tokens)
+    max_T = max(batches)
+    peaks, peak_src = load_peaks()
+
+    # ---- layers (generated and packed on the GPU, then re-tiled by scion_layer_create)
+    layers = []
+    for l in range(n_layers):
+        W = synth.layer_device(cfg, l, dev)
+        banks = {n: tq.scion_pack_device(cfg.fmt, W.pop(n + "_codes"), W.pop(n + "_scales")) for n in
+                 ("gate", "up", "down")}
+        layers.append(tq.scion_layer_create(
+            d=cfg.d, n_experts=cfg.n_experts, top_k=cfg.top_k, ffn=cfg.ffn, fmt=cfg.fmt, w_router=W["w_router"],
+            w_router_delta=W["w_delta"], gate_exps=banks["gate"], up_exps=banks["up"], down_exps=banks["down"],
+            shared_ffn=cfg.shared_ffn, sh_gate=W.get("sh_gate"), sh_up=W.get("sh_up"), sh_down=W.get("sh_down"),
+            rank=cfg.rank, corr_a=W.get("corr_a"), corr_b=W.get("corr_b"), max_tokens=max_T))
+        del banks, W
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    weight_bytes = sum(tq.scion_layer_device_bytes(L) for L in layers)
+
+    xs = {T: synth.x_device(cfg, T, dev) for T in batches}
+    outs = {T: torch.empty((T, cfg.d), dtype=torch.float32, device=dev) for T in batches}
+    stream = torch.cuda.current_stream(dev)
+    nb = len(batches)
+
+    def step(s):
+        for i, T in enumerate(batches):
+            tq.scion_moe_forward(xs[T], T, layers[(s * nb + i) % n_layers], outs[T], stream)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def timed(fn, K):
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(K):
+            fn(s)
+        e1.record(stream)
+        e1.synchronize()
+        ms = e0.elapsed_time(e1)
+        barrier()
+        return max_over_ranks(ms)
+
+    for s in range(args.warmup):
+        step(s)
+    K = args.steps
+
+    # ---- headline: device-timed region, inputs resident in HBM
+    launches0 = tq.scion_kernel_launches()
+    with ClockSampler(dev) as clocks:
+        ms = timed(step, K)
+    launches = tq.scion_kernel_launches() - launches0
+    tokens_per_step = sum(batches)
+    value = world * tokens_per_step * K / (ms / 1000.0)
+
+    # ---- per-kernel device time (CUDA events around every launch, same schedule)
+    barrier()
+    tq.scion_profile_begin(int(launches) + 64)
+    for s in range(K):
+        step(s)
+    stages = tq.scion_profile_end()
+
+    # ---- realised routing: distinct active experts of every (layer, batch) pair
+    U = {}
+    counts = torch.empty(cfg.n_experts, dtype=torch.int32, device=dev)
+    for li in range(n_layers):
+        for T in batches:
+            if T <= 64:
+                tq.scion_moe_forward_debug(xs[T], T, layers[li], outs[T], stream, counts=counts)
+                U[(li, T)] = int((counts > 0).sum().item())
+            else:
+                U[(li, T)] = cfg.n_experts
+    sched = [((s * nb + i) % n_layers, T) for s in range(K) for i, T in enumerate(batches)]
+    bytes_total = sum(workload_bytes(cfg, T, U[(li, T)]) for li, T in sched)
+    sbytes = {}
+    for li, T in sched:
+        for k_, v in stage_bytes(cfg, T, U[(li, T)]).items():
+            sbytes[k_] = sbytes.get(k_, 0) + v
+    flops_total = sum(workload_flops(cfg, T) for _, T in sched)
+
+    # ---- per batch size (each batch alone, cycling layers)
+    per_batch = {}
+    for T in batches:
+        def one(s, T=T):
+            tq.scion_moe_forward(xs[T], T, layers[s % n_layers], outs[T], stream)
+        msT = timed(one, K)
+        bT = sum(workload_bytes(cfg, T, U[(s % n_layers, T)]) for s in range(K))
+        per_batch[str(T)] = {"tokens_per_s": world * T * K / (msT / 1000.0), "us_per_call": 1000.0 * msT / K,
+                             "hbm_frac": (bT / (msT / 1000.0)) / (peaks["hbm_gbs"] * 1e9)}
+
+    # ---- end to end through the host-buffer entry point (pinned host x in, out back to host)
+    xh = {T: xs[T].cpu().pin_memory() for T in batches}
+    oh = {T: torch.empty((T, cfg.d), dtype=torch.float32).pin_memory() for T in batches}
+
+    def step_host(s):
+        for i, T in enumerate(batches):
+            tq.scion_moe_forward_host(xh[T], T, layers[(s * nb + i) % n_layers], oh[T], stream)
+
+    ms_e2e = timed(step_host, K)
+    e2e = {"value": world * tokens_per_step * K / (ms_e2e / 1000.0), "unit": "tokens/s",
+           "h2d_bytes_per_step": sum(T * cfg.d * 2 for T in batches),
+           "d2h_bytes_per_step": sum(T * cfg.d * 4 for T in batches)}
+
+    # ---- roofline of the dominant kernel
+    dom = max((k_ for k_ in stages if stages[k_][1] > 0), key=lambda k_: stages[k_][0])
+    dom_ms, dom_n = stages[dom]
+    decode = max_T <= 64
+    if decode:
+        achieved = (sbytes[dom] / dom_n) / (dom_ms / dom_n / 1000.0) / 1e9
+        roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                "bytes_per_launch": sbytes[dom] / dom_n, "us_per_launch": 1000.0 * dom_ms / dom_n}
+    else:
+        fl = flops_total  # attributed to the dominant (expert GEMM) kernel when prefill
+        achieved = fl / (dom_ms / 1000.0) / 1e12
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": peak_src}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "d": cfg.d, "experts": cfg.n_experts, "top_k": cfg.top_k, "ffn": cfg.ffn,
+                   "shared_ffn": cfg.shared_ffn, "rank": cfg.rank, "format": "PQ2_0" if cfg.fmt == 0 else "PTQ1_0",
+                   "batches": batches, "layers_cycled": n_layers, "tokens_per_step": tokens_per_step,
+                   "l2": "inputs larger than L2: %.1f GB of layers cycled" % (weight_bytes / 1e9),
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "roofline": roof,
+        "step_roofline": {"bytes_per_step": bytes_total / K, "hbm_frac": (bytes_total / (ms / 1000.0)) /
+                          (peaks["hbm_gbs"] * 1e9), "tflops": flops_total / (ms / 1000.0) / 1e12},
+        "per_batch": per_batch,
+        "stages_us_per_launch": {k_: 1000.0 * v[0] / v[1] for k_, v in stages.items() if v[1]},
+        "stages_share": {k_: v[0] / sum(x[0] for x in stages.values()) for k_, v in stages.items() if v[1]},
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg)
+    for L in layers:
+        L.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    run_gpu(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

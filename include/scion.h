@@ -1,0 +1,208 @@
+/*
+ * scion.h -- C ABI of libscion: the forward pass of one mixture-of-experts block
+ * whose expert banks are ternary ({-1, 0, +1} codes with one fp16 scale per 128
+ * weights), plus a rank-r low-rank correction added to the block output.
+ * All compute runs in hand-written CUDA kernels for sm_100a (NVIDIA B200).
+ *
+ * Sources (page titles and sections):
+ *  [P1] "Scion: ternary MoE quantization with trained corrections", The idea:
+ *       ternary expert banks at 2.125 bpw; rank-512 correction branches on the
+ *       MoE block output; router deltas.
+ *  [P3] "Scion-35B-A3B" model card: Model Overview (256 experts, top-8 plus a
+ *       shared expert), Weight Representation (codes in {-1,0,+1} plus one fp16
+ *       group scale per 128 weights = 2.125 bpw; routers stay F32).
+ *  [P4] "Scion-FlashNext-176B-A6B" model card: Model Overview (512 experts,
+ *       top-10 routed + 1 shared), Highlights and Weight Representation (PTQ1_0:
+ *       base-3 trits plus an fp16 scale, 28 bytes per 128 weights = 1.75 bpw).
+ *  [P1 Serving notes] the expert matmul computes k experts per token.
+ *
+ * Conventions for every entry point:
+ *  - Returns an int status (scion_status); never throws, never aborts.
+ *  - "device" pointers are CUDA global memory of the current device; "host"
+ *    pointers are CPU memory.  The caller owns every buffer it passes.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy stream).
+ *    Device work is enqueued asynchronously; no entry point synchronises the
+ *    stream except scion_layer_create (which validates codes once).
+ *  - Asynchronous CUDA faults surface as SCION_ECUDA on a later call.
+ */
+#ifndef SCION_H
+#define SCION_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SCION_OK = 0,
+  SCION_EINVAL = -1,   /* bad argument: null pointer, size out of range, bad descriptor */
+  SCION_ENOMEM = -2,   /* device or host allocation failed */
+  SCION_ECUDA = -3,    /* a CUDA runtime call or kernel launch failed */
+  SCION_EFORMAT = -4,  /* a packed block holds an invalid code (PQ2_0 field 3, PTQ1_0 byte > 242 / tail > 26) */
+  SCION_ETIMEOUT = -5  /* a bounded device-side wait gave up */
+} scion_status;
+
+/* Container formats.  Bit orders are this library's container specification
+ * (the pages give only the sizes):
+ *  SCION_PQ2_0  (34 B / 128 weights, [P3] Weight Representation): byte i < 32
+ *     holds weights 4i..4i+3, weight 4i+j in bits 2j..2j+1; field 0 -> -1,
+ *     1 -> 0, 2 -> +1, 3 invalid; bytes 32..33 = fp16 scale, little-endian.
+ *  SCION_PTQ1_0 (28 B / 128 weights, [P4] Weight Representation): byte q < 25 =
+ *     sum_{j<5} t_{5q+j} 3^j; byte 25 = t125 + 3 t126 + 9 t127; trit t -> code
+ *     t - 1; bytes 26..27 = fp16 scale, little-endian.
+ * A weight is code * scale. */
+typedef enum { SCION_PQ2_0 = 0, SCION_PTQ1_0 = 1 } scion_fmt;
+
+/* Bytes per 128-weight block: 34 (PQ2_0), 28 (PTQ1_0), 0 for an unknown format. */
+size_t scion_block_bytes(int fmt);
+
+/* Human-readable name of a status code (static storage). */
+const char* scion_status_str(int status);
+
+/* ------------------------------------------------------------------ packing
+ * Host packers.  codes: n_groups*128 int8 values in {-1,0,+1}; scales:
+ * n_groups fp16 bit patterns; out: n_groups*scion_block_bytes(fmt) bytes.  All
+ * host memory, caller-owned.  EINVAL on a null pointer, n_groups < 0 or a code
+ * outside {-1,0,+1} (out is then unspecified). */
+int scion_pack_pq2(const int8_t* codes, const uint16_t* scales, int64_t n_groups, uint8_t* out);
+int scion_pack_ptq1(const int8_t* codes, const uint16_t* scales, int64_t n_groups, uint8_t* out);
+
+/* Host unpacker, the inverse of the packers.  Invalid fields decode to code 0
+ * and the call returns SCION_EFORMAT after decoding everything. */
+int scion_unpack(int fmt, const uint8_t* in, int64_t n_groups, int8_t* codes, uint16_t* scales);
+
+/* Device packer: same contract as the host packers, all three pointers device
+ * memory, enqueued on `stream`.  A code outside {-1,0,+1} is packed as 0 and
+ * counted; if `bad_count` (device int64, may be NULL) is given, the number of
+ * such codes is ADDED to it. */
+int scion_pack_device(int fmt, const int8_t* codes, const uint16_t* scales, int64_t n_groups, uint8_t* out,
+                      int64_t* bad_count, void* stream);
+
+/* Device unpacker: inverse of scion_pack_device.  Invalid fields decode to 0;
+ * if `bad_count` (device int64, may be NULL) is given the number of invalid
+ * fields is ADDED to it. */
+int scion_unpack_device(int fmt, const uint8_t* in, int64_t n_groups, int8_t* codes, uint16_t* scales,
+                        int64_t* bad_count, void* stream);
+
+/* -------------------------------------------------------------------- layer
+ * One MoE block.  d = hidden size, E = experts, k = top-k, F = expert ffn,
+ * Fs = shared-expert ffn (0 = no shared expert), r = correction rank (0 = none).
+ * d and F must be multiples of 128; 1 <= k <= E <= 4096; Fs % 128 == 0;
+ * r % 16 == 0.
+ *
+ * Expert banks (device, packed blocks in `fmt`, groups of 128 along each row's
+ * reduction axis; [P3]/[P4] Weight Representation):
+ *   gate_exps, up_exps : [E][F][d/128] blocks     (rows = ffn units, K = d)
+ *   down_exps          : [E][d][F/128] blocks     (rows = hidden units, K = F)
+ * Router ([P1] The idea; [P3] Weight Representation): w_router and
+ * w_router_delta are [E][d], fp32 when router_fp32 = 1, else bf16; the logit of
+ * expert e is x.w_router[e] + x.w_router_delta[e].
+ * Shared expert ([P3]/[P4] Model Overview), bf16: sh_gate, sh_up [Fs][d];
+ * sh_down [d][Fs]; sh_gate_vec [d] or NULL (if given, the shared output is
+ * multiplied by sigmoid(x . sh_gate_vec)).
+ * Correction ([P1] The idea: rank-r branch on the MoE block output), bf16:
+ * corr_a [r][d], corr_b [d][r]; it adds corr_b (corr_a x) to the output, where x
+ * is the block input (the branch runs beside the block on the residual stream,
+ * scale 1).
+ * Gates: norm_topk = 1 -> softmax over the k selected logits; 0 -> the selected
+ * entries of a softmax over all E logits. */
+typedef struct {
+  int d, n_experts, top_k, ffn, shared_ffn, rank;
+  int fmt;         /* scion_fmt */
+  int router_fp32; /* 1: router and delta fp32; 0: bf16 */
+  int norm_topk;   /* 1 (default reading) or 0 */
+  const void* w_router;
+  const void* w_router_delta;
+  const void* gate_exps;
+  const void* up_exps;
+  const void* down_exps;
+  const void* sh_gate;
+  const void* sh_up;
+  const void* sh_down;
+  const void* sh_gate_vec;
+  const void* corr_a;
+  const void* corr_b;
+} scion_layer_desc;
+
+typedef struct scion_layer scion_layer;
+
+/* Builds a layer handle for batches of up to max_tokens tokens.
+ * Copies the expert banks into the device layout used by the kernels (same
+ * bytes per 128 weights, regrouped into 16-byte-aligned tiles), converts
+ * sh_down and corr_b to an fp16 copy, and allocates the workspace.  After it
+ * returns, the caller may free gate_exps / up_exps / down_exps / sh_down /
+ * corr_b; w_router, w_router_delta, sh_gate, sh_up, sh_gate_vec and corr_a are
+ * read in place and must outlive the handle.  Synchronises `stream` once to
+ * validate every code: SCION_EFORMAT if a block holds an invalid code (no
+ * handle is returned), EINVAL on a bad descriptor, ENOMEM, ECUDA. */
+int scion_layer_create(const scion_layer_desc* desc, int max_tokens, void* stream, scion_layer** out);
+
+/* Frees the handle and everything it allocated (synchronises the device). */
+void scion_layer_destroy(scion_layer* layer);
+
+/* Bytes of device memory owned by the handle (banks, fp16 copies, workspace). */
+size_t scion_layer_device_bytes(const scion_layer* layer);
+
+/* The block forward ([P1] The idea; [P3]/[P4] Model Overview):
+ *   out[t] = sum_{j<k} g_{t,j} E_{e(t,j)}(x_t) + S(x_t) + B (A x_t)
+ * with E_e(x) = W_d,e (silu(W_g,e x) * (W_u,e x)), S the shared expert and
+ * g, e(t, .) the gates and ids of the top-k router logits.
+ * x: device bf16 [T][d]; out: device fp32 [T][d], OVERWRITTEN (no residual add).
+ * 0 <= T <= max_tokens (T = 0 is a no-op).  Calls on one handle must not
+ * overlap on the GPU (they share its workspace): issue them on one stream.
+ * EINVAL on a null pointer or T out of range; ECUDA if a launch fails. */
+int scion_moe_forward(const void* x, int T, const scion_layer* layer, float* out, void* stream);
+
+/* Same forward with x and out in HOST memory (pinned for asynchronous copies):
+ * enqueues the host-to-device copy of x, the forward and the device-to-host copy
+ * of out on `stream`.  The caller synchronises the stream before reading out. */
+int scion_moe_forward_host(const void* x_host, int T, const scion_layer* layer, float* out_host, void* stream);
+
+/* Intermediate results of a forward, for tests and debugging.  Every pointer is
+ * device memory and may be NULL (not written). */
+typedef struct {
+  float* logits;    /* [T][E] router logits (fp32) */
+  int32_t* ids;     /* [T][k] selected experts, descending logit, ties -> lower id */
+  float* gates;     /* [T][k] gate weights */
+  int32_t* counts;  /* [E] tokens routed to each expert */
+  int32_t* offsets; /* [E+1] exclusive scan of counts */
+  int32_t* perm;    /* [T*k] entries t*k+j, grouped by expert, token order within an expert */
+  uint16_t* h;      /* fp16 [T*k][F] expert SwiGLU hidden, row p for perm[p] */
+  uint16_t* hz;     /* fp16 [T][Fs + r] shared SwiGLU hidden then correction z = A x */
+} scion_debug_out;
+
+/* scion_moe_forward, then copies the intermediates requested in `dbg`. */
+int scion_moe_forward_debug(const void* x, int T, const scion_layer* layer, float* out, const scion_debug_out* dbg,
+                            void* stream);
+
+/* ------------------------------------------------------------ measurement
+ * Kernel-level timing for benchmarks.  Between scion_profile_begin and
+ * scion_profile_end, every kernel a forward launches is bracketed by a pair of CUDA
+ * events recorded on the stream it is launched on, tagged with its stage:           */
+enum {
+  SCION_STAGE_ROUTER_F32 = 0,  /* fp32 router logits (FFMA) */
+  SCION_STAGE_XPROJ = 1,       /* bf16 router + delta, shared gate/up + SwiGLU, correction A */
+  SCION_STAGE_ROUTE = 2,       /* top-k, gates, histogram / scan / stable scatter */
+  SCION_STAGE_GATEUP = 3,      /* ternary expert gate/up + SwiGLU */
+  SCION_STAGE_DOWN_ROUTED = 4, /* ternary expert down + gate-weighted scatter-add */
+  SCION_STAGE_DOWN_DENSE = 5,  /* shared down + correction B */
+  SCION_N_STAGES = 6
+};
+/* Creates a pool for `max_launches` launches and starts recording (EINVAL if already
+ * recording or max_launches < 1).  Launches past the pool are not recorded.  Not
+ * thread-safe: one recording per process at a time. */
+int scion_profile_begin(int max_launches);
+/* Waits for the recorded events, stops recording, and writes per stage the summed
+ * device time in milliseconds and the number of recorded launches (arrays of
+ * n_stages entries, host memory).  Frees the pool. */
+int scion_profile_end(int n_stages, double* ms_total, int64_t* launches);
+/* Number of kernels the forward entry points have launched since the library loaded. */
+int64_t scion_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SCION_H */

@@ -1,0 +1,195 @@
+// k_route.cu -- router logits (fp32 routers), top-k gating and token-to-expert grouping.
+//
+// Router: logit[t][e] = x_t . W_r[e] + x_t . D[e] ("Scion: ternary MoE quantization with
+// trained corrections", The idea: router deltas; "Scion-35B-A3B" model card, Weight
+// Representation: routers stay F32).  Top-k: the k largest logits ("Scion-35B-A3B"
+// Model Overview: top-8 of 256; FlashNext Model Overview: top-10 of 512), ties to the
+// lower expert id; gates = softmax over the selected logits (or the selected entries
+// of a softmax over all E).  Grouping: histogram of the T*k ids, exclusive scan, and a
+// stable scatter in (token, slot) order -- the per-expert token lists that the expert
+// GEMMs consume ("Scion: ..." Serving notes: the expert matmul computes k experts per
+// token).
+#include <float.h>
+#include <math.h>
+
+#include "scion_internal.cuh"
+
+namespace scion {
+namespace {
+
+constexpr int kRouteThreads = 256;
+
+// One warp per (token, expert): FFMA in fp32 over d (no TF32).
+__global__ void router_f32_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ wr,
+                                  const float* __restrict__ wd, int d, int E, float* __restrict__ logits) {
+  int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int e = blockIdx.x * 8 + warp, t = blockIdx.y;
+  if (e >= E) return;
+  const __nv_bfloat16* xt = x + int64_t(t) * d;
+  const float* a = wr + int64_t(e) * d;
+  const float* b = wd + int64_t(e) * d;
+  float sa = 0.f, sb = 0.f;
+  for (int i = lane; i < d; i += 32) {
+    float xv = __bfloat162float(xt[i]);
+    sa = fmaf(xv, a[i], sa);
+    sb = fmaf(xv, b[i], sb);
+  }
+  for (int o = 16; o; o >>= 1) {
+    sa += __shfl_xor_sync(0xffffffffu, sa, o);
+    sb += __shfl_xor_sync(0xffffffffu, sb, o);
+  }
+  if (lane == 0) logits[int64_t(t) * E + e] = sa + sb;
+}
+
+__device__ __forceinline__ void argmax_merge(float& v, int& i, float v2, int i2) {
+  if (v2 > v || (v2 == v && i2 < i)) {
+    v = v2;
+    i = i2;
+  }
+}
+
+// Single CTA for one pass of T <= SCION_TDEC tokens.
+// smem: vals[8][E] f32 | counts[E] | cursor[E] | ids[T*k]
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                              int norm_topk, int32_t* __restrict__ ids_out,
+                                                              float* __restrict__ gates_out,
+                                                              int32_t* __restrict__ counts_out,
+                                                              int32_t* __restrict__ offsets_out,
+                                                              int32_t* __restrict__ perm_out,
+                                                              int32_t* __restrict__ active_out,
+                                                              int32_t* __restrict__ n_active_out) {
+  extern __shared__ float smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = kRouteThreads / 32;
+  float* vals = smem + warp * E;
+  int32_t* counts = reinterpret_cast<int32_t*>(smem + nwarps * E);
+  int32_t* cursor = counts + E;
+  int32_t* ids_s = cursor + E;
+
+  for (int e = threadIdx.x; e < E; e += kRouteThreads) counts[e] = 0;
+
+  // ---- top-k and gates, one warp per token
+  for (int t = warp; t < T; t += nwarps) {
+    const float* row = logits + int64_t(t) * E;
+    float mx = -INFINITY;
+    for (int e = lane; e < E; e += 32) {
+      // NaN / -inf rank below every finite logit but above "taken" (-inf), so each of the
+      // k rounds always selects an index in [0, E) that was not selected before.
+      float v = row[e];
+      if (!(v >= -FLT_MAX)) v = -FLT_MAX;
+      vals[e] = v;
+      mx = fmaxf(mx, v);
+    }
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float zall = 0.f;
+    if (!norm_topk) {
+      for (int e = lane; e < E; e += 32) zall += expf(vals[e] - mx);
+      for (int o = 16; o; o >>= 1) zall += __shfl_xor_sync(0xffffffffu, zall, o);
+    }
+    __syncwarp();
+    float my_v = -INFINITY;
+    int my_id = -1;
+    for (int j = 0; j < k; ++j) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int e = lane; e < E; e += 32) argmax_merge(bv, bi, vals[e], e);
+      for (int o = 16; o; o >>= 1) {
+        float v2 = __shfl_xor_sync(0xffffffffu, bv, o);
+        int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
+        argmax_merge(bv, bi, v2, i2);
+      }
+      if (lane == j) {
+        my_v = bv;
+        my_id = bi;
+      }
+      __syncwarp();
+      if (lane == (bi & 31)) vals[bi] = -INFINITY;
+      __syncwarp();
+    }
+    float top = __shfl_sync(0xffffffffu, my_v, 0);
+    float ex = 0.f;
+    if (lane < k) ex = norm_topk ? expf(my_v - top) : expf(my_v - mx);
+    float z = ex;
+    for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (!norm_topk) z = zall;
+    if (lane < k) {
+      ids_out[t * k + lane] = my_id;
+      gates_out[t * k + lane] = ex / z;
+      ids_s[t * k + lane] = my_id;
+      atomicAdd(&counts[my_id], 1);
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+
+  // ---- exclusive scan of counts and the active-expert list (warp 0)
+  if (warp == 0) {
+    const int per = (E + 31) / 32;
+    const int e0 = lane * per, e1 = min(E, e0 + per);
+    int s = 0, a = 0;
+    for (int e = e0; e < e1; ++e) {
+      s += counts[e];
+      a += counts[e] > 0;
+    }
+    int si = s, ai = a;
+    for (int o = 1; o < 32; o <<= 1) {
+      int s2 = __shfl_up_sync(0xffffffffu, si, o), a2 = __shfl_up_sync(0xffffffffu, ai, o);
+      if (lane >= o) {
+        si += s2;
+        ai += a2;
+      }
+    }
+    int run = si - s, arun = ai - a;
+    for (int e = e0; e < e1; ++e) {
+      int c = counts[e];
+      offsets_out[e] = run;
+      cursor[e] = run;
+      counts_out[e] = c;
+      if (c > 0) active_out[arun++] = e;
+      run += c;
+    }
+    if (lane == 31) {
+      offsets_out[E] = si;
+      *n_active_out = ai;
+    }
+    __syncwarp();
+    // ---- stable scatter in (token, slot) order, 32 entries at a time
+    const int n = T * k;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = 0; base < n; base += 32) {
+      int i = base + lane;
+      int e = i < n ? ids_s[i] : -1 - lane;  // unique dummies never match real ids
+      unsigned mask = __match_any_sync(0xffffffffu, e);
+      int rank = __popc(mask & lt);
+      int cur = i < n ? cursor[e] : 0;
+      __syncwarp();
+      if (i < n) {
+        perm_out[cur + rank] = i;
+        if (rank == 0) cursor[e] = cur + __popc(mask);
+      }
+      __syncwarp();
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_router_f32(const scion_layer* L, const __nv_bfloat16* x, int T, cudaStream_t s) {
+  dim3 grid((L->E + 7) / 8, T);
+  router_f32_kernel<<<grid, 256, 0, s>>>(x, static_cast<const float*>(L->desc.w_router),
+                                         static_cast<const float*>(L->desc.w_router_delta), L->d, L->E, L->logits);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s) {
+  size_t smem = sizeof(float) * (size_t(kRouteThreads / 32) * L->E) + sizeof(int32_t) * (2 * size_t(L->E)) +
+                sizeof(int32_t) * size_t(T) * L->k;
+  route_kernel<<<1, kRouteThreads, smem, s>>>(L->logits, T, L->E, L->k, L->desc.norm_topk, L->ids, L->gates,
+                                               L->counts, L->offsets, L->perm, L->active, L->n_active);
+  return cudaGetLastError();
+}
+
+cudaError_t configure_route_kernels() {
+  return cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+}
+
+}  // namespace scion

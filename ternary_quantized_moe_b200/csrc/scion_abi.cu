@@ -1,0 +1,323 @@
+// scion_abi.cu -- the extern "C" entry points of libscion (declared in include/scion.h).
+//
+// Everything here is argument checking, memory management and launch sequencing; the
+// arithmetic of the block runs in the kernels of k_route.cu and k_decode.cu.
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <atomic>
+#include <new>
+#include <vector>
+
+#include "scion_internal.cuh"
+
+namespace {
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SCION_OK;
+  if (e == cudaErrorMemoryAllocation) return SCION_ENOMEM;
+  return SCION_ECUDA;
+}
+
+#define SCION_TRY(expr)                 \
+  do {                                  \
+    cudaError_t e_ = (expr);            \
+    if (e_ != cudaSuccess) {            \
+      st = cuda_status(e_);             \
+      goto fail;                        \
+    }                                   \
+  } while (0)
+
+template <typename T>
+cudaError_t dev_alloc(scion_layer* L, T** p, size_t bytes) {
+  *p = nullptr;
+  if (bytes == 0) return cudaSuccess;
+  cudaError_t e = cudaMalloc(reinterpret_cast<void**>(p), bytes);
+  if (e == cudaSuccess) L->device_bytes += bytes;
+  return e;
+}
+
+void free_layer(scion_layer* L) {
+  if (!L) return;
+  void* ptrs[] = {L->gu_bank, L->dn_bank, L->dense_down, L->xunits,  L->logits, L->ids,      L->gates,
+                  L->counts,  L->offsets, L->perm,       L->active,  L->n_active, L->h,      L->hz,
+                  L->xfrag,   L->xpartial, L->xcount,    L->x_stage, L->out_stage, L->bad};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+  delete L;
+}
+
+int check_desc(const scion_layer_desc* D, int max_tokens) {
+  if (!D || max_tokens < 1) return SCION_EINVAL;
+  if (D->d <= 0 || D->d % 128 || D->ffn <= 0 || D->ffn % 128) return SCION_EINVAL;
+  if (D->n_experts < 1 || D->n_experts > 4096 || D->top_k < 1 || D->top_k > D->n_experts || D->top_k > 32)
+    return SCION_EINVAL;
+  if (D->shared_ffn < 0 || D->shared_ffn % 128 || D->rank < 0 || D->rank % 16) return SCION_EINVAL;
+  if (D->fmt != SCION_PQ2_0 && D->fmt != SCION_PTQ1_0) return SCION_EINVAL;
+  if ((D->router_fp32 != 0 && D->router_fp32 != 1) || (D->norm_topk != 0 && D->norm_topk != 1)) return SCION_EINVAL;
+  if (!D->w_router || !D->w_router_delta || !D->gate_exps || !D->up_exps || !D->down_exps) return SCION_EINVAL;
+  if (D->shared_ffn > 0 && (!D->sh_gate || !D->sh_up || !D->sh_down)) return SCION_EINVAL;
+  if (D->rank > 0 && (!D->corr_a || !D->corr_b)) return SCION_EINVAL;
+  if (D->sh_gate_vec) return SCION_EINVAL;  // shared-expert sigmoid gate: not supported by the kernels yet
+  return SCION_OK;
+}
+
+// ---- kernel timing for benchmarks (see scion_profile_begin in include/scion.h)
+struct Profiler {
+  bool on = false;
+  std::vector<cudaEvent_t> ev;  // 2 per launch
+  std::vector<int> stage;
+  int used = 0;
+};
+Profiler g_prof;
+std::atomic<long long> g_launches{0};
+
+struct StageScope {
+  cudaStream_t s;
+  bool rec = false;
+  StageScope(int stage, cudaStream_t st) : s(st) {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (g_prof.on && g_prof.used < int(g_prof.stage.size())) {
+      rec = true;
+      g_prof.stage[g_prof.used] = stage;
+      cudaEventRecord(g_prof.ev[2 * g_prof.used], s);
+    }
+  }
+  ~StageScope() {
+    if (rec) cudaEventRecord(g_prof.ev[2 * g_prof.used++ + 1], s);
+  }
+};
+
+#define SCION_STAGE(stage, call)                     \
+  do {                                               \
+    cudaError_t e_;                                  \
+    {                                                \
+      StageScope scope_(stage, s);                   \
+      e_ = (call);                                   \
+    }                                                \
+    if (e_ != cudaSuccess) return cuda_status(e_);   \
+  } while (0)
+
+// One pass of T <= SCION_TDEC tokens.
+int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, cudaStream_t s) {
+  if (L->desc.router_fp32) SCION_STAGE(SCION_STAGE_ROUTER_F32, scion::launch_router_f32(L, x, T, s));
+  SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_xproj(L, x, T, out, s));
+  SCION_STAGE(SCION_STAGE_ROUTE, scion::launch_route(L, T, s));
+  SCION_STAGE(SCION_STAGE_GATEUP, scion::launch_gateup(L, x, T, s));
+  SCION_STAGE(SCION_STAGE_DOWN_ROUTED, scion::launch_down_routed(L, T, out, s));
+  if (L->Kdense) SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
+  return SCION_OK;
+}
+
+}  // namespace
+
+extern "C" const char* scion_status_str(int status) {
+  switch (status) {
+    case SCION_OK: return "ok";
+    case SCION_EINVAL: return "invalid argument";
+    case SCION_ENOMEM: return "out of memory";
+    case SCION_ECUDA: return "CUDA error";
+    case SCION_EFORMAT: return "invalid code in a packed block";
+    case SCION_ETIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int scion_pack_device(int fmt, const int8_t* codes, const uint16_t* scales, int64_t n_groups, uint8_t* out,
+                                 int64_t* bad_count, void* stream) {
+  if ((fmt != SCION_PQ2_0 && fmt != SCION_PTQ1_0) || n_groups < 0) return SCION_EINVAL;
+  if (n_groups > 0 && (!codes || !scales || !out)) return SCION_EINVAL;
+  return cuda_status(scion::launch_pack(fmt, codes, scales, n_groups, out, bad_count, as_stream(stream)));
+}
+
+extern "C" int scion_unpack_device(int fmt, const uint8_t* in, int64_t n_groups, int8_t* codes, uint16_t* scales,
+                                   int64_t* bad_count, void* stream) {
+  if ((fmt != SCION_PQ2_0 && fmt != SCION_PTQ1_0) || n_groups < 0) return SCION_EINVAL;
+  if (n_groups > 0 && (!in || !codes || !scales)) return SCION_EINVAL;
+  return cuda_status(scion::launch_unpack(fmt, in, n_groups, codes, scales, bad_count, as_stream(stream)));
+}
+
+extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, void* stream, scion_layer** out) {
+  if (!out) return SCION_EINVAL;
+  *out = nullptr;
+  int st = check_desc(desc, max_tokens);
+  if (st != SCION_OK) return st;
+  scion_layer* L = new (std::nothrow) scion_layer;
+  if (!L) return SCION_ENOMEM;
+  memset(L, 0, sizeof(*L));
+  L->desc = *desc;
+  L->d = desc->d, L->E = desc->n_experts, L->k = desc->top_k, L->F = desc->ffn;
+  L->Fs = desc->shared_ffn, L->r = desc->rank, L->fmt = desc->fmt, L->max_tokens = max_tokens;
+  L->Gd = L->d / 128, L->GF = L->F / 128;
+  L->Kdense = L->Fs + L->r;
+  L->Kd = (L->Kdense + 31) / 32 * 32;
+  cudaStream_t s = as_stream(stream);
+  const int tb = scion::tile_bytes(L->fmt);
+  const int TD = SCION_TDEC;
+  std::vector<scion::XUnit> units;
+  int64_t bad_host = 0;
+
+  if (!desc->router_fp32)
+    for (int e0 = 0; e0 < L->E; e0 += 16) units.push_back({scion::kUnitRouter, e0});
+  for (int f0 = 0; f0 < L->Fs; f0 += 16) units.push_back({scion::kUnitSwiglu, f0});
+  for (int q0 = 0; q0 < L->r; q0 += 16) units.push_back({scion::kUnitPlain, q0});
+  L->n_xunits = int(units.size());
+  L->n_xchunks = (L->d + SCION_XPROJ_KC - 1) / SCION_XPROJ_KC;
+
+  SCION_TRY(scion::configure_kernels());
+  SCION_TRY(dev_alloc(L, &L->gu_bank, size_t(L->E) * (L->F / 128) * L->Gd * 2 * 8 * tb));
+  SCION_TRY(dev_alloc(L, &L->dn_bank, size_t(L->E) * (L->d / 128) * L->GF * 8 * tb));
+  SCION_TRY(dev_alloc(L, &L->dense_down, size_t(L->d) * L->Kd * sizeof(__half)));
+  SCION_TRY(dev_alloc(L, &L->xunits, sizeof(scion::XUnit) * (units.size() ? units.size() : 1)));
+  SCION_TRY(dev_alloc(L, &L->logits, sizeof(float) * TD * L->E));
+  SCION_TRY(dev_alloc(L, &L->ids, sizeof(int32_t) * TD * L->k));
+  SCION_TRY(dev_alloc(L, &L->gates, sizeof(float) * TD * L->k));
+  SCION_TRY(dev_alloc(L, &L->counts, sizeof(int32_t) * L->E));
+  SCION_TRY(dev_alloc(L, &L->offsets, sizeof(int32_t) * (L->E + 1)));
+  SCION_TRY(dev_alloc(L, &L->perm, sizeof(int32_t) * TD * L->k));
+  SCION_TRY(dev_alloc(L, &L->active, sizeof(int32_t) * L->E));
+  SCION_TRY(dev_alloc(L, &L->n_active, sizeof(int32_t)));
+  SCION_TRY(dev_alloc(L, &L->h, sizeof(__half) * TD * L->k * L->F));
+  SCION_TRY(dev_alloc(L, &L->hz, sizeof(__half) * TD * (L->Kd ? L->Kd : 1)));
+  SCION_TRY(dev_alloc(L, &L->xfrag, sizeof(__half) * TD * L->d));
+  SCION_TRY(dev_alloc(L, &L->xpartial, sizeof(float) * (L->n_xunits ? L->n_xunits : 1) * L->n_xchunks * 2 * 16 * TD));
+  SCION_TRY(dev_alloc(L, &L->xcount, sizeof(unsigned) * (L->n_xunits ? L->n_xunits : 1)));
+  SCION_TRY(dev_alloc(L, &L->x_stage, sizeof(__nv_bfloat16) * size_t(max_tokens) * L->d));
+  SCION_TRY(dev_alloc(L, &L->out_stage, sizeof(float) * size_t(max_tokens) * L->d));
+  SCION_TRY(dev_alloc(L, &L->bad, sizeof(int64_t)));
+
+  if (!units.empty())
+    SCION_TRY(cudaMemcpyAsync(L->xunits, units.data(), sizeof(scion::XUnit) * units.size(), cudaMemcpyHostToDevice, s));
+  SCION_TRY(cudaMemsetAsync(L->xcount, 0, sizeof(unsigned) * (L->n_xunits ? L->n_xunits : 1), s));
+  SCION_TRY(cudaMemsetAsync(L->hz, 0, sizeof(__half) * TD * (L->Kd ? L->Kd : 1), s));
+  SCION_TRY(cudaMemsetAsync(L->bad, 0, sizeof(int64_t), s));
+  if (L->Kd) {
+    SCION_TRY(cudaMemsetAsync(L->dense_down, 0, size_t(L->d) * L->Kd * sizeof(__half), s));
+    if (L->Fs)
+      SCION_TRY(scion::launch_bf16_to_f16_rows(static_cast<const __nv_bfloat16*>(desc->sh_down), L->d, L->Fs,
+                                               L->dense_down, L->Kd, s));
+    if (L->r)
+      SCION_TRY(scion::launch_bf16_to_f16_rows(static_cast<const __nv_bfloat16*>(desc->corr_b), L->d, L->r,
+                                               L->dense_down + L->Fs, L->Kd, s));
+  }
+  SCION_TRY(scion::launch_retile(L->fmt, static_cast<const uint8_t*>(desc->gate_exps), L->E, L->F, L->Gd, 2, 0,
+                                 L->gu_bank, L->bad, s));
+  SCION_TRY(scion::launch_retile(L->fmt, static_cast<const uint8_t*>(desc->up_exps), L->E, L->F, L->Gd, 2, 1,
+                                 L->gu_bank, L->bad, s));
+  SCION_TRY(scion::launch_retile(L->fmt, static_cast<const uint8_t*>(desc->down_exps), L->E, L->d, L->GF, 1, 0,
+                                 L->dn_bank, L->bad, s));
+  SCION_TRY(cudaMemcpyAsync(&bad_host, L->bad, sizeof(int64_t), cudaMemcpyDeviceToHost, s));
+  SCION_TRY(cudaStreamSynchronize(s));
+  if (bad_host != 0) {
+    st = SCION_EFORMAT;
+    goto fail;
+  }
+  *out = L;
+  return SCION_OK;
+fail:
+  free_layer(L);
+  return st;
+}
+
+extern "C" void scion_layer_destroy(scion_layer* layer) {
+  if (!layer) return;
+  cudaDeviceSynchronize();
+  free_layer(layer);
+}
+
+extern "C" size_t scion_layer_device_bytes(const scion_layer* layer) { return layer ? layer->device_bytes : 0; }
+
+extern "C" int scion_moe_forward(const void* x, int T, const scion_layer* L, float* out, void* stream) {
+  if (!L || T < 0 || T > L->max_tokens) return SCION_EINVAL;
+  if (T == 0) return SCION_OK;
+  if (!x || !out) return SCION_EINVAL;
+  cudaStream_t s = as_stream(stream);
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  for (int t0 = 0; t0 < T; t0 += SCION_TDEC) {
+    const int n = T - t0 < SCION_TDEC ? T - t0 : SCION_TDEC;
+    int st = forward_pass(L, xb + int64_t(t0) * L->d, n, out + int64_t(t0) * L->d, s);
+    if (st != SCION_OK) return st;
+  }
+  return SCION_OK;
+}
+
+extern "C" int scion_moe_forward_host(const void* x_host, int T, const scion_layer* L, float* out_host, void* stream) {
+  if (!L || T < 0 || T > L->max_tokens) return SCION_EINVAL;
+  if (T == 0) return SCION_OK;
+  if (!x_host || !out_host) return SCION_EINVAL;
+  cudaStream_t s = as_stream(stream);
+  cudaError_t e = cudaMemcpyAsync(L->x_stage, x_host, sizeof(__nv_bfloat16) * size_t(T) * L->d,
+                                  cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  int st = scion_moe_forward(L->x_stage, T, L, L->out_stage, stream);
+  if (st != SCION_OK) return st;
+  e = cudaMemcpyAsync(out_host, L->out_stage, sizeof(float) * size_t(T) * L->d, cudaMemcpyDeviceToHost, s);
+  return cuda_status(e);
+}
+
+extern "C" int scion_moe_forward_debug(const void* x, int T, const scion_layer* L, float* out,
+                                       const scion_debug_out* dbg, void* stream) {
+  if (!L || !dbg || T < 0 || T > L->max_tokens || T > SCION_TDEC) return SCION_EINVAL;
+  int st = scion_moe_forward(x, T, L, out, stream);
+  if (st != SCION_OK || T == 0) return st;
+  cudaStream_t s = as_stream(stream);
+  cudaError_t e = cudaSuccess;
+  auto cp = [&](void* dst, const void* src, size_t bytes) {
+    if (dst && e == cudaSuccess) e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s);
+  };
+  cp(dbg->logits, L->logits, sizeof(float) * size_t(T) * L->E);
+  cp(dbg->ids, L->ids, sizeof(int32_t) * size_t(T) * L->k);
+  cp(dbg->gates, L->gates, sizeof(float) * size_t(T) * L->k);
+  cp(dbg->counts, L->counts, sizeof(int32_t) * size_t(L->E));
+  cp(dbg->offsets, L->offsets, sizeof(int32_t) * size_t(L->E + 1));
+  cp(dbg->perm, L->perm, sizeof(int32_t) * size_t(T) * L->k);
+  if (dbg->h && e == cudaSuccess)
+    e = scion::launch_unfrag(L->fmt, L->h, T * L->k, L->GF, reinterpret_cast<__half*>(dbg->h), s);
+  if (dbg->hz && e == cudaSuccess && L->Kdense)
+    e = cudaMemcpy2DAsync(dbg->hz, sizeof(__half) * L->Kdense, L->hz, sizeof(__half) * L->Kd,
+                          sizeof(__half) * L->Kdense, T, cudaMemcpyDeviceToDevice, s);
+  return cuda_status(e);
+}
+
+extern "C" int scion_profile_begin(int max_launches) {
+  if (g_prof.on || max_launches < 1) return SCION_EINVAL;
+  g_prof.ev.assign(size_t(2) * max_launches, nullptr);
+  g_prof.stage.assign(size_t(max_launches), -1);
+  for (auto& e : g_prof.ev) {
+    cudaError_t err = cudaEventCreate(&e);
+    if (err != cudaSuccess) {
+      for (auto& f : g_prof.ev)
+        if (f) cudaEventDestroy(f);
+      g_prof.ev.clear();
+      g_prof.stage.clear();
+      return cuda_status(err);
+    }
+  }
+  g_prof.used = 0;
+  g_prof.on = true;
+  return SCION_OK;
+}
+
+extern "C" int scion_profile_end(int n_stages, double* ms_total, int64_t* launches) {
+  if (!g_prof.on || n_stages < 0 || (n_stages > 0 && (!ms_total || !launches))) return SCION_EINVAL;
+  g_prof.on = false;
+  for (int i = 0; i < n_stages; ++i) ms_total[i] = 0.0, launches[i] = 0;
+  cudaError_t err = cudaSuccess;
+  if (g_prof.used > 0) err = cudaEventSynchronize(g_prof.ev[2 * g_prof.used - 1]);
+  for (int i = 0; i < g_prof.used && err == cudaSuccess; ++i) {
+    float ms = 0.f;
+    err = cudaEventElapsedTime(&ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]);
+    int st = g_prof.stage[i];
+    if (err == cudaSuccess && st >= 0 && st < n_stages) ms_total[st] += ms, launches[st] += 1;
+  }
+  for (auto& e : g_prof.ev) cudaEventDestroy(e);
+  g_prof.ev.clear();
+  g_prof.stage.clear();
+  g_prof.used = 0;
+  return cuda_status(err);
+}
+
+extern "C" int64_t scion_kernel_launches(void) { return g_launches.load(); }

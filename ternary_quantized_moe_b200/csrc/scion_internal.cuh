@@ -1,0 +1,152 @@
+// scion_internal.cuh -- shared internals of libscion (not part of the ABI).
+//
+// Device layout of the ternary expert banks (built once by scion_layer_create):
+// every expert matrix [R rows][K] is cut into 16-row x 128-column tiles ("sub-tile
+// blocks").  A sub-tile block holds exactly the bytes of its sixteen 128-weight
+// container blocks, regrouped so that lane L = 4*r + c of a warp (r = L/4 in 0..7,
+// c = L%4) finds what it needs for rows r and r+8 in one contiguous run:
+//
+//   PQ2_0, 544 B = 16 x 34:
+//     [16L + j]        row r,   code byte 8c + j   (j < 8)
+//     [16L + 8 + j]    row r+8, code byte 8c + j
+//     [512 + 4r + 0/2] fp16 scale of row r / row r+8
+//   PTQ1_0, 448 B = 16 x 28:
+//     [12L + m]        row r,   quintet byte 6c + m (m < 6)
+//     [12L + 6 + m]    row r+8, quintet byte 6c + m
+//     [384 + 4r + 0/1] row r: quintet byte 24 / tail byte 25
+//     [384 + 4r + 2/3] row r+8: quintet byte 24 / tail byte 25
+//     [416 + 4r + 0/2] fp16 scale of row r / row r+8
+//
+// Sub-tile blocks are ordered [expert][row/128][group][matrix][row%128/16] with
+// matrix = {gate, up} interleaved for the gate/up bank and a single matrix for the
+// down bank, so a 128-row x 128-column stage of either bank is one contiguous run.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/scion.h"
+
+#define SCION_TDEC 64         // tokens per decode pass (larger batches run in passes)
+#define SCION_XPROJ_KC 512    // K columns per x-projection CTA (4 warps x 128)
+
+namespace scion {
+
+constexpr int kPq2Block = 34;
+constexpr int kPtq1Block = 28;
+constexpr int kPq2Tile = 544;   // 16 rows x 34 B
+constexpr int kPtq1Tile = 448;  // 16 rows x 28 B
+
+__host__ __device__ inline int tile_bytes(int fmt) { return fmt == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile; }
+__host__ __device__ inline int block_bytes(int fmt) { return fmt == SCION_PQ2_0 ? kPq2Block : kPtq1Block; }
+
+// x-projection work unit: 16 output rows of one kind.
+enum UnitKind : int { kUnitRouter = 0, kUnitSwiglu = 1, kUnitPlain = 2 };
+struct XUnit {
+  int kind;
+  int row0;  // first row of the unit within its matrices
+};
+
+}  // namespace scion
+
+struct scion_layer {
+  scion_layer_desc desc;
+  int d, E, k, F, Fs, r, fmt, max_tokens;
+  int Gd, GF;       // 128-groups along d and along F
+  int Kdense;       // Fs + r
+  int Kd;           // Kdense rounded up to 32: row stride of dense_down and hz (pad = 0)
+  // owned device memory
+  uint8_t* gu_bank;    // [E][F/128][Gd][2][8][tile]
+  uint8_t* dn_bank;    // [E][d/128][GF][8][tile]
+  __half* dense_down;  // [d][Kd] fp16: sh_down | corr_b | 0
+  scion::XUnit* xunits;
+  int n_xunits;
+  int n_xchunks;
+  // workspace (sized for SCION_TDEC tokens per pass, max_tokens for staging)
+  float* logits;     // [TDEC][E]
+  int32_t* ids;      // [TDEC][k]
+  float* gates;      // [TDEC][k]
+  int32_t* counts;   // [E]
+  int32_t* offsets;  // [E+1]
+  int32_t* perm;     // [TDEC*k]
+  int32_t* active;   // [E]
+  int32_t* n_active; // [1]
+  __half* h;         // [TDEC*k][F]
+  __half* hz;        // [TDEC][Kd] (pad columns stay 0)
+  __half* xfrag;     // [TDEC][Gd][128] x in fragment order (fp16)
+  float* xpartial;   // [n_xunits][n_xchunks][2][16][TDEC]
+  unsigned* xcount;  // [n_xunits]
+  void* x_stage;     // [max_tokens][d] bf16 (host-buffer forward)
+  float* out_stage;  // [max_tokens][d]
+  int64_t* bad;      // [1] invalid-code counter used at create
+  size_t device_bytes;
+};
+
+namespace scion {
+
+// ---------------------------------------------------------------- launchers
+// k_format.cu
+cudaError_t launch_pack(int fmt, const int8_t* codes, const uint16_t* scales, int64_t n_groups, uint8_t* out,
+                        int64_t* bad, cudaStream_t s);
+cudaError_t launch_unpack(int fmt, const uint8_t* in, int64_t n_groups, int8_t* codes, uint16_t* scales,
+                          int64_t* bad, cudaStream_t s);
+// Re-tile a packed bank [E][R][G] blocks into sub-tile blocks; `nmat`/`mat` select
+// the matrix slot of the interleaved gate/up bank (nmat = 1 for the down bank).
+cudaError_t launch_retile(int fmt, const uint8_t* src, int E, int R, int G, int nmat, int mat, uint8_t* dst,
+                          int64_t* bad, cudaStream_t s);
+cudaError_t launch_bf16_to_f16_rows(const __nv_bfloat16* src, int rows, int cols, __half* dst, int ld_dst,
+                                    cudaStream_t s);
+
+// k_route.cu
+cudaError_t launch_router_f32(const scion_layer* L, const __nv_bfloat16* x, int T, cudaStream_t s);
+cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s);
+cudaError_t configure_route_kernels();
+
+// k_decode.cu
+cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, cudaStream_t s);
+cudaError_t launch_gateup(const scion_layer* L, const __nv_bfloat16* x, int T, cudaStream_t s);
+cudaError_t launch_down_routed(const scion_layer* L, int T, float* out, cudaStream_t s);
+cudaError_t launch_down_dense(const scion_layer* L, int T, float* out, cudaStream_t s);
+// fragment-ordered rows [rows][G][128] -> natural order [rows][G*128]
+cudaError_t launch_unfrag(int fmt, const __half* src, int rows, int G, __half* dst, cudaStream_t s);
+cudaError_t configure_kernels();
+
+// ------------------------------------------------------------ device helpers
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_f16_1688(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
+__device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
+  // (a & mask) | magic in one LOP3
+  uint32_t r;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n" : "=r"(r) : "r"(a), "r"(mask), "r"(magic));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+
+}  // namespace scion

@@ -85,3 +85,44 @@ def bf16(bits: np.ndarray) -> np.ndarray:
 
     t = torch.from_numpy(np.ascontiguousarray(bits, np.uint16).view(np.int16)).view(torch.bfloat16)
     return t.double().numpy()
+
+
+# ------------------------------------------------------------ device layers
+def packed_banks(cfg: synth.Config, L: dict) -> dict:
+    """Expert banks packed by the oracle's packer (the bytes both sides consume)."""
+    return {n: oracle.pack(cfg.fmt, L[n + "_codes"], L[n + "_scales"]) for n in ("gate", "up", "down")}
+
+
+def oracle_layer_packed(cfg: synth.Config, L: dict, banks: dict, **kw) -> oracle.OracleLayer:
+    return oracle.OracleLayer(
+        d=cfg.d, n_experts=cfg.n_experts, top_k=cfg.top_k, ffn=cfg.ffn, fmt=cfg.fmt,
+        w_router=L["w_router"], w_delta=L["w_delta"], gate_exps=banks["gate"], up_exps=banks["up"],
+        down_exps=banks["down"], shared_ffn=cfg.shared_ffn, sh_gate=L.get("sh_gate"), sh_up=L.get("sh_up"),
+        sh_down=L.get("sh_down"), rank=cfg.rank, corr_a=L.get("corr_a"), corr_b=L.get("corr_b"), **kw)
+
+
+def u16_to_dev(a, dtype, dev):
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(dtype).to(dev)
+
+
+def device_layer(cfg: synth.Config, L: dict, banks: dict, max_tokens: int, dev="cuda", norm_topk: int = 1):
+    import torch
+
+    import ternary_quantized_moe_b200 as tq
+
+    bf = torch.bfloat16
+    if L["w_router"].dtype == np.float32:
+        wr = torch.from_numpy(L["w_router"]).to(dev)
+        wd = torch.from_numpy(L["w_delta"]).to(dev)
+    else:
+        wr = u16_to_dev(L["w_router"], bf, dev)
+        wd = u16_to_dev(L["w_delta"], bf, dev)
+    opt = lambda n: u16_to_dev(L[n], bf, dev) if n in L else None  # noqa: E731
+    return tq.scion_layer_create(
+        d=cfg.d, n_experts=cfg.n_experts, top_k=cfg.top_k, ffn=cfg.ffn, fmt=cfg.fmt, w_router=wr, w_router_delta=wd,
+        gate_exps=torch.from_numpy(banks["gate"]).to(dev), up_exps=torch.from_numpy(banks["up"]).to(dev),
+        down_exps=torch.from_numpy(banks["down"]).to(dev), shared_ffn=cfg.shared_ffn, sh_gate=opt("sh_gate"),
+        sh_up=opt("sh_up"), sh_down=opt("sh_down"), rank=cfg.rank, corr_a=opt("corr_a"), corr_b=opt("corr_b"),
+        norm_topk=norm_topk, max_tokens=max_tokens)

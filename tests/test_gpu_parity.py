@@ -1,0 +1,287 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same
+seeded inputs.  Integer work (packing, routing ids, counts, offsets, the grouping
+permutation) must match bit for bit; floating-point outputs must meet the block
+tolerance (per-token relative L2 <= 1e-3, max-abs <= 5e-3 * max|ref|)."""
+import numpy as np
+import pytest
+
+import oracle
+from tests.helpers import (check_output, device_layer, oracle_layer_packed, packed_banks, u16_to_dev,
+                           with_margin)
+from workloads import synth
+
+torch = pytest.importorskip("torch")
+import ternary_quantized_moe_b200 as tq  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def small(name, fmt, router_f32, E=16, k=4, d=256, F=128, Fs=128, r=16, index=20):
+    return synth.Config(name, index, d, E, k, F, Fs, fmt, r, router_f32, [8], 1)
+
+
+def run_forward(layer, x_u16, T, debug=False, E=None, k=None, F=None, Kdense=None):
+    x = u16_to_dev(x_u16, torch.bfloat16, DEV)
+    out = torch.full((max(T, 1), layer.d), float("nan"), dtype=torch.float32, device=DEV)
+    bufs = {}
+    if debug:
+        bufs = dict(
+            logits=torch.empty((T, E), dtype=torch.float32, device=DEV),
+            ids=torch.empty((T, k), dtype=torch.int32, device=DEV),
+            gates=torch.empty((T, k), dtype=torch.float32, device=DEV),
+            counts=torch.empty((E,), dtype=torch.int32, device=DEV),
+            offsets=torch.empty((E + 1,), dtype=torch.int32, device=DEV),
+            perm=torch.empty((T * k,), dtype=torch.int32, device=DEV),
+            h=torch.empty((T * k, F), dtype=torch.float16, device=DEV),
+        )
+        if Kdense:
+            bufs["hz"] = torch.empty((T, Kdense), dtype=torch.float16, device=DEV)
+        tq.scion_moe_forward_debug(x, T, layer, out, **bufs)
+    else:
+        tq.scion_moe_forward(x, T, layer, out)
+    torch.cuda.synchronize()
+    return out[:T].cpu().numpy().astype(np.float64), {k_: v.cpu().numpy() for k_, v in bufs.items()}
+
+
+# ------------------------------------------------------------------ formats
+@pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
+@pytest.mark.parametrize("n_groups", [1, 37, 1001])
+def test_device_pack_unpack_match_oracle(fmt, n_groups):
+    rng = np.random.default_rng(n_groups)
+    codes = rng.integers(-1, 2, size=(n_groups, 128)).astype(np.int8)
+    scales = rng.integers(0, 1 << 16, size=(n_groups, 1)).astype(np.uint16)
+    ref = oracle.pack(fmt, codes, scales)
+    dc = torch.from_numpy(codes).to(DEV)
+    ds = torch.from_numpy(scales.view(np.int16)).to(DEV)
+    bad = torch.zeros(1, dtype=torch.int64, device=DEV)
+    blocks = tq.scion_pack_device(fmt, dc, ds, bad_count=bad)
+    np.testing.assert_array_equal(blocks.cpu().numpy(), ref)
+    assert int(bad.item()) == 0
+    c2, s2 = tq.scion_unpack_device(fmt, torch.from_numpy(ref).to(DEV), bad_count=bad)
+    np.testing.assert_array_equal(c2.cpu().numpy(), codes)
+    np.testing.assert_array_equal(s2.cpu().numpy().view(np.uint16), scales)
+    assert int(bad.item()) == 0
+
+
+@pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
+def test_device_unpack_counts_invalid_codes(fmt):
+    blk = oracle.pack(fmt, np.zeros((4, 128), np.int8), np.zeros((4, 1), np.uint16))
+    blk[1, 0] = 0xFF  # PQ2: four fields of 3; PTQ1: one quintet byte above 242
+    if fmt == synth.PTQ1_0:
+        blk[2, 25] = 27  # tail byte above 26
+    bad = torch.zeros(1, dtype=torch.int64, device=DEV)
+    codes, _ = tq.scion_unpack_device(fmt, torch.from_numpy(blk).to(DEV), bad_count=bad)
+    ref_codes, _, st = oracle.unpack(fmt, blk)
+    assert st == oracle.EFORMAT
+    np.testing.assert_array_equal(codes.cpu().numpy(), ref_codes)
+    assert int(bad.item()) == (4 if fmt == synth.PQ2_0 else 2)
+
+
+def test_device_pack_counts_out_of_range_codes():
+    codes = np.zeros((2, 128), np.int8)
+    codes[0, 5] = 3
+    codes[1, 7] = -4
+    bad = torch.zeros(1, dtype=torch.int64, device=DEV)
+    tq.scion_pack_device(synth.PQ2_0, torch.from_numpy(codes).to(DEV),
+                         torch.zeros((2, 1), dtype=torch.int16, device=DEV), bad_count=bad)
+    assert int(bad.item()) == 2
+
+
+@pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
+def test_create_rejects_invalid_bank(fmt):
+    cfg = small("bad", fmt, False)
+    L = synth.layer_host(cfg)
+    banks = packed_banks(cfg, L)
+    banks["down"] = banks["down"].copy()
+    banks["down"][3, 17, 5] = 0xFF
+    with pytest.raises(tq.ScionError) as ei:
+        device_layer(cfg, L, banks, 8)
+    assert ei.value.status == tq.SCION_EFORMAT
+
+
+# ------------------------------------------------------------------ forward
+def _case(cfg, T, norm_topk=1, stream=0):
+    L = synth.layer_host(cfg)
+    banks = packed_banks(cfg, L)
+    ol = oracle_layer_packed(cfg, L, banks, norm_topk=norm_topk)
+    x = synth.x_host(cfg, T, stream)
+    if T:
+        x = with_margin(cfg, ol, x)
+    return L, banks, ol, x
+
+
+def _check_routing(cfg, dbg, ol, x, T):
+    E, k = cfg.n_experts, cfg.top_k
+    logits, ids, gates = oracle.route(ol, x)
+    np.testing.assert_allclose(dbg["logits"], logits, rtol=0, atol=2e-4 * max(1.0, np.abs(logits).max()))
+    np.testing.assert_array_equal(np.sort(dbg["ids"], 1), np.sort(ids, 1))
+    # gates per (token, expert)
+    for t in range(T):
+        ref = dict(zip(ids[t].tolist(), gates[t].tolist()))
+        for j in range(k):
+            assert abs(dbg["gates"][t, j] - ref[int(dbg["ids"][t, j])]) <= 1e-5 * max(1e-3, ref[int(dbg["ids"][t, j])])
+    counts, offsets, perm = oracle.group(ids, E)
+    np.testing.assert_array_equal(dbg["counts"], counts)
+    np.testing.assert_array_equal(dbg["offsets"], offsets)
+    # within each expert the tokens appear in increasing token order (unique); the slot
+    # part of each entry must point at that expert in the GPU's own ids
+    np.testing.assert_array_equal(dbg["perm"] // k, perm // k)
+    gp = dbg["perm"]
+    for e in range(E):
+        seg = gp[offsets[e]:offsets[e + 1]]
+        assert (dbg["ids"].reshape(-1)[seg] == e).all()
+    return ids
+
+
+def _check_hidden(cfg, dbg, ol, x, T):
+    """Expert SwiGLU hidden of every routed (token, expert) pair vs the oracle."""
+    k = cfg.top_k
+    worst = 0.0
+    for p, entry in enumerate(dbg["perm"]):
+        t, j = divmod(int(entry), k)
+        e = int(dbg["ids"][t, j])
+        h_ref, _ = oracle.expert(ol, e, x[t])
+        got = dbg["h"][p].astype(np.float64)
+        worst = max(worst, np.linalg.norm(got - h_ref) / max(np.linalg.norm(h_ref), 1e-30))
+    assert worst <= 1e-3, worst
+
+
+@pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
+@pytest.mark.parametrize("router_f32", [True, False])
+@pytest.mark.parametrize("T", [1, 5, 13])
+def test_forward_small_stagewise(fmt, router_f32, T):
+    cfg = small("s", fmt, router_f32)
+    L, banks, ol, x = _case(cfg, T)
+    layer = device_layer(cfg, L, banks, 64)
+    got, dbg = run_forward(layer, x, T, debug=True, E=cfg.n_experts, k=cfg.top_k, F=cfg.ffn,
+                           Kdense=cfg.shared_ffn + cfg.rank)
+    _check_routing(cfg, dbg, ol, x, T)
+    _check_hidden(cfg, dbg, ol, x, T)
+    hs, _ = oracle.shared(ol, x)
+    z, _ = oracle.corr(ol, x)
+    hz_ref = np.concatenate([hs, z], axis=1)
+    check_output(dbg["hz"].astype(np.float64), hz_ref, rel_l2=1e-3)
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
+
+
+@pytest.mark.parametrize("variant", ["tiny", "no_shared_no_corr", "norm_topk0", "k_eq_E", "E_not_mult16",
+                                     "wide_d", "ptq1_F384"])
+def test_forward_variants(variant):
+    T, norm_topk = 16, 1
+    if variant == "tiny":
+        cfg = synth.CONFIGS["tiny"]
+    elif variant == "no_shared_no_corr":
+        cfg = small("v", synth.PQ2_0, False, Fs=0, r=0)
+    elif variant == "norm_topk0":
+        cfg, norm_topk = small("v", synth.PTQ1_0, False), 0
+    elif variant == "k_eq_E":
+        cfg = small("v", synth.PQ2_0, True, E=4, k=4)
+    elif variant == "E_not_mult16":
+        cfg = small("v", synth.PTQ1_0, False, E=24, k=3)
+    elif variant == "wide_d":
+        cfg = small("v", synth.PQ2_0, False, d=1152, F=256, Fs=256, r=48, E=32, k=6)
+    else:
+        cfg = small("v", synth.PTQ1_0, False, d=384, F=384, Fs=384, r=32, E=16, k=2)
+    L, banks, ol, x = _case(cfg, T, norm_topk)
+    layer = device_layer(cfg, L, banks, 64, norm_topk=norm_topk)
+    got, dbg = run_forward(layer, x, T, debug=True, E=cfg.n_experts, k=cfg.top_k, F=cfg.ffn,
+                           Kdense=cfg.shared_ffn + cfg.rank)
+    _check_routing(cfg, dbg, ol, x, T)
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
+
+
+@pytest.mark.parametrize("T", [64, 65, 150])
+def test_forward_multi_pass(T):
+    """Batches above one decode pass (64 tokens) run in passes; ragged tails included."""
+    cfg = small("mp", synth.PTQ1_0, False, E=32, k=4)
+    L, banks, ol, x = _case(cfg, T)
+    layer = device_layer(cfg, L, banks, 160)
+    got, _ = run_forward(layer, x, T)
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
+
+
+def test_empty_batch_and_limits():
+    cfg = small("e", synth.PQ2_0, False)
+    L, banks, ol, x = _case(cfg, 4)
+    layer = device_layer(cfg, L, banks, 4)
+    out = torch.zeros((4, cfg.d), device=DEV)
+    xd = u16_to_dev(x, torch.bfloat16, DEV)
+    tq.scion_moe_forward(xd, 0, layer, out)
+    torch.cuda.synchronize()
+    assert float(out.abs().sum()) == 0.0
+    with pytest.raises(tq.ScionError) as ei:
+        tq.scion_moe_forward(xd, 5, layer, out)
+    assert ei.value.status == tq.SCION_EINVAL
+
+
+def test_host_buffer_forward_matches_device_forward():
+    cfg = small("h", synth.PQ2_0, False)
+    L, banks, ol, x = _case(cfg, 9)
+    layer = device_layer(cfg, L, banks, 16)
+    got_dev, _ = run_forward(layer, x, 9)
+    xh = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    oh = torch.empty((9, cfg.d), dtype=torch.float32).pin_memory()
+    tq.scion_moe_forward_host(xh, 9, layer, oh)
+    torch.cuda.synchronize()
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(oh.numpy().astype(np.float64), ref)
+    check_output(got_dev, ref)
+
+
+def test_repeated_calls_are_stable():
+    """Back-to-back calls on one handle reuse the workspace (split-K counters reset)."""
+    cfg = small("r", synth.PQ2_0, False, d=1024)
+    L, banks, ol, x = _case(cfg, 8)
+    layer = device_layer(cfg, L, banks, 8)
+    a, _ = run_forward(layer, x, 8)
+    for _ in range(3):
+        b, _ = run_forward(layer, x, 8)
+        check_output(b, a, rel_l2=1e-5, max_abs=1e-5)
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(a, ref)
+
+
+# ------------------------------------------------------------- full sizes
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["a3b_decode", "flashnext_decode"])
+def test_full_size_decode(name):
+    """One full layer of the decode shapes, every batch size the workload uses, all tokens."""
+    cfg = synth.CONFIGS[name]
+    L = synth.layer_host(cfg)
+    banks = packed_banks(cfg, L)
+    ol = oracle_layer_packed(cfg, L, banks)
+    layer = device_layer(cfg, L, banks, max(cfg.tokens))
+    del banks
+    for T in cfg.tokens:
+        x = with_margin(cfg, ol, synth.x_host(cfg, T))
+        got, dbg = run_forward(layer, x, T, debug=True, E=cfg.n_experts, k=cfg.top_k, F=cfg.ffn,
+                               Kdense=cfg.shared_ffn + cfg.rank)
+        _check_routing(cfg, dbg, ol, x, T)
+        ref, _, _ = oracle.forward(ol, x)
+        check_output(got, ref)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,n_sample", [("a3b_prefill", 256), ("flashnext_prefill", 256)])
+def test_full_size_prefill_sampled(name, n_sample):
+    """Full prefill batch on the GPU; the oracle checks a seeded sample of tokens (tokens are
+    independent, so the sampled rows of the GPU output must equal the oracle's rows)."""
+    cfg = synth.CONFIGS[name]
+    T = cfg.tokens[0]
+    L = synth.layer_host(cfg)
+    banks = packed_banks(cfg, L)
+    ol = oracle_layer_packed(cfg, L, banks)
+    layer = device_layer(cfg, L, banks, T)
+    del banks
+    x = synth.x_host(cfg, T)
+    rng = np.random.default_rng(4242)
+    sample = np.sort(rng.choice(T, size=n_sample, replace=False))
+    x[sample] = with_margin(cfg, ol, x[sample])
+    got, _ = run_forward(layer, x, T)
+    assert np.isfinite(got).all()
+    ref, _, _ = oracle.forward(ol, x[sample])
+    check_output(got[sample], ref)
