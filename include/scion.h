@@ -150,10 +150,17 @@ size_t scion_layer_device_bytes(const scion_layer* layer);
  * with E_e(x) = W_d,e (silu(W_g,e x) * (W_u,e x)), S the shared expert and
  * g, e(t, .) the gates and ids of the top-k router logits.
  * x: device bf16 [T][d]; out: device fp32 [T][d], OVERWRITTEN (no residual add).
- * 0 <= T <= max_tokens (T = 0 is a no-op).  Calls on one handle must not
+ * 0 <= T <= max_tokens (T = 0 is a no-op).  Batches of at most 64 tokens stream the
+ * weights through warp-level MMA kernels; larger batches (layers created with
+ * max_tokens > 64) run as tcgen05 grouped GEMMs.  Calls on one handle must not
  * overlap on the GPU (they share its workspace): issue them on one stream.
  * EINVAL on a null pointer or T out of range; ECUDA if a launch fails. */
 int scion_moe_forward(const void* x, int T, const scion_layer* layer, float* out, void* stream);
+
+/* Waits for `stream`, then returns the layer's device status word and clears it:
+ * SCION_ETIMEOUT if a tensor-core kernel of an earlier forward gave up a bounded wait
+ * (its outputs are then invalid), SCION_ECUDA on an asynchronous CUDA fault, else OK. */
+int scion_layer_check(const scion_layer* layer, void* stream);
 
 /* Same forward with x and out in HOST memory (pinned for asynchronous copies):
  * enqueues the host-to-device copy of x, the forward and the device-to-host copy
@@ -188,7 +195,8 @@ enum {
   SCION_STAGE_GATEUP = 3,      /* ternary expert gate/up + SwiGLU */
   SCION_STAGE_DOWN_ROUTED = 4, /* ternary expert down + gate-weighted scatter-add */
   SCION_STAGE_DOWN_DENSE = 5,  /* shared down + correction B */
-  SCION_N_STAGES = 6
+  SCION_STAGE_X16 = 6,         /* x -> fp16 in container column order (tensor-core path) */
+  SCION_N_STAGES = 7
 };
 /* Creates a pool for `max_launches` launches and starts recording (EINVAL if already
  * recording or max_launches < 1).  Launches past the pool are not recorded.  Not

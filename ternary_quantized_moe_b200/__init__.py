@@ -25,7 +25,7 @@ __all__ = [
     "scion_pack_pq2", "scion_pack_ptq1", "scion_unpack", "scion_pack_device", "scion_unpack_device",
     "scion_layer_create", "scion_layer_destroy", "scion_layer_device_bytes", "scion_moe_forward",
     "scion_moe_forward_host", "scion_moe_forward_debug", "Layer", "library_path", "EXPORTS",
-    "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "STAGES",
+    "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "STAGES", "scion_layer_check",
 ]
 
 SCION_PQ2_0 = 0
@@ -42,9 +42,9 @@ EXPORTS = (
     "scion_block_bytes", "scion_status_str", "scion_pack_pq2", "scion_pack_ptq1", "scion_unpack",
     "scion_pack_device", "scion_unpack_device", "scion_layer_create", "scion_layer_destroy",
     "scion_layer_device_bytes", "scion_moe_forward", "scion_moe_forward_host", "scion_moe_forward_debug",
-    "scion_profile_begin", "scion_profile_end", "scion_kernel_launches",
+    "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "scion_layer_check",
 )
-STAGES = ("router_f32", "xproj", "route", "gateup", "down_routed", "down_dense")
+STAGES = ("router_f32", "xproj", "route", "gateup", "down_routed", "down_dense", "x16")
 
 
 class ScionError(RuntimeError):
@@ -100,6 +100,7 @@ def _load():
             "scion_profile_begin": (ci, [ci]),
             "scion_profile_end": (ci, [ci, C.POINTER(C.c_double), C.POINTER(C.c_int64)]),
             "scion_kernel_launches": (C.c_int64, []),
+            "scion_layer_check": (ci, [vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -276,6 +277,11 @@ def scion_layer_destroy(layer: Layer) -> None:
         _load().scion_layer_destroy(C.c_void_p(layer.handle))
         layer.handle = 0
         layer._keep = {}
+
+
+def scion_layer_check(layer: Layer, stream=None) -> int:
+    """Waits for the stream and returns (and clears) the layer's device status word."""
+    return int(_load().scion_layer_check(C.c_void_p(layer.handle), _stream(stream)))
 
 
 def scion_layer_device_bytes(layer: Layer) -> int:

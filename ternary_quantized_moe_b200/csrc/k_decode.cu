@@ -648,6 +648,9 @@ cudaError_t launch_unfrag(int fmt, const __half* src, int rows, int G, __half* d
   return cudaGetLastError();
 }
 
-cudaError_t configure_kernels() { return configure_route_kernels(); }
+cudaError_t configure_kernels() {
+  cudaError_t e = configure_route_kernels();
+  return e != cudaSuccess ? e : configure_prefill_kernels();
+}
 
 }  // namespace scion

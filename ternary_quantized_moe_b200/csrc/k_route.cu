@@ -173,10 +173,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
 
 }  // namespace
 
-cudaError_t launch_router_f32(const scion_layer* L, const __nv_bfloat16* x, int T, cudaStream_t s) {
+cudaError_t launch_router_f32(const scion_layer* L, const __nv_bfloat16* x, int T, float* logits, cudaStream_t s) {
   dim3 grid((L->E + 7) / 8, T);
   router_f32_kernel<<<grid, 256, 0, s>>>(x, static_cast<const float*>(L->desc.w_router),
-                                         static_cast<const float*>(L->desc.w_router_delta), L->d, L->E, L->logits);
+                                         static_cast<const float*>(L->desc.w_router_delta), L->d, L->E, logits);
   return cudaGetLastError();
 }
 

@@ -44,10 +44,68 @@ void free_layer(scion_layer* L) {
   if (!L) return;
   void* ptrs[] = {L->gu_bank, L->dn_bank, L->dense_down, L->xunits,  L->logits, L->ids,      L->gates,
                   L->counts,  L->offsets, L->perm,       L->active,  L->n_active, L->h,      L->hz,
-                  L->xfrag,   L->xpartial, L->xcount,    L->x_stage, L->out_stage, L->bad};
+                  L->xfrag,   L->xpartial, L->xcount,    L->x_stage, L->out_stage, L->bad,   L->err};
   for (void* p : ptrs)
     if (p) cudaFree(p);
+  if (L->pre) {
+    scion::PrefillState* P = L->pre;
+    void* pp[] = {P->xunits, P->dunits, P->logits, P->ids, P->gates, P->counts, P->offsets,
+                  P->perm,   P->tiles,  P->n_tiles, P->x16, P->h,    P->hz};
+    for (void* p : pp)
+      if (p) cudaFree(p);
+    delete P;
+  }
   delete L;
+}
+
+// Buffers, unit tables and tensor maps of the tensor-core path (batches > SCION_TDEC).
+int create_prefill(scion_layer* L, cudaStream_t s) {
+  if (L->E > 2048) return SCION_EINVAL;  // grouping keeps one histogram row per warp in shared memory
+  scion::PrefillState* P = new (std::nothrow) scion::PrefillState;
+  if (!P) return SCION_ENOMEM;
+  memset(P, 0, sizeof(*P));
+  L->pre = P;
+  const size_t T = L->max_tokens, Tk = T * L->k;
+  const size_t max_tiles = (Tk + 127) / 128 + L->E;
+  cudaError_t e;
+#define PTRY(x)                              \
+  if ((e = (x)) != cudaSuccess) return cuda_status(e)
+  PTRY(dev_alloc(L, &P->logits, sizeof(float) * T * L->E));
+  PTRY(dev_alloc(L, &P->ids, sizeof(int32_t) * Tk));
+  PTRY(dev_alloc(L, &P->gates, sizeof(float) * Tk));
+  PTRY(dev_alloc(L, &P->counts, sizeof(int32_t) * L->E));
+  PTRY(dev_alloc(L, &P->offsets, sizeof(int32_t) * (L->E + 1)));
+  PTRY(dev_alloc(L, &P->perm, sizeof(int32_t) * Tk));
+  PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->tiles), scion::prefill_tile_bytes() * max_tiles));
+  PTRY(dev_alloc(L, &P->n_tiles, sizeof(int32_t)));
+  PTRY(dev_alloc(L, &P->x16, sizeof(__half) * T * L->d));
+  PTRY(dev_alloc(L, &P->h, sizeof(__half) * Tk * L->F));
+  PTRY(dev_alloc(L, &P->hz, sizeof(__half) * T * (L->Kd ? L->Kd : 64)));
+  PTRY(cudaMemsetAsync(P->hz, 0, sizeof(__half) * T * (L->Kd ? L->Kd : 64), s));
+  const int max_units = scion::prefill_max_units(L);
+  std::vector<uint8_t> xu(scion::prefill_unit_bytes() * max_units), du(scion::prefill_unit_bytes() * max_units);
+  scion::prefill_units(L, xu.data(), &P->n_xunits, du.data(), &P->n_dunits);
+  PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->xunits), scion::prefill_unit_bytes() * max_units));
+  PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->dunits), scion::prefill_unit_bytes() * max_units));
+  PTRY(cudaMemcpyAsync(P->xunits, xu.data(), xu.size(), cudaMemcpyHostToDevice, s));
+  PTRY(cudaMemcpyAsync(P->dunits, du.data(), du.size(), cudaMemcpyHostToDevice, s));
+#undef PTRY
+  int st;
+  const scion_layer_desc& D = L->desc;
+  if (!D.router_fp32) {
+    if ((st = scion::make_tmap_2d(&P->maps[0], D.w_router, 1, L->E, L->d))) return st;
+    if ((st = scion::make_tmap_2d(&P->maps[1], D.w_router_delta, 1, L->E, L->d))) return st;
+  }
+  if (L->Fs) {
+    if ((st = scion::make_tmap_2d(&P->maps[2], D.sh_gate, 1, L->Fs, L->d))) return st;
+    if ((st = scion::make_tmap_2d(&P->maps[3], D.sh_up, 1, L->Fs, L->d))) return st;
+  }
+  if (L->r && (st = scion::make_tmap_2d(&P->maps[4], D.corr_a, 1, L->r, L->d))) return st;
+  if (L->Kd) {
+    if ((st = scion::make_tmap_2d(&P->maps[5], L->dense_down, 0, L->d, L->Kd))) return st;
+    if ((st = scion::make_tmap_2d(&P->hz_map, P->hz, 0, L->max_tokens, L->Kd))) return st;
+  }
+  return SCION_OK;
 }
 
 int check_desc(const scion_layer_desc* D, int max_tokens) {
@@ -101,9 +159,22 @@ struct StageScope {
     if (e_ != cudaSuccess) return cuda_status(e_);   \
   } while (0)
 
+// Whole batch on the tensor-core path (T > SCION_TDEC).
+int forward_prefill(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, cudaStream_t s) {
+  if (L->desc.router_fp32)
+    SCION_STAGE(SCION_STAGE_ROUTER_F32, scion::launch_router_f32(L, x, T, L->pre->logits, s));
+  SCION_STAGE(SCION_STAGE_X16, scion::launch_prefill_stage(SCION_STAGE_X16, L, x, T, out, s));
+  SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_prefill_stage(SCION_STAGE_XPROJ, L, x, T, out, s));
+  SCION_STAGE(SCION_STAGE_ROUTE, scion::launch_prefill_stage(SCION_STAGE_ROUTE, L, x, T, out, s));
+  SCION_STAGE(SCION_STAGE_GATEUP, scion::launch_prefill_stage(SCION_STAGE_GATEUP, L, x, T, out, s));
+  SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_prefill_stage(SCION_STAGE_DOWN_DENSE, L, x, T, out, s));
+  SCION_STAGE(SCION_STAGE_DOWN_ROUTED, scion::launch_prefill_stage(SCION_STAGE_DOWN_ROUTED, L, x, T, out, s));
+  return SCION_OK;
+}
+
 // One pass of T <= SCION_TDEC tokens.
 int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, cudaStream_t s) {
-  if (L->desc.router_fp32) SCION_STAGE(SCION_STAGE_ROUTER_F32, scion::launch_router_f32(L, x, T, s));
+  if (L->desc.router_fp32) SCION_STAGE(SCION_STAGE_ROUTER_F32, scion::launch_router_f32(L, x, T, L->logits, s));
   SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_xproj(L, x, T, out, s));
   SCION_STAGE(SCION_STAGE_ROUTE, scion::launch_route(L, T, s));
   SCION_STAGE(SCION_STAGE_GATEUP, scion::launch_gateup(L, x, T, s));
@@ -153,7 +224,7 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   L->Fs = desc->shared_ffn, L->r = desc->rank, L->fmt = desc->fmt, L->max_tokens = max_tokens;
   L->Gd = L->d / 128, L->GF = L->F / 128;
   L->Kdense = L->Fs + L->r;
-  L->Kd = (L->Kdense + 31) / 32 * 32;
+  L->Kd = (L->Kdense + 63) / 64 * 64;
   cudaStream_t s = as_stream(stream);
   const int tb = scion::tile_bytes(L->fmt);
   const int TD = SCION_TDEC;
@@ -188,6 +259,8 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   SCION_TRY(dev_alloc(L, &L->x_stage, sizeof(__nv_bfloat16) * size_t(max_tokens) * L->d));
   SCION_TRY(dev_alloc(L, &L->out_stage, sizeof(float) * size_t(max_tokens) * L->d));
   SCION_TRY(dev_alloc(L, &L->bad, sizeof(int64_t)));
+  SCION_TRY(dev_alloc(L, &L->err, sizeof(int)));
+  SCION_TRY(cudaMemsetAsync(L->err, 0, sizeof(int), s));
 
   if (!units.empty())
     SCION_TRY(cudaMemcpyAsync(L->xunits, units.data(), sizeof(scion::XUnit) * units.size(), cudaMemcpyHostToDevice, s));
@@ -209,6 +282,10 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
                                  L->gu_bank, L->bad, s));
   SCION_TRY(scion::launch_retile(L->fmt, static_cast<const uint8_t*>(desc->down_exps), L->E, L->d, L->GF, 1, 0,
                                  L->dn_bank, L->bad, s));
+  if (max_tokens > SCION_TDEC) {
+    st = create_prefill(L, s);
+    if (st != SCION_OK) goto fail;
+  }
   SCION_TRY(cudaMemcpyAsync(&bad_host, L->bad, sizeof(int64_t), cudaMemcpyDeviceToHost, s));
   SCION_TRY(cudaStreamSynchronize(s));
   if (bad_host != 0) {
@@ -236,6 +313,7 @@ extern "C" int scion_moe_forward(const void* x, int T, const scion_layer* L, flo
   if (!x || !out) return SCION_EINVAL;
   cudaStream_t s = as_stream(stream);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  if (T > SCION_TDEC && L->pre) return forward_prefill(L, xb, T, out, s);
   for (int t0 = 0; t0 < T; t0 += SCION_TDEC) {
     const int n = T - t0 < SCION_TDEC ? T - t0 : SCION_TDEC;
     int st = forward_pass(L, xb + int64_t(t0) * L->d, n, out + int64_t(t0) * L->d, s);
@@ -260,7 +338,9 @@ extern "C" int scion_moe_forward_host(const void* x_host, int T, const scion_lay
 
 extern "C" int scion_moe_forward_debug(const void* x, int T, const scion_layer* L, float* out,
                                        const scion_debug_out* dbg, void* stream) {
-  if (!L || !dbg || T < 0 || T > L->max_tokens || T > SCION_TDEC) return SCION_EINVAL;
+  if (!L || !dbg || T < 0 || T > L->max_tokens) return SCION_EINVAL;
+  const bool pre = T > SCION_TDEC;
+  if (pre && !L->pre) return SCION_EINVAL;
   int st = scion_moe_forward(x, T, L, out, stream);
   if (st != SCION_OK || T == 0) return st;
   cudaStream_t s = as_stream(stream);
@@ -268,18 +348,36 @@ extern "C" int scion_moe_forward_debug(const void* x, int T, const scion_layer* 
   auto cp = [&](void* dst, const void* src, size_t bytes) {
     if (dst && e == cudaSuccess) e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s);
   };
-  cp(dbg->logits, L->logits, sizeof(float) * size_t(T) * L->E);
-  cp(dbg->ids, L->ids, sizeof(int32_t) * size_t(T) * L->k);
-  cp(dbg->gates, L->gates, sizeof(float) * size_t(T) * L->k);
-  cp(dbg->counts, L->counts, sizeof(int32_t) * size_t(L->E));
-  cp(dbg->offsets, L->offsets, sizeof(int32_t) * size_t(L->E + 1));
-  cp(dbg->perm, L->perm, sizeof(int32_t) * size_t(T) * L->k);
+  const scion::PrefillState* P = L->pre;
+  cp(dbg->logits, pre ? P->logits : L->logits, sizeof(float) * size_t(T) * L->E);
+  cp(dbg->ids, pre ? P->ids : L->ids, sizeof(int32_t) * size_t(T) * L->k);
+  cp(dbg->gates, pre ? P->gates : L->gates, sizeof(float) * size_t(T) * L->k);
+  cp(dbg->counts, pre ? P->counts : L->counts, sizeof(int32_t) * size_t(L->E));
+  cp(dbg->offsets, pre ? P->offsets : L->offsets, sizeof(int32_t) * size_t(L->E + 1));
+  cp(dbg->perm, pre ? P->perm : L->perm, sizeof(int32_t) * size_t(T) * L->k);
   if (dbg->h && e == cudaSuccess)
-    e = scion::launch_unfrag(L->fmt, L->h, T * L->k, L->GF, reinterpret_cast<__half*>(dbg->h), s);
+    e = pre ? scion::launch_unperm_prefill(L->fmt, P->h, int64_t(T) * L->k * L->F, reinterpret_cast<__half*>(dbg->h), s)
+            : scion::launch_unfrag(L->fmt, L->h, T * L->k, L->GF, reinterpret_cast<__half*>(dbg->h), s);
   if (dbg->hz && e == cudaSuccess && L->Kdense)
-    e = cudaMemcpy2DAsync(dbg->hz, sizeof(__half) * L->Kdense, L->hz, sizeof(__half) * L->Kd,
+    e = cudaMemcpy2DAsync(dbg->hz, sizeof(__half) * L->Kdense, pre ? P->hz : L->hz, sizeof(__half) * L->Kd,
                           sizeof(__half) * L->Kdense, T, cudaMemcpyDeviceToDevice, s);
   return cuda_status(e);
+}
+
+extern "C" int scion_layer_check(const scion_layer* L, void* stream) {
+  if (!L) return SCION_EINVAL;
+  cudaStream_t s = as_stream(stream);
+  int err = 0;
+  cudaError_t e = cudaMemcpyAsync(&err, L->err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (err != 0) {
+    const int zero = 0;
+    e = cudaMemcpyAsync(L->err, &zero, sizeof(int), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    return err;
+  }
+  return SCION_OK;
 }
 
 extern "C" int scion_profile_begin(int max_launches) {

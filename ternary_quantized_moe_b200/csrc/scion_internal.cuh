@@ -22,6 +22,7 @@
 // down bank, so a 128-row x 128-column stage of either bank is one contiguous run.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -49,6 +50,28 @@ struct XUnit {
   int row0;  // first row of the unit within its matrices
 };
 
+// Buffers and tensor maps of the tensor-core (prefill) path, present when the layer
+// accepts batches above one decode pass.
+struct PrefillState {
+  CUtensorMap maps[6];  // A operands: router, delta, sh_gate, sh_up, corr_a, dense_down
+  CUtensorMap hz_map;   // B operand of the dense down GEMM
+  void* xunits;         // DenseUnit[] (device)
+  int n_xunits;
+  void* dunits;
+  int n_dunits;
+  float* logits;        // [maxT][E]
+  int32_t* ids;         // [maxT][k]
+  float* gates;         // [maxT][k]
+  int32_t* counts;      // [E]
+  int32_t* offsets;     // [E+1]
+  int32_t* perm;        // [maxT*k]
+  void* tiles;          // 128-token tiles, [maxT*k/128 + E]
+  int32_t* n_tiles;
+  __half* x16;          // [maxT][d]   x in the container column order (fp16)
+  __half* h;            // [maxT*k][F] expert SwiGLU hidden, container column order
+  __half* hz;           // [maxT][Kd]
+};
+
 }  // namespace scion
 
 struct scion_layer {
@@ -56,7 +79,7 @@ struct scion_layer {
   int d, E, k, F, Fs, r, fmt, max_tokens;
   int Gd, GF;       // 128-groups along d and along F
   int Kdense;       // Fs + r
-  int Kd;           // Kdense rounded up to 32: row stride of dense_down and hz (pad = 0)
+  int Kd;           // Kdense rounded up to 64: row stride of dense_down and hz (pad = 0)
   // owned device memory
   uint8_t* gu_bank;    // [E][F/128][Gd][2][8][tile]
   uint8_t* dn_bank;    // [E][d/128][GF][8][tile]
@@ -81,6 +104,8 @@ struct scion_layer {
   void* x_stage;     // [max_tokens][d] bf16 (host-buffer forward)
   float* out_stage;  // [max_tokens][d]
   int64_t* bad;      // [1] invalid-code counter used at create
+  int* err;          // [1] device status word (a bounded wait that gave up writes ETIMEOUT)
+  scion::PrefillState* pre;  // tensor-core path (nullptr when max_tokens <= SCION_TDEC)
   size_t device_bytes;
 };
 
@@ -100,7 +125,7 @@ cudaError_t launch_bf16_to_f16_rows(const __nv_bfloat16* src, int rows, int cols
                                     cudaStream_t s);
 
 // k_route.cu
-cudaError_t launch_router_f32(const scion_layer* L, const __nv_bfloat16* x, int T, cudaStream_t s);
+cudaError_t launch_router_f32(const scion_layer* L, const __nv_bfloat16* x, int T, float* logits, cudaStream_t s);
 cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s);
 cudaError_t configure_route_kernels();
 
@@ -112,6 +137,17 @@ cudaError_t launch_down_dense(const scion_layer* L, int T, float* out, cudaStrea
 // fragment-ordered rows [rows][G][128] -> natural order [rows][G*128]
 cudaError_t launch_unfrag(int fmt, const __half* src, int rows, int G, __half* dst, cudaStream_t s);
 cudaError_t configure_kernels();
+
+// k_prefill.cu
+int make_tmap_2d(CUtensorMap* map, const void* ptr, int bf16, int64_t rows, int64_t K);
+cudaError_t configure_prefill_kernels();
+size_t prefill_unit_bytes();
+size_t prefill_tile_bytes();
+int prefill_max_units(const scion_layer* L);
+void prefill_units(const scion_layer* L, void* xunits_host, int* n_x, void* dunits_host, int* n_d);
+cudaError_t launch_unperm_prefill(int fmt, const __half* src, int64_t n, __half* dst, cudaStream_t s);
+cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfloat16* x, int T, float* out,
+                                 cudaStream_t s);
 
 // ------------------------------------------------------------ device helpers
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {

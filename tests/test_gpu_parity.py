@@ -285,3 +285,52 @@ def test_full_size_prefill_sampled(name, n_sample):
     assert np.isfinite(got).all()
     ref, _, _ = oracle.forward(ol, x[sample])
     check_output(got[sample], ref)
+
+
+# --------------------------------------------------------- tensor-core path
+@pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
+@pytest.mark.parametrize("router_f32", [False, True])
+def test_prefill_stagewise(fmt, router_f32):
+    """Batches above 64 tokens run as tcgen05 GEMMs; routing bit-exact, hidden and output
+    within tolerance."""
+    cfg = small("p", fmt, router_f32, E=16, k=4, d=256, F=256, Fs=128, r=32)
+    T = 200
+    L, banks, ol, x = _case(cfg, T)
+    layer = device_layer(cfg, L, banks, 256)
+    got, dbg = run_forward(layer, x, T, debug=True, E=cfg.n_experts, k=cfg.top_k, F=cfg.ffn,
+                           Kdense=cfg.shared_ffn + cfg.rank)
+    assert tq.scion_layer_check(layer) == 0
+    _check_routing(cfg, dbg, ol, x, T)
+    _check_hidden(cfg, dbg, ol, x, T)
+    hs, _ = oracle.shared(ol, x)
+    z, _ = oracle.corr(ol, x)
+    check_output(dbg["hz"].astype(np.float64), np.concatenate([hs, z], axis=1), rel_l2=1e-3)
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
+
+
+@pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
+@pytest.mark.parametrize("T", [65, 129, 500])
+def test_prefill_multi_tile_experts(fmt, T):
+    """Few experts, many tokens each: experts span several 128-token tiles, ragged tails."""
+    cfg = small("m", fmt, False, E=4, k=2, d=384, F=128, Fs=0, r=16)
+    L, banks, ol, x = _case(cfg, T)
+    layer = device_layer(cfg, L, banks, T)
+    got, dbg = run_forward(layer, x, T, debug=True, E=cfg.n_experts, k=cfg.top_k, F=cfg.ffn,
+                           Kdense=cfg.shared_ffn + cfg.rank)
+    assert tq.scion_layer_check(layer) == 0
+    _check_routing(cfg, dbg, ol, x, T)
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
+
+
+def test_prefill_matches_decode_passes():
+    """The same tokens through both paths (a 64-token layer in two calls vs one 128-token call)."""
+    cfg = small("pd", synth.PTQ1_0, False, E=32, k=4)
+    L, banks, ol, x = _case(cfg, 128)
+    dec = device_layer(cfg, L, banks, 64)
+    pre = device_layer(cfg, L, banks, 128)
+    a0, _ = run_forward(dec, x[:64], 64)
+    a1, _ = run_forward(dec, x[64:], 64)
+    b, _ = run_forward(pre, x, 128)
+    check_output(b, np.concatenate([a0, a1]), rel_l2=1e-4, max_abs=1e-3)
