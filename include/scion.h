@@ -209,6 +209,23 @@ int scion_profile_end(int n_stages, double* ms_total, int64_t* launches);
 /* Number of kernels the forward entry points have launched since the library loaded. */
 int64_t scion_kernel_launches(void);
 
+/* ------------------------------------------------------- no-allocation entry
+ * Router logits for callers that cannot allocate device memory (their memory belongs
+ * to another allocator, or they run where allocation is not allowed).  The pages
+ * describe no counterpart of this entry point; it is a deployment aid.
+ *   logits[t][e] = x_t . w_router[e] + x_t . w_router_delta[e]      (fp32)
+ * x: device bf16 [T][d]; w_router, w_router_delta: device bf16 [E][d]; logits: device
+ * fp32 [T][E], written.  Limits: T <= 64, E <= 512, d <= 4096 and d % 128 == 0; larger
+ * sizes return SCION_EINVAL and launch nothing.  The split-K scratch lives in a static
+ * device array inside the library (1 MiB + 128 B on every GPU that loads it, held until
+ * the process exits); the call allocates nothing.  The first call on a device looks the
+ * array's address up (cudaGetSymbolAddress) with that device current -- make that first
+ * call before any stream capture.  All calls share the array, so calls that could
+ * overlap on the GPU (different streams, or devices sharing a context) race: issue them
+ * in order on one stream.  Each call clears the array's counters before its kernel. */
+int scion_router_logits_static(const void* x, int T, const void* w_router, const void* w_router_delta, int n_experts,
+                               int d, float* logits, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,6 +26,7 @@ __all__ = [
     "scion_layer_create", "scion_layer_destroy", "scion_layer_device_bytes", "scion_moe_forward",
     "scion_moe_forward_host", "scion_moe_forward_debug", "Layer", "library_path", "EXPORTS",
     "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "STAGES", "scion_layer_check",
+    "scion_router_logits_static",
 ]
 
 SCION_PQ2_0 = 0
@@ -43,6 +44,7 @@ EXPORTS = (
     "scion_pack_device", "scion_unpack_device", "scion_layer_create", "scion_layer_destroy",
     "scion_layer_device_bytes", "scion_moe_forward", "scion_moe_forward_host", "scion_moe_forward_debug",
     "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "scion_layer_check",
+    "scion_router_logits_static",
 )
 STAGES = ("router_f32", "xproj", "route", "gateup", "down_routed", "down_dense", "x16")
 
@@ -101,6 +103,7 @@ def _load():
             "scion_profile_end": (ci, [ci, C.POINTER(C.c_double), C.POINTER(C.c_int64)]),
             "scion_kernel_launches": (C.c_int64, []),
             "scion_layer_check": (ci, [vp, vp]),
+            "scion_router_logits_static": (ci, [vp, ci, vp, vp, ci, ci, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -338,3 +341,19 @@ def scion_profile_end() -> dict:
 
 def scion_kernel_launches() -> int:
     return int(_load().scion_kernel_launches())
+
+
+# ------------------------------------------------------- no-allocation entry
+def scion_router_logits_static(x, T: int, w_router, w_router_delta, logits, stream=None) -> None:
+    """Router logits (x . W_r + x . delta, fp32) for callers that cannot allocate device
+    memory: the library keeps the split-K scratch in a static device array.  x: bf16 CUDA
+    [T, d]; weights: bf16 CUDA [E, d]; logits: fp32 CUDA [T, E].  T <= 64, E <= 512,
+    d <= 4096.  Calls share the scratch, so issue them in order on one stream."""
+    import torch
+
+    E, d = w_router.shape
+    st = _load().scion_router_logits_static(
+        _dptr(x, "x", (torch.bfloat16,)), int(T), _dptr(w_router, "w_router", (torch.bfloat16,)),
+        _dptr(w_router_delta, "w_router_delta", (torch.bfloat16,)), int(E), int(d),
+        _dptr(logits, "logits", (torch.float32,)), _stream(stream))
+    _check(st, "scion_router_logits_static")
