@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--impl", default="scion", choices=["scion", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0, help="override the number of cycled layers")
+    ap.add_argument("--stream-min-tokens", type=int, default=0,
+                    help="decode batches of at least this many tokens use the bulk-copy ring expert kernels")
     return ap.parse_args()
 
 
@@ -248,6 +250,8 @@ def run_gpu(args, rank, world, local_rank):
             shared_ffn=cfg.shared_ffn, sh_gate=W.get("sh_gate"), sh_up=W.get("sh_up"), sh_down=W.get("sh_down"),
             rank=cfg.rank, corr_a=W.get("corr_a"), corr_b=W.get("corr_b"), max_tokens=max_T))
         del banks, W
+        if args.stream_min_tokens:
+            tq.scion_layer_set_option(layers[-1], tq.SCION_OPT_STREAM_MIN_TOKENS, args.stream_min_tokens)
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     weight_bytes = sum(tq.scion_layer_device_bytes(L) for L in layers)

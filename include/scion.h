@@ -157,6 +157,15 @@ size_t scion_layer_device_bytes(const scion_layer* layer);
  * EINVAL on a null pointer or T out of range; ECUDA if a launch fails. */
 int scion_moe_forward(const void* x, int T, const scion_layer* layer, float* out, void* stream);
 
+/* Tuning options of a layer (scion_layer_set_option).
+ *  SCION_OPT_STREAM_MIN_TOKENS (default 65 = off): batches of at least this many tokens
+ *    (and at most 64) run the expert GEMVs on the kernels fed by a bulk-copy ring (one CTA
+ *    per 128 expert rows); other batches split K over the warps of one CTA per 16 rows.
+ *    Both give the same result up to fp32 summation order.
+ * EINVAL for an unknown option or an out-of-range value. */
+enum { SCION_OPT_STREAM_MIN_TOKENS = 1 };
+int scion_layer_set_option(scion_layer* layer, int option, int value);
+
 /* Waits for `stream`, then returns the layer's device status word and clears it:
  * SCION_ETIMEOUT if a tensor-core kernel of an earlier forward gave up a bounded wait
  * (its outputs are then invalid), SCION_ECUDA on an asynchronous CUDA fault, else OK. */
@@ -196,7 +205,8 @@ enum {
   SCION_STAGE_DOWN_ROUTED = 4, /* ternary expert down + gate-weighted scatter-add */
   SCION_STAGE_DOWN_DENSE = 5,  /* shared down + correction B */
   SCION_STAGE_X16 = 6,         /* x -> fp16 in container column order (tensor-core path) */
-  SCION_N_STAGES = 7
+  SCION_STAGE_COMBINE = 7,     /* sum of the k gate-weighted expert rows per token (tensor-core path) */
+  SCION_N_STAGES = 8
 };
 /* Creates a pool for `max_launches` launches and starts recording (EINVAL if already
  * recording or max_launches < 1).  Launches past the pool are not recorded.  Not

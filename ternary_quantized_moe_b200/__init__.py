@@ -26,7 +26,7 @@ __all__ = [
     "scion_layer_create", "scion_layer_destroy", "scion_layer_device_bytes", "scion_moe_forward",
     "scion_moe_forward_host", "scion_moe_forward_debug", "Layer", "library_path", "EXPORTS",
     "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "STAGES", "scion_layer_check",
-    "scion_router_logits_static",
+    "scion_router_logits_static", "scion_layer_set_option", "SCION_OPT_STREAM_MIN_TOKENS",
 ]
 
 SCION_PQ2_0 = 0
@@ -44,9 +44,10 @@ EXPORTS = (
     "scion_pack_device", "scion_unpack_device", "scion_layer_create", "scion_layer_destroy",
     "scion_layer_device_bytes", "scion_moe_forward", "scion_moe_forward_host", "scion_moe_forward_debug",
     "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "scion_layer_check",
-    "scion_router_logits_static",
+    "scion_router_logits_static", "scion_layer_set_option",
 )
-STAGES = ("router_f32", "xproj", "route", "gateup", "down_routed", "down_dense", "x16")
+SCION_OPT_STREAM_MIN_TOKENS = 1
+STAGES = ("router_f32", "xproj", "route", "gateup", "down_routed", "down_dense", "x16", "combine")
 
 
 class ScionError(RuntimeError):
@@ -104,6 +105,7 @@ def _load():
             "scion_kernel_launches": (C.c_int64, []),
             "scion_layer_check": (ci, [vp, vp]),
             "scion_router_logits_static": (ci, [vp, ci, vp, vp, ci, ci, vp, vp]),
+            "scion_layer_set_option": (ci, [vp, ci, ci]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -285,6 +287,11 @@ def scion_layer_destroy(layer: Layer) -> None:
 def scion_layer_check(layer: Layer, stream=None) -> int:
     """Waits for the stream and returns (and clears) the layer's device status word."""
     return int(_load().scion_layer_check(C.c_void_p(layer.handle), _stream(stream)))
+
+
+def scion_layer_set_option(layer: Layer, option: int, value: int) -> None:
+    _check(_load().scion_layer_set_option(C.c_void_p(layer.handle), int(option), int(value)),
+           "scion_layer_set_option")
 
 
 def scion_layer_device_bytes(layer: Layer) -> int:

@@ -20,8 +20,8 @@
 //
 // Column orders (the A expansion and the B rows must agree):
 //   PQ2_0 : inside every 16 columns, position 2s+h holds column s + 8h (s < 8, h < 2)
-//   PTQ1_0: inside every 128 columns, position 2q+h (q < 60) holds column 10(q/5) + 5h + q%5,
-//           positions 120..127 hold columns 120..127.
+//   PTQ1_0: each 64-column half of a 128-column group is self-contained: quintets 12h..12h+11
+//           in pairs, then remainder trits 4h..4h+3 (see perm_pos).
 #include <cudaTypedefs.h>
 #include <float.h>
 #include <math.h>
@@ -29,6 +29,7 @@
 #include <string.h>
 
 #include "tc_common.cuh"
+#include "topk_warp.cuh"
 
 namespace scion {
 
@@ -46,19 +47,32 @@ __device__ __forceinline__ int perm_pos(int fmt, int col) {  // physical column 
     int c16 = col & 15;
     return (col & ~15) | (2 * (c16 & 7) + (c16 >> 3));
   }
-  int g = col & ~127, k = col & 127;
-  if (k >= 120) return col;
-  int i = k / 10, r = k % 10;
-  return g | (2 * (5 * i + r % 5) + r / 5);
+  // PTQ1_0: half h of the group (positions 64h .. 64h+63) holds quintets 12h .. 12h+11 as
+  // pairs (2i, 2i+1) -- position 10i + 2j + u <-> column 5(12h + 2i + u) + j -- and then
+  // remainder trits 4h .. 4h+3 (columns 120 + 4h ..) in natural order.
+  const int g = col & ~127, k = col & 127;
+  if (k >= 120) return g | (64 * ((k - 120) >> 2) + 60 + ((k - 120) & 3));
+  const int q = k / 5, j = k % 5, half = q / 12, i = (q % 12) >> 1, u = q & 1;
+  return g | (64 * half + 10 * i + 2 * j + u);
 }
 
-__global__ void x16_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, int fmt, __half* __restrict__ xp) {
-  int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  // n = T*d; columns are permuted within their own row (d % 128 == 0)
-  int64_t base = i & ~int64_t(127);
-  int col = int(i & 127);
-  xp[base + perm_pos(fmt, col)] = __float2half_rn(__bfloat162float(x[i]));
+// x (bf16) -> fp16 in the container's column order; one thread per 16 columns (PQ2_0) or
+// per 128-column group (PTQ1_0).
+template <int FMT>
+__global__ void x16_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, __half* __restrict__ xp) {
+  constexpr int W = FMT == SCION_PQ2_0 ? 16 : 128;
+  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n / W) return;
+  const uint4* src = reinterpret_cast<const uint4*>(x + i * W);
+  uint4* dst = reinterpret_cast<uint4*>(xp + i * W);
+  __align__(16) __nv_bfloat16 in[W];
+  __align__(16) __half outv[W];
+#pragma unroll
+  for (int j = 0; j < W / 8; ++j) reinterpret_cast<uint4*>(in)[j] = src[j];
+#pragma unroll
+  for (int col = 0; col < W; ++col) outv[perm_pos(FMT, col) & (W - 1)] = __float2half_rn(__bfloat162float(in[col]));
+#pragma unroll
+  for (int j = 0; j < W / 8; ++j) dst[j] = reinterpret_cast<uint4*>(outv)[j];
 }
 
 // ---------------------------------------------------------------- dense GEMM
@@ -212,59 +226,51 @@ struct TernParams {
   const float* gates;
   int k;
   __half* h;  int F;     // gate/up output
-  float* out; int d;     // down output
+  float* y;   int d;     // down output: gate-weighted rows per routed (token, slot), [T*k][d]
   int* err;
 };
 
-constexpr int kTernStages = 2;
 constexpr uint32_t kAtom = 128 * 128;  // bytes of one 128-row x 64-column swizzled atom
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-// Expand row t (0..127) of one 128-row x 128-column group from its PQ2_0 sub-tile block
-// into the swizzled fp16 A tile (2 atoms).  Values are code * scale, exact in fp16.
-__device__ __forceinline__ void expand_pq2_row(const uint8_t* codes, int t, uint32_t a_tile) {
+// Expand half h (64 columns) of row t (0..127) of one 128-row group from its sub-tile block
+// into a 128-row x 64-column swizzled fp16 atom.  Values are code * scale, exact in fp16.
+__device__ __forceinline__ void expand_pq2_half(const uint8_t* codes, int t, int h, uint32_t atom) {
   const uint8_t* blk = codes + (t >> 4) * kPq2Tile;
   const int rho = t & 15, r8 = rho & 7, hi = rho >> 3;
   const __half2 sc = __half2half2(__ushort_as_half(*reinterpret_cast<const uint16_t*>(blk + 512 + 4 * r8 + 2 * hi)));
   const __half2 bias = u32_as_h2(0x64016401u);
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int cc = 0; cc < 2; ++cc) {
+    const int c = 2 * h + cc;  // container code bytes 8c .. 8c+7 = words 2c, 2c+1
     const uint2 w2 = *reinterpret_cast<const uint2*>(blk + 16 * (4 * r8 + c) + 8 * hi);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const uint32_t w = half ? w2.y : w2.x;
-      const int m = 2 * c + half;  // container word: columns 16m .. 16m+15
       uint32_t v[8];
 #pragma unroll
       for (int s = 0; s < 8; ++s)
         v[s] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w >> (2 * s), 0x00030003u, 0x64006400u)), bias), sc));
-      const int j0 = 2 * m;  // 16-byte chunk index along the 128 columns
-      st_shared_v4(a_tile + (j0 >> 3) * kAtom + sw128_offset(t, j0 & 7), v[0], v[1], v[2], v[3]);
-      st_shared_v4(a_tile + ((j0 + 1) >> 3) * kAtom + sw128_offset(t, (j0 + 1) & 7), v[4], v[5], v[6], v[7]);
+      const int j0 = 2 * (2 * cc + half);  // chunk index inside the atom
+      st_shared_v4(atom + sw128_offset(t, j0), v[0], v[1], v[2], v[3]);
+      st_shared_v4(atom + sw128_offset(t, j0 + 1), v[4], v[5], v[6], v[7]);
     }
   }
 }
 
-__device__ __forceinline__ int trit_at(int v, int digit) {
-  for (int i = 0; i < digit; ++i) v /= 3;
-  return v % 3;
-}
-
-// Same for PTQ1_0: quintet pairs (2i, 2i+1) give positions 10i + j | 10i + 5 + j through
-// the exact fp16 base-3 digit recurrence; columns 120..127 come from byte 24 and the tail.
-__device__ __forceinline__ void expand_ptq1_row(const uint8_t* codes, int t, uint32_t a_tile) {
+__device__ __forceinline__ void expand_ptq1_half(const uint8_t* codes, int t, int h, uint32_t atom) {
   const uint8_t* blk = codes + (t >> 4) * kPtq1Tile;
   const int rho = t & 15, r8 = rho & 7, hi = rho >> 3;
   const __half2 sc = __half2half2(__ushort_as_half(*reinterpret_cast<const uint16_t*>(blk + 416 + 4 * r8 + 2 * hi)));
   const __half2 third = __float2half2_rn(0.333251953125f), c1 = __float2half2_rn(682.5f);
   const __half2 m3 = __float2half2_rn(-3.0f), c2047 = __float2half2_rn(2047.0f);
-  uint32_t v[64];
+  uint32_t v[32];
 #pragma unroll
-  for (int i = 0; i < 12; ++i) {
-    const int q = 2 * i;
+  for (int i = 0; i < 6; ++i) {
+    const int q = 12 * h + 2 * i;
     const uint32_t x = *reinterpret_cast<const uint16_t*>(blk + 12 * (4 * r8 + q / 6) + 6 * hi + q % 6);
     uint32_t pr;
     asm("prmt.b32 %0, %1, 0, 0x4140;" : "=r"(pr) : "r"(x));
@@ -277,48 +283,78 @@ __device__ __forceinline__ void expand_ptq1_row(const uint8_t* codes, int t, uin
       v[5 * i + j] = h2_as_u32(__hmul2(code, sc));
     }
   }
-  const int q24 = blk[384 + 4 * r8 + 2 * hi], tail = blk[384 + 4 * r8 + 2 * hi + 1];
+  {
+    // remainder trits: digits 0..4 of byte 24 and 0..2 of the tail byte, one digit chain
+    const uint32_t qt = *reinterpret_cast<const uint16_t*>(blk + 384 + 4 * r8 + 2 * hi);
+    uint32_t pr;
+    asm("prmt.b32 %0, %1, 0, 0x4140;" : "=r"(pr) : "r"(qt));
+    __half2 V = u32_as_h2(pr | 0x64006400u);
+    uint32_t pd[5];
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int k0 = 2 * m, k1 = 2 * m + 1;  // columns 120 + k
-    const int t0 = k0 < 5 ? trit_at(q24, k0) : trit_at(tail, k0 - 5);
-    const int t1 = k1 < 5 ? trit_at(q24, k1) : trit_at(tail, k1 - 5);
-    v[60 + m] = h2_as_u32(__hmul2(__halves2half2(__int2half_rn(t0 - 1), __int2half_rn(t1 - 1)), sc));
+    for (int j = 0; j < 5; ++j) {
+      __half2 Vn = __hfma2(V, third, c1);
+      pd[j] = h2_as_u32(__hadd2(__hfma2(Vn, m3, V), c2047));
+      V = Vn;
+    }
+    uint32_t r0, r1;
+    if (h == 0) {  // columns 120..123 = byte-24 digits 0..3
+      asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r0) : "r"(pd[0]), "r"(pd[1]));
+      asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r1) : "r"(pd[2]), "r"(pd[3]));
+    } else {       // columns 124..127 = byte-24 digit 4, tail digits 0..2
+      asm("prmt.b32 %0, %1, %2, 0x7610;" : "=r"(r0) : "r"(pd[4]), "r"(pd[0]));
+      asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r1) : "r"(pd[1]), "r"(pd[2]));
+    }
+    v[30] = h2_as_u32(__hmul2(u32_as_h2(r0), sc));
+    v[31] = h2_as_u32(__hmul2(u32_as_h2(r1), sc));
   }
 #pragma unroll
-  for (int j = 0; j < 16; ++j)
-    st_shared_v4(a_tile + (j >> 3) * kAtom + sw128_offset(t, j & 7), v[4 * j], v[4 * j + 1], v[4 * j + 2],
-                 v[4 * j + 3]);
+  for (int j = 0; j < 8; ++j)
+    st_shared_v4(atom + sw128_offset(t, j), v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
 }
 
 template <int FMT, int NA>
-__global__ void __launch_bounds__(kThreads, 1) tern_gemm_kernel(const __grid_constant__ TernParams p) {
+struct TernRing {
+  static constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
+  static constexpr int kA = 3;                    // expanded 64-column A stages
+  static constexpr int kB = 4;                    // gathered 64-column B stages
+  static constexpr int kC = NA == 2 ? 3 : 4;      // packed code groups
+  static constexpr uint32_t a_bytes = NA * kAtom;  // one A stage: NA matrices x 128 rows x 128 B
+  static constexpr uint32_t c_bytes = NA * 8 * tb;
+  static constexpr uint32_t slab_bytes = 2 * 16 * 128 * 4;  // epilogue: two 16-token slabs (fp32 worst case)
+  static constexpr uint32_t a_off = 0, b_off = kA * a_bytes, c_off = b_off + kB * kAtom;
+  static constexpr uint32_t slab_off = (c_off + kC * c_bytes + 127) & ~127u;
+  static constexpr uint32_t bytes = slab_off + slab_bytes;
+};
+
+constexpr int kTernThreads = 384;  // 12 warps: codes, MMA, B rows, (idle), 4 expansion, 4 epilogue
+
+// Persistent grouped GEMM: CTA b walks the work items b, b + gridDim.x, ... where item =
+// (128-token tile, 128-row weight tile).  All roles walk the same sequence; the rings and the
+// two TMEM accumulators carry over from one item to the next, so loads, expansion and MMAs of
+// item i+1 overlap the epilogue of item i.
+template <int FMT, int NA>
+__global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid_constant__ TernParams p) {
+  using R = TernRing<FMT, NA>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t codes_full[kTernStages], b_full[kTernStages], a_full[kTernStages], empty[kTernStages], accf;
+  __shared__ uint64_t c_full[R::kC], c_empty[R::kC], a_full[R::kA], a_empty[R::kA], b_full[R::kB], b_empty[R::kB];
+  __shared__ uint64_t acc_full[2], acc_empty[2], mma_done;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
-  if (int(blockIdx.x) >= *p.n_tiles) return;
-  const TernTile tile = p.tiles[blockIdx.x];
-  const int rt = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int p0 = p.offsets[tile.e];
-  const int nn = min(kBN, p.counts[tile.e] - tile.c0);
-  const int nmma = (nn + 15) & ~15;
-  constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
-  constexpr uint32_t a_bytes = 2 * kAtom, b_bytes = 2 * kAtom, c_bytes = 8 * tb;
-  constexpr uint32_t stage_bytes = (NA * a_bytes + b_bytes + NA * c_bytes + 1023) & ~1023u;  // atoms 1024-aligned
-  constexpr uint32_t ncols = NA * kBN;
+  const int RT = p.R >> 7;                     // 128-row weight tiles per expert matrix
+  const int n_items = *p.n_tiles * RT;
+  const int nkb = 2 * p.G;                     // 64-column stages per item
+  constexpr uint32_t acc_cols = NA * kBN;      // one accumulator: NA x 128 columns
+  constexpr uint32_t ncols = 2 * acc_cols;     // ping-pong
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kTernStages; ++s) {
-      mbar_init(&codes_full[s], 1);
-      mbar_init(&b_full[s], 32);
-      mbar_init(&a_full[s], 128);
-      mbar_init(&empty[s], 1);
-    }
-    mbar_init(&accf, 1);
+    for (int i = 0; i < R::kC; ++i) mbar_init(&c_full[i], 1), mbar_init(&c_empty[i], 128);
+    for (int i = 0; i < R::kA; ++i) mbar_init(&a_full[i], 128), mbar_init(&a_empty[i], 1);
+    for (int i = 0; i < R::kB; ++i) mbar_init(&b_full[i], 32), mbar_init(&b_empty[i], 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&acc_full[i], 1), mbar_init(&acc_empty[i], 128);
+    mbar_init(&mma_done, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -330,113 +366,185 @@ __global__ void __launch_bounds__(kThreads, 1) tern_gemm_kernel(const __grid_con
   const uint32_t sbase = smem_u32(smem);
 
   if (warp == 0) {
-    // ---------------- producer: packed code blocks (bulk copy) + gathered B rows (cp.async)
-    const __half* rows[kBN / 32];
+    // ---------------- packed code blocks, one 128-row group per bulk copy and matrix
+    if (lane == 0) {
+      const int64_t mat_stride = int64_t(8) * R::tb, grp_stride = NA * mat_stride;
+      int gs = 0;  // running group-stage counter
+      for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
+        const TernTile tile = p.tiles[item / RT];
+        const int rt = item % RT;
+        const uint8_t* ebase = p.bank + (int64_t(tile.e) * RT + rt) * p.G * grp_stride;
+        for (int g = 0; g < p.G; ++g, ++gs) {
+          const int s = gs % R::kC;
+          if (gs >= R::kC && !mbar_wait(&c_empty[s], ((gs / R::kC) - 1) & 1, &abort_flag, p.err)) break;
+          uint8_t* dst = smem + R::c_off + s * R::c_bytes;
+          mbar_arrive_expect_tx(&c_full[s], R::c_bytes);
 #pragma unroll
-    for (int i = 0; i < kBN / 32; ++i) {
-      const int r = lane + 32 * i;
-      rows[i] = nullptr;
-      if (r < nn) {
-        const int64_t src = NA == 2 ? int64_t(p.perm[p0 + tile.c0 + r] / p.k) : int64_t(p0 + tile.c0 + r);
-        rows[i] = p.bsrc + src * p.ldb;
+          for (int m = 0; m < NA; ++m)
+            bulk_load(dst + m * mat_stride, ebase + g * grp_stride + m * mat_stride, mat_stride, &c_full[s]);
+        }
       }
+      // the last kC groups issued may still be in flight if a consumer gave up: let them land
+      for (int i = max(0, gs - R::kC); i < gs; ++i) mbar_drain(&c_full[i % R::kC], (i / R::kC) & 1);
     }
-    const int64_t mat_stride = int64_t(8) * tb;
-    const int64_t grp_stride = NA * mat_stride;
-    const uint8_t* ebase = p.bank + (int64_t(tile.e) * (p.R >> 7) + rt) * p.G * grp_stride;
-    for (int kb = 0; kb < p.G; ++kb) {
-      const int s = kb % kTernStages;
-      if (kb >= kTernStages && !mbar_wait(&empty[s], ((kb / kTernStages) - 1) & 1, &abort_flag, p.err)) break;
-      uint8_t* st = smem + s * stage_bytes;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&codes_full[s], NA * c_bytes);
-#pragma unroll
-        for (int m = 0; m < NA; ++m)
-          bulk_load(st + NA * a_bytes + b_bytes + m * c_bytes, ebase + kb * grp_stride + m * mat_stride, c_bytes,
-                    &codes_full[s]);
-      }
-      const uint32_t bt = smem_u32(st + NA * a_bytes);
+  } else if (warp == 2) {
+    // ---------------- gathered B rows, 64 columns (128 B) per stage
+    int ks = 0;  // running stage counter
+    for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
+      const TernTile tile = p.tiles[item / RT];
+      const int p0 = p.offsets[tile.e];
+      const int nn = min(kBN, p.counts[tile.e] - tile.c0);
+      const __half* rows[kBN / 32];
 #pragma unroll
       for (int i = 0; i < kBN / 32; ++i) {
         const int r = lane + 32 * i;
-        if (rows[i]) {
-          const __half* src = rows[i] + kb * 128;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const uint32_t dst = bt + (j >> 3) * kAtom + sw128_offset(r, j & 7);
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src + 8 * j) : "memory");
-          }
+        rows[i] = nullptr;
+        if (r < nn) {
+          const int64_t src = NA == 2 ? int64_t(p.perm[p0 + tile.c0 + r] / p.k) : int64_t(p0 + tile.c0 + r);
+          rows[i] = p.bsrc + src * p.ldb;
         }
       }
-      cp_async_arrive_noinc(&b_full[s]);
+      for (int kb = 0; kb < nkb; ++kb, ++ks) {
+        const int s = ks % R::kB;
+        if (ks >= R::kB && !mbar_wait(&b_empty[s], ((ks / R::kB) - 1) & 1, &abort_flag, p.err)) break;
+        const uint32_t bt = sbase + R::b_off + s * kAtom;
+#pragma unroll
+        for (int i = 0; i < kBN / 32; ++i) {
+          if (!rows[i]) continue;
+          const int r = lane + 32 * i;
+          const __half* src = rows[i] + kb * 64;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(bt + sw128_offset(r, j)), "l"(src + 8 * j)
+                         : "memory");
+        }
+        cp_async_arrive_noinc(&b_full[s]);
+      }
     }
     cp_async_wait_all();
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer
-      const uint32_t idesc = umma_idesc(kBM, nmma, 0);
-      for (int kb = 0; kb < p.G; ++kb) {
-        const int s = kb % kTernStages;
-        const uint32_t par = (kb / kTernStages) & 1;
-        if (!mbar_wait(&a_full[s], par, &abort_flag, p.err)) break;
-        if (!mbar_wait(&b_full[s], par, &abort_flag, p.err)) break;
+      int ks = 0, li = 0;
+      for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x, ++li) {
+        const TernTile tile = p.tiles[item / RT];
+        const int nn = min(kBN, p.counts[tile.e] - tile.c0);
+        const uint32_t idesc = umma_idesc(kBM, (nn + 15) & ~15, 0);
+        const int ab = li & 1;
+        if (li >= 2 && !mbar_wait(&acc_empty[ab], ((li >> 1) - 1) & 1, &abort_flag, p.err)) break;
         tc_fence_after();
-        fence_proxy_async();
-        const uint32_t st = sbase + s * stage_bytes;
+        const uint32_t acc = tmem + ab * acc_cols;
+        for (int kb = 0; kb < nkb; ++kb, ++ks) {
+          const int sa = ks % R::kA, sb = ks % R::kB;
+          if (!mbar_wait(&a_full[sa], (ks / R::kA) & 1, &abort_flag, p.err)) break;
+          if (!mbar_wait(&b_full[sb], (ks / R::kB) & 1, &abort_flag, p.err)) break;
+          tc_fence_after();
+          fence_proxy_async();
+          const uint32_t at = sbase + R::a_off + sa * R::a_bytes, bt = sbase + R::b_off + sb * kAtom;
 #pragma unroll
-        for (int k16 = 0; k16 < 8; ++k16) {
-          const uint32_t off = (k16 >> 2) * kAtom + 32 * (k16 & 3);
-          const uint64_t db = umma_desc_sw128(st + NA * a_bytes + off);
+          for (int k16 = 0; k16 < 4; ++k16) {
+            const uint64_t db = umma_desc_sw128(bt + 32 * k16);
 #pragma unroll
-          for (int m = 0; m < NA; ++m)
-            umma_f16(tmem + m * kBN, umma_desc_sw128(st + m * a_bytes + off), db, idesc, (kb | k16) != 0);
+            for (int m = 0; m < NA; ++m)
+              umma_f16(acc + m * kBN, umma_desc_sw128(at + m * kAtom + 32 * k16), db, idesc, (kb | k16) != 0);
+          }
+          umma_commit(&a_empty[sa]);
+          umma_commit(&b_empty[sb]);
         }
-        umma_commit(&empty[s]);
+        umma_commit(&acc_full[ab]);
       }
-      umma_commit(&accf);
+      // every MMA issued above has finished before TMEM is released
+      umma_commit(&mma_done);
+      mbar_drain(&mma_done, 0);
     }
-  } else if (warp >= 4) {
-    // ---------------- expansion (one weight row per thread), then the epilogue
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------- expansion (one weight row per thread, one 64-column half per stage)
     const int t = threadIdx.x - 128;
-    for (int kb = 0; kb < p.G; ++kb) {
-      const int s = kb % kTernStages;
-      if (!mbar_wait(&codes_full[s], (kb / kTernStages) & 1, &abort_flag, p.err)) break;
-      const uint8_t* st = smem + s * stage_bytes;
+    int ks = 0, gs = 0;
+    for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
+      for (int kb = 0; kb < nkb; ++kb, ++ks) {
+        const int h = kb & 1, sc = gs % R::kC, sa = ks % R::kA;
+        if (h == 0 && !mbar_wait(&c_full[sc], (gs / R::kC) & 1, &abort_flag, p.err)) break;
+        if (ks >= R::kA && !mbar_wait(&a_empty[sa], ((ks / R::kA) - 1) & 1, &abort_flag, p.err)) break;
+        const uint8_t* codes = smem + R::c_off + sc * R::c_bytes;
 #pragma unroll
-      for (int m = 0; m < NA; ++m) {
-        const uint8_t* codes = st + NA * a_bytes + b_bytes + m * c_bytes;
-        const uint32_t at = sbase + s * stage_bytes + m * a_bytes;
-        if constexpr (FMT == SCION_PQ2_0)
-          expand_pq2_row(codes, t, at);
-        else
-          expand_ptq1_row(codes, t, at);
+        for (int m = 0; m < NA; ++m) {
+          const uint32_t atom = sbase + R::a_off + sa * R::a_bytes + m * kAtom;
+          if constexpr (FMT == SCION_PQ2_0)
+            expand_pq2_half(codes + m * 8 * R::tb, t, h, atom);
+          else
+            expand_ptq1_half(codes + m * 8 * R::tb, t, h, atom);
+        }
+        fence_proxy_async();
+        mbar_arrive(&a_full[sa]);
+        if (h == 1) {
+          mbar_arrive(&c_empty[sc]);
+          ++gs;
+        }
       }
-      fence_proxy_async();
-      mbar_arrive(&a_full[s]);
     }
-    const int q = warp - 4;
-    if (mbar_wait(&accf, 0, &abort_flag, p.err) && !abort_flag) {
+  } else if (warp >= 8) {
+    // ---------------- epilogue: TMEM lane quarter q = rows 32q .. 32q+31 of the weight tile
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int et = threadIdx.x - 256;  // 0..127
+    int li = 0;
+    // no abort-flag test in the loop condition: the 128 threads leave only together, by the vote
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++li) {
+      const TernTile tile = p.tiles[item / RT];
+      const int rt = item % RT;
+      const int p0 = p.offsets[tile.e];
+      const int nn = min(kBN, p.counts[tile.e] - tile.c0);
+      const int ab = li & 1;
+      if (!named_bar_and(1, 128, mbar_wait(&acc_full[ab], (li >> 1) & 1, &abort_flag, p.err))) break;
       tc_fence_after();
-      const int row = q * 32 + lane;
-      const int grow = rt * kBM + row;
+      const uint32_t acc = tmem + ab * acc_cols;
+      float* slab = reinterpret_cast<float*>(smem + R::slab_off);
       for (int c = 0; c * 16 < nn; ++c) {
+        const int buf = c & 1;
         float v0[16], v1[16];
-        const uint32_t ta = tmem + (uint32_t(q * 32) << 16) + c * 16;
+        const uint32_t ta = acc + (uint32_t(q * 32) << 16) + c * 16;
         tmem_ld16(ta, v0);
         if (NA == 2) tmem_ld16(ta + kBN, v1);
+        if constexpr (NA == 2) {
+          __half* hs = reinterpret_cast<__half*>(slab) + buf * 16 * 128;
+          const int pcol = perm_pos(FMT, row);  // position of this row inside its 128-column group
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int n = c * 16 + i;
-          if (n >= nn) break;
-          const int pos = p0 + tile.c0 + n;
-          if constexpr (NA == 2) {
-            p.h[int64_t(pos) * p.F + perm_pos(FMT, grow)] = __float2half_rn(silu_f(v0[i]) * v1[i]);
-          } else {
-            const int entry = p.perm[pos];
-            atomicAdd(&p.out[int64_t(entry / p.k) * p.d + grow], p.gates[entry] * v0[i]);
+          for (int i = 0; i < 16; ++i) hs[i * 128 + pcol] = __float2half_rn(silu_f(v0[i]) * v1[i]);
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          for (int j = et; j < 16 * 16; j += 128) {
+            const int i = j >> 4, ch = j & 15, n = c * 16 + i;
+            if (n < nn) {
+              const int64_t pos = p0 + tile.c0 + n;
+              *reinterpret_cast<uint4*>(p.h + pos * p.F + int64_t(rt) * kBM + ch * 8) =
+                  *reinterpret_cast<const uint4*>(hs + i * 128 + ch * 8);
+            }
+          }
+        } else {
+          float* fs = slab + buf * 16 * 128;
+          float gv[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int n = c * 16 + i;
+            gv[i] = n < nn ? p.gates[p.perm[p0 + tile.c0 + n]] : 0.f;
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) fs[i * 128 + row] = gv[i] * v0[i];
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          for (int j = et; j < 16 * 32; j += 128) {
+            const int i = j >> 5, ch = j & 31, n = c * 16 + i;
+            if (n < nn) {
+              const int64_t pos = p0 + tile.c0 + n;
+              *reinterpret_cast<float4*>(p.y + pos * p.d + int64_t(rt) * kBM + ch * 4) =
+                  *reinterpret_cast<const float4*>(fs + i * 128 + ch * 4);
+            }
           }
         }
       }
+      // accumulator drained (tcgen05.ld waited inside tmem_ld16): hand it back to the MMA warp
+      tc_fence_before();
+      mbar_arrive(&acc_empty[ab]);
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // slabs free before the next item writes them
     }
   }
   tc_fence_before();
@@ -448,59 +556,13 @@ __global__ void __launch_bounds__(kThreads, 1) tern_gemm_kernel(const __grid_con
 }
 
 // ------------------------------------------------------------------- routing
-__device__ __forceinline__ void argmax_merge2(float& v, int& i, float v2, int i2) {
-  if (v2 > v || (v2 == v && i2 < i)) v = v2, i = i2;
-}
-
-// One warp per token: top-k (ties -> lower id), gates.  smem: vals[8][E].
+// One warp per token (8 per CTA), logits in registers.
+template <int VPL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                    int norm_topk, int32_t* __restrict__ ids, float* __restrict__ gates) {
-  extern __shared__ float vals_all[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
-  if (t >= T) return;
-  float* vals = vals_all + warp * E;
-  const float* row = logits + int64_t(t) * E;
-  float mx = -INFINITY;
-  for (int e = lane; e < E; e += 32) {
-    float v = row[e];
-    if (!(v >= -FLT_MAX)) v = -FLT_MAX;
-    vals[e] = v;
-    mx = fmaxf(mx, v);
-  }
-  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  float zall = 0.f;
-  if (!norm_topk) {
-    for (int e = lane; e < E; e += 32) zall += expf(vals[e] - mx);
-    for (int o = 16; o; o >>= 1) zall += __shfl_xor_sync(0xffffffffu, zall, o);
-  }
-  __syncwarp();
-  float my_v = -INFINITY;
-  int my_id = -1;
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
-    for (int e = lane; e < E; e += 32) argmax_merge2(bv, bi, vals[e], e);
-    for (int o = 16; o; o >>= 1) {
-      float v2 = __shfl_xor_sync(0xffffffffu, bv, o);
-      int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
-      argmax_merge2(bv, bi, v2, i2);
-    }
-    if (lane == j) my_v = bv, my_id = bi;
-    __syncwarp();
-    if (lane == (bi & 31)) vals[bi] = -INFINITY;
-    __syncwarp();
-  }
-  const float top = __shfl_sync(0xffffffffu, my_v, 0);
-  float ex = 0.f;
-  if (lane < k) ex = norm_topk ? expf(my_v - top) : expf(my_v - mx);
-  float z = ex;
-  for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-  if (!norm_topk) z = zall;
-  if (lane < k) {
-    ids[int64_t(t) * k + lane] = my_id;
-    gates[int64_t(t) * k + lane] = ex / z;
-  }
+  if (t < T) warp_topk<VPL>(logits + int64_t(t) * E, E, k, norm_topk, lane, ids + int64_t(t) * k, gates + int64_t(t) * k);
 }
 
 constexpr int kGroupWarps = 16;
@@ -511,6 +573,7 @@ __global__ void __launch_bounds__(kGroupWarps * 32) group_kernel(const int32_t* 
                                                                  int32_t* __restrict__ counts,
                                                                  int32_t* __restrict__ offsets,
                                                                  int32_t* __restrict__ perm,
+                                                                 int32_t* __restrict__ inv,
                                                                  TernTile* __restrict__ tiles,
                                                                  int32_t* __restrict__ n_tiles) {
   extern __shared__ int32_t gsm[];
@@ -581,6 +644,7 @@ __global__ void __launch_bounds__(kGroupWarps * 32) group_kernel(const int32_t* 
     __syncwarp();
     if (i < i1) {
       perm[c + rank] = i;
+      inv[i] = c + rank;
       if (rank == 0) cur[e] = c + __popc(mask);
     }
     __syncwarp();
@@ -607,10 +671,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  }
+  return n;
+}
+
 size_t tern_smem(int na, int fmt) {
-  const size_t tb = fmt == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
-  const size_t stage = (size_t(na) * 2 * kAtom + 2 * kAtom + na * 8 * tb + 1023) & ~size_t(1023);
-  return kTernStages * stage + 1024;
+  size_t b;
+  if (fmt == SCION_PQ2_0) b = na == 2 ? TernRing<SCION_PQ2_0, 2>::bytes : TernRing<SCION_PQ2_0, 1>::bytes;
+  else b = na == 2 ? TernRing<SCION_PTQ1_0, 2>::bytes : TernRing<SCION_PTQ1_0, 1>::bytes;
+  return b + 1024;
 }
 constexpr size_t kDenseSmem = kDenseStages * (2 * 128 * 64 * 2 + 128 * 64 * 2) + 1024;
 
@@ -647,8 +722,24 @@ cudaError_t configure_prefill_kernels() {
   if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PTQ1_0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 int(tern_smem(1, SCION_PTQ1_0)))))
     return e;
-  if ((e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024))) return e;
   return cudaFuncSetAttribute(group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+}
+
+// out[t] (= dense part, or 0 when the layer has no shared expert and no correction)
+// += sum over slots j < k of y[inv[t*k + j]], in slot order.  One CTA per token.
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y, const int32_t* __restrict__ inv,
+                                                     int k, int d, int has_dense, float* __restrict__ out) {
+  const int t = blockIdx.x;
+  const int32_t* iv = inv + int64_t(t) * k;
+  float4* o = reinterpret_cast<float4*>(out + int64_t(t) * d);
+  for (int c4 = threadIdx.x; c4 < d / 4; c4 += blockDim.x) {
+    float4 acc = has_dense ? o[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const float4 v = reinterpret_cast<const float4*>(y + int64_t(iv[j]) * d)[c4];
+      acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+    }
+    o[c4] = acc;
+  }
 }
 
 __global__ void unperm_prefill_kernel(int fmt, const __half* __restrict__ src, int64_t n, __half* __restrict__ dst) {
@@ -691,7 +782,10 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
   switch (stage) {
     case SCION_STAGE_X16: {
       const int64_t n = int64_t(T) * L->d;
-      x16_kernel<<<unsigned((n + 255) / 256), 256, 0, s>>>(x, n, L->fmt, P.x16);
+      if (L->fmt == SCION_PQ2_0)
+        x16_kernel<SCION_PQ2_0><<<unsigned((n / 16 + 255) / 256), 256, 0, s>>>(x, n, P.x16);
+      else
+        x16_kernel<SCION_PTQ1_0><<<unsigned((n / 128 + 127) / 128), 128, 0, s>>>(x, n, P.x16);
       return cudaGetLastError();
     }
     case SCION_STAGE_XPROJ: {
@@ -707,12 +801,20 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       return cudaGetLastError();
     }
     case SCION_STAGE_ROUTE: {
-      topk_kernel<<<(T + 7) / 8, 256, sizeof(float) * 8 * L->E, s>>>(P.logits, T, L->E, L->k, L->desc.norm_topk,
-                                                                    P.ids, P.gates);
+      const int vpl = (L->E + 31) / 32;
+#define SCION_TOPK(V) topk_kernel<V><<<(T + 7) / 8, 256, 0, s>>>(P.logits, T, L->E, L->k, L->desc.norm_topk, P.ids, P.gates)
+      if (vpl <= 1) SCION_TOPK(1);
+      else if (vpl <= 2) SCION_TOPK(2);
+      else if (vpl <= 4) SCION_TOPK(4);
+      else if (vpl <= 8) SCION_TOPK(8);
+      else if (vpl <= 16) SCION_TOPK(16);
+      else if (vpl <= 32) SCION_TOPK(32);
+      else SCION_TOPK(64);
+#undef SCION_TOPK
       cudaError_t e = cudaGetLastError();
       if (e != cudaSuccess) return e;
       const size_t gsm = sizeof(int32_t) * (size_t(kGroupWarps) * L->E + L->E);
-      group_kernel<<<1, kGroupWarps * 32, gsm, s>>>(P.ids, T, L->E, L->k, P.counts, P.offsets, P.perm,
+      group_kernel<<<1, kGroupWarps * 32, gsm, s>>>(P.ids, T, L->E, L->k, P.counts, P.offsets, P.perm, P.inv,
                                                    static_cast<TernTile*>(P.tiles), P.n_tiles);
       return cudaGetLastError();
     }
@@ -722,17 +824,20 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       tp.bsrc = P.x16, tp.ldb = L->d;
       tp.tiles = static_cast<const TernTile*>(P.tiles), tp.n_tiles = P.n_tiles;
       tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gates = P.gates, tp.k = L->k;
-      tp.h = P.h, tp.F = L->F, tp.out = nullptr, tp.d = L->d, tp.err = L->err;
-      const int max_tiles = (T * L->k + kBN - 1) / kBN + L->E;
-      dim3 grid(max_tiles, L->F / kBM);
+      tp.h = P.h, tp.F = L->F, tp.y = nullptr, tp.d = L->d, tp.err = L->err;
+      const dim3 grid(num_sms());
       if (L->fmt == SCION_PQ2_0)
-        tern_gemm_kernel<SCION_PQ2_0, 2><<<grid, kThreads, tern_smem(2, L->fmt), s>>>(tp);
+        tern_gemm_kernel<SCION_PQ2_0, 2><<<grid, kTernThreads, tern_smem(2, L->fmt), s>>>(tp);
       else
-        tern_gemm_kernel<SCION_PTQ1_0, 2><<<grid, kThreads, tern_smem(2, L->fmt), s>>>(tp);
+        tern_gemm_kernel<SCION_PTQ1_0, 2><<<grid, kTernThreads, tern_smem(2, L->fmt), s>>>(tp);
+      return cudaGetLastError();
+    }
+    case SCION_STAGE_COMBINE: {
+      combine_kernel<<<T, 256, 0, s>>>(P.y, P.inv, L->k, L->d, P.n_dunits > 0, out);
       return cudaGetLastError();
     }
     case SCION_STAGE_DOWN_DENSE: {
-      if (P.n_dunits == 0) return cudaMemsetAsync(out, 0, sizeof(float) * size_t(T) * L->d, s);
+      if (P.n_dunits == 0) return cudaSuccess;
       DenseParams dp;
       memcpy(dp.a, P.maps, sizeof(dp.a));
       dp.b = P.hz_map;
@@ -749,13 +854,12 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       tp.bsrc = P.h, tp.ldb = L->F;
       tp.tiles = static_cast<const TernTile*>(P.tiles), tp.n_tiles = P.n_tiles;
       tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gates = P.gates, tp.k = L->k;
-      tp.h = nullptr, tp.F = L->F, tp.out = out, tp.d = L->d, tp.err = L->err;
-      const int max_tiles = (T * L->k + kBN - 1) / kBN + L->E;
-      dim3 grid(max_tiles, L->d / kBM);
+      tp.h = nullptr, tp.F = L->F, tp.y = P.y, tp.d = L->d, tp.err = L->err;
+      const dim3 grid(num_sms());
       if (L->fmt == SCION_PQ2_0)
-        tern_gemm_kernel<SCION_PQ2_0, 1><<<grid, kThreads, tern_smem(1, L->fmt), s>>>(tp);
+        tern_gemm_kernel<SCION_PQ2_0, 1><<<grid, kTernThreads, tern_smem(1, L->fmt), s>>>(tp);
       else
-        tern_gemm_kernel<SCION_PTQ1_0, 1><<<grid, kThreads, tern_smem(1, L->fmt), s>>>(tp);
+        tern_gemm_kernel<SCION_PTQ1_0, 1><<<grid, kTernThreads, tern_smem(1, L->fmt), s>>>(tp);
       return cudaGetLastError();
     }
     default:

@@ -13,6 +13,7 @@
 #include <math.h>
 
 #include "scion_internal.cuh"
+#include "topk_warp.cuh"
 
 namespace scion {
 namespace {
@@ -171,6 +172,83 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
   }
 }
 
+// ---------------------------------------------------------------- decode route v2
+// One warp per token (VPL logits per lane held in registers), then the last CTA to finish
+// groups all T*k entries: histogram, scan, active list, per-slot records and the stable
+// scatter.  Grid: ceil(T / 4) CTAs of 4 warps.
+template <int VPL>
+__global__ void __launch_bounds__(128) route_par_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                        int norm_topk, int32_t* __restrict__ ids,
+                                                        float* __restrict__ gates, int32_t* __restrict__ counts_out,
+                                                        int32_t* __restrict__ offsets_out,
+                                                        int32_t* __restrict__ perm_out,
+                                                        int32_t* __restrict__ active_out,
+                                                        int32_t* __restrict__ n_active_out,
+                                                        int4* __restrict__ slot_info, unsigned* __restrict__ done) {
+  extern __shared__ int32_t rsm[];  // counts[E] | cursor[E]
+  __shared__ int last;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 4 + warp;
+  pdl_trigger();
+  pdl_wait();
+  if (t < T) warp_topk<VPL>(logits + int64_t(t) * E, E, k, norm_topk, lane, ids + t * k, gates + t * k);
+  // ---- the last CTA groups everything
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = (atomicAdd(done, 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  int32_t* counts = rsm;
+  int32_t* cursor = rsm + E;
+  const int n = T * k;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) counts[e] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) atomicAdd(&counts[__ldcg(&ids[i])], 1);
+  __syncthreads();
+  if (warp == 0) {
+    const int per = (E + 31) / 32;
+    const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+    int sc = 0, ac = 0;
+    for (int e = e0; e < e1; ++e) sc += counts[e], ac += counts[e] > 0;
+    int si = sc, ai = ac;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int s2 = __shfl_up_sync(0xffffffffu, si, o), a2 = __shfl_up_sync(0xffffffffu, ai, o);
+      if (lane >= o) si += s2, ai += a2;
+    }
+    int run = si - sc, arun = ai - ac;
+    for (int e = e0; e < e1; ++e) {
+      const int c = counts[e];
+      offsets_out[e] = run;
+      cursor[e] = run;
+      counts_out[e] = c;
+      if (c > 0) {
+        active_out[arun] = e;
+        slot_info[arun] = make_int4(e, run, c, 0);
+        ++arun;
+      }
+      run += c;
+    }
+    if (lane == 31) offsets_out[E] = si, *n_active_out = ai;
+    __syncwarp();
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = 0; base < n; base += 32) {
+      const int i = base + lane;
+      const int e = i < n ? __ldcg(&ids[i]) : -1 - lane;
+      const unsigned mask = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(mask & lt);
+      const int cur = i < n ? cursor[e] : 0;
+      __syncwarp();
+      if (i < n) {
+        perm_out[cur + rank] = i;
+        if (rank == 0) cursor[e] = cur + __popc(mask);
+      }
+      __syncwarp();
+    }
+  }
+  if (threadIdx.x == 0) *done = 0;
+}
+
 }  // namespace
 
 cudaError_t launch_router_f32(const scion_layer* L, const __nv_bfloat16* x, int T, float* logits, cudaStream_t s) {
@@ -181,10 +259,43 @@ cudaError_t launch_router_f32(const scion_layer* L, const __nv_bfloat16* x, int 
 }
 
 cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s) {
+  if (L->E <= 512) {
+    const size_t smem = sizeof(int32_t) * 2 * size_t(L->E);
+    const dim3 grid((T + 3) / 4);
+#define SCION_ROUTE_PAR(V)                                                                                 \
+  return launch_pdl(route_par_kernel<V>, grid, dim3(128), smem, s, L->logits, T, L->E, L->k, L->desc.norm_topk, \
+                    L->ids, L->gates, L->counts, L->offsets, L->perm, L->active, L->n_active,                 \
+                    reinterpret_cast<int4*>(L->slot_info), L->route_done)
+    const int vpl = (L->E + 31) / 32;
+    if (vpl <= 1) SCION_ROUTE_PAR(1);
+    else if (vpl <= 2) SCION_ROUTE_PAR(2);
+    else if (vpl <= 4) SCION_ROUTE_PAR(4);
+    else if (vpl <= 8) SCION_ROUTE_PAR(8);
+    else SCION_ROUTE_PAR(16);
+#undef SCION_ROUTE_PAR
+    return cudaGetLastError();
+  }
   size_t smem = sizeof(float) * (size_t(kRouteThreads / 32) * L->E) + sizeof(int32_t) * (2 * size_t(L->E)) +
                 sizeof(int32_t) * size_t(T) * L->k;
   route_kernel<<<1, kRouteThreads, smem, s>>>(L->logits, T, L->E, L->k, L->desc.norm_topk, L->ids, L->gates,
                                                L->counts, L->offsets, L->perm, L->active, L->n_active);
+  if (cudaError_t e = cudaGetLastError()) return e;
+  return launch_slot_info(L, s);
+}
+
+__global__ void slot_info_kernel(const int32_t* __restrict__ active, const int32_t* __restrict__ n_active,
+                                 const int32_t* __restrict__ offsets, const int32_t* __restrict__ counts,
+                                 int4* __restrict__ slot_info, int E) {
+  const int n = *n_active;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int e = active[i];
+    slot_info[i] = make_int4(e, offsets[e], counts[e], 0);
+  }
+}
+
+cudaError_t launch_slot_info(const scion_layer* L, cudaStream_t s) {
+  slot_info_kernel<<<(L->E + 255) / 256, 256, 0, s>>>(L->active, L->n_active, L->offsets, L->counts,
+                                                       reinterpret_cast<int4*>(L->slot_info), L->E);
   return cudaGetLastError();
 }
 

@@ -42,15 +42,16 @@ cudaError_t dev_alloc(scion_layer* L, T** p, size_t bytes) {
 
 void free_layer(scion_layer* L) {
   if (!L) return;
-  void* ptrs[] = {L->gu_bank, L->dn_bank, L->dense_down, L->xunits,  L->logits, L->ids,      L->gates,
-                  L->counts,  L->offsets, L->perm,       L->active,  L->n_active, L->h,      L->hz,
-                  L->xfrag,   L->xpartial, L->xcount,    L->x_stage, L->out_stage, L->bad,   L->err};
+  void* ptrs[] = {L->gu_bank, L->dn_bank,  L->dense_down, L->xunits,  L->logits,    L->ids,       L->gates,
+                  L->counts,  L->offsets,  L->perm,       L->active,  L->n_active,  L->h,         L->hz,
+                  L->xfrag,   L->xpartial, L->xcount,     L->x_stage, L->out_stage, L->bad,       L->err,
+                  L->slot_info, L->route_done};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   if (L->pre) {
     scion::PrefillState* P = L->pre;
     void* pp[] = {P->xunits, P->dunits, P->logits, P->ids, P->gates, P->counts, P->offsets,
-                  P->perm,   P->tiles,  P->n_tiles, P->x16, P->h,    P->hz};
+                  P->perm,   P->inv,    P->y,       P->tiles, P->n_tiles, P->x16, P->h, P->hz};
     for (void* p : pp)
       if (p) cudaFree(p);
     delete P;
@@ -76,6 +77,8 @@ int create_prefill(scion_layer* L, cudaStream_t s) {
   PTRY(dev_alloc(L, &P->counts, sizeof(int32_t) * L->E));
   PTRY(dev_alloc(L, &P->offsets, sizeof(int32_t) * (L->E + 1)));
   PTRY(dev_alloc(L, &P->perm, sizeof(int32_t) * Tk));
+  PTRY(dev_alloc(L, &P->inv, sizeof(int32_t) * Tk));
+  PTRY(dev_alloc(L, &P->y, sizeof(float) * Tk * L->d));
   PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->tiles), scion::prefill_tile_bytes() * max_tiles));
   PTRY(dev_alloc(L, &P->n_tiles, sizeof(int32_t)));
   PTRY(dev_alloc(L, &P->x16, sizeof(__half) * T * L->d));
@@ -169,6 +172,7 @@ int forward_prefill(const scion_layer* L, const __nv_bfloat16* x, int T, float* 
   SCION_STAGE(SCION_STAGE_GATEUP, scion::launch_prefill_stage(SCION_STAGE_GATEUP, L, x, T, out, s));
   SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_prefill_stage(SCION_STAGE_DOWN_DENSE, L, x, T, out, s));
   SCION_STAGE(SCION_STAGE_DOWN_ROUTED, scion::launch_prefill_stage(SCION_STAGE_DOWN_ROUTED, L, x, T, out, s));
+  SCION_STAGE(SCION_STAGE_COMBINE, scion::launch_prefill_stage(SCION_STAGE_COMBINE, L, x, T, out, s));
   return SCION_OK;
 }
 
@@ -177,8 +181,10 @@ int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out
   if (L->desc.router_fp32) SCION_STAGE(SCION_STAGE_ROUTER_F32, scion::launch_router_f32(L, x, T, L->logits, s));
   SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_xproj(L, x, T, out, s));
   SCION_STAGE(SCION_STAGE_ROUTE, scion::launch_route(L, T, s));
-  SCION_STAGE(SCION_STAGE_GATEUP, scion::launch_gateup(L, x, T, s));
-  SCION_STAGE(SCION_STAGE_DOWN_ROUTED, scion::launch_down_routed(L, T, out, s));
+  const bool ring = T >= L->stream_min_tokens;
+  SCION_STAGE(SCION_STAGE_GATEUP, ring ? scion::launch_stream_gateup(L, T, s) : scion::launch_gateup(L, x, T, s));
+  SCION_STAGE(SCION_STAGE_DOWN_ROUTED,
+              ring ? scion::launch_stream_down(L, T, out, s) : scion::launch_down_routed(L, T, out, s));
   if (L->Kdense) SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
   return SCION_OK;
 }
@@ -225,6 +231,7 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   L->Gd = L->d / 128, L->GF = L->F / 128;
   L->Kdense = L->Fs + L->r;
   L->Kd = (L->Kdense + 63) / 64 * 64;
+  L->stream_min_tokens = SCION_TDEC + 1;  // the split-K register kernels measured faster at every decode batch size
   cudaStream_t s = as_stream(stream);
   const int tb = scion::tile_bytes(L->fmt);
   const int TD = SCION_TDEC;
@@ -251,6 +258,9 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   SCION_TRY(dev_alloc(L, &L->perm, sizeof(int32_t) * TD * L->k));
   SCION_TRY(dev_alloc(L, &L->active, sizeof(int32_t) * L->E));
   SCION_TRY(dev_alloc(L, &L->n_active, sizeof(int32_t)));
+  SCION_TRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&L->slot_info), sizeof(int4) * L->E));
+  SCION_TRY(dev_alloc(L, &L->route_done, sizeof(unsigned)));
+  SCION_TRY(cudaMemsetAsync(L->route_done, 0, sizeof(unsigned), s));
   SCION_TRY(dev_alloc(L, &L->h, sizeof(__half) * TD * L->k * L->F));
   SCION_TRY(dev_alloc(L, &L->hz, sizeof(__half) * TD * (L->Kd ? L->Kd : 1)));
   SCION_TRY(dev_alloc(L, &L->xfrag, sizeof(__half) * TD * L->d));
@@ -419,3 +429,15 @@ extern "C" int scion_profile_end(int n_stages, double* ms_total, int64_t* launch
 }
 
 extern "C" int64_t scion_kernel_launches(void) { return g_launches.load(); }
+
+extern "C" int scion_layer_set_option(scion_layer* L, int option, int value) {
+  if (!L) return SCION_EINVAL;
+  switch (option) {
+    case SCION_OPT_STREAM_MIN_TOKENS:
+      if (value < 1) return SCION_EINVAL;
+      L->stream_min_tokens = value;
+      return SCION_OK;
+    default:
+      return SCION_EINVAL;
+  }
+}

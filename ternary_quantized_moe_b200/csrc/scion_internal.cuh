@@ -28,6 +28,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/scion.h"
 
 #define SCION_TDEC 64         // tokens per decode pass (larger batches run in passes)
@@ -65,6 +67,8 @@ struct PrefillState {
   int32_t* counts;      // [E]
   int32_t* offsets;     // [E+1]
   int32_t* perm;        // [maxT*k]
+  int32_t* inv;         // [maxT*k] position of entry t*k+j in perm
+  float* y;             // [maxT*k][d] gate-weighted expert outputs, one row per routed (token, slot)
   void* tiles;          // 128-token tiles, [maxT*k/128 + E]
   int32_t* n_tiles;
   __half* x16;          // [maxT][d]   x in the container column order (fp16)
@@ -96,6 +100,8 @@ struct scion_layer {
   int32_t* perm;     // [TDEC*k]
   int32_t* active;   // [E]
   int32_t* n_active; // [1]
+  void* slot_info;    // int4 [E]: {expert, first position, token count, 0} per active slot
+  unsigned* route_done;  // [1] arrival counter of the decode route kernel
   __half* h;         // [TDEC*k][F]
   __half* hz;        // [TDEC][Kd] (pad columns stay 0)
   __half* xfrag;     // [TDEC][Gd][128] x in fragment order (fp16)
@@ -106,6 +112,7 @@ struct scion_layer {
   int64_t* bad;      // [1] invalid-code counter used at create
   int* err;          // [1] device status word (a bounded wait that gave up writes ETIMEOUT)
   scion::PrefillState* pre;  // tensor-core path (nullptr when max_tokens <= SCION_TDEC)
+  int stream_min_tokens;     // decode batches of at least this many tokens use the bulk-copy ring kernels
   size_t device_bytes;
 };
 
@@ -128,6 +135,7 @@ cudaError_t launch_bf16_to_f16_rows(const __nv_bfloat16* src, int rows, int cols
 cudaError_t launch_router_f32(const scion_layer* L, const __nv_bfloat16* x, int T, float* logits, cudaStream_t s);
 cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s);
 cudaError_t configure_route_kernels();
+cudaError_t launch_slot_info(const scion_layer* L, cudaStream_t s);
 
 // k_decode.cu
 cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, cudaStream_t s);
@@ -137,6 +145,11 @@ cudaError_t launch_down_dense(const scion_layer* L, int T, float* out, cudaStrea
 // fragment-ordered rows [rows][G][128] -> natural order [rows][G*128]
 cudaError_t launch_unfrag(int fmt, const __half* src, int rows, int G, __half* dst, cudaStream_t s);
 cudaError_t configure_kernels();
+
+// k_stream.cu (bulk-copy-ring expert kernels for decode batches)
+cudaError_t configure_stream_kernels();
+cudaError_t launch_stream_gateup(const scion_layer* L, int T, cudaStream_t s);
+cudaError_t launch_stream_down(const scion_layer* L, int T, float* out, cudaStream_t s);
 
 // k_prefill.cu
 int make_tmap_2d(CUtensorMap* map, const void* ptr, int bf16, int64_t rows, int64_t K);
@@ -149,7 +162,31 @@ cudaError_t launch_unperm_prefill(int fmt, const __half* src, int64_t n, __half*
 cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfloat16* x, int T, float* out,
                                  cudaStream_t s);
 
+// Launch with programmatic dependent launch: the kernel may start while its predecessor
+// on the stream drains; it must execute pdl_wait() before touching anything the
+// predecessor (or anything earlier on the stream) writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ------------------------------------------------------------ device helpers
+// Wait until the preceding grid on the stream has completed and its writes are visible.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the next grid on the stream to be scheduled (it still waits in pdl_wait()).
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
