@@ -80,6 +80,18 @@ def stage_bytes(cfg, T, U):
     }
 
 
+def stage_flops(cfg, T):
+    """Algorithmic tensor-core FLOPs per launch of each GEMM stage (no padding counted)."""
+    d, F, k, Fs, r, E = cfg.d, cfg.ffn, cfg.top_k, cfg.shared_ffn, cfg.rank, cfg.n_experts
+    return {
+        "router_f32": 2 * T * 2 * E * d,
+        "xproj": 2 * T * ((0 if cfg.router_f32 else 2 * E * d) + 2 * Fs * d + r * d),
+        "gateup": 2 * T * k * 2 * d * F,
+        "down_routed": 2 * T * k * d * F,
+        "down_dense": 2 * T * d * (Fs + r),
+    }
+
+
 def workload_flops(cfg, T):
     return 2 * T * (cfg.top_k * 3 * cfg.d * cfg.ffn + 3 * cfg.d * cfg.shared_ffn + 2 * cfg.n_experts * cfg.d
                     + 2 * cfg.rank * cfg.d)
@@ -320,10 +332,12 @@ def run_gpu(args, rank, world, local_rank):
                 U[(li, T)] = cfg.n_experts
     sched = [((s * nb + i) % n_layers, T) for s in range(K) for i, T in enumerate(batches)]
     bytes_total = sum(workload_bytes(cfg, T, U[(li, T)]) for li, T in sched)
-    sbytes = {}
+    sbytes, sflops = {}, {}
     for li, T in sched:
         for k_, v in stage_bytes(cfg, T, U[(li, T)]).items():
             sbytes[k_] = sbytes.get(k_, 0) + v
+        for k_, v in stage_flops(cfg, T).items():
+            sflops[k_] = sflops.get(k_, 0) + v
     flops_total = sum(workload_flops(cfg, T) for _, T in sched)
 
     # ---- per batch size (each batch alone, cycling layers)
@@ -359,11 +373,11 @@ def run_gpu(args, rank, world, local_rank):
                 "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
                 "bytes_per_launch": sbytes[dom] / dom_n, "us_per_launch": 1000.0 * dom_ms / dom_n}
     else:
-        fl = flops_total  # attributed to the dominant (expert GEMM) kernel when prefill
-        achieved = fl / (dom_ms / 1000.0) / 1e12
+        achieved = sflops[dom] / (dom_ms / 1000.0) / 1e12  # the dominant kernel's own FLOPs / its time
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
-                "peak_source": peak_src}
+                "peak_source": peak_src, "flops_per_launch": sflops[dom] / dom_n,
+                "us_per_launch": 1000.0 * dom_ms / dom_n}
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -379,6 +393,10 @@ def run_gpu(args, rank, world, local_rank):
                           (peaks["hbm_gbs"] * 1e9), "tflops": flops_total / (ms / 1000.0) / 1e12},
         "per_batch": per_batch,
         "stages_us_per_launch": {k_: 1000.0 * v[0] / v[1] for k_, v in stages.items() if v[1]},
+        "stages_rate": {k_: (sbytes[k_] / (v[0] / 1000.0) / 1e9 if decode else
+                             sflops.get(k_, 0) / (v[0] / 1000.0) / 1e12)
+                        for k_, v in stages.items() if v[1] and k_ in sbytes},
+        "stages_rate_unit": "GB/s" if decode else "TFLOP/s",
         "stages_share": {k_: v[0] / sum(x[0] for x in stages.values()) for k_, v in stages.items() if v[1]},
         "e2e": e2e,
         "gpu_launches": int(launches),

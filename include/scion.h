@@ -205,7 +205,7 @@ enum {
   SCION_STAGE_DOWN_ROUTED = 4, /* ternary expert down + gate-weighted scatter-add */
   SCION_STAGE_DOWN_DENSE = 5,  /* shared down + correction B */
   SCION_STAGE_X16 = 6,         /* x -> fp16 in container column order (tensor-core path) */
-  SCION_STAGE_COMBINE = 7,     /* sum of the k gate-weighted expert rows per token (tensor-core path) */
+  SCION_STAGE_COMBINE = 7,     /* gate-weighted sum of the k expert rows per token (tensor-core path) */
   SCION_N_STAGES = 8
 };
 /* Creates a pool for `max_launches` launches and starts recording (EINVAL if already

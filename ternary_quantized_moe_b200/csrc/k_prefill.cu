@@ -104,7 +104,7 @@ constexpr int kBK = 64;
 
 __global__ void __launch_bounds__(kThreads, 1) dense_gemm_kernel(const __grid_constant__ DenseParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // 1024-aligned, still __shared__
   __shared__ uint64_t full[kDenseStages], empty[kDenseStages], accf;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
@@ -210,12 +210,20 @@ namespace scion {
 namespace {
 
 // -------------------------------------------------------------- ternary GEMM
-struct TernTile {
-  int e;   // expert
-  int c0;  // first token (within the expert's group) of this 128-token tile
+struct __align__(16) TernTile {
+  int e;     // expert
+  int c0;    // first token (within the expert's group) of this 128-token tile
+  int n;     // tokens in the tile (1..128)
+  int pos0;  // routed-order position of its first token (offsets[e] + c0)
 };
 
+__device__ __forceinline__ TernTile load_tile(const TernTile* tiles, int i) {
+  const int4 v = __ldg(reinterpret_cast<const int4*>(tiles) + i);
+  return TernTile{v.x, v.y, v.z, v.w};
+}
+
 struct TernParams {
+  CUtensorMap bmap;     // down projection: B = h [T*k][F], box {64, 128}
   const uint8_t* bank;  // re-tiled gate/up bank (na = 2) or down bank (na = 1)
   int fmt, na, G, R;    // groups along K, rows per expert matrix
   const __half* bsrc;   // B rows: x16 [T][d] (gate/up) or h [T*k][F] (down)
@@ -226,27 +234,24 @@ struct TernParams {
   const float* gates;
   int k;
   __half* h;  int F;     // gate/up output
-  float* y;   int d;     // down output: gate-weighted rows per routed (token, slot), [T*k][d]
+  float* y;   int d;     // down output: one row per routed (token, slot), [T*k][d], gates applied by the combine
   int* err;
 };
 
 constexpr uint32_t kAtom = 128 * 128;  // bytes of one 128-row x 64-column swizzled atom
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-
 // Expand half h (64 columns) of row t (0..127) of one 128-row group from its sub-tile block
-// into a 128-row x 64-column swizzled fp16 atom.  Values are code * scale, exact in fp16.
-__device__ __forceinline__ void expand_pq2_half(const uint8_t* codes, int t, int h, uint32_t atom) {
-  const uint8_t* blk = codes + (t >> 4) * kPq2Tile;
+// into 32 registers of fp16 pairs, in position order (v[i] = positions 2i, 2i+1 of the half).
+// Values are code * scale, exact in fp16.
+__device__ __forceinline__ void expand_pq2_half(uint32_t codes, int t, int h, uint32_t (&out)[32]) {
+  const uint32_t blk = codes + (t >> 4) * kPq2Tile;
   const int rho = t & 15, r8 = rho & 7, hi = rho >> 3;
-  const __half2 sc = __half2half2(__ushort_as_half(*reinterpret_cast<const uint16_t*>(blk + 512 + 4 * r8 + 2 * hi)));
+  const __half2 sc = __half2half2(__ushort_as_half(uint16_t(lds_u16(blk + 512 + 4 * r8 + 2 * hi))));
   const __half2 bias = u32_as_h2(0x64016401u);
 #pragma unroll
   for (int cc = 0; cc < 2; ++cc) {
     const int c = 2 * h + cc;  // container code bytes 8c .. 8c+7 = words 2c, 2c+1
-    const uint2 w2 = *reinterpret_cast<const uint2*>(blk + 16 * (4 * r8 + c) + 8 * hi);
+    const uint2 w2 = lds_v2(blk + 16 * (4 * r8 + c) + 8 * hi);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const uint32_t w = half ? w2.y : w2.x;
@@ -254,24 +259,23 @@ __device__ __forceinline__ void expand_pq2_half(const uint8_t* codes, int t, int
 #pragma unroll
       for (int s = 0; s < 8; ++s)
         v[s] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w >> (2 * s), 0x00030003u, 0x64006400u)), bias), sc));
-      const int j0 = 2 * (2 * cc + half);  // chunk index inside the atom
-      st_shared_v4(atom + sw128_offset(t, j0), v[0], v[1], v[2], v[3]);
-      st_shared_v4(atom + sw128_offset(t, j0 + 1), v[4], v[5], v[6], v[7]);
+      const int j0 = 2 * (2 * cc + half);  // 8-position chunk index inside the half
+#pragma unroll
+      for (int i = 0; i < 8; ++i) out[4 * j0 + i] = v[i];
     }
   }
 }
 
-__device__ __forceinline__ void expand_ptq1_half(const uint8_t* codes, int t, int h, uint32_t atom) {
-  const uint8_t* blk = codes + (t >> 4) * kPtq1Tile;
+__device__ __forceinline__ void expand_ptq1_half(uint32_t codes, int t, int h, uint32_t (&v)[32]) {
+  const uint32_t blk = codes + (t >> 4) * kPtq1Tile;
   const int rho = t & 15, r8 = rho & 7, hi = rho >> 3;
-  const __half2 sc = __half2half2(__ushort_as_half(*reinterpret_cast<const uint16_t*>(blk + 416 + 4 * r8 + 2 * hi)));
+  const __half2 sc = __half2half2(__ushort_as_half(uint16_t(lds_u16(blk + 416 + 4 * r8 + 2 * hi))));
   const __half2 third = __float2half2_rn(0.333251953125f), c1 = __float2half2_rn(682.5f);
   const __half2 m3 = __float2half2_rn(-3.0f), c2047 = __float2half2_rn(2047.0f);
-  uint32_t v[32];
 #pragma unroll
   for (int i = 0; i < 6; ++i) {
     const int q = 12 * h + 2 * i;
-    const uint32_t x = *reinterpret_cast<const uint16_t*>(blk + 12 * (4 * r8 + q / 6) + 6 * hi + q % 6);
+    const uint32_t x = lds_u16(blk + 12 * (4 * r8 + q / 6) + 6 * hi + q % 6);
     uint32_t pr;
     asm("prmt.b32 %0, %1, 0, 0x4140;" : "=r"(pr) : "r"(x));
     __half2 V = u32_as_h2(pr | 0x64006400u);
@@ -285,7 +289,7 @@ __device__ __forceinline__ void expand_ptq1_half(const uint8_t* codes, int t, in
   }
   {
     // remainder trits: digits 0..4 of byte 24 and 0..2 of the tail byte, one digit chain
-    const uint32_t qt = *reinterpret_cast<const uint16_t*>(blk + 384 + 4 * r8 + 2 * hi);
+    const uint32_t qt = lds_u16(blk + 384 + 4 * r8 + 2 * hi);
     uint32_t pr;
     asm("prmt.b32 %0, %1, 0, 0x4140;" : "=r"(pr) : "r"(qt));
     __half2 V = u32_as_h2(pr | 0x64006400u);
@@ -307,36 +311,44 @@ __device__ __forceinline__ void expand_ptq1_half(const uint8_t* codes, int t, in
     v[30] = h2_as_u32(__hmul2(u32_as_h2(r0), sc));
     v[31] = h2_as_u32(__hmul2(u32_as_h2(r1), sc));
   }
-#pragma unroll
-  for (int j = 0; j < 8; ++j)
-    st_shared_v4(atom + sw128_offset(t, j), v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
 }
 
+// Pipeline granularity: one 128-column code group along K ("group" = two 64-column halves).
 template <int FMT, int NA>
 struct TernRing {
   static constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
-  static constexpr int kA = 3;                    // expanded 64-column A stages
-  static constexpr int kB = 4;                    // gathered 64-column B stages
-  static constexpr int kC = NA == 2 ? 3 : 4;      // packed code groups
-  static constexpr uint32_t a_bytes = NA * kAtom;  // one A stage: NA matrices x 128 rows x 128 B
+  // shared memory: B groups (two 128-row x 128 B atoms each) and packed code groups
+  static constexpr int kB = 4;
+  static constexpr int kC = 4;
+  static constexpr uint32_t b_bytes = 2 * kAtom;
   static constexpr uint32_t c_bytes = NA * 8 * tb;
-  static constexpr uint32_t slab_bytes = 2 * 16 * 128 * 4;  // epilogue: two 16-token slabs (fp32 worst case)
-  static constexpr uint32_t a_off = 0, b_off = kA * a_bytes, c_off = b_off + kB * kAtom;
-  static constexpr uint32_t slab_off = (c_off + kC * c_bytes + 127) & ~127u;
-  static constexpr uint32_t bytes = slab_off + slab_bytes;
+  static constexpr uint32_t b_off = 0, c_off = kB * b_bytes;
+  static constexpr uint32_t bytes = c_off + kC * c_bytes;
+  // tensor memory: accumulators, then the ring of expanded A groups
+  static constexpr int n_acc = NA == 2 ? 1 : 2;   // gate/up: one NA x 128 accumulator; down: ping-pong
+  static constexpr uint32_t acc_cols = NA * kBN;
+  static constexpr int kA = 2;
+  static constexpr uint32_t a_cols = NA * 64;     // one group: NA matrices x 64 columns (128 fp16 per lane)
+  static constexpr uint32_t a_col0 = n_acc * acc_cols;
+  static constexpr uint32_t tmem_cols = 512;
+  static_assert(a_col0 + kA * a_cols <= tmem_cols, "TMEM budget");
 };
 
-constexpr int kTernThreads = 384;  // 12 warps: codes, MMA, B rows, (idle), 4 expansion, 4 epilogue
+constexpr int kTernThreads = 512;  // 16 warps: codes, MMA, 2 x B rows, 8 expansion, 4 epilogue
+constexpr int kEpiThreads = 128;
 
 // Persistent grouped GEMM: CTA b walks the work items b, b + gridDim.x, ... where item =
-// (128-token tile, 128-row weight tile).  All roles walk the same sequence; the rings and the
-// two TMEM accumulators carry over from one item to the next, so loads, expansion and MMAs of
-// item i+1 overlap the epilogue of item i.
+// (128-token tile, 128-row weight tile).  The expansion warps decode the packed codes of each
+// 128-column group straight into tensor memory (one weight row per TMEM lane), and the MMA
+// reads A from there and the tokens (B) from shared memory.  All roles walk the same item
+// sequence; rings carry over from one item to the next.  The MMA issuer waits on a single
+// barrier per group: the expansion side folds the B-ready condition into its own arrival.
 template <int FMT, int NA>
 __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid_constant__ TernParams p) {
   using R = TernRing<FMT, NA>;
+  constexpr bool kBTma = NA == 1;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // 1024-aligned, still __shared__
   __shared__ uint64_t c_full[R::kC], c_empty[R::kC], a_full[R::kA], a_empty[R::kA], b_full[R::kB], b_empty[R::kB];
   __shared__ uint64_t acc_full[2], acc_empty[2], mma_done;
   __shared__ uint32_t tmem_slot;
@@ -345,20 +357,17 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int RT = p.R >> 7;                     // 128-row weight tiles per expert matrix
   const int n_items = *p.n_tiles * RT;
-  const int nkb = 2 * p.G;                     // 64-column stages per item
-  constexpr uint32_t acc_cols = NA * kBN;      // one accumulator: NA x 128 columns
-  constexpr uint32_t ncols = 2 * acc_cols;     // ping-pong
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < R::kC; ++i) mbar_init(&c_full[i], 1), mbar_init(&c_empty[i], 128);
-    for (int i = 0; i < R::kA; ++i) mbar_init(&a_full[i], 128), mbar_init(&a_empty[i], 1);
-    for (int i = 0; i < R::kB; ++i) mbar_init(&b_full[i], 32), mbar_init(&b_empty[i], 1);
-    for (int i = 0; i < 2; ++i) mbar_init(&acc_full[i], 1), mbar_init(&acc_empty[i], 128);
+    for (int i = 0; i < R::kC; ++i) mbar_init(&c_full[i], 1), mbar_init(&c_empty[i], 256);
+    for (int i = 0; i < R::kA; ++i) mbar_init(&a_full[i], 256), mbar_init(&a_empty[i], 1);
+    for (int i = 0; i < R::kB; ++i) mbar_init(&b_full[i], kBTma ? 1 : 64), mbar_init(&b_empty[i], 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&acc_full[i], 1), mbar_init(&acc_empty[i], kEpiThreads);
     mbar_init(&mma_done, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(&tmem_slot, ncols);
+  if (warp == 1) tmem_alloc(&tmem_slot, R::tmem_cols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -369,9 +378,9 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
     // ---------------- packed code blocks, one 128-row group per bulk copy and matrix
     if (lane == 0) {
       const int64_t mat_stride = int64_t(8) * R::tb, grp_stride = NA * mat_stride;
-      int gs = 0;  // running group-stage counter
+      int gs = 0;  // running group counter
       for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
-        const TernTile tile = p.tiles[item / RT];
+        const TernTile tile = load_tile(p.tiles, item / RT);
         const int rt = item % RT;
         const uint8_t* ebase = p.bank + (int64_t(tile.e) * RT + rt) * p.G * grp_stride;
         for (int g = 0; g < p.G; ++g, ++gs) {
@@ -387,66 +396,88 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
       // the last kC groups issued may still be in flight if a consumer gave up: let them land
       for (int i = max(0, gs - R::kC); i < gs; ++i) mbar_drain(&c_full[i % R::kC], (i / R::kC) & 1);
     }
-  } else if (warp == 2) {
-    // ---------------- gathered B rows, 64 columns (128 B) per stage
-    int ks = 0;  // running stage counter
-    for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
-      const TernTile tile = p.tiles[item / RT];
-      const int p0 = p.offsets[tile.e];
-      const int nn = min(kBN, p.counts[tile.e] - tile.c0);
-      const __half* rows[kBN / 32];
-#pragma unroll
-      for (int i = 0; i < kBN / 32; ++i) {
-        const int r = lane + 32 * i;
-        rows[i] = nullptr;
-        if (r < nn) {
-          const int64_t src = NA == 2 ? int64_t(p.perm[p0 + tile.c0 + r] / p.k) : int64_t(p0 + tile.c0 + r);
-          rows[i] = p.bsrc + src * p.ldb;
+  } else if (kBTma && warp == 2) {
+    // ---------------- B rows are contiguous (h in routed order): two TMA boxes per group
+    if (lane == 0) {
+      int gs = 0;
+      for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
+        const int row0 = load_tile(p.tiles, item / RT).pos0;
+        for (int g = 0; g < p.G; ++g, ++gs) {
+          const int s = gs % R::kB;
+          if (gs >= R::kB && !mbar_wait(&b_empty[s], ((gs / R::kB) - 1) & 1, &abort_flag, p.err)) break;
+          uint8_t* dst = smem + R::b_off + s * R::b_bytes;
+          mbar_arrive_expect_tx(&b_full[s], R::b_bytes);
+          tma_load_2d(dst, &p.bmap, g * 128, row0, &b_full[s]);
+          tma_load_2d(dst + kAtom, &p.bmap, g * 128 + 64, row0, &b_full[s]);
         }
       }
-      for (int kb = 0; kb < nkb; ++kb, ++ks) {
-        const int s = ks % R::kB;
-        if (ks >= R::kB && !mbar_wait(&b_empty[s], ((ks / R::kB) - 1) & 1, &abort_flag, p.err)) break;
-        const uint32_t bt = sbase + R::b_off + s * kAtom;
+      for (int i = max(0, gs - R::kB); i < gs; ++i) mbar_drain(&b_full[i % R::kB], (i / R::kB) & 1);
+    }
+  } else if (!kBTma && (warp == 2 || warp == 3)) {
+    // ---------------- gathered B rows (tokens of the tile), 128 columns (two atoms) per group;
+    // warp 2 takes rows 0..63, warp 3 rows 64..127
+    const int rbase = (warp - 2) * 64;
+    constexpr int kLag = R::kB / 2;  // groups in flight per thread before the oldest is published
+    int gs = 0;                      // running group counter
+    for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
+      const TernTile tile = load_tile(p.tiles, item / RT);
+      const __half* rows[2];
 #pragma unroll
-        for (int i = 0; i < kBN / 32; ++i) {
+      for (int i = 0; i < 2; ++i) {
+        const int r = rbase + lane + 32 * i;
+        rows[i] = r < tile.n ? p.bsrc + int64_t(p.perm[tile.pos0 + r] / p.k) * p.ldb : nullptr;
+      }
+      for (int g = 0; g < p.G; ++g, ++gs) {
+        const int s = gs % R::kB;
+        if (gs >= R::kB && !mbar_wait(&b_empty[s], ((gs / R::kB) - 1) & 1, &abort_flag, p.err)) break;
+        const uint32_t bt = sbase + R::b_off + s * R::b_bytes;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
           if (!rows[i]) continue;
-          const int r = lane + 32 * i;
-          const __half* src = rows[i] + kb * 64;
+          const int r = rbase + lane + 32 * i;
+          const __half* src = rows[i] + g * 128;
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(bt + sw128_offset(r, j)), "l"(src + 8 * j)
+          for (int j = 0; j < 16; ++j)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(bt + (j >> 3) * kAtom + sw128_offset(r, j & 7)),
+                         "l"(src + 8 * j)
                          : "memory");
         }
-        cp_async_arrive_noinc(&b_full[s]);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        // group gs - kLag has landed: make it visible to the tensor cores (async proxy), then publish it
+        if (gs >= kLag) {
+          asm volatile("cp.async.wait_group %0;" ::"n"(kLag) : "memory");
+          fence_proxy_async();
+          mbar_arrive(&b_full[(gs - kLag) % R::kB]);
+        }
       }
     }
     cp_async_wait_all();
+    fence_proxy_async();
+    for (int i = max(0, gs - kLag); i < gs; ++i) mbar_arrive(&b_full[i % R::kB]);
   } else if (warp == 1) {
     if (lane == 0) {
-      // ---------------- MMA issuer
-      int ks = 0, li = 0;
+      // ---------------- MMA issuer: A from tensor memory, B from shared memory
+      int gs = 0, li = 0;
+      TernTile next = blockIdx.x < n_items ? load_tile(p.tiles, blockIdx.x / RT) : TernTile{};
       for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x, ++li) {
-        const TernTile tile = p.tiles[item / RT];
-        const int nn = min(kBN, p.counts[tile.e] - tile.c0);
-        const uint32_t idesc = umma_idesc(kBM, (nn + 15) & ~15, 0);
-        const int ab = li & 1;
-        if (li >= 2 && !mbar_wait(&acc_empty[ab], ((li >> 1) - 1) & 1, &abort_flag, p.err)) break;
+        const TernTile tile = next;  // loaded one item ahead: no global-load latency between items
+        if (item + int(gridDim.x) < n_items) next = load_tile(p.tiles, (item + gridDim.x) / RT);
+        const uint32_t idesc = umma_idesc(kBM, (tile.n + 15) & ~15, 0);
+        const int ab = li % R::n_acc;
+        if (li >= R::n_acc && !mbar_wait(&acc_empty[ab], ((li / R::n_acc) - 1) & 1, &abort_flag, p.err)) break;
         tc_fence_after();
-        const uint32_t acc = tmem + ab * acc_cols;
-        for (int kb = 0; kb < nkb; ++kb, ++ks) {
-          const int sa = ks % R::kA, sb = ks % R::kB;
-          if (!mbar_wait(&a_full[sa], (ks / R::kA) & 1, &abort_flag, p.err)) break;
-          if (!mbar_wait(&b_full[sb], (ks / R::kB) & 1, &abort_flag, p.err)) break;
+        const uint32_t acc = tmem + ab * R::acc_cols;
+        for (int g = 0; g < p.G; ++g, ++gs) {
+          const int sa = gs % R::kA, sb = gs % R::kB;
+          // A expanded and (folded into the same arrival) B landed
+          if (!mbar_wait(&a_full[sa], (gs / R::kA) & 1, &abort_flag, p.err)) break;
           tc_fence_after();
-          fence_proxy_async();
-          const uint32_t at = sbase + R::a_off + sa * R::a_bytes, bt = sbase + R::b_off + sb * kAtom;
+          const uint32_t at = tmem + R::a_col0 + sa * R::a_cols, bt = sbase + R::b_off + sb * R::b_bytes;
 #pragma unroll
-          for (int k16 = 0; k16 < 4; ++k16) {
-            const uint64_t db = umma_desc_sw128(bt + 32 * k16);
+          for (int k16 = 0; k16 < 8; ++k16) {
+            const uint64_t db = umma_desc_sw128(bt + (k16 >> 2) * kAtom + 32 * (k16 & 3));
 #pragma unroll
-            for (int m = 0; m < NA; ++m)
-              umma_f16(acc + m * kBN, umma_desc_sw128(at + m * kAtom + 32 * k16), db, idesc, (kb | k16) != 0);
+            for (int m = 0; m < NA; ++m) umma_ts(acc + m * kBN, at + m * 64 + 8 * k16, db, idesc, (g | k16) != 0);
           }
           umma_commit(&a_empty[sa]);
           umma_commit(&b_empty[sb]);
@@ -457,101 +488,83 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
       umma_commit(&mma_done);
       mbar_drain(&mma_done, 0);
     }
-  } else if (warp >= 4 && warp < 8) {
-    // ---------------- expansion (one weight row per thread, one 64-column half per stage)
-    const int t = threadIdx.x - 128;
-    int ks = 0, gs = 0;
+  } else if (warp >= 4 && warp < 12) {
+    // ---------------- expansion: two warpgroups; group `part` decodes the 64-column half
+    // h == part of every code group, thread t of a warpgroup decoding weight row t into TMEM lane t
+    const int part = (warp - 4) >> 2;
+    const int t = (threadIdx.x - 128) & 127;
+    const bool b_watch = part == 0 && t == 0;  // this thread also waits for the group's B rows
+    const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16) + R::a_col0 + part * 32;
+    int gs = 0;  // running code-group counter
     for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
-      for (int kb = 0; kb < nkb; ++kb, ++ks) {
-        const int h = kb & 1, sc = gs % R::kC, sa = ks % R::kA;
-        if (h == 0 && !mbar_wait(&c_full[sc], (gs / R::kC) & 1, &abort_flag, p.err)) break;
-        if (ks >= R::kA && !mbar_wait(&a_empty[sa], ((ks / R::kA) - 1) & 1, &abort_flag, p.err)) break;
-        const uint8_t* codes = smem + R::c_off + sc * R::c_bytes;
+      for (int g = 0; g < p.G; ++g, ++gs) {
+        const int sc = gs % R::kC, sa = gs % R::kA;
+        if (!mbar_wait(&c_full[sc], (gs / R::kC) & 1, &abort_flag, p.err)) break;
+        if (gs >= R::kA && !mbar_wait(&a_empty[sa], ((gs / R::kA) - 1) & 1, &abort_flag, p.err)) break;
+        tc_fence_after();
+        const uint32_t codes = sbase + R::c_off + sc * R::c_bytes;
 #pragma unroll
         for (int m = 0; m < NA; ++m) {
-          const uint32_t atom = sbase + R::a_off + sa * R::a_bytes + m * kAtom;
+          uint32_t v[32];
           if constexpr (FMT == SCION_PQ2_0)
-            expand_pq2_half(codes + m * 8 * R::tb, t, h, atom);
+            expand_pq2_half(codes + m * 8 * R::tb, t, part, v);
           else
-            expand_ptq1_half(codes + m * 8 * R::tb, t, h, atom);
+            expand_ptq1_half(codes + m * 8 * R::tb, t, part, v);
+          tmem_st32(lane_base + sa * R::a_cols + m * 64, v);
         }
-        fence_proxy_async();
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&c_empty[sc]);
+        if (b_watch && !mbar_wait(&b_full[gs % R::kB], (gs / R::kB) & 1, &abort_flag, p.err)) break;
         mbar_arrive(&a_full[sa]);
-        if (h == 1) {
-          mbar_arrive(&c_empty[sc]);
-          ++gs;
-        }
       }
     }
-  } else if (warp >= 8) {
-    // ---------------- epilogue: TMEM lane quarter q = rows 32q .. 32q+31 of the weight tile
+  } else if (warp >= 12) {
+    // ---------------- epilogue: TMEM lane quarter q = weight rows 32q .. 32q+31, 16 tokens per
+    // chunk.  Stores go straight to global memory.
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    const int et = threadIdx.x - 256;  // 0..127
+    const int pcol = perm_pos(FMT, row);  // gate/up: position of this row inside its 128-column group of h
     int li = 0;
     // no abort-flag test in the loop condition: the 128 threads leave only together, by the vote
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++li) {
-      const TernTile tile = p.tiles[item / RT];
+      const TernTile tile = load_tile(p.tiles, item / RT);
       const int rt = item % RT;
-      const int p0 = p.offsets[tile.e];
-      const int nn = min(kBN, p.counts[tile.e] - tile.c0);
-      const int ab = li & 1;
-      if (!named_bar_and(1, 128, mbar_wait(&acc_full[ab], (li >> 1) & 1, &abort_flag, p.err))) break;
+      const int64_t pos0 = tile.pos0;
+      const int nn = tile.n;
+      const int ab = li % R::n_acc;
+      if (!named_bar_and(1, kEpiThreads, mbar_wait(&acc_full[ab], (li / R::n_acc) & 1, &abort_flag, p.err))) break;
       tc_fence_after();
-      const uint32_t acc = tmem + ab * acc_cols;
-      float* slab = reinterpret_cast<float*>(smem + R::slab_off);
+      const uint32_t acc = tmem + ab * R::acc_cols + (uint32_t(q * 32) << 16);
       for (int c = 0; c * 16 < nn; ++c) {
-        const int buf = c & 1;
         float v0[16], v1[16];
-        const uint32_t ta = acc + (uint32_t(q * 32) << 16) + c * 16;
-        tmem_ld16(ta, v0);
-        if (NA == 2) tmem_ld16(ta + kBN, v1);
+        if constexpr (NA == 2)
+          tmem_ld16x2(acc + c * 16, acc + kBN + c * 16, v0, v1);
+        else
+          tmem_ld16(acc + c * 16, v0);
+        const int n0 = c * 16;
         if constexpr (NA == 2) {
-          __half* hs = reinterpret_cast<__half*>(slab) + buf * 16 * 128;
-          const int pcol = perm_pos(FMT, row);  // position of this row inside its 128-column group
+          __half* dst = p.h + (pos0 + n0) * p.F + int64_t(rt) * kBM + pcol;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) hs[i * 128 + pcol] = __float2half_rn(silu_f(v0[i]) * v1[i]);
-          asm volatile("bar.sync 1, 128;" ::: "memory");
-          for (int j = et; j < 16 * 16; j += 128) {
-            const int i = j >> 4, ch = j & 15, n = c * 16 + i;
-            if (n < nn) {
-              const int64_t pos = p0 + tile.c0 + n;
-              *reinterpret_cast<uint4*>(p.h + pos * p.F + int64_t(rt) * kBM + ch * 8) =
-                  *reinterpret_cast<const uint4*>(hs + i * 128 + ch * 8);
-            }
-          }
+          for (int i = 0; i < 16; ++i)
+            if (n0 + i < nn) dst[int64_t(i) * p.F] = __float2half_rn(silu_f(v0[i]) * v1[i]);
         } else {
-          float* fs = slab + buf * 16 * 128;
-          float gv[16];
+          float* dst = p.y + (pos0 + n0) * p.d + int64_t(rt) * kBM + row;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int n = c * 16 + i;
-            gv[i] = n < nn ? p.gates[p.perm[p0 + tile.c0 + n]] : 0.f;
-          }
-#pragma unroll
-          for (int i = 0; i < 16; ++i) fs[i * 128 + row] = gv[i] * v0[i];
-          asm volatile("bar.sync 1, 128;" ::: "memory");
-          for (int j = et; j < 16 * 32; j += 128) {
-            const int i = j >> 5, ch = j & 31, n = c * 16 + i;
-            if (n < nn) {
-              const int64_t pos = p0 + tile.c0 + n;
-              *reinterpret_cast<float4*>(p.y + pos * p.d + int64_t(rt) * kBM + ch * 4) =
-                  *reinterpret_cast<const float4*>(fs + i * 128 + ch * 4);
-            }
-          }
+          for (int i = 0; i < 16; ++i)
+            if (n0 + i < nn) dst[int64_t(i) * p.d] = v0[i];
         }
       }
-      // accumulator drained (tcgen05.ld waited inside tmem_ld16): hand it back to the MMA warp
+      // accumulator drained: hand it back to the MMA warp
       tc_fence_before();
       mbar_arrive(&acc_empty[ab]);
-      asm volatile("bar.sync 1, 128;" ::: "memory");  // slabs free before the next item writes them
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, ncols);
+    tmem_dealloc(tmem, R::tmem_cols);
   }
 }
 
@@ -624,7 +637,7 @@ __global__ void __launch_bounds__(kGroupWarps * 32) group_kernel(const int32_t* 
     for (int e = e0; e < e1; ++e) {
       const int c = tot[e];
       offsets[e] = run;
-      for (int c0 = 0; c0 < c; c0 += kBN) tiles[trun++] = TernTile{e, c0};
+      for (int c0 = 0; c0 < c; c0 += kBN) tiles[trun++] = TernTile{e, c0, min(kBN, c - c0), run + c0};
       tot[e] = run;  // becomes the expert's base offset
       run += c;
     }
@@ -728,15 +741,18 @@ cudaError_t configure_prefill_kernels() {
 // out[t] (= dense part, or 0 when the layer has no shared expert and no correction)
 // += sum over slots j < k of y[inv[t*k + j]], in slot order.  One CTA per token.
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y, const int32_t* __restrict__ inv,
-                                                     int k, int d, int has_dense, float* __restrict__ out) {
+                                                     const float* __restrict__ gates, int k, int d, int has_dense,
+                                                     float* __restrict__ out) {
   const int t = blockIdx.x;
   const int32_t* iv = inv + int64_t(t) * k;
+  const float* gt = gates + int64_t(t) * k;
   float4* o = reinterpret_cast<float4*>(out + int64_t(t) * d);
   for (int c4 = threadIdx.x; c4 < d / 4; c4 += blockDim.x) {
     float4 acc = has_dense ? o[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < k; ++j) {
       const float4 v = reinterpret_cast<const float4*>(y + int64_t(iv[j]) * d)[c4];
-      acc.x += v.x, acc.y += v.y, acc.z += v.z, acc.w += v.w;
+      const float g = gt[j];
+      acc.x += g * v.x, acc.y += g * v.y, acc.z += g * v.z, acc.w += g * v.w;
     }
     o[c4] = acc;
   }
@@ -833,7 +849,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       return cudaGetLastError();
     }
     case SCION_STAGE_COMBINE: {
-      combine_kernel<<<T, 256, 0, s>>>(P.y, P.inv, L->k, L->d, P.n_dunits > 0, out);
+      combine_kernel<<<T, 256, 0, s>>>(P.y, P.inv, P.gates, L->k, L->d, P.n_dunits > 0, out);
       return cudaGetLastError();
     }
     case SCION_STAGE_DOWN_DENSE: {
@@ -855,6 +871,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       tp.tiles = static_cast<const TernTile*>(P.tiles), tp.n_tiles = P.n_tiles;
       tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gates = P.gates, tp.k = L->k;
       tp.h = nullptr, tp.F = L->F, tp.y = P.y, tp.d = L->d, tp.err = L->err;
+      if (make_tmap_2d(&tp.bmap, P.h, 0, int64_t(T) * L->k, L->F) != SCION_OK) return cudaErrorInvalidValue;
       const dim3 grid(num_sms());
       if (L->fmt == SCION_PQ2_0)
         tern_gemm_kernel<SCION_PQ2_0, 1><<<grid, kTernThreads, tern_smem(1, L->fmt), s>>>(tp);

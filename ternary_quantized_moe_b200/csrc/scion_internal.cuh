@@ -68,7 +68,7 @@ struct PrefillState {
   int32_t* offsets;     // [E+1]
   int32_t* perm;        // [maxT*k]
   int32_t* inv;         // [maxT*k] position of entry t*k+j in perm
-  float* y;             // [maxT*k][d] gate-weighted expert outputs, one row per routed (token, slot)
+  float* y;             // [maxT*k][d] expert down outputs (gate not yet applied), one row per routed (token, slot)
   void* tiles;          // 128-token tiles, [maxT*k/128 + E]
   int32_t* n_tiles;
   __half* x16;          // [maxT][d]   x in the container column order (fp16)
@@ -220,6 +220,8 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint3
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+// x * sigmoid(x) with the fast exponential and division (a few ulp of fp32; the result is
+// rounded to fp16 or multiplied into an fp32 accumulation well above that error).
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 }  // namespace scion
