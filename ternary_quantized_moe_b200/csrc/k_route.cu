@@ -57,6 +57,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
                                                               int32_t* __restrict__ counts_out,
                                                               int32_t* __restrict__ offsets_out,
                                                               int32_t* __restrict__ perm_out,
+                                                              float* __restrict__ gperm_out,
                                                               int32_t* __restrict__ active_out,
                                                               int32_t* __restrict__ n_active_out) {
   extern __shared__ float smem[];
@@ -165,6 +166,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
       __syncwarp();
       if (i < n) {
         perm_out[cur + rank] = i;
+        gperm_out[cur + rank] = gates_out[i];
         if (rank == 0) cursor[e] = cur + __popc(mask);
       }
       __syncwarp();
@@ -182,6 +184,7 @@ __global__ void __launch_bounds__(128) route_par_kernel(const float* __restrict_
                                                         float* __restrict__ gates, int32_t* __restrict__ counts_out,
                                                         int32_t* __restrict__ offsets_out,
                                                         int32_t* __restrict__ perm_out,
+                                                        float* __restrict__ gperm_out,
                                                         int32_t* __restrict__ active_out,
                                                         int32_t* __restrict__ n_active_out,
                                                         int4* __restrict__ slot_info, unsigned* __restrict__ done) {
@@ -241,6 +244,7 @@ __global__ void __launch_bounds__(128) route_par_kernel(const float* __restrict_
       __syncwarp();
       if (i < n) {
         perm_out[cur + rank] = i;
+        gperm_out[cur + rank] = __ldcg(&gates[i]);
         if (rank == 0) cursor[e] = cur + __popc(mask);
       }
       __syncwarp();
@@ -264,7 +268,7 @@ cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s) {
     const dim3 grid((T + 3) / 4);
 #define SCION_ROUTE_PAR(V)                                                                                 \
   return launch_pdl(route_par_kernel<V>, grid, dim3(128), smem, s, L->logits, T, L->E, L->k, L->desc.norm_topk, \
-                    L->ids, L->gates, L->counts, L->offsets, L->perm, L->active, L->n_active,                 \
+                    L->ids, L->gates, L->counts, L->offsets, L->perm, L->gperm, L->active, L->n_active,       \
                     reinterpret_cast<int4*>(L->slot_info), L->route_done)
     const int vpl = (L->E + 31) / 32;
     if (vpl <= 1) SCION_ROUTE_PAR(1);
@@ -278,7 +282,7 @@ cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s) {
   size_t smem = sizeof(float) * (size_t(kRouteThreads / 32) * L->E) + sizeof(int32_t) * (2 * size_t(L->E)) +
                 sizeof(int32_t) * size_t(T) * L->k;
   route_kernel<<<1, kRouteThreads, smem, s>>>(L->logits, T, L->E, L->k, L->desc.norm_topk, L->ids, L->gates,
-                                               L->counts, L->offsets, L->perm, L->active, L->n_active);
+                                               L->counts, L->offsets, L->perm, L->gperm, L->active, L->n_active);
   if (cudaError_t e = cudaGetLastError()) return e;
   return launch_slot_info(L, s);
 }

@@ -45,7 +45,7 @@ void free_layer(scion_layer* L) {
   void* ptrs[] = {L->gu_bank, L->dn_bank,  L->dense_down, L->xunits,  L->logits,    L->ids,       L->gates,
                   L->counts,  L->offsets,  L->perm,       L->active,  L->n_active,  L->h,         L->hz,
                   L->xfrag,   L->xpartial, L->xcount,     L->x_stage, L->out_stage, L->bad,       L->err,
-                  L->slot_info, L->route_done};
+                  L->slot_info, L->route_done, L->gperm};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   if (L->pre) {
@@ -256,6 +256,7 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   SCION_TRY(dev_alloc(L, &L->counts, sizeof(int32_t) * L->E));
   SCION_TRY(dev_alloc(L, &L->offsets, sizeof(int32_t) * (L->E + 1)));
   SCION_TRY(dev_alloc(L, &L->perm, sizeof(int32_t) * TD * L->k));
+  SCION_TRY(dev_alloc(L, &L->gperm, sizeof(float) * TD * L->k));
   SCION_TRY(dev_alloc(L, &L->active, sizeof(int32_t) * L->E));
   SCION_TRY(dev_alloc(L, &L->n_active, sizeof(int32_t)));
   SCION_TRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&L->slot_info), sizeof(int4) * L->E));

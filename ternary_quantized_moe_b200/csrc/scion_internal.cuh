@@ -98,6 +98,7 @@ struct scion_layer {
   int32_t* counts;   // [E]
   int32_t* offsets;  // [E+1]
   int32_t* perm;     // [TDEC*k]
+  float* gperm;      // [TDEC*k] gate of the entry at each routed position
   int32_t* active;   // [E]
   int32_t* n_active; // [1]
   void* slot_info;    // int4 [E]: {expert, first position, token count, 0} per active slot

@@ -193,6 +193,23 @@ def test_forward_variants(variant):
     check_output(got, ref)
 
 
+@pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
+@pytest.mark.parametrize("T,E,k", [(1, 16, 4), (5, 16, 4), (13, 16, 4), (64, 16, 4), (64, 4, 2), (37, 6, 3)])
+def test_forward_stream_kernels(fmt, T, E, k):
+    """The persistent bulk-copy ring expert kernels (selected with SCION_OPT_STREAM_MIN_TOKENS):
+    stage by stage against the oracle, including experts with more than one 8-token pass."""
+    cfg = small("st", fmt, False, E=E, k=k)
+    L, banks, ol, x = _case(cfg, T)
+    layer = device_layer(cfg, L, banks, 64)
+    tq.scion_layer_set_option(layer, tq.SCION_OPT_STREAM_MIN_TOKENS, 1)
+    got, dbg = run_forward(layer, x, T, debug=True, E=cfg.n_experts, k=cfg.top_k, F=cfg.ffn,
+                           Kdense=cfg.shared_ffn + cfg.rank)
+    _check_routing(cfg, dbg, ol, x, T)
+    _check_hidden(cfg, dbg, ol, x, T)
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
+
+
 @pytest.mark.parametrize("T", [64, 65, 150])
 def test_forward_multi_pass(T):
     """Batches above one decode pass (64 tokens) run in passes; ragged tails included."""
