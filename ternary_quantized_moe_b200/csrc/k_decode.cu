@@ -40,17 +40,71 @@ struct XProjArgs {
   unsigned* count;
   float* logits;
   __half* hz;
-  __half* xfrag;  // [T][d/128][128] fp16 in fragment order
+  __half* xfrag;  // [T][d/128][SCION_BROW] fp16 in fragment order + group sums
+  __half* h;      // [T*k][F/128][SCION_BROW] expert hidden: group-sum tails zeroed here
+  int k, GF;
   float* out;     // zeroed here
 };
 
-// One CTA = (unit, 512-column chunk); 4 warps x 128 columns.  NT = token tiles of 8.
+// One CTA = (unit, 512-column chunk); 4 warps x 128 columns.  NT = token tiles of 8.  With
+// several chunks, each CTA adds its unit's partial sums into the unit's fp32 accumulation rows
+// (red.add) and the last CTA of the unit to arrive applies the epilogue and clears the rows.
+// kXAux extra CTA columns convert x to the fragment order and clear out and the hidden tails.
 constexpr int kXRow = SCION_XPROJ_KC + 8;  // bf16 elements per staged token row (+16 B pad)
+constexpr int kXAux = 8;
+
+template <int NT>
+constexpr size_t xproj_smem(int T) {
+  return (size_t(T) * kXRow * 2 > size_t(4) * 2 * NT * 32 * 4 * 4) ? size_t(T) * kXRow * 2
+                                                                    : size_t(4) * 2 * NT * 32 * 4 * 4;
+}
+
+__device__ __forceinline__ void xproj_aux(const XProjArgs& a, int aux, int n_aux) {
+  const int Gd = a.d >> 7;
+  const int lane = threadIdx.x & 31;
+  // x -> fragment order: item = (token, group, 8-element part); the 16 parts of a group sit in
+  // 16 consecutive lanes, which sum the group's B * 4^f for the row tail.
+  const int total = a.T * Gd * 16;
+  for (int base = aux * 128 + (threadIdx.x & ~31); base < total; base += n_aux * 128) {
+    const int item = base + lane;
+    const bool ok = item < total;
+    const int grp = ok ? item >> 4 : 0, part = item & 15;
+    const int t = grp / Gd, g = grp % Gd;
+    const __nv_bfloat16* src = a.x + int64_t(t) * a.d + g * 128;
+    __align__(16) __half o[8];
+    float sum = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int idx = part * 8 + e;
+      const float v = ok ? __bfloat162float(src[brow_col(a.fmt, idx)]) : 0.f;
+      if (a.fmt == SCION_PQ2_0) {
+        const float up = 1.0f / brow_bscale(idx);
+        o[e] = __float2half_rn(v / up);
+        sum += __half2float(o[e]) * up;
+      } else {
+        o[e] = __float2half_rn(v);
+      }
+    }
+#pragma unroll
+    for (int off = 8; off; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    __half* dst = a.xfrag + int64_t(grp) * SCION_BROW;
+    if (ok) {
+      *reinterpret_cast<uint4*>(dst + part * 8) = *reinterpret_cast<const uint4*>(o);
+      if (part == 0) *reinterpret_cast<float4*>(dst + 128) = make_float4(-5.9604644775390625e-08f * sum, 0.f, 0.f, 0.f);
+    }
+  }
+  const int tid = aux * 128 + threadIdx.x, nth = n_aux * 128;
+  float4* o4 = reinterpret_cast<float4*>(a.out);
+  for (int64_t i = tid; i < int64_t(a.T) * a.d / 4; i += nth) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  // the expert hidden's group sums are accumulated by the gate/up epilogue
+  for (int i = tid; i < a.T * a.k * a.GF; i += nth)
+    *reinterpret_cast<float4*>(a.h + int64_t(i) * SCION_BROW + 128) = make_float4(0.f, 0.f, 0.f, 0.f);
+}
 
 template <int NT>
 __global__ void __launch_bounds__(128) xproj_kernel(XProjArgs a) {
-  extern __shared__ __align__(16) __nv_bfloat16 xs[];  // [NT*8][kXRow]
-  __shared__ float red[4][2][NT][32][4];
+  extern __shared__ __align__(16) uint8_t xsm[];
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(xsm);  // [NT*8][kXRow], then the warp reduction
   __shared__ int last_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, c = lane & 3;
@@ -58,21 +112,9 @@ __global__ void __launch_bounds__(128) xproj_kernel(XProjArgs a) {
   const int kbase = chunk * SCION_XPROJ_KC;
 
   pdl_trigger();
-  if (blockIdx.x == a.n_units) {
+  if (blockIdx.x >= a.n_units) {
     pdl_wait();
-    // aux column: x in fragment order (one thread per token x 128-column group), zero out.
-    const int Gd = a.d >> 7;
-    for (int item = chunk * blockDim.x + threadIdx.x; item < a.T * Gd; item += a.n_chunks * blockDim.x) {
-      const int t = item / Gd, g = item % Gd;
-      if (a.fmt == SCION_PQ2_0)
-        xfrag_group<SCION_PQ2_0>(a.x + int64_t(t) * a.d + g * 128, a.xfrag + (int64_t(t) * Gd + g) * 128);
-      else
-        xfrag_group<SCION_PTQ1_0>(a.x + int64_t(t) * a.d + g * 128, a.xfrag + (int64_t(t) * Gd + g) * 128);
-    }
-    const int64_t n4 = int64_t(a.T) * a.d / 4;
-    float4* o4 = reinterpret_cast<float4*>(a.out);
-    for (int64_t i = int64_t(chunk) * blockDim.x + threadIdx.x; i < n4; i += int64_t(a.n_chunks) * blockDim.x)
-      o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    xproj_aux(a, (blockIdx.x - a.n_units) * a.n_chunks + chunk, kXAux * a.n_chunks);
     return;
   }
 
@@ -147,7 +189,8 @@ __global__ void __launch_bounds__(128) xproj_kernel(XProjArgs a) {
       }
     }
   }
-  // reduce the 4 warps
+  __syncthreads();  // the x stage is dead: its space holds the warp reduction
+  float(*red)[2][NT][32][4] = reinterpret_cast<float(*)[2][NT][32][4]>(xsm);
 #pragma unroll
   for (int m = 0; m < 2; ++m)
 #pragma unroll
@@ -156,24 +199,24 @@ __global__ void __launch_bounds__(128) xproj_kernel(XProjArgs a) {
       for (int i = 0; i < 4; ++i) red[warp][m][nt][lane][i] = acc[m][nt][i];
   __syncthreads();
 
-  // thread -> (nt, lane) pairs; NT*32 pairs over 128 threads
-  const int npairs = NT * 32;
-  float* part = a.partial + (int64_t(blockIdx.x) * a.n_chunks) * (2 * 16 * SCION_TDEC);
-  for (int p = threadIdx.x; p < npairs; p += blockDim.x) {
-    int nt = p >> 5, ln = p & 31;
+  // thread -> (nt, lane) pairs; sum the 4 warps
+  float* accum = a.partial + int64_t(blockIdx.x) * (2 * 16 * SCION_TDEC);  // [m][row][tok]
+  for (int p = threadIdx.x; p < NT * 32; p += blockDim.x) {
+    const int nt = p >> 5, ln = p & 31;
     for (int m = 0; m < nacc; ++m)
+#pragma unroll
       for (int i = 0; i < 4; ++i) {
-        float v = red[0][m][nt][ln][i] + red[1][m][nt][ln][i] + red[2][m][nt][ln][i] + red[3][m][nt][ln][i];
-        int row = (ln >> 2) + 8 * (i >> 1), tok = nt * 8 + 2 * (ln & 3) + (i & 1);
+        const float v = red[0][m][nt][ln][i] + red[1][m][nt][ln][i] + red[2][m][nt][ln][i] + red[3][m][nt][ln][i];
+        const int row = (ln >> 2) + 8 * (i >> 1), tok = nt * 8 + 2 * (ln & 3) + (i & 1);
         red[0][m][nt][ln][i] = v;
-        if (a.n_chunks > 1) part[(int64_t(chunk) * 2 + m) * 16 * SCION_TDEC + row * SCION_TDEC + tok] = v;
+        if (a.n_chunks > 1 && tok < a.T) atomicAdd(&accum[(m * 16 + row) * SCION_TDEC + tok], v);
       }
   }
   if (a.n_chunks > 1) {
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
-      unsigned prev = atomicAdd(&a.count[blockIdx.x], 1u);
+      const unsigned prev = atomicAdd(&a.count[blockIdx.x], 1u);
       last_flag = (prev == unsigned(a.n_chunks - 1));
     }
     __syncthreads();
@@ -183,27 +226,37 @@ __global__ void __launch_bounds__(128) xproj_kernel(XProjArgs a) {
     __syncthreads();
   }
 
-  // epilogue: thread -> (row, tok)
-  const int nrows_u = 16;
-  for (int p = threadIdx.x; p < nrows_u * a.T; p += blockDim.x) {
-    int row = p / a.T, tok = p % a.T;
-    int grow = u.row0 + row;
-    if (grow >= nrows) continue;
-    float v[2] = {0.f, 0.f};
+  // epilogue: thread -> (row, tok); all loads of the thread are issued together
+  constexpr int kIt = 16 * SCION_TDEC / 128;
+  float v[kIt][2];
+#pragma unroll
+  for (int it = 0; it < kIt; ++it) {
+    const int p = threadIdx.x + 128 * it;
+    v[it][0] = v[it][1] = 0.f;
+    if (p >= 16 * a.T) continue;
+    const int row = p / a.T, tok = p % a.T;
     if (a.n_chunks > 1) {
-      for (int ch = 0; ch < a.n_chunks; ++ch)
-        for (int m = 0; m < nacc; ++m)
-          v[m] += __ldcg(&part[(int64_t(ch) * 2 + m) * 16 * SCION_TDEC + row * SCION_TDEC + tok]);
+      for (int m = 0; m < nacc; ++m) v[it][m] = __ldcg(&accum[(m * 16 + row) * SCION_TDEC + tok]);
     } else {
-      int nt = tok >> 3, ln = (row & 7) * 4 + ((tok & 7) >> 1), i = (row >> 3) * 2 + (tok & 1);
-      for (int m = 0; m < nacc; ++m) v[m] = red[0][m][nt][ln][i];
+      const int nt = tok >> 3, ln = (row & 7) * 4 + ((tok & 7) >> 1), i = (row >> 3) * 2 + (tok & 1);
+      for (int m = 0; m < nacc; ++m) v[it][m] = red[0][m][nt][ln][i];
     }
+  }
+#pragma unroll
+  for (int it = 0; it < kIt; ++it) {
+    const int p = threadIdx.x + 128 * it;
+    if (p >= 16 * a.T) continue;
+    const int row = p / a.T, tok = p % a.T;
+    const int grow = u.row0 + row;
+    if (a.n_chunks > 1)
+      for (int m = 0; m < nacc; ++m) accum[(m * 16 + row) * SCION_TDEC + tok] = 0.f;  // ready for the next call
+    if (grow >= nrows) continue;
     if (u.kind == kUnitRouter) {
-      a.logits[int64_t(tok) * a.E + grow] = v[0];
+      a.logits[int64_t(tok) * a.E + grow] = v[it][0];
     } else if (u.kind == kUnitSwiglu) {
-      a.hz[int64_t(tok) * a.Kd + grow] = __float2half_rn(silu_f(v[0]) * v[1]);
+      a.hz[int64_t(tok) * a.Kd + grow] = __float2half_rn(silu_f(v[it][0]) * v[it][1]);
     } else {
-      a.hz[int64_t(tok) * a.Kd + a.Fs + grow] = __float2half_rn(v[0]);
+      a.hz[int64_t(tok) * a.Kd + a.Fs + grow] = __float2half_rn(v[it][0]);
     }
   }
   if (a.n_chunks > 1 && threadIdx.x == 0) a.count[blockIdx.x] = 0;
@@ -258,7 +311,7 @@ __global__ void __launch_bounds__(kGuWarps * 32) gateup_kernel(GateUpArgs a) {
       const int g = warp + kGuWarps * i;
       if (g < a.Gd) {
         uint32_t b[16];
-        load_b(a.xfrag, int64_t(a.Gd) * 128, tok, g, c, b);
+        load_b(a.xfrag, int64_t(a.Gd) * SCION_BROW, tok, g, c, b);
         tile_mma<FMT>(rg[i], b, tg, c);
         tile_mma<FMT>(ru[i], b, tu, c);
       }
@@ -275,10 +328,10 @@ __global__ void __launch_bounds__(kGuWarps * 32) gateup_kernel(GateUpArgs a) {
       if (tcol < nn) {
         const int f = ft * 16 + row;
         const int64_t pos = p0 + pc + tcol;
-        const int idx = frag_index(a.fmt, f & 127);
+        const int idx = brow_pos(a.fmt, f & 127);
         float h = silu_f(gs) * us;
-        if (a.fmt == SCION_PQ2_0) h *= pq2_bscale(idx);
-        a.hfrag[(pos * GF + (f >> 7)) * 128 + idx] = __float2half_rn(h);
+        if (a.fmt == SCION_PQ2_0) h *= brow_bscale(idx);
+        a.hfrag[(pos * GF + (f >> 7)) * SCION_BROW + idx] = __float2half_rn(h);
       }
     }
     __syncthreads();
@@ -328,7 +381,7 @@ __global__ void __launch_bounds__(kDnWarps * 32) down_routed_kernel(DownArgs a) 
       const int g = warp + kDnWarps * i;
       if (g < a.GF) {
         uint32_t b[16];
-        load_b(a.hfrag, int64_t(a.GF) * 128, pos, g, c, b);
+        load_b(a.hfrag, int64_t(a.GF) * SCION_BROW, pos, g, c, b);
         tile_mma<FMT>(rw[i], b, acc, c);
       }
     }
@@ -351,7 +404,10 @@ __global__ void __launch_bounds__(kDnWarps * 32) down_routed_kernel(DownArgs a) 
 }
 
 // [sh_down | corr_b] (fp16 [d][Kd]) x hz ([T][Kd] fp16, natural order) -> out += .
-// One CTA per 16 output rows; 8 warps split K in 32-column chunks.
+// CTA = (32 output rows, 256-column K chunk): the chunk of hz is staged in shared memory, the
+// 8 warps take (16 rows, 64 columns) each with their weights loaded before the dependency
+// wait, and the 4 K slices of each row pair are summed in shared memory before one fp32
+// red.add per output.
 struct DenseArgs {
   const __half* w;  // [d][Kd]
   const __half* hz; // [T][Kd]
@@ -359,51 +415,78 @@ struct DenseArgs {
   float* out;
 };
 
+constexpr int kDnKc = 256;            // K columns per CTA
+constexpr int kDnRowH = kDnKc + 32;   // staged hz row (halves): 576 B, rows 16 banks apart
+
 template <int NT>
 __global__ void __launch_bounds__(256) down_dense_kernel(DenseArgs a) {
-  __shared__ float red[8][NT][32][4];
+  extern __shared__ __align__(16) uint8_t dsm[];
+  __half* hs = reinterpret_cast<__half*>(dsm);                                 // [NT*8][kDnRowH]
+  float* red = reinterpret_cast<float*>(dsm + NT * 8 * kDnRowH * sizeof(__half));  // [8][NT][32][4]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g8 = lane >> 2, c = lane & 3;
-  const int row0 = blockIdx.x * 16;
+  const int row0 = blockIdx.x * 32 + 16 * (warp & 1);
+  const int kc0 = blockIdx.y * kDnKc;
+  const int kw = kc0 + 64 * (warp >> 1);
   pdl_trigger();
-  {
-    const char* wbase = reinterpret_cast<const char*>(a.w + int64_t(row0) * a.Kd);
-    const int64_t bytes = int64_t(16) * a.Kd * 2;
-    for (int64_t off = int64_t(threadIdx.x) * 128; off < bytes; off += int64_t(blockDim.x) * 128)
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(wbase + off));
+  // weights first (they do not depend on earlier kernels): 64 columns of rows g8 and g8 + 8
+  uint4 wa[2], wb[2];
+  const bool kin = kw < a.Kd;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    wa[q] = kin ? ldg_stream(a.w + int64_t(row0 + g8) * a.Kd + kw + 32 * q + 8 * c) : make_uint4(0, 0, 0, 0);
+    wb[q] = kin ? ldg_stream(a.w + int64_t(row0 + g8 + 8) * a.Kd + kw + 32 * q + 8 * c) : make_uint4(0, 0, 0, 0);
   }
   pdl_wait();
+  const int kcols = min(kDnKc, a.Kd - kc0);  // multiple of 64
+  for (int i = threadIdx.x; i < a.T * (kcols >> 3); i += blockDim.x) {
+    const int t = i / (kcols >> 3), j = i % (kcols >> 3);
+    const uint32_t dst = uint32_t(__cvta_generic_to_shared(hs + t * kDnRowH + 8 * j));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(a.hz + int64_t(t) * a.Kd + kc0 + 8 * j)
+                 : "memory");
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
   float acc[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-  for (int kc = warp * 32; kc < a.Kd; kc += 8 * 32) {
-    const uint4 wa = ldg_stream(a.w + int64_t(row0 + g8) * a.Kd + kc + 8 * c);
-    const uint4 wb = ldg_stream(a.w + int64_t(row0 + g8 + 8) * a.Kd + kc + 8 * c);
-    uint32_t fa0[4] = {wa.x, wb.x, wa.y, wb.y};
-    uint32_t fa1[4] = {wa.z, wb.z, wa.w, wb.w};
+  if (kin) {
+    const int kwl = kw - kc0;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int tok = nt * 8 + g8;
-      uint4 xb = tok < a.T ? *reinterpret_cast<const uint4*>(a.hz + int64_t(tok) * a.Kd + kc + 8 * c)
-                           : make_uint4(0, 0, 0, 0);
-      mma_f16_16816(acc[nt], fa0, xb.x, xb.y);
-      mma_f16_16816(acc[nt], fa1, xb.z, xb.w);
+    for (int q = 0; q < 2; ++q) {
+      const uint32_t fa0[4] = {wa[q].x, wb[q].x, wa[q].y, wb[q].y};
+      const uint32_t fa1[4] = {wa[q].z, wb[q].z, wa[q].w, wb[q].w};
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int tok = nt * 8 + g8;
+        const uint4 xb = tok < a.T ? *reinterpret_cast<const uint4*>(hs + tok * kDnRowH + kwl + 32 * q + 8 * c)
+                                   : make_uint4(0, 0, 0, 0);
+        mma_f16_16816(acc[nt], fa0, xb.x, xb.y);
+        mma_f16_16816(acc[nt], fa1, xb.z, xb.w);
+      }
     }
   }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) red[warp][nt][lane][i] = acc[nt][i];
+    for (int i = 0; i < 4; ++i) red[((warp * NT + nt) * 32 + lane) * 4 + i] = acc[nt][i];
   __syncthreads();
-  for (int idx = threadIdx.x; idx < NT * 128; idx += blockDim.x) {
-    const int nt = idx >> 7, ln = (idx >> 2) & 31, i = idx & 3;
+  // thread -> (row half h, nt, lane, i): sum the 4 K slices (warps h, h+2, h+4, h+6)
+  for (int idx = threadIdx.x; idx < 2 * NT * 128; idx += blockDim.x) {
+    const int h = idx / (NT * 128), rem = idx % (NT * 128);
+    const int nt = rem >> 7, ln = (rem >> 2) & 31, i = rem & 3;
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) v += red[w][nt][ln][i];
-    const int row = (ln >> 2) + 8 * (i >> 1), tok = nt * 8 + 2 * (ln & 3) + (i & 1);
-    if (tok < a.T) atomicAdd(&a.out[int64_t(tok) * a.d + row0 + row], v);
+    for (int ks = 0; ks < 4; ++ks) v += red[(((h + 2 * ks) * NT + nt) * 32 + ln) * 4 + i];
+    const int row = blockIdx.x * 32 + 16 * h + (ln >> 2) + 8 * (i >> 1), tok = nt * 8 + 2 * (ln & 3) + (i & 1);
+    if (tok < a.T) atomicAdd(&a.out[int64_t(tok) * a.d + row], v);
   }
+}
+
+template <int NT>
+constexpr size_t down_dense_smem() {
+  return size_t(NT) * 8 * kDnRowH * sizeof(__half) + size_t(8) * NT * 32 * 4 * sizeof(float);
 }
 
 __global__ void unfrag_kernel(int fmt, const __half* __restrict__ src, int64_t n, __half* __restrict__ dst) {
@@ -411,9 +494,9 @@ __global__ void unfrag_kernel(int fmt, const __half* __restrict__ src, int64_t n
   if (i >= n) return;
   int64_t grp = i >> 7;
   int col = int(i & 127);
-  const int idx = frag_index(fmt, col);
-  float v = __half2float(src[grp * 128 + idx]);
-  if (fmt == SCION_PQ2_0) v /= pq2_bscale(idx);  // undo the exact power-of-two B pre-scaling
+  const int idx = brow_pos(fmt, col);
+  float v = __half2float(src[grp * SCION_BROW + idx]);
+  if (fmt == SCION_PQ2_0) v /= brow_bscale(idx);  // undo the exact power-of-two B pre-scaling
   dst[grp * 128 + col] = __float2half_rn(v);
 }
 
@@ -431,14 +514,14 @@ cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, fl
   a.corr_a = static_cast<const __nv_bfloat16*>(L->desc.corr_a);
   a.units = L->xunits, a.n_units = L->n_xunits, a.n_chunks = L->n_xchunks;
   a.partial = L->xpartial, a.count = L->xcount, a.logits = L->logits, a.hz = L->hz, a.xfrag = L->xfrag, a.out = out;
-  dim3 grid(L->n_xunits + 1, L->n_xchunks);
+  a.h = L->h, a.k = L->k, a.GF = L->GF;
+  dim3 grid(L->n_xunits + kXAux, L->n_xchunks);
   const int nt = (T + 7) / 8;
-  const size_t smem = sizeof(__nv_bfloat16) * size_t(T) * kXRow;
   switch (nt) {
-    case 1: return launch_pdl(xproj_kernel<1>, grid, dim3(128), smem, s, a);
-    case 2: return launch_pdl(xproj_kernel<2>, grid, dim3(128), smem, s, a);
-    case 3: case 4: return launch_pdl(xproj_kernel<4>, grid, dim3(128), smem, s, a);
-    default: return launch_pdl(xproj_kernel<8>, grid, dim3(128), smem, s, a);
+    case 1: return launch_pdl(xproj_kernel<1>, grid, dim3(128), xproj_smem<1>(T), s, a);
+    case 2: return launch_pdl(xproj_kernel<2>, grid, dim3(128), xproj_smem<2>(T), s, a);
+    case 3: case 4: return launch_pdl(xproj_kernel<4>, grid, dim3(128), xproj_smem<4>(T), s, a);
+    default: return launch_pdl(xproj_kernel<8>, grid, dim3(128), xproj_smem<8>(T), s, a);
   }
   return cudaGetLastError();
 }
@@ -494,12 +577,12 @@ cudaError_t launch_down_dense(const scion_layer* L, int T, float* out, cudaStrea
   DenseArgs b;
   b.w = L->dense_down, b.hz = L->hz, b.d = L->d, b.Kd = L->Kd, b.T = T, b.out = out;
   const int nt = (T + 7) / 8;
-  dim3 g2(L->d / 16);
+  const dim3 g2(L->d / 32, (L->Kd + kDnKc - 1) / kDnKc);
   switch (nt) {
-    case 1: return launch_pdl(down_dense_kernel<1>, g2, dim3(256), 0, s, b);
-    case 2: return launch_pdl(down_dense_kernel<2>, g2, dim3(256), 0, s, b);
-    case 3: case 4: return launch_pdl(down_dense_kernel<4>, g2, dim3(256), 0, s, b);
-    default: return launch_pdl(down_dense_kernel<8>, g2, dim3(256), 0, s, b);
+    case 1: return launch_pdl(down_dense_kernel<1>, g2, dim3(256), down_dense_smem<1>(), s, b);
+    case 2: return launch_pdl(down_dense_kernel<2>, g2, dim3(256), down_dense_smem<2>(), s, b);
+    case 3: case 4: return launch_pdl(down_dense_kernel<4>, g2, dim3(256), down_dense_smem<4>(), s, b);
+    default: return launch_pdl(down_dense_kernel<8>, g2, dim3(256), down_dense_smem<8>(), s, b);
   }
   return cudaGetLastError();
 }
@@ -512,12 +595,24 @@ cudaError_t launch_unfrag(int fmt, const __half* src, int rows, int G, __half* d
 }
 
 cudaError_t configure_kernels() {
-  const int xs_max = int(sizeof(__nv_bfloat16)) * SCION_TDEC * kXRow;
+  const int xs_max = int(xproj_smem<8>(SCION_TDEC));
   cudaError_t e;
   if ((e = cudaFuncSetAttribute(xproj_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, xs_max))) return e;
   if ((e = cudaFuncSetAttribute(xproj_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, xs_max))) return e;
   if ((e = cudaFuncSetAttribute(xproj_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, xs_max))) return e;
   if ((e = cudaFuncSetAttribute(xproj_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, xs_max))) return e;
+  if ((e = cudaFuncSetAttribute(down_dense_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(down_dense_smem<1>()))))
+    return e;
+  if ((e = cudaFuncSetAttribute(down_dense_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(down_dense_smem<2>()))))
+    return e;
+  if ((e = cudaFuncSetAttribute(down_dense_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(down_dense_smem<4>()))))
+    return e;
+  if ((e = cudaFuncSetAttribute(down_dense_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(down_dense_smem<8>()))))
+    return e;
   if ((e = configure_route_kernels())) return e;
   if ((e = configure_stream_kernels())) return e;
   return configure_prefill_kernels();

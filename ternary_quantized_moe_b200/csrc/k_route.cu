@@ -174,84 +174,88 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
   }
 }
 
-// ---------------------------------------------------------------- decode route v2
-// One warp per token (VPL logits per lane held in registers), then the last CTA to finish
-// groups all T*k entries: histogram, scan, active list, per-slot records and the stable
-// scatter.  Grid: ceil(T / 4) CTAs of 4 warps.
+// ---------------------------------------------------------------- decode route
+// One pass of T <= SCION_TDEC tokens (E <= 512): one warp per token selects the top k and the
+// gates (ceil(T/4) CTAs of 4 warps), then the last CTA to finish stages the T*k (id, gate)
+// entries in shared memory with one sweep and groups them there: histogram, exclusive scan,
+// active-expert list with the per-slot records, and the stable scatter in (token, slot) order.
+constexpr int kRcThreads = 128;
+
 template <int VPL>
-__global__ void __launch_bounds__(128) route_par_kernel(const float* __restrict__ logits, int T, int E, int k,
-                                                        int norm_topk, int32_t* __restrict__ ids,
-                                                        float* __restrict__ gates, int32_t* __restrict__ counts_out,
-                                                        int32_t* __restrict__ offsets_out,
-                                                        int32_t* __restrict__ perm_out,
-                                                        float* __restrict__ gperm_out,
-                                                        int32_t* __restrict__ active_out,
-                                                        int32_t* __restrict__ n_active_out,
-                                                        int4* __restrict__ slot_info, unsigned* __restrict__ done) {
-  extern __shared__ int32_t rsm[];  // counts[E] | cursor[E]
+__global__ void __launch_bounds__(kRcThreads) route_cta_kernel(
+    const float* __restrict__ logits, int T, int E, int k, int norm_topk, int32_t* __restrict__ ids,
+    float* __restrict__ gates, int32_t* __restrict__ counts_out, int32_t* __restrict__ offsets_out,
+    int32_t* __restrict__ perm_out, float* __restrict__ gperm_out, int32_t* __restrict__ active_out,
+    int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info, unsigned* __restrict__ done) {
+  extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [E] | cursor [E]
   __shared__ int last;
+  const int n = T * k;
+  int32_t* ids_s = reinterpret_cast<int32_t*>(rs);
+  float* gates_s = rs + n;
+  int32_t* counts = reinterpret_cast<int32_t*>(rs + 2 * n);
+  int32_t* cursor = counts + E;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 4 + warp;
+  const int t = blockIdx.x * (kRcThreads / 32) + warp;
   pdl_trigger();
   pdl_wait();
   if (t < T) warp_topk<VPL>(logits + int64_t(t) * E, E, k, norm_topk, lane, ids + t * k, gates + t * k);
-  // ---- the last CTA groups everything
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) last = (atomicAdd(done, 1u) == gridDim.x - 1);
   __syncthreads();
   if (!last) return;
   __threadfence();
-  int32_t* counts = rsm;
-  int32_t* cursor = rsm + E;
-  const int n = T * k;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) counts[e] = 0;
+  for (int e = threadIdx.x; e < E; e += kRcThreads) counts[e] = 0;
+  for (int i = threadIdx.x; i < n; i += kRcThreads) ids_s[i] = __ldcg(&ids[i]), gates_s[i] = __ldcg(&gates[i]);
   __syncthreads();
-  for (int i = threadIdx.x; i < n; i += blockDim.x) atomicAdd(&counts[__ldcg(&ids[i])], 1);
+  for (int i = threadIdx.x; i < n; i += kRcThreads) atomicAdd(&counts[ids_s[i]], 1);
   __syncthreads();
-  if (warp == 0) {
-    const int per = (E + 31) / 32;
-    const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
-    int sc = 0, ac = 0;
-    for (int e = e0; e < e1; ++e) sc += counts[e], ac += counts[e] > 0;
-    int si = sc, ai = ac;
-    for (int o = 1; o < 32; o <<= 1) {
-      const int s2 = __shfl_up_sync(0xffffffffu, si, o), a2 = __shfl_up_sync(0xffffffffu, ai, o);
-      if (lane >= o) si += s2, ai += a2;
-    }
-    int run = si - sc, arun = ai - ac;
-    for (int e = e0; e < e1; ++e) {
-      const int c = counts[e];
-      offsets_out[e] = run;
-      cursor[e] = run;
-      counts_out[e] = c;
-      if (c > 0) {
-        active_out[arun] = e;
-        slot_info[arun] = make_int4(e, run, c, 0);
-        ++arun;
-      }
-      run += c;
-    }
-    if (lane == 31) offsets_out[E] = si, *n_active_out = ai;
-    __syncwarp();
-    const unsigned lt = (1u << lane) - 1u;
-    for (int base = 0; base < n; base += 32) {
-      const int i = base + lane;
-      const int e = i < n ? __ldcg(&ids[i]) : -1 - lane;
-      const unsigned mask = __match_any_sync(0xffffffffu, e);
-      const int rank = __popc(mask & lt);
-      const int cur = i < n ? cursor[e] : 0;
-      __syncwarp();
-      if (i < n) {
-        perm_out[cur + rank] = i;
-        gperm_out[cur + rank] = __ldcg(&gates[i]);
-        if (rank == 0) cursor[e] = cur + __popc(mask);
-      }
-      __syncwarp();
-    }
+  if (warp != 0) return;
+  if (lane == 0) *done = 0;
+  // ---- exclusive scan of the counts, active list and slot records (warp 0)
+  const int per = (E + 31) / 32;
+  const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+  int sc = 0, ac = 0;
+  for (int e = e0; e < e1; ++e) sc += counts[e], ac += counts[e] > 0;
+  int si = sc, ai = ac;
+  for (int o = 1; o < 32; o <<= 1) {
+    const int s2 = __shfl_up_sync(0xffffffffu, si, o), a2 = __shfl_up_sync(0xffffffffu, ai, o);
+    if (lane >= o) si += s2, ai += a2;
   }
-  if (threadIdx.x == 0) *done = 0;
+  int run = si - sc, arun = ai - ac;
+  for (int e = e0; e < e1; ++e) {
+    const int c = counts[e];
+    offsets_out[e] = run;
+    cursor[e] = run;
+    counts_out[e] = c;
+    if (c > 0) {
+      active_out[arun] = e;
+      slot_info[arun] = make_int4(e, run, c, 0);
+      ++arun;
+    }
+    run += c;
+  }
+  if (lane == 31) offsets_out[E] = si, *n_active_out = ai;
+  __syncwarp();
+  // ---- stable scatter in (token, slot) order, 32 entries at a time
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const int e = i < n ? ids_s[i] : -1 - lane;  // unique dummies never match real ids
+    const unsigned mask = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(mask & lt);
+    const int cur = i < n ? cursor[e] : 0;
+    __syncwarp();
+    if (i < n) {
+      perm_out[cur + rank] = i;
+      gperm_out[cur + rank] = gates_s[i];
+      if (rank == 0) cursor[e] = cur + __popc(mask);
+    }
+    __syncwarp();
+  }
 }
+
+size_t route_cta_smem(int T, int E, int k) { return sizeof(float) * (2 * size_t(T) * k + 2 * size_t(E)); }
 
 }  // namespace
 
@@ -264,19 +268,18 @@ cudaError_t launch_router_f32(const scion_layer* L, const __nv_bfloat16* x, int 
 
 cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s) {
   if (L->E <= 512) {
-    const size_t smem = sizeof(int32_t) * 2 * size_t(L->E);
-    const dim3 grid((T + 3) / 4);
-#define SCION_ROUTE_PAR(V)                                                                                 \
-  return launch_pdl(route_par_kernel<V>, grid, dim3(128), smem, s, L->logits, T, L->E, L->k, L->desc.norm_topk, \
-                    L->ids, L->gates, L->counts, L->offsets, L->perm, L->gperm, L->active, L->n_active,       \
-                    reinterpret_cast<int4*>(L->slot_info), L->route_done)
+    const size_t smem = route_cta_smem(T, L->E, L->k);
+#define SCION_ROUTE_CTA(V)                                                                                     \
+  return launch_pdl(route_cta_kernel<V>, dim3((T + 3) / 4), dim3(kRcThreads), smem, s, L->logits, T, L->E,   \
+                    L->k, L->desc.norm_topk, L->ids, L->gates, L->counts, L->offsets, L->perm, L->gperm,       \
+                    L->active, L->n_active, reinterpret_cast<int4*>(L->slot_info), L->route_done)
     const int vpl = (L->E + 31) / 32;
-    if (vpl <= 1) SCION_ROUTE_PAR(1);
-    else if (vpl <= 2) SCION_ROUTE_PAR(2);
-    else if (vpl <= 4) SCION_ROUTE_PAR(4);
-    else if (vpl <= 8) SCION_ROUTE_PAR(8);
-    else SCION_ROUTE_PAR(16);
-#undef SCION_ROUTE_PAR
+    if (vpl <= 1) SCION_ROUTE_CTA(1);
+    else if (vpl <= 2) SCION_ROUTE_CTA(2);
+    else if (vpl <= 4) SCION_ROUTE_CTA(4);
+    else if (vpl <= 8) SCION_ROUTE_CTA(8);
+    else SCION_ROUTE_CTA(16);
+#undef SCION_ROUTE_CTA
     return cudaGetLastError();
   }
   size_t smem = sizeof(float) * (size_t(kRouteThreads / 32) * L->E) + sizeof(int32_t) * (2 * size_t(L->E)) +
@@ -304,6 +307,13 @@ cudaError_t launch_slot_info(const scion_layer* L, cudaStream_t s) {
 }
 
 cudaError_t configure_route_kernels() {
+  cudaError_t e;
+  const int cta_max = int(route_cta_smem(SCION_TDEC, 512, 32));
+  if ((e = cudaFuncSetAttribute(route_cta_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, cta_max))) return e;
+  if ((e = cudaFuncSetAttribute(route_cta_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, cta_max))) return e;
+  if ((e = cudaFuncSetAttribute(route_cta_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, cta_max))) return e;
+  if ((e = cudaFuncSetAttribute(route_cta_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, cta_max))) return e;
+  if ((e = cudaFuncSetAttribute(route_cta_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, cta_max))) return e;
   return cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
 }
 

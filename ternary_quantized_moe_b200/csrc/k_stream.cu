@@ -7,11 +7,12 @@
 //
 // Work item = one active expert x 128 weight rows; a persistent CTA walks many.  In the
 // re-tiled bank the 128 x 128 codes of one group (gate and up interleaved for the gate/up
-// bank) are one contiguous block, so a producer warp streams group after group with
-// cp.async.bulk into an mbarrier ring, together with the 256-byte fragment-ordered rows of the
-// slot's tokens.  Eight consumer warps each own a 16-row sub-tile over the whole K range:
-// codes come from shared memory, are unpacked in registers into mma.sync fragments, and no
-// cross-warp reduction is needed.
+// bank) are one contiguous block and consecutive groups follow each other, so a producer
+// warp streams GPS groups per stage with one cp.async.bulk into an mbarrier ring, together
+// with the fragment-ordered B rows (x or h, plus their group-sum tails) of the item's tokens.
+// Eight consumer warps each own a 16-row sub-tile over the whole K range: codes come from
+// shared memory, are unpacked in registers into mma.sync fragments (PQ2_0 as fp16
+// subnormals, PTQ1_0 through the base-3 digit chain), and no cross-warp reduction is needed.
 #include "tc_common.cuh"
 #include "tern_tile.cuh"
 
@@ -20,19 +21,20 @@ namespace {
 
 using namespace tc;
 
-constexpr int kRing = 8;    // stages in flight
+constexpr int kRing = 4;    // stages in flight
 constexpr int kCons = 8;    // consumer warps (one 16-row sub-tile each)
 constexpr int kTok = 8;     // tokens per pass (one mma n-tile)
-constexpr int kRowB = 256;  // bytes of one token's 128-column group (fp16)
+constexpr int kRowB = SCION_BROW * 2;  // bytes of one token's 128-column group row (fp16 + sum tail)
 constexpr int kHdr = 256;   // stage header
+constexpr float kTwoP24 = 16777216.0f;  // 2^24
 
 // Written by the producer into every stage; the consumers are driven by it alone.
 struct StageHdr {
   int nn;     // tokens of the pass (1..kTok); -1: no more work for this CTA
-  int flags;  // bit 0: first group of the pass, bit 1: last group of the pass
+  int flags;  // bit 0: first stage of the pass, bit 1: last stage of the pass
   int rb;     // 128-row block of the item
-  int pad;
-  int pos[kTok];     // routed positions of the pass's tokens (last group only)
+  int ng;     // 128-column groups in this stage (1..GPS)
+  int pos[kTok];     // routed positions of the pass's tokens (last stage only)
   int orow[kTok];    // output token row (entry / k)
   float gate[kTok];  // gate of the entry
 };
@@ -40,7 +42,7 @@ static_assert(sizeof(StageHdr) <= kHdr, "stage header");
 
 struct StreamArgs {
   const uint8_t* bank;
-  const __half* bsrc;  // gate/up: xfrag [T][Gd][128]; down: hfrag [T*k][GF][128]
+  const __half* bsrc;  // gate/up: xfrag [T][Gd][SCION_BROW]; down: h [T*k][GF][SCION_BROW]
   int bld;             // 128-column groups per B row (Gd or GF)
   const int4* slot_info;
   const int32_t *n_active, *perm;
@@ -56,8 +58,120 @@ struct TokInfo {
   float gate;
 };
 
+// Groups per stage: two for the gate/up bank (each group holds both matrices), four for down.
+template <int NMAT>
+constexpr int gps() {
+  return NMAT == 2 ? 2 : 4;
+}
+template <int FMT, int NMAT>
+constexpr uint32_t code_bytes() {
+  return NMAT * 8 * (FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile);
+}
+// B rows in a stage: token n at n * tok_stride + 16 * (n / 2).  The stride is 64 (mod 128)
+// bytes, so tokens n and n + 1 fall on opposite halves of the shared-memory banks (a 16-byte
+// load of lanes (n, 0..3) and (n + 1, 0..3) is conflict-free), and the 16-byte skew spreads the
+// group-sum tails of tokens 0, 2, 4, 6 over different banks.
+template <int NMAT>
+constexpr uint32_t tok_stride() {
+  return (gps<NMAT>() * kRowB + 63) / 128 * 128 + 64;
+}
+__device__ __forceinline__ uint32_t tok_off(uint32_t stride, int n) { return n * stride + 16 * (n >> 1); }
+template <int FMT, int NMAT>
+constexpr uint32_t stage_bytes() {
+  return kHdr + gps<NMAT>() * code_bytes<FMT, NMAT>() + kTok * tok_stride<NMAT>() + 64;
+}
+
+// mma.sync m16n8k16 (fp16 in, fp32 accumulate) without `volatile`, so that independent
+// accumulation chains of several tiles can be interleaved by the compiler.
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// One stage's groups [j0, j0 + J) for this warp: J x NMAT independent PQ2_0 tiles (subnormal
+// unpack, accumulators started at the group-sum tails) or PTQ1_0 tiles (digit chain).
+template <int FMT, int NMAT, int J>
+__device__ __forceinline__ void stage_groups(const uint8_t* stg, int j0, int nn, int warp, int lane,
+                                             float (&acc)[NMAT][4]) {
+  constexpr int G = gps<NMAT>();
+  constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
+  constexpr uint32_t cb = code_bytes<FMT, NMAT>();
+  constexpr uint32_t ts = tok_stride<NMAT>();
+  const int c = lane & 3, n = lane >> 2;
+  const uint8_t* codes = stg + kHdr;
+  const uint8_t* brows = stg + kHdr + G * cb;
+  uint32_t b[J][16];
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    // only the pass's tokens are read (the columns of the others are dropped by the epilogue)
+    const uint8_t* bp = brows + tok_off(ts, n) + (j0 + j) * kRowB + 16 * c;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint4 v = n < nn ? *reinterpret_cast<const uint4*>(bp + 64 * i) : make_uint4(0, 0, 0, 0);
+      b[j][4 * i] = v.x, b[j][4 * i + 1] = v.y, b[j][4 * i + 2] = v.z, b[j][4 * i + 3] = v.w;
+    }
+  }
+  if constexpr (FMT == SCION_PQ2_0) {
+    uint4 w[J][NMAT];
+    uint32_t sc[J][NMAT];
+    float g[J][NMAT][4];
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      // -2^-24 * group sums of the lane's token columns 2c, 2c+1
+      const float xn0 = 2 * c < nn ? *reinterpret_cast<const float*>(brows + tok_off(ts, 2 * c) + (j0 + j) * kRowB + 256) : 0.f;
+      const float xn1 =
+          2 * c + 1 < nn ? *reinterpret_cast<const float*>(brows + tok_off(ts, 2 * c + 1) + (j0 + j) * kRowB + 256) : 0.f;
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m) {
+        const uint8_t* blk = codes + (j0 + j) * cb + (m * 8 + warp) * tb;
+        w[j][m] = *reinterpret_cast<const uint4*>(blk + 16 * lane);
+        sc[j][m] = *reinterpret_cast<const uint32_t*>(blk + 512 + 4 * (lane >> 2));
+        g[j][m][0] = xn0, g[j][m][1] = xn1, g[j][m][2] = xn0, g[j][m][3] = xn1;
+      }
+    }
+    uint32_t w10[J][NMAT][4];
+#pragma unroll
+    for (int j = 0; j < J; ++j)
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m)
+        w10[j][m][0] = w[j][m].x >> 10, w10[j][m][1] = w[j][m].y >> 10, w10[j][m][2] = w[j][m].z >> 10,
+        w10[j][m][3] = w[j][m].w >> 10;
+#define SCION_SUB_STEP(S)                                                                              \
+  _Pragma("unroll") for (int j = 0; j < J; ++j) _Pragma("unroll") for (int m = 0; m < NMAT; ++m) {     \
+    const uint32_t fa[4] = {pq2_pair_sub<S>(w[j][m].x, w10[j][m][0]), pq2_pair_sub<S>(w[j][m].z, w10[j][m][2]), \
+                            pq2_pair_sub<S>(w[j][m].y, w10[j][m][1]), pq2_pair_sub<S>(w[j][m].w, w10[j][m][3])}; \
+    mma_f16(g[j][m], fa, b[j][2 * S], b[j][2 * S + 1]);                                                \
+  }
+    SCION_SUB_STEP(0) SCION_SUB_STEP(1) SCION_SUB_STEP(2) SCION_SUB_STEP(3)
+    SCION_SUB_STEP(4) SCION_SUB_STEP(5) SCION_SUB_STEP(6) SCION_SUB_STEP(7)
+#undef SCION_SUB_STEP
+#pragma unroll
+    for (int j = 0; j < J; ++j)
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m) {
+        const float s_lo = __half2float(__ushort_as_half(uint16_t(sc[j][m] & 0xffff)));
+        const float s_hi = __half2float(__ushort_as_half(uint16_t(sc[j][m] >> 16)));
+        acc[m][0] = fmaf(s_lo, g[j][m][0], acc[m][0]);
+        acc[m][1] = fmaf(s_lo, g[j][m][1], acc[m][1]);
+        acc[m][2] = fmaf(s_hi, g[j][m][2], acc[m][2]);
+        acc[m][3] = fmaf(s_hi, g[j][m][3], acc[m][3]);
+      }
+  } else {
+#pragma unroll
+    for (int j = 0; j < J; ++j)
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m) {
+        TileRegs<FMT> t;
+        t.load_shared(smem_u32(codes + (j0 + j) * cb + (m * 8 + warp) * tb), lane);
+        tile_mma<FMT>(t, b[j], acc[m], c);
+      }
+  }
+}
+
 // Persistent: CTA b walks the items b, b + gridDim.x, ... with item = (active slot, 128-row
-// block).  One producer warp streams, per 128-column group, the item's codes and the
+// block).  One producer warp streams, per stage, GPS groups of the item's codes and the
 // fragment-ordered B rows of up to kTok tokens into a ring of stages, each with a header that
 // tells the consumers what it holds; routing records are fetched one (tokens) and two (slot)
 // items ahead, so no pointer chase sits between two items.
@@ -66,9 +180,9 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ uint64_t full[kRing], empty[kRing];
   __shared__ int abort_flag;
-  constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
-  constexpr uint32_t code_bytes = NMAT * 8 * tb;
-  constexpr uint32_t stage_bytes = kHdr + code_bytes + kTok * kRowB;
+  constexpr int GPS = gps<NMAT>();
+  constexpr uint32_t cb = code_bytes<FMT, NMAT>();
+  constexpr uint32_t sb = stage_bytes<FMT, NMAT>();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int RB = a.R >> 7;
 
@@ -103,18 +217,20 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
       const int4 si_n2 = slot_rec(item + 2 * gridDim.x);
       const TokInfo tk_nxt = tok_info(si_nxt, 0);
       const int rb = item % RB;
-      const uint8_t* src0 = a.bank + (int64_t(si_cur.x) * RB + rb) * a.G * code_bytes;
+      const uint8_t* src0 = a.bank + (int64_t(si_cur.x) * RB + rb) * a.G * cb;
       for (int pc = 0; pc < si_cur.z && ok; pc += kTok) {
         const TokInfo tk = pc == 0 ? tk_cur : tok_info(si_cur, pc);
         const int nn = min(kTok, si_cur.z - pc);
-        for (int g = 0; g < a.G; ++g, ++st) {
+        for (int g0 = 0; g0 < a.G; g0 += GPS, ++st) {
+          const int ng = min(GPS, a.G - g0);
           const int s = st % kRing;
           if (lane == 0 && st >= kRing) ok = mbar_wait(&empty[s], ((st / kRing) - 1) & 1, &abort_flag, a.err);
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
-          uint8_t* stg = ring + s * stage_bytes;
+          uint8_t* stg = ring + s * sb;
           StageHdr* hd = reinterpret_cast<StageHdr*>(stg);
-          if (g == a.G - 1) {
+          const bool last = g0 + GPS >= a.G;
+          if (last) {
             // the epilogue's per-token records, written by lane 0 so its arrive publishes them
 #pragma unroll
             for (int i = 0; i < kTok; ++i) {
@@ -125,15 +241,16 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
           }
           if (lane == 0) {
             hd->nn = nn;
-            hd->flags = (g == 0 ? 1 : 0) | (g == a.G - 1 ? 2 : 0);
+            hd->flags = (g0 == 0 ? 1 : 0) | (last ? 2 : 0);
             hd->rb = rb;
-            mbar_arrive_expect_tx(&full[s], code_bytes + nn * kRowB);
+            hd->ng = ng;
+            mbar_arrive_expect_tx(&full[s], ng * cb + nn * ng * kRowB);
           }
           __syncwarp();
-          if (lane == 0) bulk_load(stg + kHdr, src0 + int64_t(g) * code_bytes, code_bytes, &full[s]);
+          if (lane == 0) bulk_load(stg + kHdr, src0 + int64_t(g0) * cb, ng * cb, &full[s]);
           if (lane < nn)
-            bulk_load(stg + kHdr + code_bytes + lane * kRowB, a.bsrc + (int64_t(tk.brow) * a.bld + g) * 128, kRowB,
-                      &full[s]);
+            bulk_load(stg + kHdr + GPS * cb + tok_off(tok_stride<NMAT>(), lane),
+                      a.bsrc + (int64_t(tk.brow) * a.bld + g0) * SCION_BROW, ng * kRowB, &full[s]);
         }
       }
       si_cur = si_nxt, si_nxt = si_n2, tk_cur = tk_nxt;
@@ -143,7 +260,7 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
         // end-of-work sentinel (the consumers wait for every earlier stage before reaching it)
         const int s = st % kRing;
         if (st < kRing || mbar_wait(&empty[s], ((st / kRing) - 1) & 1, &abort_flag, a.err)) {
-          reinterpret_cast<StageHdr*>(ring + s * stage_bytes)->nn = -1;
+          reinterpret_cast<StageHdr*>(ring + s * sb)->nn = -1;
           mbar_arrive(&full[s]);
         }
       } else {
@@ -156,58 +273,65 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
   }
 
   // ---------------- consumers: warp w owns rows 16w .. 16w+15 of every item
-  const int c = lane & 3, n = lane >> 2;
-  const uint32_t ring_u32 = smem_u32(ring);
+  const int c = lane & 3;
   float acc[NMAT][4];
   for (int st = 0;; ++st) {
     const int s = st % kRing;
     if (!mbar_wait(&full[s], (st / kRing) & 1, &abort_flag, a.err)) break;
-    const StageHdr* hd = reinterpret_cast<const StageHdr*>(ring + s * stage_bytes);
+    const uint8_t* stg = ring + s * sb;
+    const StageHdr* hd = reinterpret_cast<const StageHdr*>(stg);
     const int nn = hd->nn;
     if (nn < 0) break;
-    const int flags = hd->flags;
+    const int flags = hd->flags, ng = hd->ng;
     if (flags & 1) {
 #pragma unroll
       for (int m = 0; m < NMAT; ++m)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
     }
-    const uint32_t stg = ring_u32 + s * stage_bytes;
-    TileRegs<FMT> tr[NMAT];
 #pragma unroll
-    for (int m = 0; m < NMAT; ++m) tr[m].load_shared(stg + kHdr + m * 8 * tb + warp * tb, lane);
-    {
-      uint32_t b[16];
-      if (n < nn) {
-        const uint32_t bp = stg + kHdr + code_bytes + n * kRowB + 64 * c;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                       : "=r"(b[4 * i]), "=r"(b[4 * i + 1]), "=r"(b[4 * i + 2]), "=r"(b[4 * i + 3])
-                       : "r"(bp + 16 * i));
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) b[i] = 0u;
-      }
-#pragma unroll
-      for (int m = 0; m < NMAT; ++m) tile_mma<FMT>(tr[m], b, acc[m], c);
+    for (int j0 = 0; j0 < GPS; j0 += 2) {
+      if (j0 + 1 < ng)
+        stage_groups<FMT, NMAT, 2>(stg, j0, nn, warp, lane, acc);
+      else if (j0 < ng)
+        stage_groups<FMT, NMAT, 1>(stg, j0, nn, warp, lane, acc);
     }
     if (flags & 2) {
       // epilogue: this warp's 16 rows x the pass's tokens
       const int rb = hd->rb;
+      constexpr float unit = FMT == SCION_PQ2_0 ? kTwoP24 : 1.0f;  // undo the subnormal 2^-24
+      float hs[2] = {0.f, 0.f};  // PQ2_0: this lane's share of the hidden group sums (tokens 2c, 2c+1)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int row = warp * 16 + (lane >> 2) + 8 * (i >> 1);
         const int tcol = 2 * c + (i & 1);
-        if (tcol >= nn) continue;
         if constexpr (NMAT == 2) {
           const int f = rb * 128 + row;
-          const int idx = frag_index(FMT, f & 127);
-          float h = silu_f(acc[0][i]) * acc[1][i];
-          if (FMT == SCION_PQ2_0) h *= pq2_bscale(idx);
-          a.hfrag[(int64_t(hd->pos[tcol]) * (a.F >> 7) + (f >> 7)) * 128 + idx] = __float2half_rn(h);
+          const int idx = brow_pos(FMT, f & 127);
+          float h = silu_f(acc[0][i] * unit) * (acc[1][i] * unit);
+          if (FMT == SCION_PQ2_0) h *= brow_bscale(idx);
+          const __half h16 = __float2half_rn(h);
+          if (tcol < nn) a.hfrag[(int64_t(hd->pos[tcol]) * (a.F >> 7) + (f >> 7)) * SCION_BROW + idx] = h16;
+          if (FMT == SCION_PQ2_0) hs[i & 1] += __half2float(h16) / brow_bscale(idx);
         } else {
-          atomicAdd(&a.out[int64_t(hd->orow[tcol]) * a.d + rb * 128 + row], hd->gate[tcol] * acc[0][i]);
+          if (tcol < nn)
+            atomicAdd(&a.out[int64_t(hd->orow[tcol]) * a.d + rb * 128 + row], hd->gate[tcol] * (acc[0][i] * unit));
+        }
+      }
+      if constexpr (NMAT == 2 && FMT == SCION_PQ2_0) {
+        // sum over the warp's 16 rows, then add -2^-24 x that into the hidden rows' group-sum tails
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          hs[0] += __shfl_xor_sync(0xffffffffu, hs[0], o);
+          hs[1] += __shfl_xor_sync(0xffffffffu, hs[1], o);
+        }
+        if (lane < 4) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            if (2 * c + j < nn)
+              atomicAdd(reinterpret_cast<float*>(a.hfrag + (int64_t(hd->pos[2 * c + j]) * (a.F >> 7) + rb) *
+                                                               SCION_BROW + 128),
+                        -hs[j] * (1.0f / kTwoP24));
         }
       }
     }
@@ -218,8 +342,7 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
 
 template <int FMT, int NMAT>
 constexpr size_t stream_smem() {
-  constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
-  return size_t(kRing) * (kHdr + NMAT * 8 * tb + kTok * kRowB);
+  return size_t(kRing) * stage_bytes<FMT, NMAT>();
 }
 
 template <int FMT, int NMAT>
@@ -249,21 +372,20 @@ cudaError_t launch_stream(const StreamArgs& a, int max_items, cudaStream_t s) {
   return launch_pdl(stream_kernel<FMT, NMAT>, dim3(grid), dim3((kCons + 1) * 32), stream_smem<FMT, NMAT>(), s, a);
 }
 
+template <int FMT, int NMAT>
+cudaError_t set_smem() {
+  return cudaFuncSetAttribute(stream_kernel<FMT, NMAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              int(stream_smem<FMT, NMAT>()));
+}
+
 }  // namespace
 
 cudaError_t configure_stream_kernels() {
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(stream_kernel<SCION_PQ2_0, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                int(stream_smem<SCION_PQ2_0, 2>()))))
-    return e;
-  if ((e = cudaFuncSetAttribute(stream_kernel<SCION_PQ2_0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                int(stream_smem<SCION_PQ2_0, 1>()))))
-    return e;
-  if ((e = cudaFuncSetAttribute(stream_kernel<SCION_PTQ1_0, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                int(stream_smem<SCION_PTQ1_0, 2>()))))
-    return e;
-  return cudaFuncSetAttribute(stream_kernel<SCION_PTQ1_0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              int(stream_smem<SCION_PTQ1_0, 1>()));
+  if ((e = set_smem<SCION_PQ2_0, 2>())) return e;
+  if ((e = set_smem<SCION_PQ2_0, 1>())) return e;
+  if ((e = set_smem<SCION_PTQ1_0, 2>())) return e;
+  return set_smem<SCION_PTQ1_0, 1>();
 }
 
 cudaError_t launch_stream_gateup(const scion_layer* L, int T, cudaStream_t s) {

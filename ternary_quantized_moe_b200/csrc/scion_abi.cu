@@ -45,7 +45,7 @@ void free_layer(scion_layer* L) {
   void* ptrs[] = {L->gu_bank, L->dn_bank,  L->dense_down, L->xunits,  L->logits,    L->ids,       L->gates,
                   L->counts,  L->offsets,  L->perm,       L->active,  L->n_active,  L->h,         L->hz,
                   L->xfrag,   L->xpartial, L->xcount,     L->x_stage, L->out_stage, L->bad,       L->err,
-                  L->slot_info, L->route_done, L->gperm};
+                  L->slot_info, L->gperm, L->route_done};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   if (L->pre) {
@@ -262,10 +262,11 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   SCION_TRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&L->slot_info), sizeof(int4) * L->E));
   SCION_TRY(dev_alloc(L, &L->route_done, sizeof(unsigned)));
   SCION_TRY(cudaMemsetAsync(L->route_done, 0, sizeof(unsigned), s));
-  SCION_TRY(dev_alloc(L, &L->h, sizeof(__half) * TD * L->k * L->F));
+  SCION_TRY(dev_alloc(L, &L->h, sizeof(__half) * TD * L->k * L->GF * SCION_BROW));
   SCION_TRY(dev_alloc(L, &L->hz, sizeof(__half) * TD * (L->Kd ? L->Kd : 1)));
-  SCION_TRY(dev_alloc(L, &L->xfrag, sizeof(__half) * TD * L->d));
-  SCION_TRY(dev_alloc(L, &L->xpartial, sizeof(float) * (L->n_xunits ? L->n_xunits : 1) * L->n_xchunks * 2 * 16 * TD));
+  SCION_TRY(dev_alloc(L, &L->xfrag, sizeof(__half) * TD * L->Gd * SCION_BROW));
+  SCION_TRY(dev_alloc(L, &L->xpartial, sizeof(float) * (L->n_xunits ? L->n_xunits : 1) * 2 * 16 * TD));
+  SCION_TRY(cudaMemsetAsync(L->xpartial, 0, sizeof(float) * (L->n_xunits ? L->n_xunits : 1) * 2 * 16 * TD, s));
   SCION_TRY(dev_alloc(L, &L->xcount, sizeof(unsigned) * (L->n_xunits ? L->n_xunits : 1)));
   SCION_TRY(dev_alloc(L, &L->x_stage, sizeof(__nv_bfloat16) * size_t(max_tokens) * L->d));
   SCION_TRY(dev_alloc(L, &L->out_stage, sizeof(float) * size_t(max_tokens) * L->d));

@@ -35,6 +35,12 @@
 #define SCION_TDEC 64         // tokens per decode pass (larger batches run in passes)
 #define SCION_XPROJ_KC 512    // K columns per x-projection CTA (4 warps x 128)
 
+// Fragment-ordered B operands of the decode expert kernels (x for gate/up, h for down) are
+// stored per 128-column group as 128 fp16 values followed by a 16-byte tail; the first 4
+// bytes of the tail hold  -2^-24 * sum_k B_k * 4^f(k)  in fp32 (the start value of the PQ2_0
+// subnormal unpack's accumulators, see tern_tile.cuh).
+#define SCION_BROW 136        // halves per group row (128 + 8)
+
 namespace scion {
 
 constexpr int kPq2Block = 34;
@@ -102,11 +108,11 @@ struct scion_layer {
   int32_t* active;   // [E]
   int32_t* n_active; // [1]
   void* slot_info;    // int4 [E]: {expert, first position, token count, 0} per active slot
-  unsigned* route_done;  // [1] arrival counter of the decode route kernel
-  __half* h;         // [TDEC*k][F]
+  unsigned* route_done;  // [1] arrival counter of the decode route kernel (zero between calls)
+  __half* h;         // [TDEC*k][GF][SCION_BROW] fragment order + group-sum tails
   __half* hz;        // [TDEC][Kd] (pad columns stay 0)
-  __half* xfrag;     // [TDEC][Gd][128] x in fragment order (fp16)
-  float* xpartial;   // [n_xunits][n_xchunks][2][16][TDEC]
+  __half* xfrag;     // [TDEC][Gd][SCION_BROW] x in fragment order (fp16) + group-sum tails
+  float* xpartial;   // [n_xunits][2][16][TDEC] x-projection accumulation rows (zero between calls)
   unsigned* xcount;  // [n_xunits]
   void* x_stage;     // [max_tokens][d] bf16 (host-buffer forward)
   float* out_stage;  // [max_tokens][d]
@@ -143,7 +149,7 @@ cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, fl
 cudaError_t launch_gateup(const scion_layer* L, const __nv_bfloat16* x, int T, cudaStream_t s);
 cudaError_t launch_down_routed(const scion_layer* L, int T, float* out, cudaStream_t s);
 cudaError_t launch_down_dense(const scion_layer* L, int T, float* out, cudaStream_t s);
-// fragment-ordered rows [rows][G][128] -> natural order [rows][G*128]
+// fragment-ordered rows [rows][G][SCION_BROW] -> natural order [rows][G*128]
 cudaError_t launch_unfrag(int fmt, const __half* src, int rows, int G, __half* dst, cudaStream_t s);
 cudaError_t configure_kernels();
 

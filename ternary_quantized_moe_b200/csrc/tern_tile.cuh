@@ -46,6 +46,21 @@ __device__ __forceinline__ int frag_index(int fmt, int col) {
   return 32 * c + 2 * (5 * m + j) + h;
 }
 
+// Stored order of a B group row (SCION_BROW halves): lane (n, c) consumes the 32 elements
+// idx = 32c + w (w = 0..31) as four 16-byte chunks w / 8; chunk i of lane-column c is stored at
+// halves 32i + 8c, so the four lane-columns of one 16-byte load read 64 contiguous bytes.
+__device__ __forceinline__ int brow_pos_of(int c, int w) { return 32 * (w >> 3) + 8 * c + (w & 7); }
+// column held by stored position p
+__device__ __forceinline__ int brow_col(int fmt, int p) {
+  const int w = 8 * (p >> 5) + (p & 7), c = (p >> 3) & 3;
+  return frag_col(fmt, 32 * c + w);
+}
+// stored position of column col
+__device__ __forceinline__ int brow_pos(int fmt, int col) {
+  const int idx = frag_index(fmt, col);
+  return brow_pos_of(idx >> 5, idx & 31);
+}
+
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   uint4 v;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
@@ -68,6 +83,8 @@ __device__ __forceinline__ uint32_t ldg_stream32(const void* p) {
 // the B operand when it is written (an exact power-of-two scaling of the fp16 values).
 __device__ __forceinline__ int pq2_f(int s) { return s < 5 ? s : s - 5; }
 __device__ __forceinline__ float pq2_bscale(int idx) { return exp2f(-2.0f * pq2_f((idx & 31) >> 2)); }
+// the same factor for stored position p of a B group row
+__device__ __forceinline__ float brow_bscale(int p) { return exp2f(-2.0f * pq2_f(((p >> 5) * 8 + (p & 7)) >> 2)); }
 
 template <int S>
 __device__ __forceinline__ uint32_t pq2_pair_nf(uint32_t w, uint32_t w10) {
@@ -76,6 +93,18 @@ __device__ __forceinline__ uint32_t pq2_pair_nf(uint32_t w, uint32_t w10) {
   constexpr uint32_t biash = 0x6400u + (1u << (2 * f));  // fp16 bits of 1024 + 4^f (exact, < 2048)
   const __half2 v = u32_as_h2(lop3_and_or(S < 5 ? w : w10, mask, kMagic));
   return h2_as_u32(__hsub2(v, u32_as_h2(biash | (biash << 16))));
+}
+
+// PQ2_0 unpack to fp16 subnormals (one AND per two weights).  Masking the field of pair s
+// (bits 2f..2f+1 of each 16-bit half, f = s < 5 ? s : s - 5, pairs 5..7 taken from w >> 10)
+// leaves the bit pattern b * 4^f with a zero exponent field: the fp16 subnormal
+// b * 4^f * 2^-24, where b = code + 1 is the stored field (0..2).  With the B operand
+// pre-scaled by 4^-f the MMA sums 2^-24 * b * x; starting the accumulator at
+// -2^-24 * sum(x) (the group-row tail) leaves 2^-24 * sum(code * x).
+template <int S>
+__device__ __forceinline__ uint32_t pq2_pair_sub(uint32_t w, uint32_t w10) {
+  constexpr int f = S < 5 ? S : S - 5;
+  return (S < 5 ? w : w10) & (0x00030003u << (2 * f));
 }
 
 // Registers of one 16-row x 128-column sub-tile block for lane (r8, c).
@@ -204,14 +233,38 @@ __device__ __forceinline__ void tile_mma(const TileRegs<FMT>& t, const uint32_t 
   acc[3] = fmaf(s_hi, g[3], acc[3]);
 }
 
-// B fragment of one group for lane (n, c): 64 contiguous bytes of row `row` (or zeros).
+// PQ2_0, subnormal unpack: acc += scale_row * 2^-24 * (codes . B) for one tile and one token
+// tile of 8.  xn0 / xn1 = -2^-24 * (group sum of B) of the lane's token columns 2c, 2c+1.
+__device__ __forceinline__ void tile_mma_pq2_sub(const TileRegs<SCION_PQ2_0>& t, const uint32_t (&b)[16],
+                                                 float (&acc)[4], float xn0, float xn1) {
+  float g[4] = {xn0, xn1, xn0, xn1};
+  const uint32_t x10 = t.w.x >> 10, y10 = t.w.y >> 10, z10 = t.w.z >> 10, w10 = t.w.w >> 10;
+#define SCION_PQ2_SUB_STEP(S)                                                                      \
+  {                                                                                                \
+    const uint32_t fa[4] = {pq2_pair_sub<S>(t.w.x, x10), pq2_pair_sub<S>(t.w.z, z10),              \
+                            pq2_pair_sub<S>(t.w.y, y10), pq2_pair_sub<S>(t.w.w, w10)};             \
+    mma_f16_16816(g, fa, b[2 * S], b[2 * S + 1]);                                                  \
+  }
+  SCION_PQ2_SUB_STEP(0) SCION_PQ2_SUB_STEP(1) SCION_PQ2_SUB_STEP(2) SCION_PQ2_SUB_STEP(3)
+  SCION_PQ2_SUB_STEP(4) SCION_PQ2_SUB_STEP(5) SCION_PQ2_SUB_STEP(6) SCION_PQ2_SUB_STEP(7)
+#undef SCION_PQ2_SUB_STEP
+  const float s_lo = __half2float(__ushort_as_half(uint16_t(t.sc & 0xffff)));
+  const float s_hi = __half2float(__ushort_as_half(uint16_t(t.sc >> 16)));
+  acc[0] = fmaf(s_lo, g[0], acc[0]);
+  acc[1] = fmaf(s_lo, g[1], acc[1]);
+  acc[2] = fmaf(s_hi, g[2], acc[2]);
+  acc[3] = fmaf(s_hi, g[3], acc[3]);
+}
+
+// B fragment of one group for lane (n, c): its 64 bytes of row `row` (or zeros); group rows are
+// SCION_BROW halves apart.
 __device__ __forceinline__ void load_b(const __half* base, int64_t row_stride_h, int row, int g, int c,
                                        uint32_t (&b)[16]) {
   if (row >= 0) {
-    const uint4* p = reinterpret_cast<const uint4*>(base + int64_t(row) * row_stride_h + int64_t(g) * 128 + 32 * c);
+    const __half* rp = base + int64_t(row) * row_stride_h + int64_t(g) * SCION_BROW + 8 * c;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const uint4 v = p[i];
+      const uint4 v = *reinterpret_cast<const uint4*>(rp + 32 * i);
       b[4 * i] = v.x, b[4 * i + 1] = v.y, b[4 * i + 2] = v.z, b[4 * i + 3] = v.w;
     }
   } else {
@@ -219,29 +272,5 @@ __device__ __forceinline__ void load_b(const __half* base, int64_t row_stride_h,
     for (int i = 0; i < 16; ++i) b[i] = 0u;
   }
 }
-
-
-// One 128-column group of x (bf16) -> fp16 in the decode fragment order of the format, with
-// the exact power-of-two B scaling of the PQ2_0 shift-free unpack.
-template <int FMT>
-__device__ __forceinline__ void xfrag_group(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst) {
-  __align__(16) __nv_bfloat16 in[128];
-  __align__(16) __half outv[128];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) reinterpret_cast<uint4*>(in)[j] = reinterpret_cast<const uint4*>(src)[j];
-#pragma unroll
-  for (int idx = 0; idx < 128; ++idx) {
-    float v = __bfloat162float(in[frag_col(FMT, idx)]);
-    if (FMT == SCION_PQ2_0) {
-      const int s = (idx & 31) >> 2;
-      v *= 1.0f / float(1 << (2 * (s < 5 ? s : s - 5)));
-    }
-    outv[idx] = __float2half_rn(v);
-  }
-#pragma unroll
-  for (int j = 0; j < 16; ++j) reinterpret_cast<uint4*>(dst)[j] = reinterpret_cast<uint4*>(outv)[j];
-}
-
-
 
 }  // namespace scion
