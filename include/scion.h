@@ -158,9 +158,10 @@ size_t scion_layer_device_bytes(const scion_layer* layer);
 int scion_moe_forward(const void* x, int T, const scion_layer* layer, float* out, void* stream);
 
 /* Tuning options of a layer (scion_layer_set_option).
- *  SCION_OPT_STREAM_MIN_TOKENS (default 65 = off): batches of at least this many tokens
- *    (and at most 64) run the expert GEMVs on the kernels fed by a bulk-copy ring (one CTA
- *    per 128 expert rows); other batches split K over the warps of one CTA per 16 rows.
+ *  SCION_OPT_STREAM_MIN_TOKENS (default 16): batches of at least this many tokens (and at
+ *    most 64) run the expert GEMVs on the persistent kernels fed by a bulk-copy ring (128
+ *    expert rows per work item); smaller batches split K over the warps of one CTA per 16
+ *    rows, which spreads the few active experts over more SMs.
  *    Both give the same result up to fp32 summation order.
  * EINVAL for an unknown option or an out-of-range value. */
 enum { SCION_OPT_STREAM_MIN_TOKENS = 1 };

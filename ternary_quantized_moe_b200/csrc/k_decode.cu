@@ -46,17 +46,18 @@ struct XProjArgs {
   float* out;     // zeroed here
 };
 
-// One CTA = (unit, 512-column chunk); 4 warps x 128 columns.  NT = token tiles of 8.  With
+// One CTA = (unit, 512-column chunk); 8 warps x 64 columns.  NT = token tiles of 8.  With
 // several chunks, each CTA adds its unit's partial sums into the unit's fp32 accumulation rows
 // (red.add) and the last CTA of the unit to arrive applies the epilogue and clears the rows.
 // kXAux extra CTA columns convert x to the fragment order and clear out and the hidden tails.
 constexpr int kXRow = SCION_XPROJ_KC + 8;  // bf16 elements per staged token row (+16 B pad)
-constexpr int kXAux = 8;
+constexpr int kXAux = 4;
+constexpr int kXThreads = 256;  // 8 warps x 64 columns
 
 template <int NT>
 constexpr size_t xproj_smem(int T) {
-  return (size_t(T) * kXRow * 2 > size_t(4) * 2 * NT * 32 * 4 * 4) ? size_t(T) * kXRow * 2
-                                                                    : size_t(4) * 2 * NT * 32 * 4 * 4;
+  return (size_t(T) * kXRow * 2 > size_t(8) * 2 * NT * 32 * 4 * 4) ? size_t(T) * kXRow * 2
+                                                                    : size_t(8) * 2 * NT * 32 * 4 * 4;
 }
 
 __device__ __forceinline__ void xproj_aux(const XProjArgs& a, int aux, int n_aux) {
@@ -65,7 +66,7 @@ __device__ __forceinline__ void xproj_aux(const XProjArgs& a, int aux, int n_aux
   // x -> fragment order: item = (token, group, 8-element part); the 16 parts of a group sit in
   // 16 consecutive lanes, which sum the group's B * 4^f for the row tail.
   const int total = a.T * Gd * 16;
-  for (int base = aux * 128 + (threadIdx.x & ~31); base < total; base += n_aux * 128) {
+  for (int base = aux * kXThreads + (threadIdx.x & ~31); base < total; base += n_aux * kXThreads) {
     const int item = base + lane;
     const bool ok = item < total;
     const int grp = ok ? item >> 4 : 0, part = item & 15;
@@ -93,7 +94,7 @@ __device__ __forceinline__ void xproj_aux(const XProjArgs& a, int aux, int n_aux
       if (part == 0) *reinterpret_cast<float4*>(dst + 128) = make_float4(-5.9604644775390625e-08f * sum, 0.f, 0.f, 0.f);
     }
   }
-  const int tid = aux * 128 + threadIdx.x, nth = n_aux * 128;
+  const int tid = aux * kXThreads + threadIdx.x, nth = n_aux * kXThreads;
   float4* o4 = reinterpret_cast<float4*>(a.out);
   for (int64_t i = tid; i < int64_t(a.T) * a.d / 4; i += nth) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   // the expert hidden's group sums are accumulated by the gate/up epilogue
@@ -102,7 +103,7 @@ __device__ __forceinline__ void xproj_aux(const XProjArgs& a, int aux, int n_aux
 }
 
 template <int NT>
-__global__ void __launch_bounds__(128) xproj_kernel(XProjArgs a) {
+__global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
   extern __shared__ __align__(16) uint8_t xsm[];
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(xsm);  // [NT*8][kXRow], then the warp reduction
   __shared__ int last_flag;
@@ -137,16 +138,16 @@ __global__ void __launch_bounds__(128) xproj_kernel(XProjArgs a) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[m][nt][i] = 0.f;
 
-  const int kw = kbase + warp * 128;
+  const int kw = kbase + warp * 64;
   const int row_a = u.row0 + g8, row_b = u.row0 + g8 + 8;
   const bool ok_a = row_a < nrows, ok_b = row_b < nrows;
   const bool active_warp = kw < a.d;
-  // weights first (they do not depend on x): both matrices, this warp's 128 columns
-  uint4 wa[2][4], wb[2][4];
+  // weights first (they do not depend on x): both matrices, this warp's 64 columns
+  uint4 wa[2][2], wb[2][2];
 #pragma unroll
   for (int m = 0; m < 2; ++m)
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 2; ++q) {
       const int kk = kw + 32 * q + 8 * c;
       const bool ld = active_warp && m < nmat;
       wa[m][q] = (ld && ok_a) ? ldg_stream(mats[m] + int64_t(row_a) * a.d + kk) : make_uint4(0, 0, 0, 0);
@@ -154,9 +155,10 @@ __global__ void __launch_bounds__(128) xproj_kernel(XProjArgs a) {
     }
   pdl_wait();  // everything below reads x or writes the workspace
   // stage x[0..T)[kbase .. kbase+512) in shared memory (rows padded by 16 B: conflict-free reads)
-  const int kcols = min(SCION_XPROJ_KC, a.d - kbase);
-  for (int i = threadIdx.x; i < a.T * (kcols >> 3); i += blockDim.x) {
-    const int t = i / (kcols >> 3), j = i % (kcols >> 3);
+  const int kchunks = min(SCION_XPROJ_KC, a.d - kbase) >> 3;  // 16-byte chunks per token row (<= 64)
+  for (int i = threadIdx.x; i < a.T * 64; i += kXThreads) {
+    const int t = i >> 6, j = i & 63;
+    if (j >= kchunks) continue;
     const uint32_t dst = uint32_t(__cvta_generic_to_shared(xs + t * kXRow + 8 * j));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(a.x + int64_t(t) * a.d + kbase + 8 * j)
                  : "memory");
@@ -165,7 +167,7 @@ __global__ void __launch_bounds__(128) xproj_kernel(XProjArgs a) {
   __syncthreads();
   if (active_warp) {
     const bool second_acc = (u.kind == kUnitSwiglu);
-    const int kwl = warp * 128;
+    const int kwl = warp * 64;
 #pragma unroll
     for (int m = 0; m < 2; ++m) {
       if (m >= nmat) break;
@@ -173,7 +175,7 @@ __global__ void __launch_bounds__(128) xproj_kernel(XProjArgs a) {
       for (int nt = 0; nt < NT; ++nt) {
         const int tok = nt * 8 + g8;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
           const uint4 xb = tok < a.T ? *reinterpret_cast<const uint4*>(xs + tok * kXRow + kwl + 32 * q + 8 * c)
                                      : make_uint4(0, 0, 0, 0);
           const uint32_t fa0[4] = {wa[m][q].x, wb[m][q].x, wa[m][q].y, wb[m][q].y};
@@ -199,14 +201,16 @@ __global__ void __launch_bounds__(128) xproj_kernel(XProjArgs a) {
       for (int i = 0; i < 4; ++i) red[warp][m][nt][lane][i] = acc[m][nt][i];
   __syncthreads();
 
-  // thread -> (nt, lane) pairs; sum the 4 warps
+  // thread -> (nt, lane) pairs; sum the 8 warps
   float* accum = a.partial + int64_t(blockIdx.x) * (2 * 16 * SCION_TDEC);  // [m][row][tok]
   for (int p = threadIdx.x; p < NT * 32; p += blockDim.x) {
     const int nt = p >> 5, ln = p & 31;
     for (int m = 0; m < nacc; ++m)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const float v = red[0][m][nt][ln][i] + red[1][m][nt][ln][i] + red[2][m][nt][ln][i] + red[3][m][nt][ln][i];
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) v += red[w][m][nt][ln][i];
         const int row = (ln >> 2) + 8 * (i >> 1), tok = nt * 8 + 2 * (ln & 3) + (i & 1);
         red[0][m][nt][ln][i] = v;
         if (a.n_chunks > 1 && tok < a.T) atomicAdd(&accum[(m * 16 + row) * SCION_TDEC + tok], v);
@@ -227,14 +231,14 @@ __global__ void __launch_bounds__(128) xproj_kernel(XProjArgs a) {
   }
 
   // epilogue: thread -> (row, tok); all loads of the thread are issued together
-  constexpr int kIt = 16 * SCION_TDEC / 128;
+  constexpr int kIt = 16 * SCION_TDEC / kXThreads;
   float v[kIt][2];
 #pragma unroll
   for (int it = 0; it < kIt; ++it) {
-    const int p = threadIdx.x + 128 * it;
+    const int p = threadIdx.x + kXThreads * it;
+    const int row = p / SCION_TDEC, tok = p % SCION_TDEC;
     v[it][0] = v[it][1] = 0.f;
-    if (p >= 16 * a.T) continue;
-    const int row = p / a.T, tok = p % a.T;
+    if (tok >= a.T) continue;
     if (a.n_chunks > 1) {
       for (int m = 0; m < nacc; ++m) v[it][m] = __ldcg(&accum[(m * 16 + row) * SCION_TDEC + tok]);
     } else {
@@ -244,9 +248,9 @@ __global__ void __launch_bounds__(128) xproj_kernel(XProjArgs a) {
   }
 #pragma unroll
   for (int it = 0; it < kIt; ++it) {
-    const int p = threadIdx.x + 128 * it;
-    if (p >= 16 * a.T) continue;
-    const int row = p / a.T, tok = p % a.T;
+    const int p = threadIdx.x + kXThreads * it;
+    const int row = p / SCION_TDEC, tok = p % SCION_TDEC;
+    if (tok >= a.T) continue;
     const int grow = u.row0 + row;
     if (a.n_chunks > 1)
       for (int m = 0; m < nacc; ++m) accum[(m * 16 + row) * SCION_TDEC + tok] = 0.f;  // ready for the next call
@@ -518,10 +522,10 @@ cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, fl
   dim3 grid(L->n_xunits + kXAux, L->n_xchunks);
   const int nt = (T + 7) / 8;
   switch (nt) {
-    case 1: return launch_pdl(xproj_kernel<1>, grid, dim3(128), xproj_smem<1>(T), s, a);
-    case 2: return launch_pdl(xproj_kernel<2>, grid, dim3(128), xproj_smem<2>(T), s, a);
-    case 3: case 4: return launch_pdl(xproj_kernel<4>, grid, dim3(128), xproj_smem<4>(T), s, a);
-    default: return launch_pdl(xproj_kernel<8>, grid, dim3(128), xproj_smem<8>(T), s, a);
+    case 1: return launch_pdl(xproj_kernel<1>, grid, dim3(kXThreads), xproj_smem<1>(T), s, a);
+    case 2: return launch_pdl(xproj_kernel<2>, grid, dim3(kXThreads), xproj_smem<2>(T), s, a);
+    case 3: case 4: return launch_pdl(xproj_kernel<4>, grid, dim3(kXThreads), xproj_smem<4>(T), s, a);
+    default: return launch_pdl(xproj_kernel<8>, grid, dim3(kXThreads), xproj_smem<8>(T), s, a);
   }
   return cudaGetLastError();
 }

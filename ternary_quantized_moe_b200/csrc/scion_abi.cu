@@ -231,7 +231,7 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   L->Gd = L->d / 128, L->GF = L->F / 128;
   L->Kdense = L->Fs + L->r;
   L->Kd = (L->Kdense + 63) / 64 * 64;
-  L->stream_min_tokens = SCION_TDEC + 1;  // the split-K register kernels measured faster at every decode batch size
+  L->stream_min_tokens = 16;  // below this the few active experts spread better over the split-K kernels
   cudaStream_t s = as_stream(stream);
   const int tb = scion::tile_bytes(L->fmt);
   const int TD = SCION_TDEC;
