@@ -90,45 +90,71 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Predicated shared-memory loads: lanes whose token lies past the pass's count issue no bank
+// access and keep the old register contents (their accumulator columns are dropped later).
+__device__ __forceinline__ void lds128_if(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, uint32_t addr,
+                                          bool p) {
+  asm volatile(
+      "{\n .reg .pred q;\n setp.ne.u32 q, %5, 0;\n @q ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n}\n"
+      : "+r"(r0), "+r"(r1), "+r"(r2), "+r"(r3)
+      : "r"(addr), "r"(uint32_t(p)));
+}
+__device__ __forceinline__ float ldsf_if(uint32_t addr, bool p) {
+  float v = 0.f;
+  asm volatile("{\n .reg .pred q;\n setp.ne.u32 q, %2, 0;\n @q ld.shared.f32 %0, [%1];\n}\n"
+               : "+f"(v)
+               : "r"(addr), "r"(uint32_t(p)));
+  return v;
+}
+
+// Per-lane shared-memory offsets within a stage (loop invariant).
+struct LaneOffs {
+  uint32_t code;   // this warp's tile of matrix 0, lane's 16 bytes
+  uint32_t scale;  // this warp's tile of matrix 0, the scales of rows r, r + 8
+  uint32_t brow;   // B row of token n, lane-column c
+  uint32_t tail0, tail1;  // group-sum tails of tokens 2c, 2c + 1
+};
+
+// First MMA of a chain: d = a b + c with c in other registers (no copies into the accumulator).
+__device__ __forceinline__ void mma_f16_c(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1, float c0,
+                                          float c1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%11,%10,%11};\n"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c0), "f"(c1));
+}
+
 // One stage's groups [j0, j0 + J) for this warp: J x NMAT independent PQ2_0 tiles (subnormal
 // unpack, accumulators started at the group-sum tails) or PTQ1_0 tiles (digit chain).
 template <int FMT, int NMAT, int J>
-__device__ __forceinline__ void stage_groups(const uint8_t* stg, int j0, int nn, int warp, int lane,
+__device__ __forceinline__ void stage_groups(uint32_t stg, const LaneOffs& o, int j0, int nn, int lane,
                                              float (&acc)[NMAT][4]) {
-  constexpr int G = gps<NMAT>();
   constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
   constexpr uint32_t cb = code_bytes<FMT, NMAT>();
-  constexpr uint32_t ts = tok_stride<NMAT>();
   const int c = lane & 3, n = lane >> 2;
-  const uint8_t* codes = stg + kHdr;
-  const uint8_t* brows = stg + kHdr + G * cb;
   uint32_t b[J][16];
 #pragma unroll
-  for (int j = 0; j < J; ++j) {
-    // only the pass's tokens are read (the columns of the others are dropped by the epilogue)
-    const uint8_t* bp = brows + tok_off(ts, n) + (j0 + j) * kRowB + 16 * c;
+  for (int j = 0; j < J; ++j)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint4 v = n < nn ? *reinterpret_cast<const uint4*>(bp + 64 * i) : make_uint4(0, 0, 0, 0);
-      b[j][4 * i] = v.x, b[j][4 * i + 1] = v.y, b[j][4 * i + 2] = v.z, b[j][4 * i + 3] = v.w;
-    }
-  }
+    for (int i = 0; i < 4; ++i)
+      lds128_if(b[j][4 * i], b[j][4 * i + 1], b[j][4 * i + 2], b[j][4 * i + 3],
+                stg + o.brow + (j0 + j) * kRowB + 64 * i, n < nn);
   if constexpr (FMT == SCION_PQ2_0) {
     uint4 w[J][NMAT];
     uint32_t sc[J][NMAT];
-    float g[J][NMAT][4];
+    float g[J][NMAT][4], xn[J][2];
 #pragma unroll
     for (int j = 0; j < J; ++j) {
-      // -2^-24 * group sums of the lane's token columns 2c, 2c+1
-      const float xn0 = 2 * c < nn ? *reinterpret_cast<const float*>(brows + tok_off(ts, 2 * c) + (j0 + j) * kRowB + 256) : 0.f;
-      const float xn1 =
-          2 * c + 1 < nn ? *reinterpret_cast<const float*>(brows + tok_off(ts, 2 * c + 1) + (j0 + j) * kRowB + 256) : 0.f;
+      // -2^-24 * group sums of the lane's token columns 2c, 2c+1: the chains' start values
+      xn[j][0] = ldsf_if(stg + o.tail0 + (j0 + j) * kRowB, 2 * c < nn);
+      xn[j][1] = ldsf_if(stg + o.tail1 + (j0 + j) * kRowB, 2 * c + 1 < nn);
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) {
-        const uint8_t* blk = codes + (j0 + j) * cb + (m * 8 + warp) * tb;
-        w[j][m] = *reinterpret_cast<const uint4*>(blk + 16 * lane);
-        sc[j][m] = *reinterpret_cast<const uint32_t*>(blk + 512 + 4 * (lane >> 2));
-        g[j][m][0] = xn0, g[j][m][1] = xn1, g[j][m][2] = xn0, g[j][m][3] = xn1;
+        const uint32_t blk = stg + (j0 + j) * cb + m * 8 * tb;
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(w[j][m].x), "=r"(w[j][m].y), "=r"(w[j][m].z), "=r"(w[j][m].w)
+                     : "r"(blk + o.code));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sc[j][m]) : "r"(blk + o.scale));
       }
     }
     uint32_t w10[J][NMAT][4];
@@ -138,25 +164,34 @@ __device__ __forceinline__ void stage_groups(const uint8_t* stg, int j0, int nn,
       for (int m = 0; m < NMAT; ++m)
         w10[j][m][0] = w[j][m].x >> 10, w10[j][m][1] = w[j][m].y >> 10, w10[j][m][2] = w[j][m].z >> 10,
         w10[j][m][3] = w[j][m].w >> 10;
-#define SCION_SUB_STEP(S)                                                                              \
-  _Pragma("unroll") for (int j = 0; j < J; ++j) _Pragma("unroll") for (int m = 0; m < NMAT; ++m) {     \
-    const uint32_t fa[4] = {pq2_pair_sub<S>(w[j][m].x, w10[j][m][0]), pq2_pair_sub<S>(w[j][m].z, w10[j][m][2]), \
-                            pq2_pair_sub<S>(w[j][m].y, w10[j][m][1]), pq2_pair_sub<S>(w[j][m].w, w10[j][m][3])}; \
-    mma_f16(g[j][m], fa, b[j][2 * S], b[j][2 * S + 1]);                                                \
-  }
-    SCION_SUB_STEP(0) SCION_SUB_STEP(1) SCION_SUB_STEP(2) SCION_SUB_STEP(3)
-    SCION_SUB_STEP(4) SCION_SUB_STEP(5) SCION_SUB_STEP(6) SCION_SUB_STEP(7)
-#undef SCION_SUB_STEP
+#define SCION_SUB_FA(S)                                                                                  \
+  const uint32_t fa[4] = {pq2_pair_sub<S>(w[j][m].x, w10[j][m][0]), pq2_pair_sub<S>(w[j][m].z, w10[j][m][2]), \
+                          pq2_pair_sub<S>(w[j][m].y, w10[j][m][1]), pq2_pair_sub<S>(w[j][m].w, w10[j][m][3])};
 #pragma unroll
     for (int j = 0; j < J; ++j)
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) {
-        const float s_lo = __half2float(__ushort_as_half(uint16_t(sc[j][m] & 0xffff)));
-        const float s_hi = __half2float(__ushort_as_half(uint16_t(sc[j][m] >> 16)));
-        acc[m][0] = fmaf(s_lo, g[j][m][0], acc[m][0]);
-        acc[m][1] = fmaf(s_lo, g[j][m][1], acc[m][1]);
-        acc[m][2] = fmaf(s_hi, g[j][m][2], acc[m][2]);
-        acc[m][3] = fmaf(s_hi, g[j][m][3], acc[m][3]);
+        SCION_SUB_FA(0)
+        mma_f16_c(g[j][m], fa, b[j][0], b[j][1], xn[j][0], xn[j][1]);
+      }
+#define SCION_SUB_STEP(S)                                                                              \
+  _Pragma("unroll") for (int j = 0; j < J; ++j) _Pragma("unroll") for (int m = 0; m < NMAT; ++m) {     \
+    SCION_SUB_FA(S)                                                                                    \
+    mma_f16(g[j][m], fa, b[j][2 * S], b[j][2 * S + 1]);                                                \
+  }
+    SCION_SUB_STEP(1) SCION_SUB_STEP(2) SCION_SUB_STEP(3)
+    SCION_SUB_STEP(4) SCION_SUB_STEP(5) SCION_SUB_STEP(6) SCION_SUB_STEP(7)
+#undef SCION_SUB_STEP
+#undef SCION_SUB_FA
+#pragma unroll
+    for (int j = 0; j < J; ++j)
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m) {
+        const float2 sf = __half22float2(u32_as_h2(sc[j][m]));  // scales of rows r, r + 8
+        acc[m][0] = fmaf(sf.x, g[j][m][0], acc[m][0]);
+        acc[m][1] = fmaf(sf.x, g[j][m][1], acc[m][1]);
+        acc[m][2] = fmaf(sf.y, g[j][m][2], acc[m][2]);
+        acc[m][3] = fmaf(sf.y, g[j][m][3], acc[m][3]);
       }
   } else {
 #pragma unroll
@@ -164,7 +199,7 @@ __device__ __forceinline__ void stage_groups(const uint8_t* stg, int j0, int nn,
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) {
         TileRegs<FMT> t;
-        t.load_shared(smem_u32(codes + (j0 + j) * cb + (m * 8 + warp) * tb), lane);
+        t.load_shared(stg + (j0 + j) * cb + m * 8 * tb + o.code - 16 * lane, lane);
         tile_mma<FMT>(t, b[j], acc[m], c);
       }
   }
@@ -274,12 +309,31 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
 
   // ---------------- consumers: warp w owns rows 16w .. 16w+15 of every item
   const int c = lane & 3;
+  constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
+  LaneOffs lo;
+  lo.code = kHdr + warp * tb + 16 * lane;
+  lo.scale = kHdr + warp * tb + 512 + 4 * (lane >> 2);
+  lo.brow = kHdr + GPS * cb + tok_off(tok_stride<NMAT>(), lane >> 2) + 16 * c;
+  lo.tail0 = kHdr + GPS * cb + tok_off(tok_stride<NMAT>(), 2 * c) + 256;
+  lo.tail1 = kHdr + GPS * cb + tok_off(tok_stride<NMAT>(), 2 * c + 1) + 256;
+  const uint32_t ring_u32 = smem_u32(ring);
+  // epilogue constants of this lane's rows r = 16 warp + lane / 4 and r + 8 (the same in every
+  // 128-row block): stored position of the row in the hidden's group row and its 4^-f factor
+  int hpos[2];
+  float hsc[2], hinv[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    hpos[h] = brow_pos(FMT, warp * 16 + (lane >> 2) + 8 * h);
+    hsc[h] = FMT == SCION_PQ2_0 ? brow_bscale(hpos[h]) : 1.0f;
+    hinv[h] = 1.0f / hsc[h];
+  }
   float acc[NMAT][4];
   for (int st = 0;; ++st) {
     const int s = st % kRing;
     if (!mbar_wait(&full[s], (st / kRing) & 1, &abort_flag, a.err)) break;
-    const uint8_t* stg = ring + s * sb;
-    const StageHdr* hd = reinterpret_cast<const StageHdr*>(stg);
+    const uint8_t* stgp = ring + s * sb;
+    const uint32_t stg = ring_u32 + s * sb;
+    const StageHdr* hd = reinterpret_cast<const StageHdr*>(stgp);
     const int nn = hd->nn;
     if (nn < 0) break;
     const int flags = hd->flags, ng = hd->ng;
@@ -291,10 +345,14 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
     }
 #pragma unroll
     for (int j0 = 0; j0 < GPS; j0 += 2) {
-      if (j0 + 1 < ng)
-        stage_groups<FMT, NMAT, 2>(stg, j0, nn, warp, lane, acc);
-      else if (j0 < ng)
-        stage_groups<FMT, NMAT, 1>(stg, j0, nn, warp, lane, acc);
+      // PQ2_0 takes groups in pairs (more independent MMA chains); the PTQ1_0 digit chains
+      // already need most of the registers, so it takes them one at a time
+      if (FMT == SCION_PQ2_0 && j0 + 1 < ng) {
+        stage_groups<FMT, NMAT, 2>(stg, lo, j0, nn, lane, acc);
+      } else {
+        if (j0 < ng) stage_groups<FMT, NMAT, 1>(stg, lo, j0, nn, lane, acc);
+        if (j0 + 1 < ng) stage_groups<FMT, NMAT, 1>(stg, lo, j0 + 1, nn, lane, acc);
+      }
     }
     if (flags & 2) {
       // epilogue: this warp's 16 rows x the pass's tokens
@@ -306,13 +364,10 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
         const int row = warp * 16 + (lane >> 2) + 8 * (i >> 1);
         const int tcol = 2 * c + (i & 1);
         if constexpr (NMAT == 2) {
-          const int f = rb * 128 + row;
-          const int idx = brow_pos(FMT, f & 127);
-          float h = silu_f(acc[0][i] * unit) * (acc[1][i] * unit);
-          if (FMT == SCION_PQ2_0) h *= brow_bscale(idx);
+          const float h = silu_f(acc[0][i] * unit) * (acc[1][i] * unit) * hsc[i >> 1];
           const __half h16 = __float2half_rn(h);
-          if (tcol < nn) a.hfrag[(int64_t(hd->pos[tcol]) * (a.F >> 7) + (f >> 7)) * SCION_BROW + idx] = h16;
-          if (FMT == SCION_PQ2_0) hs[i & 1] += __half2float(h16) / brow_bscale(idx);
+          if (tcol < nn) a.hfrag[(int64_t(hd->pos[tcol]) * (a.F >> 7) + rb) * SCION_BROW + hpos[i >> 1]] = h16;
+          if (FMT == SCION_PQ2_0) hs[i & 1] += __half2float(h16) * hinv[i >> 1];
         } else {
           if (tcol < nn)
             atomicAdd(&a.out[int64_t(hd->orow[tcol]) * a.d + rb * 128 + row], hd->gate[tcol] * (acc[0][i] * unit));
