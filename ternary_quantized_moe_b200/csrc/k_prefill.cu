@@ -80,7 +80,7 @@ enum DenseEpi : int { kEpiLogits = 0, kEpiSwiglu = 1, kEpiPlain = 2, kEpiStore =
 
 struct DenseUnit {
   int epi;     // DenseEpi
-  int na;      // A matrices in this unit (1 or 2)
+  int na;      // A matrices in this unit (1 or 2); units with 2 run 128-token tiles, the others 256
   int map1;    // accumulator of the second matrix (0 = same as the first)
   int mat0, mat1;  // indices into the A tensor-map table
   int row0;    // first weight row
@@ -92,6 +92,8 @@ struct DenseParams {
   CUtensorMap a[6];  // A matrices, box {64, 128}
   CUtensorMap b;     // B (tokens x K), box {64, 128}
   const DenseUnit* units;
+  int n_units2;      // units with two A matrices (listed first)
+  int n_units;
   int K, T, ab_bf16;
   float* logits;  int ld_logits;
   __half* hz;     int ld_hz;
@@ -101,31 +103,50 @@ struct DenseParams {
 
 constexpr int kDenseStages = 4;
 constexpr int kBK = 64;
+constexpr uint32_t kDenseStage = 3 * 128 * kBK * 2;  // 48 KB: two A boxes + one B box, or one A + two B
 
+// Tile t of the persistent schedule: 256-token block b = t / per_block; inside a block the
+// two-matrix units come first with two 128-token tiles each, then the one-matrix units with
+// one 256-token tile each.  Every role derives the same sequence from the same arithmetic.
+struct DenseTile {
+  int unit, tok0, ntok;  // ntok = 128 or 256 (tokens past T are not stored)
+};
+__device__ __forceinline__ DenseTile dense_tile(const DenseParams& p, int t) {
+  const int per_block = 2 * p.n_units2 + (p.n_units - p.n_units2);
+  const int b = t / per_block, r = t % per_block;
+  DenseTile d;
+  if (r < 2 * p.n_units2) {
+    d.unit = r >> 1, d.tok0 = 256 * b + 128 * (r & 1), d.ntok = 128;
+  } else {
+    d.unit = p.n_units2 + (r - 2 * p.n_units2), d.tok0 = 256 * b, d.ntok = 256;
+  }
+  return d;
+}
+
+// Persistent tcgen05 GEMM over (weight-row unit, token block) tiles: one TMA producer thread,
+// one MMA thread, four epilogue warps; the stage ring runs on across tiles and the fp32
+// accumulator is double-buffered in tensor memory (2 x 256 columns), so the epilogue of a tile
+// overlaps the main loop of the next.
 __global__ void __launch_bounds__(kThreads, 1) dense_gemm_kernel(const __grid_constant__ DenseParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // 1024-aligned, still __shared__
-  __shared__ uint64_t full[kDenseStages], empty[kDenseStages], accf;
+  __shared__ uint64_t full[kDenseStages], empty[kDenseStages], acc_full[2], acc_empty[2], mma_done;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const DenseUnit u = p.units[blockIdx.x];
-  const int tok0 = blockIdx.y * kBN;
-  const int na = u.na;
-  const int nacc = (na == 2 && u.map1 == 1) ? 2 : 1;
-  const uint32_t a_bytes = kBM * kBK * 2, b_bytes = kBN * kBK * 2;
-  const uint32_t stage_bytes = 2 * a_bytes + b_bytes;
+  const int per_block = 2 * p.n_units2 + (p.n_units - p.n_units2);
+  const int n_tiles = per_block * ((p.T + 255) / 256);
   const int nk = p.K / kBK;
-  const uint32_t ncols = nacc == 2 ? 2 * kBN : kBN;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDenseStages; ++s) mbar_init(&full[s], 1), mbar_init(&empty[s], 1);
-    mbar_init(&accf, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&acc_full[i], 1), mbar_init(&acc_empty[i], 128);
+    mbar_init(&mma_done, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(&tmem_slot, ncols);
+  if (warp == 1) tmem_alloc(&tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -133,73 +154,120 @@ __global__ void __launch_bounds__(kThreads, 1) dense_gemm_kernel(const __grid_co
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % kDenseStages;
-      if (kb >= kDenseStages && !mbar_wait(&empty[s], ((kb / kDenseStages) - 1) & 1, &abort_flag, p.err)) break;
-      uint8_t* st = smem + s * stage_bytes;
-      mbar_arrive_expect_tx(&full[s], na * a_bytes + b_bytes);
-      tma_load_2d(st, &p.a[u.mat0], kb * kBK, u.row0, &full[s]);
-      if (na == 2) tma_load_2d(st + a_bytes, &p.a[u.mat1], kb * kBK, u.row0, &full[s]);
-      tma_load_2d(st + 2 * a_bytes, &p.b, kb * kBK, tok0, &full[s]);
+    int ks = 0;  // running k-block counter (ring position)
+    for (int t = blockIdx.x; t < n_tiles && !abort_flag; t += gridDim.x) {
+      const DenseTile dt = dense_tile(p, t);
+      if (dt.tok0 >= p.T) continue;
+      const DenseUnit u = p.units[dt.unit];
+      const uint32_t bytes = u.na * 128 * kBK * 2 + dt.ntok * kBK * 2;
+      for (int kb = 0; kb < nk; ++kb, ++ks) {
+        const int s = ks % kDenseStages;
+        if (ks >= kDenseStages && !mbar_wait(&empty[s], ((ks / kDenseStages) - 1) & 1, &abort_flag, p.err)) break;
+        uint8_t* st = smem + s * kDenseStage;
+        mbar_arrive_expect_tx(&full[s], bytes);
+        tma_load_2d(st, &p.a[u.mat0], kb * kBK, u.row0, &full[s]);
+        uint8_t* bdst = st + 128 * kBK * 2;
+        if (u.na == 2) {
+          tma_load_2d(bdst, &p.a[u.mat1], kb * kBK, u.row0, &full[s]);
+          bdst += 128 * kBK * 2;
+        }
+        tma_load_2d(bdst, &p.b, kb * kBK, dt.tok0, &full[s]);
+        if (dt.ntok == 256) tma_load_2d(bdst + 128 * kBK * 2, &p.b, kb * kBK, dt.tok0 + 128, &full[s]);
+      }
     }
+    // copies of the last ring positions may still be in flight if a consumer gave up
+    for (int i = max(0, ks - kDenseStages); i < ks; ++i) mbar_drain(&full[i % kDenseStages], (i / kDenseStages) & 1);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer
-    const uint32_t idesc = umma_idesc(kBM, kBN, p.ab_bf16);
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % kDenseStages;
-      if (!mbar_wait(&full[s], (kb / kDenseStages) & 1, &abort_flag, p.err)) break;
+    int ks = 0, li = 0;
+    for (int t = blockIdx.x; t < n_tiles && !abort_flag; t += gridDim.x) {
+      const DenseTile dt = dense_tile(p, t);
+      if (dt.tok0 >= p.T) continue;
+      const DenseUnit u = p.units[dt.unit];
+      const int ab = li & 1;
+      if (li >= 2 && !mbar_wait(&acc_empty[ab], ((li >> 1) - 1) & 1, &abort_flag, p.err)) break;
       tc_fence_after();
-      const uint32_t st = smem_u32(smem + s * stage_bytes);
-#pragma unroll
-      for (int k16 = 0; k16 < kBK / 16; ++k16) {
-        const uint64_t db = umma_desc_sw128(st + 2 * a_bytes + 32 * k16);
-        const uint64_t da0 = umma_desc_sw128(st + 32 * k16);
-        umma_f16(tmem, da0, db, idesc, (kb | k16) != 0);
-        if (na == 2) {
-          const uint64_t da1 = umma_desc_sw128(st + a_bytes + 32 * k16);
-          const uint32_t acc = u.map1 ? tmem + kBN : tmem;
-          umma_f16(acc, da1, db, idesc, u.map1 ? uint32_t((kb | k16) != 0) : 1u);
+      const uint32_t acc = tmem + 256 * ab;
+      const uint32_t idesc = umma_idesc(kBM, dt.ntok, p.ab_bf16);
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb, ++ks) {
+        const int s = ks % kDenseStages;
+        if (!mbar_wait(&full[s], (ks / kDenseStages) & 1, &abort_flag, p.err)) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * kDenseStage);
+        const uint32_t bst = st + u.na * 128 * kBK * 2;
+#pragma unroll
+        for (int k16 = 0; k16 < kBK / 16; ++k16) {
+          const uint64_t db = umma_desc_sw128(bst + 32 * k16);
+          umma_f16(acc, umma_desc_sw128(st + 32 * k16), db, idesc, (kb | k16) != 0);
+          if (u.na == 2) {
+            const uint64_t da1 = umma_desc_sw128(st + 128 * kBK * 2 + 32 * k16);
+            umma_f16(u.map1 ? acc + 128 : acc, da1, db, idesc, u.map1 ? uint32_t((kb | k16) != 0) : 1u);
+          }
+        }
+        umma_commit(&empty[s]);
       }
-      umma_commit(&empty[s]);
+      if (!ok) break;
+      umma_commit(&acc_full[ab]);
+      ++li;
     }
-    umma_commit(&accf);
+    // every MMA issued above has finished before TMEM is released
+    umma_commit(&mma_done);
+    mbar_drain(&mma_done, 0);
   } else if (warp >= 4) {
     // ---------------- epilogue: TMEM lanes 32q..32q+31 = weight rows
     const int q = warp - 4;
-    if (mbar_wait(&accf, 0, &abort_flag, p.err) && !abort_flag) {
+    const int row = q * 32 + lane;
+    int li = 0;
+    // no abort-flag test in the loop condition: the 128 threads leave only together, by the vote
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+      const DenseTile dt = dense_tile(p, t);
+      if (dt.tok0 >= p.T) continue;
+      const DenseUnit u = p.units[dt.unit];
+      const int ab = li & 1;
+      if (!named_bar_and(1, 128, mbar_wait(&acc_full[ab], (li >> 1) & 1, &abort_flag, p.err))) break;
       tc_fence_after();
-      const int row = q * 32 + lane;
       const int grow = u.row0 + row;
       const bool rok = grow < u.nrows;
-      for (int c = 0; c < kBN / 16; ++c) {
+      const uint32_t acc = tmem + 256 * ab + (uint32_t(q * 32) << 16);
+      const int nt = min(dt.ntok, p.T - dt.tok0);
+      for (int c = 0; c * 16 < nt; ++c) {
         float v0[16], v1[16];
-        const uint32_t ta = tmem + (uint32_t(q * 32) << 16) + c * 16;
-        tmem_ld16(ta, v0);
-        if (nacc == 2) tmem_ld16(ta + kBN, v1);
+        if (u.epi == kEpiSwiglu)
+          tmem_ld16x2(acc + c * 16, acc + 128 + c * 16, v0, v1);
+        else
+          tmem_ld16(acc + c * 16, v0);
         if (!rok) continue;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const int t = tok0 + c * 16 + i;
-          if (t >= p.T) break;
+          const int tk = c * 16 + i;
+          if (tk >= nt) break;
+          const int64_t tt = dt.tok0 + tk;
           if (u.epi == kEpiLogits) {
-            p.logits[int64_t(t) * p.ld_logits + u.col0 + grow] = v0[i];
+            p.logits[tt * p.ld_logits + u.col0 + grow] = v0[i];
           } else if (u.epi == kEpiSwiglu) {
-            p.hz[int64_t(t) * p.ld_hz + u.col0 + grow] = __float2half_rn(silu_f(v0[i]) * v1[i]);
+            p.hz[tt * p.ld_hz + u.col0 + grow] = __float2half_rn(silu_f(v0[i]) * v1[i]);
           } else if (u.epi == kEpiPlain) {
-            p.hz[int64_t(t) * p.ld_hz + u.col0 + grow] = __float2half_rn(v0[i]);
+            p.hz[tt * p.ld_hz + u.col0 + grow] = __float2half_rn(v0[i]);
           } else {
-            p.out[int64_t(t) * p.ld_out + u.col0 + grow] = v0[i];
+            p.out[tt * p.ld_out + u.col0 + grow] = v0[i];
           }
         }
       }
+      // accumulator drained: hand it back to the MMA thread
+      tc_fence_before();
+      mbar_arrive(&acc_empty[ab]);
+      ++li;
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, ncols);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -694,13 +762,18 @@ int num_sms() {
   return n;
 }
 
+int dense_grid(const DenseParams& dp) {
+  const int n_tiles = (2 * dp.n_units2 + (dp.n_units - dp.n_units2)) * ((dp.T + 255) / 256);
+  return max(1, min(n_tiles, num_sms()));
+}
+
 size_t tern_smem(int na, int fmt) {
   size_t b;
   if (fmt == SCION_PQ2_0) b = na == 2 ? TernRing<SCION_PQ2_0, 2>::bytes : TernRing<SCION_PQ2_0, 1>::bytes;
   else b = na == 2 ? TernRing<SCION_PTQ1_0, 2>::bytes : TernRing<SCION_PTQ1_0, 1>::bytes;
   return b + 1024;
 }
-constexpr size_t kDenseSmem = kDenseStages * (2 * 128 * 64 * 2 + 128 * 64 * 2) + 1024;
+constexpr size_t kDenseSmem = kDenseStages * kDenseStage + 1024;
 
 }  // namespace
 
@@ -780,6 +853,7 @@ void prefill_units(const scion_layer* L, void* xunits_host, int* n_x, void* duni
   DenseUnit* du = static_cast<DenseUnit*>(dunits_host);
   int nx = 0, nd = 0;
   // A map table: 0 router, 1 delta, 2 sh_gate, 3 sh_up, 4 corr_a, 5 dense_down
+  // the dense kernel expects the two-matrix units first
   if (!L->desc.router_fp32)
     for (int r0 = 0; r0 < L->E; r0 += 128) xu[nx++] = DenseUnit{kEpiLogits, 2, 0, 0, 1, r0, L->E, 0};
   for (int r0 = 0; r0 < L->Fs; r0 += 128) xu[nx++] = DenseUnit{kEpiSwiglu, 2, 1, 2, 3, r0, L->Fs, 0};
@@ -810,10 +884,11 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       memcpy(dp.a, P.maps, sizeof(dp.a));
       if (make_tmap_2d(&dp.b, x, 1, T, L->d) != SCION_OK) return cudaErrorInvalidValue;
       dp.units = static_cast<const DenseUnit*>(P.xunits), dp.K = L->d, dp.T = T, dp.ab_bf16 = 1;
+      dp.n_units = P.n_xunits;
+      dp.n_units2 = (L->desc.router_fp32 ? 0 : (L->E + 127) / 128) + (L->Fs + 127) / 128;
       dp.logits = P.logits, dp.ld_logits = L->E, dp.hz = P.hz, dp.ld_hz = L->Kd, dp.out = nullptr, dp.ld_out = 0;
       dp.err = L->err;
-      dim3 grid(P.n_xunits, (T + kBN - 1) / kBN);
-      dense_gemm_kernel<<<grid, kThreads, kDenseSmem, s>>>(dp);
+      dense_gemm_kernel<<<dense_grid(dp), kThreads, kDenseSmem, s>>>(dp);
       return cudaGetLastError();
     }
     case SCION_STAGE_ROUTE: {
@@ -858,10 +933,10 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       memcpy(dp.a, P.maps, sizeof(dp.a));
       dp.b = P.hz_map;
       dp.units = static_cast<const DenseUnit*>(P.dunits), dp.K = L->Kd, dp.T = T, dp.ab_bf16 = 0;
+      dp.n_units = P.n_dunits, dp.n_units2 = 0;
       dp.logits = nullptr, dp.ld_logits = 0, dp.hz = nullptr, dp.ld_hz = 0, dp.out = out, dp.ld_out = L->d;
       dp.err = L->err;
-      dim3 grid(P.n_dunits, (T + kBN - 1) / kBN);
-      dense_gemm_kernel<<<grid, kThreads, kDenseSmem, s>>>(dp);
+      dense_gemm_kernel<<<dense_grid(dp), kThreads, kDenseSmem, s>>>(dp);
       return cudaGetLastError();
     }
     case SCION_STAGE_DOWN_ROUTED: {
