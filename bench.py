@@ -31,6 +31,20 @@ METRIC = "MoE-layer tokens/s (decode b=1..64, prefill 4K/16K); % HBM or bf16 roo
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def load_traffic(workload, stage):
+    """DRAM bytes per launch of `stage` measured by ncu for `workload` (profiles/dram_traffic.txt),
+    or None when no capture of the current kernel is recorded."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        for line in f:
+            parts = line.split("#", 1)[0].split()
+            if len(parts) == 3 and parts[0] == workload and parts[1] == stage:
+                return float(parts[2])
+    return None
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -370,12 +384,12 @@ def run_gpu(args, rank, world, local_rank):
     if decode:
         achieved = (sbytes[dom] / dom_n) / (dom_ms / dom_n / 1000.0) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                "frac": achieved / peaks["hbm_gbs"], "traffic": load_traffic(cfg.name, dom), "peak_source": peak_src,
                 "bytes_per_launch": sbytes[dom] / dom_n, "us_per_launch": 1000.0 * dom_ms / dom_n}
     else:
         achieved = sflops[dom] / (dom_ms / 1000.0) / 1e12  # the dominant kernel's own FLOPs / its time
         roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": load_traffic(cfg.name, dom),
                 "peak_source": peak_src, "flops_per_launch": sflops[dom] / dom_n,
                 "us_per_launch": 1000.0 * dom_ms / dom_n}
 
