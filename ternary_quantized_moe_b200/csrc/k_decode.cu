@@ -36,8 +36,6 @@ struct XProjArgs {
   const __nv_bfloat16 *w_router, *w_delta, *sh_gate, *sh_up, *corr_a;
   const XUnit* units;
   int n_units, n_chunks;
-  float* partial;
-  unsigned* count;
   float* logits;
   __half* hz;
   __half* xfrag;  // [T][d/128][SCION_BROW] fp16 in fragment order + group sums
@@ -46,9 +44,8 @@ struct XProjArgs {
   float* out;     // zeroed here
 };
 
-// One CTA = (unit, 512-column chunk); 8 warps x 64 columns.  NT = token tiles of 8.  With
-// several chunks, each CTA adds its unit's partial sums into the unit's fp32 accumulation rows
-// (red.add) and the last CTA of the unit to arrive applies the epilogue and clears the rows.
+// One CTA = (unit, 512-column chunk); 8 warps x 64 columns.  NT = token tiles of 8.  The
+// chunks of a unit are one thread-block cluster, reduced through distributed shared memory.
 // kXAux extra CTA columns convert x to the fragment order and clear out and the hidden tails.
 constexpr int kXRow = SCION_XPROJ_KC + 8;  // bf16 elements per staged token row (+16 B pad)
 constexpr int kXAux = 4;
@@ -106,7 +103,6 @@ template <int NT>
 __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
   extern __shared__ __align__(16) uint8_t xsm[];
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(xsm);  // [NT*8][kXRow], then the warp reduction
-  __shared__ int last_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, c = lane & 3;
   const int chunk = blockIdx.y;
@@ -201,8 +197,7 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
       for (int i = 0; i < 4; ++i) red[warp][m][nt][lane][i] = acc[m][nt][i];
   __syncthreads();
 
-  // thread -> (nt, lane) pairs; sum the 8 warps
-  float* accum = a.partial + int64_t(blockIdx.x) * (2 * 16 * SCION_TDEC);  // [m][row][tok]
+  // thread -> (nt, lane) pairs; sum the 8 warps into warp 0's slot
   for (int p = threadIdx.x; p < NT * 32; p += blockDim.x) {
     const int nt = p >> 5, ln = p & 31;
     for (int m = 0; m < nacc; ++m)
@@ -211,49 +206,41 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
         float v = 0.f;
 #pragma unroll
         for (int w = 0; w < 8; ++w) v += red[w][m][nt][ln][i];
-        const int row = (ln >> 2) + 8 * (i >> 1), tok = nt * 8 + 2 * (ln & 3) + (i & 1);
         red[0][m][nt][ln][i] = v;
-        if (a.n_chunks > 1 && tok < a.T) atomicAdd(&accum[(m * 16 + row) * SCION_TDEC + tok], v);
       }
   }
-  if (a.n_chunks > 1) {
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      const unsigned prev = atomicAdd(&a.count[blockIdx.x], 1u);
-      last_flag = (prev == unsigned(a.n_chunks - 1));
-    }
-    __syncthreads();
-    if (!last_flag) return;
-    __threadfence();
-  } else {
-    __syncthreads();
-  }
-
-  // epilogue: thread -> (row, tok); all loads of the thread are issued together
+  // the K chunks of a unit form one thread-block cluster: after a cluster barrier the chunk-0
+  // CTA adds the other chunks' sums straight from their shared memory, then a second barrier
+  // keeps them resident until it has read them
+  cluster_sync();
+  const bool lead = blockIdx.y == 0;
+  // epilogue (chunk 0): thread -> (row, tok); all remote loads of the thread are issued together
   constexpr int kIt = 16 * SCION_TDEC / kXThreads;
   float v[kIt][2];
+  if (lead) {
 #pragma unroll
-  for (int it = 0; it < kIt; ++it) {
-    const int p = threadIdx.x + kXThreads * it;
-    const int row = p / SCION_TDEC, tok = p % SCION_TDEC;
-    v[it][0] = v[it][1] = 0.f;
-    if (tok >= a.T) continue;
-    if (a.n_chunks > 1) {
-      for (int m = 0; m < nacc; ++m) v[it][m] = __ldcg(&accum[(m * 16 + row) * SCION_TDEC + tok]);
-    } else {
+    for (int it = 0; it < kIt; ++it) {
+      const int p = threadIdx.x + kXThreads * it;
+      const int row = p / SCION_TDEC, tok = p % SCION_TDEC;
+      v[it][0] = v[it][1] = 0.f;
+      if (tok >= a.T) continue;
       const int nt = tok >> 3, ln = (row & 7) * 4 + ((tok & 7) >> 1), i = (row >> 3) * 2 + (tok & 1);
-      for (int m = 0; m < nacc; ++m) v[it][m] = red[0][m][nt][ln][i];
+      for (int m = 0; m < nacc; ++m) {
+        const uint32_t off = smem_addr(&red[0][m][nt][ln][i]);
+        float sum = red[0][m][nt][ln][i];
+        for (int ch = 1; ch < a.n_chunks; ++ch) sum += ld_dsmem_f32(map_cluster_rank(off, ch));
+        v[it][m] = sum;
+      }
     }
   }
+  cluster_sync();
+  if (!lead) return;
 #pragma unroll
   for (int it = 0; it < kIt; ++it) {
     const int p = threadIdx.x + kXThreads * it;
     const int row = p / SCION_TDEC, tok = p % SCION_TDEC;
     if (tok >= a.T) continue;
     const int grow = u.row0 + row;
-    if (a.n_chunks > 1)
-      for (int m = 0; m < nacc; ++m) accum[(m * 16 + row) * SCION_TDEC + tok] = 0.f;  // ready for the next call
     if (grow >= nrows) continue;
     if (u.kind == kUnitRouter) {
       a.logits[int64_t(tok) * a.E + grow] = v[it][0];
@@ -263,7 +250,6 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
       a.hz[int64_t(tok) * a.Kd + a.Fs + grow] = __float2half_rn(v[it][0]);
     }
   }
-  if (a.n_chunks > 1 && threadIdx.x == 0) a.count[blockIdx.x] = 0;
 }
 
 // ======================================================================= gate/up
@@ -517,15 +503,17 @@ cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, fl
   a.sh_up = static_cast<const __nv_bfloat16*>(L->desc.sh_up);
   a.corr_a = static_cast<const __nv_bfloat16*>(L->desc.corr_a);
   a.units = L->xunits, a.n_units = L->n_xunits, a.n_chunks = L->n_xchunks;
-  a.partial = L->xpartial, a.count = L->xcount, a.logits = L->logits, a.hz = L->hz, a.xfrag = L->xfrag, a.out = out;
+  a.logits = L->logits, a.hz = L->hz, a.xfrag = L->xfrag, a.out = out;
   a.h = L->h, a.k = L->k, a.GF = L->GF;
   dim3 grid(L->n_xunits + kXAux, L->n_xchunks);
+  const dim3 cluster(1, L->n_xchunks, 1);
   const int nt = (T + 7) / 8;
   switch (nt) {
-    case 1: return launch_pdl(xproj_kernel<1>, grid, dim3(kXThreads), xproj_smem<1>(T), s, a);
-    case 2: return launch_pdl(xproj_kernel<2>, grid, dim3(kXThreads), xproj_smem<2>(T), s, a);
-    case 3: case 4: return launch_pdl(xproj_kernel<4>, grid, dim3(kXThreads), xproj_smem<4>(T), s, a);
-    default: return launch_pdl(xproj_kernel<8>, grid, dim3(kXThreads), xproj_smem<8>(T), s, a);
+    case 1: return launch_pdl_cluster(xproj_kernel<1>, grid, dim3(kXThreads), cluster, xproj_smem<1>(T), s, a);
+    case 2: return launch_pdl_cluster(xproj_kernel<2>, grid, dim3(kXThreads), cluster, xproj_smem<2>(T), s, a);
+    case 3: case 4:
+      return launch_pdl_cluster(xproj_kernel<4>, grid, dim3(kXThreads), cluster, xproj_smem<4>(T), s, a);
+    default: return launch_pdl_cluster(xproj_kernel<8>, grid, dim3(kXThreads), cluster, xproj_smem<8>(T), s, a);
   }
   return cudaGetLastError();
 }

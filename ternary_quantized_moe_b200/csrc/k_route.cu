@@ -175,43 +175,44 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
 }
 
 // ---------------------------------------------------------------- decode route
-// One pass of T <= SCION_TDEC tokens (E <= 512): one warp per token selects the top k and the
-// gates (ceil(T/4) CTAs of 4 warps), then the last CTA to finish stages the T*k (id, gate)
-// entries in shared memory with one sweep and groups them there: histogram, exclusive scan,
-// active-expert list with the per-slot records, and the stable scatter in (token, slot) order.
-constexpr int kRcThreads = 128;
+// One CTA for one pass of T <= SCION_TDEC tokens (E <= 512), everything between the logits
+// and the outputs in shared memory: warp w selects the top k and the gates of tokens w,
+// w + 32, ..., then the CTA groups the T*k entries -- histogram, exclusive scan, active-expert
+// list with the per-slot records, and the stable scatter in (token, slot) order.
+// 1024 threads (one warp per token up to 32 tokens); 512 when each lane holds 16 logits, to
+// keep the sorted lane lists in registers.
+template <int VPL>
+constexpr int rc_threads() {
+  return VPL >= 16 ? 512 : 1024;
+}
 
 template <int VPL>
-__global__ void __launch_bounds__(kRcThreads) route_cta_kernel(
+__global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
     const float* __restrict__ logits, int T, int E, int k, int norm_topk, int32_t* __restrict__ ids,
     float* __restrict__ gates, int32_t* __restrict__ counts_out, int32_t* __restrict__ offsets_out,
     int32_t* __restrict__ perm_out, float* __restrict__ gperm_out, int32_t* __restrict__ active_out,
-    int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info, unsigned* __restrict__ done) {
+    int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info) {
   extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [E] | cursor [E]
-  __shared__ int last;
   const int n = T * k;
   int32_t* ids_s = reinterpret_cast<int32_t*>(rs);
   float* gates_s = rs + n;
   int32_t* counts = reinterpret_cast<int32_t*>(rs + 2 * n);
   int32_t* cursor = counts + E;
+  constexpr int kRcThreads = rc_threads<VPL>();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (kRcThreads / 32) + warp;
   pdl_trigger();
-  pdl_wait();
-  if (t < T) warp_topk<VPL>(logits + int64_t(t) * E, E, k, norm_topk, lane, ids + t * k, gates + t * k);
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) last = (atomicAdd(done, 1u) == gridDim.x - 1);
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
   for (int e = threadIdx.x; e < E; e += kRcThreads) counts[e] = 0;
-  for (int i = threadIdx.x; i < n; i += kRcThreads) ids_s[i] = __ldcg(&ids[i]), gates_s[i] = __ldcg(&gates[i]);
+  pdl_wait();
+  for (int t = warp; t < T; t += kRcThreads / 32)
+    warp_topk<VPL>(logits + int64_t(t) * E, E, k, norm_topk, lane, ids_s + t * k, gates_s + t * k);
   __syncthreads();
-  for (int i = threadIdx.x; i < n; i += kRcThreads) atomicAdd(&counts[ids_s[i]], 1);
+  for (int i = threadIdx.x; i < n; i += kRcThreads) {
+    ids[i] = ids_s[i];
+    gates[i] = gates_s[i];
+    atomicAdd(&counts[ids_s[i]], 1);
+  }
   __syncthreads();
   if (warp != 0) return;
-  if (lane == 0) *done = 0;
   // ---- exclusive scan of the counts, active list and slot records (warp 0)
   const int per = (E + 31) / 32;
   const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
@@ -270,9 +271,9 @@ cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s) {
   if (L->E <= 512) {
     const size_t smem = route_cta_smem(T, L->E, L->k);
 #define SCION_ROUTE_CTA(V)                                                                                     \
-  return launch_pdl(route_cta_kernel<V>, dim3((T + 3) / 4), dim3(kRcThreads), smem, s, L->logits, T, L->E,   \
-                    L->k, L->desc.norm_topk, L->ids, L->gates, L->counts, L->offsets, L->perm, L->gperm,       \
-                    L->active, L->n_active, reinterpret_cast<int4*>(L->slot_info), L->route_done)
+  return launch_pdl(route_cta_kernel<V>, dim3(1), dim3(rc_threads<V>()), smem, s, L->logits, T, L->E, L->k,\
+                    L->desc.norm_topk, L->ids, L->gates, L->counts, L->offsets, L->perm, L->gperm, L->active, \
+                    L->n_active, reinterpret_cast<int4*>(L->slot_info))
     const int vpl = (L->E + 31) / 32;
     if (vpl <= 1) SCION_ROUTE_CTA(1);
     else if (vpl <= 2) SCION_ROUTE_CTA(2);

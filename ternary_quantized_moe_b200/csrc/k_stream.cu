@@ -194,14 +194,18 @@ __device__ __forceinline__ void stage_groups(uint32_t stg, const LaneOffs& o, in
         acc[m][3] = fmaf(sf.y, g[j][m][3], acc[m][3]);
       }
   } else {
+    // all code words of the stage's tiles first, then the digit chains and MMAs
+    TileRegs<SCION_PTQ1_0> t[J][NMAT];
 #pragma unroll
     for (int j = 0; j < J; ++j)
 #pragma unroll
       for (int m = 0; m < NMAT; ++m) {
-        TileRegs<FMT> t;
-        t.load_shared(stg + (j0 + j) * cb + m * 8 * tb + o.code - 16 * lane, lane);
-        tile_mma<FMT>(t, b[j], acc[m], c);
+        t[j][m].load_shared(stg + (j0 + j) * cb + m * 8 * tb + o.code - 16 * lane, lane);
       }
+#pragma unroll
+    for (int j = 0; j < J; ++j)
+#pragma unroll
+      for (int m = 0; m < NMAT; ++m) tile_mma_ptq1_nv(t[j][m], b[j], acc[m], c);
   }
 }
 

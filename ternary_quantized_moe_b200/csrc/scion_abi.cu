@@ -44,8 +44,8 @@ void free_layer(scion_layer* L) {
   if (!L) return;
   void* ptrs[] = {L->gu_bank, L->dn_bank,  L->dense_down, L->xunits,  L->logits,    L->ids,       L->gates,
                   L->counts,  L->offsets,  L->perm,       L->active,  L->n_active,  L->h,         L->hz,
-                  L->xfrag,   L->xpartial, L->xcount,     L->x_stage, L->out_stage, L->bad,       L->err,
-                  L->slot_info, L->gperm, L->route_done};
+                  L->xfrag,   L->x_stage, L->out_stage, L->bad,       L->err,
+                  L->slot_info, L->gperm};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   if (L->pre) {
@@ -114,6 +114,8 @@ int create_prefill(scion_layer* L, cudaStream_t s) {
 int check_desc(const scion_layer_desc* D, int max_tokens) {
   if (!D || max_tokens < 1) return SCION_EINVAL;
   if (D->d <= 0 || D->d % 128 || D->ffn <= 0 || D->ffn % 128) return SCION_EINVAL;
+  // the decode x-projection reduces its 512-column chunks inside one thread-block cluster (<= 8)
+  if (D->d > 8 * SCION_XPROJ_KC) return SCION_EINVAL;
   if (D->n_experts < 1 || D->n_experts > 4096 || D->top_k < 1 || D->top_k > D->n_experts || D->top_k > 32)
     return SCION_EINVAL;
   if (D->shared_ffn < 0 || D->shared_ffn % 128 || D->rank < 0 || D->rank % 16) return SCION_EINVAL;
@@ -260,14 +262,9 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   SCION_TRY(dev_alloc(L, &L->active, sizeof(int32_t) * L->E));
   SCION_TRY(dev_alloc(L, &L->n_active, sizeof(int32_t)));
   SCION_TRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&L->slot_info), sizeof(int4) * L->E));
-  SCION_TRY(dev_alloc(L, &L->route_done, sizeof(unsigned)));
-  SCION_TRY(cudaMemsetAsync(L->route_done, 0, sizeof(unsigned), s));
   SCION_TRY(dev_alloc(L, &L->h, sizeof(__half) * TD * L->k * L->GF * SCION_BROW));
   SCION_TRY(dev_alloc(L, &L->hz, sizeof(__half) * TD * (L->Kd ? L->Kd : 1)));
   SCION_TRY(dev_alloc(L, &L->xfrag, sizeof(__half) * TD * L->Gd * SCION_BROW));
-  SCION_TRY(dev_alloc(L, &L->xpartial, sizeof(float) * (L->n_xunits ? L->n_xunits : 1) * 2 * 16 * TD));
-  SCION_TRY(cudaMemsetAsync(L->xpartial, 0, sizeof(float) * (L->n_xunits ? L->n_xunits : 1) * 2 * 16 * TD, s));
-  SCION_TRY(dev_alloc(L, &L->xcount, sizeof(unsigned) * (L->n_xunits ? L->n_xunits : 1)));
   SCION_TRY(dev_alloc(L, &L->x_stage, sizeof(__nv_bfloat16) * size_t(max_tokens) * L->d));
   SCION_TRY(dev_alloc(L, &L->out_stage, sizeof(float) * size_t(max_tokens) * L->d));
   SCION_TRY(dev_alloc(L, &L->bad, sizeof(int64_t)));
@@ -276,7 +273,6 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
 
   if (!units.empty())
     SCION_TRY(cudaMemcpyAsync(L->xunits, units.data(), sizeof(scion::XUnit) * units.size(), cudaMemcpyHostToDevice, s));
-  SCION_TRY(cudaMemsetAsync(L->xcount, 0, sizeof(unsigned) * (L->n_xunits ? L->n_xunits : 1), s));
   SCION_TRY(cudaMemsetAsync(L->hz, 0, sizeof(__half) * TD * (L->Kd ? L->Kd : 1), s));
   SCION_TRY(cudaMemsetAsync(L->bad, 0, sizeof(int64_t), s));
   if (L->Kd) {

@@ -108,12 +108,9 @@ struct scion_layer {
   int32_t* active;   // [E]
   int32_t* n_active; // [1]
   void* slot_info;    // int4 [E]: {expert, first position, token count, 0} per active slot
-  unsigned* route_done;  // [1] arrival counter of the decode route kernel (zero between calls)
   __half* h;         // [TDEC*k][GF][SCION_BROW] fragment order + group-sum tails
   __half* hz;        // [TDEC][Kd] (pad columns stay 0)
   __half* xfrag;     // [TDEC][Gd][SCION_BROW] x in fragment order (fp16) + group-sum tails
-  float* xpartial;   // [n_xunits][2][16][TDEC] x-projection accumulation rows (zero between calls)
-  unsigned* xcount;  // [n_xunits]
   void* x_stage;     // [max_tokens][d] bf16 (host-buffer forward)
   float* out_stage;  // [max_tokens][d]
   int64_t* bad;      // [1] invalid-code counter used at create
@@ -188,6 +185,27 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Same with a thread-block cluster of `cluster` CTAs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, dim3 cluster, size_t smem,
+                               cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster.x;
+  attr[1].val.clusterDim.y = cluster.y;
+  attr[1].val.clusterDim.z = cluster.z;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ------------------------------------------------------------ device helpers
 // Wait until the preceding grid on the stream has completed and its writes are visible.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -215,6 +233,24 @@ __device__ __forceinline__ void mma_f16_1688(float (&d)[4], uint32_t a0, uint32_
       "mma.sync.aligned.m16n8k8.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};\n"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(b0));
+}
+
+// Thread-block cluster: full barrier of all threads of the cluster (release / acquire), the
+// shared-window address of a variable, its address in the CTA of cluster rank `rank`, and a
+// load through that address.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t smem_addr(const void* p) { return uint32_t(__cvta_generic_to_shared(p)); }
+__device__ __forceinline__ uint32_t map_cluster_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {

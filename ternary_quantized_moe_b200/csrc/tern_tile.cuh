@@ -188,6 +188,51 @@ __device__ __forceinline__ uint32_t ptq1_rem_slot(uint32_t qt, int c) {
   return r;
 }
 
+// Same as ptq1_rem_slot without a branch on c (the four lane-columns pick their pair by selects).
+__device__ __forceinline__ uint32_t ptq1_rem_slot_nb(uint32_t qt, int c) {
+  uint32_t pr;
+  asm("prmt.b32 %0, %1, 0, 0x4140;" : "=r"(pr) : "r"(qt));
+  Ptq1Digits d{u32_as_h2(pr | kMagic)};
+  const uint32_t p0 = d.next(), p1 = d.next(), p2 = d.next(), p3 = d.next(), p4 = d.next();
+  const uint32_t a = c == 0 ? p0 : c == 1 ? p2 : c == 2 ? p4 : p1;
+  const uint32_t b = c == 0 ? p1 : c == 1 ? p3 : c == 2 ? p0 : p2;
+  const uint32_t sel = c < 2 ? 0x5410u : (c == 2 ? 0x7610u : 0x7632u);
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// PTQ1_0 tile for the ring kernels: the digit chains, then eight MMAs issued without `volatile`
+// (independent tiles of a stage can interleave), no branch on the lane-column.
+__device__ __forceinline__ void tile_mma_ptq1_nv(const TileRegs<SCION_PTQ1_0>& t, const uint32_t (&b)[16],
+                                                 float (&acc)[4], int c) {
+  const uint32_t sel_r[3] = {0x0300u, 0x0401u, 0x0502u};
+  const uint32_t sel_h[3] = {0x0502u, 0x0603u, 0x0704u};
+  uint32_t ar[16], ah[16];
+#pragma unroll
+  for (int m = 0; m < 3; ++m) {
+    Ptq1Digits dr{ptq1_v0(t.q0, t.q1, sel_r[m])}, dh{ptq1_v0(t.q1, t.q2, sel_h[m])};
+#pragma unroll
+    for (int j = 0; j < 5; ++j) ar[5 * m + j] = dr.next(), ah[5 * m + j] = dh.next();
+  }
+  ar[15] = ptq1_rem_slot_nb(t.rem & 0xffffu, c);
+  ah[15] = ptq1_rem_slot_nb(t.rem >> 16, c);
+  float g[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int s2 = 0; s2 < 8; ++s2) {
+    const uint32_t fa[4] = {ar[2 * s2], ah[2 * s2], ar[2 * s2 + 1], ah[2 * s2 + 1]};
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(g[0]), "+f"(g[1]), "+f"(g[2]), "+f"(g[3])
+        : "r"(fa[0]), "r"(fa[1]), "r"(fa[2]), "r"(fa[3]), "r"(b[2 * s2]), "r"(b[2 * s2 + 1]));
+  }
+  const float2 sf = __half22float2(u32_as_h2(t.sc));
+  acc[0] = fmaf(sf.x, g[0], acc[0]);
+  acc[1] = fmaf(sf.x, g[1], acc[1]);
+  acc[2] = fmaf(sf.y, g[2], acc[2]);
+  acc[3] = fmaf(sf.y, g[3], acc[3]);
+}
+
 // acc += scale_row * (codes . B) for one loaded tile and one token tile of 8.
 // b: the lane's 64 bytes of the group (16 u32) in fragment order.
 template <int FMT>
