@@ -56,8 +56,17 @@ __device__ __forceinline__ int perm_pos(int fmt, int col) {  // physical column 
   return g | (64 * half + 10 * i + 2 * j + u);
 }
 
-// x (bf16) -> fp16 in the container's column order; one thread per 16 columns (PQ2_0) or
-// per 128-column group (PTQ1_0).
+// PQ2_0 B-operand factor of position p: positions (2s, 2s+1) of every 16 hold the pair of
+// columns (s, s + 8) that the expansion builds with the field at bits 2f..2f+1 of a 16-bit code
+// half (f = s < 5 ? s : s - 5), i.e. scaled by 4^f; the B operands (x and h) carry 4^-f, an exact
+// power-of-two scaling.
+__device__ __forceinline__ float pq2_pos_scale(int p) {
+  const int s = (p & 15) >> 1;
+  return 1.0f / float(1 << (2 * (s < 5 ? s : s - 5)));
+}
+
+// x (bf16) -> fp16 in the container's column order (PQ2_0: times the factor of its position);
+// one thread per 16 columns (PQ2_0) or per 128-column group (PTQ1_0).
 template <int FMT>
 __global__ void x16_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, __half* __restrict__ xp) {
   constexpr int W = FMT == SCION_PQ2_0 ? 16 : 128;
@@ -70,7 +79,11 @@ __global__ void x16_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, __hal
 #pragma unroll
   for (int j = 0; j < W / 8; ++j) reinterpret_cast<uint4*>(in)[j] = src[j];
 #pragma unroll
-  for (int col = 0; col < W; ++col) outv[perm_pos(FMT, col) & (W - 1)] = __float2half_rn(__bfloat162float(in[col]));
+  for (int col = 0; col < W; ++col) {
+    const int p = perm_pos(FMT, col) & (W - 1);
+    const float v = __bfloat162float(in[col]);
+    outv[p] = __float2half_rn(FMT == SCION_PQ2_0 ? v * pq2_pos_scale(p) : v);
+  }
 #pragma unroll
   for (int j = 0; j < W / 8; ++j) dst[j] = reinterpret_cast<uint4*>(outv)[j];
 }
@@ -315,18 +328,25 @@ __device__ __forceinline__ void expand_pq2_half(uint32_t codes, int t, int h, ui
   const uint32_t blk = codes + (t >> 4) * kPq2Tile;
   const int rho = t & 15, r8 = rho & 7, hi = rho >> 3;
   const __half2 sc = __half2half2(__ushort_as_half(uint16_t(lds_u16(blk + 512 + 4 * r8 + 2 * hi))));
-  const __half2 bias = u32_as_h2(0x64016401u);
 #pragma unroll
   for (int cc = 0; cc < 2; ++cc) {
     const int c = 2 * h + cc;  // container code bytes 8c .. 8c+7 = words 2c, 2c+1
     const uint2 w2 = lds_v2(blk + 16 * (4 * r8 + c) + 8 * hi);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-      const uint32_t w = half ? w2.y : w2.x;
+      const uint32_t w = half ? w2.y : w2.x, w10 = w >> 10;
+      // pair s = columns (s, s + 8): the field at bits 2f..2f+1 of each 16-bit half (f = s, or
+      // s - 5 in w >> 10) ORed into 1024 is 1024 + 4^f b; minus 1024 + 4^f, times the scale, is
+      // 4^f * code * scale exactly (the 4^f is divided out of B)
       uint32_t v[8];
 #pragma unroll
-      for (int s = 0; s < 8; ++s)
-        v[s] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(w >> (2 * s), 0x00030003u, 0x64006400u)), bias), sc));
+      for (int s = 0; s < 8; ++s) {
+        const int f = s < 5 ? s : s - 5;
+        const uint32_t bias = 0x6400u + (1u << (2 * f));
+        v[s] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(s < 5 ? w : w10, 0x00030003u << (2 * f), 0x64006400u)),
+                                         u32_as_h2(bias | (bias << 16))),
+                                 sc));
+      }
       const int j0 = 2 * (2 * cc + half);  // 8-position chunk index inside the half
 #pragma unroll
       for (int i = 0; i < 8; ++i) out[4 * j0 + i] = v[i];
@@ -593,6 +613,7 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
     const int q = warp & 3;
     const int row = q * 32 + lane;
     const int pcol = perm_pos(FMT, row);  // gate/up: position of this row inside its 128-column group of h
+    const float hscale = FMT == SCION_PQ2_0 ? pq2_pos_scale(pcol) : 1.0f;
     int li = 0;
     // no abort-flag test in the loop condition: the 128 threads leave only together, by the vote
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++li) {
@@ -615,7 +636,7 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
           __half* dst = p.h + (pos0 + n0) * p.F + int64_t(rt) * kBM + pcol;
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            if (n0 + i < nn) dst[int64_t(i) * p.F] = __float2half_rn(silu_f(v0[i]) * v1[i]);
+            if (n0 + i < nn) dst[int64_t(i) * p.F] = __float2half_rn(silu_f(v0[i]) * v1[i] * hscale);
         } else {
           float* dst = p.y + (pos0 + n0) * p.d + int64_t(rt) * kBM + row;
 #pragma unroll
@@ -835,7 +856,9 @@ __global__ void unperm_prefill_kernel(int fmt, const __half* __restrict__ src, i
   int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const int64_t base = i & ~int64_t(127);
-  dst[i] = src[base + perm_pos(fmt, int(i & 127))];
+  const int p = perm_pos(fmt, int(i & 127));
+  const float v = __half2float(src[base + p]);
+  dst[i] = __float2half_rn(fmt == SCION_PQ2_0 ? v / pq2_pos_scale(p) : v);
 }
 
 cudaError_t launch_unperm_prefill(int fmt, const __half* src, int64_t n, __half* dst, cudaStream_t s) {
