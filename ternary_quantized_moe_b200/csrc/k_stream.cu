@@ -209,11 +209,10 @@ __device__ __forceinline__ void stage_groups(uint32_t stg, const LaneOffs& o, in
   }
 }
 
-// Persistent: CTA b walks the items b, b + gridDim.x, ... with item = (active slot, 128-row
+// Persistent: CTA b walks a contiguous range of the items, item = (active slot, 128-row
 // block).  One producer warp streams, per stage, GPS groups of the item's codes and the
 // fragment-ordered B rows of up to kTok tokens into a ring of stages, each with a header that
-// tells the consumers what it holds; routing records are fetched one (tokens) and two (slot)
-// items ahead, so no pointer chase sits between two items.
+// tells the consumers what it holds.
 template <int FMT, int NMAT>
 __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __grid_constant__ StreamArgs a) {
   extern __shared__ __align__(128) uint8_t ring[];
@@ -248,13 +247,23 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
       }
       return t;
     };
-    int4 si_cur = slot_rec(blockIdx.x), si_nxt = slot_rec(blockIdx.x + gridDim.x);
+    // this CTA's items are a contiguous range, so consecutive items mostly share their slot and
+    // its token records (loaded again only when the slot changes); the next slot's record is
+    // fetched one slot ahead
+    const int i0 = int(int64_t(n_items) * blockIdx.x / gridDim.x);
+    const int i1 = int(int64_t(n_items) * (blockIdx.x + 1) / gridDim.x);
+    int cur_slot = i0 / RB;
+    int4 si_cur = slot_rec(i0), si_nxt = slot_rec((cur_slot + 1) * RB);
     TokInfo tk_cur = tok_info(si_cur, 0);
     int st = 0;  // running stage counter
     bool ok = true;
-    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-      const int4 si_n2 = slot_rec(item + 2 * gridDim.x);
-      const TokInfo tk_nxt = tok_info(si_nxt, 0);
+    for (int item = i0; item < i1 && ok; ++item) {
+      if (item / RB != cur_slot) {
+        cur_slot = item / RB;
+        si_cur = si_nxt;
+        si_nxt = slot_rec((cur_slot + 1) * RB);
+        tk_cur = tok_info(si_cur, 0);
+      }
       const int rb = item % RB;
       const uint8_t* src0 = a.bank + (int64_t(si_cur.x) * RB + rb) * a.G * cb;
       for (int pc = 0; pc < si_cur.z && ok; pc += kTok) {
@@ -292,7 +301,6 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
                       a.bsrc + (int64_t(tk.brow) * a.bld + g0) * SCION_BROW, ng * kRowB, &full[s]);
         }
       }
-      si_cur = si_nxt, si_nxt = si_n2, tk_cur = tk_nxt;
     }
     if (lane == 0) {
       if (ok) {
@@ -347,17 +355,10 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[m][i] = 0.f;
     }
+    // one group at a time (taking two per call measured slower: more registers, less overlap)
 #pragma unroll
-    for (int j0 = 0; j0 < GPS; j0 += 2) {
-      // PQ2_0 takes groups in pairs (more independent MMA chains); the PTQ1_0 digit chains
-      // already need most of the registers, so it takes them one at a time
-      if (FMT == SCION_PQ2_0 && j0 + 1 < ng) {
-        stage_groups<FMT, NMAT, 2>(stg, lo, j0, nn, lane, acc);
-      } else {
-        if (j0 < ng) stage_groups<FMT, NMAT, 1>(stg, lo, j0, nn, lane, acc);
-        if (j0 + 1 < ng) stage_groups<FMT, NMAT, 1>(stg, lo, j0 + 1, nn, lane, acc);
-      }
-    }
+    for (int j = 0; j < GPS; ++j)
+      if (j < ng) stage_groups<FMT, NMAT, 1>(stg, lo, j, nn, lane, acc);
     if (flags & 2) {
       // epilogue: this warp's 16 rows x the pass's tokens
       const int rb = hd->rb;
