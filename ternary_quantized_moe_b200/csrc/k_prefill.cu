@@ -315,7 +315,7 @@ struct TernParams {
   const float* gates;
   int k;
   __half* h;  int F;     // gate/up output
-  float* y;   int d;     // down output: one row per routed (token, slot), [T*k][d], gates applied by the combine
+  __half* y;  int d;     // down output: one fp16 row per routed (token, slot), [T*k][d], gates applied by the combine
   int* err;
 };
 
@@ -638,10 +638,10 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
           for (int i = 0; i < 16; ++i)
             if (n0 + i < nn) dst[int64_t(i) * p.F] = __float2half_rn(silu_f(v0[i]) * v1[i] * hscale);
         } else {
-          float* dst = p.y + (pos0 + n0) * p.d + int64_t(rt) * kBM + row;
+          __half* dst = p.y + (pos0 + n0) * p.d + int64_t(rt) * kBM + row;
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            if (n0 + i < nn) dst[int64_t(i) * p.d] = v0[i];
+            if (n0 + i < nn) dst[int64_t(i) * p.d] = __float2half_rn(v0[i]);
         }
       }
       // accumulator drained: hand it back to the MMA warp
@@ -834,7 +834,7 @@ cudaError_t configure_prefill_kernels() {
 
 // out[t] (= dense part, or 0 when the layer has no shared expert and no correction)
 // += sum over slots j < k of y[inv[t*k + j]], in slot order.  One CTA per token.
-__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ y, const int32_t* __restrict__ inv,
+__global__ void __launch_bounds__(256) combine_kernel(const __half* __restrict__ y, const int32_t* __restrict__ inv,
                                                      const float* __restrict__ gates, int k, int d, int has_dense,
                                                      float* __restrict__ out) {
   const int t = blockIdx.x;
@@ -844,7 +844,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
   for (int c4 = threadIdx.x; c4 < d / 4; c4 += blockDim.x) {
     float4 acc = has_dense ? o[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < k; ++j) {
-      const float4 v = reinterpret_cast<const float4*>(y + int64_t(iv[j]) * d)[c4];
+      const uint2 raw = reinterpret_cast<const uint2*>(y + int64_t(iv[j]) * d)[c4];
+      const float2 lo = __half22float2(u32_as_h2(raw.x)), hi = __half22float2(u32_as_h2(raw.y));
+      const float4 v = make_float4(lo.x, lo.y, hi.x, hi.y);
       const float g = gt[j];
       acc.x += g * v.x, acc.y += g * v.y, acc.z += g * v.z, acc.w += g * v.w;
     }

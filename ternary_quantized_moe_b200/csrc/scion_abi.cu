@@ -78,7 +78,7 @@ int create_prefill(scion_layer* L, cudaStream_t s) {
   PTRY(dev_alloc(L, &P->offsets, sizeof(int32_t) * (L->E + 1)));
   PTRY(dev_alloc(L, &P->perm, sizeof(int32_t) * Tk));
   PTRY(dev_alloc(L, &P->inv, sizeof(int32_t) * Tk));
-  PTRY(dev_alloc(L, &P->y, sizeof(float) * Tk * L->d));
+  PTRY(dev_alloc(L, &P->y, sizeof(__half) * Tk * L->d));
   PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->tiles), scion::prefill_tile_bytes() * max_tiles));
   PTRY(dev_alloc(L, &P->n_tiles, sizeof(int32_t)));
   PTRY(dev_alloc(L, &P->x16, sizeof(__half) * T * L->d));

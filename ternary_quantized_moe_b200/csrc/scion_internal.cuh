@@ -74,7 +74,7 @@ struct PrefillState {
   int32_t* offsets;     // [E+1]
   int32_t* perm;        // [maxT*k]
   int32_t* inv;         // [maxT*k] position of entry t*k+j in perm
-  float* y;             // [maxT*k][d] expert down outputs (gate not yet applied), one row per routed (token, slot)
+  __half* y;            // [maxT*k][d] expert down outputs in fp16 (gate not yet applied), one row per routed entry
   void* tiles;          // 128-token tiles, [maxT*k/128 + E]
   int32_t* n_tiles;
   __half* x16;          // [maxT][d]   x in the container column order (fp16)
