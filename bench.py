@@ -111,6 +111,25 @@ def workload_flops(cfg, T):
                     + 2 * cfg.rank * cfg.d)
 
 
+# ------------------------------------------------------------------- ranks
+def max_over_ranks(v, world, device):
+    """Maximum of a per-rank float over the process group (the job's time is its slowest rank)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(world, tokens_per_step, steps, ms_max):
+    """Whole-job throughput: every rank runs its own replica (weak scaling) on the same schedule,
+    so the job processes world x tokens_per_step x steps tokens in the slowest rank's time."""
+    return world * tokens_per_step * steps / (ms_max / 1000.0)
+
+
 # ------------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock and throttle reasons of one GPU through NVML (read-only)."""
@@ -296,12 +315,6 @@ def run_gpu(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     def timed(fn, K):
         barrier()
@@ -313,7 +326,7 @@ def run_gpu(args, rank, world, local_rank):
         e1.synchronize()
         ms = e0.elapsed_time(e1)
         barrier()
-        return max_over_ranks(ms)
+        return max_over_ranks(ms, world, dev)
 
     for s in range(args.warmup):
         step(s)
@@ -325,7 +338,7 @@ def run_gpu(args, rank, world, local_rank):
         ms = timed(step, K)
     launches = tq.scion_kernel_launches() - launches0
     tokens_per_step = sum(batches)
-    value = world * tokens_per_step * K / (ms / 1000.0)
+    value = job_tokens_per_s(world, tokens_per_step, K, ms)
 
     # ---- per-kernel device time (CUDA events around every launch, same schedule)
     barrier()
@@ -361,7 +374,7 @@ def run_gpu(args, rank, world, local_rank):
             tq.scion_moe_forward(xs[T], T, layers[s % n_layers], outs[T], stream)
         msT = timed(one, K)
         bT = sum(workload_bytes(cfg, T, U[(s % n_layers, T)]) for s in range(K))
-        per_batch[str(T)] = {"tokens_per_s": world * T * K / (msT / 1000.0), "us_per_call": 1000.0 * msT / K,
+        per_batch[str(T)] = {"tokens_per_s": job_tokens_per_s(world, T, K, msT), "us_per_call": 1000.0 * msT / K,
                              "hbm_frac": (bT / (msT / 1000.0)) / (peaks["hbm_gbs"] * 1e9)}
 
     # ---- end to end through the host-buffer entry point (pinned host x in, out back to host)
@@ -373,7 +386,7 @@ def run_gpu(args, rank, world, local_rank):
             tq.scion_moe_forward_host(xh[T], T, layers[(s * nb + i) % n_layers], oh[T], stream)
 
     ms_e2e = timed(step_host, K)
-    e2e = {"value": world * tokens_per_step * K / (ms_e2e / 1000.0), "unit": "tokens/s",
+    e2e = {"value": job_tokens_per_s(world, tokens_per_step, K, ms_e2e), "unit": "tokens/s",
            "h2d_bytes_per_step": sum(T * cfg.d * 2 for T in batches),
            "d2h_bytes_per_step": sum(T * cfg.d * 4 for T in batches)}
 
