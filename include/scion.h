@@ -136,7 +136,9 @@ typedef struct scion_layer scion_layer;
  * corr_b; w_router, w_router_delta, sh_gate, sh_up, sh_gate_vec and corr_a are
  * read in place and must outlive the handle.  Synchronises `stream` once to
  * validate every code: SCION_EFORMAT if a block holds an invalid code (no
- * handle is returned), EINVAL on a bad descriptor, ENOMEM, ECUDA. */
+ * handle is returned), EINVAL on a bad descriptor, ENOMEM, ECUDA.  Descriptor
+ * limits: d and ffn multiples of 128 with d <= 4096, shared_ffn a multiple of 128,
+ * rank a multiple of 16, 1 <= top_k <= min(E, 32), E <= 4096. */
 int scion_layer_create(const scion_layer_desc* desc, int max_tokens, void* stream, scion_layer** out);
 
 /* Frees the handle and everything it allocated (synchronises the device). */

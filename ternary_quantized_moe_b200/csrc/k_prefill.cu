@@ -10,8 +10,8 @@
 //   dense     tcgen05 GEMM with both operands loaded by TMA (128B swizzle):
 //               x-projection  router + delta -> logits; shared gate/up -> SwiGLU; corr A -> z
 //               dense down    [shared down | correction B] x [h_s | z] -> out (store)
-//   route     top-k per token (warp per token), then one CTA groups the T*k entries by
-//             expert (histogram, scan, stable scatter) and lists 128-token tiles
+//   route     top-k per token (warp per token) with a histogram of the selections, one CTA
+//             scans it and lists the 128-token tiles, one thread per entry takes its position
 //   ternary   tcgen05 grouped GEMM over the routed tiles: packed code blocks arrive by
 //             bulk copy, four warps expand them to fp16 (code * scale, exact) in the
 //             swizzled layout, gathered token rows arrive by cp.async:
@@ -661,96 +661,75 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
 // One warp per token (8 per CTA), logits in registers.
 template <int VPL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
-                                                   int norm_topk, int32_t* __restrict__ ids, float* __restrict__ gates) {
+                                                   int norm_topk, int32_t* __restrict__ ids, float* __restrict__ gates,
+                                                   int32_t* __restrict__ counts) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + warp;
-  if (t < T) warp_topk<VPL>(logits + int64_t(t) * E, E, k, norm_topk, lane, ids + int64_t(t) * k, gates + int64_t(t) * k);
+  if (t >= T) return;
+  warp_topk<VPL>(logits + int64_t(t) * E, E, k, norm_topk, lane, ids + int64_t(t) * k, gates + int64_t(t) * k);
+  if (lane < k) atomicAdd(&counts[ids[int64_t(t) * k + lane]], 1);  // histogram of the selections
 }
 
-constexpr int kGroupWarps = 16;
+// Grouping by expert.  The order of the tokens inside an expert's segment is free (each token
+// column of the grouped GEMMs is computed independently, and the combine sums a token's k rows
+// in slot order), so the scatter takes positions with one atomic per entry.
+//
+// One CTA: exclusive scan of the histogram, the per-expert cursors, and the 128-token tiles.
+constexpr int kScanThreads = 1024;
+__global__ void __launch_bounds__(kScanThreads) group_scan_kernel(const int32_t* __restrict__ counts, int E,
+                                                                  int32_t* __restrict__ offsets,
+                                                                  int32_t* __restrict__ cursor,
+                                                                  TernTile* __restrict__ tiles,
+                                                                  int32_t* __restrict__ n_tiles) {
+  __shared__ int32_t wsum[kScanThreads / 32], wtile[kScanThreads / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per = (E + kScanThreads - 1) / kScanThreads;  // experts per thread, contiguous
+  const int e0 = min(E, threadIdx.x * per), e1 = min(E, e0 + per);
+  int cs = 0, ts = 0;
+  for (int e = e0; e < e1; ++e) {
+    const int c = counts[e];
+    cs += c, ts += (c + kBN - 1) / kBN;
+  }
+  // block-wide exclusive scan of (cs, ts)
+  int ic = cs, it = ts;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int c2 = __shfl_up_sync(0xffffffffu, ic, o), t2 = __shfl_up_sync(0xffffffffu, it, o);
+    if (lane >= o) ic += c2, it += t2;
+  }
+  if (lane == 31) wsum[warp] = ic, wtile[warp] = it;
+  __syncthreads();
+  if (warp == 0) {
+    int a = wsum[lane], b = wtile[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a2 = __shfl_up_sync(0xffffffffu, a, o), b2 = __shfl_up_sync(0xffffffffu, b, o);
+      if (lane >= o) a += a2, b += b2;
+    }
+    wsum[lane] = a, wtile[lane] = b;
+    if (lane == 31) offsets[E] = a, *n_tiles = b;
+  }
+  __syncthreads();
+  int run = (warp ? wsum[warp - 1] : 0) + ic - cs;
+  int trun = (warp ? wtile[warp - 1] : 0) + it - ts;
+  for (int e = e0; e < e1; ++e) {
+    const int c = counts[e];
+    offsets[e] = run;
+    cursor[e] = run;
+    for (int c0 = 0; c0 < c; c0 += kBN) tiles[trun++] = TernTile{e, c0, min(kBN, c - c0), run + c0};
+    run += c;
+  }
+}
 
-// One CTA: histogram per warp-range, scan, stable scatter, and the 128-token tile list.
-// smem: hist[kGroupWarps][E] int32 | tot[E] | tscan[E]
-__global__ void __launch_bounds__(kGroupWarps * 32) group_kernel(const int32_t* __restrict__ ids, int T, int E, int k,
-                                                                 int32_t* __restrict__ counts,
-                                                                 int32_t* __restrict__ offsets,
-                                                                 int32_t* __restrict__ perm,
-                                                                 int32_t* __restrict__ inv,
-                                                                 TernTile* __restrict__ tiles,
-                                                                 int32_t* __restrict__ n_tiles) {
-  extern __shared__ int32_t gsm[];
-  int32_t* hist = gsm;                  // [W][E]
-  int32_t* tot = gsm + kGroupWarps * E; // [E]
-  __shared__ int32_t wsum[kGroupWarps], wtile[kGroupWarps];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nthr = blockDim.x;
-  const int n = T * k;
-  const int per = (n + kGroupWarps - 1) / kGroupWarps;
-  const int i0 = min(n, warp * per), i1 = min(n, i0 + per);
-  for (int i = threadIdx.x; i < kGroupWarps * E; i += nthr) hist[i] = 0;
-  __syncthreads();
-  for (int i = i0 + lane; i < i1; i += 32) atomicAdd(&hist[warp * E + ids[i]], 1);
-  __syncthreads();
-  // per expert: total, and per-warp exclusive prefix (in place)
-  for (int e = threadIdx.x; e < E; e += nthr) {
-    int run = 0;
-    for (int w = 0; w < kGroupWarps; ++w) {
-      int c = hist[w * E + e];
-      hist[w * E + e] = run;
-      run += c;
-    }
-    tot[e] = run;
-    counts[e] = run;
-  }
-  __syncthreads();
-  // exclusive scan of totals and of tile counts: each warp scans a contiguous slice
-  const int eper = (E + kGroupWarps - 1) / kGroupWarps;
-  const int e0 = min(E, warp * eper), e1 = min(E, e0 + eper);
-  int ls = 0, lt = 0;
-  for (int e = e0 + lane; e < e1; e += 32) ls += tot[e], lt += (tot[e] + kBN - 1) / kBN;
-  for (int o = 16; o; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o), lt += __shfl_xor_sync(0xffffffffu, lt, o);
-  if (lane == 0) wsum[warp] = ls, wtile[warp] = lt;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int a = 0, b = 0;
-    for (int w = 0; w < kGroupWarps; ++w) {
-      int x = wsum[w], y = wtile[w];
-      wsum[w] = a, wtile[w] = b;
-      a += x, b += y;
-    }
-    offsets[E] = a;
-    *n_tiles = b;
-  }
-  __syncthreads();
-  if (lane == 0) {
-    int run = wsum[warp], trun = wtile[warp];
-    for (int e = e0; e < e1; ++e) {
-      const int c = tot[e];
-      offsets[e] = run;
-      for (int c0 = 0; c0 < c; c0 += kBN) tiles[trun++] = TernTile{e, c0, min(kBN, c - c0), run + c0};
-      tot[e] = run;  // becomes the expert's base offset
-      run += c;
-    }
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < kGroupWarps * E; i += nthr) hist[i] += tot[i % E];
-  __syncthreads();
-  // stable scatter: warp w walks its range in order
-  const unsigned ltm = (1u << lane) - 1u;
-  int32_t* cur = hist + warp * E;
-  for (int base = i0; base < i1; base += 32) {
-    const int i = base + lane;
-    const int e = i < i1 ? ids[i] : -1 - lane;
-    const unsigned mask = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(mask & ltm);
-    const int c = i < i1 ? cur[e] : 0;
-    __syncwarp();
-    if (i < i1) {
-      perm[c + rank] = i;
-      inv[i] = c + rank;
-      if (rank == 0) cur[e] = c + __popc(mask);
-    }
-    __syncwarp();
-  }
+// One thread per entry: position inside its expert's segment.
+__global__ void __launch_bounds__(256) group_scatter_kernel(const int32_t* __restrict__ ids, int n,
+                                                            int32_t* __restrict__ cursor, int32_t* __restrict__ perm,
+                                                            int32_t* __restrict__ inv) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const int pos = atomicAdd(&cursor[ids[i]], 1);
+  perm[pos] = i;
+  inv[i] = pos;
 }
 
 }  // namespace
@@ -829,7 +808,7 @@ cudaError_t configure_prefill_kernels() {
   if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PTQ1_0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 int(tern_smem(1, SCION_PTQ1_0)))))
     return e;
-  return cudaFuncSetAttribute(group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  return cudaSuccess;
 }
 
 // out[t] (= dense part, or 0 when the layer has no shared expert and no correction)
@@ -918,7 +897,10 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
     }
     case SCION_STAGE_ROUTE: {
       const int vpl = (L->E + 31) / 32;
-#define SCION_TOPK(V) topk_kernel<V><<<(T + 7) / 8, 256, 0, s>>>(P.logits, T, L->E, L->k, L->desc.norm_topk, P.ids, P.gates)
+      cudaError_t e = cudaMemsetAsync(P.counts, 0, sizeof(int32_t) * L->E, s);
+      if (e != cudaSuccess) return e;
+#define SCION_TOPK(V) \
+  topk_kernel<V><<<(T + 7) / 8, 256, 0, s>>>(P.logits, T, L->E, L->k, L->desc.norm_topk, P.ids, P.gates, P.counts)
       if (vpl <= 1) SCION_TOPK(1);
       else if (vpl <= 2) SCION_TOPK(2);
       else if (vpl <= 4) SCION_TOPK(4);
@@ -927,11 +909,12 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       else if (vpl <= 32) SCION_TOPK(32);
       else SCION_TOPK(64);
 #undef SCION_TOPK
-      cudaError_t e = cudaGetLastError();
-      if (e != cudaSuccess) return e;
-      const size_t gsm = sizeof(int32_t) * (size_t(kGroupWarps) * L->E + L->E);
-      group_kernel<<<1, kGroupWarps * 32, gsm, s>>>(P.ids, T, L->E, L->k, P.counts, P.offsets, P.perm, P.inv,
-                                                   static_cast<TernTile*>(P.tiles), P.n_tiles);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      group_scan_kernel<<<1, kScanThreads, 0, s>>>(P.counts, L->E, P.offsets, P.cursor,
+                                                  static_cast<TernTile*>(P.tiles), P.n_tiles);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      const int n = T * L->k;
+      group_scatter_kernel<<<(n + 255) / 256, 256, 0, s>>>(P.ids, n, P.cursor, P.perm, P.inv);
       return cudaGetLastError();
     }
     case SCION_STAGE_GATEUP: {

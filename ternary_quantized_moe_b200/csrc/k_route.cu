@@ -175,45 +175,18 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
 }
 
 // ---------------------------------------------------------------- decode route
-// One CTA for one pass of T <= SCION_TDEC tokens (E <= 512), everything between the logits
-// and the outputs in shared memory: warp w selects the top k and the gates of tokens w,
-// w + 32, ..., then the CTA groups the T*k entries -- histogram, exclusive scan, active-expert
-// list with the per-slot records, and the stable scatter in (token, slot) order.
-// 1024 threads (one warp per token up to 32 tokens); 512 when each lane holds 16 logits, to
-// keep the sorted lane lists in registers.
-template <int VPL>
-constexpr int rc_threads() {
-  return VPL >= 16 ? 512 : 1024;
-}
+// One pass of T <= SCION_TDEC tokens (E <= 512).  Top-k and gates by one warp per token, then
+// the grouping of the T*k entries inside one CTA's shared memory: histogram, exclusive scan,
+// active-expert list with the per-slot records, and the stable scatter in (token, slot) order.
+// Up to 32 tokens one CTA does everything; above that the top-k is spread over ceil(T/4) CTAs
+// and the last one to finish stages the entries and groups them.
 
-template <int VPL>
-__global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
-    const float* __restrict__ logits, int T, int E, int k, int norm_topk, int32_t* __restrict__ ids,
-    float* __restrict__ gates, int32_t* __restrict__ counts_out, int32_t* __restrict__ offsets_out,
-    int32_t* __restrict__ perm_out, float* __restrict__ gperm_out, int32_t* __restrict__ active_out,
-    int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info) {
-  extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [E] | cursor [E]
-  const int n = T * k;
-  int32_t* ids_s = reinterpret_cast<int32_t*>(rs);
-  float* gates_s = rs + n;
-  int32_t* counts = reinterpret_cast<int32_t*>(rs + 2 * n);
-  int32_t* cursor = counts + E;
-  constexpr int kRcThreads = rc_threads<VPL>();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_trigger();
-  for (int e = threadIdx.x; e < E; e += kRcThreads) counts[e] = 0;
-  pdl_wait();
-  for (int t = warp; t < T; t += kRcThreads / 32)
-    warp_topk<VPL>(logits + int64_t(t) * E, E, k, norm_topk, lane, ids_s + t * k, gates_s + t * k);
-  __syncthreads();
-  for (int i = threadIdx.x; i < n; i += kRcThreads) {
-    ids[i] = ids_s[i];
-    gates[i] = gates_s[i];
-    atomicAdd(&counts[ids_s[i]], 1);
-  }
-  __syncthreads();
-  if (warp != 0) return;
-  // ---- exclusive scan of the counts, active list and slot records (warp 0)
+// Warp 0 of the grouping CTA: counts[] holds the histogram of the n staged entries.
+__device__ __forceinline__ void group_staged(const int32_t* ids_s, const float* gates_s, int n, int E, int lane,
+                                             int32_t* counts, int32_t* cursor, int32_t* __restrict__ counts_out,
+                                             int32_t* __restrict__ offsets_out, int32_t* __restrict__ perm_out,
+                                             float* __restrict__ gperm_out, int32_t* __restrict__ active_out,
+                                             int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info) {
   const int per = (E + 31) / 32;
   const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
   int sc = 0, ac = 0;
@@ -238,7 +211,7 @@ __global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
   }
   if (lane == 31) offsets_out[E] = si, *n_active_out = ai;
   __syncwarp();
-  // ---- stable scatter in (token, slot) order, 32 entries at a time
+  // stable scatter in (token, slot) order, 32 entries at a time
   const unsigned lt = (1u << lane) - 1u;
   for (int base = 0; base < n; base += 32) {
     const int i = base + lane;
@@ -256,6 +229,82 @@ __global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
   }
 }
 
+// Single CTA (T <= 32): 1024 threads, one warp per token; 512 when each lane holds 16 logits,
+// to keep the sorted lane lists in registers.
+template <int VPL>
+constexpr int rc_threads() {
+  return VPL >= 16 ? 512 : 1024;
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
+    const float* __restrict__ logits, int T, int E, int k, int norm_topk, int32_t* __restrict__ ids,
+    float* __restrict__ gates, int32_t* __restrict__ counts_out, int32_t* __restrict__ offsets_out,
+    int32_t* __restrict__ perm_out, float* __restrict__ gperm_out, int32_t* __restrict__ active_out,
+    int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info) {
+  extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [E] | cursor [E]
+  const int n = T * k;
+  int32_t* ids_s = reinterpret_cast<int32_t*>(rs);
+  float* gates_s = rs + n;
+  int32_t* counts = reinterpret_cast<int32_t*>(rs + 2 * n);
+  int32_t* cursor = counts + E;
+  constexpr int kThr = rc_threads<VPL>();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_trigger();
+  for (int e = threadIdx.x; e < E; e += kThr) counts[e] = 0;
+  pdl_wait();
+  for (int t = warp; t < T; t += kThr / 32)
+    warp_topk<VPL>(logits + int64_t(t) * E, E, k, norm_topk, lane, ids_s + t * k, gates_s + t * k);
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += kThr) {
+    ids[i] = ids_s[i];
+    gates[i] = gates_s[i];
+    atomicAdd(&counts[ids_s[i]], 1);
+  }
+  __syncthreads();
+  if (warp == 0)
+    group_staged(ids_s, gates_s, n, E, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out,
+                 active_out, n_active_out, slot_info);
+}
+
+// ceil(T/4) CTAs of 4 warps (T > 32); the last CTA to finish groups.
+constexpr int kRmThreads = 128;
+
+template <int VPL>
+__global__ void __launch_bounds__(kRmThreads) route_multi_kernel(
+    const float* __restrict__ logits, int T, int E, int k, int norm_topk, int32_t* __restrict__ ids,
+    float* __restrict__ gates, int32_t* __restrict__ counts_out, int32_t* __restrict__ offsets_out,
+    int32_t* __restrict__ perm_out, float* __restrict__ gperm_out, int32_t* __restrict__ active_out,
+    int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info, unsigned* __restrict__ done) {
+  extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [E] | cursor [E]
+  __shared__ int last;
+  const int n = T * k;
+  int32_t* ids_s = reinterpret_cast<int32_t*>(rs);
+  float* gates_s = rs + n;
+  int32_t* counts = reinterpret_cast<int32_t*>(rs + 2 * n);
+  int32_t* cursor = counts + E;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (kRmThreads / 32) + warp;
+  pdl_trigger();
+  pdl_wait();
+  if (t < T) warp_topk<VPL>(logits + int64_t(t) * E, E, k, norm_topk, lane, ids + t * k, gates + t * k);
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = (atomicAdd(done, 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  for (int e = threadIdx.x; e < E; e += kRmThreads) counts[e] = 0;
+  for (int i = threadIdx.x; i < n; i += kRmThreads) ids_s[i] = __ldcg(&ids[i]), gates_s[i] = __ldcg(&gates[i]);
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += kRmThreads) atomicAdd(&counts[ids_s[i]], 1);
+  __syncthreads();
+  if (warp != 0) return;
+  if (lane == 0) *done = 0;
+  group_staged(ids_s, gates_s, n, E, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out, active_out,
+               n_active_out, slot_info);
+}
+
 size_t route_cta_smem(int T, int E, int k) { return sizeof(float) * (2 * size_t(T) * k + 2 * size_t(E)); }
 
 }  // namespace
@@ -270,11 +319,15 @@ cudaError_t launch_router_f32(const scion_layer* L, const __nv_bfloat16* x, int 
 cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s) {
   if (L->E <= 512) {
     const size_t smem = route_cta_smem(T, L->E, L->k);
-#define SCION_ROUTE_CTA(V)                                                                                     \
-  return launch_pdl(route_cta_kernel<V>, dim3(1), dim3(rc_threads<V>()), smem, s, L->logits, T, L->E, L->k,\
-                    L->desc.norm_topk, L->ids, L->gates, L->counts, L->offsets, L->perm, L->gperm, L->active, \
-                    L->n_active, reinterpret_cast<int4*>(L->slot_info))
     const int vpl = (L->E + 31) / 32;
+#define SCION_ROUTE_CTA(V)                                                                                     \
+  return T <= 32 ? launch_pdl(route_cta_kernel<V>, dim3(1), dim3(rc_threads<V>()), smem, s, L->logits, T, L->E, \
+                              L->k, L->desc.norm_topk, L->ids, L->gates, L->counts, L->offsets, L->perm,       \
+                              L->gperm, L->active, L->n_active, reinterpret_cast<int4*>(L->slot_info))        \
+                 : launch_pdl(route_multi_kernel<V>, dim3((T + 3) / 4), dim3(kRmThreads), smem, s, L->logits, T, \
+                              L->E, L->k, L->desc.norm_topk, L->ids, L->gates, L->counts, L->offsets, L->perm, \
+                              L->gperm, L->active, L->n_active, reinterpret_cast<int4*>(L->slot_info),         \
+                              L->route_done)
     if (vpl <= 1) SCION_ROUTE_CTA(1);
     else if (vpl <= 2) SCION_ROUTE_CTA(2);
     else if (vpl <= 4) SCION_ROUTE_CTA(4);
@@ -315,6 +368,11 @@ cudaError_t configure_route_kernels() {
   if ((e = cudaFuncSetAttribute(route_cta_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, cta_max))) return e;
   if ((e = cudaFuncSetAttribute(route_cta_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, cta_max))) return e;
   if ((e = cudaFuncSetAttribute(route_cta_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, cta_max))) return e;
+  if ((e = cudaFuncSetAttribute(route_multi_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, cta_max))) return e;
+  if ((e = cudaFuncSetAttribute(route_multi_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, cta_max))) return e;
+  if ((e = cudaFuncSetAttribute(route_multi_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, cta_max))) return e;
+  if ((e = cudaFuncSetAttribute(route_multi_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, cta_max))) return e;
+  if ((e = cudaFuncSetAttribute(route_multi_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, cta_max))) return e;
   return cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
 }
 

@@ -45,13 +45,13 @@ void free_layer(scion_layer* L) {
   void* ptrs[] = {L->gu_bank, L->dn_bank,  L->dense_down, L->xunits,  L->logits,    L->ids,       L->gates,
                   L->counts,  L->offsets,  L->perm,       L->active,  L->n_active,  L->h,         L->hz,
                   L->xfrag,   L->x_stage, L->out_stage, L->bad,       L->err,
-                  L->slot_info, L->gperm};
+                  L->slot_info, L->gperm, L->route_done};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   if (L->pre) {
     scion::PrefillState* P = L->pre;
     void* pp[] = {P->xunits, P->dunits, P->logits, P->ids, P->gates, P->counts, P->offsets,
-                  P->perm,   P->inv,    P->y,       P->tiles, P->n_tiles, P->x16, P->h, P->hz};
+                  P->perm,   P->inv,    P->y,       P->tiles, P->n_tiles, P->x16, P->h, P->hz, P->cursor};
     for (void* p : pp)
       if (p) cudaFree(p);
     delete P;
@@ -78,6 +78,7 @@ int create_prefill(scion_layer* L, cudaStream_t s) {
   PTRY(dev_alloc(L, &P->offsets, sizeof(int32_t) * (L->E + 1)));
   PTRY(dev_alloc(L, &P->perm, sizeof(int32_t) * Tk));
   PTRY(dev_alloc(L, &P->inv, sizeof(int32_t) * Tk));
+  PTRY(dev_alloc(L, &P->cursor, sizeof(int32_t) * L->E));
   PTRY(dev_alloc(L, &P->y, sizeof(__half) * Tk * L->d));
   PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->tiles), scion::prefill_tile_bytes() * max_tiles));
   PTRY(dev_alloc(L, &P->n_tiles, sizeof(int32_t)));
@@ -262,6 +263,8 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   SCION_TRY(dev_alloc(L, &L->active, sizeof(int32_t) * L->E));
   SCION_TRY(dev_alloc(L, &L->n_active, sizeof(int32_t)));
   SCION_TRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&L->slot_info), sizeof(int4) * L->E));
+  SCION_TRY(dev_alloc(L, &L->route_done, sizeof(unsigned)));
+  SCION_TRY(cudaMemsetAsync(L->route_done, 0, sizeof(unsigned), s));
   SCION_TRY(dev_alloc(L, &L->h, sizeof(__half) * TD * L->k * L->GF * SCION_BROW));
   SCION_TRY(dev_alloc(L, &L->hz, sizeof(__half) * TD * (L->Kd ? L->Kd : 1)));
   SCION_TRY(dev_alloc(L, &L->xfrag, sizeof(__half) * TD * L->Gd * SCION_BROW));

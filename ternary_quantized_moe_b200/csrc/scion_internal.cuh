@@ -74,6 +74,7 @@ struct PrefillState {
   int32_t* offsets;     // [E+1]
   int32_t* perm;        // [maxT*k]
   int32_t* inv;         // [maxT*k] position of entry t*k+j in perm
+  int32_t* cursor;      // [E] next free position of each expert's segment (grouping scratch)
   __half* y;            // [maxT*k][d] expert down outputs in fp16 (gate not yet applied), one row per routed entry
   void* tiles;          // 128-token tiles, [maxT*k/128 + E]
   int32_t* n_tiles;
@@ -108,6 +109,7 @@ struct scion_layer {
   int32_t* active;   // [E]
   int32_t* n_active; // [1]
   void* slot_info;    // int4 [E]: {expert, first position, token count, 0} per active slot
+  unsigned* route_done;  // [1] arrival counter of the multi-CTA decode route kernel (zero between calls)
   __half* h;         // [TDEC*k][GF][SCION_BROW] fragment order + group-sum tails
   __half* hz;        // [TDEC][Kd] (pad columns stay 0)
   __half* xfrag;     // [TDEC][Gd][SCION_BROW] x in fragment order (fp16) + group-sum tails
