@@ -155,7 +155,10 @@ size_t scion_layer_device_bytes(const scion_layer* layer);
  * 0 <= T <= max_tokens (T = 0 is a no-op).  Batches of at most 64 tokens stream the
  * weights through warp-level MMA kernels; larger batches (layers created with
  * max_tokens > 64) run as tcgen05 grouped GEMMs.  Calls on one handle must not
- * overlap on the GPU (they share its workspace): issue them on one stream.
+ * overlap on the GPU (they share its workspace): issue them on one stream.  Batches of
+ * 16..64 tokens fork the dense down projection onto a stream owned by the handle and
+ * join it back (events) before the call's work on `stream` ends; stream capture into
+ * a CUDA graph records the fork and the join.
  * EINVAL on a null pointer or T out of range; ECUDA if a launch fails. */
 int scion_moe_forward(const void* x, int T, const scion_layer* layer, float* out, void* stream);
 

@@ -48,6 +48,9 @@ void free_layer(scion_layer* L) {
                   L->slot_info, L->gperm, L->route_done};
   for (void* p : ptrs)
     if (p) cudaFree(p);
+  if (L->side) cudaStreamDestroy(L->side);
+  if (L->ev_x) cudaEventDestroy(L->ev_x);
+  if (L->ev_dense) cudaEventDestroy(L->ev_dense);
   if (L->pre) {
     scion::PrefillState* P = L->pre;
     void* pp[] = {P->xunits, P->dunits, P->logits, P->ids, P->gates, P->counts, P->offsets,
@@ -183,11 +186,26 @@ int forward_prefill(const scion_layer* L, const __nv_bfloat16* x, int T, float* 
 int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, cudaStream_t s) {
   if (L->desc.router_fp32) SCION_STAGE(SCION_STAGE_ROUTER_F32, scion::launch_router_f32(L, x, T, L->logits, s));
   SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_xproj(L, x, T, out, s));
-  SCION_STAGE(SCION_STAGE_ROUTE, scion::launch_route(L, T, s));
   const bool ring = T >= L->stream_min_tokens;
+  // batches on the ring kernels run the dense down projection (it needs only the x-projection)
+  // on the layer's side stream, beside routing and the expert kernels; the caller's stream
+  // joins it before the forward ends
+  const bool side = ring && L->Kdense;
+  if (side) {
+    cudaError_t e = cudaEventRecord(L->ev_x, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(L->side, L->ev_x, 0);
+    if (e != cudaSuccess) return cuda_status(e);
+    {
+      cudaStream_t s = L->side;  // SCION_STAGE launches and records on `s`
+      SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
+    }
+    if ((e = cudaEventRecord(L->ev_dense, L->side)) != cudaSuccess) return cuda_status(e);
+  }
+  SCION_STAGE(SCION_STAGE_ROUTE, scion::launch_route(L, T, s));
   SCION_STAGE(SCION_STAGE_GATEUP, ring ? scion::launch_stream_gateup(L, T, s) : scion::launch_gateup(L, x, T, s));
   SCION_STAGE(SCION_STAGE_DOWN_ROUTED,
               ring ? scion::launch_stream_down(L, T, out, s) : scion::launch_down_routed(L, T, out, s));
+  if (side) return cuda_status(cudaStreamWaitEvent(s, L->ev_dense, 0));
   if (L->Kdense) SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
   return SCION_OK;
 }
@@ -272,6 +290,9 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   SCION_TRY(dev_alloc(L, &L->out_stage, sizeof(float) * size_t(max_tokens) * L->d));
   SCION_TRY(dev_alloc(L, &L->bad, sizeof(int64_t)));
   SCION_TRY(dev_alloc(L, &L->err, sizeof(int)));
+  SCION_TRY(cudaStreamCreateWithFlags(&L->side, cudaStreamNonBlocking));
+  SCION_TRY(cudaEventCreateWithFlags(&L->ev_x, cudaEventDisableTiming));
+  SCION_TRY(cudaEventCreateWithFlags(&L->ev_dense, cudaEventDisableTiming));
   SCION_TRY(cudaMemsetAsync(L->err, 0, sizeof(int), s));
 
   if (!units.empty())

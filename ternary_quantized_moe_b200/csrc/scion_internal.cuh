@@ -119,6 +119,8 @@ struct scion_layer {
   int* err;          // [1] device status word (a bounded wait that gave up writes ETIMEOUT)
   scion::PrefillState* pre;  // tensor-core path (nullptr when max_tokens <= SCION_TDEC)
   int stream_min_tokens;     // decode batches of at least this many tokens use the bulk-copy ring kernels
+  cudaStream_t side;         // the dense down projection of ring-kernel batches runs here
+  cudaEvent_t ev_x, ev_dense;  // x-projection done (fork) / dense down done (join)
   size_t device_bytes;
 };
 
