@@ -34,8 +34,9 @@ struct XProjArgs {
   int T, d, E, Fs, r, Kd;  // Kd = padded row stride of hz
   int fmt;
   const __nv_bfloat16 *w_router, *w_delta, *sh_gate, *sh_up, *corr_a;
-  const XUnit* units;
+  const XUnit* units;  // this launch's units (a slice of the layer's table)
   int n_units, n_chunks;
+  int n_aux;           // CTA columns after the units that run xproj_aux (0 or kXAux)
   float* logits;
   __half* hz;
   __half* xfrag;  // [T][d/128][SCION_BROW] fp16 in fragment order + group sums
@@ -111,7 +112,7 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
   pdl_trigger();
   if (blockIdx.x >= a.n_units) {
     pdl_wait();
-    xproj_aux(a, (blockIdx.x - a.n_units) * a.n_chunks + chunk, kXAux * a.n_chunks);
+    xproj_aux(a, (blockIdx.x - a.n_units) * a.n_chunks + chunk, a.n_aux * a.n_chunks);
     return;
   }
 
@@ -493,7 +494,8 @@ __global__ void unfrag_kernel(int fmt, const __half* __restrict__ src, int64_t n
 }  // namespace
 
 // ------------------------------------------------------------------- launchers
-cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, cudaStream_t s) {
+cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, int unit0, int n_units,
+                         bool aux, cudaStream_t s) {
   XProjArgs a;
   a.x = x;
   a.T = T, a.d = L->d, a.E = L->E, a.Fs = L->Fs, a.r = L->r, a.Kd = L->Kd, a.fmt = L->fmt;
@@ -502,10 +504,11 @@ cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, fl
   a.sh_gate = static_cast<const __nv_bfloat16*>(L->desc.sh_gate);
   a.sh_up = static_cast<const __nv_bfloat16*>(L->desc.sh_up);
   a.corr_a = static_cast<const __nv_bfloat16*>(L->desc.corr_a);
-  a.units = L->xunits, a.n_units = L->n_xunits, a.n_chunks = L->n_xchunks;
+  a.units = L->xunits + unit0, a.n_units = n_units, a.n_chunks = L->n_xchunks, a.n_aux = aux ? kXAux : 0;
   a.logits = L->logits, a.hz = L->hz, a.xfrag = L->xfrag, a.out = out;
   a.h = L->h, a.k = L->k, a.GF = L->GF;
-  dim3 grid(L->n_xunits + kXAux, L->n_xchunks);
+  if (n_units + a.n_aux == 0) return cudaSuccess;
+  dim3 grid(n_units + a.n_aux, L->n_xchunks);
   const dim3 cluster(1, L->n_xchunks, 1);
   const int nt = (T + 7) / 8;
   switch (nt) {

@@ -185,18 +185,22 @@ int forward_prefill(const scion_layer* L, const __nv_bfloat16* x, int T, float* 
 // One pass of T <= SCION_TDEC tokens.
 int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, cudaStream_t s) {
   if (L->desc.router_fp32) SCION_STAGE(SCION_STAGE_ROUTER_F32, scion::launch_router_f32(L, x, T, L->logits, s));
-  SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_xproj(L, x, T, out, s));
   const bool ring = T >= L->stream_min_tokens;
-  // batches on the ring kernels run the dense down projection (it needs only the x-projection)
-  // on the layer's side stream, beside routing and the expert kernels; the caller's stream
-  // joins it before the forward ends
+  // Batches on the ring kernels split the dense work off the expert path: the caller's stream
+  // runs the router part of the x-projection (with x's fragment rows and the clearing of out),
+  // the layer's side stream the shared-expert / correction part and the dense down projection,
+  // beside routing and the expert kernels; the caller's stream joins it at the end.
   const bool side = ring && L->Kdense;
+  const int nx_main = side ? L->n_xrouter : L->n_xunits;
+  SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_xproj(L, x, T, out, 0, nx_main, true, s));
   if (side) {
     cudaError_t e = cudaEventRecord(L->ev_x, s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(L->side, L->ev_x, 0);
     if (e != cudaSuccess) return cuda_status(e);
     {
       cudaStream_t s = L->side;  // SCION_STAGE launches and records on `s`
+      SCION_STAGE(SCION_STAGE_XPROJ,
+                  scion::launch_xproj(L, x, T, out, L->n_xrouter, L->n_xunits - L->n_xrouter, false, s));
       SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
     }
     if ((e = cudaEventRecord(L->ev_dense, L->side)) != cudaSuccess) return cuda_status(e);
@@ -264,6 +268,7 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   for (int f0 = 0; f0 < L->Fs; f0 += 16) units.push_back({scion::kUnitSwiglu, f0});
   for (int q0 = 0; q0 < L->r; q0 += 16) units.push_back({scion::kUnitPlain, q0});
   L->n_xunits = int(units.size());
+  L->n_xrouter = desc->router_fp32 ? 0 : (L->E + 15) / 16;
   L->n_xchunks = (L->d + SCION_XPROJ_KC - 1) / SCION_XPROJ_KC;
 
   SCION_TRY(scion::configure_kernels());

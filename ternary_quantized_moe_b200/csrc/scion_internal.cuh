@@ -97,6 +97,7 @@ struct scion_layer {
   __half* dense_down;  // [d][Kd] fp16: sh_down | corr_b | 0
   scion::XUnit* xunits;
   int n_xunits;
+  int n_xrouter;     // router units (the first n_xrouter entries of xunits)
   int n_xchunks;
   // workspace (sized for SCION_TDEC tokens per pass, max_tokens for staging)
   float* logits;     // [TDEC][E]
@@ -146,7 +147,11 @@ cudaError_t configure_route_kernels();
 cudaError_t launch_slot_info(const scion_layer* L, cudaStream_t s);
 
 // k_decode.cu
-cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, cudaStream_t s);
+// Units [unit0, unit0 + n_units) of the layer's x-projection table (router units first, then
+// shared gate/up, then correction A); `aux` adds the CTAs that write x's fragment rows and
+// clear out and the hidden's group-sum tails.
+cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, int unit0, int n_units,
+                         bool aux, cudaStream_t s);
 cudaError_t launch_gateup(const scion_layer* L, const __nv_bfloat16* x, int T, cudaStream_t s);
 cudaError_t launch_down_routed(const scion_layer* L, int T, float* out, cudaStream_t s);
 cudaError_t launch_down_dense(const scion_layer* L, int T, float* out, cudaStream_t s);
