@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_gemm_kernel(const __grid_co
     const int q = warp - 4;
     const int row = q * 32 + lane;
     int li = 0;
-    // no abort-flag test in the loop condition: the 128 threads leave only together, by the vote
+    // no abort-flag test in the loop condition: the epilogue threads leave only together, by the vote
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x) {
       const DenseTile dt = dense_tile(p, t);
       if (dt.tok0 >= p.T) continue;
@@ -422,8 +422,8 @@ struct TernRing {
   static_assert(a_col0 + kA * a_cols <= tmem_cols, "TMEM budget");
 };
 
-constexpr int kTernThreads = 512;  // 16 warps: codes, MMA, 2 x B rows, 8 expansion, 4 epilogue
-constexpr int kEpiThreads = 128;
+constexpr int kTernThreads = 640;  // 20 warps: codes, MMA, 2 x B rows, 8 expansion, 8 epilogue
+constexpr int kEpiThreads = 256;
 
 // Persistent grouped GEMM: CTA b walks the work items b, b + gridDim.x, ... where item =
 // (128-token tile, 128-row weight tile).  The expansion warps decode the packed codes of each
@@ -503,32 +503,36 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
     }
   } else if (!kBTma && (warp == 2 || warp == 3)) {
     // ---------------- gathered B rows (tokens of the tile), 128 columns (two atoms) per group;
-    // warp 2 takes rows 0..63, warp 3 rows 64..127
-    const int rbase = (warp - 2) * 64;
+    // warp 2 takes rows 0..63, warp 3 rows 64..127.  Lanes 2m and 2m+1 copy the two 16-byte
+    // halves of one 32-byte sector of the same row, so every request is a whole L2 sector:
+    // lane (m, hf) handles rows rbase + m + 16i (i < 4), 16-byte chunks 2j + hf (j < 8).
+    const int rbase = (warp - 2) * 64 + (lane >> 1), hf = lane & 1;
     constexpr int kLag = R::kB / 2;  // groups in flight per thread before the oldest is published
     int gs = 0;                      // running group counter
     for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
       const TernTile tile = load_tile(p.tiles, item / RT);
-      const __half* rows[2];
+      const __half* rows[4];
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int r = rbase + lane + 32 * i;
-        rows[i] = r < tile.n ? p.bsrc + int64_t(p.perm[tile.pos0 + r] / p.k) * p.ldb : nullptr;
+      for (int i = 0; i < 4; ++i) {
+        const int r = rbase + 16 * i;
+        rows[i] = r < tile.n ? p.bsrc + int64_t(p.perm[tile.pos0 + r] / p.k) * p.ldb + 8 * hf : nullptr;
       }
       for (int g = 0; g < p.G; ++g, ++gs) {
         const int s = gs % R::kB;
         if (gs >= R::kB && !mbar_wait(&b_empty[s], ((gs / R::kB) - 1) & 1, &abort_flag, p.err)) break;
         const uint32_t bt = sbase + R::b_off + s * R::b_bytes;
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < 4; ++i) {
           if (!rows[i]) continue;
-          const int r = rbase + lane + 32 * i;
+          const int r = rbase + 16 * i;
           const __half* src = rows[i] + g * 128;
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(bt + (j >> 3) * kAtom + sw128_offset(r, j & 7)),
-                         "l"(src + 8 * j)
+          for (int j = 0; j < 8; ++j) {
+            const int ch = 2 * j + hf;  // 16-byte chunk of the row's 256 bytes
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(bt + (ch >> 3) * kAtom + sw128_offset(r, ch & 7)),
+                         "l"(src + 16 * j)
                          : "memory");
+          }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
         // group gs - kLag has landed: make it visible to the tensor cores (async proxy), then publish it
@@ -609,13 +613,14 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
     }
   } else if (warp >= 12) {
     // ---------------- epilogue: TMEM lane quarter q = weight rows 32q .. 32q+31, 16 tokens per
-    // chunk.  Stores go straight to global memory.
-    const int q = warp & 3;
+    // chunk; the two warps of a quarter take alternate chunks.  Stores go straight to global
+    // memory.
+    const int q = warp & 3, half = (warp - 12) >> 2;
     const int row = q * 32 + lane;
     const int pcol = perm_pos(FMT, row);  // gate/up: position of this row inside its 128-column group of h
     const float hscale = FMT == SCION_PQ2_0 ? pq2_pos_scale(pcol) : 1.0f;
     int li = 0;
-    // no abort-flag test in the loop condition: the 128 threads leave only together, by the vote
+    // no abort-flag test in the loop condition: the epilogue threads leave only together, by the vote
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++li) {
       const TernTile tile = load_tile(p.tiles, item / RT);
       const int rt = item % RT;
@@ -625,7 +630,7 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
       if (!named_bar_and(1, kEpiThreads, mbar_wait(&acc_full[ab], (li / R::n_acc) & 1, &abort_flag, p.err))) break;
       tc_fence_after();
       const uint32_t acc = tmem + ab * R::acc_cols + (uint32_t(q * 32) << 16);
-      for (int c = 0; c * 16 < nn; ++c) {
+      for (int c = half; c * 16 < nn; c += 2) {
         float v0[16], v1[16];
         if constexpr (NA == 2)
           tmem_ld16x2(acc + c * 16, acc + kBN + c * 16, v0, v1);
