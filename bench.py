@@ -391,9 +391,10 @@ def run_gpu(args, rank, world, local_rank):
            "d2h_bytes_per_step": sum(T * cfg.d * 4 for T in batches)}
 
     # ---- roofline of the dominant kernel
-    dom = max((k_ for k_ in stages if stages[k_][1] > 0), key=lambda k_: stages[k_][0])
-    dom_ms, dom_n = stages[dom]
     decode = max_T <= 64
+    work = sbytes if decode else sflops  # the roofline is taken on a stage that moves weights / does MMAs
+    dom = max((k_ for k_ in stages if stages[k_][1] > 0 and work.get(k_, 0) > 0), key=lambda k_: stages[k_][0])
+    dom_ms, dom_n = stages[dom]
     if decode:
         achieved = (sbytes[dom] / dom_n) / (dom_ms / dom_n / 1000.0) / 1e9
         roof = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",

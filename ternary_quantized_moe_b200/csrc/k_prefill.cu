@@ -415,7 +415,7 @@ struct TernRing {
   // tensor memory: accumulators, then the ring of expanded A groups
   static constexpr int n_acc = NA == 2 ? 1 : 2;   // gate/up: one NA x 128 accumulator; down: ping-pong
   static constexpr uint32_t acc_cols = NA * kBN;
-  static constexpr int kA = 2;
+  static constexpr int kA = NA == 2 ? 2 : 4;      // down: the TMEM left over by the accumulators
   static constexpr uint32_t a_cols = NA * 64;     // one group: NA matrices x 64 columns (128 fp16 per lane)
   static constexpr uint32_t a_col0 = n_acc * acc_cols;
   static constexpr uint32_t tmem_cols = 512;
@@ -663,16 +663,29 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
 }
 
 // ------------------------------------------------------------------- routing
-// One warp per token (8 per CTA), logits in registers.
+// One warp per token, kTopkTokensPerWarp tokens per warp, logits in registers.  The expert
+// histogram is counted in shared memory and added to the global one once per CTA and expert
+// (a hot expert of a skewed router would otherwise take one global atomic per selection).
+constexpr int kTopkTokensPerWarp = 4;
+constexpr int kTopkTokensPerCta = 8 * kTopkTokensPerWarp;
 template <int VPL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                    int norm_topk, int32_t* __restrict__ ids, float* __restrict__ gates,
                                                    int32_t* __restrict__ counts) {
+  extern __shared__ int32_t hist[];  // [E]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + warp;
-  if (t >= T) return;
-  warp_topk<VPL>(logits + int64_t(t) * E, E, k, norm_topk, lane, ids + int64_t(t) * k, gates + int64_t(t) * k);
-  if (lane < k) atomicAdd(&counts[ids[int64_t(t) * k + lane]], 1);  // histogram of the selections
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  for (int i = 0; i < kTopkTokensPerWarp; ++i) {
+    const int t = blockIdx.x * kTopkTokensPerCta + i * 8 + warp;
+    if (t >= T) break;
+    warp_topk<VPL>(logits + int64_t(t) * E, E, k, norm_topk, lane, ids + int64_t(t) * k, gates + int64_t(t) * k);
+    __syncwarp();
+    if (lane < k) atomicAdd(&hist[ids[int64_t(t) * k + lane]], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (hist[e]) atomicAdd(&counts[e], hist[e]);
 }
 
 // Grouping by expert.  The order of the tokens inside an expert's segment is free (each token
@@ -726,15 +739,37 @@ __global__ void __launch_bounds__(kScanThreads) group_scan_kernel(const int32_t*
   }
 }
 
-// One thread per entry: position inside its expert's segment.
-__global__ void __launch_bounds__(256) group_scatter_kernel(const int32_t* __restrict__ ids, int n,
+// Positions inside the experts' segments: kScatterPerThread entries per thread.  Each CTA
+// ranks its entries per expert in shared memory, then reserves one block of positions per
+// expert it touches with a single global atomic.
+constexpr int kScatterPerThread = 8;
+constexpr int kScatterPerCta = 256 * kScatterPerThread;
+__global__ void __launch_bounds__(256) group_scatter_kernel(const int32_t* __restrict__ ids, int n, int E,
                                                             int32_t* __restrict__ cursor, int32_t* __restrict__ perm,
                                                             int32_t* __restrict__ inv) {
-  const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n) return;
-  const int pos = atomicAdd(&cursor[ids[i]], 1);
-  perm[pos] = i;
-  inv[i] = pos;
+  extern __shared__ int32_t sh[];  // cnt[E], base[E]
+  int32_t *cnt = sh, *base = sh + E;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  int id[kScatterPerThread], local[kScatterPerThread];
+  const int i0 = blockIdx.x * kScatterPerCta + threadIdx.x;
+#pragma unroll
+  for (int j = 0; j < kScatterPerThread; ++j) {
+    const int i = i0 + 256 * j;
+    id[j] = i < n ? ids[i] : -1;
+    local[j] = id[j] >= 0 ? atomicAdd(&cnt[id[j]], 1) : 0;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (cnt[e]) base[e] = atomicAdd(&cursor[e], cnt[e]);
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < kScatterPerThread; ++j) {
+    if (id[j] < 0) continue;
+    const int i = i0 + 256 * j, pos = base[id[j]] + local[j];
+    perm[pos] = i;
+    inv[i] = pos;
+  }
 }
 
 }  // namespace
@@ -905,7 +940,8 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       cudaError_t e = cudaMemsetAsync(P.counts, 0, sizeof(int32_t) * L->E, s);
       if (e != cudaSuccess) return e;
 #define SCION_TOPK(V) \
-  topk_kernel<V><<<(T + 7) / 8, 256, 0, s>>>(P.logits, T, L->E, L->k, L->desc.norm_topk, P.ids, P.gates, P.counts)
+  topk_kernel<V><<<(T + kTopkTokensPerCta - 1) / kTopkTokensPerCta, 256, sizeof(int32_t) * L->E, s>>>( \
+      P.logits, T, L->E, L->k, L->desc.norm_topk, P.ids, P.gates, P.counts)
       if (vpl <= 1) SCION_TOPK(1);
       else if (vpl <= 2) SCION_TOPK(2);
       else if (vpl <= 4) SCION_TOPK(4);
@@ -919,7 +955,8 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
                                                   static_cast<TernTile*>(P.tiles), P.n_tiles);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
       const int n = T * L->k;
-      group_scatter_kernel<<<(n + 255) / 256, 256, 0, s>>>(P.ids, n, P.cursor, P.perm, P.inv);
+      group_scatter_kernel<<<(n + kScatterPerCta - 1) / kScatterPerCta, 256, 2 * sizeof(int32_t) * L->E, s>>>(
+          P.ids, n, L->E, P.cursor, P.perm, P.inv);
       return cudaGetLastError();
     }
     case SCION_STAGE_GATEUP: {

@@ -33,61 +33,55 @@ __device__ __forceinline__ void warp_topk(const float* __restrict__ row, int E, 
     for (int o = 16; o; o >>= 1) zall += __shfl_xor_sync(0xffffffffu, zall, o);
   }
   static_assert(VPL <= 64, "at most 2048 experts");
-  float my_v = -INFINITY;
-  int my_id = -1;
-  if constexpr (VPL <= 16) {
-    // each lane sorts its values (descending, lower id first on ties) ...
-    int id[VPL];
+  // Order-preserving 32-bit keys of the logits (larger logit <-> larger key; -0 is taken as +0,
+  // so equal logits stay ties); entries past E get key 0, below every logit's key (-FLT_MAX maps
+  // to 0x00800000).
+  uint32_t key[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const uint32_t b = v[i] == 0.f ? 0u : __float_as_uint(v[i]);
+    key[i] = lane + 32 * i < E ? ((b >> 31) ? ~b : (b | 0x80000000u)) : 0u;
+  }
+  // Each lane keeps its L best entries in (key descending, slot ascending) order: the slot order
+  // is the id order inside a lane, so strict comparisons in ascending slot order keep ties on the
+  // lower id.  A lane whose list runs dry refills it from the entries after the last one taken.
+  constexpr int L = VPL < 4 ? VPL : 4;
+  uint32_t lk[L];
+  int ls[L];
+  auto fill = [&](uint32_t after_key, int after_slot) {
+#pragma unroll
+    for (int j = 0; j < L; ++j) lk[j] = 0u, ls[j] = VPL;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      id[i] = lane + 32 * i;
-      if (id[i] >= E) v[i] = -INFINITY, id[i] = 0x7fffffff;
+      const uint32_t x = key[i];
+      if (x == 0u || x > after_key || (x == after_key && i <= after_slot)) continue;
+      bool c[L];
+#pragma unroll
+      for (int j = 0; j < L; ++j) c[j] = x > lk[j];
+#pragma unroll
+      for (int j = L - 1; j > 0; --j) {
+        lk[j] = c[j - 1] ? lk[j - 1] : (c[j] ? x : lk[j]);
+        ls[j] = c[j - 1] ? ls[j - 1] : (c[j] ? i : ls[j]);
+      }
+      if (c[0]) lk[0] = x, ls[0] = i;
     }
+  };
+  fill(0xffffffffu, -1);
+  float my_v = -INFINITY;
+  int my_id = -1;
+  for (int j = 0; j < k; ++j) {
+    // the best head of the warp, then the lowest id among the lanes holding that key
+    const uint32_t m = __reduce_max_sync(0xffffffffu, lk[0]);
+    const unsigned cand = lk[0] == m ? unsigned(lane + 32 * ls[0]) : 0xffffffffu;
+    const int bi = int(__reduce_min_sync(0xffffffffu, cand));
+    if (lane == j) my_v = __uint_as_float((m >> 31) ? (m & 0x7fffffffu) : ~m), my_id = bi;
+    if ((bi & 31) == lane) {
+      const uint32_t tk = lk[0];
+      const int ts = ls[0];
 #pragma unroll
-    for (int r = 0; r < VPL; ++r)
-#pragma unroll
-      for (int i = r & 1; i + 1 < VPL; i += 2)
-        if (v[i + 1] > v[i] || (v[i + 1] == v[i] && id[i + 1] < id[i])) {
-          const float tv = v[i];
-          const int ti = id[i];
-          v[i] = v[i + 1], id[i] = id[i + 1], v[i + 1] = tv, id[i + 1] = ti;
-        }
-    // ... then every round the warp takes the best lane head and that lane pops it
-    for (int j = 0; j < k; ++j) {
-      float bv = v[0];
-      int bi = id[0];
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        const float v2 = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (v2 > bv || (v2 == bv && i2 < bi)) bv = v2, bi = i2;
-      }
-      if (lane == j) my_v = bv, my_id = bi;
-      if ((bi & 31) == lane) {
-#pragma unroll
-        for (int i = 0; i + 1 < VPL; ++i) v[i] = v[i + 1], id[i] = id[i + 1];
-        v[VPL - 1] = -INFINITY, id[VPL - 1] = 0x7fffffff;
-      }
-    }
-  } else {
-    // many logits per lane: each round scans the lane's untaken entries
-    unsigned long long taken = 0;
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E && !((taken >> i) & 1ull) && (bi == 0x7fffffff || v[i] > bv)) bv = v[i], bi = e;
-      }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        const float v2 = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int i2 = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (v2 > bv || (v2 == bv && i2 < bi)) bv = v2, bi = i2;
-      }
-      if (lane == j) my_v = bv, my_id = bi;
-      if ((bi & 31) == lane) taken |= 1ull << (bi >> 5);
+      for (int q = 0; q + 1 < L; ++q) lk[q] = lk[q + 1], ls[q] = ls[q + 1];
+      lk[L - 1] = 0u, ls[L - 1] = VPL;
+      if (lk[0] == 0u) fill(tk, ts);
     }
   }
   const float top = __shfl_sync(0xffffffffu, my_v, 0);
