@@ -663,21 +663,20 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
 }
 
 // ------------------------------------------------------------------- routing
-// One warp per token, kTopkTokensPerWarp tokens per warp, logits in registers.  The expert
-// histogram is counted in shared memory and added to the global one once per CTA and expert
-// (a hot expert of a skewed router would otherwise take one global atomic per selection).
-constexpr int kTopkTokensPerWarp = 4;
-constexpr int kTopkTokensPerCta = 8 * kTopkTokensPerWarp;
+// One warp per token, `tpw` tokens per warp (more for long batches, so that each CTA's
+// histogram covers more selections), logits in registers.  The expert histogram is counted in
+// shared memory and added to the global one once per CTA and expert (a hot expert of a skewed
+// router would otherwise take one global atomic per selection).
 template <int VPL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
-                                                   int norm_topk, int32_t* __restrict__ ids, float* __restrict__ gates,
-                                                   int32_t* __restrict__ counts) {
+                                                   int norm_topk, int tpw, int32_t* __restrict__ ids,
+                                                   float* __restrict__ gates, int32_t* __restrict__ counts) {
   extern __shared__ int32_t hist[];  // [E]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  for (int i = 0; i < kTopkTokensPerWarp; ++i) {
-    const int t = blockIdx.x * kTopkTokensPerCta + i * 8 + warp;
+  for (int i = 0; i < tpw; ++i) {
+    const int t = (blockIdx.x * tpw + i) * 8 + warp;
     if (t >= T) break;
     warp_topk<VPL>(logits + int64_t(t) * E, E, k, norm_topk, lane, ids + int64_t(t) * k, gates + int64_t(t) * k);
     __syncwarp();
@@ -739,24 +738,23 @@ __global__ void __launch_bounds__(kScanThreads) group_scan_kernel(const int32_t*
   }
 }
 
-// Positions inside the experts' segments: kScatterPerThread entries per thread.  Each CTA
-// ranks its entries per expert in shared memory, then reserves one block of positions per
-// expert it touches with a single global atomic.
-constexpr int kScatterPerThread = 8;
-constexpr int kScatterPerCta = 256 * kScatterPerThread;
-__global__ void __launch_bounds__(256) group_scatter_kernel(const int32_t* __restrict__ ids, int n, int E,
+// Positions inside the experts' segments: `ept` (<= kScatterMaxPerThread) entries per thread.
+// Each CTA ranks its entries per expert in shared memory, then reserves one block of positions
+// per expert it touches with a single global atomic.
+constexpr int kScatterMaxPerThread = 8;
+__global__ void __launch_bounds__(256) group_scatter_kernel(const int32_t* __restrict__ ids, int n, int E, int ept,
                                                             int32_t* __restrict__ cursor, int32_t* __restrict__ perm,
                                                             int32_t* __restrict__ inv) {
   extern __shared__ int32_t sh[];  // cnt[E], base[E]
   int32_t *cnt = sh, *base = sh + E;
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
-  int id[kScatterPerThread], local[kScatterPerThread];
-  const int i0 = blockIdx.x * kScatterPerCta + threadIdx.x;
+  int id[kScatterMaxPerThread], local[kScatterMaxPerThread];
+  const int i0 = blockIdx.x * 256 * ept + threadIdx.x;
 #pragma unroll
-  for (int j = 0; j < kScatterPerThread; ++j) {
+  for (int j = 0; j < kScatterMaxPerThread; ++j) {
     const int i = i0 + 256 * j;
-    id[j] = i < n ? ids[i] : -1;
+    id[j] = j < ept && i < n ? ids[i] : -1;
     local[j] = id[j] >= 0 ? atomicAdd(&cnt[id[j]], 1) : 0;
   }
   __syncthreads();
@@ -764,7 +762,7 @@ __global__ void __launch_bounds__(256) group_scatter_kernel(const int32_t* __res
     if (cnt[e]) base[e] = atomicAdd(&cursor[e], cnt[e]);
   __syncthreads();
 #pragma unroll
-  for (int j = 0; j < kScatterPerThread; ++j) {
+  for (int j = 0; j < kScatterMaxPerThread; ++j) {
     if (id[j] < 0) continue;
     const int i = i0 + 256 * j, pos = base[id[j]] + local[j];
     perm[pos] = i;
@@ -937,11 +935,14 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
     }
     case SCION_STAGE_ROUTE: {
       const int vpl = (L->E + 31) / 32;
+      // at least two CTAs per SM for the top-k and one for the scatter, then fewer global atomics
+      const int tpw = max(1, min(4, T / (8 * 2 * num_sms())));
+      const int n = T * L->k, ept = max(1, min(kScatterMaxPerThread, n / (256 * num_sms())));
       cudaError_t e = cudaMemsetAsync(P.counts, 0, sizeof(int32_t) * L->E, s);
       if (e != cudaSuccess) return e;
 #define SCION_TOPK(V) \
-  topk_kernel<V><<<(T + kTopkTokensPerCta - 1) / kTopkTokensPerCta, 256, sizeof(int32_t) * L->E, s>>>( \
-      P.logits, T, L->E, L->k, L->desc.norm_topk, P.ids, P.gates, P.counts)
+  topk_kernel<V><<<(T + 8 * tpw - 1) / (8 * tpw), 256, sizeof(int32_t) * L->E, s>>>( \
+      P.logits, T, L->E, L->k, L->desc.norm_topk, tpw, P.ids, P.gates, P.counts)
       if (vpl <= 1) SCION_TOPK(1);
       else if (vpl <= 2) SCION_TOPK(2);
       else if (vpl <= 4) SCION_TOPK(4);
@@ -954,9 +955,8 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       group_scan_kernel<<<1, kScanThreads, 0, s>>>(P.counts, L->E, P.offsets, P.cursor,
                                                   static_cast<TernTile*>(P.tiles), P.n_tiles);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      const int n = T * L->k;
-      group_scatter_kernel<<<(n + kScatterPerCta - 1) / kScatterPerCta, 256, 2 * sizeof(int32_t) * L->E, s>>>(
-          P.ids, n, L->E, P.cursor, P.perm, P.inv);
+      group_scatter_kernel<<<(n + 256 * ept - 1) / (256 * ept), 256, 2 * sizeof(int32_t) * L->E, s>>>(
+          P.ids, n, L->E, ept, P.cursor, P.perm, P.inv);
       return cudaGetLastError();
     }
     case SCION_STAGE_GATEUP: {
