@@ -39,7 +39,8 @@ using namespace tc;
 
 constexpr int kBM = 128;  // weight rows per tile
 constexpr int kBN = 128;  // tokens per tile
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;   // dense GEMM: TMA warp, MMA warp, 2 idle, 8 epilogue warps
+constexpr int kDenseEpi = 256;  // epilogue threads (two warps per TMEM lane quarter)
 
 // ------------------------------------------------------------- column orders
 __device__ __forceinline__ int perm_pos(int fmt, int col) {  // physical column -> position
@@ -154,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_gemm_kernel(const __grid_co
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDenseStages; ++s) mbar_init(&full[s], 1), mbar_init(&empty[s], 1);
-    for (int i = 0; i < 2; ++i) mbar_init(&acc_full[i], 1), mbar_init(&acc_empty[i], 128);
+    for (int i = 0; i < 2; ++i) mbar_init(&acc_full[i], 1), mbar_init(&acc_empty[i], kDenseEpi);
     mbar_init(&mma_done, 1);
     abort_flag = 0;
     fence_barrier_init();
@@ -231,8 +232,10 @@ __global__ void __launch_bounds__(kThreads, 1) dense_gemm_kernel(const __grid_co
     umma_commit(&mma_done);
     mbar_drain(&mma_done, 0);
   } else if (warp >= 4) {
-    // ---------------- epilogue: TMEM lanes 32q..32q+31 = weight rows
-    const int q = warp - 4;
+    // ---------------- epilogue: TMEM lanes 32q..32q+31 = weight rows; the two warps of a lane
+    // quarter take alternate 16-token chunks.  Each thread writes its row's element of every
+    // token (consecutive rows across the lanes: one contiguous segment per warp and token).
+    const int q = warp & 3, half = (warp - 4) >> 2;
     const int row = q * 32 + lane;
     int li = 0;
     // no abort-flag test in the loop condition: the epilogue threads leave only together, by the vote
@@ -241,33 +244,38 @@ __global__ void __launch_bounds__(kThreads, 1) dense_gemm_kernel(const __grid_co
       if (dt.tok0 >= p.T) continue;
       const DenseUnit u = p.units[dt.unit];
       const int ab = li & 1;
-      if (!named_bar_and(1, 128, mbar_wait(&acc_full[ab], (li >> 1) & 1, &abort_flag, p.err))) break;
+      if (!named_bar_and(1, kDenseEpi, mbar_wait(&acc_full[ab], (li >> 1) & 1, &abort_flag, p.err))) break;
       tc_fence_after();
       const int grow = u.row0 + row;
       const bool rok = grow < u.nrows;
       const uint32_t acc = tmem + 256 * ab + (uint32_t(q * 32) << 16);
       const int nt = min(dt.ntok, p.T - dt.tok0);
-      for (int c = 0; c * 16 < nt; ++c) {
+      const int64_t col = u.col0 + grow;
+      for (int c = half; c * 16 < nt; c += 2) {
         float v0[16], v1[16];
         if (u.epi == kEpiSwiglu)
           tmem_ld16x2(acc + c * 16, acc + 128 + c * 16, v0, v1);
         else
           tmem_ld16(acc + c * 16, v0);
         if (!rok) continue;
+        const int n16 = min(16, nt - c * 16);
+        const int64_t t0 = dt.tok0 + c * 16;
+        if (u.epi == kEpiLogits) {
+          float* dst = p.logits + t0 * p.ld_logits + col;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int tk = c * 16 + i;
-          if (tk >= nt) break;
-          const int64_t tt = dt.tok0 + tk;
-          if (u.epi == kEpiLogits) {
-            p.logits[tt * p.ld_logits + u.col0 + grow] = v0[i];
-          } else if (u.epi == kEpiSwiglu) {
-            p.hz[tt * p.ld_hz + u.col0 + grow] = __float2half_rn(silu_f(v0[i]) * v1[i]);
-          } else if (u.epi == kEpiPlain) {
-            p.hz[tt * p.ld_hz + u.col0 + grow] = __float2half_rn(v0[i]);
-          } else {
-            p.out[tt * p.ld_out + u.col0 + grow] = v0[i];
-          }
+          for (int i = 0; i < 16; ++i)
+            if (i < n16) dst[int64_t(i) * p.ld_logits] = v0[i];
+        } else if (u.epi == kEpiStore) {
+          float* dst = p.out + t0 * p.ld_out + col;
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (i < n16) dst[int64_t(i) * p.ld_out] = v0[i];
+        } else {
+          __half* dst = p.hz + t0 * p.ld_hz + col;
+          const bool sw = u.epi == kEpiSwiglu;
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (i < n16) dst[int64_t(i) * p.ld_hz] = __float2half_rn(sw ? silu_f(v0[i]) * v1[i] : v0[i]);
         }
       }
       // accumulator drained: hand it back to the MMA thread
