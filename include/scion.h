@@ -151,7 +151,8 @@ size_t scion_layer_device_bytes(const scion_layer* layer);
  *   out[t] = sum_{j<k} g_{t,j} E_{e(t,j)}(x_t) + S(x_t) + B (A x_t)
  * with E_e(x) = W_d,e (silu(W_g,e x) * (W_u,e x)), S the shared expert and
  * g, e(t, .) the gates and ids of the top-k router logits.
- * x: device bf16 [T][d]; out: device fp32 [T][d], OVERWRITTEN (no residual add).
+ * x: device bf16 [T][d]; out: device fp32 [T][d], OVERWRITTEN (no residual add); both
+ * 16-byte aligned.
  * 0 <= T <= max_tokens (T = 0 is a no-op).  Batches of at most 64 tokens stream the
  * weights through warp-level MMA kernels; larger batches (layers created with
  * max_tokens > 64) run as tcgen05 grouped GEMMs.  Calls on one handle must not
@@ -159,8 +160,18 @@ size_t scion_layer_device_bytes(const scion_layer* layer);
  * 16..64 tokens fork the dense down projection onto a stream owned by the handle and
  * join it back (events) before the call's work on `stream` ends; stream capture into
  * a CUDA graph records the fork and the join.
- * EINVAL on a null pointer or T out of range; ECUDA if a launch fails. */
+ * EINVAL on a null or misaligned pointer or T out of range; ECUDA if a launch fails. */
 int scion_moe_forward(const void* x, int T, const scion_layer* layer, float* out, void* stream);
+
+/* The block added to the residual stream ("Scion: ternary MoE quantization with trained
+ * corrections", The idea: the block output and its correction are added to the residual
+ * stream):  out[t] = resid[t] + block(x_t), with block(x_t) the output of scion_moe_forward.
+ * resid: device fp32 [T][d], 16-byte aligned; it may be the same buffer as out (in-place
+ * accumulation), otherwise it is only read.  The residual enters where out is first written
+ * (the first kernel of the call), so the cost is one read of resid.
+ * EINVAL on a null or misaligned pointer or T out of range; ECUDA if a launch fails. */
+int scion_moe_forward_residual(const void* x, int T, const scion_layer* layer, const float* resid, float* out,
+                               void* stream);
 
 /* Tuning options of a layer (scion_layer_set_option).
  *  SCION_OPT_STREAM_MIN_TOKENS (default 16): batches of at least this many tokens (and at

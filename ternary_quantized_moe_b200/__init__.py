@@ -27,6 +27,7 @@ __all__ = [
     "scion_moe_forward_host", "scion_moe_forward_debug", "Layer", "library_path", "EXPORTS",
     "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "STAGES", "scion_layer_check",
     "scion_router_logits_static", "scion_layer_set_option", "SCION_OPT_STREAM_MIN_TOKENS",
+    "scion_moe_forward_residual",
 ]
 
 SCION_PQ2_0 = 0
@@ -44,7 +45,7 @@ EXPORTS = (
     "scion_pack_device", "scion_unpack_device", "scion_layer_create", "scion_layer_destroy",
     "scion_layer_device_bytes", "scion_moe_forward", "scion_moe_forward_host", "scion_moe_forward_debug",
     "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "scion_layer_check",
-    "scion_router_logits_static", "scion_layer_set_option",
+    "scion_router_logits_static", "scion_layer_set_option", "scion_moe_forward_residual",
 )
 SCION_OPT_STREAM_MIN_TOKENS = 1
 STAGES = ("router_f32", "xproj", "route", "gateup", "down_routed", "down_dense", "x16", "combine")
@@ -98,6 +99,7 @@ def _load():
             "scion_layer_destroy": (None, [vp]),
             "scion_layer_device_bytes": (C.c_size_t, [vp]),
             "scion_moe_forward": (ci, [vp, ci, vp, vp, vp]),
+            "scion_moe_forward_residual": (ci, [vp, ci, vp, vp, vp, vp]),
             "scion_moe_forward_host": (ci, [vp, ci, vp, vp, vp]),
             "scion_moe_forward_debug": (ci, [vp, ci, vp, vp, C.POINTER(_Debug), vp]),
             "scion_profile_begin": (ci, [ci]),
@@ -305,6 +307,16 @@ def scion_moe_forward(x, T: int, layer: Layer, out, stream=None) -> None:
     st = _load().scion_moe_forward(_dptr(x, "x", (torch.bfloat16,)), int(T), C.c_void_p(layer.handle),
                                    _dptr(out, "out", (torch.float32,)), _stream(stream))
     _check(st, "scion_moe_forward")
+
+
+def scion_moe_forward_residual(x, T: int, layer: Layer, resid, out, stream=None) -> None:
+    """x: bf16 CUDA [T, d]; resid: fp32 CUDA [T, d] (may be `out` itself); out = resid + block(x)."""
+    import torch
+
+    st = _load().scion_moe_forward_residual(_dptr(x, "x", (torch.bfloat16,)), int(T), C.c_void_p(layer.handle),
+                                            _dptr(resid, "resid", (torch.float32,)),
+                                            _dptr(out, "out", (torch.float32,)), _stream(stream))
+    _check(st, "scion_moe_forward_residual")
 
 
 def scion_moe_forward_host(x_host, T: int, layer: Layer, out_host, stream=None) -> None:

@@ -42,7 +42,8 @@ struct XProjArgs {
   __half* xfrag;  // [T][d/128][SCION_BROW] fp16 in fragment order + group sums
   __half* h;      // [T*k][F/128][SCION_BROW] expert hidden: group-sum tails zeroed here
   int k, GF;
-  float* out;     // zeroed here
+  float* out;     // set here to the residual (or zero)
+  const float* resid;  // nullptr: out starts at zero; may equal out (then out is left as it is)
 };
 
 // One CTA = (unit, 512-column chunk); 8 warps x 64 columns.  NT = token tiles of 8.  The
@@ -94,7 +95,12 @@ __device__ __forceinline__ void xproj_aux(const XProjArgs& a, int aux, int n_aux
   }
   const int tid = aux * kXThreads + threadIdx.x, nth = n_aux * kXThreads;
   float4* o4 = reinterpret_cast<float4*>(a.out);
-  for (int64_t i = tid; i < int64_t(a.T) * a.d / 4; i += nth) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (!a.resid) {
+    for (int64_t i = tid; i < int64_t(a.T) * a.d / 4; i += nth) o4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  } else if (a.resid != a.out) {
+    const float4* r4 = reinterpret_cast<const float4*>(a.resid);
+    for (int64_t i = tid; i < int64_t(a.T) * a.d / 4; i += nth) o4[i] = r4[i];
+  }
   // the expert hidden's group sums are accumulated by the gate/up epilogue
   for (int i = tid; i < a.T * a.k * a.GF; i += nth)
     *reinterpret_cast<float4*>(a.h + int64_t(i) * SCION_BROW + 128) = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -494,9 +500,10 @@ __global__ void unfrag_kernel(int fmt, const __half* __restrict__ src, int64_t n
 }  // namespace
 
 // ------------------------------------------------------------------- launchers
-cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, int unit0, int n_units,
-                         bool aux, cudaStream_t s) {
+cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, const float* resid,
+                         int unit0, int n_units, bool aux, cudaStream_t s) {
   XProjArgs a;
+  a.resid = resid;
   a.x = x;
   a.T = T, a.d = L->d, a.E = L->E, a.Fs = L->Fs, a.r = L->r, a.Kd = L->Kd, a.fmt = L->fmt;
   a.w_router = static_cast<const __nv_bfloat16*>(L->desc.w_router);

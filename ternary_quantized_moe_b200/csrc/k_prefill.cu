@@ -66,27 +66,39 @@ __device__ __forceinline__ float pq2_pos_scale(int p) {
   return 1.0f / float(1 << (2 * (s < 5 ? s : s - 5)));
 }
 
-// x (bf16) -> fp16 in the container's column order (PQ2_0: times the factor of its position);
-// one thread per 16 columns (PQ2_0) or per 128-column group (PTQ1_0).
+// Column held by position p of a 128-column group (the inverse of perm_pos).
+__device__ __forceinline__ int pos_col(int fmt, int p) {
+  if (fmt == SCION_PQ2_0) return (p & ~15) | (((p & 15) >> 1) + 8 * (p & 1));
+  const int half = p >> 6, r = p & 63;
+  if (r >= 60) return 120 + 4 * half + (r - 60);
+  const int i = r / 10, rem = r % 10;
+  return 5 * (12 * half + 2 * i + (rem & 1)) + (rem >> 1);
+}
+
+// x (bf16) -> fp16 in the container's column order (PQ2_0: times the factor of its position).
+// A warp takes two 128-column groups per step: coalesced 16-byte loads into shared memory,
+// then each lane gathers the columns of its 8 output positions and stores 16 bytes.
 template <int FMT>
-__global__ void x16_kernel(const __nv_bfloat16* __restrict__ x, int64_t n, __half* __restrict__ xp) {
-  constexpr int W = FMT == SCION_PQ2_0 ? 16 : 128;
-  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n / W) return;
-  const uint4* src = reinterpret_cast<const uint4*>(x + i * W);
-  uint4* dst = reinterpret_cast<uint4*>(xp + i * W);
-  __align__(16) __nv_bfloat16 in[W];
-  __align__(16) __half outv[W];
+__global__ void __launch_bounds__(256) x16_kernel(const __nv_bfloat16* __restrict__ x, int64_t n_groups,
+                                                  __half* __restrict__ xp) {
+  __shared__ __align__(16) __nv_bfloat16 buf[8][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gl = lane >> 4, p0 = 8 * (lane & 15);  // group of the pair, first output position
+  const int64_t n_pairs = (n_groups + 1) / 2;
+  for (int64_t i = int64_t(blockIdx.x) * 8 + warp; i < n_pairs; i += int64_t(gridDim.x) * 8) {
+    const bool ok = 2 * i + gl < n_groups;  // an odd group count leaves the last pair half empty
+    if (ok) *reinterpret_cast<uint4*>(&buf[warp][8 * lane]) = __ldg(reinterpret_cast<const uint4*>(x + i * 256) + lane);
+    __syncwarp();
+    __align__(16) __half o[8];
 #pragma unroll
-  for (int j = 0; j < W / 8; ++j) reinterpret_cast<uint4*>(in)[j] = src[j];
-#pragma unroll
-  for (int col = 0; col < W; ++col) {
-    const int p = perm_pos(FMT, col) & (W - 1);
-    const float v = __bfloat162float(in[col]);
-    outv[p] = __float2half_rn(FMT == SCION_PQ2_0 ? v * pq2_pos_scale(p) : v);
+    for (int e = 0; e < 8; ++e) {
+      const int p = p0 + e;
+      const float v = __bfloat162float(buf[warp][128 * gl + pos_col(FMT, p)]);
+      o[e] = __float2half_rn(FMT == SCION_PQ2_0 ? v * pq2_pos_scale(p) : v);
+    }
+    if (ok) reinterpret_cast<uint4*>(xp + i * 256)[lane] = *reinterpret_cast<const uint4*>(o);
+    __syncwarp();
   }
-#pragma unroll
-  for (int j = 0; j < W / 8; ++j) dst[j] = reinterpret_cast<uint4*>(outv)[j];
 }
 
 // ---------------------------------------------------------------- dense GEMM
@@ -112,6 +124,7 @@ struct DenseParams {
   float* logits;  int ld_logits;
   __half* hz;     int ld_hz;
   float* out;     int ld_out;
+  const float* resid;  // kEpiStore: added to the stored value (same layout as out; may equal out)
   int* err;
 };
 
@@ -267,9 +280,16 @@ __global__ void __launch_bounds__(kThreads, 1) dense_gemm_kernel(const __grid_co
             if (i < n16) dst[int64_t(i) * p.ld_logits] = v0[i];
         } else if (u.epi == kEpiStore) {
           float* dst = p.out + t0 * p.ld_out + col;
+          if (p.resid) {
+            const float* rs = p.resid + t0 * p.ld_out + col;
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (i < n16) dst[int64_t(i) * p.ld_out] = v0[i];
+            for (int i = 0; i < 16; ++i)
+              if (i < n16) dst[int64_t(i) * p.ld_out] = v0[i] + rs[int64_t(i) * p.ld_out];
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (i < n16) dst[int64_t(i) * p.ld_out] = v0[i];
+          }
         } else {
           __half* dst = p.hz + t0 * p.ld_hz + col;
           const bool sw = u.epi == kEpiSwiglu;
@@ -857,17 +877,18 @@ cudaError_t configure_prefill_kernels() {
   return cudaSuccess;
 }
 
-// out[t] (= dense part, or 0 when the layer has no shared expert and no correction)
-// += sum over slots j < k of y[inv[t*k + j]], in slot order.  One CTA per token.
+// out[t] = base[t] + sum over slots j < k (in slot order) of gates[t][j] y[inv[t k + j]];
+// base = out (the dense down projection stored its part there, residual included), the
+// residual (a layer without shared expert and correction), or zero.  One CTA per token.
 __global__ void __launch_bounds__(256) combine_kernel(const __half* __restrict__ y, const int32_t* __restrict__ inv,
-                                                     const float* __restrict__ gates, int k, int d, int has_dense,
-                                                     float* __restrict__ out) {
+                                                     const float* __restrict__ gates, int k, int d,
+                                                     const float* base, float* out) {
   const int t = blockIdx.x;
   const int32_t* iv = inv + int64_t(t) * k;
   const float* gt = gates + int64_t(t) * k;
   float4* o = reinterpret_cast<float4*>(out + int64_t(t) * d);
   for (int c4 = threadIdx.x; c4 < d / 4; c4 += blockDim.x) {
-    float4 acc = has_dense ? o[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 acc = base ? reinterpret_cast<const float4*>(base + int64_t(t) * d)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j = 0; j < k; ++j) {
       const uint2 raw = reinterpret_cast<const uint2*>(y + int64_t(iv[j]) * d)[c4];
       const float2 lo = __half22float2(u32_as_h2(raw.x)), hi = __half22float2(u32_as_h2(raw.y));
@@ -917,15 +938,17 @@ void prefill_units(const scion_layer* L, void* xunits_host, int* n_x, void* duni
 int prefill_max_units(const scion_layer* L) { return (L->E + 127) / 128 + (L->Fs + 127) / 128 + (L->r + 127) / 128 + L->d / 128; }
 
 cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfloat16* x, int T, float* out,
-                                 cudaStream_t s) {
+                                 const float* resid, cudaStream_t s) {
   const PrefillState& P = *L->pre;
   switch (stage) {
     case SCION_STAGE_X16: {
       const int64_t n = int64_t(T) * L->d;
+      const int64_t groups = n / 128, pairs = (groups + 1) / 2;
+      const unsigned grid = unsigned(std::min((pairs + 7) / 8, int64_t(num_sms()) * 8));
       if (L->fmt == SCION_PQ2_0)
-        x16_kernel<SCION_PQ2_0><<<unsigned((n / 16 + 255) / 256), 256, 0, s>>>(x, n, P.x16);
+        x16_kernel<SCION_PQ2_0><<<grid, 256, 0, s>>>(x, groups, P.x16);
       else
-        x16_kernel<SCION_PTQ1_0><<<unsigned((n / 128 + 127) / 128), 128, 0, s>>>(x, n, P.x16);
+        x16_kernel<SCION_PTQ1_0><<<grid, 256, 0, s>>>(x, groups, P.x16);
       return cudaGetLastError();
     }
     case SCION_STAGE_XPROJ: {
@@ -937,6 +960,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       dp.n_units = P.n_xunits;
       dp.n_units2 = (L->desc.router_fp32 ? 0 : (L->E + 127) / 128) + (L->Fs + 127) / 128;
       dp.logits = P.logits, dp.ld_logits = L->E, dp.hz = P.hz, dp.ld_hz = L->Kd, dp.out = nullptr, dp.ld_out = 0;
+      dp.resid = nullptr;
       dp.err = L->err;
       dense_gemm_kernel<<<dense_grid(dp), kThreads, kDenseSmem, s>>>(dp);
       return cudaGetLastError();
@@ -982,7 +1006,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       return cudaGetLastError();
     }
     case SCION_STAGE_COMBINE: {
-      combine_kernel<<<T, 256, 0, s>>>(P.y, P.inv, P.gates, L->k, L->d, P.n_dunits > 0, out);
+      combine_kernel<<<T, 256, 0, s>>>(P.y, P.inv, P.gates, L->k, L->d, P.n_dunits > 0 ? out : resid, out);
       return cudaGetLastError();
     }
     case SCION_STAGE_DOWN_DENSE: {
@@ -993,6 +1017,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       dp.units = static_cast<const DenseUnit*>(P.dunits), dp.K = L->Kd, dp.T = T, dp.ab_bf16 = 0;
       dp.n_units = P.n_dunits, dp.n_units2 = 0;
       dp.logits = nullptr, dp.ld_logits = 0, dp.hz = nullptr, dp.ld_hz = 0, dp.out = out, dp.ld_out = L->d;
+      dp.resid = resid;
       dp.err = L->err;
       dense_gemm_kernel<<<dense_grid(dp), kThreads, kDenseSmem, s>>>(dp);
       return cudaGetLastError();

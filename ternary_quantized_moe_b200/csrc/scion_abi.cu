@@ -169,21 +169,22 @@ struct StageScope {
   } while (0)
 
 // Whole batch on the tensor-core path (T > SCION_TDEC).
-int forward_prefill(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, cudaStream_t s) {
+int forward_prefill(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, const float* resid,
+                    cudaStream_t s) {
   if (L->desc.router_fp32)
     SCION_STAGE(SCION_STAGE_ROUTER_F32, scion::launch_router_f32(L, x, T, L->pre->logits, s));
-  SCION_STAGE(SCION_STAGE_X16, scion::launch_prefill_stage(SCION_STAGE_X16, L, x, T, out, s));
-  SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_prefill_stage(SCION_STAGE_XPROJ, L, x, T, out, s));
-  SCION_STAGE(SCION_STAGE_ROUTE, scion::launch_prefill_stage(SCION_STAGE_ROUTE, L, x, T, out, s));
-  SCION_STAGE(SCION_STAGE_GATEUP, scion::launch_prefill_stage(SCION_STAGE_GATEUP, L, x, T, out, s));
-  SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_prefill_stage(SCION_STAGE_DOWN_DENSE, L, x, T, out, s));
-  SCION_STAGE(SCION_STAGE_DOWN_ROUTED, scion::launch_prefill_stage(SCION_STAGE_DOWN_ROUTED, L, x, T, out, s));
-  SCION_STAGE(SCION_STAGE_COMBINE, scion::launch_prefill_stage(SCION_STAGE_COMBINE, L, x, T, out, s));
+  SCION_STAGE(SCION_STAGE_X16, scion::launch_prefill_stage(SCION_STAGE_X16, L, x, T, out, resid, s));
+  SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_prefill_stage(SCION_STAGE_XPROJ, L, x, T, out, resid, s));
+  SCION_STAGE(SCION_STAGE_ROUTE, scion::launch_prefill_stage(SCION_STAGE_ROUTE, L, x, T, out, resid, s));
+  SCION_STAGE(SCION_STAGE_GATEUP, scion::launch_prefill_stage(SCION_STAGE_GATEUP, L, x, T, out, resid, s));
+  SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_prefill_stage(SCION_STAGE_DOWN_DENSE, L, x, T, out, resid, s));
+  SCION_STAGE(SCION_STAGE_DOWN_ROUTED, scion::launch_prefill_stage(SCION_STAGE_DOWN_ROUTED, L, x, T, out, resid, s));
+  SCION_STAGE(SCION_STAGE_COMBINE, scion::launch_prefill_stage(SCION_STAGE_COMBINE, L, x, T, out, resid, s));
   return SCION_OK;
 }
 
 // One pass of T <= SCION_TDEC tokens.
-int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, cudaStream_t s) {
+int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, const float* resid, cudaStream_t s) {
   if (L->desc.router_fp32) SCION_STAGE(SCION_STAGE_ROUTER_F32, scion::launch_router_f32(L, x, T, L->logits, s));
   const bool ring = T >= L->stream_min_tokens;
   // Batches on the ring kernels split the dense work off the expert path: the caller's stream
@@ -192,7 +193,7 @@ int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out
   // beside routing and the expert kernels; the caller's stream joins it at the end.
   const bool side = ring && L->Kdense;
   const int nx_main = side ? L->n_xrouter : L->n_xunits;
-  SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_xproj(L, x, T, out, 0, nx_main, true, s));
+  SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_xproj(L, x, T, out, resid, 0, nx_main, true, s));
   if (side) {
     cudaError_t e = cudaEventRecord(L->ev_x, s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(L->side, L->ev_x, 0);
@@ -200,7 +201,7 @@ int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out
     {
       cudaStream_t s = L->side;  // SCION_STAGE launches and records on `s`
       SCION_STAGE(SCION_STAGE_XPROJ,
-                  scion::launch_xproj(L, x, T, out, L->n_xrouter, L->n_xunits - L->n_xrouter, false, s));
+                  scion::launch_xproj(L, x, T, out, nullptr, L->n_xrouter, L->n_xunits - L->n_xrouter, false, s));
       SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
     }
     if ((e = cudaEventRecord(L->ev_dense, L->side)) != cudaSuccess) return cuda_status(e);
@@ -344,19 +345,35 @@ extern "C" void scion_layer_destroy(scion_layer* layer) {
 
 extern "C" size_t scion_layer_device_bytes(const scion_layer* layer) { return layer ? layer->device_bytes : 0; }
 
-extern "C" int scion_moe_forward(const void* x, int T, const scion_layer* L, float* out, void* stream) {
+namespace {
+int forward_any(const void* x, int T, const scion_layer* L, const float* resid, float* out, void* stream) {
   if (!L || T < 0 || T > L->max_tokens) return SCION_EINVAL;
   if (T == 0) return SCION_OK;
   if (!x || !out) return SCION_EINVAL;
+  // 16-byte accesses
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(resid)) & 15)
+    return SCION_EINVAL;
   cudaStream_t s = as_stream(stream);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  if (T > SCION_TDEC && L->pre) return forward_prefill(L, xb, T, out, s);
+  if (T > SCION_TDEC && L->pre) return forward_prefill(L, xb, T, out, resid, s);
   for (int t0 = 0; t0 < T; t0 += SCION_TDEC) {
     const int n = T - t0 < SCION_TDEC ? T - t0 : SCION_TDEC;
-    int st = forward_pass(L, xb + int64_t(t0) * L->d, n, out + int64_t(t0) * L->d, s);
+    int st = forward_pass(L, xb + int64_t(t0) * L->d, n, out + int64_t(t0) * L->d,
+                          resid ? resid + int64_t(t0) * L->d : nullptr, s);
     if (st != SCION_OK) return st;
   }
   return SCION_OK;
+}
+}  // namespace
+
+extern "C" int scion_moe_forward(const void* x, int T, const scion_layer* L, float* out, void* stream) {
+  return forward_any(x, T, L, nullptr, out, stream);
+}
+
+extern "C" int scion_moe_forward_residual(const void* x, int T, const scion_layer* L, const float* resid, float* out,
+                                          void* stream) {
+  if (!resid) return SCION_EINVAL;
+  return forward_any(x, T, L, resid, out, stream);
 }
 
 extern "C" int scion_moe_forward_host(const void* x_host, int T, const scion_layer* L, float* out_host, void* stream) {

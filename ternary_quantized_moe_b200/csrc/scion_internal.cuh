@@ -150,8 +150,8 @@ cudaError_t launch_slot_info(const scion_layer* L, cudaStream_t s);
 // Units [unit0, unit0 + n_units) of the layer's x-projection table (router units first, then
 // shared gate/up, then correction A); `aux` adds the CTAs that write x's fragment rows and
 // clear out and the hidden's group-sum tails.
-cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, int unit0, int n_units,
-                         bool aux, cudaStream_t s);
+cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, const float* resid,
+                         int unit0, int n_units, bool aux, cudaStream_t s);
 cudaError_t launch_gateup(const scion_layer* L, const __nv_bfloat16* x, int T, cudaStream_t s);
 cudaError_t launch_down_routed(const scion_layer* L, int T, float* out, cudaStream_t s);
 cudaError_t launch_down_dense(const scion_layer* L, int T, float* out, cudaStream_t s);
@@ -173,7 +173,7 @@ int prefill_max_units(const scion_layer* L);
 void prefill_units(const scion_layer* L, void* xunits_host, int* n_x, void* dunits_host, int* n_d);
 cudaError_t launch_unperm_prefill(int fmt, const __half* src, int64_t n, __half* dst, cudaStream_t s);
 cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfloat16* x, int T, float* out,
-                                 cudaStream_t s);
+                                 const float* resid, cudaStream_t s);
 
 // Launch with programmatic dependent launch: the kernel may start while its predecessor
 // on the stream drains; it must execute pdl_wait() before touching anything the

@@ -250,6 +250,29 @@ def test_topk_one_lane_holds_the_top(E, k, T):
     check_output(got, ref)
 
 
+@pytest.mark.parametrize("T,max_tokens,dense,in_place", [(5, 64, True, False), (40, 64, True, True),
+                                                          (64, 64, False, True), (150, 150, True, False),
+                                                          (300, 300, False, True), (300, 300, True, True)])
+def test_forward_residual(T, max_tokens, dense, in_place):
+    """out = resid + block(x) on the decode kernels (split-K and ring passes) and the
+    tensor-core path (with and without the shared expert and correction, whose dense down
+    projection adds the residual; without them the combine does), in place and not."""
+    cfg = small("rs", synth.PTQ1_0, False, E=16, k=4, Fs=128 if dense else 0, r=16 if dense else 0)
+    L, banks, ol, x = _case(cfg, T)
+    layer = device_layer(cfg, L, banks, max_tokens)
+    rng = np.random.default_rng(77 + T)
+    resid_h = rng.standard_normal((T, cfg.d)).astype(np.float32)
+    resid = torch.from_numpy(resid_h).to(DEV)
+    out = resid if in_place else torch.full((T, cfg.d), float("nan"), dtype=torch.float32, device=DEV)
+    tq.scion_moe_forward_residual(u16_to_dev(x, torch.bfloat16, DEV), T, layer, resid, out)
+    torch.cuda.synchronize()
+    assert tq.scion_layer_check(layer) == 0
+    if not in_place:
+        np.testing.assert_array_equal(resid.cpu().numpy(), resid_h)  # only read
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(out.cpu().numpy().astype(np.float64) - resid_h.astype(np.float64), ref)
+
+
 @pytest.mark.parametrize("T", [64, 65, 150])
 def test_forward_multi_pass(T):
     """Batches above one decode pass (64 tokens) run in passes; ragged tails included."""
@@ -272,6 +295,11 @@ def test_empty_batch_and_limits():
     assert float(out.abs().sum()) == 0.0
     with pytest.raises(tq.ScionError) as ei:
         tq.scion_moe_forward(xd, 5, layer, out)
+    assert ei.value.status == tq.SCION_EINVAL
+    # out must be 16-byte aligned (the kernels store it with 16-byte accesses)
+    flat = torch.zeros(4 * cfg.d + 1, device=DEV)
+    with pytest.raises(tq.ScionError) as ei:
+        tq.scion_moe_forward(xd, 4, layer, flat[1:].view(4, cfg.d))
     assert ei.value.status == tq.SCION_EINVAL
 
 
