@@ -100,6 +100,10 @@ def _load():
             lib.oracle_shared.argtypes = [C.POINTER(_Layer), vp, ci, vp, vp]
             lib.oracle_corr.restype = ci
             lib.oracle_corr.argtypes = [C.POINTER(_Layer), vp, ci, vp, vp]
+            lib.oracle_f64_to_f16_nonneg.restype = C.c_uint16
+            lib.oracle_f64_to_f16_nonneg.argtypes = [C.c_double]
+            lib.oracle_quantize.restype = ci
+            lib.oracle_quantize.argtypes = [ci, vp, i64, ci, vp, vp]
             _lib = lib
     return _lib
 
@@ -319,6 +323,30 @@ def corr(layer: OracleLayer, x: np.ndarray):
     if st != OK:
         raise RuntimeError("oracle_corr: %d" % st)
     return z, y
+
+
+ABSMEAN = 0
+LLOYD = 1
+
+
+def f64_to_f16(v: float) -> int:
+    """Nearest binary16 bit pattern of a finite v >= 0 (ties to even)."""
+    return int(_load().oracle_f64_to_f16_nonneg(float(v)))
+
+
+def quantize(method: int, w: np.ndarray, iters: int = 30):
+    """Ternary codes int8 [n, 128] and fp16 scales (uint16 bits) [n] of fp32 groups w [n, 128]
+    ("Scion: ternary MoE quantization with trained corrections", Findings; "Scion-35B-A3B" model
+    card, Highlights): ABSMEAN (s = mean |w|, codes by rounding w / s) or LLOYD (centroid /
+    nearest-level rounds from the absmean start).  Decisions in fp64; see scion_oracle.c."""
+    w = np.ascontiguousarray(w, dtype=np.float32).reshape(-1, 128)
+    n = w.shape[0]
+    codes = np.empty((n, 128), np.int8)
+    scales = np.empty(n, np.uint16)
+    st = _load().oracle_quantize(int(method), _ptr(w), n, int(iters), _ptr(codes), _ptr(scales))
+    if st != OK:
+        raise ValueError("oracle_quantize failed: %d" % st)
+    return codes, scales
 
 
 def cores_used() -> int:

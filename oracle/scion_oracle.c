@@ -598,3 +598,84 @@ int oracle_corr(const oracle_layer* L, const uint16_t* x, int T, double* z_out, 
   free(xv);
   return ORACLE_OK;
 }
+
+/* ------------------------------------------------------------- quantizers */
+/* Float -> ternary quantizers of groups of 128 consecutive weights ("Scion: ternary MoE
+ * quantization with trained corrections", Findings: the deployable Lloyd quantizer against
+ * one-shot absmean; "Scion-35B-A3B" model card, Highlights: ternary Lloyd g128).  Each group
+ * gets codes in {-1, 0, +1} and one scale s, w ~ code * s.
+ *   absmean: s = mean |w| over the group; code = w / s rounded half away from zero and
+ *            clamped to [-1, 1], i.e. sign(w) where 2|w| >= s, else 0.
+ *   Lloyd:   Lloyd's algorithm for the levels {-s, 0, +s}: starting from the absmean codes,
+ *            alternately set s to the centroid of the nonzero cells (mean |w| over codes != 0)
+ *            and re-partition to the nearest level (the same rule as above), until the codes
+ *            stop changing or `iters` rounds have run; the stored s is the centroid of the
+ *            final codes.
+ * Decisions are taken in fp64; the scale is stored as the nearest binary16. */
+
+/* Nearest binary16 (ties to even) of a finite v >= 0, as its bit pattern (+inf at >= 65520). */
+uint16_t oracle_f64_to_f16_nonneg(double v) {
+  if (!(v > 0.0)) return 0;
+  if (v >= 65520.0) return 0x7c00;
+  int e;
+  frexp(v, &e);                              /* v = m 2^e with 0.5 <= m < 1: v in [2^(e-1), 2^e) */
+  const int E = e - 1;                       /* unbiased exponent of v */
+  const int q = E >= -14 ? E - 10 : -24;     /* weight of the last fraction bit (normal / subnormal) */
+  double r = nearbyint(ldexp(v, -q));        /* v in units of that bit, rounded half to even */
+  if (q == -24) return (uint16_t)r;          /* subnormal (r = 1024 is the smallest normal) */
+  int Eo = E;
+  if (r >= 2048.0) r /= 2.0, Eo += 1;        /* rounding carried into the next binade */
+  if (Eo > 15) return 0x7c00;
+  return (uint16_t)(((Eo + 15) << 10) | ((int)r - 1024));
+}
+
+static int quant_finite(const float* w) {
+  for (int i = 0; i < 128; i++)
+    if (!isfinite(w[i])) return 0;
+  return 1;
+}
+
+/* sign(w) where 2|w| >= s, else 0; returns how many codes differ from c_old (if given). */
+static int quant_partition(const float* w, double s, int8_t* c) {
+  int changed = 0;
+  for (int i = 0; i < 128; i++) {
+    const double a = fabs((double)w[i]);
+    const int8_t v = (w[i] != 0.0f && 2.0 * a >= s) ? (w[i] > 0.0f ? 1 : -1) : 0;
+    changed += v != c[i];
+    c[i] = v;
+  }
+  return changed;
+}
+
+static double quant_centroid(const float* w, const int8_t* c) {
+  double sum = 0.0;
+  int n = 0;
+  for (int i = 0; i < 128; i++)
+    if (c[i]) sum += fabs((double)w[i]), n++;
+  return n ? sum / n : 0.0;
+}
+
+int oracle_quantize(int method, const float* w, int64_t n_groups, int iters, int8_t* codes, uint16_t* scales) {
+  if ((method != 0 && method != 1) || n_groups < 0 || iters < 0) return ORACLE_EINVAL;
+  for (int64_t g = 0; g < n_groups; g++)
+    if (!quant_finite(w + g * 128)) return ORACLE_EINVAL;
+#pragma omp parallel for schedule(static)
+  for (int64_t g = 0; g < n_groups; g++) {
+    const float* wg = w + g * 128;
+    int8_t* c = codes + g * 128;
+    double s = 0.0;
+    for (int i = 0; i < 128; i++) s += fabs((double)wg[i]);
+    s /= 128.0;
+    for (int i = 0; i < 128; i++) c[i] = 0;
+    quant_partition(wg, s, c);
+    if (method == 1) {
+      for (int it = 0; it < iters; it++) {
+        s = quant_centroid(wg, c);
+        if (quant_partition(wg, s, c) == 0) break;
+      }
+      s = quant_centroid(wg, c);
+    }
+    scales[g] = oracle_f64_to_f16_nonneg(s);
+  }
+  return ORACLE_OK;
+}
