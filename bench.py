@@ -441,8 +441,56 @@ def run_gpu(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_quantize(args):
+    """The float -> ternary quantizers over one 35B-A3B-class layer's expert weights (256 experts x
+    (gate, up, down) x 512 x 2048 = 805M N(0,1) fp32 weights, 3.2 GB): one step = one call of the
+    Lloyd quantizer (30 rounds at most) over all groups.  Device-timed with CUDA events; the
+    roofline is the HBM traffic (fp32 in, int8 codes and fp16 scales out)."""
+    import torch
+
+    import ternary_quantized_moe_b200 as tq
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    n = 256 * 3 * 512 * 2048 // 128
+    g = torch.Generator(device=dev)
+    g.manual_seed(4242)
+    w = torch.randn((n, 128), generator=g, device=dev)
+    codes = torch.empty((n, 128), dtype=torch.int8, device=dev)
+    scales = torch.empty(n, dtype=torch.int16, device=dev)
+    bytes_per_call = n * 128 * 5 + n * 2
+    res = {}
+    for name, method in (("lloyd", tq.SCION_QUANT_LLOYD), ("absmean", tq.SCION_QUANT_ABSMEAN)):
+        for _ in range(max(3, args.warmup)):
+            tq.scion_quantize_device(method, w, codes, scales, iters=30)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            tq.scion_quantize_device(method, w, codes, scales, iters=30)
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        res[name] = {"ms_per_call": ms, "weights_per_s": n * 128 / (ms / 1000.0),
+                     "hbm_gbs": bytes_per_call / (ms / 1000.0) / 1e9}
+    line = {"metric": "ternary quantizer weights/s (Lloyd g128)", "value": res["lloyd"]["weights_per_s"],
+            "unit": "weights/s", "n_gpus": 1, "steps": args.steps, "warmup": max(3, args.warmup),
+            "ms_per_step": res["lloyd"]["ms_per_call"], "higher_is_better": True, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": "quantize_a3b_experts", "weights": n * 128,
+                                             "l2": "inputs larger than L2: 3.2 GB"},
+            "roofline": {"bound": "hbm", "achieved": res["lloyd"]["hbm_gbs"], "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": res["lloyd"]["hbm_gbs"] / peaks["hbm_gbs"], "traffic": None,
+                         "peak_source": peak_src},
+            "absmean": res["absmean"]}
+    print(json.dumps(line))
+
+
 def main():
     args = parse()
+    if args.workload == "quantize_a3b_experts":
+        run_quantize(args)
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

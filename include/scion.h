@@ -86,6 +86,23 @@ int scion_pack_device(int fmt, const int8_t* codes, const uint16_t* scales, int6
 int scion_unpack_device(int fmt, const uint8_t* in, int64_t n_groups, int8_t* codes, uint16_t* scales,
                         int64_t* bad_count, void* stream);
 
+/* Float -> ternary quantizers ("Scion: ternary MoE quantization with trained corrections",
+ * Findings: the deployable Lloyd quantizer against one-shot absmean; "Scion-35B-A3B" model
+ * card, Highlights: ternary Lloyd g128).  w: device fp32, n_groups groups of 128 consecutive
+ * weights (a row-major [rows][K] matrix with K % 128 == 0 is rows * K / 128 groups along K),
+ * 16-byte aligned, finite, |w| <= 65504.  Writes codes (device int8 [n_groups][128], 4-byte
+ * aligned) in {-1, 0, +1} and scale_f16 (device binary16 bits [n_groups]) such that
+ * w ~ code * scale; feed them to scion_pack_device for the PQ2_0 / PTQ1_0 containers.
+ *   SCION_QUANT_ABSMEAN: s = mean |w| of the group; code = sign(w) where 2|w| >= s, else 0.
+ *   SCION_QUANT_LLOYD:   Lloyd's algorithm for the levels {-s, 0, +s} from the absmean start:
+ *     s = mean |w| over the nonzero codes, then every code re-chosen by the rule above, until
+ *     no code changes or `iters` (0..1000) rounds ran; s = mean |w| over the final nonzero codes.
+ * Sums and decisions in fp64; the scale is rounded to the nearest binary16.  Enqueued on
+ * `stream`.  EINVAL on a bad method, count, iteration limit, null or misaligned pointer. */
+enum { SCION_QUANT_ABSMEAN = 0, SCION_QUANT_LLOYD = 1 };
+int scion_quantize_device(int method, const float* w, int64_t n_groups, int iters, int8_t* codes, uint16_t* scale_f16,
+                          void* stream);
+
 /* -------------------------------------------------------------------- layer
  * One MoE block.  d = hidden size, E = experts, k = top-k, F = expert ffn,
  * Fs = shared-expert ffn (0 = no shared expert), r = correction rank (0 = none).

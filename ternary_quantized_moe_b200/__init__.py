@@ -27,7 +27,7 @@ __all__ = [
     "scion_moe_forward_host", "scion_moe_forward_debug", "Layer", "library_path", "EXPORTS",
     "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "STAGES", "scion_layer_check",
     "scion_router_logits_static", "scion_layer_set_option", "SCION_OPT_STREAM_MIN_TOKENS",
-    "scion_moe_forward_residual",
+    "scion_moe_forward_residual", "scion_quantize_device", "SCION_QUANT_ABSMEAN", "SCION_QUANT_LLOYD",
 ]
 
 SCION_PQ2_0 = 0
@@ -45,8 +45,9 @@ EXPORTS = (
     "scion_pack_device", "scion_unpack_device", "scion_layer_create", "scion_layer_destroy",
     "scion_layer_device_bytes", "scion_moe_forward", "scion_moe_forward_host", "scion_moe_forward_debug",
     "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "scion_layer_check",
-    "scion_router_logits_static", "scion_layer_set_option", "scion_moe_forward_residual",
+    "scion_router_logits_static", "scion_layer_set_option", "scion_moe_forward_residual", "scion_quantize_device",
 )
+SCION_QUANT_ABSMEAN, SCION_QUANT_LLOYD = 0, 1
 SCION_OPT_STREAM_MIN_TOKENS = 1
 STAGES = ("router_f32", "xproj", "route", "gateup", "down_routed", "down_dense", "x16", "combine")
 
@@ -100,6 +101,7 @@ def _load():
             "scion_layer_device_bytes": (C.c_size_t, [vp]),
             "scion_moe_forward": (ci, [vp, ci, vp, vp, vp]),
             "scion_moe_forward_residual": (ci, [vp, ci, vp, vp, vp, vp]),
+            "scion_quantize_device": (ci, [ci, vp, i64, ci, vp, vp, vp]),
             "scion_moe_forward_host": (ci, [vp, ci, vp, vp, vp]),
             "scion_moe_forward_debug": (ci, [vp, ci, vp, vp, C.POINTER(_Debug), vp]),
             "scion_profile_begin": (ci, [ci]),
@@ -203,6 +205,20 @@ def scion_pack_device(fmt: int, codes, scales, out=None, bad_count=None, stream=
                                    _stream(stream))
     _check(st, "scion_pack_device")
     return out
+
+
+def scion_quantize_device(method: int, w, codes, scales, iters: int = 30, stream=None) -> None:
+    """w: fp32 CUDA [n, 128] (groups of 128); codes: int8 CUDA [n, 128]; scales: int16 CUDA [n]
+    (binary16 bit patterns).  method: SCION_QUANT_ABSMEAN or SCION_QUANT_LLOYD."""
+    import torch
+
+    n = w.numel() // 128
+    if w.numel() != n * 128 or codes.numel() != n * 128 or scales.numel() != n:
+        raise ValueError("w / codes / scales sizes do not match")
+    st = _load().scion_quantize_device(int(method), _dptr(w, "w", (torch.float32,)), n, int(iters),
+                                       _dptr(codes, "codes", (torch.int8,)),
+                                       _dptr(scales, "scales", (torch.int16, torch.uint16)), _stream(stream))
+    _check(st, "scion_quantize_device")
 
 
 def scion_unpack_device(fmt: int, blocks, codes=None, scales=None, bad_count=None, stream=None):

@@ -419,3 +419,52 @@ def test_prefill_matches_decode_passes():
     a1, _ = run_forward(dec, x[64:], 64)
     b, _ = run_forward(pre, x, 128)
     check_output(b, np.concatenate([a0, a1]), rel_l2=1e-4, max_abs=1e-3)
+
+
+# ------------------------------------------------------------------ quantizers
+def _quant_inputs():
+    rng = np.random.default_rng(2024)
+    w = np.concatenate([rng.standard_normal((300, 128)), 0.01 * rng.laplace(size=(300, 128)),
+                        rng.standard_t(3, size=(300, 128)), 1e3 * rng.standard_normal((20, 128)),
+                        1e-4 * rng.standard_normal((20, 128))]).astype(np.float32)
+    edge = np.zeros((6, 128), np.float32)
+    edge[1] = 0.25
+    edge[2] = np.where(np.arange(128) % 2, 3.0, -3.0)
+    edge[3, 17] = -2.0
+    edge[4, :64] = 1.0
+    edge[5] = np.linspace(-1, 1, 128)
+    return np.concatenate([w, edge])
+
+
+@pytest.mark.parametrize("method", [tq.SCION_QUANT_ABSMEAN, tq.SCION_QUANT_LLOYD])
+def test_quantize_matches_oracle(method):
+    """Codes and fp16 scales bit-exact against the oracle (decisions in fp64 on both sides),
+    then packed on the device into both containers and read back by the oracle's unpacker."""
+    w = _quant_inputs()
+    ref_c, ref_s = oracle.quantize(method, w, iters=30)
+    wd = torch.from_numpy(w).to(DEV)
+    codes = torch.empty(w.shape, dtype=torch.int8, device=DEV)
+    scales = torch.empty(w.shape[0], dtype=torch.int16, device=DEV)
+    tq.scion_quantize_device(method, wd, codes, scales, iters=30)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(codes.cpu().numpy(), ref_c)
+    np.testing.assert_array_equal(scales.cpu().numpy().view(np.uint16), ref_s)
+    for fmt in (synth.PQ2_0, synth.PTQ1_0):
+        blocks = tq.scion_pack_device(fmt, codes, scales)
+        c2, s2, st = oracle.unpack(fmt, blocks.cpu().numpy())
+        assert st == oracle.OK
+        np.testing.assert_array_equal(c2.reshape(ref_c.shape), ref_c)
+        np.testing.assert_array_equal(s2.reshape(-1), ref_s)
+
+
+def test_quantize_rejects_bad_arguments():
+    w = torch.zeros((2, 128), dtype=torch.float32, device=DEV)
+    codes = torch.empty((2, 128), dtype=torch.int8, device=DEV)
+    scales = torch.empty(2, dtype=torch.int16, device=DEV)
+    with pytest.raises(tq.ScionError) as ei:
+        tq.scion_quantize_device(7, w, codes, scales)
+    assert ei.value.status == tq.SCION_EINVAL
+    flat = torch.zeros(2 * 128 + 1, dtype=torch.float32, device=DEV)
+    with pytest.raises(tq.ScionError) as ei:  # w must be 16-byte aligned
+        tq.scion_quantize_device(tq.SCION_QUANT_ABSMEAN, flat[1:], codes, scales)
+    assert ei.value.status == tq.SCION_EINVAL
