@@ -968,7 +968,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
     case SCION_STAGE_ROUTE: {
       const int vpl = (L->E + 31) / 32;
       // at least two CTAs per SM for the top-k and one for the scatter, then fewer global atomics
-      const int tpw = max(1, min(4, T / (8 * 2 * num_sms())));
+      const int tpw = max(1, min(2, T / (8 * 2 * num_sms())));
       const int n = T * L->k, ept = max(1, min(kScatterMaxPerThread, n / (256 * num_sms())));
       cudaError_t e = cudaMemsetAsync(P.counts, 0, sizeof(int32_t) * L->E, s);
       if (e != cudaSuccess) return e;
