@@ -274,17 +274,15 @@ constexpr int kGuWarps = 8;
 // CTA = (16 ffn rows, active-expert slot); the 8 warps split the d/128 groups, keep their
 // groups' codes in registers, and run the slot's tokens 8 at a time.
 template <int FMT, int GPW>
-__global__ void __launch_bounds__(kGuWarps * 32) gateup_kernel(GateUpArgs a) {
+__device__ __forceinline__ void gateup_body(const GateUpArgs& a, int slot, int ft) {
   __shared__ float red[kGuWarps][2][32][4];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, c = lane & 3;
-  const int slot = blockIdx.y;
   pdl_trigger();
   pdl_wait();
   const int nact = *a.n_active;
   const int4 si = a.slot_info[slot];
   if (slot >= nact) return;
   const int e = si.x, p0 = si.y, ne = si.z;
-  const int ft = blockIdx.x;
   constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
   const uint8_t* tile0 = a.bank + ((int64_t(e) * (a.F >> 7) + (ft >> 3)) * a.Gd * 2 * 8 + (ft & 7)) * tb;
   TileRegs<FMT> rg[GPW], ru[GPW];
@@ -333,6 +331,11 @@ __global__ void __launch_bounds__(kGuWarps * 32) gateup_kernel(GateUpArgs a) {
     }
     __syncthreads();
   }
+}
+
+template <int FMT, int GPW>
+__global__ void __launch_bounds__(kGuWarps * 32) gateup_kernel(GateUpArgs a) {
+  gateup_body<FMT, GPW>(a, blockIdx.y, blockIdx.x);
 }
 
 // ======================================================================== down
@@ -416,13 +419,13 @@ constexpr int kDnKc = 256;            // K columns per CTA
 constexpr int kDnRowH = kDnKc + 32;   // staged hz row (halves): 576 B, rows 16 banks apart
 
 template <int NT>
-__global__ void __launch_bounds__(256) down_dense_kernel(DenseArgs a) {
+__device__ __forceinline__ void dense_body(const DenseArgs& a, int bx, int by) {
   extern __shared__ __align__(16) uint8_t dsm[];
   __half* hs = reinterpret_cast<__half*>(dsm);                                 // [NT*8][kDnRowH]
   float* red = reinterpret_cast<float*>(dsm + NT * 8 * kDnRowH * sizeof(__half));  // [8][NT][32][4]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g8 = lane >> 2, c = lane & 3;
-  const int row0 = blockIdx.x * 32 + 16 * (warp & 1);
-  const int kc0 = blockIdx.y * kDnKc;
+  const int row0 = bx * 32 + 16 * (warp & 1);
+  const int kc0 = by * kDnKc;
   const int kw = kc0 + 64 * (warp >> 1);
   pdl_trigger();
   // weights first (they do not depend on earlier kernels): 64 columns of rows g8 and g8 + 8
@@ -476,9 +479,28 @@ __global__ void __launch_bounds__(256) down_dense_kernel(DenseArgs a) {
     float v = 0.f;
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) v += red[(((h + 2 * ks) * NT + nt) * 32 + ln) * 4 + i];
-    const int row = blockIdx.x * 32 + 16 * h + (ln >> 2) + 8 * (i >> 1), tok = nt * 8 + 2 * (ln & 3) + (i & 1);
+    const int row = bx * 32 + 16 * h + (ln >> 2) + 8 * (i >> 1), tok = nt * 8 + 2 * (ln & 3) + (i & 1);
     if (tok < a.T) atomicAdd(&a.out[int64_t(tok) * a.d + row], v);
   }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(256) down_dense_kernel(DenseArgs a) {
+  dense_body<NT>(a, blockIdx.x, blockIdx.y);
+}
+
+// Batches below the ring kernels' threshold: the expert gate/up and the dense down projection
+// (which needs only the x-projection) in one launch, so the dense part leaves the critical
+// path.  Rows [0, gu_rows) of the grid are gate/up CTAs, the rows after them dense-down tiles
+// (dense_x tiles of 32 output rows per K chunk).
+template <int FMT, int GPW, int NT>
+__global__ void __launch_bounds__(256) gateup_dense_kernel(GateUpArgs a, DenseArgs b, int gu_rows, int dense_x) {
+  if (int(blockIdx.y) < gu_rows) {
+    gateup_body<FMT, GPW>(a, blockIdx.y, blockIdx.x);
+    return;
+  }
+  const int lin = (int(blockIdx.y) - gu_rows) * int(gridDim.x) + int(blockIdx.x);
+  if (lin < dense_x * ((b.Kd + kDnKc - 1) / kDnKc)) dense_body<NT>(b, lin % dense_x, lin / dense_x);
 }
 
 template <int NT>
@@ -548,6 +570,42 @@ cudaError_t launch_gateup(const scion_layer* L, const __nv_bfloat16* /*x*/, int 
     else return cudaErrorInvalidValue;
   }
 #undef SCION_GU
+  return cudaGetLastError();
+}
+
+bool gateup_merges_dense(const scion_layer* L, int T) { return L->Kdense > 0 && (T + 7) / 8 <= 2; }
+
+// The gate/up of the split-K path with the dense down projection in the same launch
+// (gateup_merges_dense).
+cudaError_t launch_gateup_dense(const scion_layer* L, int T, float* out, cudaStream_t s) {
+  GateUpArgs a;
+  a.bank = L->gu_bank, a.xfrag = L->xfrag;
+  a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
+  a.d = L->d, a.F = L->F, a.k = L->k, a.Gd = L->Gd, a.fmt = L->fmt;
+  a.hfrag = L->h;
+  DenseArgs b;
+  b.w = L->dense_down, b.hz = L->hz, b.d = L->d, b.Kd = L->Kd, b.T = T, b.out = out;
+  const int slots = min(L->E, T * L->k);
+  const int gx = L->F / 16, dense_x = L->d / 32;
+  const int dense_tiles = dense_x * ((L->Kd + kDnKc - 1) / kDnKc);
+  const dim3 grid(gx, slots + (dense_tiles + gx - 1) / gx);
+  const int gpw = (L->Gd + kGuWarps - 1) / kGuWarps;
+  const bool two = (T + 7) / 8 == 2;
+#define SCION_GUD(F_, G_)                                                                                        \
+  return two ? launch_pdl(gateup_dense_kernel<F_, G_, 2>, grid, dim3(kGuWarps * 32), down_dense_smem<2>(), s, a, b, \
+                          slots, dense_x)                                                                        \
+             : launch_pdl(gateup_dense_kernel<F_, G_, 1>, grid, dim3(kGuWarps * 32), down_dense_smem<1>(), s, a, b, \
+                          slots, dense_x)
+  if (L->fmt == SCION_PQ2_0) {
+    if (gpw <= 1) SCION_GUD(SCION_PQ2_0, 1); else if (gpw == 2) SCION_GUD(SCION_PQ2_0, 2);
+    else if (gpw == 3) SCION_GUD(SCION_PQ2_0, 3); else if (gpw == 4) SCION_GUD(SCION_PQ2_0, 4);
+    else return cudaErrorInvalidValue;
+  } else {
+    if (gpw <= 1) SCION_GUD(SCION_PTQ1_0, 1); else if (gpw == 2) SCION_GUD(SCION_PTQ1_0, 2);
+    else if (gpw == 3) SCION_GUD(SCION_PTQ1_0, 3); else if (gpw == 4) SCION_GUD(SCION_PTQ1_0, 4);
+    else return cudaErrorInvalidValue;
+  }
+#undef SCION_GUD
   return cudaGetLastError();
 }
 

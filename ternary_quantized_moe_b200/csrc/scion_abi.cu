@@ -207,11 +207,16 @@ int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out
     if ((e = cudaEventRecord(L->ev_dense, L->side)) != cudaSuccess) return cuda_status(e);
   }
   SCION_STAGE(SCION_STAGE_ROUTE, scion::launch_route(L, T, s));
-  SCION_STAGE(SCION_STAGE_GATEUP, ring ? scion::launch_stream_gateup(L, T, s) : scion::launch_gateup(L, x, T, s));
+  // small batches: the dense down projection rides in the gate/up launch (it needs only the
+  // x-projection), off the critical path of the routed kernels
+  const bool merged = !ring && scion::gateup_merges_dense(L, T);
+  SCION_STAGE(SCION_STAGE_GATEUP, ring     ? scion::launch_stream_gateup(L, T, s)
+                                  : merged ? scion::launch_gateup_dense(L, T, out, s)
+                                           : scion::launch_gateup(L, x, T, s));
   SCION_STAGE(SCION_STAGE_DOWN_ROUTED,
               ring ? scion::launch_stream_down(L, T, out, s) : scion::launch_down_routed(L, T, out, s));
   if (side) return cuda_status(cudaStreamWaitEvent(s, L->ev_dense, 0));
-  if (L->Kdense) SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
+  if (L->Kdense && !merged) SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
   return SCION_OK;
 }
 

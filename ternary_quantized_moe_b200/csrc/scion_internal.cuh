@@ -155,6 +155,8 @@ cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, fl
 cudaError_t launch_gateup(const scion_layer* L, const __nv_bfloat16* x, int T, cudaStream_t s);
 cudaError_t launch_down_routed(const scion_layer* L, int T, float* out, cudaStream_t s);
 cudaError_t launch_down_dense(const scion_layer* L, int T, float* out, cudaStream_t s);
+bool gateup_merges_dense(const scion_layer* L, int T);
+cudaError_t launch_gateup_dense(const scion_layer* L, int T, float* out, cudaStream_t s);
 // fragment-ordered rows [rows][G][SCION_BROW] -> natural order [rows][G*128]
 cudaError_t launch_unfrag(int fmt, const __half* src, int rows, int G, __half* dst, cudaStream_t s);
 cudaError_t configure_kernels();
