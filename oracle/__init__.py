@@ -56,6 +56,7 @@ class _Layer(C.Structure):
         ("gate_exps", C.c_void_p), ("up_exps", C.c_void_p), ("down_exps", C.c_void_p),
         ("sh_gate", C.c_void_p), ("sh_up", C.c_void_p), ("sh_down", C.c_void_p),
         ("sh_gate_vec", C.c_void_p), ("corr_a", C.c_void_p), ("corr_b", C.c_void_p),
+        ("corr_packed", C.c_int),
     ]
 
 
@@ -190,10 +191,11 @@ class OracleLayer:
     sh_down: Optional[np.ndarray] = None   # uint16 bf16 [d, Fs]
     sh_gate_vec: Optional[np.ndarray] = None  # uint16 bf16 [d]
     rank: int = 0
-    corr_a: Optional[np.ndarray] = None    # uint16 bf16 [r, d]
-    corr_b: Optional[np.ndarray] = None    # uint16 bf16 [d, r]
+    corr_a: Optional[np.ndarray] = None    # uint16 bf16 [r, d], or uint8 PQ2_0 blocks [r, d/128*34]
+    corr_b: Optional[np.ndarray] = None    # uint16 bf16 [d, r], or uint8 PQ2_0 blocks [d, r/128*34]
     norm_topk: int = 1
     corr_on_output: int = 0
+    corr_packed: int = 0                   # 1: the correction factors are the PQ2_0 blocks
 
     def _c(self) -> _Layer:
         rf32 = 1 if self.w_router.dtype == np.float32 else 0
@@ -210,6 +212,7 @@ class OracleLayer:
         L.gate_exps, L.up_exps, L.down_exps = _ptr(self.gate_exps), _ptr(self.up_exps), _ptr(self.down_exps)
         L.sh_gate, L.sh_up, L.sh_down = _ptr(self.sh_gate), _ptr(self.sh_up), _ptr(self.sh_down)
         L.sh_gate_vec, L.corr_a, L.corr_b = _ptr(self.sh_gate_vec), _ptr(self.corr_a), _ptr(self.corr_b)
+        L.corr_packed = self.corr_packed
         return L
 
 

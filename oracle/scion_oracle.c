@@ -219,8 +219,11 @@ typedef struct {
   const uint16_t* sh_up;    /* bf16 [shared_ffn][d] */
   const uint16_t* sh_down;  /* bf16 [d][shared_ffn] */
   const uint16_t* sh_gate_vec; /* bf16 [d] or NULL */
-  const uint16_t* corr_a;   /* bf16 [rank][d] */
-  const uint16_t* corr_b;   /* bf16 [d][rank] */
+  const uint16_t* corr_a;   /* bf16 [rank][d] (or PQ2_0 blocks, see corr_packed) */
+  const uint16_t* corr_b;   /* bf16 [d][rank] (or PQ2_0 blocks) */
+  int corr_packed;          /* 1: corr_a = PQ2_0 blocks [rank][d/128], corr_b = [d][rank/128]: ternary
+                               correction factors, w = code * scale ("Scion-35B-A3B" model card, Model
+                               Overview: the release ships its corrections ternary, q1_0_g128) */
 } oracle_layer;
 
 static double router_weight(const oracle_layer* L, const void* w, long idx) {
@@ -378,6 +381,26 @@ static void shared_one(const oracle_layer* L, const double* xv, double* h, doubl
 /* Step 6: rank-r correction c = B (A in). */
 static void corr_one(const oracle_layer* L, const double* in, double* z, double* y) {
   int d = L->d, r = L->rank;
+  if (L->corr_packed) {
+    /* dequantize one row at a time with the container decoder above */
+    const uint8_t* A = (const uint8_t*)L->corr_a;
+    const uint8_t* B = (const uint8_t*)L->corr_b;
+    double* w = (double*)malloc(sizeof(double) * (d > r ? d : r));
+    for (int q = 0; q < r; q++) {
+      oracle_dequant_row(ORACLE_PQ2_0, A + (long)q * (d / 128) * 34, d, w);
+      double a = 0.0;
+      for (int i = 0; i < d; i++) a += w[i] * in[i];
+      z[q] = a;
+    }
+    for (int i = 0; i < d; i++) {
+      oracle_dequant_row(ORACLE_PQ2_0, B + (long)i * (r / 128) * 34, r, w);
+      double a = 0.0;
+      for (int q = 0; q < r; q++) a += w[q] * z[q];
+      y[i] = a;
+    }
+    free(w);
+    return;
+  }
   for (int q = 0; q < r; q++) {
     double a = 0.0;
     for (int i = 0; i < d; i++) a += oracle_bf16_to_f64(L->corr_a[(long)q * d + i]) * in[i];
@@ -417,6 +440,7 @@ static int check_layer(const oracle_layer* L) {
   if (L->n_experts <= 0 || L->top_k <= 0 || L->top_k > L->n_experts) return ORACLE_EINVAL;
   if (L->fmt != ORACLE_PQ2_0 && L->fmt != ORACLE_PTQ1_0) return ORACLE_EINVAL;
   if (L->shared_ffn < 0 || L->rank < 0) return ORACLE_EINVAL;
+  if (L->corr_packed && L->rank % 128) return ORACLE_EINVAL; /* groups of 128 along B's rank axis */
   return ORACLE_OK;
 }
 

@@ -234,3 +234,31 @@ def test_expert_hidden_matches_forward():
     for t in range(2):
         _, y = oracle.expert(lay, int(ids[t, 0]), x[t])
         np.testing.assert_allclose(out[t], y, rtol=1e-14, atol=1e-300)
+
+
+def test_packed_correction_matches_numpy_from_codes():
+    """Ternary correction factors in PQ2_0 blocks: the oracle's z = A x and c = B z from the
+    packed bytes against numpy from the generating codes and scales (groups of 128 along each
+    factor's reduction axis: d for A, r for B), and the block with the packed correction minus
+    the block without any correction is c."""
+    cfg = small_cfg(fmt=synth.PTQ1_0, r=256)
+    L = synth.layer_host(cfg)
+    rng = np.random.default_rng(31)
+    ca = synth.ternary_codes(rng, (cfg.rank, cfg.d))
+    sa = synth.group_scales(rng, (cfg.rank, cfg.d // 128))
+    cb = synth.ternary_codes(rng, (cfg.d, cfg.rank))
+    sb = synth.group_scales(rng, (cfg.d, cfg.rank // 128))
+    ol = oracle_layer_from(cfg, L)
+    ol.corr_a, ol.corr_b, ol.corr_packed = oracle.pack(synth.PQ2_0, ca, sa), oracle.pack(synth.PQ2_0, cb, sb), 1
+    x = synth.x_host(cfg, 5)
+    z, c = oracle.corr(ol, x)
+    A = ca.astype(np.float64) * np.repeat(f16(sa), 128, axis=1)
+    B = cb.astype(np.float64) * np.repeat(f16(sb), 128, axis=1)
+    xv = bf16(x)
+    np.testing.assert_allclose(z, xv @ A.T, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(c, z @ B.T, rtol=1e-10, atol=1e-14)
+    out, _, _ = oracle.forward(ol, x)
+    ol0 = oracle_layer_from(cfg, L)
+    ol0.rank, ol0.corr_a, ol0.corr_b = 0, None, None
+    out0, _, _ = oracle.forward(ol0, x)
+    np.testing.assert_allclose(out - out0, c, rtol=1e-9, atol=1e-12)
