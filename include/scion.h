@@ -141,6 +141,12 @@ typedef struct {
   const void* sh_gate_vec;
   const void* corr_a;
   const void* corr_b;
+  /* 0: corr_a / corr_b are bf16 [rank][d] and [d][rank].  1: ternary correction factors
+   * ("Scion-35B-A3B" model card, Weight Representation: the corrections ship as 2-bit codes
+   * plus one fp16 scale per 128, the q1_0_g128 container) as PQ2_0 blocks, corr_a [rank][d/128] and corr_b [d][rank/128] (groups of 128 along each
+   * factor's reduction axis; rank a multiple of 128).  Decode reads corr_a's blocks in place;
+   * corr_b, and corr_a for batches above 64 tokens, become exact fp16 copies (code * scale). */
+  int corr_packed;
 } scion_layer_desc;
 
 typedef struct scion_layer scion_layer;
@@ -155,7 +161,10 @@ typedef struct scion_layer scion_layer;
  * validate every code: SCION_EFORMAT if a block holds an invalid code (no
  * handle is returned), EINVAL on a bad descriptor, ENOMEM, ECUDA.  Descriptor
  * limits: d and ffn multiples of 128 with d <= 4096, shared_ffn a multiple of 128,
- * rank a multiple of 16, 1 <= top_k <= min(E, 32), E <= 4096. */
+ * rank a multiple of 16 (of 128 with corr_packed), 1 <= top_k <= min(E, 32), E <= 4096.
+ * With corr_packed, a correction-A scale whose 256-fold overflows fp16 on a PQ2_0 layer with
+ * max_tokens > 64 counts as an invalid code (its fp16 copy is stored in the experts' column
+ * order, scaled by the same powers of 4 as their inputs). */
 int scion_layer_create(const scion_layer_desc* desc, int max_tokens, void* stream, scion_layer** out);
 
 /* Frees the handle and everything it allocated (synchronises the device). */

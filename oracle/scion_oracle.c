@@ -222,8 +222,8 @@ typedef struct {
   const uint16_t* corr_a;   /* bf16 [rank][d] (or PQ2_0 blocks, see corr_packed) */
   const uint16_t* corr_b;   /* bf16 [d][rank] (or PQ2_0 blocks) */
   int corr_packed;          /* 1: corr_a = PQ2_0 blocks [rank][d/128], corr_b = [d][rank/128]: ternary
-                               correction factors, w = code * scale ("Scion-35B-A3B" model card, Model
-                               Overview: the release ships its corrections ternary, q1_0_g128) */
+                               correction factors, w = code * scale ("Scion-35B-A3B" model card, Weight
+                               Representation: 2-bit codes plus one fp16 scale per 128, q1_0_g128) */
 } oracle_layer;
 
 static double router_weight(const oracle_layer* L, const void* w, long idx) {

@@ -67,6 +67,7 @@ class _Desc(C.Structure):
         ("gate_exps", C.c_void_p), ("up_exps", C.c_void_p), ("down_exps", C.c_void_p),
         ("sh_gate", C.c_void_p), ("sh_up", C.c_void_p), ("sh_down", C.c_void_p),
         ("sh_gate_vec", C.c_void_p), ("corr_a", C.c_void_p), ("corr_b", C.c_void_p),
+        ("corr_packed", C.c_int),
     ]
 
 
@@ -264,11 +265,12 @@ class Layer:
 def scion_layer_create(*, d: int, n_experts: int, top_k: int, ffn: int, fmt: int, w_router, w_router_delta,
                        gate_exps, up_exps, down_exps, shared_ffn: int = 0, sh_gate=None, sh_up=None,
                        sh_down=None, rank: int = 0, corr_a=None, corr_b=None, norm_topk: int = 1,
-                       max_tokens: int = 64, stream=None) -> Layer:
+                       corr_packed: int = 0, max_tokens: int = 64, stream=None) -> Layer:
     """Builds a layer from CUDA tensors (see include/scion.h for layouts).
 
     w_router / w_router_delta: float32 (fp32 router) or bfloat16 [E, d]; banks: uint8 packed
-    blocks; shared and correction weights: bfloat16."""
+    blocks; shared weights: bfloat16; correction factors: bfloat16, or (corr_packed = 1) uint8
+    PQ2_0 blocks [rank, d/128*34] and [d, rank/128*34]."""
     import torch
 
     bf16 = (torch.bfloat16,)
@@ -286,8 +288,10 @@ def scion_layer_create(*, d: int, n_experts: int, top_k: int, ffn: int, fmt: int
     D.sh_up = _dptr(sh_up, "sh_up", bf16)
     D.sh_down = _dptr(sh_down, "sh_down", bf16)
     D.sh_gate_vec = None
-    D.corr_a = _dptr(corr_a, "corr_a", bf16)
-    D.corr_b = _dptr(corr_b, "corr_b", bf16)
+    cdt = (torch.uint8,) if corr_packed else bf16
+    D.corr_a = _dptr(corr_a, "corr_a", cdt)
+    D.corr_b = _dptr(corr_b, "corr_b", cdt)
+    D.corr_packed = int(corr_packed)
     h = C.c_void_p()
     st = _load().scion_layer_create(C.byref(D), int(max_tokens), _stream(stream), C.byref(h))
     _check(st, "scion_layer_create")

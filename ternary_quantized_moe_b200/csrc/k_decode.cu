@@ -42,6 +42,7 @@ struct XProjArgs {
   __half* xfrag;  // [T][d/128][SCION_BROW] fp16 in fragment order + group sums
   __half* h;      // [T*k][F/128][SCION_BROW] expert hidden: group-sum tails zeroed here
   int k, GF;
+  const uint8_t* corr_blocks;  // ternary correction A (PQ2_0 blocks [r][d/128]) or nullptr (bf16 corr_a)
   float* out;     // set here to the residual (or zero)
   const float* resid;  // nullptr: out starts at zero; may equal out (then out is left as it is)
 };
@@ -106,6 +107,16 @@ __device__ __forceinline__ void xproj_aux(const XProjArgs& a, int aux, int n_aux
     *reinterpret_cast<float4*>(a.h + int64_t(i) * SCION_BROW + 128) = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
+// Eight consecutive ternary codes (16 bits of a PQ2_0 block, low bits first: field 0/1/2 =
+// -1/0/+1) as four bf16 pairs in column order.
+__device__ __forceinline__ uint32_t tern_pair_bf16(uint32_t f) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(float(int(f & 3u) - 1), float(int((f >> 2) & 3u) - 1));
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+__device__ __forceinline__ uint4 tern8_bf16(uint32_t c16) {
+  return make_uint4(tern_pair_bf16(c16), tern_pair_bf16(c16 >> 4), tern_pair_bf16(c16 >> 8), tern_pair_bf16(c16 >> 12));
+}
+
 template <int NT>
 __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
   extern __shared__ __align__(16) uint8_t xsm[];
@@ -147,15 +158,35 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
   const bool active_warp = kw < a.d;
   // weights first (they do not depend on x): both matrices, this warp's 64 columns
   uint4 wa[2][2], wb[2][2];
-#pragma unroll
-  for (int m = 0; m < 2; ++m)
+  // ternary correction A: the warp's 64 columns lie in one group of 128 of each row's block, so
+  // its partial sums take the group scales of rows row_a / row_b after the MMAs
+  const bool tern = u.kind == kUnitPlain && a.corr_blocks != nullptr;
+  float sc_a = 0.f, sc_b = 0.f;
+  if (tern) {
+    const int G = a.d >> 7, g = kw >> 7, hoff = kw & 127;
+    const uint8_t* ba = a.corr_blocks + (int64_t(row_a) * G + g) * 34;
+    const uint8_t* bb = a.corr_blocks + (int64_t(row_b) * G + g) * 34;
+    const bool la = active_warp && ok_a, lb = active_warp && ok_b;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
-      const int kk = kw + 32 * q + 8 * c;
-      const bool ld = active_warp && m < nmat;
-      wa[m][q] = (ld && ok_a) ? ldg_stream(mats[m] + int64_t(row_a) * a.d + kk) : make_uint4(0, 0, 0, 0);
-      wb[m][q] = (ld && ok_b) ? ldg_stream(mats[m] + int64_t(row_b) * a.d + kk) : make_uint4(0, 0, 0, 0);
+      const int j0 = hoff + 32 * q + 8 * c;  // first of the lane's 8 columns in the group
+      wa[0][q] = la ? tern8_bf16(__ldg(reinterpret_cast<const unsigned short*>(ba + (j0 >> 2)))) : make_uint4(0, 0, 0, 0);
+      wb[0][q] = lb ? tern8_bf16(__ldg(reinterpret_cast<const unsigned short*>(bb + (j0 >> 2)))) : make_uint4(0, 0, 0, 0);
+      wa[1][q] = wb[1][q] = make_uint4(0, 0, 0, 0);
     }
+    sc_a = la ? __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short*>(ba + 32)))) : 0.f;
+    sc_b = lb ? __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short*>(bb + 32)))) : 0.f;
+  } else {
+#pragma unroll
+    for (int m = 0; m < 2; ++m)
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int kk = kw + 32 * q + 8 * c;
+        const bool ld = active_warp && m < nmat;
+        wa[m][q] = (ld && ok_a) ? ldg_stream(mats[m] + int64_t(row_a) * a.d + kk) : make_uint4(0, 0, 0, 0);
+        wb[m][q] = (ld && ok_b) ? ldg_stream(mats[m] + int64_t(row_b) * a.d + kk) : make_uint4(0, 0, 0, 0);
+      }
+  }
   pdl_wait();  // everything below reads x or writes the workspace
   // stage x[0..T)[kbase .. kbase+512) in shared memory (rows padded by 16 B: conflict-free reads)
   const int kchunks = min(SCION_XPROJ_KC, a.d - kbase) >> 3;  // 16-byte chunks per token row (<= 64)
@@ -193,6 +224,11 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
         }
       }
     }
+  }
+  if (tern) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+      acc[0][nt][0] *= sc_a, acc[0][nt][1] *= sc_a, acc[0][nt][2] *= sc_b, acc[0][nt][3] *= sc_b;
   }
   __syncthreads();  // the x stage is dead: its space holds the warp reduction
   float(*red)[2][NT][32][4] = reinterpret_cast<float(*)[2][NT][32][4]>(xsm);
@@ -535,6 +571,7 @@ cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, fl
   a.corr_a = static_cast<const __nv_bfloat16*>(L->desc.corr_a);
   a.units = L->xunits + unit0, a.n_units = n_units, a.n_chunks = L->n_xchunks, a.n_aux = aux ? kXAux : 0;
   a.logits = L->logits, a.hz = L->hz, a.xfrag = L->xfrag, a.out = out;
+  a.corr_blocks = L->desc.corr_packed ? static_cast<const uint8_t*>(L->desc.corr_a) : nullptr;
   a.h = L->h, a.k = L->k, a.GF = L->GF;
   if (n_units + a.n_aux == 0) return cudaSuccess;
   dim3 grid(n_units + a.n_aux, L->n_xchunks);

@@ -101,6 +101,34 @@ __global__ void __launch_bounds__(256) x16_kernel(const __nv_bfloat16* __restric
   }
 }
 
+// Ternary correction factors (PQ2_0 blocks [rows][K/128], 2-bit codes + fp16 scale) -> fp16
+// code * scale, exact.  order < 0: natural column order; otherwise the column order of the
+// layer's x16 operand for expert format `order` (PQ2_0: with its 4^f factors multiplied back
+// in), so that a GEMM against x16 computes A x.  dst == nullptr only counts.  Invalid codes (3)
+// and values past the fp16 range are counted into *bad.
+__global__ void dequant_corr_kernel(const uint8_t* __restrict__ blocks, int rows, int K, __half* __restrict__ dst,
+                                    int ld, int order, unsigned long long* __restrict__ bad) {
+  const int64_t n = int64_t(rows) * K;
+  unsigned nbad = 0;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const int row = int(i / K), col = int(i % K), j = col & 127;
+    const uint8_t* blk = blocks + (int64_t(row) * (K >> 7) + (col >> 7)) * 34;
+    const int field = (blk[j >> 2] >> (2 * (j & 3))) & 3;
+    const float sc = __half2float(__ushort_as_half(uint16_t(blk[32] | (blk[33] << 8))));
+    float v = field == 3 ? 0.f : float(field - 1) * sc;
+    nbad += field == 3;
+    int pos = col;
+    if (order >= 0) {
+      pos = perm_pos(order, col);
+      if (order == SCION_PQ2_0) v /= pq2_pos_scale(pos);  // times 4^f: exact unless it overflows
+    }
+    const __half hv = __float2half_rn(v);
+    nbad += __hisinf(hv) != 0;
+    if (dst) dst[int64_t(row) * ld + pos] = hv;
+  }
+  if (nbad) atomicAdd(bad, (unsigned long long)nbad);
+}
+
 // ---------------------------------------------------------------- dense GEMM
 enum DenseEpi : int { kEpiLogits = 0, kEpiSwiglu = 1, kEpiPlain = 2, kEpiStore = 3 };
 
@@ -919,6 +947,25 @@ size_t prefill_unit_bytes() { return sizeof(DenseUnit); }
 size_t prefill_tile_bytes() { return sizeof(TernTile); }
 
 // Builds the dense unit tables (host) for the x-projection and the dense down GEMM.
+cudaError_t launch_dequant_corr(const uint8_t* blocks, int rows, int K, __half* dst, int ld, int order,
+                                int64_t* bad, cudaStream_t s) {
+  const int64_t n = int64_t(rows) * K;
+  if (n == 0) return cudaSuccess;
+  const unsigned grid = unsigned(std::min<int64_t>((n + 255) / 256, int64_t(num_sms()) * 16));
+  dequant_corr_kernel<<<grid, 256, 0, s>>>(blocks, rows, K, dst, ld, order, reinterpret_cast<unsigned long long*>(bad));
+  return cudaGetLastError();
+}
+
+// Units of the correction A when its factors are ternary: an fp16 GEMM against x16 (the
+// fp16 copy of A is stored in x16's column order), writing z into hz after the shared part.
+void prefill_corr_units(const scion_layer* L, void* cunits_host, int* n_c) {
+  DenseUnit* cu = static_cast<DenseUnit*>(cunits_host);
+  int nc = 0;
+  if (L->desc.corr_packed)
+    for (int r0 = 0; r0 < L->r; r0 += 128) cu[nc++] = DenseUnit{kEpiPlain, 1, 0, 4, 4, r0, L->r, L->Fs};
+  *n_c = nc;
+}
+
 void prefill_units(const scion_layer* L, void* xunits_host, int* n_x, void* dunits_host, int* n_d) {
   DenseUnit* xu = static_cast<DenseUnit*>(xunits_host);
   DenseUnit* du = static_cast<DenseUnit*>(dunits_host);
@@ -928,7 +975,8 @@ void prefill_units(const scion_layer* L, void* xunits_host, int* n_x, void* duni
   if (!L->desc.router_fp32)
     for (int r0 = 0; r0 < L->E; r0 += 128) xu[nx++] = DenseUnit{kEpiLogits, 2, 0, 0, 1, r0, L->E, 0};
   for (int r0 = 0; r0 < L->Fs; r0 += 128) xu[nx++] = DenseUnit{kEpiSwiglu, 2, 1, 2, 3, r0, L->Fs, 0};
-  for (int r0 = 0; r0 < L->r; r0 += 128) xu[nx++] = DenseUnit{kEpiPlain, 1, 0, 4, 4, r0, L->r, L->Fs};
+  if (!L->desc.corr_packed)
+    for (int r0 = 0; r0 < L->r; r0 += 128) xu[nx++] = DenseUnit{kEpiPlain, 1, 0, 4, 4, r0, L->r, L->Fs};
   if (L->Kdense)
     for (int r0 = 0; r0 < L->d; r0 += 128) du[nd++] = DenseUnit{kEpiStore, 1, 0, 5, 5, r0, L->d, 0};
   *n_x = nx;
@@ -952,7 +1000,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       return cudaGetLastError();
     }
     case SCION_STAGE_XPROJ: {
-      if (P.n_xunits == 0) return cudaSuccess;
+      if (P.n_xunits == 0 && P.n_cunits == 0) return cudaSuccess;
       DenseParams dp;
       memcpy(dp.a, P.maps, sizeof(dp.a));
       if (make_tmap_2d(&dp.b, x, 1, T, L->d) != SCION_OK) return cudaErrorInvalidValue;
@@ -962,6 +1010,12 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       dp.logits = P.logits, dp.ld_logits = L->E, dp.hz = P.hz, dp.ld_hz = L->Kd, dp.out = nullptr, dp.ld_out = 0;
       dp.resid = nullptr;
       dp.err = L->err;
+      if (dp.n_units) dense_gemm_kernel<<<dense_grid(dp), kThreads, kDenseSmem, s>>>(dp);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess || P.n_cunits == 0) return e;
+      // ternary correction factors: z = A x as an fp16 GEMM of A's exact fp16 copy against x16
+      dp.b = P.x16_map, dp.ab_bf16 = 0;
+      dp.units = static_cast<const DenseUnit*>(P.cunits), dp.n_units = P.n_cunits, dp.n_units2 = 0;
       dense_gemm_kernel<<<dense_grid(dp), kThreads, kDenseSmem, s>>>(dp);
       return cudaGetLastError();
     }

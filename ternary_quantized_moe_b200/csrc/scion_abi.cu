@@ -53,8 +53,8 @@ void free_layer(scion_layer* L) {
   if (L->ev_dense) cudaEventDestroy(L->ev_dense);
   if (L->pre) {
     scion::PrefillState* P = L->pre;
-    void* pp[] = {P->xunits, P->dunits, P->logits, P->ids, P->gates, P->counts, P->offsets,
-                  P->perm,   P->inv,    P->y,       P->tiles, P->n_tiles, P->x16, P->h, P->hz, P->cursor};
+    void* pp[] = {P->xunits, P->dunits, P->logits, P->ids, P->gates, P->counts, P->offsets, P->perm, P->inv,
+                  P->y, P->tiles, P->n_tiles, P->x16, P->h, P->hz, P->cursor, P->cunits, P->corr_a16};
     for (void* p : pp)
       if (p) cudaFree(p);
     delete P;
@@ -96,6 +96,15 @@ int create_prefill(scion_layer* L, cudaStream_t s) {
   PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->dunits), scion::prefill_unit_bytes() * max_units));
   PTRY(cudaMemcpyAsync(P->xunits, xu.data(), xu.size(), cudaMemcpyHostToDevice, s));
   PTRY(cudaMemcpyAsync(P->dunits, du.data(), du.size(), cudaMemcpyHostToDevice, s));
+  std::vector<uint8_t> cu(scion::prefill_unit_bytes() * max_units);
+  scion::prefill_corr_units(L, cu.data(), &P->n_cunits);
+  if (P->n_cunits) {
+    PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->cunits), scion::prefill_unit_bytes() * P->n_cunits));
+    PTRY(cudaMemcpyAsync(P->cunits, cu.data(), scion::prefill_unit_bytes() * P->n_cunits, cudaMemcpyHostToDevice, s));
+    PTRY(dev_alloc(L, &P->corr_a16, sizeof(__half) * size_t(L->r) * L->d));
+    PTRY(scion::launch_dequant_corr(static_cast<const uint8_t*>(L->desc.corr_a), L->r, L->d, P->corr_a16, L->d, L->fmt,
+                                    L->bad, s));
+  }
 #undef PTRY
   int st;
   const scion_layer_desc& D = L->desc;
@@ -107,7 +116,11 @@ int create_prefill(scion_layer* L, cudaStream_t s) {
     if ((st = scion::make_tmap_2d(&P->maps[2], D.sh_gate, 1, L->Fs, L->d))) return st;
     if ((st = scion::make_tmap_2d(&P->maps[3], D.sh_up, 1, L->Fs, L->d))) return st;
   }
-  if (L->r && (st = scion::make_tmap_2d(&P->maps[4], D.corr_a, 1, L->r, L->d))) return st;
+  if (L->r && !D.corr_packed && (st = scion::make_tmap_2d(&P->maps[4], D.corr_a, 1, L->r, L->d))) return st;
+  if (P->n_cunits) {
+    if ((st = scion::make_tmap_2d(&P->maps[4], P->corr_a16, 0, L->r, L->d))) return st;
+    if ((st = scion::make_tmap_2d(&P->x16_map, P->x16, 0, L->max_tokens, L->d))) return st;
+  }
   if (L->Kd) {
     if ((st = scion::make_tmap_2d(&P->maps[5], L->dense_down, 0, L->d, L->Kd))) return st;
     if ((st = scion::make_tmap_2d(&P->hz_map, P->hz, 0, L->max_tokens, L->Kd))) return st;
@@ -128,6 +141,10 @@ int check_desc(const scion_layer_desc* D, int max_tokens) {
   if (!D->w_router || !D->w_router_delta || !D->gate_exps || !D->up_exps || !D->down_exps) return SCION_EINVAL;
   if (D->shared_ffn > 0 && (!D->sh_gate || !D->sh_up || !D->sh_down)) return SCION_EINVAL;
   if (D->rank > 0 && (!D->corr_a || !D->corr_b)) return SCION_EINVAL;
+  if (D->corr_packed != 0 && D->corr_packed != 1) return SCION_EINVAL;
+  if (D->corr_packed && D->rank % 128) return SCION_EINVAL;  // groups of 128 along corr_b's rows
+  if (D->corr_packed && D->rank && ((reinterpret_cast<uintptr_t>(D->corr_a) | reinterpret_cast<uintptr_t>(D->corr_b)) & 1))
+    return SCION_EINVAL;  // blocks are read with 2-byte loads
   if (D->sh_gate_vec) return SCION_EINVAL;  // shared-expert sigmoid gate: not supported by the kernels yet
   return SCION_OK;
 }
@@ -315,9 +332,17 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
     if (L->Fs)
       SCION_TRY(scion::launch_bf16_to_f16_rows(static_cast<const __nv_bfloat16*>(desc->sh_down), L->d, L->Fs,
                                                L->dense_down, L->Kd, s));
-    if (L->r)
+    if (L->r && !desc->corr_packed)
       SCION_TRY(scion::launch_bf16_to_f16_rows(static_cast<const __nv_bfloat16*>(desc->corr_b), L->d, L->r,
                                                L->dense_down + L->Fs, L->Kd, s));
+    if (L->r && desc->corr_packed) {
+      // ternary correction factors: B as its exact fp16 values beside the shared down weights;
+      // A's codes checked here (decode reads its blocks in place)
+      SCION_TRY(scion::launch_dequant_corr(static_cast<const uint8_t*>(desc->corr_b), L->d, L->r,
+                                           L->dense_down + L->Fs, L->Kd, -1, L->bad, s));
+      SCION_TRY(scion::launch_dequant_corr(static_cast<const uint8_t*>(desc->corr_a), L->r, L->d, nullptr, 0, -1,
+                                           L->bad, s));
+    }
   }
   SCION_TRY(scion::launch_retile(L->fmt, static_cast<const uint8_t*>(desc->gate_exps), L->E, L->F, L->Gd, 2, 0,
                                  L->gu_bank, L->bad, s));

@@ -107,7 +107,18 @@ def u16_to_dev(a, dtype, dev):
     return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(dtype).to(dev)
 
 
-def device_layer(cfg: synth.Config, L: dict, banks: dict, max_tokens: int, dev="cuda", norm_topk: int = 1):
+def packed_correction(cfg: synth.Config, seed: int = 55):
+    """Ternary correction factors packed as PQ2_0 blocks by the oracle's packer: (A blocks
+    [r, d/128*34], B blocks [d, r/128*34])."""
+    rng = np.random.default_rng(seed)
+    r, d = cfg.rank, cfg.d
+    ca, sa = synth.ternary_codes(rng, (r, d)), synth.group_scales(rng, (r, d // 128))
+    cb, sb = synth.ternary_codes(rng, (d, r)), synth.group_scales(rng, (d, r // 128))
+    return oracle.pack(synth.PQ2_0, ca, sa), oracle.pack(synth.PQ2_0, cb, sb)
+
+
+def device_layer(cfg: synth.Config, L: dict, banks: dict, max_tokens: int, dev="cuda", norm_topk: int = 1,
+                 packed_corr=None):
     import torch
 
     import ternary_quantized_moe_b200 as tq
@@ -124,5 +135,7 @@ def device_layer(cfg: synth.Config, L: dict, banks: dict, max_tokens: int, dev="
         d=cfg.d, n_experts=cfg.n_experts, top_k=cfg.top_k, ffn=cfg.ffn, fmt=cfg.fmt, w_router=wr, w_router_delta=wd,
         gate_exps=torch.from_numpy(banks["gate"]).to(dev), up_exps=torch.from_numpy(banks["up"]).to(dev),
         down_exps=torch.from_numpy(banks["down"]).to(dev), shared_ffn=cfg.shared_ffn, sh_gate=opt("sh_gate"),
-        sh_up=opt("sh_up"), sh_down=opt("sh_down"), rank=cfg.rank, corr_a=opt("corr_a"), corr_b=opt("corr_b"),
-        norm_topk=norm_topk, max_tokens=max_tokens)
+        sh_up=opt("sh_up"), sh_down=opt("sh_down"), rank=cfg.rank,
+        corr_a=torch.from_numpy(packed_corr[0]).to(dev) if packed_corr else opt("corr_a"),
+        corr_b=torch.from_numpy(packed_corr[1]).to(dev) if packed_corr else opt("corr_b"),
+        corr_packed=1 if packed_corr else 0, norm_topk=norm_topk, max_tokens=max_tokens)

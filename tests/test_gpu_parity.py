@@ -7,7 +7,7 @@ import pytest
 
 import oracle
 from tests.helpers import (TOPK_MARGIN, bf16, check_output, device_layer, oracle_layer_packed, packed_banks,
-                           topk_gap, u16_to_dev, with_margin)
+                           packed_correction, topk_gap, u16_to_dev, with_margin)
 from workloads import synth
 
 torch = pytest.importorskip("torch")
@@ -271,6 +271,46 @@ def test_forward_residual(T, max_tokens, dense, in_place):
         np.testing.assert_array_equal(resid.cpu().numpy(), resid_h)  # only read
     ref, _, _ = oracle.forward(ol, x)
     check_output(out.cpu().numpy().astype(np.float64) - resid_h.astype(np.float64), ref)
+
+
+@pytest.mark.parametrize("fmt,T,max_tokens", [(synth.PQ2_0, 5, 64), (synth.PTQ1_0, 13, 64), (synth.PQ2_0, 40, 64),
+                                              (synth.PTQ1_0, 64, 64), (synth.PQ2_0, 200, 200),
+                                              (synth.PTQ1_0, 300, 300)])
+def test_forward_packed_correction(fmt, T, max_tokens):
+    """Ternary correction factors in PQ2_0 blocks: decode (split-K and ring passes; A read from
+    its blocks) and the tensor-core path (exact fp16 copies) against the oracle on the same
+    packed bytes, with the stage outputs z (hz) checked too."""
+    cfg = small("pc", fmt, False, E=16, k=4, Fs=128, r=256)
+    L, banks, ol, x = _case(cfg, T)
+    pa, pb = packed_correction(cfg)
+    ol.corr_a, ol.corr_b, ol.corr_packed = pa, pb, 1
+    x = with_margin(cfg, ol, x)
+    layer = device_layer(cfg, L, banks, max_tokens, packed_corr=(pa, pb))
+    got, dbg = run_forward(layer, x, T, debug=True, E=cfg.n_experts, k=cfg.top_k, F=cfg.ffn,
+                           Kdense=cfg.shared_ffn + cfg.rank)
+    assert tq.scion_layer_check(layer) == 0
+    hs, _ = oracle.shared(ol, x)
+    z, _ = oracle.corr(ol, x)
+    check_output(dbg["hz"].astype(np.float64), np.concatenate([hs, z], axis=1), rel_l2=1e-3)
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
+
+
+def test_packed_correction_rejects_invalid_codes_and_rank():
+    cfg = small("pcx", synth.PQ2_0, False, E=16, k=4, Fs=128, r=256)
+    L = synth.layer_host(cfg)
+    banks = packed_banks(cfg, L)
+    pa, pb = packed_correction(cfg)
+    bad = pb.copy()
+    bad[3, 5] = 0xFF  # four invalid fields
+    with pytest.raises(tq.ScionError) as ei:
+        device_layer(cfg, L, banks, 64, packed_corr=(pa, bad))
+    assert ei.value.status == tq.SCION_EFORMAT
+    cfg2 = small("pcr", synth.PQ2_0, False, E=16, k=4, Fs=128, r=16)
+    L2 = synth.layer_host(cfg2)
+    with pytest.raises(tq.ScionError) as ei:  # rank must be a multiple of 128 for packed factors
+        device_layer(cfg2, L2, packed_banks(cfg2, L2), 64, packed_corr=packed_correction(cfg))
+    assert ei.value.status == tq.SCION_EINVAL
 
 
 @pytest.mark.parametrize("T", [64, 65, 150])
