@@ -144,8 +144,9 @@ typedef struct {
   /* 0: corr_a / corr_b are bf16 [rank][d] and [d][rank].  1: ternary correction factors
    * ("Scion-35B-A3B" model card, Weight Representation: the corrections ship as 2-bit codes
    * plus one fp16 scale per 128, the q1_0_g128 container) as PQ2_0 blocks, corr_a [rank][d/128] and corr_b [d][rank/128] (groups of 128 along each
-   * factor's reduction axis; rank a multiple of 128).  Decode reads corr_a's blocks in place;
-   * corr_b, and corr_a for batches above 64 tokens, become exact fp16 copies (code * scale). */
+   * factor's reduction axis; rank a multiple of 128; 2-byte aligned).  Decode reads both
+   * factors' blocks in place (they must outlive the handle); the tensor-core path (batches
+   * above 64 tokens) uses exact fp16 copies (code * scale). */
   int corr_packed;
 } scion_layer_desc;
 
@@ -156,8 +157,8 @@ typedef struct scion_layer scion_layer;
  * bytes per 128 weights, regrouped into 16-byte-aligned tiles), converts
  * sh_down and corr_b to an fp16 copy, and allocates the workspace.  After it
  * returns, the caller may free gate_exps / up_exps / down_exps / sh_down /
- * corr_b; w_router, w_router_delta, sh_gate, sh_up, sh_gate_vec and corr_a are
- * read in place and must outlive the handle.  Synchronises `stream` once to
+ * corr_b (not corr_b's blocks when corr_packed); w_router, w_router_delta, sh_gate,
+ * sh_up, sh_gate_vec and corr_a are read in place and must outlive the handle.  Synchronises `stream` once to
  * validate every code: SCION_EFORMAT if a block holds an invalid code (no
  * handle is returned), EINVAL on a bad descriptor, ENOMEM, ECUDA.  Descriptor
  * limits: d and ffn multiples of 128 with d <= 4096, shared_ffn a multiple of 128,

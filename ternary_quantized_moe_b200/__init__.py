@@ -296,6 +296,8 @@ def scion_layer_create(*, d: int, n_experts: int, top_k: int, ffn: int, fmt: int
     st = _load().scion_layer_create(C.byref(D), int(max_tokens), _stream(stream), C.byref(h))
     _check(st, "scion_layer_create")
     keep = dict(w_router=w_router, w_router_delta=w_router_delta, sh_gate=sh_gate, sh_up=sh_up, corr_a=corr_a)
+    if corr_packed:
+        keep["corr_b"] = corr_b  # decode reads both factors' blocks in place
     return Layer(h.value, keep, d, n_experts, top_k, ffn, shared_ffn, rank, max_tokens)
 
 

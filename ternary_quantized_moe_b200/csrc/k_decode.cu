@@ -117,6 +117,14 @@ __device__ __forceinline__ uint4 tern8_bf16(uint32_t c16) {
   return make_uint4(tern_pair_bf16(c16), tern_pair_bf16(c16 >> 4), tern_pair_bf16(c16 >> 8), tern_pair_bf16(c16 >> 12));
 }
 
+__device__ __forceinline__ uint32_t tern_pair_f16(uint32_t f) {
+  const __half2 v = __floats2half2_rn(float(int(f & 3u) - 1), float(int((f >> 2) & 3u) - 1));
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+__device__ __forceinline__ uint4 tern8_f16(uint32_t c16) {
+  return make_uint4(tern_pair_f16(c16), tern_pair_f16(c16 >> 4), tern_pair_f16(c16 >> 8), tern_pair_f16(c16 >> 12));
+}
+
 template <int NT>
 __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
   extern __shared__ __align__(16) uint8_t xsm[];
@@ -449,6 +457,10 @@ struct DenseArgs {
   const __half* hz; // [T][Kd]
   int d, Kd, T;
   float* out;
+  // ternary correction B (PQ2_0 blocks [d][r/128]) read in place for columns Fs .. Fs + r
+  // (nullptr: every column from w)
+  const uint8_t* corr_b;
+  int Fs, r;
 };
 
 constexpr int kDnKc = 256;            // K columns per CTA
@@ -467,10 +479,27 @@ __device__ __forceinline__ void dense_body(const DenseArgs& a, int bx, int by) {
   // weights first (they do not depend on earlier kernels): 64 columns of rows g8 and g8 + 8
   uint4 wa[2], wb[2];
   const bool kin = kw < a.Kd;
+  // ternary correction columns: one group of 128 per warp slice, scaled after the MMAs
+  const bool tern = a.corr_b != nullptr && kw >= a.Fs && kw < a.Fs + a.r;
+  float sc_a = 0.f, sc_b = 0.f;
+  if (tern) {
+    const int Gr = a.r >> 7, kk = kw - a.Fs, g = kk >> 7, hoff = kk & 127;
+    const uint8_t* ba = a.corr_b + (int64_t(row0 + g8) * Gr + g) * 34;
+    const uint8_t* bb = a.corr_b + (int64_t(row0 + g8 + 8) * Gr + g) * 34;
 #pragma unroll
-  for (int q = 0; q < 2; ++q) {
-    wa[q] = kin ? ldg_stream(a.w + int64_t(row0 + g8) * a.Kd + kw + 32 * q + 8 * c) : make_uint4(0, 0, 0, 0);
-    wb[q] = kin ? ldg_stream(a.w + int64_t(row0 + g8 + 8) * a.Kd + kw + 32 * q + 8 * c) : make_uint4(0, 0, 0, 0);
+    for (int q = 0; q < 2; ++q) {
+      const int j0 = hoff + 32 * q + 8 * c;
+      wa[q] = tern8_f16(__ldg(reinterpret_cast<const unsigned short*>(ba + (j0 >> 2))));
+      wb[q] = tern8_f16(__ldg(reinterpret_cast<const unsigned short*>(bb + (j0 >> 2))));
+    }
+    sc_a = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short*>(ba + 32))));
+    sc_b = __half2float(__ushort_as_half(__ldg(reinterpret_cast<const unsigned short*>(bb + 32))));
+  } else {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      wa[q] = kin ? ldg_stream(a.w + int64_t(row0 + g8) * a.Kd + kw + 32 * q + 8 * c) : make_uint4(0, 0, 0, 0);
+      wb[q] = kin ? ldg_stream(a.w + int64_t(row0 + g8 + 8) * a.Kd + kw + 32 * q + 8 * c) : make_uint4(0, 0, 0, 0);
+    }
   }
   pdl_wait();
   const int kcols = min(kDnKc, a.Kd - kc0);  // multiple of 64
@@ -502,6 +531,10 @@ __device__ __forceinline__ void dense_body(const DenseArgs& a, int bx, int by) {
         mma_f16_16816(acc[nt], fa1, xb.z, xb.w);
       }
     }
+  }
+  if (tern) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] *= sc_a, acc[nt][1] *= sc_a, acc[nt][2] *= sc_b, acc[nt][3] *= sc_b;
   }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
@@ -622,6 +655,7 @@ cudaError_t launch_gateup_dense(const scion_layer* L, int T, float* out, cudaStr
   a.hfrag = L->h;
   DenseArgs b;
   b.w = L->dense_down, b.hz = L->hz, b.d = L->d, b.Kd = L->Kd, b.T = T, b.out = out;
+  b.corr_b = L->desc.corr_packed ? static_cast<const uint8_t*>(L->desc.corr_b) : nullptr, b.Fs = L->Fs, b.r = L->r;
   const int slots = min(L->E, T * L->k);
   const int gx = L->F / 16, dense_x = L->d / 32;
   const int dense_tiles = dense_x * ((L->Kd + kDnKc - 1) / kDnKc);
@@ -673,6 +707,7 @@ cudaError_t launch_down_dense(const scion_layer* L, int T, float* out, cudaStrea
   if (L->Kdense == 0) return cudaSuccess;
   DenseArgs b;
   b.w = L->dense_down, b.hz = L->hz, b.d = L->d, b.Kd = L->Kd, b.T = T, b.out = out;
+  b.corr_b = L->desc.corr_packed ? static_cast<const uint8_t*>(L->desc.corr_b) : nullptr, b.Fs = L->Fs, b.r = L->r;
   const int nt = (T + 7) / 8;
   const dim3 g2(L->d / 32, (L->Kd + kDnKc - 1) / kDnKc);
   switch (nt) {
