@@ -63,34 +63,36 @@ def parse():
     ap.add_argument("--impl", default="scion", choices=["scion", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0, help="override the number of cycled layers")
+    ap.add_argument("--packed-corr", action="store_true",
+                    help="ternary correction factors (PQ2_0 blocks) instead of the workload's bf16 ones")
     ap.add_argument("--stream-min-tokens", type=int, default=0,
                     help="decode batches of at least this many tokens use the bulk-copy ring expert kernels")
     return ap.parse_args()
 
 
 # ------------------------------------------------------------------- algorithmic work
-def workload_bytes(cfg, T, U):
+def workload_bytes(cfg, T, U, cb=2.0):
     """Algorithmic HBM bytes of one forward: U active experts' packed banks, the dense
-    bf16 weights (router + delta, shared expert, correction), x in and out."""
+    bf16 weights (router + delta, shared expert), the correction factors (cb bytes per
+    weight: 2 for bf16, 34/128 for PQ2_0 blocks), x in and out."""
     bb = 34 if cfg.fmt == 0 else 28
     per_expert = 3 * cfg.ffn * cfg.d * bb // 128
-    fixed = (2 * cfg.n_experts * cfg.d + 3 * cfg.shared_ffn * cfg.d + 2 * cfg.rank * cfg.d) * 2
+    fixed = (2 * cfg.n_experts * cfg.d + 3 * cfg.shared_ffn * cfg.d) * 2 + 2 * cfg.rank * cfg.d * cb
     return U * per_expert + fixed + T * cfg.d * (2 + 4)
 
 
-def stage_bytes(cfg, T, U):
-    """Algorithmic bytes per launch of each kernel stage."""
+def stage_bytes(cfg, T, U, cb=2.0):
+    """Algorithmic bytes per launch of each kernel stage (cb as in workload_bytes)."""
     bb = 34 if cfg.fmt == 0 else 28
     d, F, k, Fs, r, E = cfg.d, cfg.ffn, cfg.top_k, cfg.shared_ffn, cfg.rank, cfg.n_experts
-    rf = 4 if cfg.router_f32 else 2
     return {
         "router_f32": 2 * E * d * 4 + T * d * 2 + T * E * 4,
-        "xproj": ((0 if cfg.router_f32 else 2 * E * d) + 2 * Fs * d + r * d) * 2 + T * d * 2 + T * E * 4
+        "xproj": ((0 if cfg.router_f32 else 2 * E * d) + 2 * Fs * d) * 2 + r * d * cb + T * d * 2 + T * E * 4
         + T * (Fs + r) * 2,
         "route": T * E * 4 + T * k * 12 + E * 12,
         "gateup": U * 2 * F * d * bb // 128 + T * d * 2 + T * k * F * 2,
         "down_routed": U * F * d * bb // 128 + T * k * F * 2 + T * d * 4,
-        "down_dense": d * (Fs + r) * 2 + T * (Fs + r) * 2 + T * d * 4,
+        "down_dense": d * Fs * 2 + d * r * cb + T * (Fs + r) * 2 + T * d * 4,
     }
 
 
@@ -285,15 +287,27 @@ def run_gpu(args, rank, world, local_rank):
 
     # ---- layers (generated and packed on the GPU, then re-tiled by scion_layer_create)
     layers = []
+    cb = 34.0 / 128.0 if args.packed_corr else 2.0
     for l in range(n_layers):
         W = synth.layer_device(cfg, l, dev)
         banks = {n: tq.scion_pack_device(cfg.fmt, W.pop(n + "_codes"), W.pop(n + "_scales")) for n in
                  ("gate", "up", "down")}
+        corr = dict(corr_a=W.get("corr_a"), corr_b=W.get("corr_b"))
+        if args.packed_corr and cfg.rank:
+            # ternary correction factors with the experts' code and scale distributions
+            corr = {}
+            for name, rows, K in (("corr_a", cfg.rank, cfg.d), ("corr_b", cfg.d, cfg.rank)):
+                g = torch.Generator(device=dev)
+                g.manual_seed(7000 + 31 * l + rows)
+                u = torch.randint(0, 10, (rows, K), generator=g, device=dev)
+                codes = torch.where(u < 4, 0, torch.where(u < 7, 1, -1)).to(torch.int8)
+                scales = (torch.rand((rows, K // 128), generator=g, device=dev) * 0.015 + 0.005).half()
+                corr[name] = tq.scion_pack_device(synth.PQ2_0, codes, scales.view(torch.int16))
         layers.append(tq.scion_layer_create(
             d=cfg.d, n_experts=cfg.n_experts, top_k=cfg.top_k, ffn=cfg.ffn, fmt=cfg.fmt, w_router=W["w_router"],
             w_router_delta=W["w_delta"], gate_exps=banks["gate"], up_exps=banks["up"], down_exps=banks["down"],
             shared_ffn=cfg.shared_ffn, sh_gate=W.get("sh_gate"), sh_up=W.get("sh_up"), sh_down=W.get("sh_down"),
-            rank=cfg.rank, corr_a=W.get("corr_a"), corr_b=W.get("corr_b"), max_tokens=max_T))
+            rank=cfg.rank, max_tokens=max_T, corr_packed=1 if args.packed_corr and cfg.rank else 0, **corr))
         del banks, W
         if args.stream_min_tokens:
             tq.scion_layer_set_option(layers[-1], tq.SCION_OPT_STREAM_MIN_TOKENS, args.stream_min_tokens)
@@ -358,10 +372,10 @@ def run_gpu(args, rank, world, local_rank):
             else:
                 U[(li, T)] = cfg.n_experts
     sched = [((s * nb + i) % n_layers, T) for s in range(K) for i, T in enumerate(batches)]
-    bytes_total = sum(workload_bytes(cfg, T, U[(li, T)]) for li, T in sched)
+    bytes_total = sum(workload_bytes(cfg, T, U[(li, T)], cb) for li, T in sched)
     sbytes, sflops = {}, {}
     for li, T in sched:
-        for k_, v in stage_bytes(cfg, T, U[(li, T)]).items():
+        for k_, v in stage_bytes(cfg, T, U[(li, T)], cb).items():
             sbytes[k_] = sbytes.get(k_, 0) + v
         for k_, v in stage_flops(cfg, T).items():
             sflops[k_] = sflops.get(k_, 0) + v
@@ -373,7 +387,7 @@ def run_gpu(args, rank, world, local_rank):
         def one(s, T=T):
             tq.scion_moe_forward(xs[T], T, layers[s % n_layers], outs[T], stream)
         msT = timed(one, K)
-        bT = sum(workload_bytes(cfg, T, U[(s % n_layers, T)]) for s in range(K))
+        bT = sum(workload_bytes(cfg, T, U[(s % n_layers, T)], cb) for s in range(K))
         per_batch[str(T)] = {"tokens_per_s": job_tokens_per_s(world, T, K, msT), "us_per_call": 1000.0 * msT / K,
                              "hbm_frac": (bT / (msT / 1000.0)) / (peaks["hbm_gbs"] * 1e9)}
 
@@ -413,7 +427,7 @@ def run_gpu(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": cfg.name, "d": cfg.d, "experts": cfg.n_experts, "top_k": cfg.top_k, "ffn": cfg.ffn,
                    "shared_ffn": cfg.shared_ffn, "rank": cfg.rank, "format": "PQ2_0" if cfg.fmt == 0 else "PTQ1_0",
-                   "batches": batches, "layers_cycled": n_layers, "tokens_per_step": tokens_per_step,
+                   "correction": "PQ2_0 blocks" if args.packed_corr else "bf16", "batches": batches, "layers_cycled": n_layers, "tokens_per_step": tokens_per_step,
                    "l2": "inputs larger than L2: %.1f GB of layers cycled" % (weight_bytes / 1e9),
                    "parallelism": "replicas" if world > 1 else "single"},
         "roofline": roof,

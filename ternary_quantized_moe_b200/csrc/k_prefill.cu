@@ -140,11 +140,13 @@ struct DenseUnit {
   int row0;    // first weight row
   int nrows;   // valid rows of the matrices
   int col0;    // output column offset (hz column, logit column or out column)
+  int b16;     // 1: fp16 operands with B = DenseParams::b16 (x16; the ternary correction A's units)
 };
 
 struct DenseParams {
   CUtensorMap a[6];  // A matrices, box {64, 128}
   CUtensorMap b;     // B (tokens x K), box {64, 128}
+  CUtensorMap b16;   // B of the units with b16 set: x16 (tokens x K fp16)
   const DenseUnit* units;
   int n_units2;      // units with two A matrices (listed first)
   int n_units;
@@ -226,8 +228,9 @@ __global__ void __launch_bounds__(kThreads, 1) dense_gemm_kernel(const __grid_co
           tma_load_2d(bdst, &p.a[u.mat1], kb * kBK, u.row0, &full[s]);
           bdst += 128 * kBK * 2;
         }
-        tma_load_2d(bdst, &p.b, kb * kBK, dt.tok0, &full[s]);
-        if (dt.ntok == 256) tma_load_2d(bdst + 128 * kBK * 2, &p.b, kb * kBK, dt.tok0 + 128, &full[s]);
+        const CUtensorMap* bm = u.b16 ? &p.b16 : &p.b;
+        tma_load_2d(bdst, bm, kb * kBK, dt.tok0, &full[s]);
+        if (dt.ntok == 256) tma_load_2d(bdst + 128 * kBK * 2, bm, kb * kBK, dt.tok0 + 128, &full[s]);
       }
     }
     // copies of the last ring positions may still be in flight if a consumer gave up
@@ -243,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_gemm_kernel(const __grid_co
       if (li >= 2 && !mbar_wait(&acc_empty[ab], ((li >> 1) - 1) & 1, &abort_flag, p.err)) break;
       tc_fence_after();
       const uint32_t acc = tmem + 256 * ab;
-      const uint32_t idesc = umma_idesc(kBM, dt.ntok, p.ab_bf16);
+      const uint32_t idesc = umma_idesc(kBM, dt.ntok, u.b16 ? 0 : p.ab_bf16);
       bool ok = true;
       for (int kb = 0; kb < nk; ++kb, ++ks) {
         const int s = ks % kDenseStages;
@@ -956,16 +959,6 @@ cudaError_t launch_dequant_corr(const uint8_t* blocks, int rows, int K, __half* 
   return cudaGetLastError();
 }
 
-// Units of the correction A when its factors are ternary: an fp16 GEMM against x16 (the
-// fp16 copy of A is stored in x16's column order), writing z into hz after the shared part.
-void prefill_corr_units(const scion_layer* L, void* cunits_host, int* n_c) {
-  DenseUnit* cu = static_cast<DenseUnit*>(cunits_host);
-  int nc = 0;
-  if (L->desc.corr_packed)
-    for (int r0 = 0; r0 < L->r; r0 += 128) cu[nc++] = DenseUnit{kEpiPlain, 1, 0, 4, 4, r0, L->r, L->Fs};
-  *n_c = nc;
-}
-
 void prefill_units(const scion_layer* L, void* xunits_host, int* n_x, void* dunits_host, int* n_d) {
   DenseUnit* xu = static_cast<DenseUnit*>(xunits_host);
   DenseUnit* du = static_cast<DenseUnit*>(dunits_host);
@@ -975,8 +968,9 @@ void prefill_units(const scion_layer* L, void* xunits_host, int* n_x, void* duni
   if (!L->desc.router_fp32)
     for (int r0 = 0; r0 < L->E; r0 += 128) xu[nx++] = DenseUnit{kEpiLogits, 2, 0, 0, 1, r0, L->E, 0};
   for (int r0 = 0; r0 < L->Fs; r0 += 128) xu[nx++] = DenseUnit{kEpiSwiglu, 2, 1, 2, 3, r0, L->Fs, 0};
-  if (!L->desc.corr_packed)
-    for (int r0 = 0; r0 < L->r; r0 += 128) xu[nx++] = DenseUnit{kEpiPlain, 1, 0, 4, 4, r0, L->r, L->Fs};
+  // ternary correction factors: A's exact fp16 copy (x16 column order) against x16
+  const int b16 = L->desc.corr_packed ? 1 : 0;
+  for (int r0 = 0; r0 < L->r; r0 += 128) xu[nx++] = DenseUnit{kEpiPlain, 1, 0, 4, 4, r0, L->r, L->Fs, b16};
   if (L->Kdense)
     for (int r0 = 0; r0 < L->d; r0 += 128) du[nd++] = DenseUnit{kEpiStore, 1, 0, 5, 5, r0, L->d, 0};
   *n_x = nx;
@@ -1000,7 +994,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       return cudaGetLastError();
     }
     case SCION_STAGE_XPROJ: {
-      if (P.n_xunits == 0 && P.n_cunits == 0) return cudaSuccess;
+      if (P.n_xunits == 0) return cudaSuccess;
       DenseParams dp;
       memcpy(dp.a, P.maps, sizeof(dp.a));
       if (make_tmap_2d(&dp.b, x, 1, T, L->d) != SCION_OK) return cudaErrorInvalidValue;
@@ -1010,12 +1004,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       dp.logits = P.logits, dp.ld_logits = L->E, dp.hz = P.hz, dp.ld_hz = L->Kd, dp.out = nullptr, dp.ld_out = 0;
       dp.resid = nullptr;
       dp.err = L->err;
-      if (dp.n_units) dense_gemm_kernel<<<dense_grid(dp), kThreads, kDenseSmem, s>>>(dp);
-      cudaError_t e = cudaGetLastError();
-      if (e != cudaSuccess || P.n_cunits == 0) return e;
-      // ternary correction factors: z = A x as an fp16 GEMM of A's exact fp16 copy against x16
-      dp.b = P.x16_map, dp.ab_bf16 = 0;
-      dp.units = static_cast<const DenseUnit*>(P.cunits), dp.n_units = P.n_cunits, dp.n_units2 = 0;
+      if (L->desc.corr_packed) dp.b16 = P.x16_map;
       dense_gemm_kernel<<<dense_grid(dp), kThreads, kDenseSmem, s>>>(dp);
       return cudaGetLastError();
     }

@@ -54,7 +54,7 @@ void free_layer(scion_layer* L) {
   if (L->pre) {
     scion::PrefillState* P = L->pre;
     void* pp[] = {P->xunits, P->dunits, P->logits, P->ids, P->gates, P->counts, P->offsets, P->perm, P->inv,
-                  P->y, P->tiles, P->n_tiles, P->x16, P->h, P->hz, P->cursor, P->cunits, P->corr_a16};
+                  P->y, P->tiles, P->n_tiles, P->x16, P->h, P->hz, P->cursor, P->corr_a16};
     for (void* p : pp)
       if (p) cudaFree(p);
     delete P;
@@ -96,11 +96,7 @@ int create_prefill(scion_layer* L, cudaStream_t s) {
   PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->dunits), scion::prefill_unit_bytes() * max_units));
   PTRY(cudaMemcpyAsync(P->xunits, xu.data(), xu.size(), cudaMemcpyHostToDevice, s));
   PTRY(cudaMemcpyAsync(P->dunits, du.data(), du.size(), cudaMemcpyHostToDevice, s));
-  std::vector<uint8_t> cu(scion::prefill_unit_bytes() * max_units);
-  scion::prefill_corr_units(L, cu.data(), &P->n_cunits);
-  if (P->n_cunits) {
-    PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->cunits), scion::prefill_unit_bytes() * P->n_cunits));
-    PTRY(cudaMemcpyAsync(P->cunits, cu.data(), scion::prefill_unit_bytes() * P->n_cunits, cudaMemcpyHostToDevice, s));
+  if (L->r && L->desc.corr_packed) {
     PTRY(dev_alloc(L, &P->corr_a16, sizeof(__half) * size_t(L->r) * L->d));
     PTRY(scion::launch_dequant_corr(static_cast<const uint8_t*>(L->desc.corr_a), L->r, L->d, P->corr_a16, L->d, L->fmt,
                                     L->bad, s));
@@ -117,7 +113,7 @@ int create_prefill(scion_layer* L, cudaStream_t s) {
     if ((st = scion::make_tmap_2d(&P->maps[3], D.sh_up, 1, L->Fs, L->d))) return st;
   }
   if (L->r && !D.corr_packed && (st = scion::make_tmap_2d(&P->maps[4], D.corr_a, 1, L->r, L->d))) return st;
-  if (P->n_cunits) {
+  if (L->r && D.corr_packed) {
     if ((st = scion::make_tmap_2d(&P->maps[4], P->corr_a16, 0, L->r, L->d))) return st;
     if ((st = scion::make_tmap_2d(&P->x16_map, P->x16, 0, L->max_tokens, L->d))) return st;
   }

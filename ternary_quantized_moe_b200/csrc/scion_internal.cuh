@@ -67,9 +67,7 @@ struct PrefillState {
   int n_xunits;
   void* dunits;
   int n_dunits;
-  void* cunits;         // correction-A units of ternary correction factors (fp16 GEMM against x16)
-  int n_cunits;
-  CUtensorMap x16_map;  // B operand of those units
+  CUtensorMap x16_map;  // B operand of the ternary correction A's units (fp16 GEMM against x16)
   __half* corr_a16;     // [r][d] exact fp16 copy of the ternary correction A in x16's column order
   float* logits;        // [maxT][E]
   int32_t* ids;         // [maxT][k]
@@ -177,7 +175,6 @@ size_t prefill_unit_bytes();
 size_t prefill_tile_bytes();
 int prefill_max_units(const scion_layer* L);
 void prefill_units(const scion_layer* L, void* xunits_host, int* n_x, void* dunits_host, int* n_d);
-void prefill_corr_units(const scion_layer* L, void* cunits_host, int* n_c);
 cudaError_t launch_dequant_corr(const uint8_t* blocks, int rows, int K, __half* dst, int ld, int order,
                                 int64_t* bad, cudaStream_t s);
 cudaError_t launch_unperm_prefill(int fmt, const __half* src, int64_t n, __half* dst, cudaStream_t s);
