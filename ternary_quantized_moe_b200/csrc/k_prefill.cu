@@ -379,6 +379,8 @@ struct TernParams {
 };
 
 constexpr uint32_t kAtom = 128 * 128;  // bytes of one 128-row x 64-column swizzled atom
+constexpr int kBN2 = 256;      // tokens per down-projection tile of long batches
+constexpr int kBig256 = 192;   // mean tokens per expert from which the down projection takes kBN2 tiles
 
 // Expand half h (64 columns) of row t (0..127) of one 128-row group from its sub-tile block
 // into 32 registers of fp16 pairs, in position order (v[i] = positions 2i, 2i+1 of the half).
@@ -461,20 +463,27 @@ __device__ __forceinline__ void expand_ptq1_half(uint32_t codes, int t, int h, u
 }
 
 // Pipeline granularity: one 128-column code group along K ("group" = two 64-column halves).
-template <int FMT, int NA>
+// TN = tokens per tile: 128 (both GEMMs) or 256 (down projection of batches whose experts
+// average at least kBig256 tokens).
+template <int FMT, int NA, int TN = kBN>
 struct TernRing {
   static constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
   // shared memory: B groups (two 128-row x 128 B atoms each) and packed code groups
-  static constexpr int kB = 4;
+  // 256-token tiles: a B group is four atoms (two 128-row boxes per 64-column K block)
+  static_assert(TN == kBN || (TN == kBN2 && NA == 1), "256-token tiles: down projection only");
+  static constexpr int kB = TN == kBN2 ? 2 : 4;
   static constexpr int kC = 4;
-  static constexpr uint32_t b_bytes = 2 * kAtom;
+  static constexpr uint32_t b_kblock = TN == kBN2 ? 2 * kAtom : kAtom;  // bytes of one 64-column K block of B
+  static constexpr uint32_t b_bytes = 2 * b_kblock;
   static constexpr uint32_t c_bytes = NA * 8 * tb;
   static constexpr uint32_t b_off = 0, c_off = kB * b_bytes;
   static constexpr uint32_t bytes = c_off + kC * c_bytes;
   // tensor memory: accumulators, then the ring of expanded A groups
-  static constexpr int n_acc = NA == 2 ? 1 : 2;   // gate/up: one NA x 128 accumulator; down: ping-pong
-  static constexpr uint32_t acc_cols = NA * kBN;
-  static constexpr int kA = NA == 2 ? 2 : 4;      // down: the TMEM left over by the accumulators
+  // gate/up: one NA x 128 accumulator; down: two 128-column accumulators (ping-pong), or one of
+  // 256 columns for 256-token tiles
+  static constexpr int n_acc = NA == 1 && TN == kBN ? 2 : 1;
+  static constexpr uint32_t acc_cols = NA * TN;
+  static constexpr int kA = NA == 2 ? 2 : 4;
   static constexpr uint32_t a_cols = NA * 64;     // one group: NA matrices x 64 columns (128 fp16 per lane)
   static constexpr uint32_t a_col0 = n_acc * acc_cols;
   static constexpr uint32_t tmem_cols = 512;
@@ -490,9 +499,9 @@ constexpr int kEpiThreads = 256;
 // reads A from there and the tokens (B) from shared memory.  All roles walk the same item
 // sequence; rings carry over from one item to the next.  The MMA issuer waits on a single
 // barrier per group: the expansion side folds the B-ready condition into its own arrival.
-template <int FMT, int NA>
+template <int FMT, int NA, int TN = kBN>
 __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid_constant__ TernParams p) {
-  using R = TernRing<FMT, NA>;
+  using R = TernRing<FMT, NA, TN>;
   constexpr bool kBTma = NA == 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);  // 1024-aligned, still __shared__
@@ -554,8 +563,11 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
           if (gs >= R::kB && !mbar_wait(&b_empty[s], ((gs / R::kB) - 1) & 1, &abort_flag, p.err)) break;
           uint8_t* dst = smem + R::b_off + s * R::b_bytes;
           mbar_arrive_expect_tx(&b_full[s], R::b_bytes);
-          tma_load_2d(dst, &p.bmap, g * 128, row0, &b_full[s]);
-          tma_load_2d(dst + kAtom, &p.bmap, g * 128 + 64, row0, &b_full[s]);
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb) {  // 64-column K blocks of the group, TN token rows each
+            tma_load_2d(dst + kb * R::b_kblock, &p.bmap, g * 128 + 64 * kb, row0, &b_full[s]);
+            if (TN == kBN2) tma_load_2d(dst + kb * R::b_kblock + kAtom, &p.bmap, g * 128 + 64 * kb, row0 + 128, &b_full[s]);
+          }
         }
       }
       for (int i = max(0, gs - R::kB); i < gs; ++i) mbar_drain(&b_full[i % R::kB], (i / R::kB) & 1);
@@ -626,7 +638,7 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
           const uint32_t at = tmem + R::a_col0 + sa * R::a_cols, bt = sbase + R::b_off + sb * R::b_bytes;
 #pragma unroll
           for (int k16 = 0; k16 < 8; ++k16) {
-            const uint64_t db = umma_desc_sw128(bt + (k16 >> 2) * kAtom + 32 * (k16 & 3));
+            const uint64_t db = umma_desc_sw128(bt + (k16 >> 2) * R::b_kblock + 32 * (k16 & 3));
 #pragma unroll
             for (int m = 0; m < NA; ++m) umma_ts(acc + m * kBN, at + m * 64 + 8 * k16, db, idesc, (g | k16) != 0);
           }
@@ -750,49 +762,56 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 // column of the grouped GEMMs is computed independently, and the combine sums a token's k rows
 // in slot order), so the scatter takes positions with one atomic per entry.
 //
-// One CTA: exclusive scan of the histogram, the per-expert cursors, and the 128-token tiles.
+// One CTA: exclusive scan of the histogram, the per-expert cursors, and the token tiles: of
+// 128 tokens (gate/up GEMM) and of 256 (down GEMM).
 constexpr int kScanThreads = 1024;
 __global__ void __launch_bounds__(kScanThreads) group_scan_kernel(const int32_t* __restrict__ counts, int E,
                                                                   int32_t* __restrict__ offsets,
                                                                   int32_t* __restrict__ cursor,
                                                                   TernTile* __restrict__ tiles,
-                                                                  int32_t* __restrict__ n_tiles) {
-  __shared__ int32_t wsum[kScanThreads / 32], wtile[kScanThreads / 32];
+                                                                  int32_t* __restrict__ n_tiles,
+                                                                  TernTile* __restrict__ tiles2,
+                                                                  int32_t* __restrict__ n_tiles2) {
+  __shared__ int32_t wsum[kScanThreads / 32], wtile[kScanThreads / 32], wtile2[kScanThreads / 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per = (E + kScanThreads - 1) / kScanThreads;  // experts per thread, contiguous
   const int e0 = min(E, threadIdx.x * per), e1 = min(E, e0 + per);
-  int cs = 0, ts = 0;
+  int cs = 0, ts = 0, ts2 = 0;
   for (int e = e0; e < e1; ++e) {
     const int c = counts[e];
-    cs += c, ts += (c + kBN - 1) / kBN;
+    cs += c, ts += (c + kBN - 1) / kBN, ts2 += (c + kBN2 - 1) / kBN2;
   }
-  // block-wide exclusive scan of (cs, ts)
-  int ic = cs, it = ts;
+  // block-wide exclusive scan of (cs, ts, ts2)
+  int ic = cs, it = ts, it2 = ts2;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int c2 = __shfl_up_sync(0xffffffffu, ic, o), t2 = __shfl_up_sync(0xffffffffu, it, o);
-    if (lane >= o) ic += c2, it += t2;
+    const int u2 = __shfl_up_sync(0xffffffffu, it2, o);
+    if (lane >= o) ic += c2, it += t2, it2 += u2;
   }
-  if (lane == 31) wsum[warp] = ic, wtile[warp] = it;
+  if (lane == 31) wsum[warp] = ic, wtile[warp] = it, wtile2[warp] = it2;
   __syncthreads();
   if (warp == 0) {
-    int a = wsum[lane], b = wtile[lane];
+    int a = wsum[lane], b = wtile[lane], b2 = wtile2[lane];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int a2 = __shfl_up_sync(0xffffffffu, a, o), b2 = __shfl_up_sync(0xffffffffu, b, o);
-      if (lane >= o) a += a2, b += b2;
+      const int a2 = __shfl_up_sync(0xffffffffu, a, o), x2 = __shfl_up_sync(0xffffffffu, b, o);
+      const int y2 = __shfl_up_sync(0xffffffffu, b2, o);
+      if (lane >= o) a += a2, b += x2, b2 += y2;
     }
-    wsum[lane] = a, wtile[lane] = b;
-    if (lane == 31) offsets[E] = a, *n_tiles = b;
+    wsum[lane] = a, wtile[lane] = b, wtile2[lane] = b2;
+    if (lane == 31) offsets[E] = a, *n_tiles = b, *n_tiles2 = b2;
   }
   __syncthreads();
   int run = (warp ? wsum[warp - 1] : 0) + ic - cs;
   int trun = (warp ? wtile[warp - 1] : 0) + it - ts;
+  int trun2 = (warp ? wtile2[warp - 1] : 0) + it2 - ts2;
   for (int e = e0; e < e1; ++e) {
     const int c = counts[e];
     offsets[e] = run;
     cursor[e] = run;
     for (int c0 = 0; c0 < c; c0 += kBN) tiles[trun++] = TernTile{e, c0, min(kBN, c - c0), run + c0};
+    for (int c0 = 0; c0 < c; c0 += kBN2) tiles2[trun2++] = TernTile{e, c0, min(kBN2, c - c0), run + c0};
     run += c;
   }
 }
@@ -864,11 +883,16 @@ int dense_grid(const DenseParams& dp) {
   return max(1, min(n_tiles, num_sms()));
 }
 
-size_t tern_smem(int na, int fmt) {
-  size_t b;
-  if (fmt == SCION_PQ2_0) b = na == 2 ? TernRing<SCION_PQ2_0, 2>::bytes : TernRing<SCION_PQ2_0, 1>::bytes;
-  else b = na == 2 ? TernRing<SCION_PTQ1_0, 2>::bytes : TernRing<SCION_PTQ1_0, 1>::bytes;
-  return b + 1024;
+template <int FMT, int NA, int TN>
+size_t tern_smem_t() {
+  return TernRing<FMT, NA, TN>::bytes + 1024;
+}
+size_t tern_smem(int na, int fmt, int tn = kBN) {
+  if (fmt == SCION_PQ2_0)
+    return na == 2 ? tern_smem_t<SCION_PQ2_0, 2, kBN>()
+                   : (tn == kBN2 ? tern_smem_t<SCION_PQ2_0, 1, kBN2>() : tern_smem_t<SCION_PQ2_0, 1, kBN>());
+  return na == 2 ? tern_smem_t<SCION_PTQ1_0, 2, kBN>()
+                 : (tn == kBN2 ? tern_smem_t<SCION_PTQ1_0, 1, kBN2>() : tern_smem_t<SCION_PTQ1_0, 1, kBN>());
 }
 constexpr size_t kDenseSmem = kDenseStages * kDenseStage + 1024;
 
@@ -904,6 +928,12 @@ cudaError_t configure_prefill_kernels() {
     return e;
   if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PTQ1_0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 int(tern_smem(1, SCION_PTQ1_0)))))
+    return e;
+  if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PQ2_0, 1, kBN2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(tern_smem(1, SCION_PQ2_0, kBN2)))))
+    return e;
+  if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PTQ1_0, 1, kBN2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(tern_smem(1, SCION_PTQ1_0, kBN2)))))
     return e;
   return cudaSuccess;
 }
@@ -1028,7 +1058,8 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
 #undef SCION_TOPK
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
       group_scan_kernel<<<1, kScanThreads, 0, s>>>(P.counts, L->E, P.offsets, P.cursor,
-                                                  static_cast<TernTile*>(P.tiles), P.n_tiles);
+                                                  static_cast<TernTile*>(P.tiles), P.n_tiles,
+                                                  static_cast<TernTile*>(P.tiles2), P.n_tiles2);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
       group_scatter_kernel<<<(n + 256 * ept - 1) / (256 * ept), 256, 2 * sizeof(int32_t) * L->E, s>>>(
           P.ids, n, L->E, ept, P.cursor, P.perm, P.inv);
@@ -1069,13 +1100,20 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       TernParams tp;
       tp.bank = L->dn_bank, tp.fmt = L->fmt, tp.na = 1, tp.G = L->GF, tp.R = L->d;
       tp.bsrc = P.h, tp.ldb = L->F;
-      tp.tiles = static_cast<const TernTile*>(P.tiles), tp.n_tiles = P.n_tiles;
+      // experts averaging many tokens: 256-token tiles (each expanded code group serves twice the
+      // tokens); otherwise 128-token tiles with a ping-pong accumulator that hides the epilogue
+      const bool big = int64_t(T) * L->k >= int64_t(kBig256) * L->E;
+      tp.tiles = static_cast<const TernTile*>(big ? P.tiles2 : P.tiles), tp.n_tiles = big ? P.n_tiles2 : P.n_tiles;
       tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gates = P.gates, tp.k = L->k;
       tp.h = nullptr, tp.F = L->F, tp.y = P.y, tp.d = L->d, tp.err = L->err;
       if (make_tmap_2d(&tp.bmap, P.h, 0, int64_t(T) * L->k, L->F) != SCION_OK) return cudaErrorInvalidValue;
       const dim3 grid(num_sms());
-      if (L->fmt == SCION_PQ2_0)
+      if (L->fmt == SCION_PQ2_0 && big)
+        tern_gemm_kernel<SCION_PQ2_0, 1, kBN2><<<grid, kTernThreads, tern_smem(1, L->fmt, kBN2), s>>>(tp);
+      else if (L->fmt == SCION_PQ2_0)
         tern_gemm_kernel<SCION_PQ2_0, 1><<<grid, kTernThreads, tern_smem(1, L->fmt), s>>>(tp);
+      else if (big)
+        tern_gemm_kernel<SCION_PTQ1_0, 1, kBN2><<<grid, kTernThreads, tern_smem(1, L->fmt, kBN2), s>>>(tp);
       else
         tern_gemm_kernel<SCION_PTQ1_0, 1><<<grid, kTernThreads, tern_smem(1, L->fmt), s>>>(tp);
       return cudaGetLastError();

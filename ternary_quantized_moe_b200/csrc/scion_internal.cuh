@@ -80,6 +80,8 @@ struct PrefillState {
   __half* y;            // [maxT*k][d] expert down outputs in fp16 (gate not yet applied), one row per routed entry
   void* tiles;          // 128-token tiles, [maxT*k/128 + E]
   int32_t* n_tiles;
+  void* tiles2;         // 256-token tiles (down projection), [maxT*k/256 + E]
+  int32_t* n_tiles2;
   __half* x16;          // [maxT][d]   x in the container column order (fp16)
   __half* h;            // [maxT*k][F] expert SwiGLU hidden, container column order
   __half* hz;           // [maxT][Kd]
