@@ -374,10 +374,16 @@ def run_gpu(args, rank, world, local_rank):
     sched = [((s * nb + i) % n_layers, T) for s in range(K) for i, T in enumerate(batches)]
     bytes_total = sum(workload_bytes(cfg, T, U[(li, T)], cb) for li, T in sched)
     sbytes, sflops = {}, {}
+    min_ring = args.stream_min_tokens or 16
     for li, T in sched:
-        for k_, v in stage_bytes(cfg, T, U[(li, T)], cb).items():
+        sb, sf = stage_bytes(cfg, T, U[(li, T)], cb), stage_flops(cfg, T)
+        if T < min_ring and (T + 7) // 8 <= 2 and cfg.shared_ffn + cfg.rank > 0:
+            # below the ring threshold the dense down projection runs inside the gate/up launch
+            sb["gateup"] += sb.pop("down_dense")
+            sf["gateup"] += sf.pop("down_dense")
+        for k_, v in sb.items():
             sbytes[k_] = sbytes.get(k_, 0) + v
-        for k_, v in stage_flops(cfg, T).items():
+        for k_, v in sf.items():
             sflops[k_] = sflops.get(k_, 0) + v
     flops_total = sum(workload_flops(cfg, T) for _, T in sched)
 
