@@ -86,6 +86,16 @@ int scion_pack_device(int fmt, const int8_t* codes, const uint16_t* scales, int6
 int scion_unpack_device(int fmt, const uint8_t* in, int64_t n_groups, int8_t* codes, uint16_t* scales,
                         int64_t* bad_count, void* stream);
 
+/* Test support for the failure path of the device-side waits: one kernel waits on a barrier
+ * phase that nothing completes, with a limit of limit_us (1 .. 10^6) microseconds; a second warp
+ * waits on another such phase with ten times the limit.  The first must give up on its clock
+ * and write SCION_ETIMEOUT, the second must leave on the abort flag the first raised.  result
+ * (host int[3]) receives {the status word, first wait's return, second wait's return} (expected
+ * {SCION_ETIMEOUT, 0, 0}); *elapsed_ms the time until both gave up.  No fault, no hang: the
+ * kernel ends after about limit_us plus the wait's suspend time (1 ms).  Synchronises `stream`.
+ * EINVAL on a bad argument, ENOMEM, ECUDA. */
+int scion_selftest_bounded_wait(int limit_us, int* result, double* elapsed_ms, void* stream);
+
 /* Float -> ternary quantizers ("Scion: ternary MoE quantization with trained corrections",
  * Findings: the deployable Lloyd quantizer against one-shot absmean; "Scion-35B-A3B" model
  * card, Highlights: ternary Lloyd g128).  w: device fp32, n_groups groups of 128 consecutive

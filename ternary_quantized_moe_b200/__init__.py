@@ -28,6 +28,7 @@ __all__ = [
     "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "STAGES", "scion_layer_check",
     "scion_router_logits_static", "scion_layer_set_option", "SCION_OPT_STREAM_MIN_TOKENS",
     "scion_moe_forward_residual", "scion_quantize_device", "SCION_QUANT_ABSMEAN", "SCION_QUANT_LLOYD",
+    "scion_selftest_bounded_wait",
 ]
 
 SCION_PQ2_0 = 0
@@ -46,6 +47,7 @@ EXPORTS = (
     "scion_layer_device_bytes", "scion_moe_forward", "scion_moe_forward_host", "scion_moe_forward_debug",
     "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "scion_layer_check",
     "scion_router_logits_static", "scion_layer_set_option", "scion_moe_forward_residual", "scion_quantize_device",
+    "scion_selftest_bounded_wait",
 )
 SCION_QUANT_ABSMEAN, SCION_QUANT_LLOYD = 0, 1
 SCION_OPT_STREAM_MIN_TOKENS = 1
@@ -103,6 +105,7 @@ def _load():
             "scion_moe_forward": (ci, [vp, ci, vp, vp, vp]),
             "scion_moe_forward_residual": (ci, [vp, ci, vp, vp, vp, vp]),
             "scion_quantize_device": (ci, [ci, vp, i64, ci, vp, vp, vp]),
+            "scion_selftest_bounded_wait": (ci, [ci, C.POINTER(C.c_int), C.POINTER(C.c_double), vp]),
             "scion_moe_forward_host": (ci, [vp, ci, vp, vp, vp]),
             "scion_moe_forward_debug": (ci, [vp, ci, vp, vp, C.POINTER(_Debug), vp]),
             "scion_profile_begin": (ci, [ci]),
@@ -206,6 +209,15 @@ def scion_pack_device(fmt: int, codes, scales, out=None, bad_count=None, stream=
                                    _stream(stream))
     _check(st, "scion_pack_device")
     return out
+
+
+def scion_selftest_bounded_wait(limit_us: int, stream=None):
+    """Runs the bounded-wait failure check; returns ((status, first_ok, second_ok), elapsed_ms)."""
+    res = (C.c_int * 3)()
+    ms = C.c_double()
+    st = _load().scion_selftest_bounded_wait(int(limit_us), res, C.byref(ms), _stream(stream))
+    _check(st, "scion_selftest_bounded_wait")
+    return (res[0], res[1], res[2]), ms.value
 
 
 def scion_quantize_device(method: int, w, codes, scales, iters: int = 30, stream=None) -> None:

@@ -508,3 +508,20 @@ def test_quantize_rejects_bad_arguments():
     with pytest.raises(tq.ScionError) as ei:  # w must be 16-byte aligned
         tq.scion_quantize_device(tq.SCION_QUANT_ABSMEAN, flat[1:], codes, scales)
     assert ei.value.status == tq.SCION_EINVAL
+
+
+# ------------------------------------------------------------------ failure path
+def test_bounded_wait_gives_up_and_context_stays_usable():
+    """A device wait on a barrier phase that nothing completes gives up after its limit with
+    SCION_ETIMEOUT in the status word; the other waiter leaves on the abort flag; the context then
+    still runs a forward correctly."""
+    (status, first_ok, second_ok), ms = tq.scion_selftest_bounded_wait(50000)  # 50 ms
+    assert status == tq.SCION_ETIMEOUT and first_ok == 0 and second_ok == 0
+    assert 50.0 <= ms < 200.0, ms
+    cfg = small("fw", synth.PQ2_0, False)
+    L, banks, ol, x = _case(cfg, 5)
+    layer = device_layer(cfg, L, banks, 64)
+    got, _ = run_forward(layer, x, 5)
+    assert tq.scion_layer_check(layer) == 0
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
