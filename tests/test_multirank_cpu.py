@@ -9,6 +9,7 @@ import os
 import socket
 import subprocess
 import sys
+import time
 
 import pytest
 import torch.multiprocessing as mp
@@ -72,3 +73,44 @@ def test_reference_arm_prints_on_rank_zero_only():
     line = json.loads(lines[0])
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _worker_leaves(rank, world, port, q):
+    from datetime import timedelta
+
+    import torch.distributed as dist
+
+    import bench
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=10))
+    if rank == 1:
+        os._exit(3)  # this rank dies between steps, before the timing collective
+    t0 = time.time()
+    try:
+        bench.max_over_ranks(1.0, world, "cpu")
+        q.put(("returned", time.time() - t0))
+    except Exception as e:  # noqa: BLE001 -- any error from the collective is the expected outcome
+        q.put((type(e).__name__, time.time() - t0))
+
+
+def test_a_rank_that_leaves_makes_the_collective_fail_not_hang():
+    """Failure handling between steps on the host: when a rank exits before the timing
+    collective, the surviving rank's collective ends with an error within the process group's
+    timeout instead of waiting for ever."""
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker_leaves, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    try:
+        kind, secs = q.get(timeout=120)
+    finally:
+        for p in procs:
+            p.join(timeout=60)
+            if p.is_alive():
+                p.kill()
+    assert kind != "returned", "the collective returned although a rank had left"
+    assert secs < 60.0
