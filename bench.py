@@ -373,6 +373,8 @@ def run_gpu(args, rank, world, local_rank):
                 U[(li, T)] = cfg.n_experts
     sched = [((s * nb + i) % n_layers, T) for s in range(K) for i, T in enumerate(batches)]
     bytes_total = sum(workload_bytes(cfg, T, U[(li, T)], cb) for li, T in sched)
+    # the active experts' packed banks alone (U distinct experts per call)
+    expert_bytes = sum(U[(li, T)] * 3 * cfg.ffn * cfg.d * (34 if cfg.fmt == 0 else 28) // 128 for li, T in sched)
     sbytes, sflops = {}, {}
     min_ring = args.stream_min_tokens or 16
     for li, T in sched:
@@ -438,7 +440,12 @@ def run_gpu(args, rank, world, local_rank):
                    "parallelism": "replicas" if world > 1 else "single"},
         "roofline": roof,
         "step_roofline": {"bytes_per_step": bytes_total / K, "hbm_frac": (bytes_total / (ms / 1000.0)) /
-                          (peaks["hbm_gbs"] * 1e9), "tflops": flops_total / (ms / 1000.0) / 1e12},
+                          (peaks["hbm_gbs"] * 1e9), "tflops": flops_total / (ms / 1000.0) / 1e12,
+                          "expert_bytes_per_step": expert_bytes / K,
+                          "expert_stage_hbm_frac": (expert_bytes / ((stages.get("gateup", (0, 0))[0] +
+                                                                     stages.get("down_routed", (0, 0))[0]) / 1000.0)
+                                                    / (peaks["hbm_gbs"] * 1e9))
+                          if stages.get("gateup", (0, 0))[0] > 0 else None},
         "per_batch": per_batch,
         "stages_us_per_launch": {k_: 1000.0 * v[0] / v[1] for k_, v in stages.items() if v[1]},
         "stages_rate": {k_: (sbytes[k_] / (v[0] / 1000.0) / 1e9 if decode else
