@@ -381,6 +381,8 @@ struct TernParams {
 constexpr uint32_t kAtom = 128 * 128;  // bytes of one 128-row x 64-column swizzled atom
 constexpr int kBN2 = 256;      // tokens per down-projection tile of long batches
 constexpr int kBig256 = 192;   // mean tokens per expert from which the down projection takes kBN2 tiles
+constexpr int kBN3 = 160;      // tokens per gate/up tile of batches whose experts average near 128
+constexpr int kMid160 = 112;   // mean tokens per expert from which (below kBig256) gate/up takes kBN3 tiles
 
 // Expand half h (64 columns) of row t (0..127) of one 128-row group from its sub-tile block
 // into 32 registers of fp16 pairs, in position order (v[i] = positions 2i, 2i+1 of the half).
@@ -463,17 +465,19 @@ __device__ __forceinline__ void expand_ptq1_half(uint32_t codes, int t, int h, u
 }
 
 // Pipeline granularity: one 128-column code group along K ("group" = two 64-column halves).
-// TN = tokens per tile: 128 (both GEMMs) or 256 (down projection of batches whose experts
-// average at least kBig256 tokens).
+// TN = tokens per tile: 128 (both GEMMs), 256 (down projection of batches whose experts
+// average at least kBig256 tokens) or 160 (gate/up of batches whose experts average between
+// kMid160 and kBig256 tokens: one tile holds nearly every expert's tokens, so each expert's
+// codes are expanded once).
 template <int FMT, int NA, int TN = kBN>
 struct TernRing {
   static constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
-  // shared memory: B groups (two 128-row x 128 B atoms each) and packed code groups
-  // 256-token tiles: a B group is four atoms (two 128-row boxes per 64-column K block)
-  static_assert(TN == kBN || (TN == kBN2 && NA == 1), "256-token tiles: down projection only");
+  // shared memory: B groups (two 64-column K blocks of TN swizzled 128-byte rows) and packed
+  // code groups
+  static_assert(TN == kBN || (TN == kBN2 && NA == 1) || (TN == kBN3 && NA == 2), "tile width");
   static constexpr int kB = TN == kBN2 ? 2 : 4;
   static constexpr int kC = 4;
-  static constexpr uint32_t b_kblock = TN == kBN2 ? 2 * kAtom : kAtom;  // bytes of one 64-column K block of B
+  static constexpr uint32_t b_kblock = uint32_t(TN) * 128;  // bytes of one 64-column K block of B
   static constexpr uint32_t b_bytes = 2 * b_kblock;
   static constexpr uint32_t c_bytes = NA * 8 * tb;
   static constexpr uint32_t b_off = 0, c_off = kB * b_bytes;
@@ -483,8 +487,12 @@ struct TernRing {
   // 256 columns for 256-token tiles
   static constexpr int n_acc = NA == 1 && TN == kBN ? 2 : 1;
   static constexpr uint32_t acc_cols = NA * TN;
-  static constexpr int kA = NA == 2 ? 2 : 4;
-  static constexpr uint32_t a_cols = NA * 64;     // one group: NA matrices x 64 columns (128 fp16 per lane)
+  // ring entries of expanded A: one group of all NA matrices, or (160-token gate/up tiles,
+  // whose accumulators leave 192 columns) one matrix of a group, EPG entries per group
+  static constexpr int EPG = TN == kBN3 ? NA : 1;
+  static constexpr int MPE = NA / EPG;           // matrices per entry
+  static constexpr int kA = TN == kBN3 ? 3 : (NA == 2 ? 2 : 4);
+  static constexpr uint32_t a_cols = MPE * 64;   // one entry: MPE matrices x 64 columns (128 fp16 per lane)
   static constexpr uint32_t a_col0 = n_acc * acc_cols;
   static constexpr uint32_t tmem_cols = 512;
   static_assert(a_col0 + kA * a_cols <= tmem_cols, "TMEM budget");
@@ -577,14 +585,15 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
     // warp 2 takes rows 0..63, warp 3 rows 64..127.  Lanes 2m and 2m+1 copy the two 16-byte
     // halves of one 32-byte sector of the same row, so every request is a whole L2 sector:
     // lane (m, hf) handles rows rbase + m + 16i (i < 4), 16-byte chunks 2j + hf (j < 8).
-    const int rbase = (warp - 2) * 64 + (lane >> 1), hf = lane & 1;
+    constexpr int kRows = TN / 32;   // rows per lane pair
+    const int rbase = (warp - 2) * (TN / 2) + (lane >> 1), hf = lane & 1;
     constexpr int kLag = R::kB / 2;  // groups in flight per thread before the oldest is published
     int gs = 0;                      // running group counter
     for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
       const TernTile tile = load_tile(p.tiles, item / RT);
-      const __half* rows[4];
+      const __half* rows[kRows];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < kRows; ++i) {
         const int r = rbase + 16 * i;
         rows[i] = r < tile.n ? p.bsrc + int64_t(p.perm[tile.pos0 + r] / p.k) * p.ldb + 8 * hf : nullptr;
       }
@@ -593,14 +602,14 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
         if (gs >= R::kB && !mbar_wait(&b_empty[s], ((gs / R::kB) - 1) & 1, &abort_flag, p.err)) break;
         const uint32_t bt = sbase + R::b_off + s * R::b_bytes;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kRows; ++i) {
           if (!rows[i]) continue;
           const int r = rbase + 16 * i;
           const __half* src = rows[i] + g * 128;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int ch = 2 * j + hf;  // 16-byte chunk of the row's 256 bytes
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(bt + (ch >> 3) * kAtom + sw128_offset(r, ch & 7)),
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(bt + (ch >> 3) * R::b_kblock + sw128_offset(r, ch & 7)),
                          "l"(src + 16 * j)
                          : "memory");
           }
@@ -620,7 +629,7 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer: A from tensor memory, B from shared memory
-      int gs = 0, li = 0;
+      int gs = 0, es = 0, li = 0;  // running group, A-entry and item counters
       TernTile next = blockIdx.x < n_items ? load_tile(p.tiles, blockIdx.x / RT) : TernTile{};
       for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x, ++li) {
         const TernTile tile = next;  // loaded one item ahead: no global-load latency between items
@@ -630,20 +639,27 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
         if (li >= R::n_acc && !mbar_wait(&acc_empty[ab], ((li / R::n_acc) - 1) & 1, &abort_flag, p.err)) break;
         tc_fence_after();
         const uint32_t acc = tmem + ab * R::acc_cols;
-        for (int g = 0; g < p.G; ++g, ++gs) {
-          const int sa = gs % R::kA, sb = gs % R::kB;
-          // A expanded and (folded into the same arrival) B landed
-          if (!mbar_wait(&a_full[sa], (gs / R::kA) & 1, &abort_flag, p.err)) break;
-          tc_fence_after();
-          const uint32_t at = tmem + R::a_col0 + sa * R::a_cols, bt = sbase + R::b_off + sb * R::b_bytes;
+        bool ok = true;
+        for (int g = 0; g < p.G && ok; ++g, ++gs) {
+          const int sb = gs % R::kB;
+          const uint32_t bt = sbase + R::b_off + sb * R::b_bytes;
 #pragma unroll
-          for (int k16 = 0; k16 < 8; ++k16) {
-            const uint64_t db = umma_desc_sw128(bt + (k16 >> 2) * R::b_kblock + 32 * (k16 & 3));
+          for (int eg = 0; eg < R::EPG; ++eg, ++es) {
+            const int sa = es % R::kA;
+            // A expanded and (folded into the group's first arrival) B landed
+            if (!(ok = mbar_wait(&a_full[sa], (es / R::kA) & 1, &abort_flag, p.err))) break;
+            tc_fence_after();
+            const uint32_t at = tmem + R::a_col0 + sa * R::a_cols;
 #pragma unroll
-            for (int m = 0; m < NA; ++m) umma_ts(acc + m * kBN, at + m * 64 + 8 * k16, db, idesc, (g | k16) != 0);
+            for (int k16 = 0; k16 < 8; ++k16) {
+              const uint64_t db = umma_desc_sw128(bt + (k16 >> 2) * R::b_kblock + 32 * (k16 & 3));
+#pragma unroll
+              for (int m = 0; m < R::MPE; ++m)
+                umma_ts(acc + (eg * R::MPE + m) * TN, at + m * 64 + 8 * k16, db, idesc, (g | k16) != 0);
+            }
+            umma_commit(&a_empty[sa]);
           }
-          umma_commit(&a_empty[sa]);
-          umma_commit(&b_empty[sb]);
+          if (ok) umma_commit(&b_empty[sb]);
         }
         umma_commit(&acc_full[ab]);
       }
@@ -658,28 +674,35 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
     const int t = (threadIdx.x - 128) & 127;
     const bool b_watch = part == 0 && t == 0;  // this thread also waits for the group's B rows
     const uint32_t lane_base = tmem + (uint32_t((warp & 3) * 32) << 16) + R::a_col0 + part * 32;
-    int gs = 0;  // running code-group counter
-    for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
-      for (int g = 0; g < p.G; ++g, ++gs) {
-        const int sc = gs % R::kC, sa = gs % R::kA;
-        if (!mbar_wait(&c_full[sc], (gs / R::kC) & 1, &abort_flag, p.err)) break;
-        if (gs >= R::kA && !mbar_wait(&a_empty[sa], ((gs / R::kA) - 1) & 1, &abort_flag, p.err)) break;
-        tc_fence_after();
+    int gs = 0, es = 0;  // running code-group and A-entry counters
+    bool ok = true;
+    for (int item = blockIdx.x; item < n_items && ok && !abort_flag; item += gridDim.x) {
+      for (int g = 0; g < p.G && ok; ++g, ++gs) {
+        const int sc = gs % R::kC;
+        if (!(ok = mbar_wait(&c_full[sc], (gs / R::kC) & 1, &abort_flag, p.err))) break;
         const uint32_t codes = sbase + R::c_off + sc * R::c_bytes;
 #pragma unroll
-        for (int m = 0; m < NA; ++m) {
-          uint32_t v[32];
-          if constexpr (FMT == SCION_PQ2_0)
-            expand_pq2_half(codes + m * 8 * R::tb, t, part, v);
-          else
-            expand_ptq1_half(codes + m * 8 * R::tb, t, part, v);
-          tmem_st32(lane_base + sa * R::a_cols + m * 64, v);
+        for (int eg = 0; eg < R::EPG; ++eg, ++es) {
+          const int sa = es % R::kA;
+          if (es >= R::kA && !(ok = mbar_wait(&a_empty[sa], ((es / R::kA) - 1) & 1, &abort_flag, p.err))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int m = 0; m < R::MPE; ++m) {
+            const int mat = eg * R::MPE + m;
+            uint32_t v[32];
+            if constexpr (FMT == SCION_PQ2_0)
+              expand_pq2_half(codes + mat * 8 * R::tb, t, part, v);
+            else
+              expand_ptq1_half(codes + mat * 8 * R::tb, t, part, v);
+            tmem_st32(lane_base + sa * R::a_cols + m * 64, v);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          if (eg == R::EPG - 1) mbar_arrive(&c_empty[sc]);
+          if (eg == 0 && b_watch && !(ok = mbar_wait(&b_full[gs % R::kB], (gs / R::kB) & 1, &abort_flag, p.err)))
+            break;
+          mbar_arrive(&a_full[sa]);
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&c_empty[sc]);
-        if (b_watch && !mbar_wait(&b_full[gs % R::kB], (gs / R::kB) & 1, &abort_flag, p.err)) break;
-        mbar_arrive(&a_full[sa]);
       }
     }
   } else if (warp >= 12) {
@@ -704,7 +727,7 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
       for (int c = half; c * 16 < nn; c += 2) {
         float v0[16], v1[16];
         if constexpr (NA == 2)
-          tmem_ld16x2(acc + c * 16, acc + kBN + c * 16, v0, v1);
+          tmem_ld16x2(acc + c * 16, acc + TN + c * 16, v0, v1);
         else
           tmem_ld16(acc + c * 16, v0);
         const int n0 = c * 16;
@@ -762,16 +785,16 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 // column of the grouped GEMMs is computed independently, and the combine sums a token's k rows
 // in slot order), so the scatter takes positions with one atomic per entry.
 //
-// One CTA: exclusive scan of the histogram, the per-expert cursors, and the token tiles: of
-// 128 tokens (gate/up GEMM) and of 256 (down GEMM).
+// One CTA: exclusive scan of the histogram, the per-expert cursors, and the token tiles of the
+// two ternary GEMMs: w1 tokens for gate/up (128 or 160), w2 for down (128 or 256).
 constexpr int kScanThreads = 1024;
 __global__ void __launch_bounds__(kScanThreads) group_scan_kernel(const int32_t* __restrict__ counts, int E,
                                                                   int32_t* __restrict__ offsets,
                                                                   int32_t* __restrict__ cursor,
                                                                   TernTile* __restrict__ tiles,
-                                                                  int32_t* __restrict__ n_tiles,
+                                                                  int32_t* __restrict__ n_tiles, int w1,
                                                                   TernTile* __restrict__ tiles2,
-                                                                  int32_t* __restrict__ n_tiles2) {
+                                                                  int32_t* __restrict__ n_tiles2, int w2) {
   __shared__ int32_t wsum[kScanThreads / 32], wtile[kScanThreads / 32], wtile2[kScanThreads / 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per = (E + kScanThreads - 1) / kScanThreads;  // experts per thread, contiguous
@@ -779,7 +802,7 @@ __global__ void __launch_bounds__(kScanThreads) group_scan_kernel(const int32_t*
   int cs = 0, ts = 0, ts2 = 0;
   for (int e = e0; e < e1; ++e) {
     const int c = counts[e];
-    cs += c, ts += (c + kBN - 1) / kBN, ts2 += (c + kBN2 - 1) / kBN2;
+    cs += c, ts += (c + w1 - 1) / w1, ts2 += (c + w2 - 1) / w2;
   }
   // block-wide exclusive scan of (cs, ts, ts2)
   int ic = cs, it = ts, it2 = ts2;
@@ -810,8 +833,8 @@ __global__ void __launch_bounds__(kScanThreads) group_scan_kernel(const int32_t*
     const int c = counts[e];
     offsets[e] = run;
     cursor[e] = run;
-    for (int c0 = 0; c0 < c; c0 += kBN) tiles[trun++] = TernTile{e, c0, min(kBN, c - c0), run + c0};
-    for (int c0 = 0; c0 < c; c0 += kBN2) tiles2[trun2++] = TernTile{e, c0, min(kBN2, c - c0), run + c0};
+    for (int c0 = 0; c0 < c; c0 += w1) tiles[trun++] = TernTile{e, c0, min(w1, c - c0), run + c0};
+    for (int c0 = 0; c0 < c; c0 += w2) tiles2[trun2++] = TernTile{e, c0, min(w2, c - c0), run + c0};
     run += c;
   }
 }
@@ -889,11 +912,16 @@ size_t tern_smem_t() {
 }
 size_t tern_smem(int na, int fmt, int tn = kBN) {
   if (fmt == SCION_PQ2_0)
-    return na == 2 ? tern_smem_t<SCION_PQ2_0, 2, kBN>()
+    return na == 2 ? (tn == kBN3 ? tern_smem_t<SCION_PQ2_0, 2, kBN3>() : tern_smem_t<SCION_PQ2_0, 2, kBN>())
                    : (tn == kBN2 ? tern_smem_t<SCION_PQ2_0, 1, kBN2>() : tern_smem_t<SCION_PQ2_0, 1, kBN>());
-  return na == 2 ? tern_smem_t<SCION_PTQ1_0, 2, kBN>()
+  return na == 2 ? (tn == kBN3 ? tern_smem_t<SCION_PTQ1_0, 2, kBN3>() : tern_smem_t<SCION_PTQ1_0, 2, kBN>())
                  : (tn == kBN2 ? tern_smem_t<SCION_PTQ1_0, 1, kBN2>() : tern_smem_t<SCION_PTQ1_0, 1, kBN>());
 }
+// Tile widths: gate/up takes 160-token tiles when the experts average at least kMid160 tokens
+// (fewer tiles of a few tokens past 128, each of which expands all of its expert's codes again),
+// down 256-token tiles from kBig256; 128 otherwise.
+int gateup_width(int64_t Tk, int E) { return Tk >= int64_t(kMid160) * E ? kBN3 : kBN; }
+int down_width(int64_t Tk, int E) { return Tk >= int64_t(kBig256) * E ? kBN2 : kBN; }
 constexpr size_t kDenseSmem = kDenseStages * kDenseStage + 1024;
 
 }  // namespace
@@ -934,6 +962,12 @@ cudaError_t configure_prefill_kernels() {
     return e;
   if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PTQ1_0, 1, kBN2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 int(tern_smem(1, SCION_PTQ1_0, kBN2)))))
+    return e;
+  if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PQ2_0, 2, kBN3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(tern_smem(2, SCION_PQ2_0, kBN3)))))
+    return e;
+  if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PTQ1_0, 2, kBN3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(tern_smem(2, SCION_PTQ1_0, kBN3)))))
     return e;
   return cudaSuccess;
 }
@@ -1059,7 +1093,9 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
       group_scan_kernel<<<1, kScanThreads, 0, s>>>(P.counts, L->E, P.offsets, P.cursor,
                                                   static_cast<TernTile*>(P.tiles), P.n_tiles,
-                                                  static_cast<TernTile*>(P.tiles2), P.n_tiles2);
+                                                  gateup_width(int64_t(T) * L->k, L->E),
+                                                  static_cast<TernTile*>(P.tiles2), P.n_tiles2,
+                                                  down_width(int64_t(T) * L->k, L->E));
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
       group_scatter_kernel<<<(n + 256 * ept - 1) / (256 * ept), 256, 2 * sizeof(int32_t) * L->E, s>>>(
           P.ids, n, L->E, ept, P.cursor, P.perm, P.inv);
@@ -1069,12 +1105,17 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       TernParams tp;
       tp.bank = L->gu_bank, tp.fmt = L->fmt, tp.na = 2, tp.G = L->Gd, tp.R = L->F;
       tp.bsrc = P.x16, tp.ldb = L->d;
+      const bool mid = gateup_width(int64_t(T) * L->k, L->E) == kBN3;
       tp.tiles = static_cast<const TernTile*>(P.tiles), tp.n_tiles = P.n_tiles;
       tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gates = P.gates, tp.k = L->k;
       tp.h = P.h, tp.F = L->F, tp.y = nullptr, tp.d = L->d, tp.err = L->err;
       const dim3 grid(num_sms());
-      if (L->fmt == SCION_PQ2_0)
+      if (L->fmt == SCION_PQ2_0 && mid)
+        tern_gemm_kernel<SCION_PQ2_0, 2, kBN3><<<grid, kTernThreads, tern_smem(2, L->fmt, kBN3), s>>>(tp);
+      else if (L->fmt == SCION_PQ2_0)
         tern_gemm_kernel<SCION_PQ2_0, 2><<<grid, kTernThreads, tern_smem(2, L->fmt), s>>>(tp);
+      else if (mid)
+        tern_gemm_kernel<SCION_PTQ1_0, 2, kBN3><<<grid, kTernThreads, tern_smem(2, L->fmt, kBN3), s>>>(tp);
       else
         tern_gemm_kernel<SCION_PTQ1_0, 2><<<grid, kTernThreads, tern_smem(2, L->fmt), s>>>(tp);
       return cudaGetLastError();
@@ -1102,8 +1143,8 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       tp.bsrc = P.h, tp.ldb = L->F;
       // experts averaging many tokens: 256-token tiles (each expanded code group serves twice the
       // tokens); otherwise 128-token tiles with a ping-pong accumulator that hides the epilogue
-      const bool big = int64_t(T) * L->k >= int64_t(kBig256) * L->E;
-      tp.tiles = static_cast<const TernTile*>(big ? P.tiles2 : P.tiles), tp.n_tiles = big ? P.n_tiles2 : P.n_tiles;
+      const bool big = down_width(int64_t(T) * L->k, L->E) == kBN2;
+      tp.tiles = static_cast<const TernTile*>(P.tiles2), tp.n_tiles = P.n_tiles2;
       tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gates = P.gates, tp.k = L->k;
       tp.h = nullptr, tp.F = L->F, tp.y = P.y, tp.d = L->d, tp.err = L->err;
       if (make_tmap_2d(&tp.bmap, P.h, 0, int64_t(T) * L->k, L->F) != SCION_OK) return cudaErrorInvalidValue;

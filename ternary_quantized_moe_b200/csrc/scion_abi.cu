@@ -85,7 +85,7 @@ int create_prefill(scion_layer* L, cudaStream_t s) {
   PTRY(dev_alloc(L, &P->y, sizeof(__half) * Tk * L->d));
   PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->tiles), scion::prefill_tile_bytes() * max_tiles));
   PTRY(dev_alloc(L, &P->n_tiles, sizeof(int32_t)));
-  PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->tiles2), scion::prefill_tile_bytes() * ((Tk + 255) / 256 + L->E)));
+  PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->tiles2), scion::prefill_tile_bytes() * ((Tk + 127) / 128 + L->E)));
   PTRY(dev_alloc(L, &P->n_tiles2, sizeof(int32_t)));
   PTRY(dev_alloc(L, &P->x16, sizeof(__half) * T * L->d));
   PTRY(dev_alloc(L, &P->h, sizeof(__half) * Tk * L->F));

@@ -415,13 +415,14 @@ def test_full_size_prefill_sampled(name, n_sample):
 # --------------------------------------------------------- tensor-core path
 @pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
 @pytest.mark.parametrize("router_f32", [False, True])
-def test_prefill_stagewise(fmt, router_f32):
+@pytest.mark.parametrize("T", [200, 500])
+def test_prefill_stagewise(fmt, router_f32, T):
     """Batches above 64 tokens run as tcgen05 GEMMs; routing bit-exact, hidden and output
-    within tolerance."""
+    within tolerance.  T = 200: 128-token gate/up tiles (50 tokens per expert on average);
+    T = 500: 160-token gate/up tiles (125 on average, some experts past 128 tokens)."""
     cfg = small("p", fmt, router_f32, E=16, k=4, d=256, F=256, Fs=128, r=32)
-    T = 200
     L, banks, ol, x = _case(cfg, T)
-    layer = device_layer(cfg, L, banks, 256)
+    layer = device_layer(cfg, L, banks, T)
     got, dbg = run_forward(layer, x, T, debug=True, E=cfg.n_experts, k=cfg.top_k, F=cfg.ffn,
                            Kdense=cfg.shared_ffn + cfg.rank)
     assert tq.scion_layer_check(layer) == 0
@@ -435,9 +436,10 @@ def test_prefill_stagewise(fmt, router_f32):
 
 
 @pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
-@pytest.mark.parametrize("T", [65, 129, 500])
+@pytest.mark.parametrize("T", [65, 129, 250, 300, 500])
 def test_prefill_multi_tile_experts(fmt, T):
-    """Few experts, many tokens each: experts span several 128-token tiles, ragged tails."""
+    """Few experts, many tokens each: experts span several tiles, ragged tails (T = 250, 300:
+    160-token gate/up tiles, experts on both sides of 160 tokens; T = 500: 256-token down tiles)."""
     cfg = small("m", fmt, False, E=4, k=2, d=384, F=128, Fs=0, r=16)
     L, banks, ol, x = _case(cfg, T)
     layer = device_layer(cfg, L, banks, T)
