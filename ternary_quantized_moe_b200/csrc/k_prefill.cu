@@ -474,7 +474,7 @@ struct TernRing {
   static constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
   // shared memory: B groups (two 64-column K blocks of TN swizzled 128-byte rows) and packed
   // code groups
-  static_assert(TN == kBN || (TN == kBN2 && NA == 1) || (TN == kBN3 && NA == 2), "tile width");
+  static_assert(TN == kBN || TN == kBN3 || (TN == kBN2 && NA == 1), "tile width");
   static constexpr int kB = TN == kBN2 ? 2 : 4;
   static constexpr int kC = 4;
   static constexpr uint32_t b_kblock = uint32_t(TN) * 128;  // bytes of one 64-column K block of B
@@ -483,9 +483,9 @@ struct TernRing {
   static constexpr uint32_t b_off = 0, c_off = kB * b_bytes;
   static constexpr uint32_t bytes = c_off + kC * c_bytes;
   // tensor memory: accumulators, then the ring of expanded A groups
-  // gate/up: one NA x 128 accumulator; down: two 128-column accumulators (ping-pong), or one of
+  // gate/up: one NA x TN accumulator; down: two TN-column accumulators (ping-pong), or one of
   // 256 columns for 256-token tiles
-  static constexpr int n_acc = NA == 1 && TN == kBN ? 2 : 1;
+  static constexpr int n_acc = NA == 1 && TN != kBN2 ? 2 : 1;
   static constexpr uint32_t acc_cols = NA * TN;
   // ring entries of expanded A: one group of all NA matrices, or (160-token gate/up tiles,
   // whose accumulators leave 192 columns) one matrix of a group, EPG entries per group
@@ -573,6 +573,7 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
           mbar_arrive_expect_tx(&b_full[s], R::b_bytes);
 #pragma unroll
           for (int kb = 0; kb < 2; ++kb) {  // 64-column K blocks of the group, TN token rows each
+            // the map's box is 128 rows (TN = 128, 256: one or two boxes) or 160 (TN = 160)
             tma_load_2d(dst + kb * R::b_kblock, &p.bmap, g * 128 + 64 * kb, row0, &b_full[s]);
             if (TN == kBN2) tma_load_2d(dst + kb * R::b_kblock + kAtom, &p.bmap, g * 128 + 64 * kb, row0 + 128, &b_full[s]);
           }
@@ -910,30 +911,33 @@ template <int FMT, int NA, int TN>
 size_t tern_smem_t() {
   return TernRing<FMT, NA, TN>::bytes + 1024;
 }
-size_t tern_smem(int na, int fmt, int tn = kBN) {
-  if (fmt == SCION_PQ2_0)
-    return na == 2 ? (tn == kBN3 ? tern_smem_t<SCION_PQ2_0, 2, kBN3>() : tern_smem_t<SCION_PQ2_0, 2, kBN>())
-                   : (tn == kBN2 ? tern_smem_t<SCION_PQ2_0, 1, kBN2>() : tern_smem_t<SCION_PQ2_0, 1, kBN>());
-  return na == 2 ? (tn == kBN3 ? tern_smem_t<SCION_PTQ1_0, 2, kBN3>() : tern_smem_t<SCION_PTQ1_0, 2, kBN>())
-                 : (tn == kBN2 ? tern_smem_t<SCION_PTQ1_0, 1, kBN2>() : tern_smem_t<SCION_PTQ1_0, 1, kBN>());
+template <int FMT>
+size_t tern_smem_f(int na, int tn) {
+  if (na == 2) return tn == kBN3 ? tern_smem_t<FMT, 2, kBN3>() : tern_smem_t<FMT, 2, kBN>();
+  return tn == kBN2 ? tern_smem_t<FMT, 1, kBN2>() : tn == kBN3 ? tern_smem_t<FMT, 1, kBN3>() : tern_smem_t<FMT, 1, kBN>();
 }
-// Tile widths: gate/up takes 160-token tiles when the experts average at least kMid160 tokens
-// (fewer tiles of a few tokens past 128, each of which expands all of its expert's codes again),
-// down 256-token tiles from kBig256; 128 otherwise.
+size_t tern_smem(int na, int fmt, int tn = kBN) {
+  return fmt == SCION_PQ2_0 ? tern_smem_f<SCION_PQ2_0>(na, tn) : tern_smem_f<SCION_PTQ1_0>(na, tn);
+}
+// Tile widths: 160-token tiles when the experts average at least kMid160 tokens (fewer tiles of
+// a few tokens past 128, each of which expands all of its expert's codes again), for the down
+// projection 256-token tiles from kBig256; 128 otherwise.
 int gateup_width(int64_t Tk, int E) { return Tk >= int64_t(kMid160) * E ? kBN3 : kBN; }
-int down_width(int64_t Tk, int E) { return Tk >= int64_t(kBig256) * E ? kBN2 : kBN; }
+int down_width(int64_t Tk, int E) {
+  return Tk >= int64_t(kBig256) * E ? kBN2 : (Tk >= int64_t(kMid160) * E ? kBN3 : kBN);
+}
 constexpr size_t kDenseSmem = kDenseStages * kDenseStage + 1024;
 
 }  // namespace
 
-// K-major [rows][K] 2-byte matrix, box {64 columns, 128 rows}, 128-byte swizzle.
-int make_tmap_2d(CUtensorMap* map, const void* ptr, int bf16, int64_t rows, int64_t K) {
+// K-major [rows][K] 2-byte matrix, box {64 columns, box_rows rows}, 128-byte swizzle.
+int make_tmap_2d(CUtensorMap* map, const void* ptr, int bf16, int64_t rows, int64_t K, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return SCION_ECUDA;
   if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (K * 2) % 16) return SCION_EINVAL;
   cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
   cuuint64_t strides[1] = {cuuint64_t(K * 2)};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, cuuint32_t(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
                   const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -965,6 +969,12 @@ cudaError_t configure_prefill_kernels() {
     return e;
   if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PQ2_0, 2, kBN3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 int(tern_smem(2, SCION_PQ2_0, kBN3)))))
+    return e;
+  if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PQ2_0, 1, kBN3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(tern_smem(1, SCION_PQ2_0, kBN3)))))
+    return e;
+  if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PTQ1_0, 1, kBN3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(tern_smem(1, SCION_PTQ1_0, kBN3)))))
     return e;
   if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PTQ1_0, 2, kBN3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 int(tern_smem(2, SCION_PTQ1_0, kBN3)))))
@@ -1143,20 +1153,19 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       tp.bsrc = P.h, tp.ldb = L->F;
       // experts averaging many tokens: 256-token tiles (each expanded code group serves twice the
       // tokens); otherwise 128-token tiles with a ping-pong accumulator that hides the epilogue
-      const bool big = down_width(int64_t(T) * L->k, L->E) == kBN2;
+      const int wd = down_width(int64_t(T) * L->k, L->E);
       tp.tiles = static_cast<const TernTile*>(P.tiles2), tp.n_tiles = P.n_tiles2;
       tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gates = P.gates, tp.k = L->k;
       tp.h = nullptr, tp.F = L->F, tp.y = P.y, tp.d = L->d, tp.err = L->err;
-      if (make_tmap_2d(&tp.bmap, P.h, 0, int64_t(T) * L->k, L->F) != SCION_OK) return cudaErrorInvalidValue;
+      if (make_tmap_2d(&tp.bmap, P.h, 0, int64_t(T) * L->k, L->F, wd == kBN3 ? kBN3 : 128) != SCION_OK)
+        return cudaErrorInvalidValue;
       const dim3 grid(num_sms());
-      if (L->fmt == SCION_PQ2_0 && big)
-        tern_gemm_kernel<SCION_PQ2_0, 1, kBN2><<<grid, kTernThreads, tern_smem(1, L->fmt, kBN2), s>>>(tp);
-      else if (L->fmt == SCION_PQ2_0)
-        tern_gemm_kernel<SCION_PQ2_0, 1><<<grid, kTernThreads, tern_smem(1, L->fmt), s>>>(tp);
-      else if (big)
-        tern_gemm_kernel<SCION_PTQ1_0, 1, kBN2><<<grid, kTernThreads, tern_smem(1, L->fmt, kBN2), s>>>(tp);
+#define SCION_DOWN(F, W) tern_gemm_kernel<F, 1, W><<<grid, kTernThreads, tern_smem(1, F, W), s>>>(tp)
+      if (L->fmt == SCION_PQ2_0)
+        wd == kBN2 ? SCION_DOWN(SCION_PQ2_0, kBN2) : wd == kBN3 ? SCION_DOWN(SCION_PQ2_0, kBN3) : SCION_DOWN(SCION_PQ2_0, kBN);
       else
-        tern_gemm_kernel<SCION_PTQ1_0, 1><<<grid, kTernThreads, tern_smem(1, L->fmt), s>>>(tp);
+        wd == kBN2 ? SCION_DOWN(SCION_PTQ1_0, kBN2) : wd == kBN3 ? SCION_DOWN(SCION_PTQ1_0, kBN3) : SCION_DOWN(SCION_PTQ1_0, kBN);
+#undef SCION_DOWN
       return cudaGetLastError();
     }
     default:

@@ -171,7 +171,7 @@ cudaError_t launch_stream_gateup(const scion_layer* L, int T, cudaStream_t s);
 cudaError_t launch_stream_down(const scion_layer* L, int T, float* out, cudaStream_t s);
 
 // k_prefill.cu
-int make_tmap_2d(CUtensorMap* map, const void* ptr, int bf16, int64_t rows, int64_t K);
+int make_tmap_2d(CUtensorMap* map, const void* ptr, int bf16, int64_t rows, int64_t K, int box_rows = 128);
 cudaError_t configure_prefill_kernels();
 size_t prefill_unit_bytes();
 size_t prefill_tile_bytes();
