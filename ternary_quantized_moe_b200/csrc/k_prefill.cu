@@ -379,10 +379,8 @@ struct TernParams {
 };
 
 constexpr uint32_t kAtom = 128 * 128;  // bytes of one 128-row x 64-column swizzled atom
-constexpr int kBN2 = 256;      // tokens per down-projection tile of long batches
-constexpr int kBig256 = 192;   // mean tokens per expert from which the down projection takes kBN2 tiles
-constexpr int kBN3 = 160;      // tokens per gate/up tile of batches whose experts average near 128
-constexpr int kMid160 = 112;   // mean tokens per expert from which (below kBig256) gate/up takes kBN3 tiles
+constexpr int kBN3 = 160;      // tokens per tile of batches whose experts average kMid160 or more
+constexpr int kMid160 = 112;   // mean tokens per expert from which both ternary GEMMs take kBN3 tiles
 
 // Expand half h (64 columns) of row t (0..127) of one 128-row group from its sub-tile block
 // into 32 registers of fp16 pairs, in position order (v[i] = positions 2i, 2i+1 of the half).
@@ -465,17 +463,16 @@ __device__ __forceinline__ void expand_ptq1_half(uint32_t codes, int t, int h, u
 }
 
 // Pipeline granularity: one 128-column code group along K ("group" = two 64-column halves).
-// TN = tokens per tile: 128 (both GEMMs), 256 (down projection of batches whose experts
-// average at least kBig256 tokens) or 160 (gate/up of batches whose experts average between
-// kMid160 and kBig256 tokens: one tile holds nearly every expert's tokens, so each expert's
-// codes are expanded once).
+// TN = tokens per tile: 128, or 160 when the experts average at least kMid160 tokens (a tile then
+// holds nearly all of an expert's tokens, so its codes are seldom expanded a second time for a
+// tile of a few tokens).
 template <int FMT, int NA, int TN = kBN>
 struct TernRing {
   static constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
   // shared memory: B groups (two 64-column K blocks of TN swizzled 128-byte rows) and packed
   // code groups
-  static_assert(TN == kBN || TN == kBN3 || (TN == kBN2 && NA == 1), "tile width");
-  static constexpr int kB = TN == kBN2 ? 2 : 4;
+  static_assert(TN == kBN || TN == kBN3, "tile width");
+  static constexpr int kB = 4;
   static constexpr int kC = 4;
   static constexpr uint32_t b_kblock = uint32_t(TN) * 128;  // bytes of one 64-column K block of B
   static constexpr uint32_t b_bytes = 2 * b_kblock;
@@ -483,9 +480,8 @@ struct TernRing {
   static constexpr uint32_t b_off = 0, c_off = kB * b_bytes;
   static constexpr uint32_t bytes = c_off + kC * c_bytes;
   // tensor memory: accumulators, then the ring of expanded A groups
-  // gate/up: one NA x TN accumulator; down: two TN-column accumulators (ping-pong), or one of
-  // 256 columns for 256-token tiles
-  static constexpr int n_acc = NA == 1 && TN != kBN2 ? 2 : 1;
+  // gate/up: one NA x TN accumulator; down: two TN-column accumulators (ping-pong)
+  static constexpr int n_acc = NA == 1 ? 2 : 1;
   static constexpr uint32_t acc_cols = NA * TN;
   // ring entries of expanded A: one group of all NA matrices, or (160-token gate/up tiles,
   // whose accumulators leave 192 columns) one matrix of a group, EPG entries per group
@@ -573,9 +569,8 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
           mbar_arrive_expect_tx(&b_full[s], R::b_bytes);
 #pragma unroll
           for (int kb = 0; kb < 2; ++kb) {  // 64-column K blocks of the group, TN token rows each
-            // the map's box is 128 rows (TN = 128, 256: one or two boxes) or 160 (TN = 160)
+            // the map's box is TN rows
             tma_load_2d(dst + kb * R::b_kblock, &p.bmap, g * 128 + 64 * kb, row0, &b_full[s]);
-            if (TN == kBN2) tma_load_2d(dst + kb * R::b_kblock + kAtom, &p.bmap, g * 128 + 64 * kb, row0 + 128, &b_full[s]);
           }
         }
       }
@@ -787,55 +782,49 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 // in slot order), so the scatter takes positions with one atomic per entry.
 //
 // One CTA: exclusive scan of the histogram, the per-expert cursors, and the token tiles of the
-// two ternary GEMMs: w1 tokens for gate/up (128 or 160), w2 for down (128 or 256).
+// two ternary GEMMs (w tokens: 128 or 160).
 constexpr int kScanThreads = 1024;
 __global__ void __launch_bounds__(kScanThreads) group_scan_kernel(const int32_t* __restrict__ counts, int E,
                                                                   int32_t* __restrict__ offsets,
                                                                   int32_t* __restrict__ cursor,
                                                                   TernTile* __restrict__ tiles,
-                                                                  int32_t* __restrict__ n_tiles, int w1,
-                                                                  TernTile* __restrict__ tiles2,
-                                                                  int32_t* __restrict__ n_tiles2, int w2) {
-  __shared__ int32_t wsum[kScanThreads / 32], wtile[kScanThreads / 32], wtile2[kScanThreads / 32];
+                                                                  int32_t* __restrict__ n_tiles, int w) {
+  __shared__ int32_t wsum[kScanThreads / 32], wtile[kScanThreads / 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int per = (E + kScanThreads - 1) / kScanThreads;  // experts per thread, contiguous
   const int e0 = min(E, threadIdx.x * per), e1 = min(E, e0 + per);
-  int cs = 0, ts = 0, ts2 = 0;
+  int cs = 0, ts = 0;
   for (int e = e0; e < e1; ++e) {
     const int c = counts[e];
-    cs += c, ts += (c + w1 - 1) / w1, ts2 += (c + w2 - 1) / w2;
+    cs += c, ts += (c + w - 1) / w;
   }
-  // block-wide exclusive scan of (cs, ts, ts2)
-  int ic = cs, it = ts, it2 = ts2;
+  // block-wide exclusive scan of (cs, ts)
+  int ic = cs, it = ts;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const int c2 = __shfl_up_sync(0xffffffffu, ic, o), t2 = __shfl_up_sync(0xffffffffu, it, o);
-    const int u2 = __shfl_up_sync(0xffffffffu, it2, o);
-    if (lane >= o) ic += c2, it += t2, it2 += u2;
+    if (lane >= o) ic += c2, it += t2;
   }
-  if (lane == 31) wsum[warp] = ic, wtile[warp] = it, wtile2[warp] = it2;
+  if (lane == 31) wsum[warp] = ic, wtile[warp] = it;
   __syncthreads();
   if (warp == 0) {
-    int a = wsum[lane], b = wtile[lane], b2 = wtile2[lane];
+    int a = wsum[lane], b = wtile[lane];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int a2 = __shfl_up_sync(0xffffffffu, a, o), x2 = __shfl_up_sync(0xffffffffu, b, o);
-      const int y2 = __shfl_up_sync(0xffffffffu, b2, o);
-      if (lane >= o) a += a2, b += x2, b2 += y2;
+      if (lane >= o) a += a2, b += x2;
     }
-    wsum[lane] = a, wtile[lane] = b, wtile2[lane] = b2;
-    if (lane == 31) offsets[E] = a, *n_tiles = b, *n_tiles2 = b2;
+    wsum[lane] = a, wtile[lane] = b;
+    if (lane == 31) offsets[E] = a, *n_tiles = b;
   }
   __syncthreads();
   int run = (warp ? wsum[warp - 1] : 0) + ic - cs;
   int trun = (warp ? wtile[warp - 1] : 0) + it - ts;
-  int trun2 = (warp ? wtile2[warp - 1] : 0) + it2 - ts2;
   for (int e = e0; e < e1; ++e) {
     const int c = counts[e];
     offsets[e] = run;
     cursor[e] = run;
-    for (int c0 = 0; c0 < c; c0 += w1) tiles[trun++] = TernTile{e, c0, min(w1, c - c0), run + c0};
-    for (int c0 = 0; c0 < c; c0 += w2) tiles2[trun2++] = TernTile{e, c0, min(w2, c - c0), run + c0};
+    for (int c0 = 0; c0 < c; c0 += w) tiles[trun++] = TernTile{e, c0, min(w, c - c0), run + c0};
     run += c;
   }
 }
@@ -914,18 +903,15 @@ size_t tern_smem_t() {
 template <int FMT>
 size_t tern_smem_f(int na, int tn) {
   if (na == 2) return tn == kBN3 ? tern_smem_t<FMT, 2, kBN3>() : tern_smem_t<FMT, 2, kBN>();
-  return tn == kBN2 ? tern_smem_t<FMT, 1, kBN2>() : tn == kBN3 ? tern_smem_t<FMT, 1, kBN3>() : tern_smem_t<FMT, 1, kBN>();
+  return tn == kBN3 ? tern_smem_t<FMT, 1, kBN3>() : tern_smem_t<FMT, 1, kBN>();
 }
 size_t tern_smem(int na, int fmt, int tn = kBN) {
   return fmt == SCION_PQ2_0 ? tern_smem_f<SCION_PQ2_0>(na, tn) : tern_smem_f<SCION_PTQ1_0>(na, tn);
 }
-// Tile widths: 160-token tiles when the experts average at least kMid160 tokens (fewer tiles of
-// a few tokens past 128, each of which expands all of its expert's codes again), for the down
-// projection 256-token tiles from kBig256; 128 otherwise.
-int gateup_width(int64_t Tk, int E) { return Tk >= int64_t(kMid160) * E ? kBN3 : kBN; }
-int down_width(int64_t Tk, int E) {
-  return Tk >= int64_t(kBig256) * E ? kBN2 : (Tk >= int64_t(kMid160) * E ? kBN3 : kBN);
-}
+// Tile width of both ternary GEMMs: 160 tokens when the experts average at least kMid160 tokens
+// (fewer tiles of a few tokens past 128, each of which expands all of its expert's codes again),
+// 128 otherwise.
+int tile_width(int64_t Tk, int E) { return Tk >= int64_t(kMid160) * E ? kBN3 : kBN; }
 constexpr size_t kDenseSmem = kDenseStages * kDenseStage + 1024;
 
 }  // namespace
@@ -960,12 +946,6 @@ cudaError_t configure_prefill_kernels() {
     return e;
   if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PTQ1_0, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 int(tern_smem(1, SCION_PTQ1_0)))))
-    return e;
-  if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PQ2_0, 1, kBN2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                int(tern_smem(1, SCION_PQ2_0, kBN2)))))
-    return e;
-  if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PTQ1_0, 1, kBN2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                int(tern_smem(1, SCION_PTQ1_0, kBN2)))))
     return e;
   if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PQ2_0, 2, kBN3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 int(tern_smem(2, SCION_PQ2_0, kBN3)))))
@@ -1103,9 +1083,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
       group_scan_kernel<<<1, kScanThreads, 0, s>>>(P.counts, L->E, P.offsets, P.cursor,
                                                   static_cast<TernTile*>(P.tiles), P.n_tiles,
-                                                  gateup_width(int64_t(T) * L->k, L->E),
-                                                  static_cast<TernTile*>(P.tiles2), P.n_tiles2,
-                                                  down_width(int64_t(T) * L->k, L->E));
+                                                  tile_width(int64_t(T) * L->k, L->E));
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
       group_scatter_kernel<<<(n + 256 * ept - 1) / (256 * ept), 256, 2 * sizeof(int32_t) * L->E, s>>>(
           P.ids, n, L->E, ept, P.cursor, P.perm, P.inv);
@@ -1115,7 +1093,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       TernParams tp;
       tp.bank = L->gu_bank, tp.fmt = L->fmt, tp.na = 2, tp.G = L->Gd, tp.R = L->F;
       tp.bsrc = P.x16, tp.ldb = L->d;
-      const bool mid = gateup_width(int64_t(T) * L->k, L->E) == kBN3;
+      const bool mid = tile_width(int64_t(T) * L->k, L->E) == kBN3;
       tp.tiles = static_cast<const TernTile*>(P.tiles), tp.n_tiles = P.n_tiles;
       tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gates = P.gates, tp.k = L->k;
       tp.h = P.h, tp.F = L->F, tp.y = nullptr, tp.d = L->d, tp.err = L->err;
@@ -1151,20 +1129,18 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       TernParams tp;
       tp.bank = L->dn_bank, tp.fmt = L->fmt, tp.na = 1, tp.G = L->GF, tp.R = L->d;
       tp.bsrc = P.h, tp.ldb = L->F;
-      // experts averaging many tokens: 256-token tiles (each expanded code group serves twice the
-      // tokens); otherwise 128-token tiles with a ping-pong accumulator that hides the epilogue
-      const int wd = down_width(int64_t(T) * L->k, L->E);
-      tp.tiles = static_cast<const TernTile*>(P.tiles2), tp.n_tiles = P.n_tiles2;
+      const int wd = tile_width(int64_t(T) * L->k, L->E);
+      tp.tiles = static_cast<const TernTile*>(P.tiles), tp.n_tiles = P.n_tiles;
       tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gates = P.gates, tp.k = L->k;
       tp.h = nullptr, tp.F = L->F, tp.y = P.y, tp.d = L->d, tp.err = L->err;
-      if (make_tmap_2d(&tp.bmap, P.h, 0, int64_t(T) * L->k, L->F, wd == kBN3 ? kBN3 : 128) != SCION_OK)
+      if (make_tmap_2d(&tp.bmap, P.h, 0, int64_t(T) * L->k, L->F, wd) != SCION_OK)
         return cudaErrorInvalidValue;
       const dim3 grid(num_sms());
 #define SCION_DOWN(F, W) tern_gemm_kernel<F, 1, W><<<grid, kTernThreads, tern_smem(1, F, W), s>>>(tp)
       if (L->fmt == SCION_PQ2_0)
-        wd == kBN2 ? SCION_DOWN(SCION_PQ2_0, kBN2) : wd == kBN3 ? SCION_DOWN(SCION_PQ2_0, kBN3) : SCION_DOWN(SCION_PQ2_0, kBN);
+        wd == kBN3 ? SCION_DOWN(SCION_PQ2_0, kBN3) : SCION_DOWN(SCION_PQ2_0, kBN);
       else
-        wd == kBN2 ? SCION_DOWN(SCION_PTQ1_0, kBN2) : wd == kBN3 ? SCION_DOWN(SCION_PTQ1_0, kBN3) : SCION_DOWN(SCION_PTQ1_0, kBN);
+        wd == kBN3 ? SCION_DOWN(SCION_PTQ1_0, kBN3) : SCION_DOWN(SCION_PTQ1_0, kBN);
 #undef SCION_DOWN
       return cudaGetLastError();
     }

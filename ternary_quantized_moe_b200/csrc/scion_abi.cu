@@ -54,7 +54,7 @@ void free_layer(scion_layer* L) {
   if (L->pre) {
     scion::PrefillState* P = L->pre;
     void* pp[] = {P->xunits, P->dunits, P->logits, P->ids, P->gates, P->counts, P->offsets, P->perm, P->inv,
-                  P->y, P->tiles, P->n_tiles, P->x16, P->h, P->hz, P->cursor, P->corr_a16, P->tiles2, P->n_tiles2};
+                  P->y, P->tiles, P->n_tiles, P->x16, P->h, P->hz, P->cursor, P->corr_a16};
     for (void* p : pp)
       if (p) cudaFree(p);
     delete P;
@@ -85,8 +85,6 @@ int create_prefill(scion_layer* L, cudaStream_t s) {
   PTRY(dev_alloc(L, &P->y, sizeof(__half) * Tk * L->d));
   PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->tiles), scion::prefill_tile_bytes() * max_tiles));
   PTRY(dev_alloc(L, &P->n_tiles, sizeof(int32_t)));
-  PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->tiles2), scion::prefill_tile_bytes() * ((Tk + 127) / 128 + L->E)));
-  PTRY(dev_alloc(L, &P->n_tiles2, sizeof(int32_t)));
   PTRY(dev_alloc(L, &P->x16, sizeof(__half) * T * L->d));
   PTRY(dev_alloc(L, &P->h, sizeof(__half) * Tk * L->F));
   PTRY(dev_alloc(L, &P->hz, sizeof(__half) * T * (L->Kd ? L->Kd : 64)));

@@ -78,10 +78,8 @@ struct PrefillState {
   int32_t* inv;         // [maxT*k] position of entry t*k+j in perm
   int32_t* cursor;      // [E] next free position of each expert's segment (grouping scratch)
   __half* y;            // [maxT*k][d] expert down outputs in fp16 (gate not yet applied), one row per routed entry
-  void* tiles;          // gate/up token tiles (128 or 160 tokens), [maxT*k/128 + E]
+  void* tiles;          // token tiles of the ternary GEMMs (128 or 160 tokens), [maxT*k/128 + E]
   int32_t* n_tiles;
-  void* tiles2;         // down token tiles (128 or 256 tokens), [maxT*k/128 + E]
-  int32_t* n_tiles2;
   __half* x16;          // [maxT][d]   x in the container column order (fp16)
   __half* h;            // [maxT*k][F] expert SwiGLU hidden, container column order
   __half* hz;           // [maxT][Kd]

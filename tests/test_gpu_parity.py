@@ -438,8 +438,9 @@ def test_prefill_stagewise(fmt, router_f32, T):
 @pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
 @pytest.mark.parametrize("T", [65, 129, 250, 300, 500])
 def test_prefill_multi_tile_experts(fmt, T):
-    """Few experts, many tokens each: experts span several tiles, ragged tails (T = 250, 300:
-    160-token gate/up tiles, experts on both sides of 160 tokens; T = 500: 256-token down tiles)."""
+    """Few experts, many tokens each: experts span several tiles, ragged tails (T = 65, 129:
+    128-token tiles; T = 250, 300, 500: 160-token tiles, experts on both sides of 160 tokens and,
+    at T = 500, across two tiles)."""
     cfg = small("m", fmt, False, E=4, k=2, d=384, F=128, Fs=0, r=16)
     L, banks, ol, x = _case(cfg, T)
     layer = device_layer(cfg, L, banks, T)
