@@ -445,7 +445,12 @@ def run_gpu(args, rank, world, local_rank):
                           "expert_stage_hbm_frac": (expert_bytes / ((stages.get("gateup", (0, 0))[0] +
                                                                      stages.get("down_routed", (0, 0))[0]) / 1000.0)
                                                     / (peaks["hbm_gbs"] * 1e9))
-                          if stages.get("gateup", (0, 0))[0] > 0 else None},
+                          if stages.get("gateup", (0, 0))[0] > 0 else None,
+                          # the same step against nominal figures: HBM3e at 8 TB/s, and the bf16
+                          # throughput a seconds-long GEMM sustains under the power cap
+                          "hbm_frac_vs_nominal_8tbs": (bytes_total / (ms / 1000.0)) / 8e12,
+                          "tflops_frac_vs_sustained": flops_total / (ms / 1000.0) / 1e12 /
+                          peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])},
         "per_batch": per_batch,
         "stages_us_per_launch": {k_: 1000.0 * v[0] / v[1] for k_, v in stages.items() if v[1]},
         "stages_rate": {k_: (sbytes[k_] / (v[0] / 1000.0) / 1e9 if decode else
