@@ -971,17 +971,46 @@ __global__ void __launch_bounds__(256) combine_kernel(const __half* __restrict__
   const int t = blockIdx.x;
   const int32_t* iv = inv + int64_t(t) * k;
   const float* gt = gates + int64_t(t) * k;
-  float4* o = reinterpret_cast<float4*>(out + int64_t(t) * d);
-  for (int c4 = threadIdx.x; c4 < d / 4; c4 += blockDim.x) {
-    float4 acc = base ? reinterpret_cast<const float4*>(base + int64_t(t) * d)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j = 0; j < k; ++j) {
-      const uint2 raw = reinterpret_cast<const uint2*>(y + int64_t(iv[j]) * d)[c4];
-      const float2 lo = __half22float2(u32_as_h2(raw.x)), hi = __half22float2(u32_as_h2(raw.y));
-      const float4 v = make_float4(lo.x, lo.y, hi.x, hi.y);
-      const float g = gt[j];
-      acc.x += g * v.x, acc.y += g * v.y, acc.z += g * v.z, acc.w += g * v.w;
+  // each thread: 8 columns (one 16-byte load per routed row); the k rows' loads are issued in
+  // batches of 8 before any of them is used, so each thread keeps 8 loads in flight
+  for (int c8 = threadIdx.x; c8 < d / 8; c8 += blockDim.x) {
+    float acc[8];
+    if (base) {
+      const float4 b0 = reinterpret_cast<const float4*>(base + int64_t(t) * d)[2 * c8];
+      const float4 b1 = reinterpret_cast<const float4*>(base + int64_t(t) * d)[2 * c8 + 1];
+      acc[0] = b0.x, acc[1] = b0.y, acc[2] = b0.z, acc[3] = b0.w;
+      acc[4] = b1.x, acc[5] = b1.y, acc[6] = b1.z, acc[7] = b1.w;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     }
-    o[c4] = acc;
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      uint4 raw[8];
+      float g[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j0 + j < k) {
+          raw[j] = reinterpret_cast<const uint4*>(y + int64_t(iv[j0 + j]) * d)[c8];
+          g[j] = gt[j0 + j];
+        } else {
+          raw[j] = make_uint4(0u, 0u, 0u, 0u);
+          g[j] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t w[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 v = __half22float2(u32_as_h2(w[q]));
+          acc[2 * q] = fmaf(g[j], v.x, acc[2 * q]);
+          acc[2 * q + 1] = fmaf(g[j], v.y, acc[2 * q + 1]);
+        }
+      }
+    }
+    float4* o = reinterpret_cast<float4*>(out + int64_t(t) * d);
+    o[2 * c8] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    o[2 * c8 + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
 }
 
