@@ -76,27 +76,41 @@ __device__ __forceinline__ int pos_col(int fmt, int p) {
 }
 
 // x (bf16) -> fp16 in the container's column order (PQ2_0: times the factor of its position).
-// A warp takes two 128-column groups per step: coalesced 16-byte loads into shared memory,
-// then each lane gathers the columns of its 8 output positions and stores 16 bytes.
+// A warp takes kXU pairs of 128-column groups per step: their coalesced 16-byte loads are all
+// issued first, then each pair goes through shared memory, where each lane gathers the columns
+// of its 8 output positions and stores 16 bytes.
+constexpr int kXU = 4;
 template <int FMT>
 __global__ void __launch_bounds__(256) x16_kernel(const __nv_bfloat16* __restrict__ x, int64_t n_groups,
                                                   __half* __restrict__ xp) {
-  __shared__ __align__(16) __nv_bfloat16 buf[8][256];
+  __shared__ __align__(16) __nv_bfloat16 buf[8][kXU][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gl = lane >> 4, p0 = 8 * (lane & 15);  // group of the pair, first output position
   const int64_t n_pairs = (n_groups + 1) / 2;
-  for (int64_t i = int64_t(blockIdx.x) * 8 + warp; i < n_pairs; i += int64_t(gridDim.x) * 8) {
-    const bool ok = 2 * i + gl < n_groups;  // an odd group count leaves the last pair half empty
-    if (ok) *reinterpret_cast<uint4*>(&buf[warp][8 * lane]) = __ldg(reinterpret_cast<const uint4*>(x + i * 256) + lane);
-    __syncwarp();
-    __align__(16) __half o[8];
+  for (int64_t i0 = (int64_t(blockIdx.x) * 8 + warp) * kXU; i0 < n_pairs; i0 += int64_t(gridDim.x) * 8 * kXU) {
+    uint4 v[kXU];
+    bool ok[kXU];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int p = p0 + e;
-      const float v = __bfloat162float(buf[warp][128 * gl + pos_col(FMT, p)]);
-      o[e] = __float2half_rn(FMT == SCION_PQ2_0 ? v * pq2_pos_scale(p) : v);
+    for (int u = 0; u < kXU; ++u) {
+      // past the last group (an odd group count leaves the last pair half empty) nothing moves
+      ok[u] = 2 * (i0 + u) + gl < n_groups;
+      if (ok[u]) v[u] = __ldg(reinterpret_cast<const uint4*>(x + (i0 + u) * 256) + lane);
     }
-    if (ok) reinterpret_cast<uint4*>(xp + i * 256)[lane] = *reinterpret_cast<const uint4*>(o);
+#pragma unroll
+    for (int u = 0; u < kXU; ++u)
+      if (ok[u]) *reinterpret_cast<uint4*>(&buf[warp][u][8 * lane]) = v[u];
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < kXU; ++u) {
+      __align__(16) __half o[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int p = p0 + e;
+        const float f = __bfloat162float(buf[warp][u][128 * gl + pos_col(FMT, p)]);
+        o[e] = __float2half_rn(FMT == SCION_PQ2_0 ? f * pq2_pos_scale(p) : f);
+      }
+      if (ok[u]) reinterpret_cast<uint4*>(xp + (i0 + u) * 256)[lane] = *reinterpret_cast<const uint4*>(o);
+    }
     __syncwarp();
   }
 }
@@ -1069,7 +1083,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
     case SCION_STAGE_X16: {
       const int64_t n = int64_t(T) * L->d;
       const int64_t groups = n / 128, pairs = (groups + 1) / 2;
-      const unsigned grid = unsigned(std::min((pairs + 7) / 8, int64_t(num_sms()) * 8));
+      const unsigned grid = unsigned(std::min((pairs + 8 * kXU - 1) / (8 * kXU), int64_t(num_sms()) * 8));
       if (L->fmt == SCION_PQ2_0)
         x16_kernel<SCION_PQ2_0><<<grid, 256, 0, s>>>(x, groups, P.x16);
       else
