@@ -11,12 +11,15 @@
 //               x-projection  router + delta -> logits; shared gate/up -> SwiGLU; corr A -> z
 //               dense down    [shared down | correction B] x [h_s | z] -> out (store)
 //   route     top-k per token (warp per token) with a histogram of the selections, one CTA
-//             scans it and lists the 128-token tiles, one thread per entry takes its position
+//             scans it and lists the token tiles (128 or 160 tokens), and each entry takes
+//             its position inside its expert's segment
 //   ternary   tcgen05 grouped GEMM over the routed tiles: packed code blocks arrive by
-//             bulk copy, four warps expand them to fp16 (code * scale, exact) in the
-//             swizzled layout, gathered token rows arrive by cp.async:
+//             bulk copy, eight warps expand them to fp16 (code * scale, exact) straight into
+//             tensor memory (the A operand), token rows arrive by cp.async (gathered x16 rows)
+//             or TMA (h, already in routed order):
 //               gate/up  -> SwiGLU -> h (fp16)
-//               down     -> out += gate * y   (fp32 red.add)
+//               down     -> y (fp16, one row per routed entry)
+//   combine   out = base + the gate-weighted sum of each token's k rows of y
 //
 // Column orders (the A expansion and the B rows must agree):
 //   PQ2_0 : inside every 16 columns, position 2s+h holds column s + 8h (s < 8, h < 2)
@@ -366,8 +369,8 @@ namespace {
 // -------------------------------------------------------------- ternary GEMM
 struct __align__(16) TernTile {
   int e;     // expert
-  int c0;    // first token (within the expert's group) of this 128-token tile
-  int n;     // tokens in the tile (1..128)
+  int c0;    // first token (within the expert's group) of this tile
+  int n;     // tokens in the tile (1..TN, TN = 128 or 160)
   int pos0;  // routed-order position of its first token (offsets[e] + c0)
 };
 
@@ -512,7 +515,7 @@ constexpr int kTernThreads = 640;  // 20 warps: codes, MMA, 2 x B rows, 8 expans
 constexpr int kEpiThreads = 256;
 
 // Persistent grouped GEMM: CTA b walks the work items b, b + gridDim.x, ... where item =
-// (128-token tile, 128-row weight tile).  The expansion warps decode the packed codes of each
+// (token tile of up to TN tokens, 128-row weight tile).  The expansion warps decode the packed codes of each
 // 128-column group straight into tensor memory (one weight row per TMEM lane), and the MMA
 // reads A from there and the tokens (B) from shared memory.  All roles walk the same item
 // sequence; rings carry over from one item to the next.  The MMA issuer waits on a single
