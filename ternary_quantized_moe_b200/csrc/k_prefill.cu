@@ -395,7 +395,6 @@ struct TernParams {
   int* err;
 };
 
-constexpr uint32_t kAtom = 128 * 128;  // bytes of one 128-row x 64-column swizzled atom
 constexpr int kBN3 = 160;      // tokens per tile of batches whose experts average kMid160 or more
 constexpr int kMid160 = 112;   // mean tokens per expert from which both ternary GEMMs take kBN3 tiles
 
