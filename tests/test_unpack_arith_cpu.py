@@ -1,0 +1,92 @@
+"""The fp16 arithmetic identities the CUDA kernels' in-register unpack relies on, checked
+exhaustively on the CPU with numpy's binary16 rounding (a fused multiply-add is emulated as the
+exact fp64 value rounded once to fp16; every operand here is an fp16 value, so the fp64 product
+plus addend is exact).  The expected values are the containers' definitions: a PQ2_0 field holds
+code + 1 in two bits; a PTQ1_0 quintet byte holds five base-3 digits code + 1, least significant
+first ("Scion-35B-A3B" and "Scion-FlashNext-176B-A6B" model cards, Weight Representation).
+"""
+import numpy as np
+import pytest
+
+
+def f16(v):
+    return np.asarray(v, np.float64).astype(np.float16)
+
+
+def bits_to_f64(b):
+    return np.asarray(b, np.uint16).view(np.float16).astype(np.float64)
+
+
+def fma16(a, b, c):
+    return f16(np.asarray(a, np.float64) * np.asarray(b, np.float64) + np.asarray(c, np.float64))
+
+
+HALVES = np.arange(1 << 16, dtype=np.uint32)
+
+
+@pytest.mark.parametrize("s", range(8))
+def test_pq2_subnormal_fields(s):
+    """Decode ring kernels: pair s takes the field at bits 2f..2f+1 (f = s, or s - 5 after a
+    10-bit shift); masked alone it is the fp16 subnormal b * 4^f * 2^-24 with b the stored field."""
+    f = s if s < 5 else s - 5
+    src = HALVES if s < 5 else HALVES >> 10
+    b = (src >> (2 * f)) & 3
+    masked = src & (3 << (2 * f))
+    np.testing.assert_array_equal(bits_to_f64(masked), b * 4.0 ** f * 2.0 ** -24)
+
+
+@pytest.mark.parametrize("s", range(8))
+def test_pq2_magic_fields(s):
+    """Split-K decode and prefill expansion: the field ORed into the fp16 pattern of 1024, minus
+    1024 + 4^f, is 4^f * (b - 1) = 4^f * code, with no rounding."""
+    f = s if s < 5 else s - 5
+    src = HALVES if s < 5 else HALVES >> 10
+    b = (src >> (2 * f)) & 3
+    v = bits_to_f64((src & (3 << (2 * f))) | 0x6400)
+    got = f16(v.astype(np.float16).astype(np.float64) - f16(1024 + 4 ** f).astype(np.float64))
+    np.testing.assert_array_equal(got.astype(np.float64), 4.0 ** f * (b.astype(np.float64) - 1))
+
+
+def test_pq2_scaled_expansion_exact():
+    """Prefill expansion: 4^f * code times an fp16 group scale (the 4^f divided out of B later)
+    is exact in fp16 for every scale of the workloads' range and beyond."""
+    scales = f16(np.linspace(1e-3, 4.0, 4001))
+    for f in range(5):
+        for code in (-1, 0, 1):
+            got = f16(f16(4.0 ** f * code).astype(np.float64) * scales.astype(np.float64))
+            np.testing.assert_array_equal(got.astype(np.float64), 4.0 ** f * code * scales.astype(np.float64))
+
+
+def _digit_chain(V, n):
+    """n steps of the kernels' base-3 chain on fp16 values V = 1024 + v."""
+    third, c1, m3, c2047 = f16(0.333251953125), f16(682.5), f16(-3.0), f16(2047.0)
+    out = []
+    for _ in range(n):
+        Vn = fma16(V, third, c1)
+        code = f16(fma16(Vn, m3, V).astype(np.float64) + c2047.astype(np.float64))
+        out.append(code.astype(np.float64))
+        V = Vn
+    return out
+
+
+def test_ptq1_digit_chain_all_quintets():
+    """Every valid quintet byte (0..242): the chain yields its five digits minus one, least
+    significant first."""
+    v = np.arange(243)
+    codes = _digit_chain(f16(1024 + v), 5)
+    for j in range(5):
+        np.testing.assert_array_equal(codes[j], (v // 3 ** j) % 3 - 1)
+
+
+def test_ptq1_digit_chain_tail_byte():
+    """The tail byte (0..26) holds three digits; the same chain reads them."""
+    v = np.arange(27)
+    codes = _digit_chain(f16(1024 + v), 3)
+    for j in range(3):
+        np.testing.assert_array_equal(codes[j], (v // 3 ** j) % 3 - 1)
+
+
+def test_ptq1_chain_constants_are_fp16():
+    """The chain's constants are exact fp16 values (no rounding when they are loaded)."""
+    for c in (0.333251953125, 682.5, -3.0, 2047.0):
+        assert float(f16(c)) == c
