@@ -247,6 +247,17 @@ typedef struct {
 int scion_moe_forward_debug(const void* x, int T, const scion_layer* layer, float* out, const scion_debug_out* dbg,
                             void* stream);
 
+/* The routing of a batch alone ([P3]/[P4] Model Overview: top-k of the router logits; [P1]
+ * Serving notes: tokens grouped per expert for the expert matmul).  Runs the block forward on x
+ * (bf16 [T][d], device, 16-byte aligned) with the output going to the handle's own staging
+ * buffer, then copies ids [T][k] (int32), gates [T][k] (fp32), offsets [E+1] (int32) and perm
+ * [T*k] (int32) -- the same values and orders as the fields of scion_debug_out -- into the
+ * given device buffers; any of the four may be NULL (not written).  Calls on one handle must
+ * not overlap (the staging buffer is shared with scion_moe_forward_host).  EINVAL on a null x,
+ * a misaligned x or T out of range; ECUDA if a launch or copy fails. */
+int scion_debug_route(const void* x, int T, const scion_layer* layer, int32_t* ids, float* gates, int32_t* offsets,
+                      int32_t* perm, void* stream);
+
 /* ------------------------------------------------------------ measurement
  * Kernel-level timing for benchmarks.  Between scion_profile_begin and
  * scion_profile_end, every kernel a forward launches is bracketed by a pair of CUDA
@@ -278,8 +289,9 @@ int64_t scion_kernel_launches(void);
  * to another allocator, or they run where allocation is not allowed).  The pages
  * describe no counterpart of this entry point; it is a deployment aid.
  *   logits[t][e] = x_t . w_router[e] + x_t . w_router_delta[e]      (fp32)
- * x: device bf16 [T][d]; w_router, w_router_delta: device bf16 [E][d]; logits: device
- * fp32 [T][E], written.  Limits: T <= 64, E <= 512, d <= 4096 and d % 128 == 0; larger
+ * x: device bf16 [T][d]; w_router, w_router_delta: device bf16 [E][d], all three 16-byte
+ * aligned (they are read with 16-byte loads); logits: device fp32 [T][E], 4-byte aligned,
+ * written.  A null or misaligned pointer returns SCION_EINVAL and launches nothing.  Limits: T <= 64, E <= 512, d <= 4096 and d % 128 == 0; larger
  * sizes return SCION_EINVAL and launch nothing.  The split-K scratch lives in a static
  * device array inside the library (1 MiB + 128 B on every GPU that loads it, held until
  * the process exits); the call allocates nothing.  The first call on a device looks the

@@ -28,7 +28,7 @@ __all__ = [
     "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "STAGES", "scion_layer_check",
     "scion_router_logits_static", "scion_layer_set_option", "SCION_OPT_STREAM_MIN_TOKENS",
     "scion_moe_forward_residual", "scion_quantize_device", "SCION_QUANT_ABSMEAN", "SCION_QUANT_LLOYD",
-    "scion_selftest_bounded_wait",
+    "scion_selftest_bounded_wait", "scion_debug_route",
 ]
 
 SCION_PQ2_0 = 0
@@ -47,7 +47,7 @@ EXPORTS = (
     "scion_layer_device_bytes", "scion_moe_forward", "scion_moe_forward_host", "scion_moe_forward_debug",
     "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "scion_layer_check",
     "scion_router_logits_static", "scion_layer_set_option", "scion_moe_forward_residual", "scion_quantize_device",
-    "scion_selftest_bounded_wait",
+    "scion_selftest_bounded_wait", "scion_debug_route",
 )
 SCION_QUANT_ABSMEAN, SCION_QUANT_LLOYD = 0, 1
 SCION_OPT_STREAM_MIN_TOKENS = 1
@@ -108,6 +108,7 @@ def _load():
             "scion_selftest_bounded_wait": (ci, [ci, C.POINTER(C.c_int), C.POINTER(C.c_double), vp]),
             "scion_moe_forward_host": (ci, [vp, ci, vp, vp, vp]),
             "scion_moe_forward_debug": (ci, [vp, ci, vp, vp, C.POINTER(_Debug), vp]),
+            "scion_debug_route": (ci, [vp, ci, vp, vp, vp, vp, vp, vp]),
             "scion_profile_begin": (ci, [ci]),
             "scion_profile_end": (ci, [ci, C.POINTER(C.c_double), C.POINTER(C.c_int64)]),
             "scion_kernel_launches": (C.c_int64, []),
@@ -376,6 +377,18 @@ def scion_moe_forward_debug(x, T: int, layer: Layer, out, stream=None, **bufs) -
     st = _load().scion_moe_forward_debug(_dptr(x, "x", (torch.bfloat16,)), int(T), C.c_void_p(layer.handle),
                                          _dptr(out, "out", (torch.float32,)), C.byref(dbg), _stream(stream))
     _check(st, "scion_moe_forward_debug")
+
+
+def scion_debug_route(x, T: int, layer: Layer, ids=None, gates=None, offsets=None, perm=None, stream=None) -> None:
+    """The batch's routing into the given CUDA tensors: ids int32 [T, k], gates fp32 [T, k],
+    offsets int32 [E + 1], perm int32 [T * k] (each optional)."""
+    import torch
+
+    st = _load().scion_debug_route(_dptr(x, "x", (torch.bfloat16,)), int(T), C.c_void_p(layer.handle),
+                                   _dptr(ids, "ids", (torch.int32,)), _dptr(gates, "gates", (torch.float32,)),
+                                   _dptr(offsets, "offsets", (torch.int32,)), _dptr(perm, "perm", (torch.int32,)),
+                                   _stream(stream))
+    _check(st, "scion_debug_route")
 
 
 # ------------------------------------------------------------ measurement

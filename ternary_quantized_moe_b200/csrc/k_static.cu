@@ -138,6 +138,10 @@ extern "C" int scion_router_logits_static(const void* x, int T, const void* w_ro
     return SCION_EINVAL;
   if (T == 0) return SCION_OK;
   if (!x || !w_router || !w_router_delta || !logits) return SCION_EINVAL;
+  // x and both router matrices are read with 16-byte loads, logits written as fp32
+  if (((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w_router) |
+        reinterpret_cast<uintptr_t>(w_router_delta)) & 15) || (reinterpret_cast<uintptr_t>(logits) & 3))
+    return SCION_EINVAL;
   float* scratch = nullptr;
   int st = scratch_for_current_device(&scratch);
   if (st != SCION_OK) return st;

@@ -196,7 +196,21 @@ int forward_prefill(const scion_layer* L, const __nv_bfloat16* x, int T, float* 
   return SCION_OK;
 }
 
-// One pass of T <= SCION_TDEC tokens.
+// Same, but records the first failure in `status` and skips the launch once one has failed
+// (used where work already forked onto the side stream must still be joined).
+#define SCION_STAGE_INTO(status, stage, call)          \
+  do {                                                 \
+    if ((status) == SCION_OK) {                        \
+      cudaError_t e_;                                  \
+      {                                                \
+        StageScope scope_(stage, s);                   \
+        e_ = (call);                                   \
+      }                                                \
+      if (e_ != cudaSuccess) (status) = cuda_status(e_); \
+    }                                                  \
+  } while (0)
+
+// One decode pass of T <= SCION_TDEC tokens.
 int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, const float* resid, cudaStream_t s) {
   if (L->desc.router_fp32) SCION_STAGE(SCION_STAGE_ROUTER_F32, scion::launch_router_f32(L, x, T, L->logits, s));
   const bool ring = T >= L->stream_min_tokens;
@@ -207,30 +221,41 @@ int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out
   const bool side = ring && L->Kdense;
   const int nx_main = side ? L->n_xrouter : L->n_xunits;
   SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_xproj(L, x, T, out, resid, 0, nx_main, true, s));
+  int st = SCION_OK;
   if (side) {
     cudaError_t e = cudaEventRecord(L->ev_x, s);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(L->side, L->ev_x, 0);
-    if (e != cudaSuccess) return cuda_status(e);
+    if (e != cudaSuccess) return cuda_status(e);  // nothing was launched on the side stream
+    int st_side = SCION_OK;
     {
-      cudaStream_t s = L->side;  // SCION_STAGE launches and records on `s`
-      SCION_STAGE(SCION_STAGE_XPROJ,
-                  scion::launch_xproj(L, x, T, out, nullptr, L->n_xrouter, L->n_xunits - L->n_xrouter, false, s));
-      SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
+      cudaStream_t s = L->side;  // SCION_STAGE_INTO launches and records on `s`
+      SCION_STAGE_INTO(st_side, SCION_STAGE_XPROJ,
+                       scion::launch_xproj(L, x, T, out, nullptr, L->n_xrouter, L->n_xunits - L->n_xrouter, false, s));
+      SCION_STAGE_INTO(st_side, SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
     }
-    if ((e = cudaEventRecord(L->ev_dense, L->side)) != cudaSuccess) return cuda_status(e);
+    // the join is recorded whatever happened above, so that no later work on the caller's stream
+    // (a retry, the next call) can overlap side-stream work that still writes out or hz
+    if ((e = cudaEventRecord(L->ev_dense, L->side)) != cudaSuccess) {
+      cudaStreamSynchronize(L->side);
+      st_side = cuda_status(e);
+    }
+    st = st_side;
   }
-  SCION_STAGE(SCION_STAGE_ROUTE, scion::launch_route(L, T, s));
+  SCION_STAGE_INTO(st, SCION_STAGE_ROUTE, scion::launch_route(L, T, s));
   // small batches: the dense down projection rides in the gate/up launch (it needs only the
   // x-projection), off the critical path of the routed kernels
   const bool merged = !ring && scion::gateup_merges_dense(L, T);
-  SCION_STAGE(SCION_STAGE_GATEUP, ring     ? scion::launch_stream_gateup(L, T, s)
-                                  : merged ? scion::launch_gateup_dense(L, T, out, s)
-                                           : scion::launch_gateup(L, x, T, s));
-  SCION_STAGE(SCION_STAGE_DOWN_ROUTED,
-              ring ? scion::launch_stream_down(L, T, out, s) : scion::launch_down_routed(L, T, out, s));
-  if (side) return cuda_status(cudaStreamWaitEvent(s, L->ev_dense, 0));
-  if (L->Kdense && !merged) SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
-  return SCION_OK;
+  SCION_STAGE_INTO(st, SCION_STAGE_GATEUP, ring     ? scion::launch_stream_gateup(L, T, s)
+                                           : merged ? scion::launch_gateup_dense(L, T, out, s)
+                                                    : scion::launch_gateup(L, x, T, s));
+  SCION_STAGE_INTO(st, SCION_STAGE_DOWN_ROUTED,
+                   ring ? scion::launch_stream_down(L, T, out, s) : scion::launch_down_routed(L, T, out, s));
+  if (side) {
+    const cudaError_t e = cudaStreamWaitEvent(s, L->ev_dense, 0);
+    return st != SCION_OK ? st : cuda_status(e);
+  }
+  if (L->Kdense && !merged) SCION_STAGE_INTO(st, SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
+  return st;
 }
 
 }  // namespace
@@ -381,14 +406,10 @@ int forward_any(const void* x, int T, const scion_layer* L, const float* resid, 
     return SCION_EINVAL;
   cudaStream_t s = as_stream(stream);
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-  if (T > SCION_TDEC && L->pre) return forward_prefill(L, xb, T, out, resid, s);
-  for (int t0 = 0; t0 < T; t0 += SCION_TDEC) {
-    const int n = T - t0 < SCION_TDEC ? T - t0 : SCION_TDEC;
-    int st = forward_pass(L, xb + int64_t(t0) * L->d, n, out + int64_t(t0) * L->d,
-                          resid ? resid + int64_t(t0) * L->d : nullptr, s);
-    if (st != SCION_OK) return st;
-  }
-  return SCION_OK;
+  // a layer built for more than one decode pass (max_tokens > SCION_TDEC) has the tensor-core
+  // path, so every batch is either one decode pass or one prefill
+  if (T > SCION_TDEC) return forward_prefill(L, xb, T, out, resid, s);
+  return forward_pass(L, xb, T, out, resid, s);
 }
 }  // namespace
 
@@ -442,6 +463,15 @@ extern "C" int scion_moe_forward_debug(const void* x, int T, const scion_layer* 
     e = cudaMemcpy2DAsync(dbg->hz, sizeof(__half) * L->Kdense, pre ? P->hz : L->hz, sizeof(__half) * L->Kd,
                           sizeof(__half) * L->Kdense, T, cudaMemcpyDeviceToDevice, s);
   return cuda_status(e);
+}
+
+extern "C" int scion_debug_route(const void* x, int T, const scion_layer* L, int32_t* ids, float* gates,
+                                 int32_t* offsets, int32_t* perm, void* stream) {
+  if (!L) return SCION_EINVAL;
+  scion_debug_out dbg;
+  memset(&dbg, 0, sizeof(dbg));
+  dbg.ids = ids, dbg.gates = gates, dbg.offsets = offsets, dbg.perm = perm;
+  return scion_moe_forward_debug(x, T, L, L->out_stage, &dbg, stream);
 }
 
 extern "C" int scion_layer_check(const scion_layer* L, void* stream) {

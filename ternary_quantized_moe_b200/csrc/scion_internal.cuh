@@ -32,7 +32,7 @@
 
 #include "../../include/scion.h"
 
-#define SCION_TDEC 64         // tokens per decode pass (larger batches run in passes)
+#define SCION_TDEC 64         // tokens of the decode path (larger batches take the tensor-core path)
 #define SCION_XPROJ_KC 512    // K columns per x-projection CTA (4 warps x 128)
 
 // Fragment-ordered B operands of the decode expert kernels (x for gate/up, h for down) are

@@ -101,3 +101,25 @@ def test_layer_create_rejects_null_banks_and_tokens():
     assert lib.scion_layer_create(C.byref(D), 16, None, C.byref(h)) == tq.SCION_EINVAL
     assert lib.scion_layer_create(C.byref(_desc()), 0, None, C.byref(h)) == tq.SCION_EINVAL
     assert lib.scion_moe_forward(None, 1, None, None, None) == tq.SCION_EINVAL
+
+
+@pytest.mark.parametrize("off", [(2, 0, 0, 0), (0, 8, 0, 0), (0, 0, 4, 0), (0, 0, 0, 2)])
+def test_static_router_rejects_misaligned_pointers_before_cuda(off):
+    """x and the router matrices are read with 16-byte loads and logits written as fp32: a
+    misaligned pointer is refused before any CUDA call (so this runs without a GPU; an aligned
+    call here would reach the CUDA runtime and report SCION_ECUDA instead)."""
+    lib = tq._load()
+    base = 0x10000
+    x, wr, wd, lg = (base + o for o in off)
+    assert lib.scion_router_logits_static(x, 8, wr, wd, 64, 256, lg, None) == tq.SCION_EINVAL
+
+
+def test_static_router_aligned_call_reaches_cuda():
+    """Without a GPU an aligned call passes the argument checks and stops at the CUDA runtime.
+    Skipped where a GPU is present: the pointers here are not device memory."""
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("fake pointers must not reach a real device")
+    lib = tq._load()
+    assert lib.scion_router_logits_static(0x10000, 8, 0x20000, 0x30000, 64, 256, 0x40000, None) == tq.SCION_ECUDA

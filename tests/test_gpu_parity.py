@@ -314,14 +314,64 @@ def test_packed_correction_rejects_invalid_codes_and_rank():
 
 
 @pytest.mark.parametrize("T", [64, 65, 150])
-def test_forward_multi_pass(T):
-    """Batches above one decode pass (64 tokens) run in passes; ragged tails included."""
+def test_forward_across_the_decode_limit(T):
+    """One layer built for up to 160 tokens: T = 64 runs the decode kernels, T = 65 and 150 (one
+    token past the limit, and a ragged 150) the tensor-core path; both against the oracle."""
     cfg = small("mp", synth.PTQ1_0, False, E=32, k=4)
     L, banks, ol, x = _case(cfg, T)
     layer = device_layer(cfg, L, banks, 160)
     got, _ = run_forward(layer, x, T)
     ref, _, _ = oracle.forward(ol, x)
     check_output(got, ref)
+
+
+@pytest.mark.parametrize("E,k,T", [(1024, 8, 1), (1024, 8, 13), (1024, 8, 64),
+                                   pytest.param(4096, 32, 64, marks=pytest.mark.slow)])
+def test_forward_decode_many_experts(E, k, T):
+    """Decode routing for more than 512 experts (the single-CTA grouping kernel with the logits
+    staged per warp in shared memory, then the slot records): ids, counts, offsets and the stable
+    permutation bit-exact, gates, hidden and output within tolerance; E = 4096 with k = 32 is the
+    largest layer the decode path accepts."""
+    cfg = small("me", synth.PQ2_0, False, E=E, k=k, d=256, F=128, Fs=128, r=16)
+    L, banks, ol, x = _case(cfg, T)
+    layer = device_layer(cfg, L, banks, 64)
+    del L, banks
+    got, dbg = run_forward(layer, x, T, debug=True, E=E, k=k, F=cfg.ffn, Kdense=cfg.shared_ffn + cfg.rank)
+    assert tq.scion_layer_check(layer) == 0
+    _check_routing(cfg, dbg, ol, x, T)
+    _check_hidden(cfg, dbg, ol, x, T)
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
+
+
+@pytest.mark.parametrize("T,max_tokens", [(13, 64), (200, 200)])
+def test_debug_route_matches_oracle(T, max_tokens):
+    """scion_debug_route (the routing alone): ids as sets per token, offsets and the grouping
+    bit-exact against the oracle, gates within the gate tolerance (decode and tensor-core path)."""
+    cfg = small("dr", synth.PTQ1_0, False, E=32, k=4)
+    L, banks, ol, x = _case(cfg, T)
+    layer = device_layer(cfg, L, banks, max_tokens)
+    ids = torch.empty((T, cfg.top_k), dtype=torch.int32, device=DEV)
+    gates = torch.empty((T, cfg.top_k), dtype=torch.float32, device=DEV)
+    offsets = torch.empty((cfg.n_experts + 1,), dtype=torch.int32, device=DEV)
+    perm = torch.empty((T * cfg.top_k,), dtype=torch.int32, device=DEV)
+    tq.scion_debug_route(u16_to_dev(x, torch.bfloat16, DEV), T, layer, ids=ids, gates=gates, offsets=offsets,
+                         perm=perm)
+    torch.cuda.synchronize()
+    _, rids, rgates = oracle.route(ol, x)
+    gi, gg = ids.cpu().numpy(), gates.cpu().numpy()
+    np.testing.assert_array_equal(np.sort(gi, 1), np.sort(rids, 1))
+    for t in range(T):
+        ref = dict(zip(rids[t].tolist(), rgates[t].tolist()))
+        for j in range(cfg.top_k):
+            assert abs(gg[t, j] - ref[int(gi[t, j])]) <= 1e-5 * ref[int(gi[t, j])]
+    _, roff, rperm = oracle.group(rids, cfg.n_experts)
+    np.testing.assert_array_equal(offsets.cpu().numpy(), roff)
+    gp = perm.cpu().numpy()
+    for e in range(cfg.n_experts):
+        np.testing.assert_array_equal(np.sort(gp[roff[e]:roff[e + 1]] // cfg.top_k),
+                                      np.sort(rperm[roff[e]:roff[e + 1]] // cfg.top_k))
+        assert (gi.reshape(-1)[gp[roff[e]:roff[e + 1]]] == e).all()
 
 
 def test_empty_batch_and_limits():
