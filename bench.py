@@ -1,11 +1,15 @@
 #!/usr/bin/env python
 """MoE-layer throughput of the ternary MoE block forward on B200.
 
-Default workload: the 35B-A3B-class decode layer (d=2048, 256 experts, top-8 + shared
-expert, ffn 512, PQ2_0 experts, rank-512 correction).  One step = one forward at each
-decode batch size b in {1, 8, 32, 64} (105 tokens), each call on the next of 40
-independent layers (9.1 GB of weights, far above the 126 MB L2, so every call reads
-its weights from HBM).  Metric: tokens/s over the whole job.
+One run measures the four synthetic workloads in turn and prints one JSON line: the
+headline (top-level keys) is the 35B-A3B-class decode layer (d=2048, 256 experts, top-8 +
+shared expert, ffn 512, PQ2_0 experts, rank-512 correction), where one step = one forward
+at each decode batch size b in {1, 8, 32, 64} (105 tokens), each call on the next of 40
+independent layers (9.1 GB of weights, far above the 126 MB L2, so every call reads its
+weights from HBM).  "workloads" holds the same figures for every workload: a3b_decode,
+a3b_prefill (4096 tokens), flashnext_decode (d=3072, 512 experts, top-10 + shared, PTQ1_0,
+b in {1, 16, 64}, 48 layers) and flashnext_prefill (16384 tokens, Zipf-loaded router).
+Metric: tokens/s over the whole job, with the roofline fraction of the dominant kernel.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl scion|reference]
 
@@ -57,9 +61,10 @@ def load_peaks():
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="a3b_decode")
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="all",
+                    help="all (the four measured workloads, a3b_decode first as the headline) or one name")
     ap.add_argument("--impl", default="scion", choices=["scion", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0, help="override the number of cycled layers")
@@ -179,7 +184,9 @@ class ClockSampler:
             time.sleep(0.01)
 
     def __enter__(self):
+        # re-entered once per timed region; the samples accumulate over all of them
         if self.ok:
+            self._stop.clear()
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
         return self
@@ -215,79 +222,106 @@ def oracle_sample(cfg, batches):
     return ol, xs
 
 
-def cpu_baseline(cfg):
+# Token counts of the bounded oracle samples of the prefill workloads: the first tokens of a
+# batch drawn like the workload's (same router, same x distribution, Zipf load included).
+PREFILL_SAMPLE_TOKENS = {"a3b_prefill": 256, "flashnext_prefill": 128}
+
+
+def oracle_batches(cfg):
+    """The batches one oracle step runs: the workload's own decode batches, or a bounded sample
+    of a prefill batch."""
+    if max(cfg.tokens) <= 64:
+        return list(cfg.tokens)
+    return [PREFILL_SAMPLE_TOKENS.get(cfg.name, 64)]
+
+
+def cpu_baseline(cfg, seconds=5.0):
+    """The oracle as it stands on the host cores: its batch set repeated for about `seconds` of
+    CPU work (at least once, at most 6x that)."""
     import oracle
 
-    batches = cfg.tokens if max(cfg.tokens) <= 64 else [64]
+    batches = oracle_batches(cfg)
     ol, xs = oracle_sample(cfg, batches)
     t0 = time.perf_counter()
     reps = 0
-    while True:  # repeat the batch set until about 10 s of CPU work (bounded at 30 s)
+    while True:
         for x in xs:
             oracle.forward(ol, x)
         reps += 1
         dt = time.perf_counter() - t0
-        if dt >= 10.0 or dt * (reps + 1) / reps > 30.0:
+        if dt >= seconds or dt * (reps + 1) / reps > 6 * seconds:
             break
     ntok = sum(batches) * reps
+    what = ("one forward per batch %s" % batches if max(cfg.tokens) <= 64 else
+            "one forward of the first %d tokens of a %d-token batch" % (batches[0], cfg.tokens[0]))
     return {"value": ntok / dt, "unit": "tokens/s", "cores": oracle.cores_used(), "kind": "oracle",
-            "sample": "%s layer 0 (host-generated), %d x one forward per batch %s = %d tokens, %.1f s"
-                      % (cfg.name, reps, batches, ntok, dt)}
+            "sample": "%s layer 0 (host-generated), %d x %s = %d tokens, %.1f s" % (cfg.name, reps, what, ntok, dt)}
 
 
 def run_reference(args, rank):
-    """The oracle arm: plain fp64 C reference on the host cores, rank 0 only."""
+    """The oracle arm: plain fp64 C reference on the host cores, rank 0 only.  A step is the
+    headline workload's own step (one forward at each of its decode batch sizes, or a bounded
+    sample of its prefill batch) on layer 0; the other workloads get bounded samples too."""
     if rank != 0:
         return
     import oracle
     from workloads import synth
 
-    cfg = synth.CONFIGS[args.workload]
-    ol, xs = oracle_sample(cfg, [1])
-    x = xs[0]
+    names = workload_names(args)
+    cfg = synth.CONFIGS[names[0]]
+    batches = oracle_batches(cfg)
+    ol, xs = oracle_sample(cfg, batches)
     for _ in range(args.warmup):
-        oracle.forward(ol, x)
+        for x in xs:
+            oracle.forward(ol, x)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.forward(ol, x)
+        for x in xs:
+            oracle.forward(ol, x)
     dt = time.perf_counter() - t0
-    v = args.steps / dt
+    v = sum(batches) * args.steps / dt
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic",
-            "config": {"workload": cfg.name, "d": cfg.d, "experts": cfg.n_experts, "top_k": cfg.top_k,
-                       "ffn": cfg.ffn, "format": "PQ2_0" if cfg.fmt == 0 else "PTQ1_0"},
+            "data": "synthetic", "config": workload_config(cfg, args),
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.cores_used(), "kind": "oracle",
-                             "sample": "each step: one single-token forward on layer 0 of %s" % cfg.name},
+                             "sample": "each step: one forward per batch %s on layer 0 of %s" % (batches, cfg.name)},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    if len(names) > 1:
+        line["workloads"] = {n: {"cpu_baseline": cpu_baseline(synth.CONFIGS[n], 3.0)} for n in names[1:]}
     print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------------- GPU arm
-def run_gpu(args, rank, world, local_rank):
+ALL_WORKLOADS = ("a3b_decode", "a3b_prefill", "flashnext_decode", "flashnext_prefill")
+
+
+def workload_names(args):
+    """The workloads of one run, the headline first."""
+    return list(ALL_WORKLOADS) if args.workload == "all" else [args.workload]
+
+
+def workload_config(cfg, args, n_layers=None, weight_bytes=None):
+    c = {"workload": cfg.name, "d": cfg.d, "experts": cfg.n_experts, "top_k": cfg.top_k, "ffn": cfg.ffn,
+         "shared_ffn": cfg.shared_ffn, "rank": cfg.rank, "format": "PQ2_0" if cfg.fmt == 0 else "PTQ1_0",
+         "correction": "PQ2_0 blocks" if args.packed_corr else "bf16", "batches": list(cfg.tokens),
+         "tokens_per_step": sum(cfg.tokens)}
+    if cfg.zipf_s is not None:
+        c["router_load"] = "Zipf(%.1f) over a seeded permutation of the experts" % cfg.zipf_s
+    if n_layers is not None:
+        c["layers_cycled"] = n_layers
+    if weight_bytes is not None:
+        c["l2"] = "inputs larger than L2: %.1f GB of layers cycled" % (weight_bytes / 1e9)
+    return c
+
+
+def build_layers(cfg, args, dev, n_layers, max_T):
     import torch
-    import torch.distributed as dist
 
     import ternary_quantized_moe_b200 as tq
     from workloads import synth
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    if world > 1:
-        from datetime import timedelta
-
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
-
-    cfg = synth.CONFIGS[args.workload]
-    n_layers = args.layers or cfg.n_layers
-    batches = list(cfg.tokens)
-    max_T = max(batches)
-    peaks, peak_src = load_peaks()
-
-    # ---- layers (generated and packed on the GPU, then re-tiled by scion_layer_create)
     layers = []
-    cb = 34.0 / 128.0 if args.packed_corr else 2.0
     for l in range(n_layers):
         W = synth.layer_device(cfg, l, dev)
         banks = {n: tq.scion_pack_device(cfg.fmt, W.pop(n + "_codes"), W.pop(n + "_scales")) for n in
@@ -313,6 +347,23 @@ def run_gpu(args, rank, world, local_rank):
             tq.scion_layer_set_option(layers[-1], tq.SCION_OPT_STREAM_MIN_TOKENS, args.stream_min_tokens)
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
+    return layers
+
+
+def measure(cfg, args, rank, world, dev, peaks, peak_src, clocks):
+    """Every figure of one workload: device-timed throughput, per-kernel times, rooflines, per
+    batch size, end to end through the host-buffer entry point, and the oracle baseline."""
+    import torch
+    import torch.distributed as dist
+
+    import ternary_quantized_moe_b200 as tq
+    from workloads import synth
+
+    n_layers = args.layers or cfg.n_layers
+    batches = list(cfg.tokens)
+    max_T = max(batches)
+    layers = build_layers(cfg, args, dev, n_layers, max_T)
+    cb = 34.0 / 128.0 if args.packed_corr else 2.0
     weight_bytes = sum(tq.scion_layer_device_bytes(L) for L in layers)
 
     xs = {T: synth.x_device(cfg, T, dev) for T in batches}
@@ -329,7 +380,6 @@ def run_gpu(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
-
     def timed(fn, K):
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -342,13 +392,13 @@ def run_gpu(args, rank, world, local_rank):
         barrier()
         return max_over_ranks(ms, world, dev)
 
-    for s in range(args.warmup):
+    for s in range(max(3, args.warmup)):
         step(s)
     K = args.steps
 
     # ---- headline: device-timed region, inputs resident in HBM
     launches0 = tq.scion_kernel_launches()
-    with ClockSampler(dev) as clocks:
+    with clocks:
         ms = timed(step, K)
     launches = tq.scion_kernel_launches() - launches0
     tokens_per_step = sum(batches)
@@ -366,11 +416,8 @@ def run_gpu(args, rank, world, local_rank):
     counts = torch.empty(cfg.n_experts, dtype=torch.int32, device=dev)
     for li in range(n_layers):
         for T in batches:
-            if T <= 64:
-                tq.scion_moe_forward_debug(xs[T], T, layers[li], outs[T], stream, counts=counts)
-                U[(li, T)] = int((counts > 0).sum().item())
-            else:
-                U[(li, T)] = cfg.n_experts
+            tq.scion_moe_forward_debug(xs[T], T, layers[li], outs[T], stream, counts=counts)
+            U[(li, T)] = int((counts > 0).sum().item())
     sched = [((s * nb + i) % n_layers, T) for s in range(K) for i, T in enumerate(batches)]
     bytes_total = sum(workload_bytes(cfg, T, U[(li, T)], cb) for li, T in sched)
     # the active experts' packed banks alone (U distinct experts per call)
@@ -391,13 +438,15 @@ def run_gpu(args, rank, world, local_rank):
 
     # ---- per batch size (each batch alone, cycling layers)
     per_batch = {}
-    for T in batches:
-        def one(s, T=T):
-            tq.scion_moe_forward(xs[T], T, layers[s % n_layers], outs[T], stream)
-        msT = timed(one, K)
-        bT = sum(workload_bytes(cfg, T, U[(s % n_layers, T)], cb) for s in range(K))
-        per_batch[str(T)] = {"tokens_per_s": job_tokens_per_s(world, T, K, msT), "us_per_call": 1000.0 * msT / K,
-                             "hbm_frac": (bT / (msT / 1000.0)) / (peaks["hbm_gbs"] * 1e9)}
+    if nb > 1:
+        for T in batches:
+            def one(s, T=T):
+                tq.scion_moe_forward(xs[T], T, layers[s % n_layers], outs[T], stream)
+            msT = timed(one, K)
+            bT = sum(workload_bytes(cfg, T, U[(s % n_layers, T)], cb) for s in range(K))
+            per_batch[str(T)] = {"tokens_per_s": job_tokens_per_s(world, T, K, msT),
+                                 "us_per_call": 1000.0 * msT / K,
+                                 "hbm_frac": (bT / (msT / 1000.0)) / (peaks["hbm_gbs"] * 1e9)}
 
     # ---- end to end through the host-buffer entry point (pinned host x in, out back to host)
     xh = {T: xs[T].cpu().pin_memory() for T in batches}
@@ -428,30 +477,22 @@ def run_gpu(args, rank, world, local_rank):
                 "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": load_traffic(cfg.name, dom),
                 "peak_source": peak_src, "flops_per_launch": sflops[dom] / dom_n,
                 "us_per_launch": 1000.0 * dom_ms / dom_n}
-
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
-        "data": "synthetic",
-        "config": {"workload": cfg.name, "d": cfg.d, "experts": cfg.n_experts, "top_k": cfg.top_k, "ffn": cfg.ffn,
-                   "shared_ffn": cfg.shared_ffn, "rank": cfg.rank, "format": "PQ2_0" if cfg.fmt == 0 else "PTQ1_0",
-                   "correction": "PQ2_0 blocks" if args.packed_corr else "bf16", "batches": batches, "layers_cycled": n_layers, "tokens_per_step": tokens_per_step,
-                   "l2": "inputs larger than L2: %.1f GB of layers cycled" % (weight_bytes / 1e9),
-                   "parallelism": "replicas" if world > 1 else "single"},
-        "roofline": roof,
-        "step_roofline": {"bytes_per_step": bytes_total / K, "hbm_frac": (bytes_total / (ms / 1000.0)) /
-                          (peaks["hbm_gbs"] * 1e9), "tflops": flops_total / (ms / 1000.0) / 1e12,
-                          "expert_bytes_per_step": expert_bytes / K,
-                          "expert_stage_hbm_frac": (expert_bytes / ((stages.get("gateup", (0, 0))[0] +
-                                                                     stages.get("down_routed", (0, 0))[0]) / 1000.0)
-                                                    / (peaks["hbm_gbs"] * 1e9))
-                          if stages.get("gateup", (0, 0))[0] > 0 else None,
-                          # the same step against nominal figures: HBM3e at 8 TB/s, and the bf16
-                          # throughput a seconds-long GEMM sustains under the power cap
-                          "hbm_frac_vs_nominal_8tbs": (bytes_total / (ms / 1000.0)) / 8e12,
-                          "tflops_frac_vs_sustained": flops_total / (ms / 1000.0) / 1e12 /
-                          peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])},
-        "per_batch": per_batch,
+    step_roof = {"bytes_per_step": bytes_total / K, "hbm_frac": (bytes_total / (ms / 1000.0)) / (peaks["hbm_gbs"] * 1e9),
+                 "tflops": flops_total / (ms / 1000.0) / 1e12,
+                 "tflops_frac": flops_total / (ms / 1000.0) / 1e12 / peaks["bf16_tflops"],
+                 "expert_bytes_per_step": expert_bytes / K,
+                 "expert_stage_hbm_frac": (expert_bytes / ((stages.get("gateup", (0, 0))[0] +
+                                                            stages.get("down_routed", (0, 0))[0]) / 1000.0)
+                                           / (peaks["hbm_gbs"] * 1e9)) if stages.get("gateup", (0, 0))[0] > 0 else None,
+                 # the same step against nominal figures: HBM3e at 8 TB/s, and the bf16 throughput
+                 # a seconds-long GEMM sustains under the power cap
+                 "hbm_frac_vs_nominal_8tbs": (bytes_total / (ms / 1000.0)) / 8e12,
+                 "tflops_frac_vs_sustained": flops_total / (ms / 1000.0) / 1e12 /
+                 peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])}
+    res = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "ms_per_step": ms / K,
+        "config": workload_config(cfg, args, n_layers, weight_bytes),
+        "roofline": roof, "step_roofline": step_roof,
         "stages_us_per_launch": {k_: 1000.0 * v[0] / v[1] for k_, v in stages.items() if v[1]},
         "stages_rate": {k_: (sbytes[k_] / (v[0] / 1000.0) / 1e9 if decode else
                              sflops.get(k_, 0) / (v[0] / 1000.0) / 1e12)
@@ -460,12 +501,55 @@ def run_gpu(args, rank, world, local_rank):
         "stages_share": {k_: v[0] / sum(x[0] for x in stages.values()) for k_, v in stages.items() if v[1]},
         "e2e": e2e,
         "gpu_launches": int(launches),
-        "clocks": clocks.summary(),
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg)
+    if per_batch:
+        res["per_batch"] = per_batch
+    if not decode:
+        # routing of the prefill batch: empty experts and the heaviest expert's share of the entries
+        tq.scion_moe_forward_debug(xs[max_T], max_T, layers[0], outs[max_T], stream, counts=counts)
+        c = counts.cpu()
+        res["routing"] = {"empty_experts": int((c == 0).sum()), "max_expert_tokens": int(c.max()),
+                          "mean_expert_tokens": float(c.float().mean())}
     for L in layers:
         L.close()
+    del layers, xs, outs, xh, oh
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(cfg)
+    return res
+
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from workloads import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    peaks, peak_src = load_peaks()
+    clocks = ClockSampler(dev)  # sampled during every timed region of every workload
+    names = workload_names(args)
+    results = {n: measure(synth.CONFIGS[n], args, rank, world, dev, peaks, peak_src, clocks) for n in names}
+    head = results[names[0]]
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+        "config": dict(head["config"], parallelism="replicas" if world > 1 else "single"),
+    }
+    for k_ in ("roofline", "step_roofline", "per_batch", "stages_us_per_launch", "stages_rate", "stages_rate_unit",
+               "stages_share", "e2e", "gpu_launches", "cpu_baseline"):
+        if k_ in head:
+            line[k_] = head[k_]
+    line["clocks"] = clocks.summary()
+    if len(names) > 1:
+        line["workloads"] = results
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -197,6 +197,13 @@ size_t scion_layer_device_bytes(const scion_layer* layer);
  * 16..64 tokens fork the dense down projection onto a stream owned by the handle and
  * join it back (events) before the call's work on `stream` ends; stream capture into
  * a CUDA graph records the fork and the join.
+ * Activation range: any finite bf16 x.  The expert GEMMs and the stored hidden values run in
+ * fp16; every token whose largest |x| lies outside [2^-3, 2^6) is scaled by a power of two
+ * 2^s (s = 2 - floor(log2 max|x|), clamped to [-40, 40]) on its way into them and scaled back
+ * exactly where its results enter out, so tokens with outlier channels (tested up to 3e4),
+ * tokens of tiny magnitude (tested near 1e-6) and large ones keep the block tolerance; max|x|
+ * inside [2^-38, 2^42] is fully normalised.  The output itself is fp32: a block output beyond
+ * the fp32 range overflows.
  * EINVAL on a null or misaligned pointer or T out of range; ECUDA if a launch fails. */
 int scion_moe_forward(const void* x, int T, const scion_layer* layer, float* out, void* stream);
 
@@ -239,9 +246,11 @@ typedef struct {
   int32_t* counts;  /* [E] tokens routed to each expert */
   int32_t* offsets; /* [E+1] exclusive scan of counts */
   int32_t* perm;    /* [T*k] entries t*k+j, grouped by expert, token order within an expert */
-  uint16_t* h;      /* fp16 [T*k][F] expert SwiGLU hidden, row p for perm[p] */
-  uint16_t* hz;     /* fp16 [T][Fs + r] shared SwiGLU hidden then correction z = A x */
+  uint16_t* h;      /* fp16 [T*k][F] expert SwiGLU hidden, row p for perm[p], times 2^(2s) */
+  uint16_t* hz;     /* fp16 [T][Fs + r] shared SwiGLU hidden then correction z = A x, times 2^p */
 } scion_debug_out;
+/* (s is the token's range exponent of scion_moe_forward, 0 for max|x| in [2^-3, 2^6); p = s for
+ * s > 0 on a layer with a correction, else 2s.) */
 
 /* scion_moe_forward, then copies the intermediates requested in `dbg`. */
 int scion_moe_forward_debug(const void* x, int T, const scion_layer* layer, float* out, const scion_debug_out* dbg,

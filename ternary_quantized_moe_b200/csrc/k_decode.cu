@@ -39,7 +39,8 @@ struct XProjArgs {
   int n_aux;           // CTA columns after the units that run xproj_aux (0 or kXAux)
   float* logits;
   __half* hz;
-  __half* xfrag;  // [T][d/128][SCION_BROW] fp16 in fragment order + group sums
+  __half* xfrag;  // [T][d/128][SCION_BROW] fp16 x 2^s_t in fragment order + group sums
+  int32_t* xexp;  // [T] range exponent s_t of each token (token_shift), written by the aux CTAs
   __half* h;      // [T*k][F/128][SCION_BROW] expert hidden: group-sum tails zeroed here
   int k, GF;
   const uint8_t* corr_blocks;  // ternary correction A (PQ2_0 blocks [r][d/128]) or nullptr (bf16 corr_a)
@@ -60,38 +61,52 @@ constexpr size_t xproj_smem(int T) {
                                                                     : size_t(8) * 2 * NT * 32 * 4 * 4;
 }
 
+// Largest magnitude of eight bf16 values, as the bit pattern of their absolute value.
+__device__ __forceinline__ uint32_t max_mag8(uint4 v) {
+  const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu), __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+  return max(m & 0xFFFFu, m >> 16);
+}
+
 __device__ __forceinline__ void xproj_aux(const XProjArgs& a, int aux, int n_aux) {
   const int Gd = a.d >> 7;
   const int lane = threadIdx.x & 31;
-  // x -> fragment order: item = (token, group, 8-element part); the 16 parts of a group sit in
-  // 16 consecutive lanes, which sum the group's B * 4^f for the row tail.
-  const int total = a.T * Gd * 16;
-  for (int base = aux * kXThreads + (threadIdx.x & ~31); base < total; base += n_aux * kXThreads) {
-    const int item = base + lane;
-    const bool ok = item < total;
-    const int grp = ok ? item >> 4 : 0, part = item & 15;
-    const int t = grp / Gd, g = grp % Gd;
-    const __nv_bfloat16* src = a.x + int64_t(t) * a.d + g * 128;
-    __align__(16) __half o[8];
-    float sum = 0.f;
+  const int gw = aux * (kXThreads / 32) + (threadIdx.x >> 5), nw = n_aux * (kXThreads / 32);
+  // one warp per token: the row's largest magnitude fixes its range exponent s_t, then x 2^s_t
+  // goes to the fragment order, two groups per step (16 lanes per group, 8 elements per lane);
+  // the 16 lanes of a group sum its B * 4^f for the row tail
+  for (int t = gw; t < a.T; t += nw) {
+    const __nv_bfloat16* row = a.x + int64_t(t) * a.d;
+    uint32_t mx = 0;
+    for (int i = lane; i < a.d / 8; i += 32) mx = max(mx, max_mag8(*reinterpret_cast<const uint4*>(row + 8 * i)));
+    const int sh = token_shift(__reduce_max_sync(0xffffffffu, mx));
+    if (lane == 0) a.xexp[t] = sh;
+    const float xs = pow2i(sh);
+    for (int g0 = 0; g0 < Gd; g0 += 2) {
+      const int g = g0 + (lane >> 4), part = lane & 15;
+      const bool ok = g < Gd;
+      const __nv_bfloat16* src = row + g * 128;
+      __align__(16) __half o[8];
+      float sum = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int idx = part * 8 + e;
-      const float v = ok ? __bfloat162float(src[brow_col(a.fmt, idx)]) : 0.f;
-      if (a.fmt == SCION_PQ2_0) {
-        const float up = 1.0f / brow_bscale(idx);
-        o[e] = __float2half_rn(v / up);
-        sum += __half2float(o[e]) * up;
-      } else {
-        o[e] = __float2half_rn(v);
+      for (int e = 0; e < 8; ++e) {
+        const int idx = part * 8 + e;
+        const float v = ok ? __bfloat162float(src[brow_col(a.fmt, idx)]) * xs : 0.f;
+        if (a.fmt == SCION_PQ2_0) {
+          const float up = 1.0f / brow_bscale(idx);
+          o[e] = __float2half_rn(v / up);
+          sum += __half2float(o[e]) * up;
+        } else {
+          o[e] = __float2half_rn(v);
+        }
       }
-    }
 #pragma unroll
-    for (int off = 8; off; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    __half* dst = a.xfrag + int64_t(grp) * SCION_BROW;
-    if (ok) {
-      *reinterpret_cast<uint4*>(dst + part * 8) = *reinterpret_cast<const uint4*>(o);
-      if (part == 0) *reinterpret_cast<float4*>(dst + 128) = make_float4(-5.9604644775390625e-08f * sum, 0.f, 0.f, 0.f);
+      for (int off = 8; off; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      __half* dst = a.xfrag + (int64_t(t) * Gd + g) * SCION_BROW;
+      if (ok) {
+        *reinterpret_cast<uint4*>(dst + part * 8) = *reinterpret_cast<const uint4*>(o);
+        if (part == 0)
+          *reinterpret_cast<float4*>(dst + 128) = make_float4(-5.9604644775390625e-08f * sum, 0.f, 0.f, 0.f);
+      }
     }
   }
   const int tid = aux * kXThreads + threadIdx.x, nth = n_aux * kXThreads;
@@ -129,6 +144,8 @@ template <int NT>
 __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
   extern __shared__ __align__(16) uint8_t xsm[];
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(xsm);  // [NT*8][kXRow], then the warp reduction
+  __shared__ uint32_t tmax[SCION_TDEC];  // largest |x| bits of each token over this CTA's K chunk
+  __shared__ int tshift[SCION_TDEC];     // lead CTA: range exponent of each token
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, c = lane & 3;
   const int chunk = blockIdx.y;
@@ -195,6 +212,10 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
         wb[m][q] = (ld && ok_b) ? ldg_stream(mats[m] + int64_t(row_b) * a.d + kk) : make_uint4(0, 0, 0, 0);
       }
   }
+  // the shared-expert and correction rows are stored scaled per token (hz_shift), which needs the
+  // largest |x| of each token: each chunk's CTA finds it over its columns, the lead combines them
+  const bool need_max = u.kind != kUnitRouter;
+  for (int i = threadIdx.x; i < SCION_TDEC; i += kXThreads) tmax[i] = 0;
   pdl_wait();  // everything below reads x or writes the workspace
   // stage x[0..T)[kbase .. kbase+512) in shared memory (rows padded by 16 B: conflict-free reads)
   const int kchunks = min(SCION_XPROJ_KC, a.d - kbase) >> 3;  // 16-byte chunks per token row (<= 64)
@@ -207,6 +228,11 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
+  if (need_max)
+    for (int i = threadIdx.x; i < a.T * kchunks; i += kXThreads) {
+      const int t = i / kchunks, j = i % kchunks;
+      atomicMax(&tmax[t], max_mag8(*reinterpret_cast<const uint4*>(xs + t * kXRow + 8 * j)));
+    }
   if (active_warp) {
     const bool second_acc = (u.kind == kUnitSwiglu);
     const int kwl = warp * 64;
@@ -268,6 +294,15 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
   // epilogue (chunk 0): thread -> (row, tok); all remote loads of the thread are issued together
   constexpr int kIt = 16 * SCION_TDEC / kXThreads;
   float v[kIt][2];
+  if (lead && need_max) {
+    for (int t = threadIdx.x; t < a.T; t += kXThreads) {
+      uint32_t m = tmax[t];
+      for (int ch = 1; ch < a.n_chunks; ++ch)
+        m = max(m, ld_dsmem_u32(map_cluster_rank(smem_addr(&tmax[t]), ch)));
+      tshift[t] = hz_shift(token_shift(m), a.r > 0);
+    }
+    __syncthreads();
+  }
   if (lead) {
 #pragma unroll
     for (int it = 0; it < kIt; ++it) {
@@ -296,9 +331,9 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
     if (u.kind == kUnitRouter) {
       a.logits[int64_t(tok) * a.E + grow] = v[it][0];
     } else if (u.kind == kUnitSwiglu) {
-      a.hz[int64_t(tok) * a.Kd + grow] = __float2half_rn(silu_f(v[it][0]) * v[it][1]);
+      a.hz[int64_t(tok) * a.Kd + grow] = __float2half_rn(silu_f(v[it][0]) * v[it][1] * pow2i(tshift[tok]));
     } else {
-      a.hz[int64_t(tok) * a.Kd + a.Fs + grow] = __float2half_rn(v[it][0]);
+      a.hz[int64_t(tok) * a.Kd + a.Fs + grow] = __float2half_rn(v[it][0] * pow2i(tshift[tok]));
     }
   }
 }
@@ -309,8 +344,9 @@ struct GateUpArgs {
   const __half* xfrag;  // [T][Gd][128]
   const int4* slot_info;
   const int32_t *n_active, *perm;
+  const int32_t* xexp;  // [T] range exponent of each token
   int d, F, k, Gd, fmt;
-  __half* hfrag;  // [T*k][GF][128] fragment order of the down format
+  __half* hfrag;  // [T*k][GF][128] fragment order of the down format, h 2^(2 s_t)
 };
 
 constexpr int kGuWarps = 8;
@@ -368,7 +404,8 @@ __device__ __forceinline__ void gateup_body(const GateUpArgs& a, int slot, int f
         const int f = ft * 16 + row;
         const int64_t pos = p0 + pc + tcol;
         const int idx = brow_pos(a.fmt, f & 127);
-        float h = silu_f(gs) * us;
+        const int sh = a.xexp[a.perm[pos] / a.k];  // the sums are of x 2^sh
+        float h = silu_f(gs * pow2i(-sh)) * (us * pow2i(sh));
         if (a.fmt == SCION_PQ2_0) h *= brow_bscale(idx);
         a.hfrag[(pos * GF + (f >> 7)) * SCION_BROW + idx] = __float2half_rn(h);
       }
@@ -389,6 +426,7 @@ struct DownArgs {
   const int4* slot_info;
   const int32_t *n_active, *perm;
   const float* gates;
+  const int32_t* xexp;  // [T] range exponent of each token (the hidden is h 2^(2 s_t))
   int d, F, k, GF;
   float* out;
 };
@@ -440,7 +478,8 @@ __global__ void __launch_bounds__(kDnWarps * 32) down_routed_kernel(DownArgs a) 
       const int row = (ln >> 2) + 8 * (i >> 1), tcol = 2 * (ln & 3) + (i & 1);
       if (tcol < nn) {
         const int entry = a.perm[p0 + pc + tcol];
-        atomicAdd(&a.out[int64_t(entry / a.k) * a.d + dt * 16 + row], a.gates[entry] * v);
+        const int t = entry / a.k;
+        atomicAdd(&a.out[int64_t(t) * a.d + dt * 16 + row], a.gates[entry] * pow2i(-2 * a.xexp[t]) * v);
       }
     }
     __syncthreads();
@@ -461,6 +500,7 @@ struct DenseArgs {
   // (nullptr: every column from w)
   const uint8_t* corr_b;
   int Fs, r;
+  const int32_t* xexp;  // [T] range exponent of each token: hz rows hold 2^hz_shift(s_t, r > 0) times their values
 };
 
 constexpr int kDnKc = 256;            // K columns per CTA
@@ -549,7 +589,7 @@ __device__ __forceinline__ void dense_body(const DenseArgs& a, int bx, int by) {
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) v += red[(((h + 2 * ks) * NT + nt) * 32 + ln) * 4 + i];
     const int row = bx * 32 + 16 * h + (ln >> 2) + 8 * (i >> 1), tok = nt * 8 + 2 * (ln & 3) + (i & 1);
-    if (tok < a.T) atomicAdd(&a.out[int64_t(tok) * a.d + row], v);
+    if (tok < a.T) atomicAdd(&a.out[int64_t(tok) * a.d + row], v * pow2i(-hz_shift(a.xexp[tok], a.r > 0)));
   }
 }
 
@@ -603,7 +643,7 @@ cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, fl
   a.sh_up = static_cast<const __nv_bfloat16*>(L->desc.sh_up);
   a.corr_a = static_cast<const __nv_bfloat16*>(L->desc.corr_a);
   a.units = L->xunits + unit0, a.n_units = n_units, a.n_chunks = L->n_xchunks, a.n_aux = aux ? kXAux : 0;
-  a.logits = L->logits, a.hz = L->hz, a.xfrag = L->xfrag, a.out = out;
+  a.logits = L->logits, a.hz = L->hz, a.xfrag = L->xfrag, a.xexp = L->xexp, a.out = out;
   a.corr_blocks = L->desc.corr_packed ? static_cast<const uint8_t*>(L->desc.corr_a) : nullptr;
   a.h = L->h, a.k = L->k, a.GF = L->GF;
   if (n_units + a.n_aux == 0) return cudaSuccess;
@@ -625,7 +665,7 @@ cudaError_t launch_gateup(const scion_layer* L, const __nv_bfloat16* /*x*/, int 
   a.bank = L->gu_bank, a.xfrag = L->xfrag;
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
   a.d = L->d, a.F = L->F, a.k = L->k, a.Gd = L->Gd, a.fmt = L->fmt;
-  a.hfrag = L->h;
+  a.hfrag = L->h, a.xexp = L->xexp;
   const int slots = min(L->E, T * L->k);
   const dim3 grid(L->F / 16, slots);
   const int gpw = (L->Gd + kGuWarps - 1) / kGuWarps;
@@ -652,10 +692,11 @@ cudaError_t launch_gateup_dense(const scion_layer* L, int T, float* out, cudaStr
   a.bank = L->gu_bank, a.xfrag = L->xfrag;
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
   a.d = L->d, a.F = L->F, a.k = L->k, a.Gd = L->Gd, a.fmt = L->fmt;
-  a.hfrag = L->h;
+  a.hfrag = L->h, a.xexp = L->xexp;
   DenseArgs b;
   b.w = L->dense_down, b.hz = L->hz, b.d = L->d, b.Kd = L->Kd, b.T = T, b.out = out;
   b.corr_b = L->desc.corr_packed ? static_cast<const uint8_t*>(L->desc.corr_b) : nullptr, b.Fs = L->Fs, b.r = L->r;
+  b.xexp = L->xexp;
   const int slots = min(L->E, T * L->k);
   const int gx = L->F / 16, dense_x = L->d / 32;
   const int dense_tiles = dense_x * ((L->Kd + kDnKc - 1) / kDnKc);
@@ -684,7 +725,7 @@ cudaError_t launch_down_routed(const scion_layer* L, int T, float* out, cudaStre
   DownArgs a;
   a.bank = L->dn_bank, a.hfrag = L->h;
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
-  a.gates = L->gates;
+  a.gates = L->gates, a.xexp = L->xexp;
   a.d = L->d, a.F = L->F, a.k = L->k, a.GF = L->GF, a.out = out;
   const int slots = min(L->E, T * L->k);
   const dim3 grid(L->d / 16, slots);
@@ -708,6 +749,7 @@ cudaError_t launch_down_dense(const scion_layer* L, int T, float* out, cudaStrea
   DenseArgs b;
   b.w = L->dense_down, b.hz = L->hz, b.d = L->d, b.Kd = L->Kd, b.T = T, b.out = out;
   b.corr_b = L->desc.corr_packed ? static_cast<const uint8_t*>(L->desc.corr_b) : nullptr, b.Fs = L->Fs, b.r = L->r;
+  b.xexp = L->xexp;
   const int nt = (T + 7) / 8;
   const dim3 g2(L->d / 32, (L->Kd + kDnKc - 1) / kDnKc);
   switch (nt) {

@@ -78,43 +78,54 @@ __device__ __forceinline__ int pos_col(int fmt, int p) {
   return 5 * (12 * half + 2 * i + (rem & 1)) + (rem >> 1);
 }
 
-// x (bf16) -> fp16 in the container's column order (PQ2_0: times the factor of its position).
-// A warp takes kXU pairs of 128-column groups per step: their coalesced 16-byte loads are all
-// issued first, then each pair goes through shared memory, where each lane gathers the columns
-// of its 8 output positions and stores 16 bytes.
-constexpr int kXU = 4;
+// x (bf16) -> fp16 x 2^s_t in the container's column order (PQ2_0: times the factor of its
+// position), s_t the token's range exponent (token_shift of its largest magnitude, written to
+// xexp).  One warp per token: the whole row's coalesced 16-byte loads are issued first (pairs of
+// 128-column groups, 16 bytes per lane), their maximum fixes s_t, then each pair goes through
+// shared memory, where each lane gathers the columns of its 8 output positions and stores 16
+// bytes.  d <= 4096 (16 pairs).
+constexpr int kXPairs = 16;
+__device__ __forceinline__ uint32_t max_mag8(uint4 v) {
+  const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu), __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+  return max(m & 0xFFFFu, m >> 16);
+}
 template <int FMT>
-__global__ void __launch_bounds__(256) x16_kernel(const __nv_bfloat16* __restrict__ x, int64_t n_groups,
-                                                  __half* __restrict__ xp) {
-  __shared__ __align__(16) __nv_bfloat16 buf[8][kXU][256];
+__global__ void __launch_bounds__(256) x16_kernel(const __nv_bfloat16* __restrict__ x, int T, int d,
+                                                  __half* __restrict__ xp, int32_t* __restrict__ xexp) {
+  __shared__ __align__(16) __nv_bfloat16 buf[8][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gl = lane >> 4, p0 = 8 * (lane & 15);  // group of the pair, first output position
-  const int64_t n_pairs = (n_groups + 1) / 2;
-  for (int64_t i0 = (int64_t(blockIdx.x) * 8 + warp) * kXU; i0 < n_pairs; i0 += int64_t(gridDim.x) * 8 * kXU) {
-    uint4 v[kXU];
-    bool ok[kXU];
+  const int G = d >> 7, n_pairs = (G + 1) / 2;
+  for (int t = blockIdx.x * 8 + warp; t < T; t += gridDim.x * 8) {
+    const __nv_bfloat16* row = x + int64_t(t) * d;
+    uint4 v[kXPairs];
+    uint32_t mx = 0;
 #pragma unroll
-    for (int u = 0; u < kXU; ++u) {
+    for (int i = 0; i < kXPairs; ++i) {
       // past the last group (an odd group count leaves the last pair half empty) nothing moves
-      ok[u] = 2 * (i0 + u) + gl < n_groups;
-      if (ok[u]) v[u] = __ldg(reinterpret_cast<const uint4*>(x + (i0 + u) * 256) + lane);
+      const bool ok = i < n_pairs && 2 * i + gl < G;
+      v[i] = ok ? __ldg(reinterpret_cast<const uint4*>(row + i * 256) + lane) : make_uint4(0u, 0u, 0u, 0u);
+      mx = max(mx, max_mag8(v[i]));
     }
+    const int sh = token_shift(__reduce_max_sync(0xffffffffu, mx));
+    if (lane == 0) xexp[t] = sh;
+    const float xs = pow2i(sh);
+    __half* orow = xp + int64_t(t) * d;
 #pragma unroll
-    for (int u = 0; u < kXU; ++u)
-      if (ok[u]) *reinterpret_cast<uint4*>(&buf[warp][u][8 * lane]) = v[u];
-    __syncwarp();
-#pragma unroll
-    for (int u = 0; u < kXU; ++u) {
+    for (int i = 0; i < kXPairs; ++i) {
+      if (i >= n_pairs) break;
+      __syncwarp();
+      *reinterpret_cast<uint4*>(&buf[warp][8 * lane]) = v[i];
+      __syncwarp();
       __align__(16) __half o[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int p = p0 + e;
-        const float f = __bfloat162float(buf[warp][u][128 * gl + pos_col(FMT, p)]);
+        const float f = __bfloat162float(buf[warp][128 * gl + pos_col(FMT, p)]) * xs;
         o[e] = __float2half_rn(FMT == SCION_PQ2_0 ? f * pq2_pos_scale(p) : f);
       }
-      if (ok[u]) reinterpret_cast<uint4*>(xp + (i0 + u) * 256)[lane] = *reinterpret_cast<const uint4*>(o);
+      if (2 * i + gl < G) reinterpret_cast<uint4*>(orow + i * 256)[lane] = *reinterpret_cast<const uint4*>(o);
     }
-    __syncwarp();
   }
 }
 
@@ -172,6 +183,8 @@ struct DenseParams {
   __half* hz;     int ld_hz;
   float* out;     int ld_out;
   const float* resid;  // kEpiStore: added to the stored value (same layout as out; may equal out)
+  const int32_t* xexp;  // range exponent s_t of each token: hz rows are stored times 2^hz_shift(s_t)
+  int has_corr;         // the layer has a correction (hz_shift's choice)
   int* err;
 };
 
@@ -321,6 +334,17 @@ __global__ void __launch_bounds__(kThreads, 1) dense_gemm_kernel(const __grid_co
         if (!rok) continue;
         const int n16 = min(16, nt - c * 16);
         const int64_t t0 = dt.tok0 + c * 16;
+        // per-token factors of the hz rows (see hz_shift): stored times 2^p, read back times 2^-p;
+        // the units against x16 (ternary correction A) accumulate x 2^s_t
+        float tf[16];
+        if (u.epi != kEpiLogits) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int sh = i < n16 ? p.xexp[t0 + i] : 0;
+            const int e = hz_shift(sh, p.has_corr);
+            tf[i] = pow2i(u.epi == kEpiStore ? -e : (u.b16 ? e - sh : e));
+          }
+        }
         if (u.epi == kEpiLogits) {
           float* dst = p.logits + t0 * p.ld_logits + col;
 #pragma unroll
@@ -332,18 +356,18 @@ __global__ void __launch_bounds__(kThreads, 1) dense_gemm_kernel(const __grid_co
             const float* rs = p.resid + t0 * p.ld_out + col;
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              if (i < n16) dst[int64_t(i) * p.ld_out] = v0[i] + rs[int64_t(i) * p.ld_out];
+              if (i < n16) dst[int64_t(i) * p.ld_out] = v0[i] * tf[i] + rs[int64_t(i) * p.ld_out];
           } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              if (i < n16) dst[int64_t(i) * p.ld_out] = v0[i];
+              if (i < n16) dst[int64_t(i) * p.ld_out] = v0[i] * tf[i];
           }
         } else {
           __half* dst = p.hz + t0 * p.ld_hz + col;
           const bool sw = u.epi == kEpiSwiglu;
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            if (i < n16) dst[int64_t(i) * p.ld_hz] = __float2half_rn(sw ? silu_f(v0[i]) * v1[i] : v0[i]);
+            if (i < n16) dst[int64_t(i) * p.ld_hz] = __float2half_rn((sw ? silu_f(v0[i]) * v1[i] : v0[i]) * tf[i]);
         }
       }
       // accumulator drained: hand it back to the MMA thread
@@ -390,7 +414,8 @@ struct TernParams {
   const int32_t *counts, *offsets, *perm;
   const float* gates;
   int k;
-  __half* h;  int F;     // gate/up output
+  const int32_t* pexp;   // range exponent of the token of each routed position (B rows are x 2^s)
+  __half* h;  int F;     // gate/up output, h 2^(2 s)
   __half* y;  int d;     // down output: one fp16 row per routed (token, slot), [T*k][d], gates applied by the combine
   int* err;
 };
@@ -747,7 +772,10 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
           __half* dst = p.h + (pos0 + n0) * p.F + int64_t(rt) * kBM + pcol;
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            if (n0 + i < nn) dst[int64_t(i) * p.F] = __float2half_rn(silu_f(v0[i]) * v1[i] * hscale);
+            if (n0 + i < nn) {
+              const int sh = p.pexp[pos0 + n0 + i];
+              dst[int64_t(i) * p.F] = __float2half_rn(silu_f(v0[i] * pow2i(-sh)) * (v1[i] * pow2i(sh)) * hscale);
+            }
         } else {
           __half* dst = p.y + (pos0 + n0) * p.d + int64_t(rt) * kBM + row;
 #pragma unroll
@@ -851,7 +879,9 @@ __global__ void __launch_bounds__(kScanThreads) group_scan_kernel(const int32_t*
 constexpr int kScatterMaxPerThread = 8;
 __global__ void __launch_bounds__(256) group_scatter_kernel(const int32_t* __restrict__ ids, int n, int E, int ept,
                                                             int32_t* __restrict__ cursor, int32_t* __restrict__ perm,
-                                                            int32_t* __restrict__ inv) {
+                                                            int32_t* __restrict__ inv, int k,
+                                                            const int32_t* __restrict__ xexp,
+                                                            int32_t* __restrict__ pexp) {
   extern __shared__ int32_t sh[];  // cnt[E], base[E]
   int32_t *cnt = sh, *base = sh + E;
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
@@ -874,6 +904,7 @@ __global__ void __launch_bounds__(256) group_scatter_kernel(const int32_t* __res
     const int i = i0 + 256 * j, pos = base[id[j]] + local[j];
     perm[pos] = i;
     inv[i] = pos;
+    pexp[pos] = xexp[i / k];
   }
 }
 
@@ -983,10 +1014,11 @@ cudaError_t configure_prefill_kernels() {
 // residual (a layer without shared expert and correction), or zero.  One CTA per token.
 __global__ void __launch_bounds__(256) combine_kernel(const __half* __restrict__ y, const int32_t* __restrict__ inv,
                                                      const float* __restrict__ gates, int k, int d,
-                                                     const float* base, float* out) {
+                                                     const int32_t* __restrict__ xexp, const float* base, float* out) {
   const int t = blockIdx.x;
   const int32_t* iv = inv + int64_t(t) * k;
   const float* gt = gates + int64_t(t) * k;
+  const float ys = pow2i(-2 * xexp[t]);  // the rows of y are of the hidden h 2^(2 s_t)
   // each thread: 8 columns (one 16-byte load per routed row); the k rows' loads are issued in
   // batches of 8 before any of them is used, so each thread keeps 8 loads in flight
   for (int c8 = threadIdx.x; c8 < d / 8; c8 += blockDim.x) {
@@ -1007,7 +1039,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const __half* __restrict__
       for (int j = 0; j < 8; ++j) {
         if (j0 + j < k) {
           raw[j] = reinterpret_cast<const uint4*>(y + int64_t(iv[j0 + j]) * d)[c8];
-          g[j] = gt[j0 + j];
+          g[j] = gt[j0 + j] * ys;
         } else {
           raw[j] = make_uint4(0u, 0u, 0u, 0u);
           g[j] = 0.f;
@@ -1083,13 +1115,11 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
   const PrefillState& P = *L->pre;
   switch (stage) {
     case SCION_STAGE_X16: {
-      const int64_t n = int64_t(T) * L->d;
-      const int64_t groups = n / 128, pairs = (groups + 1) / 2;
-      const unsigned grid = unsigned(std::min((pairs + 8 * kXU - 1) / (8 * kXU), int64_t(num_sms()) * 8));
+      const unsigned grid = unsigned(std::min((T + 7) / 8, num_sms() * 8));
       if (L->fmt == SCION_PQ2_0)
-        x16_kernel<SCION_PQ2_0><<<grid, 256, 0, s>>>(x, groups, P.x16);
+        x16_kernel<SCION_PQ2_0><<<grid, 256, 0, s>>>(x, T, L->d, P.x16, P.xexp);
       else
-        x16_kernel<SCION_PTQ1_0><<<grid, 256, 0, s>>>(x, groups, P.x16);
+        x16_kernel<SCION_PTQ1_0><<<grid, 256, 0, s>>>(x, T, L->d, P.x16, P.xexp);
       return cudaGetLastError();
     }
     case SCION_STAGE_XPROJ: {
@@ -1102,6 +1132,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       dp.n_units2 = (L->desc.router_fp32 ? 0 : (L->E + 127) / 128) + (L->Fs + 127) / 128;
       dp.logits = P.logits, dp.ld_logits = L->E, dp.hz = P.hz, dp.ld_hz = L->Kd, dp.out = nullptr, dp.ld_out = 0;
       dp.resid = nullptr;
+      dp.xexp = P.xexp, dp.has_corr = L->r > 0;
       dp.err = L->err;
       if (L->desc.corr_packed) dp.b16 = P.x16_map;
       dense_gemm_kernel<<<dense_grid(dp), kThreads, kDenseSmem, s>>>(dp);
@@ -1131,7 +1162,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
                                                   tile_width(int64_t(T) * L->k, L->E));
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
       group_scatter_kernel<<<(n + 256 * ept - 1) / (256 * ept), 256, 2 * sizeof(int32_t) * L->E, s>>>(
-          P.ids, n, L->E, ept, P.cursor, P.perm, P.inv);
+          P.ids, n, L->E, ept, P.cursor, P.perm, P.inv, L->k, P.xexp, P.pexp);
       return cudaGetLastError();
     }
     case SCION_STAGE_GATEUP: {
@@ -1141,6 +1172,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       const bool mid = tile_width(int64_t(T) * L->k, L->E) == kBN3;
       tp.tiles = static_cast<const TernTile*>(P.tiles), tp.n_tiles = P.n_tiles;
       tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gates = P.gates, tp.k = L->k;
+      tp.pexp = P.pexp;
       tp.h = P.h, tp.F = L->F, tp.y = nullptr, tp.d = L->d, tp.err = L->err;
       const dim3 grid(num_sms());
       if (L->fmt == SCION_PQ2_0 && mid)
@@ -1154,7 +1186,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       return cudaGetLastError();
     }
     case SCION_STAGE_COMBINE: {
-      combine_kernel<<<T, 256, 0, s>>>(P.y, P.inv, P.gates, L->k, L->d, P.n_dunits > 0 ? out : resid, out);
+      combine_kernel<<<T, 256, 0, s>>>(P.y, P.inv, P.gates, L->k, L->d, P.xexp, P.n_dunits > 0 ? out : resid, out);
       return cudaGetLastError();
     }
     case SCION_STAGE_DOWN_DENSE: {
@@ -1166,6 +1198,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       dp.n_units = P.n_dunits, dp.n_units2 = 0;
       dp.logits = nullptr, dp.ld_logits = 0, dp.hz = nullptr, dp.ld_hz = 0, dp.out = out, dp.ld_out = L->d;
       dp.resid = resid;
+      dp.xexp = P.xexp, dp.has_corr = L->r > 0;
       dp.err = L->err;
       dense_gemm_kernel<<<dense_grid(dp), kThreads, kDenseSmem, s>>>(dp);
       return cudaGetLastError();
@@ -1177,6 +1210,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       const int wd = tile_width(int64_t(T) * L->k, L->E);
       tp.tiles = static_cast<const TernTile*>(P.tiles), tp.n_tiles = P.n_tiles;
       tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gates = P.gates, tp.k = L->k;
+      tp.pexp = P.pexp;
       tp.h = nullptr, tp.F = L->F, tp.y = P.y, tp.d = L->d, tp.err = L->err;
       if (make_tmap_2d(&tp.bmap, P.h, 0, int64_t(T) * L->k, L->F, wd) != SCION_OK)
         return cudaErrorInvalidValue;

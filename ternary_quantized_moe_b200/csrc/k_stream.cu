@@ -36,7 +36,9 @@ struct StageHdr {
   int ng;     // 128-column groups in this stage (1..GPS)
   int pos[kTok];     // routed positions of the pass's tokens (last stage only)
   int orow[kTok];    // output token row (entry / k)
-  float gate[kTok];  // gate of the entry
+  float gate[kTok];  // gate of the entry (down: times 2^(-2 s_t), the hidden being h 2^(2 s_t))
+  float xdn[kTok];   // gate/up: 2^-s_t and 2^s_t of the token's range exponent (the sums are of x 2^s_t)
+  float xup[kTok];
 };
 static_assert(sizeof(StageHdr) <= kHdr, "stage header");
 
@@ -47,6 +49,7 @@ struct StreamArgs {
   const int4* slot_info;
   const int32_t *n_active, *perm;
   const float* gperm;  // gate of each routed position
+  const int32_t* xexp; // range exponent s_t of each token
   int G, R, k, F, d, fmt;
   __half* hfrag;  // gate/up output
   float* out;     // down output
@@ -55,7 +58,7 @@ struct StreamArgs {
 
 struct TokInfo {
   int pos, brow, orow;
-  float gate;
+  float gate, xdn, xup;
 };
 
 // Groups per stage: two for the gate/up bank (each group holds both matrices), four for down.
@@ -238,11 +241,13 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
     const int n_items = *a.n_active * RB;
     auto slot_rec = [&](int item) { return item < n_items ? a.slot_info[item / RB] : make_int4(0, 0, 0, 0); };
     auto tok_info = [&](int4 si, int pc) {
-      TokInfo t{0, 0, 0, 0.f};
+      TokInfo t{0, 0, 0, 0.f, 1.f, 1.f};
       if (lane < min(kTok, si.z - pc)) {
         t.pos = si.y + pc + lane;
         t.orow = a.perm[t.pos] / a.k;
-        t.gate = a.gperm[t.pos];
+        const int sh = a.xexp[t.orow];
+        t.gate = a.gperm[t.pos] * pow2i(-2 * sh);
+        t.xdn = pow2i(-sh), t.xup = pow2i(sh);
         t.brow = NMAT == 2 ? t.orow : t.pos;
       }
       return t;
@@ -284,7 +289,8 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
             for (int i = 0; i < kTok; ++i) {
               const int pos = __shfl_sync(0xffffffffu, tk.pos, i), orow = __shfl_sync(0xffffffffu, tk.orow, i);
               const float gate = __shfl_sync(0xffffffffu, tk.gate, i);
-              if (lane == 0) hd->pos[i] = pos, hd->orow[i] = orow, hd->gate[i] = gate;
+              const float xdn = __shfl_sync(0xffffffffu, tk.xdn, i), xup = __shfl_sync(0xffffffffu, tk.xup, i);
+              if (lane == 0) hd->pos[i] = pos, hd->orow[i] = orow, hd->gate[i] = gate, hd->xdn[i] = xdn, hd->xup[i] = xup;
             }
           }
           if (lane == 0) {
@@ -369,7 +375,7 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
         const int row = warp * 16 + (lane >> 2) + 8 * (i >> 1);
         const int tcol = 2 * c + (i & 1);
         if constexpr (NMAT == 2) {
-          const float h = silu_f(acc[0][i] * unit) * (acc[1][i] * unit) * hsc[i >> 1];
+          const float h = silu_f(acc[0][i] * unit * hd->xdn[tcol]) * (acc[1][i] * unit * hd->xup[tcol]) * hsc[i >> 1];
           const __half h16 = __float2half_rn(h);
           if (tcol < nn) a.hfrag[(int64_t(hd->pos[tcol]) * (a.F >> 7) + rb) * SCION_BROW + hpos[i >> 1]] = h16;
           if (FMT == SCION_PQ2_0) hs[i & 1] += __half2float(h16) * hinv[i >> 1];
@@ -452,7 +458,7 @@ cudaError_t launch_stream_gateup(const scion_layer* L, int T, cudaStream_t s) {
   StreamArgs a;
   a.bank = L->gu_bank, a.bsrc = L->xfrag, a.bld = L->Gd;
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
-  a.gperm = L->gperm, a.G = L->Gd, a.R = L->F, a.k = L->k, a.F = L->F, a.d = L->d, a.fmt = L->fmt;
+  a.gperm = L->gperm, a.xexp = L->xexp, a.G = L->Gd, a.R = L->F, a.k = L->k, a.F = L->F, a.d = L->d, a.fmt = L->fmt;
   a.hfrag = L->h, a.out = nullptr, a.err = L->err;
   const int max_items = min(L->E, T * L->k) * (L->F / 128);
   if (L->fmt == SCION_PQ2_0) return launch_stream<SCION_PQ2_0, 2>(a, max_items, s);
@@ -463,7 +469,7 @@ cudaError_t launch_stream_down(const scion_layer* L, int T, float* out, cudaStre
   StreamArgs a;
   a.bank = L->dn_bank, a.bsrc = L->h, a.bld = L->GF;
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
-  a.gperm = L->gperm, a.G = L->GF, a.R = L->d, a.k = L->k, a.F = L->F, a.d = L->d, a.fmt = L->fmt;
+  a.gperm = L->gperm, a.xexp = L->xexp, a.G = L->GF, a.R = L->d, a.k = L->k, a.F = L->F, a.d = L->d, a.fmt = L->fmt;
   a.hfrag = nullptr, a.out = out, a.err = L->err;
   const int max_items = min(L->E, T * L->k) * (L->d / 128);
   if (L->fmt == SCION_PQ2_0) return launch_stream<SCION_PQ2_0, 1>(a, max_items, s);

@@ -45,7 +45,7 @@ void free_layer(scion_layer* L) {
   void* ptrs[] = {L->gu_bank, L->dn_bank,  L->dense_down, L->xunits,  L->logits,    L->ids,       L->gates,
                   L->counts,  L->offsets,  L->perm,       L->active,  L->n_active,  L->h,         L->hz,
                   L->xfrag,   L->x_stage, L->out_stage, L->bad,       L->err,
-                  L->slot_info, L->gperm, L->route_done};
+                  L->slot_info, L->gperm, L->route_done, L->xexp};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   if (L->side) cudaStreamDestroy(L->side);
@@ -54,7 +54,7 @@ void free_layer(scion_layer* L) {
   if (L->pre) {
     scion::PrefillState* P = L->pre;
     void* pp[] = {P->xunits, P->dunits, P->logits, P->ids, P->gates, P->counts, P->offsets, P->perm, P->inv,
-                  P->y, P->tiles, P->n_tiles, P->x16, P->h, P->hz, P->cursor, P->corr_a16};
+                  P->y, P->tiles, P->n_tiles, P->x16, P->h, P->hz, P->cursor, P->corr_a16, P->xexp, P->pexp};
     for (void* p : pp)
       if (p) cudaFree(p);
     delete P;
@@ -86,6 +86,8 @@ int create_prefill(scion_layer* L, cudaStream_t s) {
   PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->tiles), scion::prefill_tile_bytes() * max_tiles));
   PTRY(dev_alloc(L, &P->n_tiles, sizeof(int32_t)));
   PTRY(dev_alloc(L, &P->x16, sizeof(__half) * T * L->d));
+  PTRY(dev_alloc(L, &P->xexp, sizeof(int32_t) * T));
+  PTRY(dev_alloc(L, &P->pexp, sizeof(int32_t) * Tk));
   PTRY(dev_alloc(L, &P->h, sizeof(__half) * Tk * L->F));
   PTRY(dev_alloc(L, &P->hz, sizeof(__half) * T * (L->Kd ? L->Kd : 64)));
   PTRY(cudaMemsetAsync(P->hz, 0, sizeof(__half) * T * (L->Kd ? L->Kd : 64), s));
@@ -335,6 +337,7 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   SCION_TRY(dev_alloc(L, &L->h, sizeof(__half) * TD * L->k * L->GF * SCION_BROW));
   SCION_TRY(dev_alloc(L, &L->hz, sizeof(__half) * TD * (L->Kd ? L->Kd : 1)));
   SCION_TRY(dev_alloc(L, &L->xfrag, sizeof(__half) * TD * L->Gd * SCION_BROW));
+  SCION_TRY(dev_alloc(L, &L->xexp, sizeof(int32_t) * TD));
   SCION_TRY(dev_alloc(L, &L->x_stage, sizeof(__nv_bfloat16) * size_t(max_tokens) * L->d));
   SCION_TRY(dev_alloc(L, &L->out_stage, sizeof(float) * size_t(max_tokens) * L->d));
   SCION_TRY(dev_alloc(L, &L->bad, sizeof(int64_t)));

@@ -80,7 +80,9 @@ struct PrefillState {
   __half* y;            // [maxT*k][d] expert down outputs in fp16 (gate not yet applied), one row per routed entry
   void* tiles;          // token tiles of the ternary GEMMs (128 or 160 tokens), [maxT*k/128 + E]
   int32_t* n_tiles;
-  __half* x16;          // [maxT][d]   x in the container column order (fp16)
+  __half* x16;          // [maxT][d]   x 2^s_t in the container column order (fp16)
+  int32_t* xexp;        // [maxT] per-token range exponent s_t (see token_shift)
+  int32_t* pexp;        // [maxT*k] s_t of the token of each routed position
   __half* h;            // [maxT*k][F] expert SwiGLU hidden, container column order
   __half* hz;           // [maxT][Kd]
 };
@@ -116,6 +118,7 @@ struct scion_layer {
   __half* h;         // [TDEC*k][GF][SCION_BROW] fragment order + group-sum tails
   __half* hz;        // [TDEC][Kd] (pad columns stay 0)
   __half* xfrag;     // [TDEC][Gd][SCION_BROW] x in fragment order (fp16) + group-sum tails
+  int32_t* xexp;     // [TDEC] per-token range exponent s_t (see token_shift)
   void* x_stage;     // [max_tokens][d] bf16 (host-buffer forward)
   float* out_stage;  // [max_tokens][d]
   int64_t* bad;      // [1] invalid-code counter used at create
@@ -268,12 +271,55 @@ __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ uint32_t ld_dsmem_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
   // (a & mask) | magic in one LOP3
   uint32_t r;
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;\n" : "=r"(r) : "r"(a), "r"(mask), "r"(magic));
   return r;
 }
+
+// ---------------------------------------------------- per-token range scaling
+// The expert GEMMs and the stored hidden values run in fp16, whose range (2^-14 .. 65504 for
+// full precision) is far narrower than bf16's.  Every token t gets an exponent s_t from the
+// largest magnitude of its activations: s_t = 0 while max|x_t| lies in [2^-3, 2^6) (the usual
+// case: nothing changes), otherwise s_t = 2 - floor(log2 max|x_t|) clamped to [-40, 40], which
+// brings max|x_t 2^s_t| into [4, 8).  All factors are powers of two, so every scaling is exact:
+//   expert input     x 2^s                  (fp16 operand of the expert gate/up GEMMs)
+//   expert hidden    h 2^(2s)               (silu(g 2^-s) * (u 2^s) from the scaled sums g, u;
+//                                            |silu(y)| <= |y| keeps it within the range of the
+//                                            hidden of the scaled token)
+//   expert output    gate 2^(-2s) y         (applied where the weighted sum enters out)
+//   shared / z rows  hz 2^p, p = s when the layer has a correction and s > 0, else 2s; the
+//                    dense down projection multiplies its output by 2^-p.  (The shared hidden
+//                    grows like x^2 and z like x: for s < 0 the x^2 terms dominate the output,
+//                    for s > 0 the correction does, so the term whose stored value may leave the
+//                    fp16 range is the one too small to matter.)
+constexpr int kShiftLo = -3, kShiftHi = 5, kShiftTarget = 2, kShiftMax = 40;
+// s_t from the largest bf16 magnitude of the token (its bit pattern with the sign cleared)
+__host__ __device__ __forceinline__ int token_shift(uint32_t max_mag_bits) {
+  if (max_mag_bits == 0) return 0;
+  const int e = int(max_mag_bits >> 7) - 127;  // floor(log2 |x|) for normal values; subnormals -> -127
+  if (e >= kShiftLo && e <= kShiftHi) return 0;
+  const int s = kShiftTarget - e;
+  return s < -kShiftMax ? -kShiftMax : (s > kShiftMax ? kShiftMax : s);
+}
+// 2^n as fp32 for |n| <= 126, built from its exponent field
+__host__ __device__ __forceinline__ float pow2i(int n) {
+  union {
+    uint32_t u;
+    float f;
+  } v;
+  v.u = uint32_t(n + 127) << 23;
+  return v.f;
+}
+// exponent p of the shared / z rows' factor (see above); has_corr = the layer has a correction
+__host__ __device__ __forceinline__ int hz_shift(int s, int has_corr) { return (has_corr && s > 0) ? s : 2 * s; }
 
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }

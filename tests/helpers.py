@@ -139,3 +139,40 @@ def device_layer(cfg: synth.Config, L: dict, banks: dict, max_tokens: int, dev="
         corr_a=torch.from_numpy(packed_corr[0]).to(dev) if packed_corr else opt("corr_a"),
         corr_b=torch.from_numpy(packed_corr[1]).to(dev) if packed_corr else opt("corr_b"),
         corr_packed=1 if packed_corr else 0, norm_topk=norm_topk, max_tokens=max_tokens)
+
+
+def range_mix(cfg: synth.Config, layer: oracle.OracleLayer, x: np.ndarray, seed: int = 4711) -> np.ndarray:
+    """Activations far from N(0, 1), built from margin-filtered tokens x (bf16 bits): token t gets
+    kind (t + 1) % 5 --
+      0  unchanged (N(0, 1));
+      1  four channels replaced by outliers of magnitude 1e2 .. 3e4 (log-uniform, random sign);
+      2  the whole token times 2^-20 (values near 1e-6);
+      3  the whole token times 2^8 (rms 256, max near 1e3);
+      4  a hundred channels replaced by values near 1e-6.
+    Power-of-two scalings are exact in bf16 and leave the fp64 logits scaled by the same factor,
+    so those tokens keep their (relative) top-k margin; the outlier tokens are redrawn until their
+    fp64 top-k gap is at least the absolute margin."""
+    rng = np.random.default_rng(seed)
+    xf = bf16(x).astype(np.float32)
+    out = xf.copy()
+    for t in range(x.shape[0]):
+        kind = (t + 1) % 5
+        if kind == 1:
+            for _ in range(50):
+                row = xf[t].copy()
+                ch = rng.choice(cfg.d, 4, replace=False)
+                row[ch] = (np.exp(rng.uniform(np.log(1e2), np.log(3e4), 4)) * rng.choice([-1.0, 1.0], 4))
+                logits, _, _ = oracle.route(layer, synth.to_bf16_bits(row[None]))
+                if topk_gap(logits, cfg.top_k)[0] >= TOPK_MARGIN:
+                    out[t] = row
+                    break
+            else:
+                raise RuntimeError("no outlier token with the top-k margin")
+        elif kind == 2:
+            out[t] = xf[t] * np.float32(2.0 ** -20)
+        elif kind == 3:
+            out[t] = xf[t] * np.float32(2.0 ** 8)
+        elif kind == 4:
+            ch = rng.choice(cfg.d, 100, replace=False)
+            out[t, ch] = rng.standard_normal(100).astype(np.float32) * np.float32(1e-6)
+    return synth.to_bf16_bits(out)

@@ -7,7 +7,7 @@ import pytest
 
 import oracle
 from tests.helpers import (TOPK_MARGIN, bf16, check_output, device_layer, oracle_layer_packed, packed_banks,
-                           packed_correction, topk_gap, u16_to_dev, with_margin)
+                           packed_correction, range_mix, topk_gap, u16_to_dev, with_margin)
 from workloads import synth
 
 torch = pytest.importorskip("torch")
@@ -344,6 +344,32 @@ def test_forward_decode_many_experts(E, k, T):
     check_output(got, ref)
 
 
+@pytest.mark.parametrize("shape", ["a3b", "flashnext"])
+@pytest.mark.parametrize("T", [1, 13, 64, 300])
+def test_forward_activation_range(shape, T):
+    """Activations far outside N(0, 1) -- outlier channels up to 3e4, whole tokens near 1e-6 or
+    scaled by 256, tiny channels inside ordinary tokens -- through the decode kernels (T <= 64:
+    split-K and ring passes) and the tensor-core path (T = 300), with the 35B-A3B-class (d 2048,
+    ffn 512, PQ2_0, shared expert, rank 512) and FlashNext-class (d 3072, ffn 768, PTQ1_0) layer
+    widths (32 experts).  Routing bit-exact, output within the block tolerance per token."""
+    if shape == "a3b":
+        cfg = small("ra", synth.PQ2_0, False, E=32, k=8, d=2048, F=512, Fs=512, r=512)
+    else:
+        cfg = small("rf", synth.PTQ1_0, False, E=32, k=10, d=3072, F=768, Fs=768, r=512)
+    L, banks, ol, x = _case(cfg, T)
+    x = range_mix(cfg, ol, x)
+    layer = device_layer(cfg, L, banks, max(T, 64))
+    del L, banks
+    got, dbg = run_forward(layer, x, T, debug=True, E=cfg.n_experts, k=cfg.top_k, F=cfg.ffn,
+                           Kdense=cfg.shared_ffn + cfg.rank)
+    assert tq.scion_layer_check(layer) == 0
+    assert np.isfinite(got).all()
+    _, ids, _ = oracle.route(ol, x)
+    np.testing.assert_array_equal(np.sort(dbg["ids"], 1), np.sort(ids, 1))
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
+
+
 @pytest.mark.parametrize("T,max_tokens", [(13, 64), (200, 200)])
 def test_debug_route_matches_oracle(T, max_tokens):
     """scion_debug_route (the routing alone): ids as sets per token, offsets and the grouping
@@ -438,6 +464,13 @@ def test_full_size_decode(name):
         _check_routing(cfg, dbg, ol, x, T)
         ref, _, _ = oracle.forward(ol, x)
         check_output(got, ref)
+    # the largest batch again with activations far from N(0, 1) (outliers, tiny and large tokens)
+    T = max(cfg.tokens)
+    x = range_mix(cfg, ol, with_margin(cfg, ol, synth.x_host(cfg, T, 1)))
+    got, _ = run_forward(layer, x, T)
+    assert np.isfinite(got).all()
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
 
 
 @pytest.mark.slow
