@@ -71,7 +71,11 @@ def parse():
     ap.add_argument("--packed-corr", action="store_true",
                     help="ternary correction factors (PQ2_0 blocks) instead of the workload's bf16 ones")
     ap.add_argument("--stream-min-tokens", type=int, default=0,
-                    help="decode batches of at least this many tokens use the bulk-copy ring expert kernels")
+                    help="decode batches of at least this many tokens use the persistent expert kernels")
+    ap.add_argument("--decode-tc", type=int, default=1, choices=[0, 1],
+                    help="1: tcgen05 expert GEMMs for those batches, 0: the mma.sync bulk-copy ring kernels")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="prefill: per-entry rows summed in slot order instead of fp32 reductions into out")
     return ap.parse_args()
 
 
@@ -305,6 +309,8 @@ def workload_config(cfg, args, n_layers=None, weight_bytes=None):
     c = {"workload": cfg.name, "d": cfg.d, "experts": cfg.n_experts, "top_k": cfg.top_k, "ffn": cfg.ffn,
          "shared_ffn": cfg.shared_ffn, "rank": cfg.rank, "format": "PQ2_0" if cfg.fmt == 0 else "PTQ1_0",
          "correction": "PQ2_0 blocks" if args.packed_corr else "bf16", "batches": list(cfg.tokens),
+         "decode_expert_kernels": "tcgen05" if args.decode_tc else "mma.sync ring",
+         "prefill_combine": "slot-order rows" if args.deterministic else "fp32 reductions",
          "tokens_per_step": sum(cfg.tokens)}
     if cfg.zipf_s is not None:
         c["router_load"] = "Zipf(%.1f) over a seeded permutation of the experts" % cfg.zipf_s
@@ -345,6 +351,9 @@ def build_layers(cfg, args, dev, n_layers, max_T):
         del banks, W
         if args.stream_min_tokens:
             tq.scion_layer_set_option(layers[-1], tq.SCION_OPT_STREAM_MIN_TOKENS, args.stream_min_tokens)
+        tq.scion_layer_set_option(layers[-1], tq.SCION_OPT_DECODE_TC, args.decode_tc)
+        if args.deterministic:
+            tq.scion_layer_set_option(layers[-1], tq.SCION_OPT_DETERMINISTIC, 1)
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     return layers

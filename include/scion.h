@@ -219,12 +219,18 @@ int scion_moe_forward_residual(const void* x, int T, const scion_layer* layer, c
 
 /* Tuning options of a layer (scion_layer_set_option).
  *  SCION_OPT_STREAM_MIN_TOKENS (default 16): batches of at least this many tokens (and at
- *    most 64) run the expert GEMVs on the persistent kernels fed by a bulk-copy ring (128
- *    expert rows per work item); smaller batches split K over the warps of one CTA per 16
- *    rows, which spreads the few active experts over more SMs.
- *    Both give the same result up to fp32 summation order.
+ *    most 64) run the expert GEMMs on persistent kernels (128 expert rows per work item);
+ *    smaller batches split K over the warps of one CTA per 16 rows, which spreads the few
+ *    active experts over more SMs.
+ *  SCION_OPT_DECODE_TC (default 1): those persistent kernels are the tcgen05 grouped GEMMs
+ *    (codes expanded into tensor memory, one tile per active expert, the down projection adding
+ *    its gate-weighted rows into out); 0 selects the mma.sync kernels fed by a bulk-copy ring.
+ *  SCION_OPT_DETERMINISTIC (default 0): 1 makes batches above 64 tokens bit-reproducible: the
+ *    down projection writes one fp16 row per routed entry and a combine kernel sums each token's
+ *    rows in slot order, instead of fp32 reductions into out in whatever order they land.
+ *    All settings give the same result up to fp32 summation order.
  * EINVAL for an unknown option or an out-of-range value. */
-enum { SCION_OPT_STREAM_MIN_TOKENS = 1 };
+enum { SCION_OPT_STREAM_MIN_TOKENS = 1, SCION_OPT_DECODE_TC = 2, SCION_OPT_DETERMINISTIC = 3 };
 int scion_layer_set_option(scion_layer* layer, int option, int value);
 
 /* Waits for `stream`, then returns the layer's device status word and clears it:

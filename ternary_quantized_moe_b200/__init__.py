@@ -26,7 +26,8 @@ __all__ = [
     "scion_layer_create", "scion_layer_destroy", "scion_layer_device_bytes", "scion_moe_forward",
     "scion_moe_forward_host", "scion_moe_forward_debug", "Layer", "library_path", "EXPORTS",
     "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "STAGES", "scion_layer_check",
-    "scion_router_logits_static", "scion_layer_set_option", "SCION_OPT_STREAM_MIN_TOKENS",
+    "scion_router_logits_static", "scion_layer_set_option", "SCION_OPT_STREAM_MIN_TOKENS", "SCION_OPT_DECODE_TC",
+    "SCION_OPT_DETERMINISTIC",
     "scion_moe_forward_residual", "scion_quantize_device", "SCION_QUANT_ABSMEAN", "SCION_QUANT_LLOYD",
     "scion_selftest_bounded_wait", "scion_debug_route",
 ]
@@ -50,7 +51,7 @@ EXPORTS = (
     "scion_selftest_bounded_wait", "scion_debug_route",
 )
 SCION_QUANT_ABSMEAN, SCION_QUANT_LLOYD = 0, 1
-SCION_OPT_STREAM_MIN_TOKENS = 1
+SCION_OPT_STREAM_MIN_TOKENS, SCION_OPT_DECODE_TC, SCION_OPT_DETERMINISTIC = 1, 2, 3
 STAGES = ("router_f32", "xproj", "route", "gateup", "down_routed", "down_dense", "x16", "combine")
 
 

@@ -22,6 +22,7 @@
 #include <math.h>
 
 #include "scion_internal.cuh"
+#include "tc_order.cuh"
 #include "tern_tile.cuh"
 
 namespace scion {
@@ -41,6 +42,7 @@ struct XProjArgs {
   __half* hz;
   __half* xfrag;  // [T][d/128][SCION_BROW] fp16 x 2^s_t in fragment order + group sums
   int32_t* xexp;  // [T] range exponent s_t of each token (token_shift), written by the aux CTAs
+  __half* x16;    // non-null: the aux CTAs write x 2^s_t here, [T][d] in the tcgen05 column order
   __half* h;      // [T*k][F/128][SCION_BROW] expert hidden: group-sum tails zeroed here
   int k, GF;
   const uint8_t* corr_blocks;  // ternary correction A (PQ2_0 blocks [r][d/128]) or nullptr (bf16 corr_a)
@@ -68,24 +70,40 @@ __device__ __forceinline__ uint32_t max_mag8(uint4 v) {
 }
 
 __device__ __forceinline__ void xproj_aux(const XProjArgs& a, int aux, int n_aux) {
-  const int Gd = a.d >> 7;
+  const int Gd = a.d >> 7, n_pairs = (Gd + 1) >> 1;
   const int lane = threadIdx.x & 31;
   const int gw = aux * (kXThreads / 32) + (threadIdx.x >> 5), nw = n_aux * (kXThreads / 32);
-  // one warp per token: the row's largest magnitude fixes its range exponent s_t, then x 2^s_t
-  // goes to the fragment order, two groups per step (16 lanes per group, 8 elements per lane);
-  // the 16 lanes of a group sum its B * 4^f for the row tail
-  for (int t = gw; t < a.T; t += nw) {
+  // Warps share the tokens out (wpt warps per token, each a slice of its pairs of 128-column
+  // groups).  Each warp finds its token's largest magnitude over the whole row (all loads in
+  // flight at once), which fixes the range exponent s_t, then writes x 2^s_t for its pairs:
+  // 16 lanes per group, 8 elements per lane, in the tcgen05 order (a.x16) or the fragment order
+  // with the group sums of B * 4^f in the row tails.
+  const int wpt = max(1, nw / max(1, a.T));
+  for (int job = gw; job < a.T * wpt; job += nw) {
+    const int t = job / wpt, slice = job % wpt;
     const __nv_bfloat16* row = a.x + int64_t(t) * a.d;
     uint32_t mx = 0;
+#pragma unroll 4
     for (int i = lane; i < a.d / 8; i += 32) mx = max(mx, max_mag8(*reinterpret_cast<const uint4*>(row + 8 * i)));
     const int sh = token_shift(__reduce_max_sync(0xffffffffu, mx));
-    if (lane == 0) a.xexp[t] = sh;
+    if (lane == 0 && slice == 0) a.xexp[t] = sh;
     const float xs = pow2i(sh);
-    for (int g0 = 0; g0 < Gd; g0 += 2) {
-      const int g = g0 + (lane >> 4), part = lane & 15;
+    for (int pr = slice; pr < n_pairs; pr += wpt) {
+      const int g = 2 * pr + (lane >> 4), part = lane & 15;
       const bool ok = g < Gd;
       const __nv_bfloat16* src = row + g * 128;
       __align__(16) __half o[8];
+      if (a.x16) {
+        // tcgen05 order: positions 8 part .. 8 part + 7 of group g
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int q = 8 * part + e;
+          const float v = ok ? __bfloat162float(src[pos_col(a.fmt, q)]) * xs : 0.f;
+          o[e] = __float2half_rn(a.fmt == SCION_PQ2_0 ? v * pq2_pos_scale(q) : v);
+        }
+        if (ok) *reinterpret_cast<uint4*>(a.x16 + int64_t(t) * a.d + g * 128 + 8 * part) = *reinterpret_cast<const uint4*>(o);
+        continue;
+      }
       float sum = 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -144,7 +162,7 @@ template <int NT>
 __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
   extern __shared__ __align__(16) uint8_t xsm[];
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(xsm);  // [NT*8][kXRow], then the warp reduction
-  __shared__ uint32_t tmax[SCION_TDEC];  // largest |x| bits of each token over this CTA's K chunk
+  __shared__ uint32_t tmax[SCION_TDEC];  // largest |x| bits of each token over this CTA's K chunk (T entries)
   __shared__ int tshift[SCION_TDEC];     // lead CTA: range exponent of each token
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, c = lane & 3;
@@ -215,7 +233,6 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
   // the shared-expert and correction rows are stored scaled per token (hz_shift), which needs the
   // largest |x| of each token: each chunk's CTA finds it over its columns, the lead combines them
   const bool need_max = u.kind != kUnitRouter;
-  for (int i = threadIdx.x; i < SCION_TDEC; i += kXThreads) tmax[i] = 0;
   pdl_wait();  // everything below reads x or writes the workspace
   // stage x[0..T)[kbase .. kbase+512) in shared memory (rows padded by 16 B: conflict-free reads)
   const int kchunks = min(SCION_XPROJ_KC, a.d - kbase) >> 3;  // 16-byte chunks per token row (<= 64)
@@ -229,9 +246,11 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
   if (need_max)
-    for (int i = threadIdx.x; i < a.T * kchunks; i += kXThreads) {
-      const int t = i / kchunks, j = i % kchunks;
-      atomicMax(&tmax[t], max_mag8(*reinterpret_cast<const uint4*>(xs + t * kXRow + 8 * j)));
+    for (int t = warp; t < a.T; t += kXThreads / 32) {  // one warp per staged token row
+      uint32_t m = 0;
+      for (int j = lane; j < kchunks; j += 32) m = max(m, max_mag8(*reinterpret_cast<const uint4*>(xs + t * kXRow + 8 * j)));
+      m = __reduce_max_sync(0xffffffffu, m);
+      if (lane == 0) tmax[t] = m;
     }
   if (active_warp) {
     const bool second_acc = (u.kind == kUnitSwiglu);
@@ -344,7 +363,7 @@ struct GateUpArgs {
   const __half* xfrag;  // [T][Gd][128]
   const int4* slot_info;
   const int32_t *n_active, *perm;
-  const int32_t* xexp;  // [T] range exponent of each token
+  const int32_t* pexp;  // [T*k] range exponent of the token of each routed position
   int d, F, k, Gd, fmt;
   __half* hfrag;  // [T*k][GF][128] fragment order of the down format, h 2^(2 s_t)
 };
@@ -404,7 +423,7 @@ __device__ __forceinline__ void gateup_body(const GateUpArgs& a, int slot, int f
         const int f = ft * 16 + row;
         const int64_t pos = p0 + pc + tcol;
         const int idx = brow_pos(a.fmt, f & 127);
-        const int sh = a.xexp[a.perm[pos] / a.k];  // the sums are of x 2^sh
+        const int sh = a.pexp[pos];  // the sums are of x 2^sh
         float h = silu_f(gs * pow2i(-sh)) * (us * pow2i(sh));
         if (a.fmt == SCION_PQ2_0) h *= brow_bscale(idx);
         a.hfrag[(pos * GF + (f >> 7)) * SCION_BROW + idx] = __float2half_rn(h);
@@ -425,8 +444,7 @@ struct DownArgs {
   const __half* hfrag;  // [T*k][GF][128]
   const int4* slot_info;
   const int32_t *n_active, *perm;
-  const float* gates;
-  const int32_t* xexp;  // [T] range exponent of each token (the hidden is h 2^(2 s_t))
+  const float* gperm;  // [T*k] gate of each routed position, times 2^(-2 s_t) (the hidden is h 2^(2 s_t))
   int d, F, k, GF;
   float* out;
 };
@@ -478,8 +496,7 @@ __global__ void __launch_bounds__(kDnWarps * 32) down_routed_kernel(DownArgs a) 
       const int row = (ln >> 2) + 8 * (i >> 1), tcol = 2 * (ln & 3) + (i & 1);
       if (tcol < nn) {
         const int entry = a.perm[p0 + pc + tcol];
-        const int t = entry / a.k;
-        atomicAdd(&a.out[int64_t(t) * a.d + dt * 16 + row], a.gates[entry] * pow2i(-2 * a.xexp[t]) * v);
+        atomicAdd(&a.out[int64_t(entry / a.k) * a.d + dt * 16 + row], a.gperm[p0 + pc + tcol] * v);
       }
     }
     __syncthreads();
@@ -632,7 +649,7 @@ __global__ void unfrag_kernel(int fmt, const __half* __restrict__ src, int64_t n
 
 // ------------------------------------------------------------------- launchers
 cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, const float* resid,
-                         int unit0, int n_units, bool aux, cudaStream_t s) {
+                         int unit0, int n_units, bool aux, bool x16, cudaStream_t s) {
   XProjArgs a;
   a.resid = resid;
   a.x = x;
@@ -644,6 +661,7 @@ cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, fl
   a.corr_a = static_cast<const __nv_bfloat16*>(L->desc.corr_a);
   a.units = L->xunits + unit0, a.n_units = n_units, a.n_chunks = L->n_xchunks, a.n_aux = aux ? kXAux : 0;
   a.logits = L->logits, a.hz = L->hz, a.xfrag = L->xfrag, a.xexp = L->xexp, a.out = out;
+  a.x16 = x16 ? L->x16d : nullptr;
   a.corr_blocks = L->desc.corr_packed ? static_cast<const uint8_t*>(L->desc.corr_a) : nullptr;
   a.h = L->h, a.k = L->k, a.GF = L->GF;
   if (n_units + a.n_aux == 0) return cudaSuccess;
@@ -665,7 +683,7 @@ cudaError_t launch_gateup(const scion_layer* L, const __nv_bfloat16* /*x*/, int 
   a.bank = L->gu_bank, a.xfrag = L->xfrag;
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
   a.d = L->d, a.F = L->F, a.k = L->k, a.Gd = L->Gd, a.fmt = L->fmt;
-  a.hfrag = L->h, a.xexp = L->xexp;
+  a.hfrag = L->h, a.pexp = L->pexp;
   const int slots = min(L->E, T * L->k);
   const dim3 grid(L->F / 16, slots);
   const int gpw = (L->Gd + kGuWarps - 1) / kGuWarps;
@@ -692,7 +710,7 @@ cudaError_t launch_gateup_dense(const scion_layer* L, int T, float* out, cudaStr
   a.bank = L->gu_bank, a.xfrag = L->xfrag;
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
   a.d = L->d, a.F = L->F, a.k = L->k, a.Gd = L->Gd, a.fmt = L->fmt;
-  a.hfrag = L->h, a.xexp = L->xexp;
+  a.hfrag = L->h, a.pexp = L->pexp;
   DenseArgs b;
   b.w = L->dense_down, b.hz = L->hz, b.d = L->d, b.Kd = L->Kd, b.T = T, b.out = out;
   b.corr_b = L->desc.corr_packed ? static_cast<const uint8_t*>(L->desc.corr_b) : nullptr, b.Fs = L->Fs, b.r = L->r;
@@ -725,7 +743,7 @@ cudaError_t launch_down_routed(const scion_layer* L, int T, float* out, cudaStre
   DownArgs a;
   a.bank = L->dn_bank, a.hfrag = L->h;
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
-  a.gates = L->gates, a.xexp = L->xexp;
+  a.gperm = L->gperm;
   a.d = L->d, a.F = L->F, a.k = L->k, a.GF = L->GF, a.out = out;
   const int slots = min(L->E, T * L->k);
   const dim3 grid(L->d / 16, slots);

@@ -32,6 +32,7 @@
 #include <string.h>
 
 #include "tc_common.cuh"
+#include "tc_order.cuh"
 #include "topk_warp.cuh"
 
 namespace scion {
@@ -45,39 +46,6 @@ constexpr int kBN = 128;  // tokens per tile
 constexpr int kThreads = 384;   // dense GEMM: TMA warp, MMA warp, 2 idle, 8 epilogue warps
 constexpr int kDenseEpi = 256;  // epilogue threads (two warps per TMEM lane quarter)
 
-// ------------------------------------------------------------- column orders
-__device__ __forceinline__ int perm_pos(int fmt, int col) {  // physical column -> position
-  if (fmt == SCION_PQ2_0) {
-    int c16 = col & 15;
-    return (col & ~15) | (2 * (c16 & 7) + (c16 >> 3));
-  }
-  // PTQ1_0: half h of the group (positions 64h .. 64h+63) holds quintets 12h .. 12h+11 as
-  // pairs (2i, 2i+1) -- position 10i + 2j + u <-> column 5(12h + 2i + u) + j -- and then
-  // remainder trits 4h .. 4h+3 (columns 120 + 4h ..) in natural order.
-  const int g = col & ~127, k = col & 127;
-  if (k >= 120) return g | (64 * ((k - 120) >> 2) + 60 + ((k - 120) & 3));
-  const int q = k / 5, j = k % 5, half = q / 12, i = (q % 12) >> 1, u = q & 1;
-  return g | (64 * half + 10 * i + 2 * j + u);
-}
-
-// PQ2_0 B-operand factor of position p: positions (2s, 2s+1) of every 16 hold the pair of
-// columns (s, s + 8) that the expansion builds with the field at bits 2f..2f+1 of a 16-bit code
-// half (f = s < 5 ? s : s - 5), i.e. scaled by 4^f; the B operands (x and h) carry 4^-f, an exact
-// power-of-two scaling.
-__device__ __forceinline__ float pq2_pos_scale(int p) {
-  const int s = (p & 15) >> 1;
-  return 1.0f / float(1 << (2 * (s < 5 ? s : s - 5)));
-}
-
-// Column held by position p of a 128-column group (the inverse of perm_pos).
-__device__ __forceinline__ int pos_col(int fmt, int p) {
-  if (fmt == SCION_PQ2_0) return (p & ~15) | (((p & 15) >> 1) + 8 * (p & 1));
-  const int half = p >> 6, r = p & 63;
-  if (r >= 60) return 120 + 4 * half + (r - 60);
-  const int i = r / 10, rem = r % 10;
-  return 5 * (12 * half + 2 * i + (rem & 1)) + (rem >> 1);
-}
-
 // x (bf16) -> fp16 x 2^s_t in the container's column order (PQ2_0: times the factor of its
 // position), s_t the token's range exponent (token_shift of its largest magnitude, written to
 // xexp).  One warp per token: the whole row's coalesced 16-byte loads are issued first (pairs of
@@ -89,9 +57,12 @@ __device__ __forceinline__ uint32_t max_mag8(uint4 v) {
   const uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu), __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
   return max(m & 0xFFFFu, m >> 16);
 }
+// init_out: also set out[t] = resid[t] (or zero) -- for layers without shared expert and
+// correction, whose routed down projection only adds into out.
 template <int FMT>
 __global__ void __launch_bounds__(256) x16_kernel(const __nv_bfloat16* __restrict__ x, int T, int d,
-                                                  __half* __restrict__ xp, int32_t* __restrict__ xexp) {
+                                                  __half* __restrict__ xp, int32_t* __restrict__ xexp,
+                                                  int init_out, const float* resid, float* out) {
   __shared__ __align__(16) __nv_bfloat16 buf[8][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gl = lane >> 4, p0 = 8 * (lane & 15);  // group of the pair, first output position
@@ -125,6 +96,11 @@ __global__ void __launch_bounds__(256) x16_kernel(const __nv_bfloat16* __restric
         o[e] = __float2half_rn(FMT == SCION_PQ2_0 ? f * pq2_pos_scale(p) : f);
       }
       if (2 * i + gl < G) reinterpret_cast<uint4*>(orow + i * 256)[lane] = *reinterpret_cast<const uint4*>(o);
+    }
+    if (init_out && resid != out) {
+      float4* o4 = reinterpret_cast<float4*>(out + int64_t(t) * d);
+      const float4* r4 = reinterpret_cast<const float4*>(resid + int64_t(t) * d);
+      for (int j = lane; j < d / 4; j += 32) o4[j] = resid ? r4[j] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
 }
@@ -398,30 +374,38 @@ struct __align__(16) TernTile {
   int pos0;  // routed-order position of its first token (offsets[e] + c0)
 };
 
-__device__ __forceinline__ TernTile load_tile(const TernTile* tiles, int i) {
+// slots = 1: the list is the decode routing's active-slot records {expert, first routed
+// position, tokens, 0}, one tile per active expert (a decode batch never fills more than one).
+__device__ __forceinline__ TernTile load_tile(const TernTile* tiles, int i, int slots) {
   const int4 v = __ldg(reinterpret_cast<const int4*>(tiles) + i);
-  return TernTile{v.x, v.y, v.z, v.w};
+  return slots ? TernTile{v.x, 0, v.z, v.y} : TernTile{v.x, v.y, v.z, v.w};
 }
 
 struct TernParams {
-  CUtensorMap bmap;     // down projection: B = h [T*k][F], box {64, 128}
+  CUtensorMap bmap;     // down projection: B = h [T*k][F], box {64, box_rows}
+  int box_rows;         // rows of one TMA box of B (the tile width, or 16 for decode tiles)
   const uint8_t* bank;  // re-tiled gate/up bank (na = 2) or down bank (na = 1)
   int fmt, na, G, R;    // groups along K, rows per expert matrix
   const __half* bsrc;   // B rows: x16 [T][d] (gate/up) or h [T*k][F] (down)
   int ldb;
   const TernTile* tiles;
+  int tile_slots;       // 1: `tiles` holds the decode routing's slot records (see load_tile)
   const int32_t* n_tiles;
   const int32_t *counts, *offsets, *perm;
-  const float* gates;
+  const float* gperm;   // [T*k] gate of the entry at each routed position, times 2^(-2 s_t)
   int k;
-  const int32_t* pexp;   // range exponent of the token of each routed position (B rows are x 2^s)
-  __half* h;  int F;     // gate/up output, h 2^(2 s)
-  __half* y;  int d;     // down output: one fp16 row per routed (token, slot), [T*k][d], gates applied by the combine
+  const int32_t* pexp;  // [T*k] range exponent s_t of the token of each routed position (gate/up B rows are x 2^s_t)
+  __half* h;  int F;     // gate/up output, h 2^(2 s_t), one row per routed position
+  // down output: y != nullptr -> one fp16 row per routed (token, slot), [T*k][d], gates applied
+  // by the combine; otherwise out[t] += gate 2^(-2 s_t) y with fp32 reductions
+  __half* y;  int d;
+  float* out;
   int* err;
 };
 
 constexpr int kBN3 = 160;      // tokens per tile of batches whose experts average kMid160 or more
 constexpr int kMid160 = 112;   // mean tokens per expert from which both ternary GEMMs take kBN3 tiles
+constexpr int kBND = 64;       // tokens per tile of decode batches (at most 64 tokens in all)
 
 // Expand half h (64 columns) of row t (0..127) of one 128-row group from its sub-tile block
 // into 32 registers of fp16 pairs, in position order (v[i] = positions 2i, 2i+1 of the half).
@@ -512,7 +496,7 @@ struct TernRing {
   static constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
   // shared memory: B groups (two 64-column K blocks of TN swizzled 128-byte rows) and packed
   // code groups
-  static_assert(TN == kBN || TN == kBN3, "tile width");
+  static_assert(TN == kBN || TN == kBN3 || TN == kBND, "tile width");
   static constexpr int kB = 4;
   static constexpr int kC = 4;
   static constexpr uint32_t b_kblock = uint32_t(TN) * 128;  // bytes of one 64-column K block of B
@@ -521,14 +505,15 @@ struct TernRing {
   static constexpr uint32_t b_off = 0, c_off = kB * b_bytes;
   static constexpr uint32_t bytes = c_off + kC * c_bytes;
   // tensor memory: accumulators, then the ring of expanded A groups
-  // gate/up: one NA x TN accumulator; down: two TN-column accumulators (ping-pong)
-  static constexpr int n_acc = NA == 1 ? 2 : 1;
+  // gate/up: one NA x TN accumulator (two, ping-pong, for decode tiles); down: two TN-column
+  // accumulators (ping-pong)
+  static constexpr int n_acc = (NA == 1 || TN == kBND) ? 2 : 1;
   static constexpr uint32_t acc_cols = NA * TN;
   // ring entries of expanded A: one group of all NA matrices, or (160-token gate/up tiles,
   // whose accumulators leave 192 columns) one matrix of a group, EPG entries per group
   static constexpr int EPG = TN == kBN3 ? NA : 1;
   static constexpr int MPE = NA / EPG;           // matrices per entry
-  static constexpr int kA = TN == kBN3 ? 3 : (NA == 2 ? 2 : 4);
+  static constexpr int kA = TN == kBN3 ? 3 : (TN == kBND ? (NA == 2 ? 2 : 6) : (NA == 2 ? 2 : 4));
   static constexpr uint32_t a_cols = MPE * 64;   // one entry: MPE matrices x 64 columns (128 fp16 per lane)
   static constexpr uint32_t a_col0 = n_acc * acc_cols;
   static constexpr uint32_t tmem_cols = 512;
@@ -581,7 +566,7 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
       const int64_t mat_stride = int64_t(8) * R::tb, grp_stride = NA * mat_stride;
       int gs = 0;  // running group counter
       for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
-        const TernTile tile = load_tile(p.tiles, item / RT);
+        const TernTile tile = load_tile(p.tiles, item / RT, p.tile_slots);
         const int rt = item % RT;
         const uint8_t* ebase = p.bank + (int64_t(tile.e) * RT + rt) * p.G * grp_stride;
         for (int g = 0; g < p.G; ++g, ++gs) {
@@ -602,17 +587,21 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
     if (lane == 0) {
       int gs = 0;
       for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
-        const int row0 = load_tile(p.tiles, item / RT).pos0;
+        const TernTile tile = load_tile(p.tiles, item / RT, p.tile_slots);
+        // boxes of box_rows rows (128-byte rows, swizzle atoms of 8 rows: consecutive boxes
+        // stack into one TN-row operand); rows past the tile's tokens are loaded but never stored
+        const int nbox = p.box_rows >= TN ? 1 : (tile.n + p.box_rows - 1) / p.box_rows;
+        const uint32_t box_bytes = uint32_t(min(p.box_rows, TN)) * 128;
         for (int g = 0; g < p.G; ++g, ++gs) {
           const int s = gs % R::kB;
           if (gs >= R::kB && !mbar_wait(&b_empty[s], ((gs / R::kB) - 1) & 1, &abort_flag, p.err)) break;
           uint8_t* dst = smem + R::b_off + s * R::b_bytes;
-          mbar_arrive_expect_tx(&b_full[s], R::b_bytes);
+          mbar_arrive_expect_tx(&b_full[s], 2 * nbox * box_bytes);
 #pragma unroll
-          for (int kb = 0; kb < 2; ++kb) {  // 64-column K blocks of the group, TN token rows each
-            // the map's box is TN rows
-            tma_load_2d(dst + kb * R::b_kblock, &p.bmap, g * 128 + 64 * kb, row0, &b_full[s]);
-          }
+          for (int kb = 0; kb < 2; ++kb)  // 64-column K blocks of the group
+            for (int bx = 0; bx < nbox; ++bx)
+              tma_load_2d(dst + kb * R::b_kblock + bx * box_bytes, &p.bmap, g * 128 + 64 * kb,
+                          tile.pos0 + bx * p.box_rows, &b_full[s]);
         }
       }
       for (int i = max(0, gs - R::kB); i < gs; ++i) mbar_drain(&b_full[i % R::kB], (i / R::kB) & 1);
@@ -627,7 +616,7 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
     constexpr int kLag = R::kB / 2;  // groups in flight per thread before the oldest is published
     int gs = 0;                      // running group counter
     for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
-      const TernTile tile = load_tile(p.tiles, item / RT);
+      const TernTile tile = load_tile(p.tiles, item / RT, p.tile_slots);
       const __half* rows[kRows];
 #pragma unroll
       for (int i = 0; i < kRows; ++i) {
@@ -667,10 +656,10 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
     if (lane == 0) {
       // ---------------- MMA issuer: A from tensor memory, B from shared memory
       int gs = 0, es = 0, li = 0;  // running group, A-entry and item counters
-      TernTile next = blockIdx.x < n_items ? load_tile(p.tiles, blockIdx.x / RT) : TernTile{};
+      TernTile next = blockIdx.x < n_items ? load_tile(p.tiles, blockIdx.x / RT, p.tile_slots) : TernTile{};
       for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x, ++li) {
         const TernTile tile = next;  // loaded one item ahead: no global-load latency between items
-        if (item + int(gridDim.x) < n_items) next = load_tile(p.tiles, (item + gridDim.x) / RT);
+        if (item + int(gridDim.x) < n_items) next = load_tile(p.tiles, (item + gridDim.x) / RT, p.tile_slots);
         const uint32_t idesc = umma_idesc(kBM, (tile.n + 15) & ~15, 0);
         const int ab = li % R::n_acc;
         if (li >= R::n_acc && !mbar_wait(&acc_empty[ab], ((li / R::n_acc) - 1) & 1, &abort_flag, p.err)) break;
@@ -753,7 +742,7 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
     int li = 0;
     // no abort-flag test in the loop condition: the epilogue threads leave only together, by the vote
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++li) {
-      const TernTile tile = load_tile(p.tiles, item / RT);
+      const TernTile tile = load_tile(p.tiles, item / RT, p.tile_slots);
       const int rt = item % RT;
       const int64_t pos0 = tile.pos0;
       const int nn = tile.n;
@@ -773,14 +762,22 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             if (n0 + i < nn) {
-              const int sh = p.pexp[pos0 + n0 + i];
+              const int sh = p.pexp[pos0 + n0 + i];  // the sums are of x 2^sh
               dst[int64_t(i) * p.F] = __float2half_rn(silu_f(v0[i] * pow2i(-sh)) * (v1[i] * pow2i(sh)) * hscale);
             }
-        } else {
+        } else if (p.y) {
           __half* dst = p.y + (pos0 + n0) * p.d + int64_t(rt) * kBM + row;
 #pragma unroll
           for (int i = 0; i < 16; ++i)
             if (n0 + i < nn) dst[int64_t(i) * p.d] = __float2half_rn(v0[i]);
+        } else {
+          // gate-weighted scatter-add: the warp's 32 rows of one token are 128 contiguous bytes
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (n0 + i < nn) {
+              const int t = p.perm[pos0 + n0 + i] / p.k;
+              atomicAdd(p.out + int64_t(t) * p.d + int64_t(rt) * kBM + row, p.gperm[pos0 + n0 + i] * v0[i]);
+            }
         }
       }
       // accumulator drained: hand it back to the MMA warp
@@ -880,8 +877,9 @@ constexpr int kScatterMaxPerThread = 8;
 __global__ void __launch_bounds__(256) group_scatter_kernel(const int32_t* __restrict__ ids, int n, int E, int ept,
                                                             int32_t* __restrict__ cursor, int32_t* __restrict__ perm,
                                                             int32_t* __restrict__ inv, int k,
+                                                            const float* __restrict__ gates,
                                                             const int32_t* __restrict__ xexp,
-                                                            int32_t* __restrict__ pexp) {
+                                                            float* __restrict__ gperm, int32_t* __restrict__ pexp) {
   extern __shared__ int32_t sh[];  // cnt[E], base[E]
   int32_t *cnt = sh, *base = sh + E;
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
@@ -902,9 +900,11 @@ __global__ void __launch_bounds__(256) group_scatter_kernel(const int32_t* __res
   for (int j = 0; j < kScatterMaxPerThread; ++j) {
     if (id[j] < 0) continue;
     const int i = i0 + 256 * j, pos = base[id[j]] + local[j];
+    const int sh = xexp[i / k];
     perm[pos] = i;
     inv[i] = pos;
-    pexp[pos] = xexp[i / k];
+    pexp[pos] = sh;
+    gperm[pos] = gates[i] * pow2i(-2 * sh);
   }
 }
 
@@ -949,6 +949,7 @@ size_t tern_smem_t() {
 }
 template <int FMT>
 size_t tern_smem_f(int na, int tn) {
+  if (tn == kBND) return na == 2 ? tern_smem_t<FMT, 2, kBND>() : tern_smem_t<FMT, 1, kBND>();
   if (na == 2) return tn == kBN3 ? tern_smem_t<FMT, 2, kBN3>() : tern_smem_t<FMT, 2, kBN>();
   return tn == kBN3 ? tern_smem_t<FMT, 1, kBN3>() : tern_smem_t<FMT, 1, kBN>();
 }
@@ -1006,6 +1007,15 @@ cudaError_t configure_prefill_kernels() {
   if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PTQ1_0, 2, kBN3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 int(tern_smem(2, SCION_PTQ1_0, kBN3)))))
     return e;
+#define SCION_TC_DEC_SMEM(F, NA)                                                                 \
+  if ((e = cudaFuncSetAttribute(tern_gemm_kernel<F, NA, kBND>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                int(tern_smem(NA, F, kBND)))))                                   \
+    return e;
+  SCION_TC_DEC_SMEM(SCION_PQ2_0, 2)
+  SCION_TC_DEC_SMEM(SCION_PQ2_0, 1)
+  SCION_TC_DEC_SMEM(SCION_PTQ1_0, 2)
+  SCION_TC_DEC_SMEM(SCION_PTQ1_0, 1)
+#undef SCION_TC_DEC_SMEM
   return cudaSuccess;
 }
 
@@ -1116,10 +1126,13 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
   switch (stage) {
     case SCION_STAGE_X16: {
       const unsigned grid = unsigned(std::min((T + 7) / 8, num_sms() * 8));
+      // without a dense down projection (which stores out first) the fused routed down
+      // projection only adds into out: set it here
+      const int init = P.n_dunits == 0 && !L->deterministic;
       if (L->fmt == SCION_PQ2_0)
-        x16_kernel<SCION_PQ2_0><<<grid, 256, 0, s>>>(x, T, L->d, P.x16, P.xexp);
+        x16_kernel<SCION_PQ2_0><<<grid, 256, 0, s>>>(x, T, L->d, P.x16, P.xexp, init, resid, out);
       else
-        x16_kernel<SCION_PTQ1_0><<<grid, 256, 0, s>>>(x, T, L->d, P.x16, P.xexp);
+        x16_kernel<SCION_PTQ1_0><<<grid, 256, 0, s>>>(x, T, L->d, P.x16, P.xexp, init, resid, out);
       return cudaGetLastError();
     }
     case SCION_STAGE_XPROJ: {
@@ -1162,7 +1175,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
                                                   tile_width(int64_t(T) * L->k, L->E));
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
       group_scatter_kernel<<<(n + 256 * ept - 1) / (256 * ept), 256, 2 * sizeof(int32_t) * L->E, s>>>(
-          P.ids, n, L->E, ept, P.cursor, P.perm, P.inv, L->k, P.xexp, P.pexp);
+          P.ids, n, L->E, ept, P.cursor, P.perm, P.inv, L->k, P.gates, P.xexp, P.gperm, P.pexp);
       return cudaGetLastError();
     }
     case SCION_STAGE_GATEUP: {
@@ -1171,8 +1184,8 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       tp.bsrc = P.x16, tp.ldb = L->d;
       const bool mid = tile_width(int64_t(T) * L->k, L->E) == kBN3;
       tp.tiles = static_cast<const TernTile*>(P.tiles), tp.n_tiles = P.n_tiles;
-      tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gates = P.gates, tp.k = L->k;
-      tp.pexp = P.pexp;
+      tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gperm = P.gperm, tp.k = L->k;
+      tp.pexp = P.pexp, tp.tile_slots = 0, tp.box_rows = kBN, tp.out = nullptr;
       tp.h = P.h, tp.F = L->F, tp.y = nullptr, tp.d = L->d, tp.err = L->err;
       const dim3 grid(num_sms());
       if (L->fmt == SCION_PQ2_0 && mid)
@@ -1209,9 +1222,11 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       tp.bsrc = P.h, tp.ldb = L->F;
       const int wd = tile_width(int64_t(T) * L->k, L->E);
       tp.tiles = static_cast<const TernTile*>(P.tiles), tp.n_tiles = P.n_tiles;
-      tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gates = P.gates, tp.k = L->k;
-      tp.pexp = P.pexp;
-      tp.h = nullptr, tp.F = L->F, tp.y = P.y, tp.d = L->d, tp.err = L->err;
+      tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gperm = P.gperm, tp.k = L->k;
+      tp.pexp = P.pexp, tp.tile_slots = 0, tp.box_rows = wd;
+      // fused gate-weighted scatter-add into out, or (deterministic) one row per entry for the combine
+      tp.out = out, tp.y = L->deterministic ? P.y : nullptr;
+      tp.h = nullptr, tp.F = L->F, tp.d = L->d, tp.err = L->err;
       if (make_tmap_2d(&tp.bmap, P.h, 0, int64_t(T) * L->k, L->F, wd) != SCION_OK)
         return cudaErrorInvalidValue;
       const dim3 grid(num_sms());
@@ -1226,6 +1241,31 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
     default:
       return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_tc_decode(int na, const scion_layer* L, int T, float* out, cudaStream_t s) {
+  TernParams tp;
+  memset(&tp, 0, sizeof(tp));
+  tp.fmt = L->fmt, tp.na = na, tp.k = L->k, tp.F = L->F, tp.d = L->d, tp.err = L->err;
+  tp.tiles = static_cast<const TernTile*>(L->slot_info), tp.tile_slots = 1, tp.n_tiles = L->n_active;
+  tp.counts = L->counts, tp.offsets = L->offsets, tp.perm = L->perm, tp.gperm = L->gperm, tp.pexp = L->pexp;
+  if (na == 2) {
+    tp.bank = L->gu_bank, tp.G = L->Gd, tp.R = L->F, tp.bsrc = L->x16d, tp.ldb = L->d, tp.h = L->hp;
+    tp.box_rows = kBND;
+  } else {
+    tp.bank = L->dn_bank, tp.G = L->GF, tp.R = L->d, tp.bsrc = L->hp, tp.ldb = L->F, tp.out = out;
+    tp.bmap = L->hp_map, tp.box_rows = 16;
+  }
+  const int items = std::min(L->E, T * L->k) * (tp.R / 128);
+  const dim3 grid(std::max(1, std::min(items, num_sms())));
+#define SCION_TCD(F, NA) tern_gemm_kernel<F, NA, kBND><<<grid, kTernThreads, tern_smem(NA, F, kBND), s>>>(tp)
+  if (L->fmt == SCION_PQ2_0) {
+    if (na == 2) SCION_TCD(SCION_PQ2_0, 2); else SCION_TCD(SCION_PQ2_0, 1);
+  } else {
+    if (na == 2) SCION_TCD(SCION_PTQ1_0, 2); else SCION_TCD(SCION_PTQ1_0, 1);
+  }
+#undef SCION_TCD
+  return cudaGetLastError();
 }
 
 }  // namespace scion

@@ -59,7 +59,9 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
                                                               int32_t* __restrict__ perm_out,
                                                               float* __restrict__ gperm_out,
                                                               int32_t* __restrict__ active_out,
-                                                              int32_t* __restrict__ n_active_out) {
+                                                              int32_t* __restrict__ n_active_out,
+                                                              const int32_t* __restrict__ xexp,
+                                                              int32_t* __restrict__ pexp_out) {
   extern __shared__ float smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = kRouteThreads / 32;
   float* vals = smem + warp * E;
@@ -165,8 +167,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
       int cur = i < n ? cursor[e] : 0;
       __syncwarp();
       if (i < n) {
+        const int sh = xexp[i / k];
         perm_out[cur + rank] = i;
-        gperm_out[cur + rank] = gates_out[i];
+        gperm_out[cur + rank] = gates_out[i] * pow2i(-2 * sh);
+        pexp_out[cur + rank] = sh;
         if (rank == 0) cursor[e] = cur + __popc(mask);
       }
       __syncwarp();
@@ -182,10 +186,14 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
 // and the last one to finish stages the entries and groups them.
 
 // Warp 0 of the grouping CTA: counts[] holds the histogram of the n staged entries.
-__device__ __forceinline__ void group_staged(const int32_t* ids_s, const float* gates_s, int n, int E, int lane,
-                                             int32_t* counts, int32_t* cursor, int32_t* __restrict__ counts_out,
-                                             int32_t* __restrict__ offsets_out, int32_t* __restrict__ perm_out,
-                                             float* __restrict__ gperm_out, int32_t* __restrict__ active_out,
+// xexp_s: the tokens' range exponents (staged); each routed position gets its token's exponent
+// (pexp_out) and its gate times 2^(-2 s_t) (gperm_out), the factor that takes the scaled expert
+// hidden back to the block's units.
+__device__ __forceinline__ void group_staged(const int32_t* ids_s, const float* gates_s, const int32_t* xexp_s, int n,
+                                             int k, int E, int lane, int32_t* counts, int32_t* cursor,
+                                             int32_t* __restrict__ counts_out, int32_t* __restrict__ offsets_out,
+                                             int32_t* __restrict__ perm_out, float* __restrict__ gperm_out,
+                                             int32_t* __restrict__ pexp_out, int32_t* __restrict__ active_out,
                                              int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info) {
   const int per = (E + 31) / 32;
   const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
@@ -221,8 +229,10 @@ __device__ __forceinline__ void group_staged(const int32_t* ids_s, const float* 
     const int cur = i < n ? cursor[e] : 0;
     __syncwarp();
     if (i < n) {
+      const int sh = xexp_s[i / k];
       perm_out[cur + rank] = i;
-      gperm_out[cur + rank] = gates_s[i];
+      gperm_out[cur + rank] = gates_s[i] * pow2i(-2 * sh);
+      pexp_out[cur + rank] = sh;
       if (rank == 0) cursor[e] = cur + __popc(mask);
     }
     __syncwarp();
@@ -241,18 +251,21 @@ __global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
     const float* __restrict__ logits, int T, int E, int k, int norm_topk, int32_t* __restrict__ ids,
     float* __restrict__ gates, int32_t* __restrict__ counts_out, int32_t* __restrict__ offsets_out,
     int32_t* __restrict__ perm_out, float* __restrict__ gperm_out, int32_t* __restrict__ active_out,
-    int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info) {
-  extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [E] | cursor [E]
+    int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info, const int32_t* __restrict__ xexp,
+    int32_t* __restrict__ pexp_out) {
+  extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [E] | cursor [E] | xexp [T]
   const int n = T * k;
   int32_t* ids_s = reinterpret_cast<int32_t*>(rs);
   float* gates_s = rs + n;
   int32_t* counts = reinterpret_cast<int32_t*>(rs + 2 * n);
   int32_t* cursor = counts + E;
+  int32_t* xexp_s = cursor + E;
   constexpr int kThr = rc_threads<VPL>();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
   for (int e = threadIdx.x; e < E; e += kThr) counts[e] = 0;
   pdl_wait();
+  for (int t = threadIdx.x; t < T; t += kThr) xexp_s[t] = xexp[t];
   for (int t = warp; t < T; t += kThr / 32)
     warp_topk<VPL>(logits + int64_t(t) * E, E, k, norm_topk, lane, ids_s + t * k, gates_s + t * k);
   __syncthreads();
@@ -263,8 +276,8 @@ __global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
   }
   __syncthreads();
   if (warp == 0)
-    group_staged(ids_s, gates_s, n, E, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out,
-                 active_out, n_active_out, slot_info);
+    group_staged(ids_s, gates_s, xexp_s, n, k, E, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out,
+                 pexp_out, active_out, n_active_out, slot_info);
 }
 
 // ceil(T/4) CTAs of 4 warps (T > 32); the last CTA to finish groups.
@@ -275,14 +288,16 @@ __global__ void __launch_bounds__(kRmThreads) route_multi_kernel(
     const float* __restrict__ logits, int T, int E, int k, int norm_topk, int32_t* __restrict__ ids,
     float* __restrict__ gates, int32_t* __restrict__ counts_out, int32_t* __restrict__ offsets_out,
     int32_t* __restrict__ perm_out, float* __restrict__ gperm_out, int32_t* __restrict__ active_out,
-    int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info, unsigned* __restrict__ done) {
-  extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [E] | cursor [E]
+    int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info, unsigned* __restrict__ done,
+    const int32_t* __restrict__ xexp, int32_t* __restrict__ pexp_out) {
+  extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [E] | cursor [E] | xexp [T]
   __shared__ int last;
   const int n = T * k;
   int32_t* ids_s = reinterpret_cast<int32_t*>(rs);
   float* gates_s = rs + n;
   int32_t* counts = reinterpret_cast<int32_t*>(rs + 2 * n);
   int32_t* cursor = counts + E;
+  int32_t* xexp_s = cursor + E;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * (kRmThreads / 32) + warp;
   pdl_trigger();
@@ -296,16 +311,17 @@ __global__ void __launch_bounds__(kRmThreads) route_multi_kernel(
   __threadfence();
   for (int e = threadIdx.x; e < E; e += kRmThreads) counts[e] = 0;
   for (int i = threadIdx.x; i < n; i += kRmThreads) ids_s[i] = __ldcg(&ids[i]), gates_s[i] = __ldcg(&gates[i]);
+  for (int i = threadIdx.x; i < T; i += kRmThreads) xexp_s[i] = xexp[i];
   __syncthreads();
   for (int i = threadIdx.x; i < n; i += kRmThreads) atomicAdd(&counts[ids_s[i]], 1);
   __syncthreads();
   if (warp != 0) return;
   if (lane == 0) *done = 0;
-  group_staged(ids_s, gates_s, n, E, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out, active_out,
-               n_active_out, slot_info);
+  group_staged(ids_s, gates_s, xexp_s, n, k, E, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out,
+               pexp_out, active_out, n_active_out, slot_info);
 }
 
-size_t route_cta_smem(int T, int E, int k) { return sizeof(float) * (2 * size_t(T) * k + 2 * size_t(E)); }
+size_t route_cta_smem(int T, int E, int k) { return sizeof(float) * (2 * size_t(T) * k + 2 * size_t(E) + size_t(T)); }
 
 }  // namespace
 
@@ -323,11 +339,12 @@ cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s) {
 #define SCION_ROUTE_CTA(V)                                                                                     \
   return T <= 32 ? launch_pdl(route_cta_kernel<V>, dim3(1), dim3(rc_threads<V>()), smem, s, L->logits, T, L->E, \
                               L->k, L->desc.norm_topk, L->ids, L->gates, L->counts, L->offsets, L->perm,       \
-                              L->gperm, L->active, L->n_active, reinterpret_cast<int4*>(L->slot_info))        \
+                              L->gperm, L->active, L->n_active, reinterpret_cast<int4*>(L->slot_info), L->xexp, \
+                              L->pexp)                                                                         \
                  : launch_pdl(route_multi_kernel<V>, dim3((T + 3) / 4), dim3(kRmThreads), smem, s, L->logits, T, \
                               L->E, L->k, L->desc.norm_topk, L->ids, L->gates, L->counts, L->offsets, L->perm, \
                               L->gperm, L->active, L->n_active, reinterpret_cast<int4*>(L->slot_info),         \
-                              L->route_done)
+                              L->route_done, L->xexp, L->pexp)
     if (vpl <= 1) SCION_ROUTE_CTA(1);
     else if (vpl <= 2) SCION_ROUTE_CTA(2);
     else if (vpl <= 4) SCION_ROUTE_CTA(4);
@@ -339,7 +356,8 @@ cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s) {
   size_t smem = sizeof(float) * (size_t(kRouteThreads / 32) * L->E) + sizeof(int32_t) * (2 * size_t(L->E)) +
                 sizeof(int32_t) * size_t(T) * L->k;
   route_kernel<<<1, kRouteThreads, smem, s>>>(L->logits, T, L->E, L->k, L->desc.norm_topk, L->ids, L->gates,
-                                               L->counts, L->offsets, L->perm, L->gperm, L->active, L->n_active);
+                                               L->counts, L->offsets, L->perm, L->gperm, L->active, L->n_active,
+                                               L->xexp, L->pexp);
   if (cudaError_t e = cudaGetLastError()) return e;
   return launch_slot_info(L, s);
 }

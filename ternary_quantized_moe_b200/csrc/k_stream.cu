@@ -36,7 +36,7 @@ struct StageHdr {
   int ng;     // 128-column groups in this stage (1..GPS)
   int pos[kTok];     // routed positions of the pass's tokens (last stage only)
   int orow[kTok];    // output token row (entry / k)
-  float gate[kTok];  // gate of the entry (down: times 2^(-2 s_t), the hidden being h 2^(2 s_t))
+  float gate[kTok];  // gate of the entry times 2^(-2 s_t) (the hidden is h 2^(2 s_t))
   float xdn[kTok];   // gate/up: 2^-s_t and 2^s_t of the token's range exponent (the sums are of x 2^s_t)
   float xup[kTok];
 };
@@ -48,8 +48,8 @@ struct StreamArgs {
   int bld;             // 128-column groups per B row (Gd or GF)
   const int4* slot_info;
   const int32_t *n_active, *perm;
-  const float* gperm;  // gate of each routed position
-  const int32_t* xexp; // range exponent s_t of each token
+  const float* gperm;  // gate of each routed position, times 2^(-2 s_t)
+  const int32_t* pexp; // range exponent s_t of the token of each routed position
   int G, R, k, F, d, fmt;
   __half* hfrag;  // gate/up output
   float* out;     // down output
@@ -245,8 +245,8 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
       if (lane < min(kTok, si.z - pc)) {
         t.pos = si.y + pc + lane;
         t.orow = a.perm[t.pos] / a.k;
-        const int sh = a.xexp[t.orow];
-        t.gate = a.gperm[t.pos] * pow2i(-2 * sh);
+        const int sh = a.pexp[t.pos];
+        t.gate = a.gperm[t.pos];
         t.xdn = pow2i(-sh), t.xup = pow2i(sh);
         t.brow = NMAT == 2 ? t.orow : t.pos;
       }
@@ -458,7 +458,7 @@ cudaError_t launch_stream_gateup(const scion_layer* L, int T, cudaStream_t s) {
   StreamArgs a;
   a.bank = L->gu_bank, a.bsrc = L->xfrag, a.bld = L->Gd;
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
-  a.gperm = L->gperm, a.xexp = L->xexp, a.G = L->Gd, a.R = L->F, a.k = L->k, a.F = L->F, a.d = L->d, a.fmt = L->fmt;
+  a.gperm = L->gperm, a.pexp = L->pexp, a.G = L->Gd, a.R = L->F, a.k = L->k, a.F = L->F, a.d = L->d, a.fmt = L->fmt;
   a.hfrag = L->h, a.out = nullptr, a.err = L->err;
   const int max_items = min(L->E, T * L->k) * (L->F / 128);
   if (L->fmt == SCION_PQ2_0) return launch_stream<SCION_PQ2_0, 2>(a, max_items, s);
@@ -469,7 +469,7 @@ cudaError_t launch_stream_down(const scion_layer* L, int T, float* out, cudaStre
   StreamArgs a;
   a.bank = L->dn_bank, a.bsrc = L->h, a.bld = L->GF;
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
-  a.gperm = L->gperm, a.xexp = L->xexp, a.G = L->GF, a.R = L->d, a.k = L->k, a.F = L->F, a.d = L->d, a.fmt = L->fmt;
+  a.gperm = L->gperm, a.pexp = L->pexp, a.G = L->GF, a.R = L->d, a.k = L->k, a.F = L->F, a.d = L->d, a.fmt = L->fmt;
   a.hfrag = nullptr, a.out = out, a.err = L->err;
   const int max_items = min(L->E, T * L->k) * (L->d / 128);
   if (L->fmt == SCION_PQ2_0) return launch_stream<SCION_PQ2_0, 1>(a, max_items, s);

@@ -45,7 +45,7 @@ void free_layer(scion_layer* L) {
   void* ptrs[] = {L->gu_bank, L->dn_bank,  L->dense_down, L->xunits,  L->logits,    L->ids,       L->gates,
                   L->counts,  L->offsets,  L->perm,       L->active,  L->n_active,  L->h,         L->hz,
                   L->xfrag,   L->x_stage, L->out_stage, L->bad,       L->err,
-                  L->slot_info, L->gperm, L->route_done, L->xexp};
+                  L->slot_info, L->gperm, L->route_done, L->xexp, L->pexp, L->x16d, L->hp};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   if (L->side) cudaStreamDestroy(L->side);
@@ -54,7 +54,7 @@ void free_layer(scion_layer* L) {
   if (L->pre) {
     scion::PrefillState* P = L->pre;
     void* pp[] = {P->xunits, P->dunits, P->logits, P->ids, P->gates, P->counts, P->offsets, P->perm, P->inv,
-                  P->y, P->tiles, P->n_tiles, P->x16, P->h, P->hz, P->cursor, P->corr_a16, P->xexp, P->pexp};
+                  P->y, P->tiles, P->n_tiles, P->x16, P->h, P->hz, P->cursor, P->corr_a16, P->xexp, P->pexp, P->gperm};
     for (void* p : pp)
       if (p) cudaFree(p);
     delete P;
@@ -88,6 +88,7 @@ int create_prefill(scion_layer* L, cudaStream_t s) {
   PTRY(dev_alloc(L, &P->x16, sizeof(__half) * T * L->d));
   PTRY(dev_alloc(L, &P->xexp, sizeof(int32_t) * T));
   PTRY(dev_alloc(L, &P->pexp, sizeof(int32_t) * Tk));
+  PTRY(dev_alloc(L, &P->gperm, sizeof(float) * Tk));
   PTRY(dev_alloc(L, &P->h, sizeof(__half) * Tk * L->F));
   PTRY(dev_alloc(L, &P->hz, sizeof(__half) * T * (L->Kd ? L->Kd : 64)));
   PTRY(cudaMemsetAsync(P->hz, 0, sizeof(__half) * T * (L->Kd ? L->Kd : 64), s));
@@ -194,7 +195,8 @@ int forward_prefill(const scion_layer* L, const __nv_bfloat16* x, int T, float* 
   SCION_STAGE(SCION_STAGE_GATEUP, scion::launch_prefill_stage(SCION_STAGE_GATEUP, L, x, T, out, resid, s));
   SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_prefill_stage(SCION_STAGE_DOWN_DENSE, L, x, T, out, resid, s));
   SCION_STAGE(SCION_STAGE_DOWN_ROUTED, scion::launch_prefill_stage(SCION_STAGE_DOWN_ROUTED, L, x, T, out, resid, s));
-  SCION_STAGE(SCION_STAGE_COMBINE, scion::launch_prefill_stage(SCION_STAGE_COMBINE, L, x, T, out, resid, s));
+  if (L->deterministic)
+    SCION_STAGE(SCION_STAGE_COMBINE, scion::launch_prefill_stage(SCION_STAGE_COMBINE, L, x, T, out, resid, s));
   return SCION_OK;
 }
 
@@ -216,13 +218,14 @@ int forward_prefill(const scion_layer* L, const __nv_bfloat16* x, int T, float* 
 int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, const float* resid, cudaStream_t s) {
   if (L->desc.router_fp32) SCION_STAGE(SCION_STAGE_ROUTER_F32, scion::launch_router_f32(L, x, T, L->logits, s));
   const bool ring = T >= L->stream_min_tokens;
+  const bool tcd = ring && L->tc_decode;  // tcgen05 expert GEMMs instead of the bulk-copy ring kernels
   // Batches on the ring kernels split the dense work off the expert path: the caller's stream
   // runs the router part of the x-projection (with x's fragment rows and the clearing of out),
   // the layer's side stream the shared-expert / correction part and the dense down projection,
   // beside routing and the expert kernels; the caller's stream joins it at the end.
   const bool side = ring && L->Kdense;
   const int nx_main = side ? L->n_xrouter : L->n_xunits;
-  SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_xproj(L, x, T, out, resid, 0, nx_main, true, s));
+  SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_xproj(L, x, T, out, resid, 0, nx_main, true, tcd, s));
   int st = SCION_OK;
   if (side) {
     cudaError_t e = cudaEventRecord(L->ev_x, s);
@@ -232,7 +235,8 @@ int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out
     {
       cudaStream_t s = L->side;  // SCION_STAGE_INTO launches and records on `s`
       SCION_STAGE_INTO(st_side, SCION_STAGE_XPROJ,
-                       scion::launch_xproj(L, x, T, out, nullptr, L->n_xrouter, L->n_xunits - L->n_xrouter, false, s));
+                       scion::launch_xproj(L, x, T, out, nullptr, L->n_xrouter, L->n_xunits - L->n_xrouter, false,
+                                           false, s));
       SCION_STAGE_INTO(st_side, SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
     }
     // the join is recorded whatever happened above, so that no later work on the caller's stream
@@ -247,11 +251,13 @@ int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out
   // small batches: the dense down projection rides in the gate/up launch (it needs only the
   // x-projection), off the critical path of the routed kernels
   const bool merged = !ring && scion::gateup_merges_dense(L, T);
-  SCION_STAGE_INTO(st, SCION_STAGE_GATEUP, ring     ? scion::launch_stream_gateup(L, T, s)
+  SCION_STAGE_INTO(st, SCION_STAGE_GATEUP, tcd      ? scion::launch_tc_decode(2, L, T, out, s)
+                                           : ring   ? scion::launch_stream_gateup(L, T, s)
                                            : merged ? scion::launch_gateup_dense(L, T, out, s)
                                                     : scion::launch_gateup(L, x, T, s));
-  SCION_STAGE_INTO(st, SCION_STAGE_DOWN_ROUTED,
-                   ring ? scion::launch_stream_down(L, T, out, s) : scion::launch_down_routed(L, T, out, s));
+  SCION_STAGE_INTO(st, SCION_STAGE_DOWN_ROUTED, tcd    ? scion::launch_tc_decode(1, L, T, out, s)
+                                                : ring ? scion::launch_stream_down(L, T, out, s)
+                                                       : scion::launch_down_routed(L, T, out, s));
   if (side) {
     const cudaError_t e = cudaStreamWaitEvent(s, L->ev_dense, 0);
     return st != SCION_OK ? st : cuda_status(e);
@@ -303,6 +309,7 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   L->Kdense = L->Fs + L->r;
   L->Kd = (L->Kdense + 63) / 64 * 64;
   L->stream_min_tokens = 16;  // below this the few active experts spread better over the split-K kernels
+  L->tc_decode = 1;
   cudaStream_t s = as_stream(stream);
   const int tb = scion::tile_bytes(L->fmt);
   const int TD = SCION_TDEC;
@@ -338,6 +345,9 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   SCION_TRY(dev_alloc(L, &L->hz, sizeof(__half) * TD * (L->Kd ? L->Kd : 1)));
   SCION_TRY(dev_alloc(L, &L->xfrag, sizeof(__half) * TD * L->Gd * SCION_BROW));
   SCION_TRY(dev_alloc(L, &L->xexp, sizeof(int32_t) * TD));
+  SCION_TRY(dev_alloc(L, &L->pexp, sizeof(int32_t) * TD * L->k));
+  SCION_TRY(dev_alloc(L, &L->x16d, sizeof(__half) * TD * L->d));
+  SCION_TRY(dev_alloc(L, &L->hp, sizeof(__half) * TD * L->k * L->F));
   SCION_TRY(dev_alloc(L, &L->x_stage, sizeof(__nv_bfloat16) * size_t(max_tokens) * L->d));
   SCION_TRY(dev_alloc(L, &L->out_stage, sizeof(float) * size_t(max_tokens) * L->d));
   SCION_TRY(dev_alloc(L, &L->bad, sizeof(int64_t)));
@@ -374,6 +384,8 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
                                  L->gu_bank, L->bad, s));
   SCION_TRY(scion::launch_retile(L->fmt, static_cast<const uint8_t*>(desc->down_exps), L->E, L->d, L->GF, 1, 0,
                                  L->dn_bank, L->bad, s));
+  // B operand of the tcgen05 decode down projection: the hidden rows, 16-row TMA boxes
+  if ((st = scion::make_tmap_2d(&L->hp_map, L->hp, 0, int64_t(TD) * L->k, L->F, 16)) != SCION_OK) goto fail;
   if (max_tokens > SCION_TDEC) {
     st = create_prefill(L, s);
     if (st != SCION_OK) goto fail;
@@ -461,6 +473,8 @@ extern "C" int scion_moe_forward_debug(const void* x, int T, const scion_layer* 
   cp(dbg->perm, pre ? P->perm : L->perm, sizeof(int32_t) * size_t(T) * L->k);
   if (dbg->h && e == cudaSuccess)
     e = pre ? scion::launch_unperm_prefill(L->fmt, P->h, int64_t(T) * L->k * L->F, reinterpret_cast<__half*>(dbg->h), s)
+        : (T >= L->stream_min_tokens && L->tc_decode)
+            ? scion::launch_unperm_prefill(L->fmt, L->hp, int64_t(T) * L->k * L->F, reinterpret_cast<__half*>(dbg->h), s)
             : scion::launch_unfrag(L->fmt, L->h, T * L->k, L->GF, reinterpret_cast<__half*>(dbg->h), s);
   if (dbg->hz && e == cudaSuccess && L->Kdense)
     e = cudaMemcpy2DAsync(dbg->hz, sizeof(__half) * L->Kdense, pre ? P->hz : L->hz, sizeof(__half) * L->Kd,
@@ -539,6 +553,14 @@ extern "C" int scion_layer_set_option(scion_layer* L, int option, int value) {
     case SCION_OPT_STREAM_MIN_TOKENS:
       if (value < 1) return SCION_EINVAL;
       L->stream_min_tokens = value;
+      return SCION_OK;
+    case SCION_OPT_DECODE_TC:
+      if (value != 0 && value != 1) return SCION_EINVAL;
+      L->tc_decode = value;
+      return SCION_OK;
+    case SCION_OPT_DETERMINISTIC:
+      if (value != 0 && value != 1) return SCION_EINVAL;
+      L->deterministic = value;
       return SCION_OK;
     default:
       return SCION_EINVAL;

@@ -83,6 +83,7 @@ struct PrefillState {
   __half* x16;          // [maxT][d]   x 2^s_t in the container column order (fp16)
   int32_t* xexp;        // [maxT] per-token range exponent s_t (see token_shift)
   int32_t* pexp;        // [maxT*k] s_t of the token of each routed position
+  float* gperm;         // [maxT*k] gate of the entry at each routed position, times 2^(-2 s_t)
   __half* h;            // [maxT*k][F] expert SwiGLU hidden, container column order
   __half* hz;           // [maxT][Kd]
 };
@@ -110,7 +111,7 @@ struct scion_layer {
   int32_t* counts;   // [E]
   int32_t* offsets;  // [E+1]
   int32_t* perm;     // [TDEC*k]
-  float* gperm;      // [TDEC*k] gate of the entry at each routed position
+  float* gperm;      // [TDEC*k] gate of the entry at each routed position, times 2^(-2 s_t)
   int32_t* active;   // [E]
   int32_t* n_active; // [1]
   void* slot_info;    // int4 [E]: {expert, first position, token count, 0} per active slot
@@ -119,6 +120,14 @@ struct scion_layer {
   __half* hz;        // [TDEC][Kd] (pad columns stay 0)
   __half* xfrag;     // [TDEC][Gd][SCION_BROW] x in fragment order (fp16) + group-sum tails
   int32_t* xexp;     // [TDEC] per-token range exponent s_t (see token_shift)
+  int32_t* pexp;     // [TDEC*k] s_t of the token of each routed position (written by the routing)
+  // tensor-core decode (batches on the ring threshold and above, tc_decode = 1): x 2^s_t in the
+  // tcgen05 column order, the expert hidden one row per routed position, and its TMA map (16-row boxes)
+  __half* x16d;      // [TDEC][d]
+  __half* hp;        // [TDEC*k][F]
+  CUtensorMap hp_map;
+  int tc_decode;     // 1 (default): decode batches of stream_min_tokens and more run the tcgen05 expert GEMMs
+  int deterministic; // 1: the prefill down projection writes one row per routed entry and a combine sums them in slot order
   void* x_stage;     // [max_tokens][d] bf16 (host-buffer forward)
   float* out_stage;  // [max_tokens][d]
   int64_t* bad;      // [1] invalid-code counter used at create
@@ -155,8 +164,10 @@ cudaError_t launch_slot_info(const scion_layer* L, cudaStream_t s);
 // Units [unit0, unit0 + n_units) of the layer's x-projection table (router units first, then
 // shared gate/up, then correction A); `aux` adds the CTAs that write x's fragment rows and
 // clear out and the hidden's group-sum tails.
+// x16 = true: the aux CTAs write x for the tcgen05 decode kernels (L->x16d) instead of the
+// fragment-ordered rows of the register kernels.
 cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, const float* resid,
-                         int unit0, int n_units, bool aux, cudaStream_t s);
+                         int unit0, int n_units, bool aux, bool x16, cudaStream_t s);
 cudaError_t launch_gateup(const scion_layer* L, const __nv_bfloat16* x, int T, cudaStream_t s);
 cudaError_t launch_down_routed(const scion_layer* L, int T, float* out, cudaStream_t s);
 cudaError_t launch_down_dense(const scion_layer* L, int T, float* out, cudaStream_t s);
@@ -173,6 +184,9 @@ cudaError_t launch_stream_down(const scion_layer* L, int T, float* out, cudaStre
 
 // k_prefill.cu
 int make_tmap_2d(CUtensorMap* map, const void* ptr, int bf16, int64_t rows, int64_t K, int box_rows = 128);
+// Expert gate/up (na = 2) or down (na = 1, gate-weighted fp32 reductions into out) of a decode
+// batch on the tcgen05 grouped GEMM, one tile per active expert.
+cudaError_t launch_tc_decode(int na, const scion_layer* L, int T, float* out, cudaStream_t s);
 cudaError_t configure_prefill_kernels();
 size_t prefill_unit_bytes();
 size_t prefill_tile_bytes();

@@ -204,15 +204,20 @@ def test_forward_variants(variant):
     check_output(got, ref)
 
 
+@pytest.mark.parametrize("tc", [0, 1])
 @pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
 @pytest.mark.parametrize("T,E,k", [(1, 16, 4), (5, 16, 4), (13, 16, 4), (64, 16, 4), (64, 4, 2), (37, 6, 3)])
-def test_forward_stream_kernels(fmt, T, E, k):
-    """The persistent bulk-copy ring expert kernels (selected with SCION_OPT_STREAM_MIN_TOKENS):
-    stage by stage against the oracle, including experts with more than one 8-token pass."""
+def test_forward_stream_kernels(tc, fmt, T, E, k):
+    """The persistent expert kernels of decode batches (selected for every batch size with
+    SCION_OPT_STREAM_MIN_TOKENS = 1): tc = 1 the tcgen05 grouped GEMMs (one tile per active
+    expert, 16-row boxes of the hidden, gate-weighted reductions into out), tc = 0 the mma.sync
+    kernels fed by a bulk-copy ring (experts with more than one 8-token pass); stage by stage
+    against the oracle, experts with up to 64 tokens (E = 4, k = 2)."""
     cfg = small("st", fmt, False, E=E, k=k)
     L, banks, ol, x = _case(cfg, T)
     layer = device_layer(cfg, L, banks, 64)
     tq.scion_layer_set_option(layer, tq.SCION_OPT_STREAM_MIN_TOKENS, 1)
+    tq.scion_layer_set_option(layer, tq.SCION_OPT_DECODE_TC, tc)
     got, dbg = run_forward(layer, x, T, debug=True, E=cfg.n_experts, k=cfg.top_k, F=cfg.ffn,
                            Kdense=cfg.shared_ffn + cfg.rank)
     _check_routing(cfg, dbg, ol, x, T)
@@ -566,6 +571,27 @@ def test_prefill_multi_tile_experts(fmt, T):
     _check_routing(cfg, dbg, ol, x, T, stable=False)
     ref, _, _ = oracle.forward(ol, x)
     check_output(got, ref)
+
+
+@pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
+@pytest.mark.parametrize("dense", [True, False])
+def test_prefill_deterministic_combine(fmt, dense):
+    """Both ways of adding the routed rows on the tensor-core path: fused fp32 reductions into out
+    (default) and, with SCION_OPT_DETERMINISTIC, one fp16 row per entry summed in slot order by
+    the combine kernel, which repeats bit for bit; with and without the dense down projection
+    (without it out starts from zero, set by the x conversion or by the combine)."""
+    cfg = small("dc", fmt, False, E=16, k=4, Fs=128 if dense else 0, r=16 if dense else 0)
+    T = 300
+    L, banks, ol, x = _case(cfg, T)
+    layer = device_layer(cfg, L, banks, T)
+    ref, _, _ = oracle.forward(ol, x)
+    fused, _ = run_forward(layer, x, T)
+    check_output(fused, ref)
+    tq.scion_layer_set_option(layer, tq.SCION_OPT_DETERMINISTIC, 1)
+    d1, _ = run_forward(layer, x, T)
+    d2, _ = run_forward(layer, x, T)
+    check_output(d1, ref)
+    np.testing.assert_array_equal(d1, d2)
 
 
 def test_prefill_matches_decode_passes():
