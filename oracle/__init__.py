@@ -105,6 +105,8 @@ def _load():
             lib.oracle_f64_to_f16_nonneg.argtypes = [C.c_double]
             lib.oracle_quantize.restype = ci
             lib.oracle_quantize.argtypes = [ci, vp, i64, ci, vp, vp]
+            lib.oracle_attn_corr.restype = ci
+            lib.oracle_attn_corr.argtypes = [ci, ci, ci, ci, vp, vp, vp, ci, vp, vp, vp]
             _lib = lib
     return _lib
 
@@ -326,6 +328,27 @@ def corr(layer: OracleLayer, x: np.ndarray):
     if st != OK:
         raise RuntimeError("oracle_corr: %d" % st)
     return z, y
+
+
+def attn_corr(v: np.ndarray, a: np.ndarray, b: np.ndarray, d_in: int, d_out: int, rank: int, packed: int = 0,
+              base: Optional[np.ndarray] = None):
+    """The correction branch on the attention output ("Scion: ternary MoE quantization with trained
+    corrections", The idea and Findings): z = A v, out = base + B z.  v: bf16 bits [T, d_in];
+    a, b: bf16 bits [rank, d_in] / [d_out, rank] or (packed) PQ2_0 blocks; base fp64 [T, d_out] or
+    None.  Returns (out fp64 [T, d_out], z fp64 [T, rank])."""
+    v = np.ascontiguousarray(v, dtype=np.uint16)
+    assert v.ndim == 2 and v.shape[1] == d_in
+    T = v.shape[0]
+    a = np.ascontiguousarray(a)
+    b = np.ascontiguousarray(b)
+    out = np.empty((T, d_out), np.float64)
+    z = np.empty((T, rank), np.float64)
+    bs = None if base is None else np.ascontiguousarray(base, dtype=np.float64)
+    st = _load().oracle_attn_corr(d_in, d_out, rank, int(packed), _ptr(a), _ptr(b), _ptr(v), T, _ptr(bs), _ptr(out),
+                                  _ptr(z))
+    if st != OK:
+        raise RuntimeError("oracle_attn_corr: %d" % st)
+    return out, z
 
 
 ABSMEAN = 0

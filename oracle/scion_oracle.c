@@ -703,3 +703,66 @@ int oracle_quantize(int method, const float* w, int64_t n_groups, int iters, int
   }
   return ORACLE_OK;
 }
+
+/*
+ * The correction branch on the attention output ("Scion: ternary MoE quantization with trained
+ * corrections", The idea: rank-512 branches on the attention output and on the MoE block output;
+ * Findings: the attention-output branch ships as a standard low-rank adapter on the attention
+ * output projection).  Reading: the branch takes that projection's input v (d_in wide) and adds
+ * its low-rank product to the projection's output (d_out wide), scale 1 (any alpha / r folded into
+ * B), on top of a given base (the projection's output, or the residual stream it joins):
+ *   z = A v,   out[t] = base[t] + B z
+ * v: bf16 [T][d_in]; A, B: bf16 [r][d_in] and [d_out][r], or (packed = 1) PQ2_0 blocks
+ * [r][d_in/128] and [d_out][r/128] decoded by oracle_dequant_row; base: fp64 [T][d_out] or NULL
+ * (zero); out: fp64 [T][d_out]; z_out: fp64 [T][r] or NULL.
+ */
+int oracle_attn_corr(int d_in, int d_out, int r, int packed, const void* A, const void* B, const uint16_t* v, int T,
+                     const double* base, double* out, double* z_out) {
+  if (d_in <= 0 || d_out <= 0 || r <= 0 || T < 0 || !A || !B || !out) return ORACLE_EINVAL;
+  if (packed && (d_in % 128 || r % 128)) return ORACLE_EINVAL;
+  double* a = (double*)malloc(sizeof(double) * (size_t)r * d_in);
+  double* b = (double*)malloc(sizeof(double) * (size_t)d_out * r);
+  if (!a || !b) {
+    free(a), free(b);
+    return ORACLE_ENOMEM;
+  }
+  int status = ORACLE_OK;
+  for (int q = 0; q < r && status == ORACLE_OK; q++) {
+    if (packed)
+      status = oracle_dequant_row(ORACLE_PQ2_0, (const uint8_t*)A + (long)q * (d_in / 128) * 34, d_in, a + (long)q * d_in);
+    else
+      for (int i = 0; i < d_in; i++) a[(long)q * d_in + i] = oracle_bf16_to_f64(((const uint16_t*)A)[(long)q * d_in + i]);
+  }
+  for (int i = 0; i < d_out && status == ORACLE_OK; i++) {
+    if (packed)
+      status = oracle_dequant_row(ORACLE_PQ2_0, (const uint8_t*)B + (long)i * (r / 128) * 34, r, b + (long)i * r);
+    else
+      for (int q = 0; q < r; q++) b[(long)i * r + q] = oracle_bf16_to_f64(((const uint16_t*)B)[(long)i * r + q]);
+  }
+  if (status == ORACLE_OK) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int t = 0; t < T; t++) {
+      double* vv = (double*)malloc(sizeof(double) * d_in);
+      double* z = (double*)malloc(sizeof(double) * r);
+      if (!vv || !z) {
+        status = ORACLE_ENOMEM;
+      } else {
+        for (int i = 0; i < d_in; i++) vv[i] = oracle_bf16_to_f64(v[(long)t * d_in + i]);
+        for (int q = 0; q < r; q++) {
+          double s = 0.0;
+          for (int i = 0; i < d_in; i++) s += a[(long)q * d_in + i] * vv[i];
+          z[q] = s;
+          if (z_out) z_out[(long)t * r + q] = s;
+        }
+        for (int i = 0; i < d_out; i++) {
+          double s = 0.0;
+          for (int q = 0; q < r; q++) s += b[(long)i * r + q] * z[q];
+          out[(long)t * d_out + i] = (base ? base[(long)t * d_out + i] : 0.0) + s;
+        }
+      }
+      free(vv), free(z);
+    }
+  }
+  free(a), free(b);
+  return status;
+}
