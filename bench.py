@@ -72,10 +72,11 @@ def parse():
                     help="ternary correction factors (PQ2_0 blocks) instead of the workload's bf16 ones")
     ap.add_argument("--stream-min-tokens", type=int, default=0,
                     help="decode batches of at least this many tokens use the persistent expert kernels")
-    ap.add_argument("--decode-tc", type=int, default=1, choices=[0, 1],
+    ap.add_argument("--decode-tc", type=int, default=0, choices=[0, 1],
                     help="1: tcgen05 expert GEMMs for those batches, 0: the mma.sync bulk-copy ring kernels")
-    ap.add_argument("--deterministic", action="store_true",
-                    help="prefill: per-entry rows summed in slot order instead of fp32 reductions into out")
+    ap.add_argument("--prefill-reduce", action="store_true",
+                    help="prefill: fp32 reductions into out from the down projection instead of per-entry rows "
+                         "summed in slot order")
     return ap.parse_args()
 
 
@@ -310,7 +311,7 @@ def workload_config(cfg, args, n_layers=None, weight_bytes=None):
          "shared_ffn": cfg.shared_ffn, "rank": cfg.rank, "format": "PQ2_0" if cfg.fmt == 0 else "PTQ1_0",
          "correction": "PQ2_0 blocks" if args.packed_corr else "bf16", "batches": list(cfg.tokens),
          "decode_expert_kernels": "tcgen05" if args.decode_tc else "mma.sync ring",
-         "prefill_combine": "slot-order rows" if args.deterministic else "fp32 reductions",
+         "prefill_combine": "fp32 reductions" if args.prefill_reduce else "slot-order rows",
          "tokens_per_step": sum(cfg.tokens)}
     if cfg.zipf_s is not None:
         c["router_load"] = "Zipf(%.1f) over a seeded permutation of the experts" % cfg.zipf_s
@@ -352,8 +353,8 @@ def build_layers(cfg, args, dev, n_layers, max_T):
         if args.stream_min_tokens:
             tq.scion_layer_set_option(layers[-1], tq.SCION_OPT_STREAM_MIN_TOKENS, args.stream_min_tokens)
         tq.scion_layer_set_option(layers[-1], tq.SCION_OPT_DECODE_TC, args.decode_tc)
-        if args.deterministic:
-            tq.scion_layer_set_option(layers[-1], tq.SCION_OPT_DETERMINISTIC, 1)
+        if args.prefill_reduce:
+            tq.scion_layer_set_option(layers[-1], tq.SCION_OPT_DETERMINISTIC, 0)
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     return layers

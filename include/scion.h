@@ -222,12 +222,14 @@ int scion_moe_forward_residual(const void* x, int T, const scion_layer* layer, c
  *    most 64) run the expert GEMMs on persistent kernels (128 expert rows per work item);
  *    smaller batches split K over the warps of one CTA per 16 rows, which spreads the few
  *    active experts over more SMs.
- *  SCION_OPT_DECODE_TC (default 1): those persistent kernels are the tcgen05 grouped GEMMs
- *    (codes expanded into tensor memory, one tile per active expert, the down projection adding
- *    its gate-weighted rows into out); 0 selects the mma.sync kernels fed by a bulk-copy ring.
- *  SCION_OPT_DETERMINISTIC (default 0): 1 makes batches above 64 tokens bit-reproducible: the
- *    down projection writes one fp16 row per routed entry and a combine kernel sums each token's
- *    rows in slot order, instead of fp32 reductions into out in whatever order they land.
+ *  SCION_OPT_DECODE_TC (default 0): 0 runs those persistent kernels as mma.sync kernels fed by a
+ *    bulk-copy ring; 1 as the tcgen05 grouped GEMMs of the large batches (codes expanded into
+ *    tensor memory, one tile per active expert, the down projection adding its gate-weighted rows
+ *    into out), measured slower at decode sizes.
+ *  SCION_OPT_DETERMINISTIC (default 1): batches above 64 tokens are bit-reproducible: the down
+ *    projection writes one fp16 row per routed entry and a combine kernel sums each token's rows
+ *    in slot order.  0: the down projection adds its rows into out with fp32 reductions (no row
+ *    buffer, order of the additions not fixed).
  *    All settings give the same result up to fp32 summation order.
  * EINVAL for an unknown option or an out-of-range value. */
 enum { SCION_OPT_STREAM_MIN_TOKENS = 1, SCION_OPT_DECODE_TC = 2, SCION_OPT_DETERMINISTIC = 3 };
@@ -272,6 +274,44 @@ int scion_moe_forward_debug(const void* x, int T, const scion_layer* layer, floa
  * a misaligned x or T out of range; ECUDA if a launch or copy fails. */
 int scion_debug_route(const void* x, int T, const scion_layer* layer, int32_t* ids, float* gates, int32_t* offsets,
                       int32_t* perm, void* stream);
+
+/* ------------------------------------------ correction branch on the attention output
+ * The second correction branch of the method ("Scion: ternary MoE quantization with trained
+ * corrections", The idea: rank-512 branches on the attention output and on the MoE block output;
+ * Findings: the attention-output branch ships as a standard low-rank adapter on the attention
+ * output projection; "Scion-35B-A3B" model card, Weight Representation: the corrections ship as
+ * 2-bit codes plus one fp16 scale per 128).  The branch takes the input v of the attention
+ * output projection (the attention heads' concatenated output, d_in wide) and adds its low-rank
+ * product to the projection's output (d_out wide), scale 1:
+ *   out[t] = base[t] + B (A v_t)
+ * The attention itself and its output projection are the caller's; base is typically that
+ * projection's output, or the residual stream with it already added.
+ *   packed = 0: corr_a bf16 [rank][d_in], corr_b bf16 [d_out][rank], 16-byte aligned, read in place
+ *              (they must outlive the handle; a fp16 copy of B is made);
+ *   packed = 1: PQ2_0 blocks, corr_a [rank][d_in/128], corr_b [d_out][rank/128] (groups of 128
+ *              along each factor's reduction axis), 2-byte aligned; rank a multiple of 128.
+ * Limits: d_in a multiple of 128 and <= 4096, d_out a multiple of 128, rank a multiple of 16 and
+ * <= 4096.  EINVAL on a bad descriptor, EFORMAT on an invalid code (packed), ENOMEM, ECUDA.
+ * Batches of up to 64 tokens run split-K weight-streaming kernels, larger ones (handles created
+ * with max_tokens > 64) tcgen05 GEMMs. */
+typedef struct {
+  int d_in, d_out, rank;
+  int packed;
+  const void* corr_a;
+  const void* corr_b;
+} scion_corr_desc;
+typedef struct scion_corr scion_corr;
+int scion_corr_create(const scion_corr_desc* desc, int max_tokens, void* stream, scion_corr** out);
+void scion_corr_destroy(scion_corr* corr);
+size_t scion_corr_device_bytes(const scion_corr* corr);
+/* v: device bf16 [T][d_in]; base: device fp32 [T][d_out] or NULL (zero), may equal out; out:
+ * device fp32 [T][d_out], written; all 16-byte aligned.  0 <= T <= max_tokens.  Activations get
+ * the same per-token power-of-two range scaling as scion_moe_forward.  Calls on one handle must
+ * not overlap on the GPU.  EINVAL on a null or misaligned pointer or T out of range; ECUDA. */
+int scion_corr_forward(const void* v, int T, const scion_corr* corr, const float* base, float* out, void* stream);
+/* Waits for `stream`, then returns and clears the handle's device status word (SCION_ETIMEOUT if
+ * a bounded wait of the tensor-core path gave up), like scion_layer_check. */
+int scion_corr_check(const scion_corr* corr, void* stream);
 
 /* ------------------------------------------------------------ measurement
  * Kernel-level timing for benchmarks.  Between scion_profile_begin and

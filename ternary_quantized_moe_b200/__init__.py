@@ -29,7 +29,7 @@ __all__ = [
     "scion_router_logits_static", "scion_layer_set_option", "SCION_OPT_STREAM_MIN_TOKENS", "SCION_OPT_DECODE_TC",
     "SCION_OPT_DETERMINISTIC",
     "scion_moe_forward_residual", "scion_quantize_device", "SCION_QUANT_ABSMEAN", "SCION_QUANT_LLOYD",
-    "scion_selftest_bounded_wait", "scion_debug_route",
+    "scion_selftest_bounded_wait", "scion_debug_route", "scion_corr_create", "scion_corr_forward", "Corr",
 ]
 
 SCION_PQ2_0 = 0
@@ -48,7 +48,8 @@ EXPORTS = (
     "scion_layer_device_bytes", "scion_moe_forward", "scion_moe_forward_host", "scion_moe_forward_debug",
     "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "scion_layer_check",
     "scion_router_logits_static", "scion_layer_set_option", "scion_moe_forward_residual", "scion_quantize_device",
-    "scion_selftest_bounded_wait", "scion_debug_route",
+    "scion_selftest_bounded_wait", "scion_debug_route", "scion_corr_create", "scion_corr_destroy",
+    "scion_corr_device_bytes", "scion_corr_forward", "scion_corr_check",
 )
 SCION_QUANT_ABSMEAN, SCION_QUANT_LLOYD = 0, 1
 SCION_OPT_STREAM_MIN_TOKENS, SCION_OPT_DECODE_TC, SCION_OPT_DETERMINISTIC = 1, 2, 3
@@ -72,6 +73,11 @@ class _Desc(C.Structure):
         ("sh_gate_vec", C.c_void_p), ("corr_a", C.c_void_p), ("corr_b", C.c_void_p),
         ("corr_packed", C.c_int),
     ]
+
+
+class _CorrDesc(C.Structure):
+    _fields_ = [("d_in", C.c_int), ("d_out", C.c_int), ("rank", C.c_int), ("packed", C.c_int),
+                ("corr_a", C.c_void_p), ("corr_b", C.c_void_p)]
 
 
 class _Debug(C.Structure):
@@ -110,6 +116,11 @@ def _load():
             "scion_moe_forward_host": (ci, [vp, ci, vp, vp, vp]),
             "scion_moe_forward_debug": (ci, [vp, ci, vp, vp, C.POINTER(_Debug), vp]),
             "scion_debug_route": (ci, [vp, ci, vp, vp, vp, vp, vp, vp]),
+            "scion_corr_create": (ci, [C.POINTER(_CorrDesc), ci, vp, C.POINTER(vp)]),
+            "scion_corr_destroy": (None, [vp]),
+            "scion_corr_device_bytes": (C.c_size_t, [vp]),
+            "scion_corr_forward": (ci, [vp, ci, vp, vp, vp, vp]),
+            "scion_corr_check": (ci, [vp, vp]),
             "scion_profile_begin": (ci, [ci]),
             "scion_profile_end": (ci, [ci, C.POINTER(C.c_double), C.POINTER(C.c_int64)]),
             "scion_kernel_launches": (C.c_int64, []),
@@ -390,6 +401,51 @@ def scion_debug_route(x, T: int, layer: Layer, ids=None, gates=None, offsets=Non
                                    _dptr(offsets, "offsets", (torch.int32,)), _dptr(perm, "perm", (torch.int32,)),
                                    _stream(stream))
     _check(st, "scion_debug_route")
+
+
+# ------------------------------------------ correction branch on the attention output
+class Corr:
+    """Handle of the correction branch on the attention output (scion_corr_*).  Keeps the
+    factor tensors alive for the handle's lifetime."""
+
+    def __init__(self, handle: int, d_in: int, d_out: int, keep):
+        self.handle, self.d_in, self.d_out, self._keep = handle, d_in, d_out, keep
+
+    def close(self):
+        if self.handle:
+            _load().scion_corr_destroy(C.c_void_p(self.handle))
+            self.handle = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def scion_corr_create(d_in: int, d_out: int, rank: int, corr_a, corr_b, packed: int = 0, max_tokens: int = 64,
+                      stream=None) -> Corr:
+    """corr_a / corr_b: bf16 CUDA [rank, d_in] / [d_out, rank], or (packed = 1) uint8 CUDA PQ2_0 blocks."""
+    D = _CorrDesc()
+    D.d_in, D.d_out, D.rank, D.packed = int(d_in), int(d_out), int(rank), int(packed)
+    D.corr_a, D.corr_b = _dptr(corr_a, "corr_a"), _dptr(corr_b, "corr_b")
+    h = C.c_void_p()
+    _check(_load().scion_corr_create(C.byref(D), int(max_tokens), _stream(stream), C.byref(h)), "scion_corr_create")
+    return Corr(h.value, d_in, d_out, (corr_a, corr_b))
+
+
+def scion_corr_forward(v, T: int, corr: Corr, out, base=None, stream=None) -> None:
+    """out = base + B (A v): v bf16 CUDA [T, d_in]; base / out fp32 CUDA [T, d_out] (base optional)."""
+    import torch
+
+    st = _load().scion_corr_forward(_dptr(v, "v", (torch.bfloat16,)), int(T), C.c_void_p(corr.handle),
+                                    _dptr(base, "base", (torch.float32,)), _dptr(out, "out", (torch.float32,)),
+                                    _stream(stream))
+    _check(st, "scion_corr_forward")
+
+
+def scion_corr_check(corr: Corr, stream=None) -> int:
+    return int(_load().scion_corr_check(C.c_void_p(corr.handle), _stream(stream)))
 
 
 # ------------------------------------------------------------ measurement

@@ -20,6 +20,7 @@
 // enter the MMA as exact fp16 {-1,0,+1}; each 128-column group accumulates separately
 // and is scaled by its fp16 group scale in fp32.
 #include <math.h>
+#include <string.h>
 
 #include "scion_internal.cuh"
 #include "tc_order.cuh"
@@ -48,6 +49,8 @@ struct XProjArgs {
   const uint8_t* corr_blocks;  // ternary correction A (PQ2_0 blocks [r][d/128]) or nullptr (bf16 corr_a)
   float* out;     // set here to the residual (or zero)
   const float* resid;  // nullptr: out starts at zero; may equal out (then out is left as it is)
+  int z_only;          // the correction branch alone: z rows scaled by 2^s_t (not hz_shift), and the
+                       // lead CTA of unit 0 writes each token's s_t to xexp
 };
 
 // One CTA = (unit, 512-column chunk); 8 warps x 64 columns.  NT = token tiles of 8.  The
@@ -318,7 +321,9 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
       uint32_t m = tmax[t];
       for (int ch = 1; ch < a.n_chunks; ++ch)
         m = max(m, ld_dsmem_u32(map_cluster_rank(smem_addr(&tmax[t]), ch)));
-      tshift[t] = hz_shift(token_shift(m), a.r > 0);
+      const int sh = token_shift(m);
+      tshift[t] = a.z_only ? sh : hz_shift(sh, a.r > 0);
+      if (a.z_only && blockIdx.x == 0) a.xexp[t] = sh;
     }
     __syncthreads();
   }
@@ -399,6 +404,9 @@ __device__ __forceinline__ void gateup_body(const GateUpArgs& a, int slot, int f
     const int nn = min(8, ne - pc);
     const int n = lane >> 2;
     const int tok = n < nn ? a.perm[p0 + pc + n] / a.k : -1;
+    // the epilogue thread's token column is fixed: fetch its range exponent before the MMAs
+    const int tcol_e = 2 * ((threadIdx.x >> 2) & 3) + (threadIdx.x & 1);
+    const int sh_e = threadIdx.x < 128 && tcol_e < nn ? a.pexp[p0 + pc + tcol_e] : 0;
     float tg[4] = {0.f, 0.f, 0.f, 0.f}, tu[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int i = 0; i < GPW; ++i) {
@@ -423,8 +431,7 @@ __device__ __forceinline__ void gateup_body(const GateUpArgs& a, int slot, int f
         const int f = ft * 16 + row;
         const int64_t pos = p0 + pc + tcol;
         const int idx = brow_pos(a.fmt, f & 127);
-        const int sh = a.pexp[pos];  // the sums are of x 2^sh
-        float h = silu_f(gs * pow2i(-sh)) * (us * pow2i(sh));
+        float h = silu_f(gs * pow2i(-sh_e)) * (us * pow2i(sh_e));  // the sums are of x 2^sh_e
         if (a.fmt == SCION_PQ2_0) h *= brow_bscale(idx);
         a.hfrag[(pos * GF + (f >> 7)) * SCION_BROW + idx] = __float2half_rn(h);
       }
@@ -518,6 +525,7 @@ struct DenseArgs {
   const uint8_t* corr_b;
   int Fs, r;
   const int32_t* xexp;  // [T] range exponent of each token: hz rows hold 2^hz_shift(s_t, r > 0) times their values
+  int z_only;           // hz holds z 2^s_t alone (the correction branch on the attention output)
 };
 
 constexpr int kDnKc = 256;            // K columns per CTA
@@ -606,7 +614,9 @@ __device__ __forceinline__ void dense_body(const DenseArgs& a, int bx, int by) {
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) v += red[(((h + 2 * ks) * NT + nt) * 32 + ln) * 4 + i];
     const int row = bx * 32 + 16 * h + (ln >> 2) + 8 * (i >> 1), tok = nt * 8 + 2 * (ln & 3) + (i & 1);
-    if (tok < a.T) atomicAdd(&a.out[int64_t(tok) * a.d + row], v * pow2i(-hz_shift(a.xexp[tok], a.r > 0)));
+    if (tok < a.T)
+      atomicAdd(&a.out[int64_t(tok) * a.d + row],
+                v * pow2i(a.z_only ? -a.xexp[tok] : -hz_shift(a.xexp[tok], a.r > 0)));
   }
 }
 
@@ -662,6 +672,7 @@ cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, fl
   a.units = L->xunits + unit0, a.n_units = n_units, a.n_chunks = L->n_xchunks, a.n_aux = aux ? kXAux : 0;
   a.logits = L->logits, a.hz = L->hz, a.xfrag = L->xfrag, a.xexp = L->xexp, a.out = out;
   a.x16 = x16 ? L->x16d : nullptr;
+  a.z_only = 0;
   a.corr_blocks = L->desc.corr_packed ? static_cast<const uint8_t*>(L->desc.corr_a) : nullptr;
   a.h = L->h, a.k = L->k, a.GF = L->GF;
   if (n_units + a.n_aux == 0) return cudaSuccess;
@@ -714,7 +725,7 @@ cudaError_t launch_gateup_dense(const scion_layer* L, int T, float* out, cudaStr
   DenseArgs b;
   b.w = L->dense_down, b.hz = L->hz, b.d = L->d, b.Kd = L->Kd, b.T = T, b.out = out;
   b.corr_b = L->desc.corr_packed ? static_cast<const uint8_t*>(L->desc.corr_b) : nullptr, b.Fs = L->Fs, b.r = L->r;
-  b.xexp = L->xexp;
+  b.xexp = L->xexp, b.z_only = 0;
   const int slots = min(L->E, T * L->k);
   const int gx = L->F / 16, dense_x = L->d / 32;
   const int dense_tiles = dense_x * ((L->Kd + kDnKc - 1) / kDnKc);
@@ -767,7 +778,7 @@ cudaError_t launch_down_dense(const scion_layer* L, int T, float* out, cudaStrea
   DenseArgs b;
   b.w = L->dense_down, b.hz = L->hz, b.d = L->d, b.Kd = L->Kd, b.T = T, b.out = out;
   b.corr_b = L->desc.corr_packed ? static_cast<const uint8_t*>(L->desc.corr_b) : nullptr, b.Fs = L->Fs, b.r = L->r;
-  b.xexp = L->xexp;
+  b.xexp = L->xexp, b.z_only = 0;
   const int nt = (T + 7) / 8;
   const dim3 g2(L->d / 32, (L->Kd + kDnKc - 1) / kDnKc);
   switch (nt) {
@@ -777,6 +788,39 @@ cudaError_t launch_down_dense(const scion_layer* L, int T, float* out, cudaStrea
     default: return launch_pdl(down_dense_kernel<8>, g2, dim3(256), down_dense_smem<8>(), s, b);
   }
   return cudaGetLastError();
+}
+
+cudaError_t launch_corr_z(const CorrState* C, const __nv_bfloat16* v, int T, cudaStream_t s) {
+  XProjArgs a;
+  memset(&a, 0, sizeof(a));
+  a.x = v, a.T = T, a.d = C->d_in, a.E = 0, a.Fs = 0, a.r = C->r, a.Kd = C->Kd, a.fmt = SCION_PQ2_0;
+  a.corr_a = static_cast<const __nv_bfloat16*>(C->a);
+  a.corr_blocks = C->packed ? static_cast<const uint8_t*>(C->a) : nullptr;
+  a.units = C->xunits, a.n_units = C->n_xunits, a.n_chunks = C->n_xchunks, a.n_aux = 0;
+  a.hz = C->hz, a.xexp = C->xexp, a.z_only = 1;
+  const dim3 grid(C->n_xunits, C->n_xchunks), cluster(1, C->n_xchunks, 1);
+  switch ((T + 7) / 8) {
+    case 1: return launch_pdl_cluster(xproj_kernel<1>, grid, dim3(kXThreads), cluster, xproj_smem<1>(T), s, a);
+    case 2: return launch_pdl_cluster(xproj_kernel<2>, grid, dim3(kXThreads), cluster, xproj_smem<2>(T), s, a);
+    case 3: case 4:
+      return launch_pdl_cluster(xproj_kernel<4>, grid, dim3(kXThreads), cluster, xproj_smem<4>(T), s, a);
+    default: return launch_pdl_cluster(xproj_kernel<8>, grid, dim3(kXThreads), cluster, xproj_smem<8>(T), s, a);
+  }
+}
+
+cudaError_t launch_corr_out(const CorrState* C, int T, float* out, cudaStream_t s) {
+  DenseArgs b;
+  memset(&b, 0, sizeof(b));
+  b.w = C->b16, b.hz = C->hz, b.d = C->d_out, b.Kd = C->Kd, b.T = T, b.out = out;
+  b.corr_b = C->packed ? static_cast<const uint8_t*>(C->b) : nullptr, b.Fs = 0, b.r = C->r;
+  b.xexp = C->xexp, b.z_only = 1;
+  const dim3 g2(C->d_out / 32, (C->Kd + kDnKc - 1) / kDnKc);
+  switch ((T + 7) / 8) {
+    case 1: return launch_pdl(down_dense_kernel<1>, g2, dim3(256), down_dense_smem<1>(), s, b);
+    case 2: return launch_pdl(down_dense_kernel<2>, g2, dim3(256), down_dense_smem<2>(), s, b);
+    case 3: case 4: return launch_pdl(down_dense_kernel<4>, g2, dim3(256), down_dense_smem<4>(), s, b);
+    default: return launch_pdl(down_dense_kernel<8>, g2, dim3(256), down_dense_smem<8>(), s, b);
+  }
 }
 
 cudaError_t launch_unfrag(int fmt, const __half* src, int rows, int G, __half* dst, cudaStream_t s) {

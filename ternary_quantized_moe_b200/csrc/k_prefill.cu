@@ -31,6 +31,8 @@
 
 #include <string.h>
 
+#include <vector>
+
 #include "tc_common.cuh"
 #include "tc_order.cuh"
 #include "topk_warp.cuh"
@@ -161,6 +163,7 @@ struct DenseParams {
   const float* resid;  // kEpiStore: added to the stored value (same layout as out; may equal out)
   const int32_t* xexp;  // range exponent s_t of each token: hz rows are stored times 2^hz_shift(s_t)
   int has_corr;         // the layer has a correction (hz_shift's choice)
+  int z_only;           // the correction branch alone: z rows are stored times 2^s_t
   int* err;
 };
 
@@ -317,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_gemm_kernel(const __grid_co
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int sh = i < n16 ? p.xexp[t0 + i] : 0;
-            const int e = hz_shift(sh, p.has_corr);
+            const int e = p.z_only ? sh : hz_shift(sh, p.has_corr);
             tf[i] = pow2i(u.epi == kEpiStore ? -e : (u.b16 ? e - sh : e));
           }
         }
@@ -379,6 +382,11 @@ struct __align__(16) TernTile {
 __device__ __forceinline__ TernTile load_tile(const TernTile* tiles, int i, int slots) {
   const int4 v = __ldg(reinterpret_cast<const int4*>(tiles) + i);
   return slots ? TernTile{v.x, 0, v.z, v.y} : TernTile{v.x, v.y, v.z, v.w};
+}
+
+// out[0..3] += (a, b, c, d): one 16-byte fp32 reduction (16-byte aligned address).
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
 struct TernParams {
@@ -503,7 +511,10 @@ struct TernRing {
   static constexpr uint32_t b_bytes = 2 * b_kblock;
   static constexpr uint32_t c_bytes = NA * 8 * tb;
   static constexpr uint32_t b_off = 0, c_off = kB * b_bytes;
-  static constexpr uint32_t bytes = c_off + kC * c_bytes;
+  // down projection: per epilogue warp a 16-token x 32-row fp32 tile, read back as 4-row vectors
+  // for the 16-byte reductions into out
+  static constexpr uint32_t e_off = c_off + kC * c_bytes;
+  static constexpr uint32_t bytes = e_off + (NA == 1 ? 8 * 16 * 32 * 4 : 0);
   // tensor memory: accumulators, then the ring of expanded A groups
   // gate/up: one NA x TN accumulator (two, ping-pong, for decode tiles); down: two TN-column
   // accumulators (ping-pong)
@@ -771,13 +782,25 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
           for (int i = 0; i < 16; ++i)
             if (n0 + i < nn) dst[int64_t(i) * p.d] = __float2half_rn(v0[i]);
         } else {
-          // gate-weighted scatter-add: the warp's 32 rows of one token are 128 contiguous bytes
+          // gate-weighted scatter-add: the warp's 32 rows x 16 tokens go through shared memory and
+          // come back as (token, 4 consecutive rows) vectors, one 16-byte fp32 reduction each
+          float* ts = reinterpret_cast<float*>(smem + R::e_off) + (warp - 12) * 512;
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
+          for (int i = 0; i < 16; ++i) ts[i * 32 + lane] = v0[i];
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int i = (lane >> 3) + 4 * j, g4 = lane & 7;  // token i of the chunk, rows 4 g4 .. 4 g4 + 3
             if (n0 + i < nn) {
-              const int t = p.perm[pos0 + n0 + i] / p.k;
-              atomicAdd(p.out + int64_t(t) * p.d + int64_t(rt) * kBM + row, p.gperm[pos0 + n0 + i] * v0[i]);
+              const float4 w = *reinterpret_cast<const float4*>(ts + i * 32 + 4 * g4);
+              const int pos = int(pos0) + n0 + i;
+              const int t = p.perm[pos] / p.k;
+              const float gg = p.gperm[pos];
+              red_add_v4(p.out + int64_t(t) * p.d + int64_t(rt) * kBM + q * 32 + 4 * g4, gg * w.x, gg * w.y,
+                         gg * w.z, gg * w.w);
             }
+          }
+          __syncwarp();
         }
       }
       // accumulator drained: hand it back to the MMA warp
@@ -1145,7 +1168,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       dp.n_units2 = (L->desc.router_fp32 ? 0 : (L->E + 127) / 128) + (L->Fs + 127) / 128;
       dp.logits = P.logits, dp.ld_logits = L->E, dp.hz = P.hz, dp.ld_hz = L->Kd, dp.out = nullptr, dp.ld_out = 0;
       dp.resid = nullptr;
-      dp.xexp = P.xexp, dp.has_corr = L->r > 0;
+      dp.xexp = P.xexp, dp.has_corr = L->r > 0, dp.z_only = 0;
       dp.err = L->err;
       if (L->desc.corr_packed) dp.b16 = P.x16_map;
       dense_gemm_kernel<<<dense_grid(dp), kThreads, kDenseSmem, s>>>(dp);
@@ -1211,7 +1234,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       dp.n_units = P.n_dunits, dp.n_units2 = 0;
       dp.logits = nullptr, dp.ld_logits = 0, dp.hz = nullptr, dp.ld_hz = 0, dp.out = out, dp.ld_out = L->d;
       dp.resid = resid;
-      dp.xexp = P.xexp, dp.has_corr = L->r > 0;
+      dp.xexp = P.xexp, dp.has_corr = L->r > 0, dp.z_only = 0;
       dp.err = L->err;
       dense_gemm_kernel<<<dense_grid(dp), kThreads, kDenseSmem, s>>>(dp);
       return cudaGetLastError();
@@ -1241,6 +1264,59 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
     default:
       return cudaErrorInvalidValue;
   }
+}
+
+// ---------------------------------------- correction branch on the attention output
+// Tensor-core path: v -> fp16 (PTQ1_0 column order, no per-position factors) with the range
+// exponents, z = A v into hz (A bf16 against v bf16, or packed A's exact fp16 copy in the same
+// column order against v16), then out = base + B z with B's fp16 copy.
+int corr_prefill_setup(CorrState* C, cudaStream_t s) {
+  std::vector<DenseUnit> uz, uo;
+  for (int r0 = 0; r0 < C->r; r0 += 128) uz.push_back(DenseUnit{kEpiPlain, 1, 0, 4, 4, r0, C->r, 0, C->packed});
+  for (int r0 = 0; r0 < C->d_out; r0 += 128) uo.push_back(DenseUnit{kEpiStore, 1, 0, 5, 5, r0, C->d_out, 0, 0});
+  C->n_units_z = int(uz.size()), C->n_units_o = int(uo.size());
+  int st;
+  if (cudaMalloc(&C->units_z, sizeof(DenseUnit) * uz.size()) != cudaSuccess) return SCION_ENOMEM;
+  if (cudaMalloc(&C->units_o, sizeof(DenseUnit) * uo.size()) != cudaSuccess) return SCION_ENOMEM;
+  C->device_bytes += sizeof(DenseUnit) * (uz.size() + uo.size());
+  if (cudaMemcpyAsync(C->units_z, uz.data(), sizeof(DenseUnit) * uz.size(), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(C->units_o, uo.data(), sizeof(DenseUnit) * uo.size(), cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)  // the host vectors go out of scope
+    return SCION_ECUDA;
+  if (C->packed) {
+    if ((st = make_tmap_2d(&C->map_a, C->a16, 0, C->r, C->d_in))) return st;
+  } else if ((st = make_tmap_2d(&C->map_a, C->a, 1, C->r, C->d_in))) {
+    return st;
+  }
+  if ((st = make_tmap_2d(&C->map_b16, C->b16, 0, C->d_out, C->Kd))) return st;
+  if ((st = make_tmap_2d(&C->map_v16, C->v16, 0, C->max_tokens, C->d_in))) return st;
+  return make_tmap_2d(&C->map_hz, C->hz, 0, C->max_tokens, C->Kd);
+}
+
+cudaError_t launch_corr_prefill(const CorrState* C, const __nv_bfloat16* v, int T, const float* base, float* out,
+                                cudaStream_t s) {
+  const unsigned grid = unsigned(std::min((T + 7) / 8, num_sms() * 8));
+  x16_kernel<SCION_PTQ1_0><<<grid, 256, 0, s>>>(v, T, C->d_in, C->v16, C->xexp, 0, nullptr, nullptr);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  DenseParams dp;
+  memset(&dp, 0, sizeof(dp));
+  dp.a[4] = C->map_a, dp.a[5] = C->map_b16;
+  if (!C->packed && make_tmap_2d(&dp.b, v, 1, T, C->d_in) != SCION_OK) return cudaErrorInvalidValue;
+  dp.b16 = C->map_v16;
+  dp.units = static_cast<const DenseUnit*>(C->units_z), dp.n_units = C->n_units_z, dp.n_units2 = 0;
+  dp.K = C->d_in, dp.T = T, dp.ab_bf16 = 1;
+  dp.hz = C->hz, dp.ld_hz = C->Kd, dp.xexp = C->xexp, dp.z_only = 1, dp.err = C->err;
+  dense_gemm_kernel<<<dense_grid(dp), kThreads, kDenseSmem, s>>>(dp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  DenseParams dq;
+  memset(&dq, 0, sizeof(dq));
+  dq.a[5] = C->map_b16, dq.b = C->map_hz;
+  dq.units = static_cast<const DenseUnit*>(C->units_o), dq.n_units = C->n_units_o, dq.n_units2 = 0;
+  dq.K = C->Kd, dq.T = T, dq.ab_bf16 = 0;
+  dq.out = out, dq.ld_out = C->d_out, dq.resid = base, dq.xexp = C->xexp, dq.z_only = 1, dq.err = C->err;
+  dense_gemm_kernel<<<dense_grid(dq), kThreads, kDenseSmem, s>>>(dq);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_tc_decode(int na, const scion_layer* L, int T, float* out, cudaStream_t s) {

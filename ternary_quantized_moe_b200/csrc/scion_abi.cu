@@ -309,7 +309,8 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   L->Kdense = L->Fs + L->r;
   L->Kd = (L->Kdense + 63) / 64 * 64;
   L->stream_min_tokens = 16;  // below this the few active experts spread better over the split-K kernels
-  L->tc_decode = 1;
+  L->tc_decode = 0;
+  L->deterministic = 1;
   cudaStream_t s = as_stream(stream);
   const int tb = scion::tile_bytes(L->fmt);
   const int TD = SCION_TDEC;
@@ -489,6 +490,147 @@ extern "C" int scion_debug_route(const void* x, int T, const scion_layer* L, int
   memset(&dbg, 0, sizeof(dbg));
   dbg.ids = ids, dbg.gates = gates, dbg.offsets = offsets, dbg.perm = perm;
   return scion_moe_forward_debug(x, T, L, L->out_stage, &dbg, stream);
+}
+
+// ------------------------------------------------ correction branch on the attention output
+namespace {
+template <typename T>
+cudaError_t corr_alloc(scion::CorrState* C, T** p, size_t bytes) {
+  *p = nullptr;
+  if (bytes == 0) return cudaSuccess;
+  cudaError_t e = cudaMalloc(reinterpret_cast<void**>(p), bytes);
+  if (e == cudaSuccess) C->device_bytes += bytes;
+  return e;
+}
+
+void free_corr(scion_corr* H) {
+  if (!H) return;
+  scion::CorrState& C = H->c;
+  void* ptrs[] = {C.b16, C.xunits, C.hz, C.xexp, C.v16, C.a16, C.units_z, C.units_o, C.err};
+  for (void* p : ptrs)
+    if (p) cudaFree(p);
+  delete H;
+}
+}  // namespace
+
+extern "C" int scion_corr_create(const scion_corr_desc* D, int max_tokens, void* stream, scion_corr** out) {
+  if (!out) return SCION_EINVAL;
+  *out = nullptr;
+  if (!D || max_tokens < 1 || !D->corr_a || !D->corr_b) return SCION_EINVAL;
+  if (D->d_in <= 0 || D->d_in % 128 || D->d_in > 8 * SCION_XPROJ_KC || D->d_out <= 0 || D->d_out % 128) return SCION_EINVAL;
+  if (D->packed != 0 && D->packed != 1) return SCION_EINVAL;
+  if (D->rank <= 0 || D->rank % 16 || D->rank > 4096 || (D->packed && D->rank % 128)) return SCION_EINVAL;
+  if (D->packed && ((reinterpret_cast<uintptr_t>(D->corr_a) | reinterpret_cast<uintptr_t>(D->corr_b)) & 1))
+    return SCION_EINVAL;  // blocks are read with 2-byte loads
+  if (!D->packed && ((reinterpret_cast<uintptr_t>(D->corr_a) | reinterpret_cast<uintptr_t>(D->corr_b)) & 15))
+    return SCION_EINVAL;  // rows are read with 16-byte loads
+  scion_corr* H = new (std::nothrow) scion_corr;
+  if (!H) return SCION_ENOMEM;
+  memset(H, 0, sizeof(*H));
+  scion::CorrState& C = H->c;
+  C.d_in = D->d_in, C.d_out = D->d_out, C.r = D->rank, C.packed = D->packed, C.max_tokens = max_tokens;
+  C.Kd = (C.r + 63) / 64 * 64;
+  C.a = D->corr_a, C.b = D->corr_b;
+  C.n_xunits = (C.r + 15) / 16, C.n_xchunks = (C.d_in + SCION_XPROJ_KC - 1) / SCION_XPROJ_KC;
+  cudaStream_t s = as_stream(stream);
+  int st = SCION_OK;
+  int64_t* bad = nullptr;
+  int64_t bad_host = 0;
+  std::vector<scion::XUnit> units;
+  for (int q0 = 0; q0 < C.r; q0 += 16) units.push_back({scion::kUnitPlain, q0});
+  const int T = max_tokens > SCION_TDEC ? max_tokens : SCION_TDEC;
+  SCION_TRY(scion::configure_kernels());
+  SCION_TRY(corr_alloc(&C, &C.b16, sizeof(__half) * size_t(C.d_out) * C.Kd));
+  SCION_TRY(corr_alloc(&C, &C.xunits, sizeof(scion::XUnit) * units.size()));
+  SCION_TRY(corr_alloc(&C, &C.hz, sizeof(__half) * size_t(T) * C.Kd));
+  SCION_TRY(corr_alloc(&C, &C.xexp, sizeof(int32_t) * T));
+  SCION_TRY(corr_alloc(&C, &C.err, sizeof(int)));
+  SCION_TRY(cudaMalloc(&bad, sizeof(int64_t)));
+  SCION_TRY(cudaMemsetAsync(bad, 0, sizeof(int64_t), s));
+  SCION_TRY(cudaMemsetAsync(C.err, 0, sizeof(int), s));
+  SCION_TRY(cudaMemsetAsync(C.hz, 0, sizeof(__half) * size_t(T) * C.Kd, s));  // pad columns stay 0
+  SCION_TRY(cudaMemsetAsync(C.b16, 0, sizeof(__half) * size_t(C.d_out) * C.Kd, s));
+  SCION_TRY(cudaMemcpyAsync(C.xunits, units.data(), sizeof(scion::XUnit) * units.size(), cudaMemcpyHostToDevice, s));
+  if (C.packed) {
+    // B's exact fp16 values (code * scale); A's codes are checked here and read in place by decode
+    SCION_TRY(scion::launch_dequant_corr(static_cast<const uint8_t*>(C.b), C.d_out, C.r, C.b16, C.Kd, -1, bad, s));
+    SCION_TRY(scion::launch_dequant_corr(static_cast<const uint8_t*>(C.a), C.r, C.d_in, nullptr, 0, -1, bad, s));
+  } else {
+    SCION_TRY(scion::launch_bf16_to_f16_rows(static_cast<const __nv_bfloat16*>(C.b), C.d_out, C.r, C.b16, C.Kd, s));
+  }
+  if (max_tokens > SCION_TDEC) {
+    SCION_TRY(corr_alloc(&C, &C.v16, sizeof(__half) * size_t(max_tokens) * C.d_in));
+    if (C.packed) {
+      SCION_TRY(corr_alloc(&C, &C.a16, sizeof(__half) * size_t(C.r) * C.d_in));
+      // in the column order of v16 (the PTQ1_0 order carries no per-position factors)
+      SCION_TRY(scion::launch_dequant_corr(static_cast<const uint8_t*>(C.a), C.r, C.d_in, C.a16, C.d_in, SCION_PTQ1_0,
+                                           bad, s));
+    }
+    if ((st = scion::corr_prefill_setup(&C, s)) != SCION_OK) goto fail;
+  }
+  SCION_TRY(cudaMemcpyAsync(&bad_host, bad, sizeof(int64_t), cudaMemcpyDeviceToHost, s));
+  SCION_TRY(cudaStreamSynchronize(s));
+  cudaFree(bad);
+  bad = nullptr;
+  if (bad_host) {
+    st = SCION_EFORMAT;
+    goto fail;
+  }
+  *out = H;
+  return SCION_OK;
+fail:
+  if (bad) cudaFree(bad);
+  free_corr(H);
+  return st;
+}
+
+extern "C" void scion_corr_destroy(scion_corr* H) {
+  if (!H) return;
+  cudaDeviceSynchronize();
+  free_corr(H);
+}
+
+extern "C" int scion_corr_forward(const void* v, int T, const scion_corr* H, const float* base, float* out,
+                                  void* stream) {
+  if (!H || T < 0 || T > H->c.max_tokens) return SCION_EINVAL;
+  if (T == 0) return SCION_OK;
+  if (!v || !out) return SCION_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(base)) & 15)
+    return SCION_EINVAL;
+  const scion::CorrState& C = H->c;
+  cudaStream_t s = as_stream(stream);
+  if (T > SCION_TDEC) {
+    g_launches.fetch_add(2, std::memory_order_relaxed);  // three kernels, the scope counts one
+    StageScope scope_(SCION_STAGE_XPROJ, s);
+    return cuda_status(scion::launch_corr_prefill(&C, static_cast<const __nv_bfloat16*>(v), T, base, out, s));
+  }
+  // out starts at base (or zero); the B z product is added with fp32 reductions
+  cudaError_t e = base ? (base != out ? cudaMemcpyAsync(out, base, sizeof(float) * size_t(T) * C.d_out,
+                                                        cudaMemcpyDeviceToDevice, s)
+                                      : cudaSuccess)
+                       : cudaMemsetAsync(out, 0, sizeof(float) * size_t(T) * C.d_out, s);
+  if (e != cudaSuccess) return cuda_status(e);
+  SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_corr_z(&C, static_cast<const __nv_bfloat16*>(v), T, s));
+  SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_corr_out(&C, T, out, s));
+  return SCION_OK;
+}
+
+extern "C" size_t scion_corr_device_bytes(const scion_corr* H) { return H ? H->c.device_bytes : 0; }
+
+extern "C" int scion_corr_check(const scion_corr* H, void* stream) {
+  if (!H) return SCION_EINVAL;
+  cudaStream_t s = as_stream(stream);
+  int err = 0;
+  cudaError_t e = cudaMemcpyAsync(&err, H->c.err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_status(e);
+  if (err != 0) {
+    const int zero = 0;
+    e = cudaMemcpyAsync(H->c.err, &zero, sizeof(int), cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    return err;
+  }
+  return SCION_OK;
 }
 
 extern "C" int scion_layer_check(const scion_layer* L, void* stream) {

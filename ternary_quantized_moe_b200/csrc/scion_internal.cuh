@@ -88,7 +88,32 @@ struct PrefillState {
   __half* hz;           // [maxT][Kd]
 };
 
+// The correction branch on the attention output (scion_corr_*): z = A v, out = base + B z.
+struct CorrState {
+  int d_in, d_out, r, Kd, packed, max_tokens;
+  const void* a;       // bf16 [r][d_in] or PQ2_0 blocks [r][d_in/128] (read in place)
+  const void* b;       // bf16 [d_out][r] or PQ2_0 blocks [d_out][r/128] (packed: read in place by decode)
+  __half* b16;         // [d_out][Kd] exact fp16 copy of B (bf16 decode and the tensor-core path)
+  XUnit* xunits;       // decode: one kind-Plain unit per 16 rows of A
+  int n_xunits, n_xchunks;
+  __half* hz;          // [max_tokens][Kd] z times 2^s_t
+  int32_t* xexp;       // [max_tokens] range exponent of each token
+  // tensor-core path (max_tokens > SCION_TDEC)
+  __half* v16;         // [max_tokens][d_in] v 2^s_t in the PTQ1_0 column order (fp16)
+  __half* a16;         // packed A: [r][d_in] exact fp16 in the same column order
+  void* units_z;       // dense-GEMM units: rows of A, then rows of B
+  void* units_o;
+  int n_units_z, n_units_o;
+  CUtensorMap map_a, map_b16, map_v16, map_hz;
+  int* err;            // device status word (a bounded wait of the tensor-core path that gave up)
+  size_t device_bytes;
+};
+
 }  // namespace scion
+
+struct scion_corr {
+  scion::CorrState c;
+};
 
 struct scion_layer {
   scion_layer_desc desc;
@@ -181,6 +206,14 @@ cudaError_t configure_kernels();
 cudaError_t configure_stream_kernels();
 cudaError_t launch_stream_gateup(const scion_layer* L, int T, cudaStream_t s);
 cudaError_t launch_stream_down(const scion_layer* L, int T, float* out, cudaStream_t s);
+
+// correction branch on the attention output: decode kernels (k_decode.cu) and the tensor-core
+// path with its unit tables (k_prefill.cu)
+cudaError_t launch_corr_z(const CorrState* C, const __nv_bfloat16* v, int T, cudaStream_t s);
+cudaError_t launch_corr_out(const CorrState* C, int T, float* out, cudaStream_t s);
+int corr_prefill_setup(CorrState* C, cudaStream_t s);
+cudaError_t launch_corr_prefill(const CorrState* C, const __nv_bfloat16* v, int T, const float* base, float* out,
+                                cudaStream_t s);
 
 // k_prefill.cu
 int make_tmap_2d(CUtensorMap* map, const void* ptr, int bf16, int64_t rows, int64_t K, int box_rows = 128);

@@ -375,6 +375,56 @@ def test_forward_activation_range(shape, T):
     check_output(got, ref)
 
 
+@pytest.mark.parametrize("packed", [0, 1])
+@pytest.mark.parametrize("T,max_tokens,in_place", [(1, 64, False), (13, 64, True), (64, 64, False),
+                                                   (300, 300, False), (300, 300, True)])
+def test_attn_out_correction(packed, T, max_tokens, in_place):
+    """The correction branch on the attention output, out = base + B (A v), with d_in != d_out:
+    decode kernels (T <= 64) and tcgen05 GEMMs (T = 300), bf16 and PQ2_0 factors, in place and
+    not, on activations that include tokens scaled by 2^-20 and 2^8 and outlier channels.  The
+    branch (out - base) must meet the block tolerance against the oracle."""
+    d_in, d_out, r = 1024, 512, 256
+    rng = np.random.default_rng(91 + T + packed)
+    if packed:
+        ca, sa = synth.ternary_codes(rng, (r, d_in)), synth.group_scales(rng, (r, d_in // 128))
+        cb, sb = synth.ternary_codes(rng, (d_out, r)), synth.group_scales(rng, (d_out, r // 128))
+        a, b = oracle.pack(synth.PQ2_0, ca, sa), oracle.pack(synth.PQ2_0, cb, sb)
+        ad, bd = torch.from_numpy(a).to(DEV), torch.from_numpy(b).to(DEV)
+    else:
+        a, b = synth.normal_bf16(rng, (r, d_in), 0.02), synth.normal_bf16(rng, (d_out, r), 0.02)
+        ad, bd = u16_to_dev(a, torch.bfloat16, DEV), u16_to_dev(b, torch.bfloat16, DEV)
+    vf = rng.standard_normal((T, d_in)).astype(np.float32)
+    for t in range(T):
+        kind = t % 4
+        if kind == 1:
+            vf[t] *= np.float32(2.0 ** -20)
+        elif kind == 2:
+            vf[t] *= np.float32(2.0 ** 8)
+        elif kind == 3:
+            vf[t, rng.choice(d_in, 3, replace=False)] = np.float32(2e4)
+    v = synth.to_bf16_bits(vf)
+    base = rng.standard_normal((T, d_out))
+    ref, _ = oracle.attn_corr(v, a, b, d_in, d_out, r, packed=packed, base=base)
+    h = tq.scion_corr_create(d_in, d_out, r, ad, bd, packed=packed, max_tokens=max_tokens)
+    base_d = torch.from_numpy(base.astype(np.float32)).to(DEV)
+    out = base_d if in_place else torch.full((T, d_out), float("nan"), dtype=torch.float32, device=DEV)
+    tq.scion_corr_forward(u16_to_dev(v, torch.bfloat16, DEV), T, h, out, base=base_d)
+    torch.cuda.synchronize()
+    assert tq.scion_corr_check(h) == 0
+    got = out.cpu().numpy().astype(np.float64)
+    base32 = base.astype(np.float32).astype(np.float64)
+    check_output(got - base32, ref - base)
+
+
+def test_attn_out_correction_rejects_bad_descriptors():
+    dummy = torch.zeros(1 << 16, dtype=torch.bfloat16, device=DEV)
+    for d_in, d_out, r, packed in [(1000, 512, 256, 0), (1024, 500, 256, 0), (1024, 512, 8, 0), (1024, 512, 64, 1),
+                                   (8192, 512, 64, 0)]:
+        with pytest.raises(tq.ScionError) as ei:
+            tq.scion_corr_create(d_in, d_out, r, dummy, dummy, packed=packed)
+        assert ei.value.status == tq.SCION_EINVAL
+
+
 @pytest.mark.parametrize("T,max_tokens", [(13, 64), (200, 200)])
 def test_debug_route_matches_oracle(T, max_tokens):
     """scion_debug_route (the routing alone): ids as sets per token, offsets and the grouping
@@ -576,15 +626,17 @@ def test_prefill_multi_tile_experts(fmt, T):
 @pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
 @pytest.mark.parametrize("dense", [True, False])
 def test_prefill_deterministic_combine(fmt, dense):
-    """Both ways of adding the routed rows on the tensor-core path: fused fp32 reductions into out
-    (default) and, with SCION_OPT_DETERMINISTIC, one fp16 row per entry summed in slot order by
-    the combine kernel, which repeats bit for bit; with and without the dense down projection
-    (without it out starts from zero, set by the x conversion or by the combine)."""
+    """Both ways of adding the routed rows on the tensor-core path: one fp16 row per entry summed
+    in slot order by the combine kernel (SCION_OPT_DETERMINISTIC = 1, the default), which repeats
+    bit for bit, and fp32 reductions into out from the down projection's epilogue (0); with and
+    without the dense down projection (without it out starts from zero, set by the x conversion
+    or by the combine)."""
     cfg = small("dc", fmt, False, E=16, k=4, Fs=128 if dense else 0, r=16 if dense else 0)
     T = 300
     L, banks, ol, x = _case(cfg, T)
     layer = device_layer(cfg, L, banks, T)
     ref, _, _ = oracle.forward(ol, x)
+    tq.scion_layer_set_option(layer, tq.SCION_OPT_DETERMINISTIC, 0)
     fused, _ = run_forward(layer, x, T)
     check_output(fused, ref)
     tq.scion_layer_set_option(layer, tq.SCION_OPT_DETERMINISTIC, 1)
