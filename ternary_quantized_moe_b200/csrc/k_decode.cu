@@ -248,13 +248,6 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
-  if (need_max)
-    for (int t = warp; t < a.T; t += kXThreads / 32) {  // one warp per staged token row
-      uint32_t m = 0;
-      for (int j = lane; j < kchunks; j += 32) m = max(m, max_mag8(*reinterpret_cast<const uint4*>(xs + t * kXRow + 8 * j)));
-      m = __reduce_max_sync(0xffffffffu, m);
-      if (lane == 0) tmax[t] = m;
-    }
   if (active_warp) {
     const bool second_acc = (u.kind == kUnitSwiglu);
     const int kwl = warp * 64;
@@ -286,6 +279,13 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
     for (int nt = 0; nt < NT; ++nt)
       acc[0][nt][0] *= sc_a, acc[0][nt][1] *= sc_a, acc[0][nt][2] *= sc_b, acc[0][nt][3] *= sc_b;
   }
+  if (need_max)  // after the MMAs, while the x stage is still intact
+    for (int t = warp; t < a.T; t += kXThreads / 32) {  // one warp per staged token row
+      uint32_t m = 0;
+      for (int j = lane; j < kchunks; j += 32) m = max(m, max_mag8(*reinterpret_cast<const uint4*>(xs + t * kXRow + 8 * j)));
+      m = __reduce_max_sync(0xffffffffu, m);
+      if (lane == 0) tmax[t] = m;
+    }
   __syncthreads();  // the x stage is dead: its space holds the warp reduction
   float(*red)[2][NT][32][4] = reinterpret_cast<float(*)[2][NT][32][4]>(xsm);
 #pragma unroll
@@ -317,6 +317,8 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
   constexpr int kIt = 16 * SCION_TDEC / kXThreads;
   float v[kIt][2];
   if (lead && need_max) {
+    // the tokens' largest |x| over all chunks (read beside the partial sums below; the cluster
+    // barrier that follows orders these shared-memory writes before the epilogue reads them)
     for (int t = threadIdx.x; t < a.T; t += kXThreads) {
       uint32_t m = tmax[t];
       for (int ch = 1; ch < a.n_chunks; ++ch)
@@ -325,7 +327,6 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
       tshift[t] = a.z_only ? sh : hz_shift(sh, a.r > 0);
       if (a.z_only && blockIdx.x == 0) a.xexp[t] = sh;
     }
-    __syncthreads();
   }
   if (lead) {
 #pragma unroll

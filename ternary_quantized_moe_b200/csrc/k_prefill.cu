@@ -310,20 +310,22 @@ __global__ void __launch_bounds__(kThreads, 1) dense_gemm_kernel(const __grid_co
           tmem_ld16x2(acc + c * 16, acc + 128 + c * 16, v0, v1);
         else
           tmem_ld16(acc + c * 16, v0);
-        if (!rok) continue;
         const int n16 = min(16, nt - c * 16);
         const int64_t t0 = dt.tok0 + c * 16;
         // per-token factors of the hz rows (see hz_shift): stored times 2^p, read back times 2^-p;
-        // the units against x16 (ternary correction A) accumulate x 2^s_t
+        // the units against x16 (ternary correction A) accumulate x 2^s_t.  One load per lane,
+        // shared by shuffles (the whole warp takes part, before rows past the unit drop out).
         float tf[16];
         if (u.epi != kEpiLogits) {
+          const int my_sh = lane < n16 ? p.xexp[t0 + lane] : 0;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const int sh = i < n16 ? p.xexp[t0 + i] : 0;
+            const int sh = __shfl_sync(0xffffffffu, my_sh, i);
             const int e = p.z_only ? sh : hz_shift(sh, p.has_corr);
             tf[i] = pow2i(u.epi == kEpiStore ? -e : (u.b16 ? e - sh : e));
           }
         }
+        if (!rok) continue;
         if (u.epi == kEpiLogits) {
           float* dst = p.logits + t0 * p.ld_logits + col;
 #pragma unroll
@@ -770,12 +772,21 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
         const int n0 = c * 16;
         if constexpr (NA == 2) {
           __half* dst = p.h + (pos0 + n0) * p.F + int64_t(rt) * kBM + pcol;
+          // range exponents of the chunk's 16 tokens: one load per lane, shared by shuffles; the
+          // common case (every token in the unscaled band) skips the scaling
+          const int my_sh = (lane < 16 && n0 + lane < nn) ? p.pexp[pos0 + n0 + lane] : 0;
+          if (__all_sync(0xffffffffu, my_sh == 0)) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (n0 + i < nn) {
-              const int sh = p.pexp[pos0 + n0 + i];  // the sums are of x 2^sh
-              dst[int64_t(i) * p.F] = __float2half_rn(silu_f(v0[i] * pow2i(-sh)) * (v1[i] * pow2i(sh)) * hscale);
+            for (int i = 0; i < 16; ++i)
+              if (n0 + i < nn) dst[int64_t(i) * p.F] = __float2half_rn(silu_f(v0[i]) * v1[i] * hscale);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int sh = __shfl_sync(0xffffffffu, my_sh, i);  // the sums are of x 2^sh
+              if (n0 + i < nn)
+                dst[int64_t(i) * p.F] = __float2half_rn(silu_f(v0[i] * pow2i(-sh)) * (v1[i] * pow2i(sh)) * hscale);
             }
+          }
         } else if (p.y) {
           __half* dst = p.y + (pos0 + n0) * p.d + int64_t(rt) * kBM + row;
 #pragma unroll

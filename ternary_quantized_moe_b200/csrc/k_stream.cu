@@ -293,9 +293,11 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
               if (lane == 0) hd->pos[i] = pos, hd->orow[i] = orow, hd->gate[i] = gate, hd->xdn[i] = xdn, hd->xup[i] = xup;
             }
           }
+          // bit 2: some token of the pass is range-scaled (its epilogue factors are not all 1)
+          const bool scaled = __any_sync(0xffffffffu, tk.xup != 1.f);
           if (lane == 0) {
             hd->nn = nn;
-            hd->flags = (g0 == 0 ? 1 : 0) | (last ? 2 : 0);
+            hd->flags = (g0 == 0 ? 1 : 0) | (last ? 2 : 0) | (scaled ? 4 : 0);
             hd->rb = rb;
             hd->ng = ng;
             mbar_arrive_expect_tx(&full[s], ng * cb + nn * ng * kRowB);
@@ -375,7 +377,9 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
         const int row = warp * 16 + (lane >> 2) + 8 * (i >> 1);
         const int tcol = 2 * c + (i & 1);
         if constexpr (NMAT == 2) {
-          const float h = silu_f(acc[0][i] * unit * hd->xdn[tcol]) * (acc[1][i] * unit * hd->xup[tcol]) * hsc[i >> 1];
+          const float h = (flags & 4) ? silu_f(acc[0][i] * unit * hd->xdn[tcol]) * (acc[1][i] * unit * hd->xup[tcol]) *
+                                            hsc[i >> 1]
+                                      : silu_f(acc[0][i] * unit) * (acc[1][i] * unit) * hsc[i >> 1];
           const __half h16 = __float2half_rn(h);
           if (tcol < nn) a.hfrag[(int64_t(hd->pos[tcol]) * (a.F >> 7) + rb) * SCION_BROW + hpos[i >> 1]] = h16;
           if (FMT == SCION_PQ2_0) hs[i & 1] += __half2float(h16) * hinv[i >> 1];

@@ -403,7 +403,10 @@ def test_attn_out_correction(packed, T, max_tokens, in_place):
         elif kind == 3:
             vf[t, rng.choice(d_in, 3, replace=False)] = np.float32(2e4)
     v = synth.to_bf16_bits(vf)
-    base = rng.standard_normal((T, d_out))
+    # base rows of the branch's own magnitude (a fp32 sum cannot hold a branch far below its base)
+    br, _ = oracle.attn_corr(v, a, b, d_in, d_out, r, packed=packed)
+    base = rng.standard_normal((T, d_out)) * np.sqrt((br ** 2).mean(axis=1, keepdims=True))
+    base = base.astype(np.float32).astype(np.float64)
     ref, _ = oracle.attn_corr(v, a, b, d_in, d_out, r, packed=packed, base=base)
     h = tq.scion_corr_create(d_in, d_out, r, ad, bd, packed=packed, max_tokens=max_tokens)
     base_d = torch.from_numpy(base.astype(np.float32)).to(DEV)
@@ -412,8 +415,7 @@ def test_attn_out_correction(packed, T, max_tokens, in_place):
     torch.cuda.synchronize()
     assert tq.scion_corr_check(h) == 0
     got = out.cpu().numpy().astype(np.float64)
-    base32 = base.astype(np.float32).astype(np.float64)
-    check_output(got - base32, ref - base)
+    check_output(got - base, ref - base)
 
 
 def test_attn_out_correction_rejects_bad_descriptors():
