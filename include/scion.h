@@ -223,9 +223,10 @@ int scion_moe_forward_residual(const void* x, int T, const scion_layer* layer, c
  *    smaller batches split K over the warps of one CTA per 16 rows, which spreads the few
  *    active experts over more SMs.
  *  SCION_OPT_DECODE_TC (default 0): 0 runs those persistent kernels as mma.sync kernels fed by a
- *    bulk-copy ring; 1 as the tcgen05 grouped GEMMs of the large batches (codes expanded into
- *    tensor memory, one tile per active expert, the down projection adding its gate-weighted rows
- *    into out), measured slower at decode sizes.
+ *    bulk-copy ring; 1 as tcgen05 kernels (codes expanded into tensor memory at one instruction
+ *    per two weights, tiles of up to 16 tokens of one expert, one accumulator per 128-column
+ *    group folded into registers with the group scales; the down projection adds its
+ *    gate-weighted rows into out).  Layers of up to 512 experts.
  *  SCION_OPT_DETERMINISTIC (default 1): batches above 64 tokens are bit-reproducible: the down
  *    projection writes one fp16 row per routed entry and a combine kernel sums each token's rows
  *    in slot order.  0: the down projection adds its rows into out with fp32 reductions (no row

@@ -43,7 +43,9 @@ struct XProjArgs {
   __half* hz;
   __half* xfrag;  // [T][d/128][SCION_BROW] fp16 x 2^s_t in fragment order + group sums
   int32_t* xexp;  // [T] range exponent s_t of each token (token_shift), written by the aux CTAs
-  __half* x16;    // non-null: the aux CTAs write x 2^s_t here, [T][d] in the tcgen05 column order
+  __half* x16;    // non-null: the aux CTAs write x 2^s_t here, [T][d] in the tcgen05 column order,
+  float* xsum;    //   with its per-group sums of B * 4^f (PQ2_0) in xsum [T][d/128],
+  float* hsum;    //   and zero the hidden's group sums hsum [T*k][F/128]
   __half* h;      // [T*k][F/128][SCION_BROW] expert hidden: group-sum tails zeroed here
   int k, GF;
   const uint8_t* corr_blocks;  // ternary correction A (PQ2_0 blocks [r][d/128]) or nullptr (bf16 corr_a)
@@ -77,53 +79,73 @@ __device__ __forceinline__ void xproj_aux(const XProjArgs& a, int aux, int n_aux
   const int lane = threadIdx.x & 31;
   const int gw = aux * (kXThreads / 32) + (threadIdx.x >> 5), nw = n_aux * (kXThreads / 32);
   // Warps share the tokens out (wpt warps per token, each a slice of its pairs of 128-column
-  // groups).  Each warp finds its token's largest magnitude over the whole row (all loads in
-  // flight at once), which fixes the range exponent s_t, then writes x 2^s_t for its pairs:
-  // 16 lanes per group, 8 elements per lane, in the tcgen05 order (a.x16) or the fragment order
-  // with the group sums of B * 4^f in the row tails.
+  // groups).  Each warp loads its token's whole row into registers (16 bytes per lane per pair,
+  // all loads in flight at once); their largest magnitude fixes the range exponent s_t.  Each of
+  // its pairs then goes through shared memory, where lane (gl, part) gathers the 8 columns of its
+  // output positions in group 2 pr + gl and writes x 2^s_t in the tcgen05 order (a.x16) or the
+  // fragment order with the group sums of B * 4^f in the row tails.
+  constexpr int kMaxPairs = 16;  // d <= 4096
+  __shared__ __align__(16) __nv_bfloat16 pbuf[kXThreads / 32][256];
+  __nv_bfloat16* buf = pbuf[threadIdx.x >> 5];
   const int wpt = max(1, nw / max(1, a.T));
+  const int gl = lane >> 4, part = lane & 15;
   for (int job = gw; job < a.T * wpt; job += nw) {
     const int t = job / wpt, slice = job % wpt;
     const __nv_bfloat16* row = a.x + int64_t(t) * a.d;
+    uint4 v[kMaxPairs];
     uint32_t mx = 0;
-#pragma unroll 4
-    for (int i = lane; i < a.d / 8; i += 32) mx = max(mx, max_mag8(*reinterpret_cast<const uint4*>(row + 8 * i)));
+#pragma unroll
+    for (int j = 0; j < kMaxPairs; ++j) {
+      const bool ld = j < n_pairs && 2 * j + gl < Gd;  // an odd group count leaves the last pair half empty
+      v[j] = ld ? *reinterpret_cast<const uint4*>(row + 256 * j + 8 * lane) : make_uint4(0u, 0u, 0u, 0u);
+      mx = max(mx, max_mag8(v[j]));
+    }
     const int sh = token_shift(__reduce_max_sync(0xffffffffu, mx));
     if (lane == 0 && slice == 0) a.xexp[t] = sh;
     const float xs = pow2i(sh);
-    for (int pr = slice; pr < n_pairs; pr += wpt) {
-      const int g = 2 * pr + (lane >> 4), part = lane & 15;
+#pragma unroll
+    for (int pr = 0; pr < kMaxPairs; ++pr) {
+      if (pr >= n_pairs) break;
+      if (pr % wpt != slice) continue;
+      const int g = 2 * pr + gl;
       const bool ok = g < Gd;
-      const __nv_bfloat16* src = row + g * 128;
+      __syncwarp();
+      *reinterpret_cast<uint4*>(buf + 8 * lane) = v[pr];
+      __syncwarp();
+      const __nv_bfloat16* src = buf + 128 * gl;
       __align__(16) __half o[8];
+      float sum = 0.f;
       if (a.x16) {
         // tcgen05 order: positions 8 part .. 8 part + 7 of group g
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int q = 8 * part + e;
-          const float v = ok ? __bfloat162float(src[pos_col(a.fmt, q)]) * xs : 0.f;
-          o[e] = __float2half_rn(a.fmt == SCION_PQ2_0 ? v * pq2_pos_scale(q) : v);
+          const float f = __bfloat162float(src[pos_col(a.fmt, q)]) * xs;
+          o[e] = __float2half_rn(a.fmt == SCION_PQ2_0 ? f * pq2_pos_scale(q) : f);
+          if (a.fmt == SCION_PQ2_0) sum += __half2float(o[e]) / pq2_pos_scale(q);
         }
-        if (ok) *reinterpret_cast<uint4*>(a.x16 + int64_t(t) * a.d + g * 128 + 8 * part) = *reinterpret_cast<const uint4*>(o);
-        continue;
-      }
-      float sum = 0.f;
+      } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int idx = part * 8 + e;
-        const float v = ok ? __bfloat162float(src[brow_col(a.fmt, idx)]) * xs : 0.f;
-        if (a.fmt == SCION_PQ2_0) {
-          const float up = 1.0f / brow_bscale(idx);
-          o[e] = __float2half_rn(v / up);
-          sum += __half2float(o[e]) * up;
-        } else {
-          o[e] = __float2half_rn(v);
+        for (int e = 0; e < 8; ++e) {
+          const int idx = part * 8 + e;
+          const float f = __bfloat162float(src[brow_col(a.fmt, idx)]) * xs;
+          if (a.fmt == SCION_PQ2_0) {
+            const float up = 1.0f / brow_bscale(idx);
+            o[e] = __float2half_rn(f / up);
+            sum += __half2float(o[e]) * up;
+          } else {
+            o[e] = __float2half_rn(f);
+          }
         }
       }
 #pragma unroll
       for (int off = 8; off; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-      __half* dst = a.xfrag + (int64_t(t) * Gd + g) * SCION_BROW;
-      if (ok) {
+      if (!ok) continue;
+      if (a.x16) {
+        *reinterpret_cast<uint4*>(a.x16 + int64_t(t) * a.d + g * 128 + 8 * part) = *reinterpret_cast<const uint4*>(o);
+        if (part == 0 && a.xsum && a.fmt == SCION_PQ2_0) a.xsum[int64_t(t) * Gd + g] = sum;
+      } else {
+        __half* dst = a.xfrag + (int64_t(t) * Gd + g) * SCION_BROW;
         *reinterpret_cast<uint4*>(dst + part * 8) = *reinterpret_cast<const uint4*>(o);
         if (part == 0)
           *reinterpret_cast<float4*>(dst + 128) = make_float4(-5.9604644775390625e-08f * sum, 0.f, 0.f, 0.f);
@@ -139,8 +161,10 @@ __device__ __forceinline__ void xproj_aux(const XProjArgs& a, int aux, int n_aux
     for (int64_t i = tid; i < int64_t(a.T) * a.d / 4; i += nth) o4[i] = r4[i];
   }
   // the expert hidden's group sums are accumulated by the gate/up epilogue
-  for (int i = tid; i < a.T * a.k * a.GF; i += nth)
+  for (int i = tid; i < a.T * a.k * a.GF; i += nth) {
     *reinterpret_cast<float4*>(a.h + int64_t(i) * SCION_BROW + 128) = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (a.hsum) a.hsum[i] = 0.f;
+  }
 }
 
 // Eight consecutive ternary codes (16 bits of a PQ2_0 block, low bits first: field 0/1/2 =
@@ -673,6 +697,8 @@ cudaError_t launch_xproj(const scion_layer* L, const __nv_bfloat16* x, int T, fl
   a.units = L->xunits + unit0, a.n_units = n_units, a.n_chunks = L->n_xchunks, a.n_aux = aux ? kXAux : 0;
   a.logits = L->logits, a.hz = L->hz, a.xfrag = L->xfrag, a.xexp = L->xexp, a.out = out;
   a.x16 = x16 ? L->x16d : nullptr;
+  a.xsum = x16 ? L->xsum : nullptr;
+  a.hsum = x16 ? L->hsum : nullptr;
   a.z_only = 0;
   a.corr_blocks = L->desc.corr_packed ? static_cast<const uint8_t*>(L->desc.corr_a) : nullptr;
   a.h = L->h, a.k = L->k, a.GF = L->GF;
@@ -852,6 +878,7 @@ cudaError_t configure_kernels() {
     return e;
   if ((e = configure_route_kernels())) return e;
   if ((e = configure_stream_kernels())) return e;
+  if ((e = configure_tdec_kernels())) return e;
   return configure_prefill_kernels();
 }
 

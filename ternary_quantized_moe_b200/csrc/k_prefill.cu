@@ -379,11 +379,9 @@ struct __align__(16) TernTile {
   int pos0;  // routed-order position of its first token (offsets[e] + c0)
 };
 
-// slots = 1: the list is the decode routing's active-slot records {expert, first routed
-// position, tokens, 0}, one tile per active expert (a decode batch never fills more than one).
-__device__ __forceinline__ TernTile load_tile(const TernTile* tiles, int i, int slots) {
+__device__ __forceinline__ TernTile load_tile(const TernTile* tiles, int i) {
   const int4 v = __ldg(reinterpret_cast<const int4*>(tiles) + i);
-  return slots ? TernTile{v.x, 0, v.z, v.y} : TernTile{v.x, v.y, v.z, v.w};
+  return TernTile{v.x, v.y, v.z, v.w};
 }
 
 // out[0..3] += (a, b, c, d): one 16-byte fp32 reduction (16-byte aligned address).
@@ -393,13 +391,12 @@ __device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, 
 
 struct TernParams {
   CUtensorMap bmap;     // down projection: B = h [T*k][F], box {64, box_rows}
-  int box_rows;         // rows of one TMA box of B (the tile width, or 16 for decode tiles)
+  int box_rows;         // rows of one TMA box of B (the tile width)
   const uint8_t* bank;  // re-tiled gate/up bank (na = 2) or down bank (na = 1)
   int fmt, na, G, R;    // groups along K, rows per expert matrix
   const __half* bsrc;   // B rows: x16 [T][d] (gate/up) or h [T*k][F] (down)
   int ldb;
   const TernTile* tiles;
-  int tile_slots;       // 1: `tiles` holds the decode routing's slot records (see load_tile)
   const int32_t* n_tiles;
   const int32_t *counts, *offsets, *perm;
   const float* gperm;   // [T*k] gate of the entry at each routed position, times 2^(-2 s_t)
@@ -415,7 +412,6 @@ struct TernParams {
 
 constexpr int kBN3 = 160;      // tokens per tile of batches whose experts average kMid160 or more
 constexpr int kMid160 = 112;   // mean tokens per expert from which both ternary GEMMs take kBN3 tiles
-constexpr int kBND = 64;       // tokens per tile of decode batches (at most 64 tokens in all)
 
 // Expand half h (64 columns) of row t (0..127) of one 128-row group from its sub-tile block
 // into 32 registers of fp16 pairs, in position order (v[i] = positions 2i, 2i+1 of the half).
@@ -506,7 +502,7 @@ struct TernRing {
   static constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
   // shared memory: B groups (two 64-column K blocks of TN swizzled 128-byte rows) and packed
   // code groups
-  static_assert(TN == kBN || TN == kBN3 || TN == kBND, "tile width");
+  static_assert(TN == kBN || TN == kBN3, "tile width");
   static constexpr int kB = 4;
   static constexpr int kC = 4;
   static constexpr uint32_t b_kblock = uint32_t(TN) * 128;  // bytes of one 64-column K block of B
@@ -518,15 +514,14 @@ struct TernRing {
   static constexpr uint32_t e_off = c_off + kC * c_bytes;
   static constexpr uint32_t bytes = e_off + (NA == 1 ? 8 * 16 * 32 * 4 : 0);
   // tensor memory: accumulators, then the ring of expanded A groups
-  // gate/up: one NA x TN accumulator (two, ping-pong, for decode tiles); down: two TN-column
-  // accumulators (ping-pong)
-  static constexpr int n_acc = (NA == 1 || TN == kBND) ? 2 : 1;
+  // gate/up: one NA x TN accumulator; down: two TN-column accumulators (ping-pong)
+  static constexpr int n_acc = NA == 1 ? 2 : 1;
   static constexpr uint32_t acc_cols = NA * TN;
   // ring entries of expanded A: one group of all NA matrices, or (160-token gate/up tiles,
   // whose accumulators leave 192 columns) one matrix of a group, EPG entries per group
   static constexpr int EPG = TN == kBN3 ? NA : 1;
   static constexpr int MPE = NA / EPG;           // matrices per entry
-  static constexpr int kA = TN == kBN3 ? 3 : (TN == kBND ? (NA == 2 ? 2 : 6) : (NA == 2 ? 2 : 4));
+  static constexpr int kA = TN == kBN3 ? 3 : (NA == 2 ? 2 : 4);
   static constexpr uint32_t a_cols = MPE * 64;   // one entry: MPE matrices x 64 columns (128 fp16 per lane)
   static constexpr uint32_t a_col0 = n_acc * acc_cols;
   static constexpr uint32_t tmem_cols = 512;
@@ -579,7 +574,7 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
       const int64_t mat_stride = int64_t(8) * R::tb, grp_stride = NA * mat_stride;
       int gs = 0;  // running group counter
       for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
-        const TernTile tile = load_tile(p.tiles, item / RT, p.tile_slots);
+        const TernTile tile = load_tile(p.tiles, item / RT);
         const int rt = item % RT;
         const uint8_t* ebase = p.bank + (int64_t(tile.e) * RT + rt) * p.G * grp_stride;
         for (int g = 0; g < p.G; ++g, ++gs) {
@@ -600,7 +595,7 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
     if (lane == 0) {
       int gs = 0;
       for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
-        const TernTile tile = load_tile(p.tiles, item / RT, p.tile_slots);
+        const TernTile tile = load_tile(p.tiles, item / RT);
         // boxes of box_rows rows (128-byte rows, swizzle atoms of 8 rows: consecutive boxes
         // stack into one TN-row operand); rows past the tile's tokens are loaded but never stored
         const int nbox = p.box_rows >= TN ? 1 : (tile.n + p.box_rows - 1) / p.box_rows;
@@ -629,7 +624,7 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
     constexpr int kLag = R::kB / 2;  // groups in flight per thread before the oldest is published
     int gs = 0;                      // running group counter
     for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x) {
-      const TernTile tile = load_tile(p.tiles, item / RT, p.tile_slots);
+      const TernTile tile = load_tile(p.tiles, item / RT);
       const __half* rows[kRows];
 #pragma unroll
       for (int i = 0; i < kRows; ++i) {
@@ -669,10 +664,10 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
     if (lane == 0) {
       // ---------------- MMA issuer: A from tensor memory, B from shared memory
       int gs = 0, es = 0, li = 0;  // running group, A-entry and item counters
-      TernTile next = blockIdx.x < n_items ? load_tile(p.tiles, blockIdx.x / RT, p.tile_slots) : TernTile{};
+      TernTile next = blockIdx.x < n_items ? load_tile(p.tiles, blockIdx.x / RT) : TernTile{};
       for (int item = blockIdx.x; item < n_items && !abort_flag; item += gridDim.x, ++li) {
         const TernTile tile = next;  // loaded one item ahead: no global-load latency between items
-        if (item + int(gridDim.x) < n_items) next = load_tile(p.tiles, (item + gridDim.x) / RT, p.tile_slots);
+        if (item + int(gridDim.x) < n_items) next = load_tile(p.tiles, (item + gridDim.x) / RT);
         const uint32_t idesc = umma_idesc(kBM, (tile.n + 15) & ~15, 0);
         const int ab = li % R::n_acc;
         if (li >= R::n_acc && !mbar_wait(&acc_empty[ab], ((li / R::n_acc) - 1) & 1, &abort_flag, p.err)) break;
@@ -755,7 +750,7 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
     int li = 0;
     // no abort-flag test in the loop condition: the epilogue threads leave only together, by the vote
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++li) {
-      const TernTile tile = load_tile(p.tiles, item / RT, p.tile_slots);
+      const TernTile tile = load_tile(p.tiles, item / RT);
       const int rt = item % RT;
       const int64_t pos0 = tile.pos0;
       const int nn = tile.n;
@@ -983,7 +978,6 @@ size_t tern_smem_t() {
 }
 template <int FMT>
 size_t tern_smem_f(int na, int tn) {
-  if (tn == kBND) return na == 2 ? tern_smem_t<FMT, 2, kBND>() : tern_smem_t<FMT, 1, kBND>();
   if (na == 2) return tn == kBN3 ? tern_smem_t<FMT, 2, kBN3>() : tern_smem_t<FMT, 2, kBN>();
   return tn == kBN3 ? tern_smem_t<FMT, 1, kBN3>() : tern_smem_t<FMT, 1, kBN>();
 }
@@ -1041,15 +1035,6 @@ cudaError_t configure_prefill_kernels() {
   if ((e = cudaFuncSetAttribute(tern_gemm_kernel<SCION_PTQ1_0, 2, kBN3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 int(tern_smem(2, SCION_PTQ1_0, kBN3)))))
     return e;
-#define SCION_TC_DEC_SMEM(F, NA)                                                                 \
-  if ((e = cudaFuncSetAttribute(tern_gemm_kernel<F, NA, kBND>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                int(tern_smem(NA, F, kBND)))))                                   \
-    return e;
-  SCION_TC_DEC_SMEM(SCION_PQ2_0, 2)
-  SCION_TC_DEC_SMEM(SCION_PQ2_0, 1)
-  SCION_TC_DEC_SMEM(SCION_PTQ1_0, 2)
-  SCION_TC_DEC_SMEM(SCION_PTQ1_0, 1)
-#undef SCION_TC_DEC_SMEM
   return cudaSuccess;
 }
 
@@ -1219,7 +1204,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       const bool mid = tile_width(int64_t(T) * L->k, L->E) == kBN3;
       tp.tiles = static_cast<const TernTile*>(P.tiles), tp.n_tiles = P.n_tiles;
       tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gperm = P.gperm, tp.k = L->k;
-      tp.pexp = P.pexp, tp.tile_slots = 0, tp.box_rows = kBN, tp.out = nullptr;
+      tp.pexp = P.pexp, tp.box_rows = kBN, tp.out = nullptr;
       tp.h = P.h, tp.F = L->F, tp.y = nullptr, tp.d = L->d, tp.err = L->err;
       const dim3 grid(num_sms());
       if (L->fmt == SCION_PQ2_0 && mid)
@@ -1257,7 +1242,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       const int wd = tile_width(int64_t(T) * L->k, L->E);
       tp.tiles = static_cast<const TernTile*>(P.tiles), tp.n_tiles = P.n_tiles;
       tp.counts = P.counts, tp.offsets = P.offsets, tp.perm = P.perm, tp.gperm = P.gperm, tp.k = L->k;
-      tp.pexp = P.pexp, tp.tile_slots = 0, tp.box_rows = wd;
+      tp.pexp = P.pexp, tp.box_rows = wd;
       // fused gate-weighted scatter-add into out, or (deterministic) one row per entry for the combine
       tp.out = out, tp.y = L->deterministic ? P.y : nullptr;
       tp.h = nullptr, tp.F = L->F, tp.d = L->d, tp.err = L->err;
@@ -1327,31 +1312,6 @@ cudaError_t launch_corr_prefill(const CorrState* C, const __nv_bfloat16* v, int 
   dq.K = C->Kd, dq.T = T, dq.ab_bf16 = 0;
   dq.out = out, dq.ld_out = C->d_out, dq.resid = base, dq.xexp = C->xexp, dq.z_only = 1, dq.err = C->err;
   dense_gemm_kernel<<<dense_grid(dq), kThreads, kDenseSmem, s>>>(dq);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_tc_decode(int na, const scion_layer* L, int T, float* out, cudaStream_t s) {
-  TernParams tp;
-  memset(&tp, 0, sizeof(tp));
-  tp.fmt = L->fmt, tp.na = na, tp.k = L->k, tp.F = L->F, tp.d = L->d, tp.err = L->err;
-  tp.tiles = static_cast<const TernTile*>(L->slot_info), tp.tile_slots = 1, tp.n_tiles = L->n_active;
-  tp.counts = L->counts, tp.offsets = L->offsets, tp.perm = L->perm, tp.gperm = L->gperm, tp.pexp = L->pexp;
-  if (na == 2) {
-    tp.bank = L->gu_bank, tp.G = L->Gd, tp.R = L->F, tp.bsrc = L->x16d, tp.ldb = L->d, tp.h = L->hp;
-    tp.box_rows = kBND;
-  } else {
-    tp.bank = L->dn_bank, tp.G = L->GF, tp.R = L->d, tp.bsrc = L->hp, tp.ldb = L->F, tp.out = out;
-    tp.bmap = L->hp_map, tp.box_rows = 16;
-  }
-  const int items = std::min(L->E, T * L->k) * (tp.R / 128);
-  const dim3 grid(std::max(1, std::min(items, num_sms())));
-#define SCION_TCD(F, NA) tern_gemm_kernel<F, NA, kBND><<<grid, kTernThreads, tern_smem(NA, F, kBND), s>>>(tp)
-  if (L->fmt == SCION_PQ2_0) {
-    if (na == 2) SCION_TCD(SCION_PQ2_0, 2); else SCION_TCD(SCION_PQ2_0, 1);
-  } else {
-    if (na == 2) SCION_TCD(SCION_PTQ1_0, 2); else SCION_TCD(SCION_PTQ1_0, 1);
-  }
-#undef SCION_TCD
   return cudaGetLastError();
 }
 

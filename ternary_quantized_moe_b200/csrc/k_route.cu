@@ -194,17 +194,19 @@ __device__ __forceinline__ void group_staged(const int32_t* ids_s, const float* 
                                              int32_t* __restrict__ counts_out, int32_t* __restrict__ offsets_out,
                                              int32_t* __restrict__ perm_out, float* __restrict__ gperm_out,
                                              int32_t* __restrict__ pexp_out, int32_t* __restrict__ active_out,
-                                             int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info) {
+                                             int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info,
+                                             int4* __restrict__ dtiles, int32_t* __restrict__ n_dtiles) {
   const int per = (E + 31) / 32;
   const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
-  int sc = 0, ac = 0;
-  for (int e = e0; e < e1; ++e) sc += counts[e], ac += counts[e] > 0;
-  int si = sc, ai = ac;
+  int sc = 0, ac = 0, tc = 0;
+  for (int e = e0; e < e1; ++e) sc += counts[e], ac += counts[e] > 0, tc += (counts[e] + kDecTile - 1) / kDecTile;
+  int si = sc, ai = ac, ti = tc;
   for (int o = 1; o < 32; o <<= 1) {
     const int s2 = __shfl_up_sync(0xffffffffu, si, o), a2 = __shfl_up_sync(0xffffffffu, ai, o);
-    if (lane >= o) si += s2, ai += a2;
+    const int t2 = __shfl_up_sync(0xffffffffu, ti, o);
+    if (lane >= o) si += s2, ai += a2, ti += t2;
   }
-  int run = si - sc, arun = ai - ac;
+  int run = si - sc, arun = ai - ac, trun = ti - tc;
   for (int e = e0; e < e1; ++e) {
     const int c = counts[e];
     offsets_out[e] = run;
@@ -215,9 +217,11 @@ __device__ __forceinline__ void group_staged(const int32_t* ids_s, const float* 
       slot_info[arun] = make_int4(e, run, c, 0);
       ++arun;
     }
+    // tiles of the tensor-core decode kernels: {expert, first token, tokens, first position}
+    for (int c0 = 0; c0 < c; c0 += kDecTile) dtiles[trun++] = make_int4(e, c0, min(kDecTile, c - c0), run + c0);
     run += c;
   }
-  if (lane == 31) offsets_out[E] = si, *n_active_out = ai;
+  if (lane == 31) offsets_out[E] = si, *n_active_out = ai, *n_dtiles = ti;
   __syncwarp();
   // stable scatter in (token, slot) order, 32 entries at a time
   const unsigned lt = (1u << lane) - 1u;
@@ -252,7 +256,7 @@ __global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
     float* __restrict__ gates, int32_t* __restrict__ counts_out, int32_t* __restrict__ offsets_out,
     int32_t* __restrict__ perm_out, float* __restrict__ gperm_out, int32_t* __restrict__ active_out,
     int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info, const int32_t* __restrict__ xexp,
-    int32_t* __restrict__ pexp_out) {
+    int32_t* __restrict__ pexp_out, int4* __restrict__ dtiles, int32_t* __restrict__ n_dtiles) {
   extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [E] | cursor [E] | xexp [T]
   const int n = T * k;
   int32_t* ids_s = reinterpret_cast<int32_t*>(rs);
@@ -277,7 +281,7 @@ __global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
   __syncthreads();
   if (warp == 0)
     group_staged(ids_s, gates_s, xexp_s, n, k, E, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out,
-                 pexp_out, active_out, n_active_out, slot_info);
+                 pexp_out, active_out, n_active_out, slot_info, dtiles, n_dtiles);
 }
 
 // ceil(T/4) CTAs of 4 warps (T > 32); the last CTA to finish groups.
@@ -289,7 +293,8 @@ __global__ void __launch_bounds__(kRmThreads) route_multi_kernel(
     float* __restrict__ gates, int32_t* __restrict__ counts_out, int32_t* __restrict__ offsets_out,
     int32_t* __restrict__ perm_out, float* __restrict__ gperm_out, int32_t* __restrict__ active_out,
     int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info, unsigned* __restrict__ done,
-    const int32_t* __restrict__ xexp, int32_t* __restrict__ pexp_out) {
+    const int32_t* __restrict__ xexp, int32_t* __restrict__ pexp_out, int4* __restrict__ dtiles,
+    int32_t* __restrict__ n_dtiles) {
   extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [E] | cursor [E] | xexp [T]
   __shared__ int last;
   const int n = T * k;
@@ -318,7 +323,7 @@ __global__ void __launch_bounds__(kRmThreads) route_multi_kernel(
   if (warp != 0) return;
   if (lane == 0) *done = 0;
   group_staged(ids_s, gates_s, xexp_s, n, k, E, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out,
-               pexp_out, active_out, n_active_out, slot_info);
+               pexp_out, active_out, n_active_out, slot_info, dtiles, n_dtiles);
 }
 
 size_t route_cta_smem(int T, int E, int k) { return sizeof(float) * (2 * size_t(T) * k + 2 * size_t(E) + size_t(T)); }
@@ -340,11 +345,11 @@ cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s) {
   return T <= 32 ? launch_pdl(route_cta_kernel<V>, dim3(1), dim3(rc_threads<V>()), smem, s, L->logits, T, L->E, \
                               L->k, L->desc.norm_topk, L->ids, L->gates, L->counts, L->offsets, L->perm,       \
                               L->gperm, L->active, L->n_active, reinterpret_cast<int4*>(L->slot_info), L->xexp, \
-                              L->pexp)                                                                         \
+                              L->pexp, reinterpret_cast<int4*>(L->dtiles), L->n_dtiles)                        \
                  : launch_pdl(route_multi_kernel<V>, dim3((T + 3) / 4), dim3(kRmThreads), smem, s, L->logits, T, \
                               L->E, L->k, L->desc.norm_topk, L->ids, L->gates, L->counts, L->offsets, L->perm, \
                               L->gperm, L->active, L->n_active, reinterpret_cast<int4*>(L->slot_info),         \
-                              L->route_done, L->xexp, L->pexp)
+                              L->route_done, L->xexp, L->pexp, reinterpret_cast<int4*>(L->dtiles), L->n_dtiles)
     if (vpl <= 1) SCION_ROUTE_CTA(1);
     else if (vpl <= 2) SCION_ROUTE_CTA(2);
     else if (vpl <= 4) SCION_ROUTE_CTA(4);

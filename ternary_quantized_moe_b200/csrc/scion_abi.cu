@@ -45,7 +45,8 @@ void free_layer(scion_layer* L) {
   void* ptrs[] = {L->gu_bank, L->dn_bank,  L->dense_down, L->xunits,  L->logits,    L->ids,       L->gates,
                   L->counts,  L->offsets,  L->perm,       L->active,  L->n_active,  L->h,         L->hz,
                   L->xfrag,   L->x_stage, L->out_stage, L->bad,       L->err,
-                  L->slot_info, L->gperm, L->route_done, L->xexp, L->pexp, L->x16d, L->hp};
+                  L->slot_info, L->gperm, L->route_done, L->xexp, L->pexp, L->x16d, L->hp,
+                  L->dtiles, L->n_dtiles, L->xsum, L->hsum};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   if (L->side) cudaStreamDestroy(L->side);
@@ -218,7 +219,9 @@ int forward_prefill(const scion_layer* L, const __nv_bfloat16* x, int T, float* 
 int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, const float* resid, cudaStream_t s) {
   if (L->desc.router_fp32) SCION_STAGE(SCION_STAGE_ROUTER_F32, scion::launch_router_f32(L, x, T, L->logits, s));
   const bool ring = T >= L->stream_min_tokens;
-  const bool tcd = ring && L->tc_decode;  // tcgen05 expert GEMMs instead of the bulk-copy ring kernels
+  // tcgen05 expert GEMMs instead of the bulk-copy ring kernels (their tiles come from the grouping
+  // kernels of up to 512 experts)
+  const bool tcd = ring && L->tc_decode && L->E <= 512;
   // Batches on the ring kernels split the dense work off the expert path: the caller's stream
   // runs the router part of the x-projection (with x's fragment rows and the clearing of out),
   // the layer's side stream the shared-expert / correction part and the dense down projection,
@@ -251,11 +254,11 @@ int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out
   // small batches: the dense down projection rides in the gate/up launch (it needs only the
   // x-projection), off the critical path of the routed kernels
   const bool merged = !ring && scion::gateup_merges_dense(L, T);
-  SCION_STAGE_INTO(st, SCION_STAGE_GATEUP, tcd      ? scion::launch_tc_decode(2, L, T, out, s)
+  SCION_STAGE_INTO(st, SCION_STAGE_GATEUP, tcd      ? scion::launch_tdec(2, L, T, out, s)
                                            : ring   ? scion::launch_stream_gateup(L, T, s)
                                            : merged ? scion::launch_gateup_dense(L, T, out, s)
                                                     : scion::launch_gateup(L, x, T, s));
-  SCION_STAGE_INTO(st, SCION_STAGE_DOWN_ROUTED, tcd    ? scion::launch_tc_decode(1, L, T, out, s)
+  SCION_STAGE_INTO(st, SCION_STAGE_DOWN_ROUTED, tcd    ? scion::launch_tdec(1, L, T, out, s)
                                                 : ring ? scion::launch_stream_down(L, T, out, s)
                                                        : scion::launch_down_routed(L, T, out, s));
   if (side) {
@@ -347,6 +350,11 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   SCION_TRY(dev_alloc(L, &L->xfrag, sizeof(__half) * TD * L->Gd * SCION_BROW));
   SCION_TRY(dev_alloc(L, &L->xexp, sizeof(int32_t) * TD));
   SCION_TRY(dev_alloc(L, &L->pexp, sizeof(int32_t) * TD * L->k));
+  SCION_TRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&L->dtiles),
+                      sizeof(int4) * (size_t(TD) * L->k / scion::kDecTile + L->E + 1)));
+  SCION_TRY(dev_alloc(L, &L->n_dtiles, sizeof(int32_t)));
+  SCION_TRY(dev_alloc(L, &L->xsum, sizeof(float) * TD * L->Gd));
+  SCION_TRY(dev_alloc(L, &L->hsum, sizeof(float) * TD * L->k * L->GF));
   SCION_TRY(dev_alloc(L, &L->x16d, sizeof(__half) * TD * L->d));
   SCION_TRY(dev_alloc(L, &L->hp, sizeof(__half) * TD * L->k * L->F));
   SCION_TRY(dev_alloc(L, &L->x_stage, sizeof(__nv_bfloat16) * size_t(max_tokens) * L->d));
@@ -474,7 +482,7 @@ extern "C" int scion_moe_forward_debug(const void* x, int T, const scion_layer* 
   cp(dbg->perm, pre ? P->perm : L->perm, sizeof(int32_t) * size_t(T) * L->k);
   if (dbg->h && e == cudaSuccess)
     e = pre ? scion::launch_unperm_prefill(L->fmt, P->h, int64_t(T) * L->k * L->F, reinterpret_cast<__half*>(dbg->h), s)
-        : (T >= L->stream_min_tokens && L->tc_decode)
+        : (T >= L->stream_min_tokens && L->tc_decode && L->E <= 512)
             ? scion::launch_unperm_prefill(L->fmt, L->hp, int64_t(T) * L->k * L->F, reinterpret_cast<__half*>(dbg->h), s)
             : scion::launch_unfrag(L->fmt, L->h, T * L->k, L->GF, reinterpret_cast<__half*>(dbg->h), s);
   if (dbg->hz && e == cudaSuccess && L->Kdense)

@@ -34,6 +34,9 @@
 
 #define SCION_TDEC 64         // tokens of the decode path (larger batches take the tensor-core path)
 #define SCION_XPROJ_KC 512    // K columns per x-projection CTA (4 warps x 128)
+namespace scion {
+constexpr int kDecTile = 16;  // tokens per tile of the tensor-core decode kernels (one MMA N)
+}
 
 // Fragment-ordered B operands of the decode expert kernels (x for gate/up, h for down) are
 // stored per 128-column group as 128 fp16 values followed by a 16-byte tail; the first 4
@@ -146,6 +149,10 @@ struct scion_layer {
   __half* xfrag;     // [TDEC][Gd][SCION_BROW] x in fragment order (fp16) + group-sum tails
   int32_t* xexp;     // [TDEC] per-token range exponent s_t (see token_shift)
   int32_t* pexp;     // [TDEC*k] s_t of the token of each routed position (written by the routing)
+  void* dtiles;      // int4 [TDEC*k/kDecTile + E]: tiles of <= kDecTile tokens per active expert (routing)
+  int32_t* n_dtiles; // [1]
+  float* xsum;       // [TDEC][Gd] per-group sums of the tensor-core decode's B values times 4^f (x)
+  float* hsum;       // [TDEC*k][GF] the same for the expert hidden
   // tensor-core decode (batches on the ring threshold and above, tc_decode = 1): x 2^s_t in the
   // tcgen05 column order, the expert hidden one row per routed position, and its TMA map (16-row boxes)
   __half* x16d;      // [TDEC][d]
@@ -217,9 +224,10 @@ cudaError_t launch_corr_prefill(const CorrState* C, const __nv_bfloat16* v, int 
 
 // k_prefill.cu
 int make_tmap_2d(CUtensorMap* map, const void* ptr, int bf16, int64_t rows, int64_t K, int box_rows = 128);
-// Expert gate/up (na = 2) or down (na = 1, gate-weighted fp32 reductions into out) of a decode
-// batch on the tcgen05 grouped GEMM, one tile per active expert.
-cudaError_t launch_tc_decode(int na, const scion_layer* L, int T, float* out, cudaStream_t s);
+// k_tdec.cu: expert gate/up (na = 2) or down (na = 1, gate-weighted fp32 reductions into out) of
+// a decode batch on the tensor cores, tiles of up to kDecTile tokens listed by the routing.
+cudaError_t configure_tdec_kernels();
+cudaError_t launch_tdec(int na, const scion_layer* L, int T, float* out, cudaStream_t s);
 cudaError_t configure_prefill_kernels();
 size_t prefill_unit_bytes();
 size_t prefill_tile_bytes();
