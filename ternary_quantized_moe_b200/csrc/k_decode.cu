@@ -79,12 +79,12 @@ __device__ __forceinline__ void xproj_aux(const XProjArgs& a, int aux, int n_aux
   const int lane = threadIdx.x & 31;
   const int gw = aux * (kXThreads / 32) + (threadIdx.x >> 5), nw = n_aux * (kXThreads / 32);
   // Warps share the tokens out (wpt warps per token, each a slice of its pairs of 128-column
-  // groups).  Each warp loads its token's whole row into registers (16 bytes per lane per pair,
-  // all loads in flight at once); their largest magnitude fixes the range exponent s_t.  Each of
-  // its pairs then goes through shared memory, where lane (gl, part) gathers the 8 columns of its
-  // output positions in group 2 pr + gl and writes x 2^s_t in the tcgen05 order (a.x16) or the
-  // fragment order with the group sums of B * 4^f in the row tails.
-  constexpr int kMaxPairs = 16;  // d <= 4096
+  // groups).  Each warp streams its token's whole row once for the largest magnitude, which
+  // fixes the range exponent s_t; each of its pairs is then read again (coalesced, from cache)
+  // into shared memory, where lane (gl, part) gathers the 8 columns of its output positions in
+  // group 2 pr + gl and writes x 2^s_t in the tcgen05 order (a.x16) or the fragment order with
+  // the group sums of B * 4^f in the row tails.  (Nothing is held across the two passes: the
+  // registers of this path would otherwise bound the x-projection CTAs' occupancy.)
   __shared__ __align__(16) __nv_bfloat16 pbuf[kXThreads / 32][256];
   __nv_bfloat16* buf = pbuf[threadIdx.x >> 5];
   const int wpt = max(1, nw / max(1, a.T));
@@ -92,25 +92,18 @@ __device__ __forceinline__ void xproj_aux(const XProjArgs& a, int aux, int n_aux
   for (int job = gw; job < a.T * wpt; job += nw) {
     const int t = job / wpt, slice = job % wpt;
     const __nv_bfloat16* row = a.x + int64_t(t) * a.d;
-    uint4 v[kMaxPairs];
     uint32_t mx = 0;
-#pragma unroll
-    for (int j = 0; j < kMaxPairs; ++j) {
-      const bool ld = j < n_pairs && 2 * j + gl < Gd;  // an odd group count leaves the last pair half empty
-      v[j] = ld ? *reinterpret_cast<const uint4*>(row + 256 * j + 8 * lane) : make_uint4(0u, 0u, 0u, 0u);
-      mx = max(mx, max_mag8(v[j]));
-    }
+#pragma unroll 1
+    for (int i = lane; i < a.d / 8; i += 32) mx = max(mx, max_mag8(*reinterpret_cast<const uint4*>(row + 8 * i)));
     const int sh = token_shift(__reduce_max_sync(0xffffffffu, mx));
     if (lane == 0 && slice == 0) a.xexp[t] = sh;
     const float xs = pow2i(sh);
-#pragma unroll
-    for (int pr = 0; pr < kMaxPairs; ++pr) {
-      if (pr >= n_pairs) break;
-      if (pr % wpt != slice) continue;
+    for (int pr = slice; pr < n_pairs; pr += wpt) {
       const int g = 2 * pr + gl;
-      const bool ok = g < Gd;
+      const bool ok = g < Gd;  // an odd group count leaves the last pair half empty
+      const uint4 v = ok ? *reinterpret_cast<const uint4*>(row + 256 * pr + 8 * lane) : make_uint4(0u, 0u, 0u, 0u);
       __syncwarp();
-      *reinterpret_cast<uint4*>(buf + 8 * lane) = v[pr];
+      *reinterpret_cast<uint4*>(buf + 8 * lane) = v;
       __syncwarp();
       const __nv_bfloat16* src = buf + 128 * gl;
       __align__(16) __half o[8];
