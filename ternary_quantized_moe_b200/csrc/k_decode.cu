@@ -59,7 +59,7 @@ struct XProjArgs {
 // chunks of a unit are one thread-block cluster, reduced through distributed shared memory.
 // kXAux extra CTA columns convert x to the fragment order and clear out and the hidden tails.
 constexpr int kXRow = SCION_XPROJ_KC + 8;  // bf16 elements per staged token row (+16 B pad)
-constexpr int kXAux = 4;
+constexpr int kXAux = 8;
 constexpr int kXThreads = 256;  // 8 warps x 64 columns
 
 template <int NT>

@@ -61,7 +61,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
                                                               int32_t* __restrict__ active_out,
                                                               int32_t* __restrict__ n_active_out,
                                                               const int32_t* __restrict__ xexp,
-                                                              int32_t* __restrict__ pexp_out) {
+                                                              int32_t* __restrict__ pexp_out,
+                                                              int32_t* __restrict__ any_scaled) {
   extern __shared__ float smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = kRouteThreads / 32;
   float* vals = smem + warp * E;
@@ -155,6 +156,10 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
       offsets_out[E] = si;
       *n_active_out = ai;
     }
+    int sc_any = 0;
+    for (int t = lane; t < T; t += 32) sc_any |= xexp[t] != 0;
+    sc_any = __any_sync(0xffffffffu, sc_any);
+    if (lane == 0) *any_scaled = sc_any;
     __syncwarp();
     // ---- stable scatter in (token, slot) order, 32 entries at a time
     const int n = T * k;
@@ -195,7 +200,8 @@ __device__ __forceinline__ void group_staged(const int32_t* ids_s, const float* 
                                              int32_t* __restrict__ perm_out, float* __restrict__ gperm_out,
                                              int32_t* __restrict__ pexp_out, int32_t* __restrict__ active_out,
                                              int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info,
-                                             int4* __restrict__ dtiles, int32_t* __restrict__ n_dtiles) {
+                                             int4* __restrict__ dtiles, int32_t* __restrict__ n_dtiles,
+                                             int32_t* __restrict__ any_scaled) {
   const int per = (E + 31) / 32;
   const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
   int sc = 0, ac = 0, tc = 0;
@@ -218,10 +224,19 @@ __device__ __forceinline__ void group_staged(const int32_t* ids_s, const float* 
       ++arun;
     }
     // tiles of the tensor-core decode kernels: {expert, first token, tokens, first position}
-    for (int c0 = 0; c0 < c; c0 += kDecTile) dtiles[trun++] = make_int4(e, c0, min(kDecTile, c - c0), run + c0);
+    if (dtiles)
+      for (int c0 = 0; c0 < c; c0 += kDecTile) dtiles[trun++] = make_int4(e, c0, min(kDecTile, c - c0), run + c0);
     run += c;
   }
-  if (lane == 31) offsets_out[E] = si, *n_active_out = ai, *n_dtiles = ti;
+  if (lane == 31) {
+    offsets_out[E] = si, *n_active_out = ai;
+    if (dtiles) *n_dtiles = ti;
+  }
+  // whether any token of the batch is range-scaled (the expert epilogues skip the factors if not)
+  int sc_any = 0;
+  for (int t = lane; t < n / k; t += 32) sc_any |= xexp_s[t] != 0;
+  sc_any = __any_sync(0xffffffffu, sc_any);
+  if (lane == 0) *any_scaled = sc_any;
   __syncwarp();
   // stable scatter in (token, slot) order, 32 entries at a time
   const unsigned lt = (1u << lane) - 1u;
@@ -256,7 +271,8 @@ __global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
     float* __restrict__ gates, int32_t* __restrict__ counts_out, int32_t* __restrict__ offsets_out,
     int32_t* __restrict__ perm_out, float* __restrict__ gperm_out, int32_t* __restrict__ active_out,
     int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info, const int32_t* __restrict__ xexp,
-    int32_t* __restrict__ pexp_out, int4* __restrict__ dtiles, int32_t* __restrict__ n_dtiles) {
+    int32_t* __restrict__ pexp_out, int4* __restrict__ dtiles, int32_t* __restrict__ n_dtiles,
+    int32_t* __restrict__ any_scaled) {
   extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [E] | cursor [E] | xexp [T]
   const int n = T * k;
   int32_t* ids_s = reinterpret_cast<int32_t*>(rs);
@@ -281,7 +297,7 @@ __global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
   __syncthreads();
   if (warp == 0)
     group_staged(ids_s, gates_s, xexp_s, n, k, E, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out,
-                 pexp_out, active_out, n_active_out, slot_info, dtiles, n_dtiles);
+                 pexp_out, active_out, n_active_out, slot_info, dtiles, n_dtiles, any_scaled);
 }
 
 // ceil(T/4) CTAs of 4 warps (T > 32); the last CTA to finish groups.
@@ -294,7 +310,7 @@ __global__ void __launch_bounds__(kRmThreads) route_multi_kernel(
     int32_t* __restrict__ perm_out, float* __restrict__ gperm_out, int32_t* __restrict__ active_out,
     int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info, unsigned* __restrict__ done,
     const int32_t* __restrict__ xexp, int32_t* __restrict__ pexp_out, int4* __restrict__ dtiles,
-    int32_t* __restrict__ n_dtiles) {
+    int32_t* __restrict__ n_dtiles, int32_t* __restrict__ any_scaled) {
   extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [E] | cursor [E] | xexp [T]
   __shared__ int last;
   const int n = T * k;
@@ -323,7 +339,7 @@ __global__ void __launch_bounds__(kRmThreads) route_multi_kernel(
   if (warp != 0) return;
   if (lane == 0) *done = 0;
   group_staged(ids_s, gates_s, xexp_s, n, k, E, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out,
-               pexp_out, active_out, n_active_out, slot_info, dtiles, n_dtiles);
+               pexp_out, active_out, n_active_out, slot_info, dtiles, n_dtiles, any_scaled);
 }
 
 size_t route_cta_smem(int T, int E, int k) { return sizeof(float) * (2 * size_t(T) * k + 2 * size_t(E) + size_t(T)); }
@@ -340,16 +356,19 @@ cudaError_t launch_router_f32(const scion_layer* L, const __nv_bfloat16* x, int 
 cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s) {
   if (L->E <= 512) {
     const size_t smem = route_cta_smem(T, L->E, L->k);
+    // tile list only for the tensor-core decode kernels (stream_min_tokens and up, option set)
+    int4* dtl = (L->tc_decode && T >= L->stream_min_tokens) ? reinterpret_cast<int4*>(L->dtiles) : nullptr;
     const int vpl = (L->E + 31) / 32;
 #define SCION_ROUTE_CTA(V)                                                                                     \
   return T <= 32 ? launch_pdl(route_cta_kernel<V>, dim3(1), dim3(rc_threads<V>()), smem, s, L->logits, T, L->E, \
                               L->k, L->desc.norm_topk, L->ids, L->gates, L->counts, L->offsets, L->perm,       \
                               L->gperm, L->active, L->n_active, reinterpret_cast<int4*>(L->slot_info), L->xexp, \
-                              L->pexp, reinterpret_cast<int4*>(L->dtiles), L->n_dtiles)                        \
+                              L->pexp, dtl, L->n_dtiles, L->any_scaled)                                        \
                  : launch_pdl(route_multi_kernel<V>, dim3((T + 3) / 4), dim3(kRmThreads), smem, s, L->logits, T, \
                               L->E, L->k, L->desc.norm_topk, L->ids, L->gates, L->counts, L->offsets, L->perm, \
                               L->gperm, L->active, L->n_active, reinterpret_cast<int4*>(L->slot_info),         \
-                              L->route_done, L->xexp, L->pexp, reinterpret_cast<int4*>(L->dtiles), L->n_dtiles)
+                              L->route_done, L->xexp, L->pexp, dtl, L->n_dtiles,                               \
+                              L->any_scaled)
     if (vpl <= 1) SCION_ROUTE_CTA(1);
     else if (vpl <= 2) SCION_ROUTE_CTA(2);
     else if (vpl <= 4) SCION_ROUTE_CTA(4);
@@ -362,7 +381,7 @@ cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s) {
                 sizeof(int32_t) * size_t(T) * L->k;
   route_kernel<<<1, kRouteThreads, smem, s>>>(L->logits, T, L->E, L->k, L->desc.norm_topk, L->ids, L->gates,
                                                L->counts, L->offsets, L->perm, L->gperm, L->active, L->n_active,
-                                               L->xexp, L->pexp);
+                                               L->xexp, L->pexp, L->any_scaled);
   if (cudaError_t e = cudaGetLastError()) return e;
   return launch_slot_info(L, s);
 }

@@ -34,11 +34,9 @@ struct StageHdr {
   int flags;  // bit 0: first stage of the pass, bit 1: last stage of the pass
   int rb;     // 128-row block of the item
   int ng;     // 128-column groups in this stage (1..GPS)
-  int pos[kTok];     // routed positions of the pass's tokens (last stage only)
-  int orow[kTok];    // output token row (entry / k)
-  float gate[kTok];  // gate of the entry times 2^(-2 s_t) (the hidden is h 2^(2 s_t))
-  float xdn[kTok];   // gate/up: 2^-s_t and 2^s_t of the token's range exponent (the sums are of x 2^s_t)
-  float xup[kTok];
+  int pos[kTok];     // gate/up: routed positions of the pass's tokens (last stage only)
+  int orow[kTok];    // down: output token row (entry / k)
+  float gate[kTok];  // down: gate of the entry times 2^(-2 s_t) (the hidden is h 2^(2 s_t))
 };
 static_assert(sizeof(StageHdr) <= kHdr, "stage header");
 
@@ -50,6 +48,7 @@ struct StreamArgs {
   const int32_t *n_active, *perm;
   const float* gperm;  // gate of each routed position, times 2^(-2 s_t)
   const int32_t* pexp; // range exponent s_t of the token of each routed position
+  const int32_t* any_scaled;  // nonzero when some token of the batch has s_t != 0 (written by the routing)
   int G, R, k, F, d, fmt;
   __half* hfrag;  // gate/up output
   float* out;     // down output
@@ -58,7 +57,7 @@ struct StreamArgs {
 
 struct TokInfo {
   int pos, brow, orow;
-  float gate, xdn, xup;
+  float gate;
 };
 
 // Groups per stage: two for the gate/up bank (each group holds both matrices), four for down.
@@ -241,13 +240,11 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
     const int n_items = *a.n_active * RB;
     auto slot_rec = [&](int item) { return item < n_items ? a.slot_info[item / RB] : make_int4(0, 0, 0, 0); };
     auto tok_info = [&](int4 si, int pc) {
-      TokInfo t{0, 0, 0, 0.f, 1.f, 1.f};
+      TokInfo t{0, 0, 0, 0.f};
       if (lane < min(kTok, si.z - pc)) {
         t.pos = si.y + pc + lane;
         t.orow = a.perm[t.pos] / a.k;
-        const int sh = a.pexp[t.pos];
-        t.gate = a.gperm[t.pos];
-        t.xdn = pow2i(-sh), t.xup = pow2i(sh);
+        if (NMAT == 1) t.gate = a.gperm[t.pos];
         t.brow = NMAT == 2 ? t.orow : t.pos;
       }
       return t;
@@ -286,18 +283,21 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
           if (last) {
             // the epilogue's per-token records, written by lane 0 so its arrive publishes them
 #pragma unroll
+            // (the producer's per-stage work bounds the ring: only what the epilogue reads)
             for (int i = 0; i < kTok; ++i) {
-              const int pos = __shfl_sync(0xffffffffu, tk.pos, i), orow = __shfl_sync(0xffffffffu, tk.orow, i);
-              const float gate = __shfl_sync(0xffffffffu, tk.gate, i);
-              const float xdn = __shfl_sync(0xffffffffu, tk.xdn, i), xup = __shfl_sync(0xffffffffu, tk.xup, i);
-              if (lane == 0) hd->pos[i] = pos, hd->orow[i] = orow, hd->gate[i] = gate, hd->xdn[i] = xdn, hd->xup[i] = xup;
+              if constexpr (NMAT == 2) {
+                const int pos = __shfl_sync(0xffffffffu, tk.pos, i);
+                if (lane == 0) hd->pos[i] = pos;
+              } else {
+                const int orow = __shfl_sync(0xffffffffu, tk.orow, i);
+                const float gate = __shfl_sync(0xffffffffu, tk.gate, i);
+                if (lane == 0) hd->orow[i] = orow, hd->gate[i] = gate;
+              }
             }
           }
-          // bit 2: some token of the pass is range-scaled (its epilogue factors are not all 1)
-          const bool scaled = __any_sync(0xffffffffu, tk.xup != 1.f);
           if (lane == 0) {
             hd->nn = nn;
-            hd->flags = (g0 == 0 ? 1 : 0) | (last ? 2 : 0) | (scaled ? 4 : 0);
+            hd->flags = (g0 == 0 ? 1 : 0) | (last ? 2 : 0);
             hd->rb = rb;
             hd->ng = ng;
             mbar_arrive_expect_tx(&full[s], ng * cb + nn * ng * kRowB);
@@ -328,6 +328,7 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
   }
 
   // ---------------- consumers: warp w owns rows 16w .. 16w+15 of every item
+  const bool scaled = NMAT == 2 && *a.any_scaled != 0;
   const int c = lane & 3;
   constexpr int tb = FMT == SCION_PQ2_0 ? kPq2Tile : kPtq1Tile;
   LaneOffs lo;
@@ -377,9 +378,13 @@ __global__ void __launch_bounds__((kCons + 1) * 32, 2) stream_kernel(const __gri
         const int row = warp * 16 + (lane >> 2) + 8 * (i >> 1);
         const int tcol = 2 * c + (i & 1);
         if constexpr (NMAT == 2) {
-          const float h = (flags & 4) ? silu_f(acc[0][i] * unit * hd->xdn[tcol]) * (acc[1][i] * unit * hd->xup[tcol]) *
-                                            hsc[i >> 1]
-                                      : silu_f(acc[0][i] * unit) * (acc[1][i] * unit) * hsc[i >> 1];
+          float h;
+          if (!scaled) {
+            h = silu_f(acc[0][i] * unit) * (acc[1][i] * unit) * hsc[i >> 1];
+          } else {  // some token of the batch is range-scaled: the sums are of x 2^sh
+            const int sh = tcol < nn ? a.pexp[hd->pos[tcol]] : 0;
+            h = silu_f(acc[0][i] * unit * pow2i(-sh)) * (acc[1][i] * unit * pow2i(sh)) * hsc[i >> 1];
+          }
           const __half h16 = __float2half_rn(h);
           if (tcol < nn) a.hfrag[(int64_t(hd->pos[tcol]) * (a.F >> 7) + rb) * SCION_BROW + hpos[i >> 1]] = h16;
           if (FMT == SCION_PQ2_0) hs[i & 1] += __half2float(h16) * hinv[i >> 1];
@@ -462,7 +467,7 @@ cudaError_t launch_stream_gateup(const scion_layer* L, int T, cudaStream_t s) {
   StreamArgs a;
   a.bank = L->gu_bank, a.bsrc = L->xfrag, a.bld = L->Gd;
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
-  a.gperm = L->gperm, a.pexp = L->pexp, a.G = L->Gd, a.R = L->F, a.k = L->k, a.F = L->F, a.d = L->d, a.fmt = L->fmt;
+  a.gperm = L->gperm, a.pexp = L->pexp, a.any_scaled = L->any_scaled, a.G = L->Gd, a.R = L->F, a.k = L->k, a.F = L->F, a.d = L->d, a.fmt = L->fmt;
   a.hfrag = L->h, a.out = nullptr, a.err = L->err;
   const int max_items = min(L->E, T * L->k) * (L->F / 128);
   if (L->fmt == SCION_PQ2_0) return launch_stream<SCION_PQ2_0, 2>(a, max_items, s);
@@ -473,7 +478,7 @@ cudaError_t launch_stream_down(const scion_layer* L, int T, float* out, cudaStre
   StreamArgs a;
   a.bank = L->dn_bank, a.bsrc = L->h, a.bld = L->GF;
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
-  a.gperm = L->gperm, a.pexp = L->pexp, a.G = L->GF, a.R = L->d, a.k = L->k, a.F = L->F, a.d = L->d, a.fmt = L->fmt;
+  a.gperm = L->gperm, a.pexp = L->pexp, a.any_scaled = L->any_scaled, a.G = L->GF, a.R = L->d, a.k = L->k, a.F = L->F, a.d = L->d, a.fmt = L->fmt;
   a.hfrag = nullptr, a.out = out, a.err = L->err;
   const int max_items = min(L->E, T * L->k) * (L->d / 128);
   if (L->fmt == SCION_PQ2_0) return launch_stream<SCION_PQ2_0, 1>(a, max_items, s);

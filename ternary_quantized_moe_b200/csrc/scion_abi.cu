@@ -46,7 +46,7 @@ void free_layer(scion_layer* L) {
                   L->counts,  L->offsets,  L->perm,       L->active,  L->n_active,  L->h,         L->hz,
                   L->xfrag,   L->x_stage, L->out_stage, L->bad,       L->err,
                   L->slot_info, L->gperm, L->route_done, L->xexp, L->pexp, L->x16d, L->hp,
-                  L->dtiles, L->n_dtiles, L->xsum, L->hsum};
+                  L->dtiles, L->n_dtiles, L->xsum, L->hsum, L->any_scaled};
   for (void* p : ptrs)
     if (p) cudaFree(p);
   if (L->side) cudaStreamDestroy(L->side);
@@ -353,6 +353,7 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   SCION_TRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&L->dtiles),
                       sizeof(int4) * (size_t(TD) * L->k / scion::kDecTile + L->E + 1)));
   SCION_TRY(dev_alloc(L, &L->n_dtiles, sizeof(int32_t)));
+  SCION_TRY(dev_alloc(L, &L->any_scaled, sizeof(int32_t)));
   SCION_TRY(dev_alloc(L, &L->xsum, sizeof(float) * TD * L->Gd));
   SCION_TRY(dev_alloc(L, &L->hsum, sizeof(float) * TD * L->k * L->GF));
   SCION_TRY(dev_alloc(L, &L->x16d, sizeof(__half) * TD * L->d));

@@ -149,6 +149,7 @@ struct scion_layer {
   __half* xfrag;     // [TDEC][Gd][SCION_BROW] x in fragment order (fp16) + group-sum tails
   int32_t* xexp;     // [TDEC] per-token range exponent s_t (see token_shift)
   int32_t* pexp;     // [TDEC*k] s_t of the token of each routed position (written by the routing)
+  int32_t* any_scaled;  // [1] nonzero when some token of the pass has s_t != 0 (written by the routing)
   void* dtiles;      // int4 [TDEC*k/kDecTile + E]: tiles of <= kDecTile tokens per active expert (routing)
   int32_t* n_dtiles; // [1]
   float* xsum;       // [TDEC][Gd] per-group sums of the tensor-core decode's B values times 4^f (x)
