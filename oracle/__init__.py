@@ -95,6 +95,8 @@ def _load():
             lib.oracle_route.argtypes = [C.POINTER(_Layer), vp, ci, vp, vp, vp]
             lib.oracle_moe_forward.restype = ci
             lib.oracle_moe_forward.argtypes = [C.POINTER(_Layer), vp, ci, vp, vp, vp]
+            lib.oracle_moe_forward_part.restype = ci
+            lib.oracle_moe_forward_part.argtypes = [C.POINTER(_Layer), vp, ci, ci, ci, ci, vp]
             lib.oracle_moe_forward_dense.restype = ci
             lib.oracle_moe_forward_dense.argtypes = [C.POINTER(_Layer), vp, ci, vp]
             lib.oracle_shared.restype = ci
@@ -291,6 +293,27 @@ def forward(layer: OracleLayer, x: np.ndarray):
     if st != OK:
         raise RuntimeError("oracle_moe_forward: %d" % st)
     return out, ids, g
+
+
+ROUTED, DENSE = 1, 2
+
+
+def forward_part(layer: OracleLayer, x: np.ndarray, expert_lo: int = 0, n_local: Optional[int] = None,
+                 parts: int = ROUTED | DENSE) -> np.ndarray:
+    """The part of the block one expert-parallel rank computes: the routed terms of the experts in
+    [expert_lo, expert_lo + n_local) (parts & ROUTED) and the shared expert + correction (parts &
+    DENSE).  Disjoint ranges covering all experts plus one dense part sum to forward()."""
+    x = _x(layer, x)
+    n_local = layer.n_experts - expert_lo if n_local is None else n_local
+    out = np.zeros((x.shape[0], layer.d), np.float64)
+    if x.shape[0] == 0:
+        return out
+    L = layer._c()
+    st = _load().oracle_moe_forward_part(C.byref(L), _ptr(x), x.shape[0], int(expert_lo), int(n_local), int(parts),
+                                         _ptr(out))
+    if st != OK:
+        raise RuntimeError("oracle_moe_forward_part: %d" % st)
+    return out
 
 
 def forward_dense(layer: OracleLayer, x: np.ndarray) -> np.ndarray:

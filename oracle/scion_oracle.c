@@ -450,8 +450,16 @@ static int check_layer(const oracle_layer* L) {
  * order; the pairs are visited expert by expert so each expert is dequantized once,
  * and the per-token sums then run in slot order.
  */
-int oracle_moe_forward(const oracle_layer* L, const uint16_t* x, int T, double* out, int32_t* ids_out,
-                       double* gates_out) {
+/*
+ * The block forward, or the part of it that one rank of an expert-parallel layout computes:
+ * routed terms only for experts e in [expert_lo, expert_lo + n_local) (parts & 1), the shared
+ * expert and the correction (parts & 2).  Disjoint expert ranges covering all E, plus the dense
+ * part once, sum to the block output.  (Expert parallelism is not on the pages; "Scion: ternary
+ * MoE quantization with trained corrections", Serving notes, places the experts of one large
+ * model on more than one device, and this is the plainest such split: by expert.)
+ */
+static int moe_forward_impl(const oracle_layer* L, const uint16_t* x, int T, double* out, int32_t* ids_out,
+                            double* gates_out, int expert_lo, int n_local, int parts) {
   int st = check_layer(L);
   if (st) return st;
   if (T <= 0) return ORACLE_OK;
@@ -471,10 +479,10 @@ int oracle_moe_forward(const oracle_layer* L, const uint16_t* x, int T, double* 
   if (st) goto done;
   oracle_group(ids, T, k, E, counts, offsets, perm);
 
-  /* Step 4: y[t][j] = expert e_{t,j} applied to x_t. */
+  /* Step 4: y[t][j] = expert e_{t,j} applied to x_t (for the experts of this part). */
 #pragma omp parallel for schedule(dynamic, 1)
   for (int e = 0; e < E; e++) {
-    if (counts[e] == 0) continue;
+    if (counts[e] == 0 || !(parts & 1) || e < expert_lo || e >= expert_lo + n_local) continue;
     long n = (long)F * d;
     double* wg = (double*)malloc(sizeof(double) * n);
     double* wu = (double*)malloc(sizeof(double) * n);
@@ -510,15 +518,19 @@ int oracle_moe_forward(const oracle_layer* L, const uint16_t* x, int T, double* 
       load_x(x + (long)t * d, d, xv);
       for (int i = 0; i < d; i++) acc[i] = 0.0;
       for (int j = 0; j < k; j++) {
+        const int e = ids[(long)t * k + j];
+        if (!(parts & 1) || e < expert_lo || e >= expert_lo + n_local) continue;
         const double* yj = y + ((long)t * k + j) * d;
         double g = gates[(long)t * k + j];
         for (int i = 0; i < d; i++) acc[i] += g * yj[i];
       }
-      if (L->shared_ffn > 0) {
+      if (!(parts & 2)) {
+        /* no dense terms in this part */
+      } else if (L->shared_ffn > 0) {
         shared_one(L, xv, hs, ys);
         for (int i = 0; i < d; i++) acc[i] += ys[i];
       }
-      if (L->rank > 0) {
+      if (L->rank > 0 && (parts & 2)) {
         const double* in = L->corr_on_output ? acc : xv;
         double* in_copy = (double*)malloc(sizeof(double) * d);
         memcpy(in_copy, in, sizeof(double) * d);
@@ -542,6 +554,18 @@ done:
  * with m_e = the gate of e if e is among the top-k of t, else 0.  Same result as
  * oracle_moe_forward; used on tiny sizes to check that the sparse form drops nothing.
  */
+int oracle_moe_forward(const oracle_layer* L, const uint16_t* x, int T, double* out, int32_t* ids_out,
+                       double* gates_out) {
+  return moe_forward_impl(L, x, T, out, ids_out, gates_out, 0, L ? L->n_experts : 0, 3);
+}
+
+int oracle_moe_forward_part(const oracle_layer* L, const uint16_t* x, int T, int expert_lo, int n_local, int parts,
+                            double* out) {
+  if (!L || expert_lo < 0 || n_local < 0 || expert_lo + n_local > L->n_experts || parts < 0 || parts > 3)
+    return ORACLE_EINVAL;
+  return moe_forward_impl(L, x, T, out, NULL, NULL, expert_lo, n_local, parts);
+}
+
 int oracle_moe_forward_dense(const oracle_layer* L, const uint16_t* x, int T, double* out) {
   int st = check_layer(L);
   if (st) return st;

@@ -262,3 +262,24 @@ def test_packed_correction_matches_numpy_from_codes():
     ol0.rank, ol0.corr_a, ol0.corr_b = 0, None, None
     out0, _, _ = oracle.forward(ol0, x)
     np.testing.assert_allclose(out - out0, c, rtol=1e-9, atol=1e-12)
+
+
+def test_expert_parallel_parts_sum_to_the_block():
+    """The parts an expert-parallel layout computes: routed terms of disjoint expert ranges that
+    cover all experts, plus the dense part (shared expert + correction) once, add up to the block
+    output; the dense part alone is the shared expert's output plus the correction's; an empty
+    range contributes nothing."""
+    cfg = synth.Config("ep", 41, 256, 12, 3, 128, 128, synth.PQ2_0, 16, False, [8], 1)
+    L = synth.layer_host(cfg)
+    ol = oracle_layer_from(cfg, L)
+    x = synth.x_host(cfg, 9)
+    full, _, _ = oracle.forward(ol, x)
+    parts = [oracle.forward_part(ol, x, lo, n, oracle.ROUTED) for lo, n in ((0, 5), (5, 4), (9, 3))]
+    dense = oracle.forward_part(ol, x, 0, 0, oracle.DENSE)
+    np.testing.assert_allclose(sum(parts) + dense, full, rtol=1e-12, atol=1e-12)
+    _, ys = oracle.shared(ol, x)
+    _, c = oracle.corr(ol, x)
+    np.testing.assert_allclose(dense, ys + c, rtol=1e-12, atol=1e-13)
+    assert (oracle.forward_part(ol, x, 4, 0, oracle.ROUTED) == 0).all()
+    np.testing.assert_allclose(oracle.forward_part(ol, x, 0, 12, oracle.ROUTED | oracle.DENSE), full, rtol=1e-12,
+                               atol=1e-13)
