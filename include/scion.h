@@ -158,6 +158,16 @@ typedef struct {
    * factors' blocks in place (they must outlive the handle); the tensor-core path (batches
    * above 64 tokens) uses exact fp16 copies (code * scale). */
   int corr_packed;
+  /* Expert parallelism: this handle holds experts [expert_lo, expert_lo + n_local_experts) of the
+   * n_experts the router scores (n_local_experts = 0: all of them, expert_lo must be 0).  The
+   * banks then hold n_local_experts experts ([n_local][F][d/128] and [n_local][d][F/128] blocks);
+   * routing still picks the top-k of all n_experts logits, and only the entries whose expert is
+   * local are grouped and computed (the grouping outputs of scion_moe_forward_debug are indexed
+   * by local expert).  With SCION_OPT_PARTS the handle computes the routed and / or the dense part
+   * (shared expert + correction) of the block; summing the routed parts of the ranks that hold all
+   * experts and one dense part gives the block output. */
+  int expert_lo;
+  int n_local_experts;
 } scion_layer_desc;
 
 typedef struct scion_layer scion_layer;
@@ -233,7 +243,11 @@ int scion_moe_forward_residual(const void* x, int T, const scion_layer* layer, c
  *    buffer, order of the additions not fixed).
  *    All settings give the same result up to fp32 summation order.
  * EINVAL for an unknown option or an out-of-range value. */
-enum { SCION_OPT_STREAM_MIN_TOKENS = 1, SCION_OPT_DECODE_TC = 2, SCION_OPT_DETERMINISTIC = 3 };
+enum { SCION_OPT_STREAM_MIN_TOKENS = 1, SCION_OPT_DECODE_TC = 2, SCION_OPT_DETERMINISTIC = 3, SCION_OPT_PARTS = 4 };
+/* SCION_OPT_PARTS (default SCION_PART_ROUTED | SCION_PART_DENSE): which part of the block a forward
+ * computes: the routed experts (the handle's local ones), the dense part (shared expert and
+ * correction), or both.  out is overwritten with the selected part (plus resid). */
+enum { SCION_PART_ROUTED = 1, SCION_PART_DENSE = 2 };
 int scion_layer_set_option(scion_layer* layer, int option, int value);
 
 /* Waits for `stream`, then returns the layer's device status word and clears it:

@@ -27,7 +27,7 @@ __all__ = [
     "scion_moe_forward_host", "scion_moe_forward_debug", "Layer", "library_path", "EXPORTS",
     "scion_profile_begin", "scion_profile_end", "scion_kernel_launches", "STAGES", "scion_layer_check",
     "scion_router_logits_static", "scion_layer_set_option", "SCION_OPT_STREAM_MIN_TOKENS", "SCION_OPT_DECODE_TC",
-    "SCION_OPT_DETERMINISTIC",
+    "SCION_OPT_DETERMINISTIC", "SCION_OPT_PARTS", "SCION_PART_ROUTED", "SCION_PART_DENSE",
     "scion_moe_forward_residual", "scion_quantize_device", "SCION_QUANT_ABSMEAN", "SCION_QUANT_LLOYD",
     "scion_selftest_bounded_wait", "scion_debug_route", "scion_corr_create", "scion_corr_forward", "Corr",
 ]
@@ -52,7 +52,8 @@ EXPORTS = (
     "scion_corr_device_bytes", "scion_corr_forward", "scion_corr_check",
 )
 SCION_QUANT_ABSMEAN, SCION_QUANT_LLOYD = 0, 1
-SCION_OPT_STREAM_MIN_TOKENS, SCION_OPT_DECODE_TC, SCION_OPT_DETERMINISTIC = 1, 2, 3
+SCION_OPT_STREAM_MIN_TOKENS, SCION_OPT_DECODE_TC, SCION_OPT_DETERMINISTIC, SCION_OPT_PARTS = 1, 2, 3, 4
+SCION_PART_ROUTED, SCION_PART_DENSE = 1, 2
 STAGES = ("router_f32", "xproj", "route", "gateup", "down_routed", "down_dense", "x16", "combine")
 
 
@@ -71,7 +72,7 @@ class _Desc(C.Structure):
         ("gate_exps", C.c_void_p), ("up_exps", C.c_void_p), ("down_exps", C.c_void_p),
         ("sh_gate", C.c_void_p), ("sh_up", C.c_void_p), ("sh_down", C.c_void_p),
         ("sh_gate_vec", C.c_void_p), ("corr_a", C.c_void_p), ("corr_b", C.c_void_p),
-        ("corr_packed", C.c_int),
+        ("corr_packed", C.c_int), ("expert_lo", C.c_int), ("n_local_experts", C.c_int),
     ]
 
 
@@ -290,7 +291,8 @@ class Layer:
 def scion_layer_create(*, d: int, n_experts: int, top_k: int, ffn: int, fmt: int, w_router, w_router_delta,
                        gate_exps, up_exps, down_exps, shared_ffn: int = 0, sh_gate=None, sh_up=None,
                        sh_down=None, rank: int = 0, corr_a=None, corr_b=None, norm_topk: int = 1,
-                       corr_packed: int = 0, max_tokens: int = 64, stream=None) -> Layer:
+                       corr_packed: int = 0, max_tokens: int = 64, expert_lo: int = 0, n_local_experts: int = 0,
+                       stream=None) -> Layer:
     """Builds a layer from CUDA tensors (see include/scion.h for layouts).
 
     w_router / w_router_delta: float32 (fp32 router) or bfloat16 [E, d]; banks: uint8 packed
@@ -317,6 +319,7 @@ def scion_layer_create(*, d: int, n_experts: int, top_k: int, ffn: int, fmt: int
     D.corr_a = _dptr(corr_a, "corr_a", cdt)
     D.corr_b = _dptr(corr_b, "corr_b", cdt)
     D.corr_packed = int(corr_packed)
+    D.expert_lo, D.n_local_experts = int(expert_lo), int(n_local_experts)
     h = C.c_void_p()
     st = _load().scion_layer_create(C.byref(D), int(max_tokens), _stream(stream), C.byref(h))
     _check(st, "scion_layer_create")

@@ -715,7 +715,7 @@ cudaError_t launch_gateup(const scion_layer* L, const __nv_bfloat16* /*x*/, int 
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
   a.d = L->d, a.F = L->F, a.k = L->k, a.Gd = L->Gd, a.fmt = L->fmt;
   a.hfrag = L->h, a.pexp = L->pexp;
-  const int slots = min(L->E, T * L->k);
+  const int slots = min(L->El, T * L->k);
   const dim3 grid(L->F / 16, slots);
   const int gpw = (L->Gd + kGuWarps - 1) / kGuWarps;
 #define SCION_GU(F_, G_) return launch_pdl(gateup_kernel<F_, G_>, grid, dim3(kGuWarps * 32), 0, s, a)
@@ -746,7 +746,7 @@ cudaError_t launch_gateup_dense(const scion_layer* L, int T, float* out, cudaStr
   b.w = L->dense_down, b.hz = L->hz, b.d = L->d, b.Kd = L->Kd, b.T = T, b.out = out;
   b.corr_b = L->desc.corr_packed ? static_cast<const uint8_t*>(L->desc.corr_b) : nullptr, b.Fs = L->Fs, b.r = L->r;
   b.xexp = L->xexp, b.z_only = 0;
-  const int slots = min(L->E, T * L->k);
+  const int slots = min(L->El, T * L->k);
   const int gx = L->F / 16, dense_x = L->d / 32;
   const int dense_tiles = dense_x * ((L->Kd + kDnKc - 1) / kDnKc);
   const dim3 grid(gx, slots + (dense_tiles + gx - 1) / gx);
@@ -776,7 +776,7 @@ cudaError_t launch_down_routed(const scion_layer* L, int T, float* out, cudaStre
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
   a.gperm = L->gperm;
   a.d = L->d, a.F = L->F, a.k = L->k, a.GF = L->GF, a.out = out;
-  const int slots = min(L->E, T * L->k);
+  const int slots = min(L->El, T * L->k);
   const dim3 grid(L->d / 16, slots);
   const int gpw = (L->GF + kDnWarps - 1) / kDnWarps;
 #define SCION_DN(F_, G_) return launch_pdl(down_routed_kernel<F_, G_>, grid, dim3(kDnWarps * 32), 0, s, a)

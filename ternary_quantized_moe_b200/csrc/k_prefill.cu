@@ -830,20 +830,24 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
 template <int VPL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                    int norm_topk, int tpw, int32_t* __restrict__ ids,
-                                                   float* __restrict__ gates, int32_t* __restrict__ counts) {
-  extern __shared__ int32_t hist[];  // [E]
+                                                   float* __restrict__ gates, int32_t* __restrict__ counts, int elo,
+                                                   int El) {
+  extern __shared__ int32_t hist[];  // [El]: the handle's local experts
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  for (int e = threadIdx.x; e < El; e += blockDim.x) hist[e] = 0;
   __syncthreads();
   for (int i = 0; i < tpw; ++i) {
     const int t = (blockIdx.x * tpw + i) * 8 + warp;
     if (t >= T) break;
     warp_topk<VPL>(logits + int64_t(t) * E, E, k, norm_topk, lane, ids + int64_t(t) * k, gates + int64_t(t) * k);
     __syncwarp();
-    if (lane < k) atomicAdd(&hist[ids[int64_t(t) * k + lane]], 1);
+    if (lane < k) {
+      const unsigned le = unsigned(ids[int64_t(t) * k + lane] - elo);
+      if (le < unsigned(El)) atomicAdd(&hist[le], 1);
+    }
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
+  for (int e = threadIdx.x; e < El; e += blockDim.x)
     if (hist[e]) atomicAdd(&counts[e], hist[e]);
 }
 
@@ -908,7 +912,8 @@ __global__ void __launch_bounds__(256) group_scatter_kernel(const int32_t* __res
                                                             int32_t* __restrict__ inv, int k,
                                                             const float* __restrict__ gates,
                                                             const int32_t* __restrict__ xexp,
-                                                            float* __restrict__ gperm, int32_t* __restrict__ pexp) {
+                                                            float* __restrict__ gperm, int32_t* __restrict__ pexp,
+                                                            int elo) {
   extern __shared__ int32_t sh[];  // cnt[E], base[E]
   int32_t *cnt = sh, *base = sh + E;
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
@@ -918,7 +923,10 @@ __global__ void __launch_bounds__(256) group_scatter_kernel(const int32_t* __res
 #pragma unroll
   for (int j = 0; j < kScatterMaxPerThread; ++j) {
     const int i = i0 + 256 * j;
-    id[j] = j < ept && i < n ? ids[i] : -1;
+    // local expert of the entry; entries of another rank's experts get no position (inv = -1)
+    id[j] = j < ept && i < n ? ids[i] - elo : -1;
+    if (id[j] >= E) id[j] = -1;
+    if (j < ept && i < n && id[j] < 0) inv[i] = -1;
     local[j] = id[j] >= 0 ? atomicAdd(&cnt[id[j]], 1) : 0;
   }
   __syncthreads();
@@ -1066,7 +1074,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const __half* __restrict__
       float g[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        if (j0 + j < k) {
+        if (j0 + j < k && iv[j0 + j] >= 0) {  // (an entry of another rank's expert has no row)
           raw[j] = reinterpret_cast<const uint4*>(y + int64_t(iv[j0 + j]) * d)[c8];
           g[j] = gt[j0 + j] * ys;
         } else {
@@ -1137,6 +1145,8 @@ void prefill_units(const scion_layer* L, void* xunits_host, int* n_x, void* duni
   *n_d = nd;
 }
 
+bool prefill_dense_down(const scion_layer* L) { return (L->parts & SCION_PART_DENSE) && L->pre->n_dunits > 0; }
+
 int prefill_max_units(const scion_layer* L) { return (L->E + 127) / 128 + (L->Fs + 127) / 128 + (L->r + 127) / 128 + L->d / 128; }
 
 cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfloat16* x, int T, float* out,
@@ -1147,7 +1157,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       const unsigned grid = unsigned(std::min((T + 7) / 8, num_sms() * 8));
       // without a dense down projection (which stores out first) the fused routed down
       // projection only adds into out: set it here
-      const int init = P.n_dunits == 0 && !L->deterministic;
+      const int init = !prefill_dense_down(L) && !L->deterministic && (L->parts & SCION_PART_ROUTED);
       if (L->fmt == SCION_PQ2_0)
         x16_kernel<SCION_PQ2_0><<<grid, 256, 0, s>>>(x, T, L->d, P.x16, P.xexp, init, resid, out);
       else
@@ -1155,13 +1165,17 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       return cudaGetLastError();
     }
     case SCION_STAGE_XPROJ: {
-      if (P.n_xunits == 0) return cudaSuccess;
+      // units of the selected parts: router units, then shared gate/up and correction units
+      const bool routed = L->parts & SCION_PART_ROUTED, dense = L->parts & SCION_PART_DENSE;
+      const int u0 = routed ? 0 : P.n_xrouter, u1 = dense ? P.n_xunits : P.n_xrouter;
+      if (u1 <= u0) return cudaSuccess;
       DenseParams dp;
       memcpy(dp.a, P.maps, sizeof(dp.a));
       if (make_tmap_2d(&dp.b, x, 1, T, L->d) != SCION_OK) return cudaErrorInvalidValue;
-      dp.units = static_cast<const DenseUnit*>(P.xunits), dp.K = L->d, dp.T = T, dp.ab_bf16 = 1;
-      dp.n_units = P.n_xunits;
-      dp.n_units2 = (L->desc.router_fp32 ? 0 : (L->E + 127) / 128) + (L->Fs + 127) / 128;
+      dp.units = static_cast<const DenseUnit*>(P.xunits) + u0, dp.K = L->d, dp.T = T, dp.ab_bf16 = 1;
+      dp.n_units = u1 - u0;
+      // two-matrix units (router + delta, shared gate/up) come first
+      dp.n_units2 = (routed ? P.n_xrouter : 0) + (dense ? (L->Fs + 127) / 128 : 0);
       dp.logits = P.logits, dp.ld_logits = L->E, dp.hz = P.hz, dp.ld_hz = L->Kd, dp.out = nullptr, dp.ld_out = 0;
       dp.resid = nullptr;
       dp.xexp = P.xexp, dp.has_corr = L->r > 0, dp.z_only = 0;
@@ -1175,11 +1189,11 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       // at least two CTAs per SM for the top-k and one for the scatter, then fewer global atomics
       const int tpw = max(1, min(2, T / (8 * 2 * num_sms())));
       const int n = T * L->k, ept = max(1, min(kScatterMaxPerThread, n / (256 * num_sms())));
-      cudaError_t e = cudaMemsetAsync(P.counts, 0, sizeof(int32_t) * L->E, s);
+      cudaError_t e = cudaMemsetAsync(P.counts, 0, sizeof(int32_t) * L->El, s);
       if (e != cudaSuccess) return e;
 #define SCION_TOPK(V) \
-  topk_kernel<V><<<(T + 8 * tpw - 1) / (8 * tpw), 256, sizeof(int32_t) * L->E, s>>>( \
-      P.logits, T, L->E, L->k, L->desc.norm_topk, tpw, P.ids, P.gates, P.counts)
+  topk_kernel<V><<<(T + 8 * tpw - 1) / (8 * tpw), 256, sizeof(int32_t) * L->El, s>>>( \
+      P.logits, T, L->E, L->k, L->desc.norm_topk, tpw, P.ids, P.gates, P.counts, L->elo, L->El)
       if (vpl <= 1) SCION_TOPK(1);
       else if (vpl <= 2) SCION_TOPK(2);
       else if (vpl <= 4) SCION_TOPK(4);
@@ -1189,12 +1203,12 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       else SCION_TOPK(64);
 #undef SCION_TOPK
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      group_scan_kernel<<<1, kScanThreads, 0, s>>>(P.counts, L->E, P.offsets, P.cursor,
+      group_scan_kernel<<<1, kScanThreads, 0, s>>>(P.counts, L->El, P.offsets, P.cursor,
                                                   static_cast<TernTile*>(P.tiles), P.n_tiles,
                                                   tile_width(int64_t(T) * L->k, L->E));
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
-      group_scatter_kernel<<<(n + 256 * ept - 1) / (256 * ept), 256, 2 * sizeof(int32_t) * L->E, s>>>(
-          P.ids, n, L->E, ept, P.cursor, P.perm, P.inv, L->k, P.gates, P.xexp, P.gperm, P.pexp);
+      group_scatter_kernel<<<(n + 256 * ept - 1) / (256 * ept), 256, 2 * sizeof(int32_t) * L->El, s>>>(
+          P.ids, n, L->El, ept, P.cursor, P.perm, P.inv, L->k, P.gates, P.xexp, P.gperm, P.pexp, L->elo);
       return cudaGetLastError();
     }
     case SCION_STAGE_GATEUP: {
@@ -1218,7 +1232,8 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       return cudaGetLastError();
     }
     case SCION_STAGE_COMBINE: {
-      combine_kernel<<<T, 256, 0, s>>>(P.y, P.inv, P.gates, L->k, L->d, P.xexp, P.n_dunits > 0 ? out : resid, out);
+      combine_kernel<<<T, 256, 0, s>>>(P.y, P.inv, P.gates, L->k, L->d, P.xexp, prefill_dense_down(L) ? out : resid,
+                                       out);
       return cudaGetLastError();
     }
     case SCION_STAGE_DOWN_DENSE: {

@@ -42,6 +42,12 @@ __global__ void router_f32_kernel(const __nv_bfloat16* __restrict__ x, const flo
   if (lane == 0) logits[int64_t(t) * E + e] = sa + sb;
 }
 
+// Local index of expert e in the handle's range [lo, lo + nl), or -1 (an entry of another rank).
+__device__ __forceinline__ int local_expert(int e, int lo, int nl) {
+  const unsigned u = unsigned(e - lo);
+  return u < unsigned(nl) ? int(u) : -1;
+}
+
 __device__ __forceinline__ void argmax_merge(float& v, int& i, float v2, int i2) {
   if (v2 > v || (v2 == v && i2 < i)) {
     v = v2;
@@ -62,15 +68,15 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
                                                               int32_t* __restrict__ n_active_out,
                                                               const int32_t* __restrict__ xexp,
                                                               int32_t* __restrict__ pexp_out,
-                                                              int32_t* __restrict__ any_scaled) {
+                                                              int32_t* __restrict__ any_scaled, int elo, int El) {
   extern __shared__ float smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = kRouteThreads / 32;
   float* vals = smem + warp * E;
-  int32_t* counts = reinterpret_cast<int32_t*>(smem + nwarps * E);
-  int32_t* cursor = counts + E;
-  int32_t* ids_s = cursor + E;
+  int32_t* counts = reinterpret_cast<int32_t*>(smem + nwarps * E);  // [El]
+  int32_t* cursor = counts + El;
+  int32_t* ids_s = cursor + El;  // local expert of each entry, -1 for another rank's
 
-  for (int e = threadIdx.x; e < E; e += kRouteThreads) counts[e] = 0;
+  for (int e = threadIdx.x; e < El; e += kRouteThreads) counts[e] = 0;
 
   // ---- top-k and gates, one warp per token
   for (int t = warp; t < T; t += nwarps) {
@@ -119,8 +125,9 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
     if (lane < k) {
       ids_out[t * k + lane] = my_id;
       gates_out[t * k + lane] = ex / z;
-      ids_s[t * k + lane] = my_id;
-      atomicAdd(&counts[my_id], 1);
+      const int le = local_expert(my_id, elo, El);
+      ids_s[t * k + lane] = le;
+      if (le >= 0) atomicAdd(&counts[le], 1);
     }
     __syncwarp();
   }
@@ -128,8 +135,8 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
 
   // ---- exclusive scan of counts and the active-expert list (warp 0)
   if (warp == 0) {
-    const int per = (E + 31) / 32;
-    const int e0 = lane * per, e1 = min(E, e0 + per);
+    const int per = (El + 31) / 32;
+    const int e0 = lane * per, e1 = min(El, e0 + per);
     int s = 0, a = 0;
     for (int e = e0; e < e1; ++e) {
       s += counts[e];
@@ -153,7 +160,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
       run += c;
     }
     if (lane == 31) {
-      offsets_out[E] = si;
+      offsets_out[El] = si;
       *n_active_out = ai;
     }
     int sc_any = 0;
@@ -166,12 +173,13 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
     const unsigned lt = (1u << lane) - 1u;
     for (int base = 0; base < n; base += 32) {
       int i = base + lane;
-      int e = i < n ? ids_s[i] : -1 - lane;  // unique dummies never match real ids
+      const bool mine = i < n && ids_s[i] >= 0;
+      int e = mine ? ids_s[i] : -1 - lane;  // unique dummies never match real ids
       unsigned mask = __match_any_sync(0xffffffffu, e);
       int rank = __popc(mask & lt);
-      int cur = i < n ? cursor[e] : 0;
+      int cur = mine ? cursor[e] : 0;
       __syncwarp();
-      if (i < n) {
+      if (mine) {
         const int sh = xexp[i / k];
         perm_out[cur + rank] = i;
         gperm_out[cur + rank] = gates_out[i] * pow2i(-2 * sh);
@@ -194,6 +202,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
 // xexp_s: the tokens' range exponents (staged); each routed position gets its token's exponent
 // (pexp_out) and its gate times 2^(-2 s_t) (gperm_out), the factor that takes the scaled expert
 // hidden back to the block's units.
+// ids_s holds local expert indices (-1: an entry of another rank, not grouped); E = local experts.
 __device__ __forceinline__ void group_staged(const int32_t* ids_s, const float* gates_s, const int32_t* xexp_s, int n,
                                              int k, int E, int lane, int32_t* counts, int32_t* cursor,
                                              int32_t* __restrict__ counts_out, int32_t* __restrict__ offsets_out,
@@ -242,12 +251,13 @@ __device__ __forceinline__ void group_staged(const int32_t* ids_s, const float* 
   const unsigned lt = (1u << lane) - 1u;
   for (int base = 0; base < n; base += 32) {
     const int i = base + lane;
-    const int e = i < n ? ids_s[i] : -1 - lane;  // unique dummies never match real ids
+    const bool mine = i < n && ids_s[i] >= 0;
+    const int e = mine ? ids_s[i] : -1 - lane;  // unique dummies never match real ids
     const unsigned mask = __match_any_sync(0xffffffffu, e);
     const int rank = __popc(mask & lt);
-    const int cur = i < n ? cursor[e] : 0;
+    const int cur = mine ? cursor[e] : 0;
     __syncwarp();
-    if (i < n) {
+    if (mine) {
       const int sh = xexp_s[i / k];
       perm_out[cur + rank] = i;
       gperm_out[cur + rank] = gates_s[i] * pow2i(-2 * sh);
@@ -272,18 +282,18 @@ __global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
     int32_t* __restrict__ perm_out, float* __restrict__ gperm_out, int32_t* __restrict__ active_out,
     int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info, const int32_t* __restrict__ xexp,
     int32_t* __restrict__ pexp_out, int4* __restrict__ dtiles, int32_t* __restrict__ n_dtiles,
-    int32_t* __restrict__ any_scaled) {
-  extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [E] | cursor [E] | xexp [T]
+    int32_t* __restrict__ any_scaled, int elo, int El) {
+  extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [El] | cursor [El] | xexp [T]
   const int n = T * k;
   int32_t* ids_s = reinterpret_cast<int32_t*>(rs);
   float* gates_s = rs + n;
   int32_t* counts = reinterpret_cast<int32_t*>(rs + 2 * n);
-  int32_t* cursor = counts + E;
-  int32_t* xexp_s = cursor + E;
+  int32_t* cursor = counts + El;
+  int32_t* xexp_s = cursor + El;
   constexpr int kThr = rc_threads<VPL>();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
-  for (int e = threadIdx.x; e < E; e += kThr) counts[e] = 0;
+  for (int e = threadIdx.x; e < El; e += kThr) counts[e] = 0;
   pdl_wait();
   for (int t = threadIdx.x; t < T; t += kThr) xexp_s[t] = xexp[t];
   for (int t = warp; t < T; t += kThr / 32)
@@ -292,11 +302,13 @@ __global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
   for (int i = threadIdx.x; i < n; i += kThr) {
     ids[i] = ids_s[i];
     gates[i] = gates_s[i];
-    atomicAdd(&counts[ids_s[i]], 1);
+    const int le = local_expert(ids_s[i], elo, El);
+    ids_s[i] = le;
+    if (le >= 0) atomicAdd(&counts[le], 1);
   }
   __syncthreads();
   if (warp == 0)
-    group_staged(ids_s, gates_s, xexp_s, n, k, E, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out,
+    group_staged(ids_s, gates_s, xexp_s, n, k, El, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out,
                  pexp_out, active_out, n_active_out, slot_info, dtiles, n_dtiles, any_scaled);
 }
 
@@ -310,15 +322,15 @@ __global__ void __launch_bounds__(kRmThreads) route_multi_kernel(
     int32_t* __restrict__ perm_out, float* __restrict__ gperm_out, int32_t* __restrict__ active_out,
     int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info, unsigned* __restrict__ done,
     const int32_t* __restrict__ xexp, int32_t* __restrict__ pexp_out, int4* __restrict__ dtiles,
-    int32_t* __restrict__ n_dtiles, int32_t* __restrict__ any_scaled) {
-  extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [E] | cursor [E] | xexp [T]
+    int32_t* __restrict__ n_dtiles, int32_t* __restrict__ any_scaled, int elo, int El) {
+  extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [El] | cursor [El] | xexp [T]
   __shared__ int last;
   const int n = T * k;
   int32_t* ids_s = reinterpret_cast<int32_t*>(rs);
   float* gates_s = rs + n;
   int32_t* counts = reinterpret_cast<int32_t*>(rs + 2 * n);
-  int32_t* cursor = counts + E;
-  int32_t* xexp_s = cursor + E;
+  int32_t* cursor = counts + El;
+  int32_t* xexp_s = cursor + El;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * (kRmThreads / 32) + warp;
   pdl_trigger();
@@ -330,19 +342,21 @@ __global__ void __launch_bounds__(kRmThreads) route_multi_kernel(
   __syncthreads();
   if (!last) return;
   __threadfence();
-  for (int e = threadIdx.x; e < E; e += kRmThreads) counts[e] = 0;
-  for (int i = threadIdx.x; i < n; i += kRmThreads) ids_s[i] = __ldcg(&ids[i]), gates_s[i] = __ldcg(&gates[i]);
+  for (int e = threadIdx.x; e < El; e += kRmThreads) counts[e] = 0;
+  for (int i = threadIdx.x; i < n; i += kRmThreads)
+    ids_s[i] = local_expert(__ldcg(&ids[i]), elo, El), gates_s[i] = __ldcg(&gates[i]);
   for (int i = threadIdx.x; i < T; i += kRmThreads) xexp_s[i] = xexp[i];
   __syncthreads();
-  for (int i = threadIdx.x; i < n; i += kRmThreads) atomicAdd(&counts[ids_s[i]], 1);
+  for (int i = threadIdx.x; i < n; i += kRmThreads)
+    if (ids_s[i] >= 0) atomicAdd(&counts[ids_s[i]], 1);
   __syncthreads();
   if (warp != 0) return;
   if (lane == 0) *done = 0;
-  group_staged(ids_s, gates_s, xexp_s, n, k, E, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out,
+  group_staged(ids_s, gates_s, xexp_s, n, k, El, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out,
                pexp_out, active_out, n_active_out, slot_info, dtiles, n_dtiles, any_scaled);
 }
 
-size_t route_cta_smem(int T, int E, int k) { return sizeof(float) * (2 * size_t(T) * k + 2 * size_t(E) + size_t(T)); }
+size_t route_cta_smem(int T, int El, int k) { return sizeof(float) * (2 * size_t(T) * k + 2 * size_t(El) + size_t(T)); }
 
 }  // namespace
 
@@ -355,7 +369,7 @@ cudaError_t launch_router_f32(const scion_layer* L, const __nv_bfloat16* x, int 
 
 cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s) {
   if (L->E <= 512) {
-    const size_t smem = route_cta_smem(T, L->E, L->k);
+    const size_t smem = route_cta_smem(T, L->El, L->k);
     // tile list only for the tensor-core decode kernels (stream_min_tokens and up, option set)
     int4* dtl = (L->tc_decode && T >= L->stream_min_tokens) ? reinterpret_cast<int4*>(L->dtiles) : nullptr;
     const int vpl = (L->E + 31) / 32;
@@ -363,12 +377,12 @@ cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s) {
   return T <= 32 ? launch_pdl(route_cta_kernel<V>, dim3(1), dim3(rc_threads<V>()), smem, s, L->logits, T, L->E, \
                               L->k, L->desc.norm_topk, L->ids, L->gates, L->counts, L->offsets, L->perm,       \
                               L->gperm, L->active, L->n_active, reinterpret_cast<int4*>(L->slot_info), L->xexp, \
-                              L->pexp, dtl, L->n_dtiles, L->any_scaled)                                        \
+                              L->pexp, dtl, L->n_dtiles, L->any_scaled, L->elo, L->El)                         \
                  : launch_pdl(route_multi_kernel<V>, dim3((T + 3) / 4), dim3(kRmThreads), smem, s, L->logits, T, \
                               L->E, L->k, L->desc.norm_topk, L->ids, L->gates, L->counts, L->offsets, L->perm, \
                               L->gperm, L->active, L->n_active, reinterpret_cast<int4*>(L->slot_info),         \
                               L->route_done, L->xexp, L->pexp, dtl, L->n_dtiles,                               \
-                              L->any_scaled)
+                              L->any_scaled, L->elo, L->El)
     if (vpl <= 1) SCION_ROUTE_CTA(1);
     else if (vpl <= 2) SCION_ROUTE_CTA(2);
     else if (vpl <= 4) SCION_ROUTE_CTA(4);
@@ -377,11 +391,11 @@ cudaError_t launch_route(const scion_layer* L, int T, cudaStream_t s) {
 #undef SCION_ROUTE_CTA
     return cudaGetLastError();
   }
-  size_t smem = sizeof(float) * (size_t(kRouteThreads / 32) * L->E) + sizeof(int32_t) * (2 * size_t(L->E)) +
+  size_t smem = sizeof(float) * (size_t(kRouteThreads / 32) * L->E) + sizeof(int32_t) * (2 * size_t(L->El)) +
                 sizeof(int32_t) * size_t(T) * L->k;
   route_kernel<<<1, kRouteThreads, smem, s>>>(L->logits, T, L->E, L->k, L->desc.norm_topk, L->ids, L->gates,
                                                L->counts, L->offsets, L->perm, L->gperm, L->active, L->n_active,
-                                               L->xexp, L->pexp, L->any_scaled);
+                                               L->xexp, L->pexp, L->any_scaled, L->elo, L->El);
   if (cudaError_t e = cudaGetLastError()) return e;
   return launch_slot_info(L, s);
 }
@@ -397,8 +411,8 @@ __global__ void slot_info_kernel(const int32_t* __restrict__ active, const int32
 }
 
 cudaError_t launch_slot_info(const scion_layer* L, cudaStream_t s) {
-  slot_info_kernel<<<(L->E + 255) / 256, 256, 0, s>>>(L->active, L->n_active, L->offsets, L->counts,
-                                                       reinterpret_cast<int4*>(L->slot_info), L->E);
+  slot_info_kernel<<<(L->El + 255) / 256, 256, 0, s>>>(L->active, L->n_active, L->offsets, L->counts,
+                                                        reinterpret_cast<int4*>(L->slot_info), L->El);
   return cudaGetLastError();
 }
 

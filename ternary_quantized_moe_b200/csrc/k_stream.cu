@@ -469,7 +469,7 @@ cudaError_t launch_stream_gateup(const scion_layer* L, int T, cudaStream_t s) {
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
   a.gperm = L->gperm, a.pexp = L->pexp, a.any_scaled = L->any_scaled, a.G = L->Gd, a.R = L->F, a.k = L->k, a.F = L->F, a.d = L->d, a.fmt = L->fmt;
   a.hfrag = L->h, a.out = nullptr, a.err = L->err;
-  const int max_items = min(L->E, T * L->k) * (L->F / 128);
+  const int max_items = min(L->El, T * L->k) * (L->F / 128);
   if (L->fmt == SCION_PQ2_0) return launch_stream<SCION_PQ2_0, 2>(a, max_items, s);
   return launch_stream<SCION_PTQ1_0, 2>(a, max_items, s);
 }
@@ -480,7 +480,7 @@ cudaError_t launch_stream_down(const scion_layer* L, int T, float* out, cudaStre
   a.slot_info = reinterpret_cast<const int4*>(L->slot_info), a.n_active = L->n_active, a.perm = L->perm;
   a.gperm = L->gperm, a.pexp = L->pexp, a.any_scaled = L->any_scaled, a.G = L->GF, a.R = L->d, a.k = L->k, a.F = L->F, a.d = L->d, a.fmt = L->fmt;
   a.hfrag = nullptr, a.out = out, a.err = L->err;
-  const int max_items = min(L->E, T * L->k) * (L->d / 128);
+  const int max_items = min(L->El, T * L->k) * (L->d / 128);
   if (L->fmt == SCION_PQ2_0) return launch_stream<SCION_PQ2_0, 1>(a, max_items, s);
   return launch_stream<SCION_PTQ1_0, 1>(a, max_items, s);
 }

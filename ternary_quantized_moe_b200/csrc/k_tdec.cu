@@ -470,7 +470,7 @@ cudaError_t launch_tdec(int na, const scion_layer* L, int T, float* out, cudaStr
     p.bank = L->dn_bank, p.G = L->GF, p.R = L->d, p.bmap = L->hp_map, p.bsum = L->hsum, p.out = out;
   }
   const int Tk = T * L->k;
-  const int max_tiles = Tk / kDecTile + std::min(L->E, Tk);
+  const int max_tiles = Tk / kDecTile + std::min(L->El, Tk);
   const int items = max_tiles * (p.R / 128);
   const dim3 grid(std::max(1, std::min(items, num_sms_td())));
 #define SCION_TD(F, NA) \

@@ -71,18 +71,18 @@ int create_prefill(scion_layer* L, cudaStream_t s) {
   memset(P, 0, sizeof(*P));
   L->pre = P;
   const size_t T = L->max_tokens, Tk = T * L->k;
-  const size_t max_tiles = (Tk + 127) / 128 + L->E;
+  const size_t max_tiles = (Tk + 127) / 128 + L->El;
   cudaError_t e;
 #define PTRY(x)                              \
   if ((e = (x)) != cudaSuccess) return cuda_status(e)
   PTRY(dev_alloc(L, &P->logits, sizeof(float) * T * L->E));
   PTRY(dev_alloc(L, &P->ids, sizeof(int32_t) * Tk));
   PTRY(dev_alloc(L, &P->gates, sizeof(float) * Tk));
-  PTRY(dev_alloc(L, &P->counts, sizeof(int32_t) * L->E));
-  PTRY(dev_alloc(L, &P->offsets, sizeof(int32_t) * (L->E + 1)));
+  PTRY(dev_alloc(L, &P->counts, sizeof(int32_t) * L->El));
+  PTRY(dev_alloc(L, &P->offsets, sizeof(int32_t) * (L->El + 1)));
   PTRY(dev_alloc(L, &P->perm, sizeof(int32_t) * Tk));
   PTRY(dev_alloc(L, &P->inv, sizeof(int32_t) * Tk));
-  PTRY(dev_alloc(L, &P->cursor, sizeof(int32_t) * L->E));
+  PTRY(dev_alloc(L, &P->cursor, sizeof(int32_t) * L->El));
   PTRY(dev_alloc(L, &P->y, sizeof(__half) * Tk * L->d));
   PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->tiles), scion::prefill_tile_bytes() * max_tiles));
   PTRY(dev_alloc(L, &P->n_tiles, sizeof(int32_t)));
@@ -96,6 +96,7 @@ int create_prefill(scion_layer* L, cudaStream_t s) {
   const int max_units = scion::prefill_max_units(L);
   std::vector<uint8_t> xu(scion::prefill_unit_bytes() * max_units), du(scion::prefill_unit_bytes() * max_units);
   scion::prefill_units(L, xu.data(), &P->n_xunits, du.data(), &P->n_dunits);
+  P->n_xrouter = L->desc.router_fp32 ? 0 : (L->E + 127) / 128;
   PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->xunits), scion::prefill_unit_bytes() * max_units));
   PTRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&P->dunits), scion::prefill_unit_bytes() * max_units));
   PTRY(cudaMemcpyAsync(P->xunits, xu.data(), xu.size(), cudaMemcpyHostToDevice, s));
@@ -146,6 +147,10 @@ int check_desc(const scion_layer_desc* D, int max_tokens) {
   if (D->corr_packed && D->rank && ((reinterpret_cast<uintptr_t>(D->corr_a) | reinterpret_cast<uintptr_t>(D->corr_b)) & 1))
     return SCION_EINVAL;  // blocks are read with 2-byte loads
   if (D->sh_gate_vec) return SCION_EINVAL;  // shared-expert sigmoid gate: not supported by the kernels yet
+  // expert range of an expert-parallel rank (0 local experts: all of them)
+  if (D->n_local_experts < 0 || D->expert_lo < 0 || (D->n_local_experts == 0 && D->expert_lo != 0) ||
+      D->expert_lo + D->n_local_experts > D->n_experts)
+    return SCION_EINVAL;
   return SCION_OK;
 }
 
@@ -188,16 +193,22 @@ struct StageScope {
 // Whole batch on the tensor-core path (T > SCION_TDEC).
 int forward_prefill(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, const float* resid,
                     cudaStream_t s) {
-  if (L->desc.router_fp32)
+  const bool routed = L->parts & SCION_PART_ROUTED;
+  if (routed && L->desc.router_fp32)
     SCION_STAGE(SCION_STAGE_ROUTER_F32, scion::launch_router_f32(L, x, T, L->pre->logits, s));
   SCION_STAGE(SCION_STAGE_X16, scion::launch_prefill_stage(SCION_STAGE_X16, L, x, T, out, resid, s));
   SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_prefill_stage(SCION_STAGE_XPROJ, L, x, T, out, resid, s));
-  SCION_STAGE(SCION_STAGE_ROUTE, scion::launch_prefill_stage(SCION_STAGE_ROUTE, L, x, T, out, resid, s));
-  SCION_STAGE(SCION_STAGE_GATEUP, scion::launch_prefill_stage(SCION_STAGE_GATEUP, L, x, T, out, resid, s));
-  SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_prefill_stage(SCION_STAGE_DOWN_DENSE, L, x, T, out, resid, s));
-  SCION_STAGE(SCION_STAGE_DOWN_ROUTED, scion::launch_prefill_stage(SCION_STAGE_DOWN_ROUTED, L, x, T, out, resid, s));
-  if (L->deterministic)
-    SCION_STAGE(SCION_STAGE_COMBINE, scion::launch_prefill_stage(SCION_STAGE_COMBINE, L, x, T, out, resid, s));
+  if (routed) {
+    SCION_STAGE(SCION_STAGE_ROUTE, scion::launch_prefill_stage(SCION_STAGE_ROUTE, L, x, T, out, resid, s));
+    SCION_STAGE(SCION_STAGE_GATEUP, scion::launch_prefill_stage(SCION_STAGE_GATEUP, L, x, T, out, resid, s));
+  }
+  if (scion::prefill_dense_down(L))
+    SCION_STAGE(SCION_STAGE_DOWN_DENSE, scion::launch_prefill_stage(SCION_STAGE_DOWN_DENSE, L, x, T, out, resid, s));
+  if (routed) {
+    SCION_STAGE(SCION_STAGE_DOWN_ROUTED, scion::launch_prefill_stage(SCION_STAGE_DOWN_ROUTED, L, x, T, out, resid, s));
+    if (L->deterministic)
+      SCION_STAGE(SCION_STAGE_COMBINE, scion::launch_prefill_stage(SCION_STAGE_COMBINE, L, x, T, out, resid, s));
+  }
   return SCION_OK;
 }
 
@@ -217,7 +228,10 @@ int forward_prefill(const scion_layer* L, const __nv_bfloat16* x, int T, float* 
 
 // One decode pass of T <= SCION_TDEC tokens.
 int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out, const float* resid, cudaStream_t s) {
-  if (L->desc.router_fp32) SCION_STAGE(SCION_STAGE_ROUTER_F32, scion::launch_router_f32(L, x, T, L->logits, s));
+  // which parts of the block this forward computes (SCION_OPT_PARTS)
+  const bool routed = L->parts & SCION_PART_ROUTED, dense = (L->parts & SCION_PART_DENSE) && L->Kdense;
+  if (routed && L->desc.router_fp32)
+    SCION_STAGE(SCION_STAGE_ROUTER_F32, scion::launch_router_f32(L, x, T, L->logits, s));
   const bool ring = T >= L->stream_min_tokens;
   // tcgen05 expert GEMMs instead of the bulk-copy ring kernels (their tiles come from the grouping
   // kernels of up to 512 experts)
@@ -226,9 +240,11 @@ int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out
   // runs the router part of the x-projection (with x's fragment rows and the clearing of out),
   // the layer's side stream the shared-expert / correction part and the dense down projection,
   // beside routing and the expert kernels; the caller's stream joins it at the end.
-  const bool side = ring && L->Kdense;
-  const int nx_main = side ? L->n_xrouter : L->n_xunits;
-  SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_xproj(L, x, T, out, resid, 0, nx_main, true, tcd, s));
+  const bool side = routed && dense && ring;
+  // x-projection units: router units first, then shared gate/up and correction A
+  const int unit0 = routed ? 0 : L->n_xrouter;
+  const int nx_main = routed ? ((dense && !side) ? L->n_xunits : L->n_xrouter) : (dense ? L->n_xunits - L->n_xrouter : 0);
+  SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_xproj(L, x, T, out, resid, unit0, nx_main, true, tcd && routed, s));
   int st = SCION_OK;
   if (side) {
     cudaError_t e = cudaEventRecord(L->ev_x, s);
@@ -250,22 +266,24 @@ int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out
     }
     st = st_side;
   }
-  SCION_STAGE_INTO(st, SCION_STAGE_ROUTE, scion::launch_route(L, T, s));
   // small batches: the dense down projection rides in the gate/up launch (it needs only the
   // x-projection), off the critical path of the routed kernels
-  const bool merged = !ring && scion::gateup_merges_dense(L, T);
-  SCION_STAGE_INTO(st, SCION_STAGE_GATEUP, tcd      ? scion::launch_tdec(2, L, T, out, s)
-                                           : ring   ? scion::launch_stream_gateup(L, T, s)
-                                           : merged ? scion::launch_gateup_dense(L, T, out, s)
-                                                    : scion::launch_gateup(L, x, T, s));
-  SCION_STAGE_INTO(st, SCION_STAGE_DOWN_ROUTED, tcd    ? scion::launch_tdec(1, L, T, out, s)
-                                                : ring ? scion::launch_stream_down(L, T, out, s)
-                                                       : scion::launch_down_routed(L, T, out, s));
+  const bool merged = routed && dense && !ring && scion::gateup_merges_dense(L, T);
+  if (routed) {
+    SCION_STAGE_INTO(st, SCION_STAGE_ROUTE, scion::launch_route(L, T, s));
+    SCION_STAGE_INTO(st, SCION_STAGE_GATEUP, tcd      ? scion::launch_tdec(2, L, T, out, s)
+                                             : ring   ? scion::launch_stream_gateup(L, T, s)
+                                             : merged ? scion::launch_gateup_dense(L, T, out, s)
+                                                      : scion::launch_gateup(L, x, T, s));
+    SCION_STAGE_INTO(st, SCION_STAGE_DOWN_ROUTED, tcd    ? scion::launch_tdec(1, L, T, out, s)
+                                                  : ring ? scion::launch_stream_down(L, T, out, s)
+                                                         : scion::launch_down_routed(L, T, out, s));
+  }
   if (side) {
     const cudaError_t e = cudaStreamWaitEvent(s, L->ev_dense, 0);
     return st != SCION_OK ? st : cuda_status(e);
   }
-  if (L->Kdense && !merged) SCION_STAGE_INTO(st, SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
+  if (dense && !merged) SCION_STAGE_INTO(st, SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
   return st;
 }
 
@@ -307,6 +325,8 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   memset(L, 0, sizeof(*L));
   L->desc = *desc;
   L->d = desc->d, L->E = desc->n_experts, L->k = desc->top_k, L->F = desc->ffn;
+  L->elo = desc->expert_lo, L->El = desc->n_local_experts ? desc->n_local_experts : desc->n_experts;
+  L->parts = SCION_PART_ROUTED | SCION_PART_DENSE;
   L->Fs = desc->shared_ffn, L->r = desc->rank, L->fmt = desc->fmt, L->max_tokens = max_tokens;
   L->Gd = L->d / 128, L->GF = L->F / 128;
   L->Kdense = L->Fs + L->r;
@@ -329,20 +349,20 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   L->n_xchunks = (L->d + SCION_XPROJ_KC - 1) / SCION_XPROJ_KC;
 
   SCION_TRY(scion::configure_kernels());
-  SCION_TRY(dev_alloc(L, &L->gu_bank, size_t(L->E) * (L->F / 128) * L->Gd * 2 * 8 * tb));
-  SCION_TRY(dev_alloc(L, &L->dn_bank, size_t(L->E) * (L->d / 128) * L->GF * 8 * tb));
+  SCION_TRY(dev_alloc(L, &L->gu_bank, size_t(L->El) * (L->F / 128) * L->Gd * 2 * 8 * tb));
+  SCION_TRY(dev_alloc(L, &L->dn_bank, size_t(L->El) * (L->d / 128) * L->GF * 8 * tb));
   SCION_TRY(dev_alloc(L, &L->dense_down, size_t(L->d) * L->Kd * sizeof(__half)));
   SCION_TRY(dev_alloc(L, &L->xunits, sizeof(scion::XUnit) * (units.size() ? units.size() : 1)));
   SCION_TRY(dev_alloc(L, &L->logits, sizeof(float) * TD * L->E));
   SCION_TRY(dev_alloc(L, &L->ids, sizeof(int32_t) * TD * L->k));
   SCION_TRY(dev_alloc(L, &L->gates, sizeof(float) * TD * L->k));
-  SCION_TRY(dev_alloc(L, &L->counts, sizeof(int32_t) * L->E));
-  SCION_TRY(dev_alloc(L, &L->offsets, sizeof(int32_t) * (L->E + 1)));
+  SCION_TRY(dev_alloc(L, &L->counts, sizeof(int32_t) * L->El));
+  SCION_TRY(dev_alloc(L, &L->offsets, sizeof(int32_t) * (L->El + 1)));
   SCION_TRY(dev_alloc(L, &L->perm, sizeof(int32_t) * TD * L->k));
   SCION_TRY(dev_alloc(L, &L->gperm, sizeof(float) * TD * L->k));
-  SCION_TRY(dev_alloc(L, &L->active, sizeof(int32_t) * L->E));
+  SCION_TRY(dev_alloc(L, &L->active, sizeof(int32_t) * L->El));
   SCION_TRY(dev_alloc(L, &L->n_active, sizeof(int32_t)));
-  SCION_TRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&L->slot_info), sizeof(int4) * L->E));
+  SCION_TRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&L->slot_info), sizeof(int4) * L->El));
   SCION_TRY(dev_alloc(L, &L->route_done, sizeof(unsigned)));
   SCION_TRY(cudaMemsetAsync(L->route_done, 0, sizeof(unsigned), s));
   SCION_TRY(dev_alloc(L, &L->h, sizeof(__half) * TD * L->k * L->GF * SCION_BROW));
@@ -351,7 +371,7 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   SCION_TRY(dev_alloc(L, &L->xexp, sizeof(int32_t) * TD));
   SCION_TRY(dev_alloc(L, &L->pexp, sizeof(int32_t) * TD * L->k));
   SCION_TRY(dev_alloc(L, reinterpret_cast<uint8_t**>(&L->dtiles),
-                      sizeof(int4) * (size_t(TD) * L->k / scion::kDecTile + L->E + 1)));
+                      sizeof(int4) * (size_t(TD) * L->k / scion::kDecTile + L->El + 1)));
   SCION_TRY(dev_alloc(L, &L->n_dtiles, sizeof(int32_t)));
   SCION_TRY(dev_alloc(L, &L->any_scaled, sizeof(int32_t)));
   SCION_TRY(dev_alloc(L, &L->xsum, sizeof(float) * TD * L->Gd));
@@ -388,11 +408,11 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
                                            L->bad, s));
     }
   }
-  SCION_TRY(scion::launch_retile(L->fmt, static_cast<const uint8_t*>(desc->gate_exps), L->E, L->F, L->Gd, 2, 0,
+  SCION_TRY(scion::launch_retile(L->fmt, static_cast<const uint8_t*>(desc->gate_exps), L->El, L->F, L->Gd, 2, 0,
                                  L->gu_bank, L->bad, s));
-  SCION_TRY(scion::launch_retile(L->fmt, static_cast<const uint8_t*>(desc->up_exps), L->E, L->F, L->Gd, 2, 1,
+  SCION_TRY(scion::launch_retile(L->fmt, static_cast<const uint8_t*>(desc->up_exps), L->El, L->F, L->Gd, 2, 1,
                                  L->gu_bank, L->bad, s));
-  SCION_TRY(scion::launch_retile(L->fmt, static_cast<const uint8_t*>(desc->down_exps), L->E, L->d, L->GF, 1, 0,
+  SCION_TRY(scion::launch_retile(L->fmt, static_cast<const uint8_t*>(desc->down_exps), L->El, L->d, L->GF, 1, 0,
                                  L->dn_bank, L->bad, s));
   // B operand of the tcgen05 decode down projection: the hidden rows, 16-row TMA boxes
   if ((st = scion::make_tmap_2d(&L->hp_map, L->hp, 0, int64_t(TD) * L->k, L->F, 16)) != SCION_OK) goto fail;
@@ -478,8 +498,8 @@ extern "C" int scion_moe_forward_debug(const void* x, int T, const scion_layer* 
   cp(dbg->logits, pre ? P->logits : L->logits, sizeof(float) * size_t(T) * L->E);
   cp(dbg->ids, pre ? P->ids : L->ids, sizeof(int32_t) * size_t(T) * L->k);
   cp(dbg->gates, pre ? P->gates : L->gates, sizeof(float) * size_t(T) * L->k);
-  cp(dbg->counts, pre ? P->counts : L->counts, sizeof(int32_t) * size_t(L->E));
-  cp(dbg->offsets, pre ? P->offsets : L->offsets, sizeof(int32_t) * size_t(L->E + 1));
+  cp(dbg->counts, pre ? P->counts : L->counts, sizeof(int32_t) * size_t(L->El));
+  cp(dbg->offsets, pre ? P->offsets : L->offsets, sizeof(int32_t) * size_t(L->El + 1));
   cp(dbg->perm, pre ? P->perm : L->perm, sizeof(int32_t) * size_t(T) * L->k);
   if (dbg->h && e == cudaSuccess)
     e = pre ? scion::launch_unperm_prefill(L->fmt, P->h, int64_t(T) * L->k * L->F, reinterpret_cast<__half*>(dbg->h), s)
@@ -712,6 +732,10 @@ extern "C" int scion_layer_set_option(scion_layer* L, int option, int value) {
     case SCION_OPT_DETERMINISTIC:
       if (value != 0 && value != 1) return SCION_EINVAL;
       L->deterministic = value;
+      return SCION_OK;
+    case SCION_OPT_PARTS:
+      if (value < 1 || value > (SCION_PART_ROUTED | SCION_PART_DENSE)) return SCION_EINVAL;
+      L->parts = value;
       return SCION_OK;
     default:
       return SCION_EINVAL;

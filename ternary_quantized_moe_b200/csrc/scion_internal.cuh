@@ -66,8 +66,9 @@ struct XUnit {
 struct PrefillState {
   CUtensorMap maps[6];  // A operands: router, delta, sh_gate, sh_up, corr_a, dense_down
   CUtensorMap hz_map;   // B operand of the dense down GEMM
-  void* xunits;         // DenseUnit[] (device)
+  void* xunits;         // DenseUnit[] (device): router units, shared gate/up units, correction units
   int n_xunits;
+  int n_xrouter;        // router units at the front of xunits
   void* dunits;
   int n_dunits;
   CUtensorMap x16_map;  // B operand of the ternary correction A's units (fp16 GEMM against x16)
@@ -121,6 +122,8 @@ struct scion_corr {
 struct scion_layer {
   scion_layer_desc desc;
   int d, E, k, F, Fs, r, fmt, max_tokens;
+  int elo, El;      // local experts [elo, elo + El) of the E the router scores (banks and grouping hold El)
+  int parts;        // SCION_PART_ROUTED | SCION_PART_DENSE: what a forward computes
   int Gd, GF;       // 128-groups along d and along F
   int Kdense;       // Fs + r
   int Kd;           // Kdense rounded up to 64: row stride of dense_down and hz (pad = 0)
@@ -239,6 +242,9 @@ cudaError_t launch_dequant_corr(const uint8_t* blocks, int rows, int K, __half* 
 cudaError_t launch_unperm_prefill(int fmt, const __half* src, int64_t n, __half* dst, cudaStream_t s);
 cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfloat16* x, int T, float* out,
                                  const float* resid, cudaStream_t s);
+// Whether a prefill forward runs the dense down projection (shared expert / correction selected
+// and present).
+bool prefill_dense_down(const scion_layer* L);
 
 // Launch with programmatic dependent launch: the kernel may start while its predecessor
 // on the stream drains; it must execute pdl_wait() before touching anything the

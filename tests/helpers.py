@@ -118,7 +118,7 @@ def packed_correction(cfg: synth.Config, seed: int = 55):
 
 
 def device_layer(cfg: synth.Config, L: dict, banks: dict, max_tokens: int, dev="cuda", norm_topk: int = 1,
-                 packed_corr=None):
+                 packed_corr=None, expert_lo: int = 0, n_local_experts: int = 0):
     import torch
 
     import ternary_quantized_moe_b200 as tq
@@ -138,7 +138,8 @@ def device_layer(cfg: synth.Config, L: dict, banks: dict, max_tokens: int, dev="
         sh_up=opt("sh_up"), sh_down=opt("sh_down"), rank=cfg.rank,
         corr_a=torch.from_numpy(packed_corr[0]).to(dev) if packed_corr else opt("corr_a"),
         corr_b=torch.from_numpy(packed_corr[1]).to(dev) if packed_corr else opt("corr_b"),
-        corr_packed=1 if packed_corr else 0, norm_topk=norm_topk, max_tokens=max_tokens)
+        corr_packed=1 if packed_corr else 0, norm_topk=norm_topk, max_tokens=max_tokens, expert_lo=expert_lo,
+        n_local_experts=n_local_experts)
 
 
 def range_mix(cfg: synth.Config, layer: oracle.OracleLayer, x: np.ndarray, seed: int = 4711) -> np.ndarray:

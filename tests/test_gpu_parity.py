@@ -427,6 +427,48 @@ def test_attn_out_correction_rejects_bad_descriptors():
         assert ei.value.status == tq.SCION_EINVAL
 
 
+@pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
+@pytest.mark.parametrize("T,max_tokens", [(5, 64), (40, 64), (300, 300)])
+def test_expert_parallel_parts(fmt, T, max_tokens):
+    """The parts of an expert-parallel layout on one GPU: three handles holding experts [0, 10),
+    [10, 18) and [18, 24) of a 24-expert layer (their slices of the banks), each computing its
+    routed part (SCION_OPT_PARTS), and one dense part (shared expert + correction).  Each part
+    against the oracle's part, their sum against the block (decode split-K and ring passes, the
+    tensor-core path)."""
+    cfg = small("ep", fmt, False, E=24, k=4)
+    L, banks, ol, x = _case(cfg, T)
+    full, _, _ = oracle.forward(ol, x)
+    scale = np.linalg.norm(full, axis=1, keepdims=True)
+    total = np.zeros_like(full)
+    for lo, n in ((0, 10), (10, 8), (18, 6)):
+        part_banks = {name: np.ascontiguousarray(banks[name][lo:lo + n]) for name in banks}
+        layer = device_layer(cfg, L, part_banks, max_tokens, expert_lo=lo, n_local_experts=n)
+        tq.scion_layer_set_option(layer, tq.SCION_OPT_PARTS, tq.SCION_PART_ROUTED)
+        got, dbg = run_forward(layer, x, T, debug=True, E=cfg.n_experts, k=cfg.top_k, F=cfg.ffn)
+        ref = oracle.forward_part(ol, x, lo, n, oracle.ROUTED)
+        assert (np.linalg.norm(got - ref, axis=1, keepdims=True) <= 1e-3 * scale).all()
+        # the grouping holds exactly the entries of the local experts (local indices)
+        _, ids, _ = oracle.route(ol, x)
+        loc = ids[(ids >= lo) & (ids < lo + n)] - lo
+        np.testing.assert_array_equal(dbg["counts"][:n], np.bincount(loc, minlength=n))
+        total += got
+    layer = device_layer(cfg, L, banks, max_tokens)
+    tq.scion_layer_set_option(layer, tq.SCION_OPT_PARTS, tq.SCION_PART_DENSE)
+    dense, _ = run_forward(layer, x, T)
+    check_output(dense, oracle.forward_part(ol, x, 0, 0, oracle.DENSE))
+    check_output(total + dense, full)
+
+
+def test_expert_range_rejects_bad_descriptors():
+    cfg = small("epx", synth.PQ2_0, False, E=16, k=4)
+    L = synth.layer_host(cfg)
+    banks = packed_banks(cfg, L)
+    for lo, n in ((3, 0), (-1, 4), (10, 8)):
+        with pytest.raises(tq.ScionError) as ei:
+            device_layer(cfg, L, banks, 64, expert_lo=lo, n_local_experts=n)
+        assert ei.value.status == tq.SCION_EINVAL
+
+
 @pytest.mark.parametrize("T,max_tokens", [(13, 64), (200, 200)])
 def test_debug_route_matches_oracle(T, max_tokens):
     """scion_debug_route (the routing alone): ids as sets per token, offsets and the grouping
