@@ -45,7 +45,7 @@ def load_traffic(workload, stage):
         for line in f:
             parts = line.split("#", 1)[0].split()
             if len(parts) == 3 and parts[0] == workload and parts[1] == stage:
-                return float(parts[2])
+                return None if parts[2] == "null" else float(parts[2])
     return None
 
 
