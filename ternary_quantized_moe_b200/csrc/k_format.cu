@@ -117,8 +117,18 @@ __global__ void retile_kernel(int fmt, const uint8_t* __restrict__ src, int E, i
       t[12 * lane + 6 * hi + q % 6] = s[q];
     }
     nbad += (s[24] > 242) + (s[25] > 26);
-    t[384 + 4 * r8 + 2 * hi] = s[24];
-    t[384 + 4 * r8 + 2 * hi + 1] = s[25];
+    // the row's 8 remainder trits (digits 0..4 of byte 24, 0..2 of the tail byte) as 2-bit
+    // fields: even trits 2i at bits 2i of byte L, odd trits 2i+1 at bits 2i of byte H
+    unsigned v24 = s[24], vt = s[25], L = 0, H = 0;
+    for (int j = 0; j < 8; ++j) {
+      unsigned dgt;
+      if (j < 5) dgt = v24 % 3, v24 /= 3;
+      else dgt = vt % 3, vt /= 3;
+      if (j & 1) H |= dgt << (j - 1);
+      else L |= dgt << j;
+    }
+    t[384 + 4 * r8 + hi] = uint8_t(L);
+    t[384 + 4 * r8 + 2 + hi] = uint8_t(H);
     t[416 + 4 * r8 + 2 * hi] = s[26];
     t[416 + 4 * r8 + 2 * hi + 1] = s[27];
   }

@@ -468,26 +468,10 @@ __device__ __forceinline__ void expand_ptq1_half(uint32_t codes, int t, int h, u
     }
   }
   {
-    // remainder trits: digits 0..4 of byte 24 and 0..2 of the tail byte, one digit chain
-    const uint32_t qt = lds_u16(blk + 384 + 4 * r8 + 2 * hi);
-    uint32_t pr;
-    asm("prmt.b32 %0, %1, 0, 0x4140;" : "=r"(pr) : "r"(qt));
-    __half2 V = u32_as_h2(pr | 0x64006400u);
-    uint32_t pd[5];
-#pragma unroll
-    for (int j = 0; j < 5; ++j) {
-      __half2 Vn = __hfma2(V, third, c1);
-      pd[j] = h2_as_u32(__hadd2(__hfma2(Vn, m3, V), c2047));
-      V = Vn;
-    }
-    uint32_t r0, r1;
-    if (h == 0) {  // columns 120..123 = byte-24 digits 0..3
-      asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r0) : "r"(pd[0]), "r"(pd[1]));
-      asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r1) : "r"(pd[2]), "r"(pd[3]));
-    } else {       // columns 124..127 = byte-24 digit 4, tail digits 0..2
-      asm("prmt.b32 %0, %1, %2, 0x7610;" : "=r"(r0) : "r"(pd[4]), "r"(pd[0]));
-      asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r1) : "r"(pd[1]), "r"(pd[2]));
-    }
+    // remainder trits (columns 120..127) as 2-bit fields: bytes (even trits, odd trits) of this row;
+    // half h takes trits 4h .. 4h + 3
+    const uint32_t x = (lds_u32(blk + 384 + 4 * r8) >> (8 * hi)) & 0x00ff00ffu;
+    const uint32_t r0 = ptq1_rem_pair(x, 4 * h), r1 = ptq1_rem_pair(x, 4 * h + 2);
     v[30] = h2_as_u32(__hmul2(u32_as_h2(r0), sc));
     v[31] = h2_as_u32(__hmul2(u32_as_h2(r1), sc));
   }

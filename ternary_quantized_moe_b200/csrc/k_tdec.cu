@@ -116,24 +116,10 @@ __device__ __forceinline__ void expand_ptq1_codes(uint32_t codes, int t, int h, 
       V = Vn;
     }
   }
-  const uint32_t qt = lds_u16(blk + 384 + 4 * r8 + 2 * hi);
-  uint32_t pr;
-  asm("prmt.b32 %0, %1, 0, 0x4140;" : "=r"(pr) : "r"(qt));
-  __half2 V = u32_as_h2(pr | 0x64006400u);
-  uint32_t pd[5];
-#pragma unroll
-  for (int j = 0; j < 5; ++j) {
-    const __half2 Vn = __hfma2(V, third, c1);
-    pd[j] = h2_as_u32(__hadd2(__hfma2(Vn, m3, V), c2047));
-    V = Vn;
-  }
-  if (h == 0) {  // columns 120..123 = byte-24 digits 0..3
-    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(v[30]) : "r"(pd[0]), "r"(pd[1]));
-    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(v[31]) : "r"(pd[2]), "r"(pd[3]));
-  } else {       // columns 124..127 = byte-24 digit 4, tail digits 0..2
-    asm("prmt.b32 %0, %1, %2, 0x7610;" : "=r"(v[30]) : "r"(pd[4]), "r"(pd[0]));
-    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(v[31]) : "r"(pd[1]), "r"(pd[2]));
-  }
+  // remainder trits (columns 120..127) as 2-bit fields: bytes (even trits, odd trits) of this row
+  const uint32_t x = (lds_u32(blk + 384 + 4 * r8) >> (8 * hi)) & 0x00ff00ffu;
+  v[30] = ptq1_rem_pair(x, 4 * h);
+  v[31] = ptq1_rem_pair(x, 4 * h + 2);
 }
 
 // fp16 group scale of row t of a 128-row group of one matrix, from the re-tiled bank in global memory.

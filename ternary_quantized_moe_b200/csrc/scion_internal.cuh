@@ -13,8 +13,12 @@
 //   PTQ1_0, 448 B = 16 x 28:
 //     [12L + m]        row r,   quintet byte 6c + m (m < 6)
 //     [12L + 6 + m]    row r+8, quintet byte 6c + m
-//     [384 + 4r + 0/1] row r: quintet byte 24 / tail byte 25
-//     [384 + 4r + 2/3] row r+8: quintet byte 24 / tail byte 25
+//     [384 + 4r + 0/1] even remainder trits of row r / row r+8
+//     [384 + 4r + 2/3] odd remainder trits of row r / row r+8
+//   The 8 remainder trits of a row (digits 0..4 of quintet byte 24, digits 0..2 of tail byte
+//   25: columns 120..127) are re-encoded as 2-bit fields (trit value 0..2): trit 2i at bits
+//   2i..2i+1 of the "even" byte, trit 2i+1 at bits 2i..2i+1 of the "odd" byte.  The same 16
+//   bits per row; lane c then takes its columns 120+2c, 121+2c with one shift and one mask.
 //     [416 + 4r + 0/2] fp16 scale of row r / row r+8
 //
 // Sub-tile blocks are ordered [expert][row/128][group][matrix][row%128/16] with
@@ -385,6 +389,14 @@ __host__ __device__ __forceinline__ int hz_shift(int s, int has_corr) { return (
 
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// PTQ1_0 remainder trits in the sub-tile layout (2-bit fields, trit value 0..2): the low two
+// bits of each half of (rem >> shift), OR-ed into fp16 1024 and less 1025, give the half2
+// (trit - 1) exactly.
+__device__ __forceinline__ uint32_t ptq1_rem_pair(uint32_t rem, int shift) {
+  const __half2 v = u32_as_h2(lop3_and_or(rem >> shift, 0x00030003u, 0x64006400u));
+  return h2_as_u32(__hsub2(v, u32_as_h2(0x64016401u)));
+}
 
 // x * sigmoid(x) with the fast exponential and division (a few ulp of fp32; the result is
 // rounded to fp16 or multiplied into an fp32 accumulation well above that error).

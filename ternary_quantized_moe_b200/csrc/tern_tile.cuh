@@ -167,43 +167,8 @@ __device__ __forceinline__ __half2 ptq1_v0(uint32_t a, uint32_t b, uint32_t sel)
   return u32_as_h2(lop3_and_or(p, 0x00ff00ffu, kMagic));
 }
 
-// The 8 remainder trits of a row are digits 0..4 of byte 24 (columns 120..124) and digits
-// 0..2 of the tail byte (125..127).  One digit chain on (1024 + q24, 1024 + tail) gives
-// p_j = (q24 digit j - 1, tail digit j - 1); returns the half2 of remainder trits 2c, 2c+1.
-// `qt` = q24 | tail << 8.
-__device__ __forceinline__ uint32_t ptq1_rem_slot(uint32_t qt, int c) {
-  uint32_t pr;
-  asm("prmt.b32 %0, %1, 0, 0x4140;" : "=r"(pr) : "r"(qt));
-  Ptq1Digits d{u32_as_h2(pr | kMagic)};
-  const uint32_t p0 = d.next(), p1 = d.next(), p2 = d.next(), p3 = d.next(), p4 = d.next();
-  uint32_t r;
-  if (c == 0)
-    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(p0), "r"(p1));  // (q24 d0, q24 d1)
-  else if (c == 1)
-    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(r) : "r"(p2), "r"(p3));  // (q24 d2, q24 d3)
-  else if (c == 2)
-    asm("prmt.b32 %0, %1, %2, 0x7610;" : "=r"(r) : "r"(p4), "r"(p0));  // (q24 d4, tail d0)
-  else
-    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(r) : "r"(p1), "r"(p2));  // (tail d1, tail d2)
-  return r;
-}
-
-// Same as ptq1_rem_slot without a branch on c (the four lane-columns pick their pair by selects).
-__device__ __forceinline__ uint32_t ptq1_rem_slot_nb(uint32_t qt, int c) {
-  uint32_t pr;
-  asm("prmt.b32 %0, %1, 0, 0x4140;" : "=r"(pr) : "r"(qt));
-  Ptq1Digits d{u32_as_h2(pr | kMagic)};
-  const uint32_t p0 = d.next(), p1 = d.next(), p2 = d.next(), p3 = d.next(), p4 = d.next();
-  const uint32_t a = c == 0 ? p0 : c == 1 ? p2 : c == 2 ? p4 : p1;
-  const uint32_t b = c == 0 ? p1 : c == 1 ? p3 : c == 2 ? p0 : p2;
-  const uint32_t sel = c < 2 ? 0x5410u : (c == 2 ? 0x7610u : 0x7632u);
-  uint32_t r;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
-  return r;
-}
-
 // PTQ1_0 tile for the ring kernels: the digit chains, then eight MMAs issued without `volatile`
-// (independent tiles of a stage can interleave), no branch on the lane-column.
+// (independent tiles of a stage can interleave).
 __device__ __forceinline__ void tile_mma_ptq1_nv(const TileRegs<SCION_PTQ1_0>& t, const uint32_t (&b)[16],
                                                  float (&acc)[4], int c) {
   const uint32_t sel_r[3] = {0x0300u, 0x0401u, 0x0502u};
@@ -215,8 +180,8 @@ __device__ __forceinline__ void tile_mma_ptq1_nv(const TileRegs<SCION_PTQ1_0>& t
 #pragma unroll
     for (int j = 0; j < 5; ++j) ar[5 * m + j] = dr.next(), ah[5 * m + j] = dh.next();
   }
-  ar[15] = ptq1_rem_slot_nb(t.rem & 0xffffu, c);
-  ah[15] = ptq1_rem_slot_nb(t.rem >> 16, c);
+  ar[15] = ptq1_rem_pair(t.rem, 2 * c);
+  ah[15] = ptq1_rem_pair(t.rem, 2 * c + 8);
   float g[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int s2 = 0; s2 < 8; ++s2) {
@@ -262,8 +227,8 @@ __device__ __forceinline__ void tile_mma(const TileRegs<FMT>& t, const uint32_t 
 #pragma unroll
       for (int j = 0; j < 5; ++j) ar[5 * m + j] = dr.next(), ah[5 * m + j] = dh.next();
     }
-    ar[15] = ptq1_rem_slot(t.rem & 0xffffu, c);
-    ah[15] = ptq1_rem_slot(t.rem >> 16, c);
+    ar[15] = ptq1_rem_pair(t.rem, 2 * c);
+    ah[15] = ptq1_rem_pair(t.rem, 2 * c + 8);
 #pragma unroll
     for (int s2 = 0; s2 < 8; ++s2) {
       const uint32_t fa[4] = {ar[2 * s2], ah[2 * s2], ar[2 * s2 + 1], ah[2 * s2 + 1]};

@@ -90,3 +90,27 @@ def test_ptq1_chain_constants_are_fp16():
     """The chain's constants are exact fp16 values (no rounding when they are loaded)."""
     for c in (0.333251953125, 682.5, -3.0, 2047.0):
         assert float(f16(c)) == c
+
+
+def test_ptq1_remainder_fields_all_bytes():
+    """The eight remainder trits of a row (digits 0..4 of quintet byte 24, 0..2 of the tail byte)
+    re-encoded as 2-bit fields, even trits in one byte and odd trits in the other, are read back
+    by lane-column c as the fp16 pair (trit 2c - 1, trit 2c+1 - 1): shift by 2c, mask the low two
+    bits of each half into fp16 1024, subtract 1025.  All 243 x 27 byte pairs, both rows of a
+    lane (the second row's bytes one byte higher)."""
+    q24, tail = np.meshgrid(np.arange(243), np.arange(27), indexing="ij")
+    q24, tail = q24.ravel(), tail.ravel()
+    trits = [(q24 // 3 ** j) % 3 for j in range(5)] + [(tail // 3 ** j) % 3 for j in range(3)]
+    even = sum(trits[2 * i] << (2 * i) for i in range(4)).astype(np.uint32)
+    odd = sum(trits[2 * i + 1] << (2 * i) for i in range(4)).astype(np.uint32)
+    for hi in range(2):
+        # bytes of the lane's word: (even r, even r+8, odd r, odd r+8); this row's pair at byte hi
+        other = (even * 7 + 3) & 0xFF  # some other row's bytes in the neighbouring slots
+        word = np.where(hi == 0, even | (other << 8) | (odd << 16) | (other << 24),
+                        other | (even << 8) | (other << 16) | (odd << 24)).astype(np.uint64)
+        for c in range(4):
+            f = ((word >> (2 * c + 8 * hi)) & 0x00030003) | 0x64006400
+            lo = bits_to_f64(f & 0xFFFF) - 1025.0
+            hi_half = bits_to_f64((f >> 16) & 0xFFFF) - 1025.0
+            np.testing.assert_array_equal(lo, trits[2 * c] - 1)
+            np.testing.assert_array_equal(hi_half, trits[2 * c + 1] - 1)
