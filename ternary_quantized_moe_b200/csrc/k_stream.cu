@@ -21,7 +21,8 @@ namespace {
 
 using namespace tc;
 
-constexpr int kRing = 4;    // stages in flight
+constexpr int kRing = 4;    // stages in flight (two CTAs per SM; three CTAs of a three-stage ring
+                            // measured slower)
 constexpr int kCons = 8;    // consumer warps (one 16-row sub-tile each)
 constexpr int kTok = 8;     // tokens per pass (one mma n-tile)
 constexpr int kRowB = SCION_BROW * 2;  // bytes of one token's 128-column group row (fp16 + sum tail)
@@ -94,11 +95,17 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], u
 
 // Predicated shared-memory loads: lanes whose token lies past the pass's count issue no bank
 // access and keep the old register contents (their accumulator columns are dropped later).
-__device__ __forceinline__ void lds128_if(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3, uint32_t addr,
-                                          bool p) {
+// lds_brow_if: the lane's 64 bytes of one B group row (four 16-byte chunks 64 bytes apart)
+// under one predicate.
+__device__ __forceinline__ void lds_brow_if(uint32_t (&r)[16], uint32_t addr, bool p) {
   asm volatile(
-      "{\n .reg .pred q;\n setp.ne.u32 q, %5, 0;\n @q ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n}\n"
-      : "+r"(r0), "+r"(r1), "+r"(r2), "+r"(r3)
+      "{\n .reg .pred q;\n setp.ne.u32 q, %17, 0;\n"
+      " @q ld.shared.v4.u32 {%0,%1,%2,%3}, [%16];\n"
+      " @q ld.shared.v4.u32 {%4,%5,%6,%7}, [%16+64];\n"
+      " @q ld.shared.v4.u32 {%8,%9,%10,%11}, [%16+128];\n"
+      " @q ld.shared.v4.u32 {%12,%13,%14,%15}, [%16+192];\n}\n"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
       : "r"(addr), "r"(uint32_t(p)));
 }
 __device__ __forceinline__ float ldsf_if(uint32_t addr, bool p) {
@@ -136,11 +143,7 @@ __device__ __forceinline__ void stage_groups(uint32_t stg, const LaneOffs& o, in
   const int c = lane & 3, n = lane >> 2;
   uint32_t b[J][16];
 #pragma unroll
-  for (int j = 0; j < J; ++j)
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      lds128_if(b[j][4 * i], b[j][4 * i + 1], b[j][4 * i + 2], b[j][4 * i + 3],
-                stg + o.brow + (j0 + j) * kRowB + 64 * i, n < nn);
+  for (int j = 0; j < J; ++j) lds_brow_if(b[j], stg + o.brow + (j0 + j) * kRowB, n < nn);
   if constexpr (FMT == SCION_PQ2_0) {
     uint4 w[J][NMAT];
     uint32_t sc[J][NMAT];
