@@ -198,19 +198,33 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(const float* __res
 // Up to 32 tokens one CTA does everything; above that the top-k is spread over ceil(T/4) CTAs
 // and the last one to finish stages the entries and groups them.
 
-// Warp 0 of the grouping CTA: counts[] holds the histogram of the n staged entries.
-// xexp_s: the tokens' range exponents (staged); each routed position gets its token's exponent
-// (pexp_out) and its gate times 2^(-2 s_t) (gperm_out), the factor that takes the scaled expert
-// hidden back to the block's units.
+// The grouping of n = T k staged entries (T <= 64) by all threads of one CTA.  An expert appears
+// at most once among a token's k entries (the top-k ids are distinct), so the rank of entry
+// (t, j) among its expert's entries in the stable (token, slot) order is the number of earlier
+// tokens that chose the expert: popc(tmask[e] & (2^t - 1)) with tmask[e] the expert's token bits.
 // ids_s holds local expert indices (-1: an entry of another rank, not grouped); E = local experts.
-__device__ __forceinline__ void group_staged(const int32_t* ids_s, const float* gates_s, const int32_t* xexp_s, int n,
-                                             int k, int E, int lane, int32_t* counts, int32_t* cursor,
-                                             int32_t* __restrict__ counts_out, int32_t* __restrict__ offsets_out,
-                                             int32_t* __restrict__ perm_out, float* __restrict__ gperm_out,
-                                             int32_t* __restrict__ pexp_out, int32_t* __restrict__ active_out,
-                                             int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info,
-                                             int4* __restrict__ dtiles, int32_t* __restrict__ n_dtiles,
-                                             int32_t* __restrict__ any_scaled) {
+
+// all threads: histogram and token bits of the staged entries (counts, tmask zeroed before)
+__device__ __forceinline__ void group_count(const int32_t* ids_s, int n, int k, int tid, int nthr, int32_t* counts,
+                                            unsigned long long* tmask) {
+  for (int i = tid; i < n; i += nthr) {
+    const int e = ids_s[i];
+    if (e >= 0) {
+      atomicAdd(&counts[e], 1);
+      atomicOr(&tmask[e], 1ull << (i / k));
+    }
+  }
+}
+
+// warp 0: exclusive scan of the counts (cursor[e] = first position of expert e), the per-expert
+// records, the active-expert list with its per-slot records, the tile list of the tensor-core
+// decode kernels, and whether any token of the batch is range-scaled.
+__device__ __forceinline__ void group_scan(const int32_t* xexp_s, int n, int k, int E, int lane, const int32_t* counts,
+                                           int32_t* cursor, int32_t* __restrict__ counts_out,
+                                           int32_t* __restrict__ offsets_out, int32_t* __restrict__ active_out,
+                                           int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info,
+                                           int4* __restrict__ dtiles, int32_t* __restrict__ n_dtiles,
+                                           int32_t* __restrict__ any_scaled) {
   const int per = (E + 31) / 32;
   const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
   int sc = 0, ac = 0, tc = 0;
@@ -246,25 +260,24 @@ __device__ __forceinline__ void group_staged(const int32_t* ids_s, const float* 
   for (int t = lane; t < n / k; t += 32) sc_any |= xexp_s[t] != 0;
   sc_any = __any_sync(0xffffffffu, sc_any);
   if (lane == 0) *any_scaled = sc_any;
-  __syncwarp();
-  // stable scatter in (token, slot) order, 32 entries at a time
-  const unsigned lt = (1u << lane) - 1u;
-  for (int base = 0; base < n; base += 32) {
-    const int i = base + lane;
-    const bool mine = i < n && ids_s[i] >= 0;
-    const int e = mine ? ids_s[i] : -1 - lane;  // unique dummies never match real ids
-    const unsigned mask = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(mask & lt);
-    const int cur = mine ? cursor[e] : 0;
-    __syncwarp();
-    if (mine) {
-      const int sh = xexp_s[i / k];
-      perm_out[cur + rank] = i;
-      gperm_out[cur + rank] = gates_s[i] * pow2i(-2 * sh);
-      pexp_out[cur + rank] = sh;
-      if (rank == 0) cursor[e] = cur + __popc(mask);
-    }
-    __syncwarp();
+}
+
+// all threads: each entry to its stable position.  Each routed position gets its token's range
+// exponent (pexp_out) and its gate times 2^(-2 s_t) (gperm_out), the factor that takes the scaled
+// expert hidden back to the block's units.
+__device__ __forceinline__ void group_scatter(const int32_t* ids_s, const float* gates_s, const int32_t* xexp_s, int n,
+                                              int k, int tid, int nthr, const int32_t* cursor,
+                                              const unsigned long long* tmask, int32_t* __restrict__ perm_out,
+                                              float* __restrict__ gperm_out, int32_t* __restrict__ pexp_out) {
+  for (int i = tid; i < n; i += nthr) {
+    const int e = ids_s[i];
+    if (e < 0) continue;
+    const int t = i / k;
+    const int pos = cursor[e] + __popcll(tmask[e] & ((1ull << t) - 1ull));
+    const int sh = xexp_s[t];
+    perm_out[pos] = i;
+    gperm_out[pos] = gates_s[i] * pow2i(-2 * sh);
+    pexp_out[pos] = sh;
   }
 }
 
@@ -283,8 +296,10 @@ __global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
     int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info, const int32_t* __restrict__ xexp,
     int32_t* __restrict__ pexp_out, int4* __restrict__ dtiles, int32_t* __restrict__ n_dtiles,
     int32_t* __restrict__ any_scaled, int elo, int El) {
-  extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [El] | cursor [El] | xexp [T]
+  extern __shared__ unsigned long long rs8[];  // tmask [El] | ids [T*k] | gates [T*k] | counts [El] | cursor [El] | xexp [T]
   const int n = T * k;
+  unsigned long long* tmask = rs8;
+  float* rs = reinterpret_cast<float*>(rs8 + El);
   int32_t* ids_s = reinterpret_cast<int32_t*>(rs);
   float* gates_s = rs + n;
   int32_t* counts = reinterpret_cast<int32_t*>(rs + 2 * n);
@@ -293,7 +308,7 @@ __global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
   constexpr int kThr = rc_threads<VPL>();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_trigger();
-  for (int e = threadIdx.x; e < El; e += kThr) counts[e] = 0;
+  for (int e = threadIdx.x; e < El; e += kThr) counts[e] = 0, tmask[e] = 0ull;
   pdl_wait();
   for (int t = threadIdx.x; t < T; t += kThr) xexp_s[t] = xexp[t];
   for (int t = warp; t < T; t += kThr / 32)
@@ -302,14 +317,16 @@ __global__ void __launch_bounds__(rc_threads<VPL>()) route_cta_kernel(
   for (int i = threadIdx.x; i < n; i += kThr) {
     ids[i] = ids_s[i];
     gates[i] = gates_s[i];
-    const int le = local_expert(ids_s[i], elo, El);
-    ids_s[i] = le;
-    if (le >= 0) atomicAdd(&counts[le], 1);
+    ids_s[i] = local_expert(ids_s[i], elo, El);
   }
   __syncthreads();
+  group_count(ids_s, n, k, threadIdx.x, kThr, counts, tmask);
+  __syncthreads();
   if (warp == 0)
-    group_staged(ids_s, gates_s, xexp_s, n, k, El, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out,
-                 pexp_out, active_out, n_active_out, slot_info, dtiles, n_dtiles, any_scaled);
+    group_scan(xexp_s, n, k, El, lane, counts, cursor, counts_out, offsets_out, active_out, n_active_out, slot_info,
+               dtiles, n_dtiles, any_scaled);
+  __syncthreads();
+  group_scatter(ids_s, gates_s, xexp_s, n, k, threadIdx.x, kThr, cursor, tmask, perm_out, gperm_out, pexp_out);
 }
 
 // ceil(T/4) CTAs of 4 warps (T > 32); the last CTA to finish groups.
@@ -323,9 +340,11 @@ __global__ void __launch_bounds__(kRmThreads) route_multi_kernel(
     int32_t* __restrict__ n_active_out, int4* __restrict__ slot_info, unsigned* __restrict__ done,
     const int32_t* __restrict__ xexp, int32_t* __restrict__ pexp_out, int4* __restrict__ dtiles,
     int32_t* __restrict__ n_dtiles, int32_t* __restrict__ any_scaled, int elo, int El) {
-  extern __shared__ float rs[];  // ids [T*k] | gates [T*k] | counts [El] | cursor [El] | xexp [T]
+  extern __shared__ unsigned long long rs8[];  // tmask [El] | ids [T*k] | gates [T*k] | counts [El] | cursor [El] | xexp [T]
   __shared__ int last;
   const int n = T * k;
+  unsigned long long* tmask = rs8;
+  float* rs = reinterpret_cast<float*>(rs8 + El);
   int32_t* ids_s = reinterpret_cast<int32_t*>(rs);
   float* gates_s = rs + n;
   int32_t* counts = reinterpret_cast<int32_t*>(rs + 2 * n);
@@ -342,21 +361,25 @@ __global__ void __launch_bounds__(kRmThreads) route_multi_kernel(
   __syncthreads();
   if (!last) return;
   __threadfence();
-  for (int e = threadIdx.x; e < El; e += kRmThreads) counts[e] = 0;
+  for (int e = threadIdx.x; e < El; e += kRmThreads) counts[e] = 0, tmask[e] = 0ull;
   for (int i = threadIdx.x; i < n; i += kRmThreads)
     ids_s[i] = local_expert(__ldcg(&ids[i]), elo, El), gates_s[i] = __ldcg(&gates[i]);
   for (int i = threadIdx.x; i < T; i += kRmThreads) xexp_s[i] = xexp[i];
   __syncthreads();
-  for (int i = threadIdx.x; i < n; i += kRmThreads)
-    if (ids_s[i] >= 0) atomicAdd(&counts[ids_s[i]], 1);
+  group_count(ids_s, n, k, threadIdx.x, kRmThreads, counts, tmask);
   __syncthreads();
-  if (warp != 0) return;
-  if (lane == 0) *done = 0;
-  group_staged(ids_s, gates_s, xexp_s, n, k, El, lane, counts, cursor, counts_out, offsets_out, perm_out, gperm_out,
-               pexp_out, active_out, n_active_out, slot_info, dtiles, n_dtiles, any_scaled);
+  if (warp == 0) {
+    if (lane == 0) *done = 0;
+    group_scan(xexp_s, n, k, El, lane, counts, cursor, counts_out, offsets_out, active_out, n_active_out, slot_info,
+               dtiles, n_dtiles, any_scaled);
+  }
+  __syncthreads();
+  group_scatter(ids_s, gates_s, xexp_s, n, k, threadIdx.x, kRmThreads, cursor, tmask, perm_out, gperm_out, pexp_out);
 }
 
-size_t route_cta_smem(int T, int El, int k) { return sizeof(float) * (2 * size_t(T) * k + 2 * size_t(El) + size_t(T)); }
+size_t route_cta_smem(int T, int El, int k) {
+  return sizeof(unsigned long long) * size_t(El) + sizeof(float) * (2 * size_t(T) * k + 2 * size_t(El) + size_t(T));
+}
 
 }  // namespace
 
