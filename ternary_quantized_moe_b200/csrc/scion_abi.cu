@@ -50,6 +50,7 @@ void free_layer(scion_layer* L) {
   for (void* p : ptrs)
     if (p) cudaFree(p);
   if (L->side) cudaStreamDestroy(L->side);
+  if (L->ev_start) cudaEventDestroy(L->ev_start);
   if (L->ev_x) cudaEventDestroy(L->ev_x);
   if (L->ev_dense) cudaEventDestroy(L->ev_dense);
   if (L->pre) {
@@ -238,24 +239,38 @@ int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out
   const bool tcd = ring && L->tc_decode && L->E <= 512;
   // Batches on the ring kernels split the dense work off the expert path: the caller's stream
   // runs the router part of the x-projection (with x's fragment rows and the clearing of out),
-  // the layer's side stream the shared-expert / correction part and the dense down projection,
-  // beside routing and the expert kernels; the caller's stream joins it at the end.
+  // the layer's side stream the shared-expert / correction part of the x-projection (from the
+  // start, beside the router part: it needs only x) and then, once out is cleared, the dense
+  // down projection, beside routing and the expert kernels; the caller's stream joins it at the end.
   const bool side = routed && dense && ring;
   // x-projection units: router units first, then shared gate/up and correction A
   const int unit0 = routed ? 0 : L->n_xrouter;
   const int nx_main = routed ? ((dense && !side) ? L->n_xunits : L->n_xrouter) : (dense ? L->n_xunits - L->n_xrouter : 0);
-  SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_xproj(L, x, T, out, resid, unit0, nx_main, true, tcd && routed, s));
+  if (!side) {
+    SCION_STAGE(SCION_STAGE_XPROJ, scion::launch_xproj(L, x, T, out, resid, unit0, nx_main, true, tcd && routed, s));
+  }
   int st = SCION_OK;
   if (side) {
-    cudaError_t e = cudaEventRecord(L->ev_x, s);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(L->side, L->ev_x, 0);
+    // fork: the side stream starts after everything issued on the caller's stream so far (x ready)
+    cudaError_t e = cudaEventRecord(L->ev_start, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(L->side, L->ev_start, 0);
     if (e != cudaSuccess) return cuda_status(e);  // nothing was launched on the side stream
+    // the router part first (the critical path), then the side stream's part
+    SCION_STAGE_INTO(st, SCION_STAGE_XPROJ,
+                     scion::launch_xproj(L, x, T, out, resid, unit0, nx_main, true, tcd && routed, s));
     int st_side = SCION_OK;
     {
       cudaStream_t s = L->side;  // SCION_STAGE_INTO launches and records on `s`
       SCION_STAGE_INTO(st_side, SCION_STAGE_XPROJ,
                        scion::launch_xproj(L, x, T, out, nullptr, L->n_xrouter, L->n_xunits - L->n_xrouter, false,
                                            false, s));
+    }
+    // the dense down projection adds into out after the caller's stream has cleared it (and
+    // written the tokens' range exponents)
+    if (st == SCION_OK && (e = cudaEventRecord(L->ev_x, s)) == cudaSuccess) e = cudaStreamWaitEvent(L->side, L->ev_x, 0);
+    if (e != cudaSuccess && st == SCION_OK) st = cuda_status(e);
+    if (st == SCION_OK) {
+      cudaStream_t s = L->side;
       SCION_STAGE_INTO(st_side, SCION_STAGE_DOWN_DENSE, scion::launch_down_dense(L, T, out, s));
     }
     // the join is recorded whatever happened above, so that no later work on the caller's stream
@@ -264,7 +279,7 @@ int forward_pass(const scion_layer* L, const __nv_bfloat16* x, int T, float* out
       cudaStreamSynchronize(L->side);
       st_side = cuda_status(e);
     }
-    st = st_side;
+    if (st == SCION_OK) st = st_side;
   }
   // small batches: the dense down projection rides in the gate/up launch (it needs only the
   // x-projection), off the critical path of the routed kernels
@@ -383,6 +398,7 @@ extern "C" int scion_layer_create(const scion_layer_desc* desc, int max_tokens, 
   SCION_TRY(dev_alloc(L, &L->bad, sizeof(int64_t)));
   SCION_TRY(dev_alloc(L, &L->err, sizeof(int)));
   SCION_TRY(cudaStreamCreateWithFlags(&L->side, cudaStreamNonBlocking));
+  SCION_TRY(cudaEventCreateWithFlags(&L->ev_start, cudaEventDisableTiming));
   SCION_TRY(cudaEventCreateWithFlags(&L->ev_x, cudaEventDisableTiming));
   SCION_TRY(cudaEventCreateWithFlags(&L->ev_dense, cudaEventDisableTiming));
   SCION_TRY(cudaMemsetAsync(L->err, 0, sizeof(int), s));

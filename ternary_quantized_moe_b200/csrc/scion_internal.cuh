@@ -175,7 +175,7 @@ struct scion_layer {
   scion::PrefillState* pre;  // tensor-core path (nullptr when max_tokens <= SCION_TDEC)
   int stream_min_tokens;     // decode batches of at least this many tokens use the bulk-copy ring kernels
   cudaStream_t side;         // the dense down projection of ring-kernel batches runs here
-  cudaEvent_t ev_x, ev_dense;  // x-projection done (fork) / dense down done (join)
+  cudaEvent_t ev_start, ev_x, ev_dense;  // fork (x ready) / out cleared / dense down done (join)
   size_t device_bytes;
 };
 
