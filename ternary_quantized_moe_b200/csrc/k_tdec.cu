@@ -148,7 +148,6 @@ __global__ void __launch_bounds__(kTdThreads, 1) tdec_kernel(const __grid_consta
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int RT = p.R >> 7;
-  const int n_items = *p.n_tiles * RT;
   const int64_t grp_stride = int64_t(R::c_bytes);
 
   if (threadIdx.x == 0) {
@@ -164,6 +163,10 @@ __global__ void __launch_bounds__(kTdThreads, 1) tdec_kernel(const __grid_consta
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the prologue above overlaps the previous kernel's tail; everything below reads its outputs
+  pdl_trigger();
+  pdl_wait();
+  const int n_items = *p.n_tiles * RT;
   const uint32_t tmem = tmem_slot;
   const uint32_t sbase = smem_u32(smem);
 
@@ -326,19 +329,36 @@ __global__ void __launch_bounds__(kTdThreads, 1) tdec_kernel(const __grid_consta
       for (int m = 0; m < NA; ++m)
 #pragma unroll
         for (int i = 0; i < kTN; ++i) acc[m][i] = 0.f;
-      float sc[NA], sc_next[NA], xg = 0.f, xg_next = 0.f;
+      // the row's group scales and the tokens' group sums, kPre groups ahead (their loads from L2
+      // are in flight while the earlier groups are folded)
+      constexpr int kPre = 4;
+      float scq[kPre][NA], xgq[kPre];
 #pragma unroll
-      for (int m = 0; m < NA; ++m) sc_next[m] = row_scale<FMT>(ebase + m * R::mat_bytes, row);
-      if (FMT == SCION_PQ2_0) xg_next = p.bsum[int64_t(my_brow) * p.G];
+      for (int j = 0; j < kPre; ++j) {
+#pragma unroll
+        for (int m = 0; m < NA; ++m)
+          scq[j][m] = j < p.G ? row_scale<FMT>(ebase + j * grp_stride + m * R::mat_bytes, row) : 0.f;
+        xgq[j] = (FMT == SCION_PQ2_0 && j < p.G) ? p.bsum[int64_t(my_brow) * p.G + j] : 0.f;
+      }
       for (int g = 0; g < p.G; ++g, ++gs) {
         const int sd = gs % R::kD;
+        float sc[NA], xg;
+        // rotate the prefetch ring (static indices: the ring shifts by one each group)
 #pragma unroll
-        for (int m = 0; m < NA; ++m) sc[m] = sc_next[m];
-        xg = xg_next;
-        if (g + 1 < p.G) {  // the next group's scales and sums, in flight during this group
+        for (int m = 0; m < NA; ++m) sc[m] = scq[0][m];
+        xg = xgq[0];
 #pragma unroll
-          for (int m = 0; m < NA; ++m) sc_next[m] = row_scale<FMT>(ebase + (g + 1) * grp_stride + m * R::mat_bytes, row);
-          if (FMT == SCION_PQ2_0) xg_next = p.bsum[int64_t(my_brow) * p.G + g + 1];
+        for (int j = 0; j + 1 < kPre; ++j) {
+#pragma unroll
+          for (int m = 0; m < NA; ++m) scq[j][m] = scq[j + 1][m];
+          xgq[j] = xgq[j + 1];
+        }
+        {
+          const int gn = g + kPre;
+#pragma unroll
+          for (int m = 0; m < NA; ++m)
+            scq[kPre - 1][m] = gn < p.G ? row_scale<FMT>(ebase + gn * grp_stride + m * R::mat_bytes, row) : 0.f;
+          xgq[kPre - 1] = (FMT == SCION_PQ2_0 && gn < p.G) ? p.bsum[int64_t(my_brow) * p.G + gn] : 0.f;
         }
         // no abort-flag test: the epilogue threads leave only together, by the vote
         if (!(ok = named_bar_and(1, kTdEpi, mbar_wait(&d_full[sd], (gs / R::kD) & 1, &abort_flag, p.err)))) break;
@@ -353,6 +373,7 @@ __global__ void __launch_bounds__(kTdThreads, 1) tdec_kernel(const __grid_consta
         mbar_arrive(&d_empty[sd]);
 #pragma unroll
         for (int i = 0; i < kTN; ++i) {
+          if (i >= nn) break;  // the tile's tokens only (nn is the same for the whole warp)
           if constexpr (FMT == SCION_PQ2_0) {
             const float x = __shfl_sync(0xffffffffu, xg, i);  // group sum of token i's B row
 #pragma unroll
@@ -459,15 +480,14 @@ cudaError_t launch_tdec(int na, const scion_layer* L, int T, float* out, cudaStr
   const int max_tiles = Tk / kDecTile + std::min(L->El, Tk);
   const int items = max_tiles * (p.R / 128);
   const dim3 grid(std::max(1, std::min(items, num_sms_td())));
-#define SCION_TD(F, NA) \
-  tdec_kernel<F, NA><<<grid, kTdThreads, td_smem<F, NA>(), s>>>(p)
+#define SCION_TD(F, NA) return launch_pdl(tdec_kernel<F, NA>, grid, dim3(kTdThreads), td_smem<F, NA>(), s, p)
   if (L->fmt == SCION_PQ2_0) {
-    if (na == 2) SCION_TD(SCION_PQ2_0, 2); else SCION_TD(SCION_PQ2_0, 1);
-  } else {
-    if (na == 2) SCION_TD(SCION_PTQ1_0, 2); else SCION_TD(SCION_PTQ1_0, 1);
+    if (na == 2) SCION_TD(SCION_PQ2_0, 2);
+    SCION_TD(SCION_PQ2_0, 1);
   }
+  if (na == 2) SCION_TD(SCION_PTQ1_0, 2);
+  SCION_TD(SCION_PTQ1_0, 1);
 #undef SCION_TD
-  return cudaGetLastError();
 }
 
 }  // namespace scion
