@@ -204,6 +204,27 @@ def test_forward_variants(variant):
     check_output(got, ref)
 
 
+@pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
+@pytest.mark.parametrize("shape", ["d_max", "d_min"])
+@pytest.mark.parametrize("T", [1, 16, 64, 100])
+def test_forward_extreme_widths(fmt, shape, T):
+    """The widest block the decode x-projection takes (d = 4096: eight 512-column chunks in one
+    cluster) with the narrowest expert (F = 128: one group along the down projection's K) and
+    k = 1, and the narrowest block (d = 128: one group along every gate/up row), on the split-K,
+    ring and tensor-core paths (max_tokens = 128)."""
+    if shape == "d_max":
+        cfg = small("xw", fmt, False, E=8, k=1, d=4096, F=128, Fs=128, r=16)
+    else:
+        cfg = small("xn", fmt, False, E=8, k=2, d=128, F=128, Fs=128, r=16)
+    L, banks, ol, x = _case(cfg, T)
+    layer = device_layer(cfg, L, banks, 128)
+    got, dbg = run_forward(layer, x, T, debug=True, E=cfg.n_experts, k=cfg.top_k, F=cfg.ffn,
+                           Kdense=cfg.shared_ffn + cfg.rank)
+    _check_routing(cfg, dbg, ol, x, T, stable=T <= 64)
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
+
+
 @pytest.mark.parametrize("tc", [0, 1])
 @pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
 @pytest.mark.parametrize("T,E,k", [(1, 16, 4), (5, 16, 4), (13, 16, 4), (64, 16, 4), (64, 4, 2), (37, 6, 3)])
