@@ -322,6 +322,27 @@ def test_forward_packed_correction(fmt, T, max_tokens):
     check_output(got, ref)
 
 
+@pytest.mark.parametrize("T,max_tokens", [(5, 64), (40, 64), (300, 300)])
+def test_forward_packed_correction_activation_range(T, max_tokens):
+    """Ternary correction factors with activations far outside N(0, 1) (outlier channels, tokens
+    near 1e-6 or scaled by 256): the correction units read A from its blocks and scale z by the
+    token's range exponent (decode), or use the exact fp16 copies (tensor-core path)."""
+    cfg = small("pcr", synth.PQ2_0, False, E=16, k=4, Fs=128, r=256)
+    L, banks, ol, x = _case(cfg, T)
+    pa, pb = packed_correction(cfg)
+    ol.corr_a, ol.corr_b, ol.corr_packed = pa, pb, 1
+    x = range_mix(cfg, ol, with_margin(cfg, ol, x))
+    layer = device_layer(cfg, L, banks, max_tokens, packed_corr=(pa, pb))
+    got, dbg = run_forward(layer, x, T, debug=True, E=cfg.n_experts, k=cfg.top_k, F=cfg.ffn,
+                           Kdense=cfg.shared_ffn + cfg.rank)
+    assert tq.scion_layer_check(layer) == 0
+    assert np.isfinite(got).all()
+    _, ids, _ = oracle.route(ol, x)
+    np.testing.assert_array_equal(np.sort(dbg["ids"], 1), np.sort(ids, 1))
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
+
+
 def test_packed_correction_rejects_invalid_codes_and_rank():
     cfg = small("pcx", synth.PQ2_0, False, E=16, k=4, Fs=128, r=256)
     L = synth.layer_host(cfg)
