@@ -204,6 +204,23 @@ def test_forward_variants(variant):
     check_output(got, ref)
 
 
+@pytest.mark.parametrize("E,k,T,norm_topk,max_tokens", [(64, 32, 1, 1, 64), (64, 32, 13, 0, 64), (64, 32, 64, 1, 64),
+                                                       (512, 32, 40, 1, 64), (64, 32, 200, 0, 200),
+                                                       (512, 32, 200, 1, 200)])
+def test_forward_widest_topk(E, k, T, norm_topk, max_tokens):
+    """k = 32 (the largest top-k the descriptor accepts) with E <= 512: the decode routing kernels
+    (one CTA, and the multi-CTA form above 32 tokens) and the prefill top-k, both gate
+    normalisations; routing bit-exact, output within the block tolerance."""
+    cfg = small("wk", synth.PQ2_0 if E == 64 else synth.PTQ1_0, False, E=E, k=k)
+    L, banks, ol, x = _case(cfg, T, norm_topk)
+    layer = device_layer(cfg, L, banks, max_tokens, norm_topk=norm_topk)
+    got, dbg = run_forward(layer, x, T, debug=True, E=cfg.n_experts, k=cfg.top_k, F=cfg.ffn,
+                           Kdense=cfg.shared_ffn + cfg.rank)
+    _check_routing(cfg, dbg, ol, x, T, stable=T <= 64)
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
+
+
 @pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
 @pytest.mark.parametrize("shape", ["d_max", "d_min"])
 @pytest.mark.parametrize("T", [1, 16, 64, 100])
