@@ -272,8 +272,9 @@ typedef struct {
   uint16_t* h;      /* fp16 [T*k][F] expert SwiGLU hidden, row p for perm[p], times 2^(2s) */
   uint16_t* hz;     /* fp16 [T][Fs + r] shared SwiGLU hidden then correction z = A x, times 2^p */
 } scion_debug_out;
-/* (s is the token's range exponent of scion_moe_forward, 0 for max|x| in [2^-3, 2^6); p = s for
- * s > 0 on a layer with a correction, else 2s.) */
+/* (s is the token's range exponent of scion_moe_forward, 0 for max|x| in [2^-3, 2^6); p = s on a
+ * layer without a shared expert, 2s on a layer without a correction, and with both s for s > 0,
+ * else 2s.) */
 
 /* scion_moe_forward, then copies the intermediates requested in `dbg`. */
 int scion_moe_forward_debug(const void* x, int T, const scion_layer* layer, float* out, const scion_debug_out* dbg,

@@ -341,7 +341,7 @@ __global__ void __launch_bounds__(kXThreads) xproj_kernel(XProjArgs a) {
       for (int ch = 1; ch < a.n_chunks; ++ch)
         m = max(m, ld_dsmem_u32(map_cluster_rank(smem_addr(&tmax[t]), ch)));
       const int sh = token_shift(m);
-      tshift[t] = a.z_only ? sh : hz_shift(sh, a.r > 0);
+      tshift[t] = a.z_only ? sh : hz_shift(sh, a.Fs > 0, a.r > 0);
       if (a.z_only && blockIdx.x == 0) a.xexp[t] = sh;
     }
   }
@@ -542,7 +542,7 @@ struct DenseArgs {
   // (nullptr: every column from w)
   const uint8_t* corr_b;
   int Fs, r;
-  const int32_t* xexp;  // [T] range exponent of each token: hz rows hold 2^hz_shift(s_t, r > 0) times their values
+  const int32_t* xexp;  // [T] range exponent of each token: hz rows hold 2^hz_shift(s_t, Fs > 0, r > 0) times their values
   int z_only;           // hz holds z 2^s_t alone (the correction branch on the attention output)
 };
 
@@ -634,7 +634,7 @@ __device__ __forceinline__ void dense_body(const DenseArgs& a, int bx, int by) {
     const int row = bx * 32 + 16 * h + (ln >> 2) + 8 * (i >> 1), tok = nt * 8 + 2 * (ln & 3) + (i & 1);
     if (tok < a.T)
       atomicAdd(&a.out[int64_t(tok) * a.d + row],
-                v * pow2i(a.z_only ? -a.xexp[tok] : -hz_shift(a.xexp[tok], a.r > 0)));
+                v * pow2i(a.z_only ? -a.xexp[tok] : -hz_shift(a.xexp[tok], a.Fs > 0, a.r > 0)));
   }
 }
 

@@ -163,6 +163,7 @@ struct DenseParams {
   const float* resid;  // kEpiStore: added to the stored value (same layout as out; may equal out)
   const int32_t* xexp;  // range exponent s_t of each token: hz rows are stored times 2^hz_shift(s_t)
   int has_corr;         // the layer has a correction (hz_shift's choice)
+  int has_shared;       // the layer has a shared expert (hz_shift's choice)
   int z_only;           // the correction branch alone: z rows are stored times 2^s_t
   int* err;
 };
@@ -321,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) dense_gemm_kernel(const __grid_co
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const int sh = __shfl_sync(0xffffffffu, my_sh, i);
-            const int e = p.z_only ? sh : hz_shift(sh, p.has_corr);
+            const int e = p.z_only ? sh : hz_shift(sh, p.has_shared, p.has_corr);
             tf[i] = pow2i(u.epi == kEpiStore ? -e : (u.b16 ? e - sh : e));
           }
         }
@@ -1162,7 +1163,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       dp.n_units2 = (routed ? P.n_xrouter : 0) + (dense ? (L->Fs + 127) / 128 : 0);
       dp.logits = P.logits, dp.ld_logits = L->E, dp.hz = P.hz, dp.ld_hz = L->Kd, dp.out = nullptr, dp.ld_out = 0;
       dp.resid = nullptr;
-      dp.xexp = P.xexp, dp.has_corr = L->r > 0, dp.z_only = 0;
+      dp.xexp = P.xexp, dp.has_corr = L->r > 0, dp.has_shared = L->Fs > 0, dp.z_only = 0;
       dp.err = L->err;
       if (L->desc.corr_packed) dp.b16 = P.x16_map;
       dense_gemm_kernel<<<dense_grid(dp), kThreads, kDenseSmem, s>>>(dp);
@@ -1229,7 +1230,7 @@ cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfl
       dp.n_units = P.n_dunits, dp.n_units2 = 0;
       dp.logits = nullptr, dp.ld_logits = 0, dp.hz = nullptr, dp.ld_hz = 0, dp.out = out, dp.ld_out = L->d;
       dp.resid = resid;
-      dp.xexp = P.xexp, dp.has_corr = L->r > 0, dp.z_only = 0;
+      dp.xexp = P.xexp, dp.has_corr = L->r > 0, dp.has_shared = L->Fs > 0, dp.z_only = 0;
       dp.err = L->err;
       dense_gemm_kernel<<<dense_grid(dp), kThreads, kDenseSmem, s>>>(dp);
       return cudaGetLastError();

@@ -361,11 +361,12 @@ __device__ __forceinline__ uint32_t lop3_and_or(uint32_t a, uint32_t mask, uint3
 //                                            |silu(y)| <= |y| keeps it within the range of the
 //                                            hidden of the scaled token)
 //   expert output    gate 2^(-2s) y         (applied where the weighted sum enters out)
-//   shared / z rows  hz 2^p, p = s when the layer has a correction and s > 0, else 2s; the
-//                    dense down projection multiplies its output by 2^-p.  (The shared hidden
-//                    grows like x^2 and z like x: for s < 0 the x^2 terms dominate the output,
-//                    for s > 0 the correction does, so the term whose stored value may leave the
-//                    fp16 range is the one too small to matter.)
+//   shared / z rows  hz 2^p, the dense down projection multiplies its output by 2^-p:
+//                    p = s on a layer without a shared expert (z alone, which grows like x),
+//                    p = 2s on a layer without a correction (the shared hidden, like x^2), and
+//                    with both p = s for s > 0, else 2s (for s < 0 the x^2 terms dominate the
+//                    output, for s > 0 the correction does, so the term whose stored value may
+//                    leave the fp16 range is the one too small to matter).
 constexpr int kShiftLo = -3, kShiftHi = 5, kShiftTarget = 2, kShiftMax = 40;
 // s_t from the largest bf16 magnitude of the token (its bit pattern with the sign cleared)
 __host__ __device__ __forceinline__ int token_shift(uint32_t max_mag_bits) {
@@ -384,8 +385,11 @@ __host__ __device__ __forceinline__ float pow2i(int n) {
   v.u = uint32_t(n + 127) << 23;
   return v.f;
 }
-// exponent p of the shared / z rows' factor (see above); has_corr = the layer has a correction
-__host__ __device__ __forceinline__ int hz_shift(int s, int has_corr) { return (has_corr && s > 0) ? s : 2 * s; }
+// exponent p of the shared / z rows' factor (see above)
+__host__ __device__ __forceinline__ int hz_shift(int s, int has_shared, int has_corr) {
+  if (!has_shared) return s;
+  return (has_corr && s > 0) ? s : 2 * s;
+}
 
 __device__ __forceinline__ uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }

@@ -204,6 +204,28 @@ def test_forward_variants(variant):
     check_output(got, ref)
 
 
+@pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
+@pytest.mark.parametrize("dense", ["shared_only", "corr_only"])
+@pytest.mark.parametrize("T,max_tokens", [(1, 64), (13, 64), (40, 64), (200, 200)])
+def test_forward_one_dense_part(fmt, dense, T, max_tokens):
+    """A shared expert without a correction (the shared hidden then stored times 2^(2 s_t)) and a
+    correction without a shared expert (z times 2^(s_t)), with range-scaled tokens, on the
+    split-K, ring and tensor-core paths, at the 35B-A3B-class widths (d 2048, ffn 512)."""
+    Fs, r = (512, 0) if dense == "shared_only" else (0, 512)
+    cfg = small("od", fmt, False, E=16, k=4, d=2048, F=512, Fs=Fs, r=r)
+    L, banks, ol, x = _case(cfg, T)
+    x = range_mix(cfg, ol, x)
+    layer = device_layer(cfg, L, banks, max_tokens)
+    got, dbg = run_forward(layer, x, T, debug=True, E=cfg.n_experts, k=cfg.top_k, F=cfg.ffn,
+                           Kdense=cfg.shared_ffn + cfg.rank)
+    assert tq.scion_layer_check(layer) == 0
+    assert np.isfinite(got).all()
+    _, ids, _ = oracle.route(ol, x)
+    np.testing.assert_array_equal(np.sort(dbg["ids"], 1), np.sort(ids, 1))
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
+
+
 @pytest.mark.parametrize("E,k,T,norm_topk,max_tokens", [(64, 32, 1, 1, 64), (64, 32, 13, 0, 64), (64, 32, 64, 1, 64),
                                                        (512, 32, 40, 1, 64), (64, 32, 200, 0, 200),
                                                        (512, 32, 200, 1, 200)])
