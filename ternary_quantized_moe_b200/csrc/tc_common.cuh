@@ -1,5 +1,5 @@
 // tc_common.cuh -- sm_100a building blocks for the tensor-core (tcgen05) kernels:
-// mbarriers with bounded waits, TMA / bulk copies (no multicast), cp.async gathers,
+// mbarriers with bounded waits, TMA / bulk copies (each into its own CTA only), cp.async gathers,
 // UMMA descriptors, tcgen05.mma / commit / ld and TMEM allocation.
 //
 // Shared-memory operand layout used everywhere: K-major, 128-byte swizzle.  A tile of
@@ -114,7 +114,7 @@ __device__ __forceinline__ void fence_proxy_async() {
 }
 
 // ------------------------------------------------------------------ copies
-// 2-D tiled TMA load (no multicast) into CTA shared memory, completing on `bar`.
+// 2-D tiled TMA load into this CTA's shared memory only, completing on `bar`.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
