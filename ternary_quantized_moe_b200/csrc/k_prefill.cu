@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(256) x16_kernel(const __nv_bfloat16* __restric
       for (int e = 0; e < 8; ++e) {
         const int p = p0 + e;
         const float f = __bfloat162float(buf[warp][128 * gl + pos_col(FMT, p)]) * xs;
-        o[e] = __float2half_rn(FMT == SCION_PQ2_0 ? f * pq2_pos_scale(p) : f);
+        o[e] = __float2half_rn(f);
       }
       if (2 * i + gl < G) reinterpret_cast<uint4*>(orow + i * 256)[lane] = *reinterpret_cast<const uint4*>(o);
     }
@@ -109,8 +109,7 @@ __global__ void __launch_bounds__(256) x16_kernel(const __nv_bfloat16* __restric
 
 // Ternary correction factors (PQ2_0 blocks [rows][K/128], 2-bit codes + fp16 scale) -> fp16
 // code * scale, exact.  order < 0: natural column order; otherwise the column order of the
-// layer's x16 operand for expert format `order` (PQ2_0: with its 4^f factors multiplied back
-// in), so that a GEMM against x16 computes A x.  dst == nullptr only counts.  Invalid codes (3)
+// layer's x16 operand for expert format `order`, so that a GEMM against x16 computes A x.  dst == nullptr only counts.  Invalid codes (3)
 // and values past the fp16 range are counted into *bad.
 __global__ void dequant_corr_kernel(const uint8_t* __restrict__ blocks, int rows, int K, __half* __restrict__ dst,
                                     int ld, int order, unsigned long long* __restrict__ bad) {
@@ -123,11 +122,7 @@ __global__ void dequant_corr_kernel(const uint8_t* __restrict__ blocks, int rows
     const float sc = __half2float(__ushort_as_half(uint16_t(blk[32] | (blk[33] << 8))));
     float v = field == 3 ? 0.f : float(field - 1) * sc;
     nbad += field == 3;
-    int pos = col;
-    if (order >= 0) {
-      pos = perm_pos(order, col);
-      if (order == SCION_PQ2_0) v /= pq2_pos_scale(pos);  // times 4^f: exact unless it overflows
-    }
+    const int pos = order >= 0 ? perm_pos(order, col) : col;
     const __half hv = __float2half_rn(v);
     nbad += __hisinf(hv) != 0;
     if (dst) dst[int64_t(row) * ld + pos] = hv;
@@ -429,14 +424,16 @@ __device__ __forceinline__ void expand_pq2_half(uint32_t codes, int t, int h, ui
     for (int half = 0; half < 2; ++half) {
       const uint32_t w = half ? w2.y : w2.x, w10 = w >> 10;
       // pair s = columns (s, s + 8): the field at bits 2f..2f+1 of each 16-bit half (f = s, or
-      // s - 5 in w >> 10) ORed into 1024 is 1024 + 4^f b; minus 1024 + 4^f, times the scale, is
-      // 4^f * code * scale exactly (the 4^f is divided out of B)
+      // s - 5 in w >> 10) ORed into the fp16 pattern of 2^(10-2f) (exponent field 25 - 2f, whose
+      // mantissa unit is 4^-f) reads 2^(10-2f) + b; minus 2^(10-2f) + 1, times the scale, is
+      // code * scale exactly, so the B operands carry no factor
       uint32_t v[8];
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
         const int f = s < 5 ? s : s - 5;
-        const uint32_t bias = 0x6400u + (1u << (2 * f));
-        v[s] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(s < 5 ? w : w10, 0x00030003u << (2 * f), 0x64006400u)),
+        const uint32_t magic = uint32_t(25 - 2 * f) << 10, bias = magic | (1u << (2 * f));
+        v[s] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(lop3_and_or(s < 5 ? w : w10, 0x00030003u << (2 * f),
+                                                               magic | (magic << 16))),
                                          u32_as_h2(bias | (bias << 16))),
                                  sc));
       }
@@ -731,7 +728,6 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
     const int q = warp & 3, half = (warp - 12) >> 2;
     const int row = q * 32 + lane;
     const int pcol = perm_pos(FMT, row);  // gate/up: position of this row inside its 128-column group of h
-    const float hscale = FMT == SCION_PQ2_0 ? pq2_pos_scale(pcol) : 1.0f;
     int li = 0;
     // no abort-flag test in the loop condition: the epilogue threads leave only together, by the vote
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++li) {
@@ -758,13 +754,13 @@ __global__ void __launch_bounds__(kTernThreads, 1) tern_gemm_kernel(const __grid
           if (__all_sync(0xffffffffu, my_sh == 0)) {
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              if (n0 + i < nn) dst[int64_t(i) * p.F] = __float2half_rn(silu_f(v0[i]) * v1[i] * hscale);
+              if (n0 + i < nn) dst[int64_t(i) * p.F] = __float2half_rn(silu_f(v0[i]) * v1[i]);
           } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int sh = __shfl_sync(0xffffffffu, my_sh, i);  // the sums are of x 2^sh
               if (n0 + i < nn)
-                dst[int64_t(i) * p.F] = __float2half_rn(silu_f(v0[i] * pow2i(-sh)) * (v1[i] * pow2i(sh)) * hscale);
+                dst[int64_t(i) * p.F] = __float2half_rn(silu_f(v0[i] * pow2i(-sh)) * (v1[i] * pow2i(sh)));
             }
           }
         } else if (p.y) {
@@ -1084,18 +1080,21 @@ __global__ void __launch_bounds__(256) combine_kernel(const __half* __restrict__
   }
 }
 
-__global__ void unperm_prefill_kernel(int fmt, const __half* __restrict__ src, int64_t n, __half* __restrict__ dst) {
+// h in the tcgen05 column order -> natural order.  pos_scaled: the values carry the PQ2_0
+// position factor 4^-f (the tensor-core decode's h), divided out here.
+__global__ void unperm_prefill_kernel(int fmt, int pos_scaled, const __half* __restrict__ src, int64_t n,
+                                      __half* __restrict__ dst) {
   int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const int64_t base = i & ~int64_t(127);
   const int p = perm_pos(fmt, int(i & 127));
   const float v = __half2float(src[base + p]);
-  dst[i] = __float2half_rn(fmt == SCION_PQ2_0 ? v / pq2_pos_scale(p) : v);
+  dst[i] = __float2half_rn(pos_scaled && fmt == SCION_PQ2_0 ? v / pq2_pos_scale(p) : v);
 }
 
-cudaError_t launch_unperm_prefill(int fmt, const __half* src, int64_t n, __half* dst, cudaStream_t s) {
+cudaError_t launch_unperm_prefill(int fmt, int pos_scaled, const __half* src, int64_t n, __half* dst, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
-  unperm_prefill_kernel<<<unsigned((n + 255) / 256), 256, 0, s>>>(fmt, src, n, dst);
+  unperm_prefill_kernel<<<unsigned((n + 255) / 256), 256, 0, s>>>(fmt, pos_scaled, src, n, dst);
   return cudaGetLastError();
 }
 

@@ -518,9 +518,9 @@ extern "C" int scion_moe_forward_debug(const void* x, int T, const scion_layer* 
   cp(dbg->offsets, pre ? P->offsets : L->offsets, sizeof(int32_t) * size_t(L->El + 1));
   cp(dbg->perm, pre ? P->perm : L->perm, sizeof(int32_t) * size_t(T) * L->k);
   if (dbg->h && e == cudaSuccess)
-    e = pre ? scion::launch_unperm_prefill(L->fmt, P->h, int64_t(T) * L->k * L->F, reinterpret_cast<__half*>(dbg->h), s)
+    e = pre ? scion::launch_unperm_prefill(L->fmt, 0, P->h, int64_t(T) * L->k * L->F, reinterpret_cast<__half*>(dbg->h), s)
         : (T >= L->stream_min_tokens && L->tc_decode && L->E <= 512)
-            ? scion::launch_unperm_prefill(L->fmt, L->hp, int64_t(T) * L->k * L->F, reinterpret_cast<__half*>(dbg->h), s)
+            ? scion::launch_unperm_prefill(L->fmt, 1, L->hp, int64_t(T) * L->k * L->F, reinterpret_cast<__half*>(dbg->h), s)
             : scion::launch_unfrag(L->fmt, L->h, T * L->k, L->GF, reinterpret_cast<__half*>(dbg->h), s);
   if (dbg->hz && e == cudaSuccess && L->Kdense)
     e = cudaMemcpy2DAsync(dbg->hz, sizeof(__half) * L->Kdense, pre ? P->hz : L->hz, sizeof(__half) * L->Kd,

@@ -243,7 +243,7 @@ int prefill_max_units(const scion_layer* L);
 void prefill_units(const scion_layer* L, void* xunits_host, int* n_x, void* dunits_host, int* n_d);
 cudaError_t launch_dequant_corr(const uint8_t* blocks, int rows, int K, __half* dst, int ld, int order,
                                 int64_t* bad, cudaStream_t s);
-cudaError_t launch_unperm_prefill(int fmt, const __half* src, int64_t n, __half* dst, cudaStream_t s);
+cudaError_t launch_unperm_prefill(int fmt, int pos_scaled, const __half* src, int64_t n, __half* dst, cudaStream_t s);
 cudaError_t launch_prefill_stage(int stage, const scion_layer* L, const __nv_bfloat16* x, int T, float* out,
                                  const float* resid, cudaStream_t s);
 // Whether a prefill forward runs the dense down projection (shared expert / correction selected

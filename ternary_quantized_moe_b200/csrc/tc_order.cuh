@@ -27,10 +27,11 @@ __device__ __forceinline__ int perm_pos(int fmt, int col) {  // physical column 
   return g | (64 * half + 10 * i + 2 * j + u);
 }
 
-// PQ2_0 B-operand factor of position p: positions (2s, 2s+1) of every 16 hold the pair of
-// columns (s, s + 8) that the expansion builds with the field at bits 2f..2f+1 of a 16-bit code
-// half (f = s < 5 ? s : s - 5), i.e. scaled by 4^f; the B operands (x and h) carry 4^-f, an exact
-// power-of-two scaling.
+// PQ2_0 B-operand factor of position p for the tensor-core decode: positions (2s, 2s+1) of
+// every 16 hold the pair of columns (s, s + 8) that its subnormal expansion builds with the field
+// at bits 2f..2f+1 of a 16-bit code half (f = s < 5 ? s : s - 5), i.e. scaled by 4^f; its B
+// operands (x and h) carry 4^-f, an exact power-of-two scaling.  The prefill expansion shifts
+// each field down first and needs no factor.
 __device__ __forceinline__ float pq2_pos_scale(int p) {
   const int s = (p & 15) >> 1;
   return 1.0f / float(1 << (2 * (s < 5 ? s : s - 5)));

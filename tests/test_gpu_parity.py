@@ -226,6 +226,22 @@ def test_forward_one_dense_part(fmt, dense, T, max_tokens):
     check_output(got, ref)
 
 
+@pytest.mark.parametrize("fmt", [synth.PQ2_0, synth.PTQ1_0])
+@pytest.mark.parametrize("T,max_tokens", [(40, 64), (200, 200)])
+def test_forward_narrow_correction_only(fmt, T, max_tokens):
+    """A narrow layer (d 256, ffn 128) with a correction and no shared expert, on range-scaled
+    tokens whose energy sits in a few outlier channels: their scaled expert hidden is small, and
+    the tensor-core path keeps it out of the fp16 subnormals (no position factor on its operands)."""
+    cfg = small("od", fmt, False, E=16, k=4, Fs=0, r=128)
+    L, banks, ol, x = _case(cfg, T)
+    x = range_mix(cfg, ol, x)
+    layer = device_layer(cfg, L, banks, max_tokens)
+    got, _ = run_forward(layer, x, T)
+    assert tq.scion_layer_check(layer) == 0
+    ref, _, _ = oracle.forward(ol, x)
+    check_output(got, ref)
+
+
 @pytest.mark.parametrize("E,k,T,norm_topk,max_tokens", [(64, 32, 1, 1, 64), (64, 32, 13, 0, 64), (64, 32, 64, 1, 64),
                                                        (512, 32, 40, 1, 64), (64, 32, 200, 0, 200),
                                                        (512, 32, 200, 1, 200)])

@@ -37,8 +37,8 @@ def test_pq2_subnormal_fields(s):
 
 @pytest.mark.parametrize("s", range(8))
 def test_pq2_magic_fields(s):
-    """Split-K decode and prefill expansion: the field ORed into the fp16 pattern of 1024, minus
-    1024 + 4^f, is 4^f * (b - 1) = 4^f * code, with no rounding."""
+    """Split-K decode expansion: the field ORed into the fp16 pattern of 1024, minus 1024 + 4^f,
+    is 4^f * (b - 1) = 4^f * code, with no rounding."""
     f = s if s < 5 else s - 5
     src = HALVES if s < 5 else HALVES >> 10
     b = (src >> (2 * f)) & 3
@@ -47,14 +47,31 @@ def test_pq2_magic_fields(s):
     np.testing.assert_array_equal(got.astype(np.float64), 4.0 ** f * (b.astype(np.float64) - 1))
 
 
+@pytest.mark.parametrize("s", range(8))
+def test_pq2_exponent_magic_fields(s):
+    """Prefill expansion: the field at bits 2f..2f+1 ORed into the fp16 pattern with exponent
+    field 25 - 2f (the value 2^(10-2f), whose mantissa unit is 4^-f) reads 2^(10-2f) + b; minus
+    2^(10-2f) + 1 (that pattern with bit 2f set) it is the code b - 1, with no rounding and no
+    position factor."""
+    f = s if s < 5 else s - 5
+    src = HALVES if s < 5 else HALVES >> 10
+    b = ((src >> (2 * f)) & 3).astype(np.float64)
+    magic = (25 - 2 * f) << 10
+    v = bits_to_f64((src & (3 << (2 * f))) | magic)
+    np.testing.assert_array_equal(v, 2.0 ** (10 - 2 * f) + b)
+    bias = float(bits_to_f64(magic | (1 << (2 * f))))
+    assert bias == 2.0 ** (10 - 2 * f) + 1
+    np.testing.assert_array_equal(f16(v - bias).astype(np.float64), b - 1)
+
+
 def test_pq2_scaled_expansion_exact():
-    """Prefill expansion: 4^f * code times an fp16 group scale (the 4^f divided out of B later)
-    is exact in fp16 for every scale of the workloads' range and beyond."""
-    scales = f16(np.linspace(1e-3, 4.0, 4001))
-    for f in range(5):
-        for code in (-1, 0, 1):
-            got = f16(f16(4.0 ** f * code).astype(np.float64) * scales.astype(np.float64))
-            np.testing.assert_array_equal(got.astype(np.float64), 4.0 ** f * code * scales.astype(np.float64))
+    """Prefill expansion: code times an fp16 group scale is exact in fp16 for every finite fp16
+    scale (the product is the scale, zero or its negation)."""
+    scales = np.arange(1 << 16, dtype=np.uint16).view(np.float16)
+    scales = scales[np.isfinite(scales)].astype(np.float64)
+    for code in (-1.0, 0.0, 1.0):
+        got = f16(f16(code).astype(np.float64) * scales)
+        np.testing.assert_array_equal(got.astype(np.float64), code * scales)
 
 
 def _digit_chain(V, n):
